@@ -1,0 +1,133 @@
+"""KV-cache quantization reference: INT8 and FP8-E5M2 with per-token-head scales.
+
+Test infrastructure only (see ``oracle/__init__``).
+
+What the pages fix:
+* KV can be stored as FP8 or INT8 and is dequantized before use
+  [KV Cache 原理与 PagedAttention, §四 "KV Cache 量化" table; the FP8 flavour named
+  there is ``fp8_e5m2``].
+* The finest granularity listed, one scale per token per attention head
+  ("per-token-head"), is the one in mainstream use
+  [bjdmk.com.cn/news/6246348, §5.2].
+
+What they leave open, and the reading taken here (plain symmetric absmax):
+* a = max |x| over the D values of one (token, head) row;
+* scale = fl32(a / QMAX), QMAX = 127 for INT8 and 57344 (largest finite E5M2) for FP8;
+* y = fl32(x / scale) (IEEE fp32 division, correctly rounded);
+* INT8 code = clamp(round-half-even(y), -127, 127);
+  E5M2 code = round-half-even of y to 1-5-2 with saturation to +-57344;
+* a == 0 gives scale 0 and all-zero codes;
+* dequantized value = code * scale.
+
+The E5M2 encoder/decoder below are written from the format definition (OCP 8-bit
+floating point specification, E5M2: 1 sign bit, 5 exponent bits with bias 15,
+2 mantissa bits, subnormals when the exponent field is 0, exponent field 31 for
+Inf/NaN), working on the raw fp32 bits.
+"""
+import numpy as np
+
+QMAX_INT8 = np.float32(127.0)
+QMAX_E5M2 = np.float32(57344.0)       # (1 + 3/4) * 2**15
+E5M2_MAX_CODE = 0x7B                  # exponent field 30, mantissa 3
+
+
+def e5m2_decode(codes):
+    """E5M2 byte(s) -> float64 value(s), from the format definition."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where((c >> 7) & 1, -1.0, 1.0)
+    e = (c >> 2) & 0x1F
+    m = (c & 3).astype(np.float64)
+    normal = np.ldexp(1.0 + m / 4.0, (e - 15).astype(np.int64))
+    subnormal = np.ldexp(m / 4.0, -14)
+    val = np.where(e == 0, subnormal, normal)
+    val = np.where(e == 31, np.where(m == 0, np.inf, np.nan), val)
+    return sign * val
+
+
+def e5m2_encode(y):
+    """float32 value(s) -> E5M2 byte(s): round to nearest, ties to even, saturating.
+
+    Magnitudes that round above the largest finite value (57344) saturate to it;
+    infinities saturate as well. NaN maps to 0x7F (never produced by quantize).
+    """
+    y = np.asarray(y, dtype=np.float32)
+    bits = y.view(np.uint32).astype(np.int64)
+    sign = (bits >> 31) & 1
+    E = (bits >> 23) & 0xFF
+    M = bits & 0x7FFFFF
+    is_nan = (E == 0xFF) & (M != 0)
+    is_inf = (E == 0xFF) & (M == 0)
+
+    # Normal results: E5M2 exponent field = E - 127 + 15 = E - 112 >= 1.
+    # Keep the top 2 mantissa bits, round on the 21 dropped bits (ties to even).
+    # A carry out of the mantissa correctly bumps the exponent field.
+    mag_n = ((E - 112) << 2) | (M >> 21)
+    rem = M & ((1 << 21) - 1)
+    half = 1 << 20
+    up = (rem > half) | ((rem == half) & ((mag_n & 1) == 1))
+    mag_n = mag_n + up.astype(np.int64)
+
+    # Subnormal results (E <= 112): the value in units of 2**-16 (the E5M2
+    # subnormal step) is sig * 2**(E - 134), sig the 24-bit significand; round
+    # that to an integer, ties to even. A result of 4 is the smallest normal
+    # (exponent field 1, mantissa 0), which the plain integer already encodes.
+    sig = np.where(E == 0, M, M | (1 << 23))
+    e_eff = np.where(E == 0, 1, E)             # fp32 subnormals share exponent -126
+    sh = np.clip(134 - e_eff, 0, 62)
+    q = sig >> sh
+    r = sig - (q << sh)
+    halfs = np.where(sh > 0, np.left_shift(np.int64(1), np.maximum(sh - 1, 0)), 0)
+    up_s = (sh > 0) & ((r > halfs) | ((r == halfs) & ((q & 1) == 1)))
+    mag_s = q + up_s.astype(np.int64)
+
+    mag = np.where(E >= 113, mag_n, mag_s)
+    mag = np.minimum(mag, E5M2_MAX_CODE)       # saturate (covers rounding into Inf)
+    mag = np.where(is_inf, E5M2_MAX_CODE, mag)
+    code = (sign << 7) | mag
+    code = np.where(is_nan, 0x7F, code)
+    return code.astype(np.uint8)
+
+
+def int8_encode(y):
+    """float32 value(s) -> INT8: round half to even, clamp to [-127, 127]."""
+    y = np.asarray(y, dtype=np.float32)
+    r = np.rint(y.astype(np.float64))          # numpy rint rounds half to even
+    return np.clip(r, -127, 127).astype(np.int8)
+
+
+def quantize_rows(x, kind):
+    """Per-row symmetric absmax quantization.
+
+    x: float32-representable values, shape [..., D]; each row of D values is one
+       (token, kv head) of K or V.
+    kind: "int8" or "e5m2".
+    Returns (codes [..., D] int8|uint8, scales [...] float32).
+    """
+    x = np.asarray(x, dtype=np.float32)
+    qmax = QMAX_INT8 if kind == "int8" else QMAX_E5M2
+    a = np.max(np.abs(x), axis=-1)                            # exact in fp32
+    scale = np.divide(a, qmax, dtype=np.float32)               # fl32(a / QMAX)
+    nz = scale > 0
+    safe = np.where(nz, scale, np.float32(1.0))
+    y = np.divide(x, safe[..., None], dtype=np.float32)        # fl32(x / scale)
+    if kind == "int8":
+        codes = int8_encode(y)
+        codes = np.where(nz[..., None], codes, np.int8(0)).astype(np.int8)
+    elif kind == "e5m2":
+        codes = e5m2_encode(y)
+        codes = np.where(nz[..., None], codes, np.uint8(0)).astype(np.uint8)
+    else:
+        raise ValueError(kind)
+    scale = np.where(nz, scale, np.float32(0.0)).astype(np.float32)
+    return codes, scale
+
+
+def dequantize(codes, scales, kind):
+    """codes [..., D], scales [...] -> float64 values code * scale (exact in fp64)."""
+    if kind == "int8":
+        v = np.asarray(codes, dtype=np.int8).astype(np.float64)
+    elif kind == "e5m2":
+        v = e5m2_decode(codes)
+    else:
+        raise ValueError(kind)
+    return v * np.asarray(scales, dtype=np.float32).astype(np.float64)[..., None]
