@@ -1,0 +1,422 @@
+"""Benchmark of one paged decode step on the LLaMA-70B-shaped GQA layer.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload gqa70b|mha13b|quant_a_int8|...] [--partition S]
+
+A step is the whole hot path for one batch: append of each sequence's new K/V
+token into the paged cache (kv_append), then paged decode attention
+(partition kernel + merge kernel), all through the library's C ABI.
+
+Workload (default): batch 32, 64 query / 8 KV heads, head_dim 128, bf16,
+16-token blocks, context lengths uniform on [512, 4096] (seed 0), pool 1.2x
+the blocks needed, shuffled placement, q/K/V ~ N(0, 1). The cache (302 MB of
+K/V) exceeds L2, and L2 is also flushed (256 MiB write) before every timed
+step, outside the timed events.
+
+Metric: KV HBM GB/s = algorithmic bytes per step / step time, where the
+bytes are K+V of every cached token read once, q read, output written, plus
+the append's reads and writes. Also reported: % of 8 TB/s, decode tokens/s
+(sequences per second per layer), the partition kernel's roofline fraction
+against the measured copy bandwidth, an end-to-end figure with host buffers,
+and the CPU oracle on a bounded sample.
+
+Multi-GPU (torchrun): replicas only. Each rank runs the same workload on its
+own GPU with no data-path collective; the step time is the max over ranks and
+the value the sum of all ranks' bytes over it.
+"""
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "paged decode attention: KV HBM GB/s (% of 8 TB/s), decode tokens/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+
+WORKLOADS = {
+    "gqa70b": ("LLaMA-70B-shaped GQA layer: 64 q / 8 kv heads, head_dim 128, bf16, block 16, "
+               "batch 32, context U[512,4096], pool 1.2x, shuffled placement",
+               lambda dev: W.gqa70b(dev)),
+    "mha13b": ("13B-shaped MHA layer: 40/40 heads, head_dim 128, fp16, block 16, batch 32 x 2048",
+               lambda dev: W.mha13b(dev)),
+    "quant_a_int8": ("INT8 per-token-head KV: 64/8 heads, head_dim 128, block 32, 64 x 4096",
+                     lambda dev: W.quant_long("int8", "a", dev)),
+    "quant_a_e5m2": ("FP8-E5M2 per-token-head KV: 64/8 heads, head_dim 128, block 32, 64 x 4096",
+                     lambda dev: W.quant_long("e5m2", "a", dev)),
+    "quant_b_int8": ("INT8 per-token-head KV: 64/8 heads, head_dim 128, block 32, 8 x 32768",
+                     lambda dev: W.quant_long("int8", "b", dev)),
+    "quant_b_e5m2": ("FP8-E5M2 per-token-head KV: 64/8 heads, head_dim 128, block 32, 8 x 32768",
+                     lambda dev: W.quant_long("e5m2", "b", dev)),
+}
+
+
+def measured_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def elt_bytes(cache):
+    return 2 if cache in ("bf16", "fp16") else 1
+
+
+def step_bytes(wl):
+    """Algorithmic bytes of one step: (decode kernel bytes, append bytes)."""
+    e = elt_bytes(wl.cache_dtype)
+    tokens = int(wl.context_lens.sum())
+    kv = tokens * wl.kv_heads * wl.head_dim * 2 * e
+    if e == 1:
+        kv += tokens * wl.kv_heads * 2 * 4                   # per-token-head scales
+    q_out = 2 * wl.batch * wl.q_heads * wl.head_dim * 2
+    rows = wl.batch * wl.kv_heads
+    append = rows * wl.head_dim * 2 * 2 + wl.batch * 8        # read new K, V and slots
+    append += rows * wl.head_dim * 2 * e + (rows * 2 * 4 if e == 1 else 0)   # write rows
+    return kv + q_out, append
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index, period=0.01):
+        self.index, self.period = index, period
+        self.samples = []
+        self.ok = False
+        self._stop = threading.Event()
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:    # no NVML: report it, do not guess
+            self.err = str(e)
+
+    def _reasons(self):
+        try:
+            return self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            return self.nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append((time.time(),
+                                     self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM),
+                                     self._reasons()))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self, t0, t1):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        s = [x for x in self.samples if t0 <= x[0] <= t1] or self.samples[-3:]
+        mhz = [x[1] for x in s]
+        bits = 0
+        for x in s:
+            bits |= x[2]
+        reasons = [n for b, n in self.REASONS.items() if bits & b and n != "gpu_idle"]
+        return {"sm_mhz": float(np.median(mhz)) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(s)}
+
+
+# ------------------------------------------------------------------ oracle arm
+
+def oracle_sample(wl, budget_s=15.0):
+    """Time the fp64 CPU oracle (as it stands) on a bounded sample of the step:
+    the append and decode of whole sequences, taken in order until ~budget_s of
+    CPU work. Returns (GB/s in the metric's bytes, seconds, sequences, threads)."""
+    from threadpoolctl import threadpool_info
+    from oracle import attention, cache_ops
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    dt = np.float16 if wl.cache_dtype == "fp16" else np.float32
+    if wl.k_fill is None:
+        raise SystemExit("the CPU baseline covers 16-bit caches only")
+    kc = wl.k_fill.float().cpu().numpy().astype(dt)
+    vc = wl.v_fill.float().cpu().numpy().astype(dt)
+    kn = wl.k_new.float().cpu().numpy().astype(dt)
+    vn = wl.v_new.float().cpu().numpy().astype(dt)
+    q = wl.q.float().cpu().numpy().astype(np.float64)
+    e = elt_bytes(wl.cache_dtype)
+    done, nbytes, t_total = 0, 0, 0.0
+    for b in range(wl.batch):
+        t0 = time.perf_counter()
+        cache_ops.append(kc, vc, kn[b:b + 1], vn[b:b + 1], wl.slot_new[b:b + 1], wl.block_size)
+        for h in range(wl.q_heads):
+            attention.decode_one(q, kc, vc, wl.block_tables, wl.context_lens, wl.scale, b, h)
+        t_total += time.perf_counter() - t0
+        done += 1
+        nbytes += int(wl.context_lens[b]) * wl.kv_heads * wl.head_dim * 2 * e \
+            + 2 * wl.q_heads * wl.head_dim * 2 + wl.kv_heads * wl.head_dim * 2 * 2 * (1 + e)
+        if t_total >= budget_s:
+            break
+    return nbytes / t_total / 1e9, t_total, done, threads
+
+
+# ------------------------------------------------------------------ ours
+
+def run_ours(args, rank, world, device):
+    import paged_kv_cache_440_b200 as pkv
+    desc, make = WORKLOADS[args.workload]
+    wl = make(device)
+    pool = pkv.KVPool(1, wl.num_blocks, wl.block_size, wl.kv_heads, wl.head_dim,
+                      wl.cache_dtype, device)
+    K, V, _, _ = pool.layer_views(0)
+    if wl.k_fill is not None:
+        K.copy_(wl.k_fill)
+        V.copy_(wl.v_fill)
+    else:
+        slots = torch.from_numpy(wl.slot_hist).to(device)
+        for s in range(0, wl.k_hist.shape[0], 65536):
+            pkv.kv_append(pool, 0, wl.k_hist[s:s + 65536].contiguous(),
+                          wl.v_hist[s:s + 65536].contiguous(), slots[s:s + 65536].contiguous())
+    tables = torch.from_numpy(wl.block_tables).to(device)
+    lens = torch.from_numpy(wl.context_lens.astype(np.int32)).to(device)
+    slot_new = torch.from_numpy(wl.slot_new).to(device)
+    max_ctx = int(wl.context_lens.max())
+    S = args.partition or pkv.default_partition(pool, wl.batch, wl.q_heads, max_ctx)
+    ws = pkv.make_workspace(pool, wl.batch, wl.q_heads, max_ctx, S)
+    out = torch.empty_like(wl.q)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+    multi = max_ctx > S
+
+    def one_step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        pkv.kv_append(pool, 0, wl.k_new, wl.v_new, slot_new)
+        if ev:
+            ev[1].record(stream)
+        pkv.paged_attn_partition(pool, 0, wl.q, tables, lens, max_ctx, wl.scale, out, ws,
+                                 partition_tokens=S)
+        if ev:
+            ev[2].record(stream)
+        if multi:
+            pkv.paged_attn_merge(pool, lens, tables.shape[1], max_ctx, out, ws,
+                                 partition_tokens=S)
+        if ev:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        one_step()
+    torch.cuda.synchronize(device)
+    pool.status_clear()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    sampler = ClockSampler(device.index if device.index is not None else 0).start()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    t0 = time.time()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)                   # evict L2 outside the timed events
+        one_step(evs[i])
+    torch.cuda.synchronize(device)
+    t1 = time.time()
+    if world > 1:
+        torch.distributed.barrier()
+    sampler.stop()
+    status = pool.status()
+    step_ms = np.array([e[0].elapsed_time(e[3]) for e in evs])
+    part_ms = np.array([e[1].elapsed_time(e[2]) for e in evs])
+    step_s = float(step_ms.mean()) / 1e3
+    part_s = float(part_ms.mean()) / 1e3
+    if world > 1:
+        t = torch.tensor([step_s, part_s], device=device, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        step_s, part_s = float(t[0]), float(t[1])
+    clocks = sampler.summary(t0, t1)
+
+    # ---------------------------------------------------------- end to end
+    e2e = None
+    if not args.no_e2e:
+        pin = lambda t: t.cpu().pin_memory()
+        h_q, h_kn, h_vn = pin(wl.q), pin(wl.k_new), pin(wl.v_new)
+        h_slot, h_tab, h_len = pin(slot_new), pin(tables), pin(lens)
+        h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        d_q, d_kn, d_vn = torch.empty_like(wl.q), torch.empty_like(wl.k_new), torch.empty_like(wl.v_new)
+        d_slot, d_tab, d_len = torch.empty_like(slot_new), torch.empty_like(tables), torch.empty_like(lens)
+        d_out = torch.empty_like(out)
+        h2d = sum(t.numel() * t.element_size() for t in (h_q, h_kn, h_vn, h_slot, h_tab, h_len))
+        d2h = h_out.numel() * h_out.element_size()
+        n_e2e = max(10, args.steps // 10)
+        times = []
+        for i in range(args.warmup + n_e2e):
+            flush.fill_(i & 0xFF)
+            torch.cuda.synchronize(device)
+            a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for d, h in ((d_q, h_q), (d_kn, h_kn), (d_vn, h_vn), (d_slot, h_slot),
+                         (d_tab, h_tab), (d_len, h_len)):
+                d.copy_(h, non_blocking=True)
+            pkv.kv_append(pool, 0, d_kn, d_vn, d_slot)
+            pkv.paged_attn_decode(pool, 0, d_q, d_tab, d_len, max_ctx, wl.scale, out=d_out,
+                                  partition_tokens=S, workspace=ws)
+            h_out.copy_(d_out, non_blocking=True)
+            b_.record(stream)
+            b_.synchronize()
+            if i >= args.warmup:
+                times.append(a.elapsed_time(b_) / 1e3)
+        e2e_s = float(np.mean(times))
+        if world > 1:
+            t = torch.tensor([e2e_s], device=device, dtype=torch.float64)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e2e_s = float(t[0])
+        e2e = (e2e_s, h2d, d2h)
+
+    dec_bytes, app_bytes = step_bytes(wl)
+    res = {"wl": wl, "desc": desc, "S": S, "step_s": step_s, "part_s": part_s,
+           "dec_bytes": dec_bytes, "app_bytes": app_bytes, "clocks": clocks,
+           "status": status, "e2e": e2e, "launches": args.steps * (3 if multi else 2),
+           "wall": t1 - t0}
+    return res
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="gqa70b")
+    ap.add_argument("--partition", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    desc, make = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        if rank == 0:
+            wl = make("cpu")
+            gbs, secs, nseq, threads = oracle_sample(wl, args.cpu_budget)
+            dec_bytes, app_bytes = step_bytes(wl)
+            step_s = (dec_bytes + app_bytes) / (gbs * 1e9)
+            line = {
+                "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": round(step_s * 1e3, 3), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": desc, "batch": wl.batch},
+                "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": threads,
+                                 "kind": "oracle",
+                                 "sample": "%d of %d sequences (all %d heads each), %.1f s" %
+                                           (nseq, wl.batch, wl.q_heads, secs)},
+                "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0},
+            }
+            print(json.dumps(line), flush=True)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    r = run_ours(args, rank, world, device)
+    wl = r["wl"]
+    total_bytes = (r["dec_bytes"] + r["app_bytes"]) * world
+    gbs = total_bytes / r["step_s"] / 1e9
+    peak, peak_kind = measured_peak()
+    achieved = r["dec_bytes"] / r["part_s"] / 1e9
+    traffic = None
+    try:
+        with open(TRAFFIC_FILE) as f:
+            tr = json.load(f).get(args.workload)
+        if tr and tr.get("kernel_source_hash") == kernel_hash():
+            traffic = tr["bytes_per_launch"]
+    except Exception:
+        pass
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and wl.k_fill is not None:
+        g_cpu, secs, nseq, threads = oracle_sample(wl, args.cpu_budget)
+        cpu = {"value": round(g_cpu, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+               "sample": "%d of %d sequences (all %d heads each), %.1f s of fp64 numpy" %
+                         (nseq, wl.batch, wl.q_heads, secs)}
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(gbs, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(r["step_s"] * 1e3, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": wl.cache_dtype if wl.cache_dtype != "e5m2" else "fp8_e5m2",
+            "data": "synthetic",
+            "config": {"workload": r["desc"], "batch": wl.batch, "q_heads": wl.q_heads,
+                       "kv_heads": wl.kv_heads, "head_dim": wl.head_dim,
+                       "block_size": wl.block_size, "cached_tokens": int(wl.context_lens.sum()),
+                       "partition_tokens": r["S"], "parallelism": "replicas" if world > 1 else "1 gpu",
+                       "l2": "inputs 3x L2 and L2 flushed (256 MiB write) before each timed step",
+                       "bytes_per_step": r["dec_bytes"] + r["app_bytes"]},
+            "pct_of_8tbs": round(100 * gbs / world / NOMINAL_HBM_GBS, 2),
+            "decode_tokens_per_s": round(wl.batch * world / r["step_s"], 1),
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
+                         "unit": "GB/s", "frac": round(achieved / peak, 4),
+                         "traffic": traffic, "kernel": "attn_partition_kernel",
+                         "peak_source": peak_kind + " (MEASURED_PEAKS.json hbm_gbs)"
+                         if peak_kind == "measured" else "fallback 6650 GB/s",
+                         "kernel_ms": round(r["part_s"] * 1e3, 5)},
+            "cpu_baseline": cpu,
+            "e2e": None if r["e2e"] is None else {
+                "value": round(total_bytes / r["e2e"][0] / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": r["e2e"][1], "d2h_bytes_per_step": r["e2e"][2]},
+            "gpu_launches": r["launches"],
+            "clocks": r["clocks"],
+            "device_status": r["status"],
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+def kernel_hash():
+    """Hash of the attention kernel source; ncu traffic figures apply only to it."""
+    import hashlib
+    with open(os.path.join(ROOT, "paged_kv_cache_440_b200", "csrc", "attn_decode.cu"), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,317 @@
+/*
+ * pagedkv.h -- C ABI of a paged KV-cache library for single-token decode on
+ * NVIDIA B200 (sm_100a).
+ *
+ * What the library does, and where the operations are defined:
+ *
+ *   The KV cache of every sequence is cut into fixed-size blocks of
+ *   block_size tokens that live anywhere in one preallocated pool; a per-sequence
+ *   block table maps logical block i to physical block p; blocks are handed out
+ *   on demand and returned when done; attention gathers the scattered blocks
+ *   back into the logical sequence.
+ *     [KV Cache 原理与 PagedAttention, §三 "工作方式" 1-4;
+ *      aiworkagent.org q17, "Block Table", "Block Size", "KV Memory Pool"]
+ *   Each decode step computes only the new token's K and V and appends them to
+ *   the cache; the new query attends over every cached token.
+ *     [KV Cache 原理与 PagedAttention, §一; bjdmk.com.cn/news/6246348, §2.1]
+ *   Attention is softmax(q K^T * scale) V; several query heads may share one
+ *   KV head (GQA / MQA).
+ *     [bjdmk.com.cn/news/6246348, §2.1; KV Cache 原理与 PagedAttention, §一 GQA/MQA]
+ *   Requests with a common prefix share its physical blocks; a write into a
+ *   shared block first copies it (copy-on-write).
+ *     [bjdmk.com.cn/news/6246348, §3.2]
+ *   The cache may be stored as INT8 or FP8-E5M2 with one fp32 scale per
+ *   (token, KV head), dequantized inside the attention kernel.
+ *     [KV Cache 原理与 PagedAttention, §四; bjdmk.com.cn/news/6246348, §5.2, §5.3]
+ *
+ * Conventions for every call:
+ *   - Device pointers are borrowed. The caller allocates all device memory
+ *     (the pool, inputs, outputs, split-K workspace) and keeps it alive until
+ *     the work queued on the stream has finished. No call allocates device memory.
+ *   - Device work is queued on the given stream; calls return after enqueueing.
+ *     A launch failure returns KV_ERR_CUDA.
+ *   - Arguments are validated on the host before anything is queued; a
+ *     rejected call queues nothing and returns KV_ERR_INVALID or
+ *     KV_ERR_UNSUPPORTED. kv_last_error() then describes the problem.
+ *   - Values only the device can see (block ids read from a block table,
+ *     context lengths, slots) are range-checked in the kernels. A bad value
+ *     never causes an out-of-bounds access: the affected row is skipped (append)
+ *     or contributes nothing (attention), and a bit is set in the pool's device
+ *     status word (see kv_pool_status).
+ *   - Tensors are dense and row-major; the shapes below list dimensions from
+ *     outermost to innermost.
+ */
+#ifndef PAGEDKV_H
+#define PAGEDKV_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; 0 is the legacy default stream. */
+typedef struct CUstream_st *kv_stream_t;
+
+typedef enum {
+  KV_OK = 0,
+  KV_ERR_INVALID = 1,      /* bad argument (null pointer, out-of-range id, ...) */
+  KV_ERR_OOM = 2,          /* the block pool has fewer free blocks than asked   */
+  KV_ERR_CUDA = 3,         /* a CUDA runtime call or kernel launch failed       */
+  KV_ERR_UNSUPPORTED = 4   /* valid but not implemented (e.g. head_dim 96)      */
+} kv_status;
+
+typedef enum {
+  KV_BF16 = 0,
+  KV_FP16 = 1,
+  KV_FP8_E5M2 = 2,         /* 1 sign, 5 exponent (bias 15), 2 mantissa bits     */
+  KV_INT8 = 3              /* two's complement, codes in [-127, 127]            */
+} kv_dtype;
+
+/* Bits of the device status word. */
+enum {
+  KV_DEVERR_BLOCK_ID = 1,  /* a block-table entry outside [0, num_blocks)        */
+  KV_DEVERR_CONTEXT = 2,   /* a context length < 0 or beyond the table/maximum   */
+  KV_DEVERR_SLOT = 4,      /* a slot >= num_blocks * block_size                  */
+  KV_DEVERR_TIMEOUT = 8    /* a kernel gave up waiting for its own tile loads    */
+};
+
+typedef struct {
+  int32_t num_layers;      /* >= 1                                              */
+  int32_t num_blocks;      /* physical blocks per layer, >= 1                   */
+  int32_t block_size;      /* tokens per block: 16 or 32                        */
+  int32_t num_kv_heads;    /* >= 1                                              */
+  int32_t head_dim;        /* 64 or 128                                         */
+  int32_t cache_dtype;     /* a kv_dtype                                        */
+} kv_pool_desc;
+
+typedef struct kv_pool kv_pool;   /* opaque host object */
+
+/* ------------------------------------------------------------------------ */
+/* Pool                                                                      */
+/* ------------------------------------------------------------------------ */
+
+/* Bytes of device memory a pool with this description needs.
+ *
+ * Layout of the caller's buffer, for each layer in order, every region
+ * starting on a 256-byte boundary:
+ *   K       [num_blocks][num_kv_heads][block_size][head_dim]  cache_dtype
+ *   V       same
+ *   K scale [num_blocks][num_kv_heads][block_size]  fp32   (INT8 / E5M2 only)
+ *   V scale same                                            (INT8 / E5M2 only)
+ * followed by one 256-byte status region. One (block, head) tile of K or V is
+ * contiguous (block_size * head_dim elements). K and V of a layer take exactly
+ * 2 * num_kv_heads * head_dim * elem_bytes * (num_blocks * block_size) bytes,
+ * the per-layer KV size formula of the pages applied to the pool's capacity
+ * [KV Cache 原理与 PagedAttention, §一 "显存占用公式"].
+ * Errors: KV_ERR_INVALID for a null pointer or a non-positive size field,
+ * KV_ERR_UNSUPPORTED for a block_size, head_dim or dtype outside the lists above. */
+kv_status kv_pool_required_bytes(const kv_pool_desc *desc, uint64_t *bytes);
+
+/* Create the host-side pool object over a caller-owned device buffer.
+ * device_base: 256-byte aligned device pointer to >= kv_pool_required_bytes
+ * bytes; borrowed, never freed by the library. Its contents are not touched;
+ * the caller zeroes the status region (kv_pool_status_clear) before first use.
+ * All blocks start free (refcount 0).
+ * Errors: KV_ERR_INVALID (null, misaligned, too small), KV_ERR_UNSUPPORTED. */
+kv_status kv_pool_create(const kv_pool_desc *desc, void *device_base,
+                         uint64_t bytes, kv_pool **out);
+
+/* Free the host object. Does not touch device memory. */
+kv_status kv_pool_destroy(kv_pool *pool);
+
+/* Device addresses of one layer's regions. k_scale / v_scale are set to NULL
+ * for 16-bit caches. Any output pointer may be NULL if not wanted. */
+kv_status kv_pool_layer_ptrs(const kv_pool *pool, int32_t layer, void **k,
+                             void **v, float **k_scale, float **v_scale);
+
+/* Device address of the pool's int32 status word (bits KV_DEVERR_*). */
+kv_status kv_pool_status_ptr(const kv_pool *pool, int32_t **status);
+
+/* Queue a reset of the status word to 0 on the stream. */
+kv_status kv_pool_status_clear(kv_pool *pool, kv_stream_t stream);
+
+/* Copy the status word to *host_bits after the stream's queued work has
+ * finished (synchronizes the stream). */
+kv_status kv_pool_status(kv_pool *pool, kv_stream_t stream, int32_t *host_bits);
+
+/* ------------------------------------------------------------------------ */
+/* Host block allocator with reference counts                                */
+/* [KV Cache 原理与 PagedAttention, §三 "工作方式" 3; bjdmk.com.cn/news/6246348,   */
+/*  §3.1-§3.2]. Thread-safe; no device work.                                  */
+/* ------------------------------------------------------------------------ */
+
+/* Take n free blocks (refcount 0 -> 1) and write their ids to out_ids[0..n).
+ * KV_ERR_OOM, with nothing taken, when fewer than n blocks are free. */
+kv_status kv_alloc_blocks(kv_pool *pool, int32_t n, int32_t *out_ids);
+
+/* Drop one reference from each listed block; a block reaching 0 is free again.
+ * KV_ERR_INVALID, with nothing changed, if any id is out of range or free. */
+kv_status kv_free_blocks(kv_pool *pool, int32_t n, const int32_t *ids);
+
+/* Add one reference to each listed (allocated) block: sharing a prefix, or
+ * forking a sequence. KV_ERR_INVALID, nothing changed, for a free/bad id. */
+kv_status kv_share_blocks(kv_pool *pool, int32_t n, const int32_t *ids);
+
+/* Before writing into `block`: if it is shared (refcount > 1), take a fresh
+ * block, drop one reference from `block`, and return the fresh id in
+ * *new_block; the caller then copies the contents with kv_block_copy and
+ * points its block table at the copy. If the block is exclusively owned,
+ * *new_block = block and nothing changes. KV_ERR_OOM when no block is free. */
+kv_status kv_cow_prepare(kv_pool *pool, int32_t block, int32_t *new_block);
+
+/* Current reference count of one block. */
+kv_status kv_block_refcount(const kv_pool *pool, int32_t block, int32_t *ref);
+
+/* used = blocks with refcount >= 1, free_ = refcount 0, shared = refcount >= 2
+ * (the cache-usage figures a serving system monitors
+ * [KV Cache 原理与 PagedAttention, §六]). Any pointer may be NULL. */
+kv_status kv_pool_stats(const kv_pool *pool, int32_t *used, int32_t *free_,
+                        int32_t *shared);
+
+/* ------------------------------------------------------------------------ */
+/* Append (reshape_and_cache), quantize, copy-on-write block copy           */
+/* ------------------------------------------------------------------------ */
+
+/* Write each new token's K and V rows into the slot it maps to.
+ * k_new, v_new: device [num_tokens][num_kv_heads][head_dim] of in_dtype
+ *   (KV_BF16 or KV_FP16), 16-byte aligned.
+ * slot_mapping: device int64 [num_tokens]; slot = physical_block * block_size
+ *   + row. A negative slot skips the token; a slot >= num_blocks * block_size
+ *   skips it and sets KV_DEVERR_SLOT. Slots must be distinct (duplicates race).
+ * 16-bit caches: in_dtype must equal the cache dtype; the rows are copied
+ *   bit for bit.
+ * INT8 / E5M2 caches: each (token, head) row x of head_dim values is
+ *   quantized as kv_quantize does and its code row and fp32 scale are stored.
+ * Errors: KV_ERR_INVALID (bad layer, null, misaligned, num_tokens < 0),
+ *   KV_ERR_UNSUPPORTED (dtype combination), KV_ERR_CUDA. */
+kv_status kv_append(kv_pool *pool, int32_t layer, const void *k_new,
+                    const void *v_new, int32_t in_dtype,
+                    const int64_t *slot_mapping, int32_t num_tokens,
+                    kv_stream_t stream);
+
+/* Per-row symmetric absmax quantization [bjdmk.com.cn/news/6246348, §5.2:
+ * one scale per token per head]:
+ *   a = max|x|; scale = fl32(a / QMAX) (QMAX 127 for INT8, 57344 for E5M2);
+ *   code = round-half-even(fl32(x / scale)), clamped to [-127, 127] (INT8) or
+ *   rounded to E5M2 with saturation to +-57344; a == 0 gives scale 0, codes 0.
+ *   Both divisions are IEEE fp32 divisions, so results are bit-reproducible.
+ * x: device [rows][head_dim] of in_dtype (BF16 / FP16), 16-byte aligned.
+ * codes: device [rows][head_dim] bytes; scales: device fp32 [rows].
+ * head_dim: 64 or 128. out_dtype: KV_INT8 or KV_FP8_E5M2. */
+kv_status kv_quantize(const void *x, int32_t in_dtype, int64_t rows,
+                      int32_t head_dim, int32_t out_dtype, void *codes,
+                      float *scales, kv_stream_t stream);
+
+/* Copy whole physical blocks, every layer, K and V (and the scales of a
+ * quantized cache): block dst := block src for each pair
+ * [bjdmk.com.cn/news/6246348, §3.2, copy-on-write].
+ * host_pairs: HOST int32 [n_pairs][2] = {src, dst}. The pairs must be
+ * disjoint: src != dst, no dst repeated, no dst that is also a src, all ids in
+ * [0, num_blocks); otherwise KV_ERR_INVALID and nothing is queued. The pair
+ * list is passed to the kernel by value (no device staging buffer). */
+kv_status kv_block_copy(kv_pool *pool, const int32_t *host_pairs,
+                        int32_t n_pairs, kv_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Paged decode attention                                                    */
+/* ------------------------------------------------------------------------ */
+/*
+ * For sequence b (context length L_b, block table row bt[b]) and query head h,
+ * with g = h / (num_q_heads / num_kv_heads):
+ *   out[b][h] = sum_t softmax_t(scale * q[b][h] . K_g[t]) V_g[t],  t in [0, L_b)
+ * where position t lives in row t % block_size of physical block
+ * bt[b][t / block_size]. L_b = 0 gives a zero output. For INT8 / E5M2 caches,
+ * K_g[t] = code * k_scale and V_g[t] = code * v_scale (dequantized in-kernel).
+ * [bjdmk.com.cn/news/6246348, §2.1; KV Cache 原理与 PagedAttention, §三 工作方式 4]
+ *
+ * Long contexts are split into partitions of partition_tokens tokens
+ * (split-K). Each partition is reduced by one CTA per (sequence, KV head,
+ * partition) to a running max m, a sum l and an unnormalized output o; a
+ * merge combines them: out = sum_p e^(m_p - M) o_p / sum_p e^(m_p - M) l_p,
+ * M = max_p m_p. Sequences with one partition are written directly.
+ *
+ * Common arguments:
+ *   q       device [num_seqs][num_q_heads][head_dim], q_dtype, 16-byte aligned.
+ *           16-bit caches need q_dtype == cache dtype; INT8/E5M2 caches take
+ *           KV_BF16 or KV_FP16 queries.
+ *   out     device [num_seqs][num_q_heads][head_dim], q_dtype, 16-byte aligned.
+ *   block_tables  device int32 [num_seqs][max_blocks_per_seq].
+ *   context_lens  device int32 [num_seqs]; each must satisfy
+ *           0 <= L_b <= min(max_context, max_blocks_per_seq * block_size),
+ *           else KV_DEVERR_CONTEXT is set and that sequence's output is 0.
+ *   max_context   host upper bound on every L_b; sizes the workspace.
+ *   partition_tokens  0 = library default, else a positive multiple of
+ *           block_size.
+ *   workspace     device, 256-byte aligned, >= paged_attn_workspace_bytes
+ *           bytes (may be NULL when that size is 0). Holds the per-partition
+ *           (m, l, o) in fp32 between the two phases; its contents are
+ *           scratch and need no initialisation.
+ */
+
+/* Workspace bytes paged_attn_decode / paged_attn_partition / paged_attn_merge
+ * need for these sizes (0 when every sequence fits one partition). */
+kv_status paged_attn_workspace_bytes(const kv_pool *pool, int32_t num_seqs,
+                                     int32_t num_q_heads, int32_t max_context,
+                                     int32_t partition_tokens, uint64_t *bytes);
+
+/* The partition size the library uses for these arguments when
+ * partition_tokens is 0. */
+kv_status paged_attn_default_partition(const kv_pool *pool, int32_t num_seqs,
+                                       int32_t num_q_heads, int32_t max_context,
+                                       int32_t *partition_tokens);
+
+/* Full decode attention: paged_attn_partition followed, when any sequence can
+ * span more than one partition, by paged_attn_merge, on the same stream. */
+kv_status paged_attn_decode(kv_pool *pool, int32_t layer, const void *q,
+                            int32_t q_dtype, int32_t num_seqs,
+                            int32_t num_q_heads, const int32_t *block_tables,
+                            int32_t max_blocks_per_seq,
+                            const int32_t *context_lens, int32_t max_context,
+                            float scale, void *out, int32_t partition_tokens,
+                            void *workspace, uint64_t workspace_bytes,
+                            kv_stream_t stream);
+
+/* Phase 1 alone: one CTA per (sequence, KV head, partition). Writes out[b]
+ * for sequences with a single partition and the workspace partials for the
+ * others. */
+kv_status paged_attn_partition(kv_pool *pool, int32_t layer, const void *q,
+                               int32_t q_dtype, int32_t num_seqs,
+                               int32_t num_q_heads, const int32_t *block_tables,
+                               int32_t max_blocks_per_seq,
+                               const int32_t *context_lens, int32_t max_context,
+                               float scale, void *out, int32_t partition_tokens,
+                               void *workspace, uint64_t workspace_bytes,
+                               kv_stream_t stream);
+
+/* Phase 2 alone: merge the partials of sequences with more than one
+ * partition into out (q_dtype). Same argument meanings as phase 1. */
+kv_status paged_attn_merge(const kv_pool *pool, int32_t num_seqs,
+                           int32_t num_q_heads, const int32_t *context_lens,
+                           int32_t max_blocks_per_seq, int32_t max_context,
+                           int32_t partition_tokens, int32_t out_dtype,
+                           void *out, const void *workspace,
+                           uint64_t workspace_bytes, kv_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+
+/* Failure-path self-test: launch one thread that waits on a shared-memory
+ * barrier nothing completes, using the same bounded wait as the attention
+ * kernel. After limit_us microseconds (1 .. 1e6) it gives up, ORs
+ * KV_DEVERR_TIMEOUT into *device_status (device int32) and exits; the
+ * context stays usable. No counterpart on the pages: it tests this library's
+ * own failure detection. */
+kv_status kv_selftest_wait_timeout(int32_t *device_status, uint32_t limit_us,
+                                   kv_stream_t stream);
+
+/* Message for the last non-OK status returned on this thread ("" if none). */
+const char *kv_last_error(void);
+
+/* Library version string. */
+const char *kv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDKV_H */

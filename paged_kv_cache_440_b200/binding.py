@@ -1,0 +1,345 @@
+"""ctypes binding of libpagedkv.so (the C ABI declared in include/pagedkv.h).
+
+Argument marshalling only: every computation runs in the library's CUDA
+kernels. torch supplies device memory and the current stream. Importing this
+module raises ImportError when the compiled library is missing; there is no
+fallback path.
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpagedkv.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        "libpagedkv.so is not built (expected at %s); run "
+        "`python -m paged_kv_cache_440_b200.build`" % LIB_PATH)
+
+lib = ctypes.CDLL(LIB_PATH)
+
+# ----------------------------------------------------------------- constants
+KV_OK, KV_ERR_INVALID, KV_ERR_OOM, KV_ERR_CUDA, KV_ERR_UNSUPPORTED = 0, 1, 2, 3, 4
+KV_BF16, KV_FP16, KV_FP8_E5M2, KV_INT8 = 0, 1, 2, 3
+KV_DEVERR_BLOCK_ID, KV_DEVERR_CONTEXT, KV_DEVERR_SLOT, KV_DEVERR_TIMEOUT = 1, 2, 4, 8
+
+DTYPE_CODES = {"bf16": KV_BF16, "fp16": KV_FP16, "e5m2": KV_FP8_E5M2, "int8": KV_INT8}
+TORCH_CODES = {torch.bfloat16: KV_BF16, torch.float16: KV_FP16}
+CACHE_TORCH = {"bf16": torch.bfloat16, "fp16": torch.float16, "e5m2": torch.uint8,
+               "int8": torch.int8}
+
+
+class PoolDesc(ctypes.Structure):
+    _fields_ = [("num_layers", ctypes.c_int32), ("num_blocks", ctypes.c_int32),
+                ("block_size", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("cache_dtype", ctypes.c_int32)]
+
+
+_P = ctypes.c_void_p
+_I32 = ctypes.c_int32
+_I64 = ctypes.c_int64
+_U64 = ctypes.c_uint64
+_PI32 = ctypes.POINTER(ctypes.c_int32)
+_PU64 = ctypes.POINTER(ctypes.c_uint64)
+_F = ctypes.c_float
+
+_SIGS = {
+    "kv_pool_required_bytes": [ctypes.POINTER(PoolDesc), _PU64],
+    "kv_pool_create": [ctypes.POINTER(PoolDesc), _P, _U64, ctypes.POINTER(_P)],
+    "kv_pool_destroy": [_P],
+    "kv_pool_layer_ptrs": [_P, _I32, ctypes.POINTER(_P), ctypes.POINTER(_P),
+                           ctypes.POINTER(_P), ctypes.POINTER(_P)],
+    "kv_pool_status_ptr": [_P, ctypes.POINTER(_P)],
+    "kv_pool_status_clear": [_P, _P],
+    "kv_pool_status": [_P, _P, _PI32],
+    "kv_alloc_blocks": [_P, _I32, _PI32],
+    "kv_free_blocks": [_P, _I32, _PI32],
+    "kv_share_blocks": [_P, _I32, _PI32],
+    "kv_cow_prepare": [_P, _I32, _PI32],
+    "kv_block_refcount": [_P, _I32, _PI32],
+    "kv_pool_stats": [_P, _PI32, _PI32, _PI32],
+    "kv_append": [_P, _I32, _P, _P, _I32, _P, _I32, _P],
+    "kv_quantize": [_P, _I32, _I64, _I32, _I32, _P, _P, _P],
+    "kv_block_copy": [_P, _PI32, _I32, _P],
+    "paged_attn_workspace_bytes": [_P, _I32, _I32, _I32, _I32, _PU64],
+    "paged_attn_default_partition": [_P, _I32, _I32, _I32, _PI32],
+    "paged_attn_decode": [_P, _I32, _P, _I32, _I32, _I32, _P, _I32, _P, _I32, _F, _P, _I32,
+                          _P, _U64, _P],
+    "paged_attn_partition": [_P, _I32, _P, _I32, _I32, _I32, _P, _I32, _P, _I32, _F, _P,
+                             _I32, _P, _U64, _P],
+    "paged_attn_merge": [_P, _I32, _I32, _P, _I32, _I32, _I32, _I32, _P, _P, _U64, _P],
+    "kv_selftest_wait_timeout": [_P, ctypes.c_uint32, _P],
+}
+for _name, _args in _SIGS.items():
+    _fn = getattr(lib, _name)
+    _fn.argtypes = _args
+    _fn.restype = ctypes.c_int
+lib.kv_last_error.argtypes = []
+lib.kv_last_error.restype = ctypes.c_char_p
+lib.kv_version.argtypes = []
+lib.kv_version.restype = ctypes.c_char_p
+
+
+class PagedKVError(RuntimeError):
+    def __init__(self, status, message):
+        super().__init__("pagedkv status %d: %s" % (status, message))
+        self.status = status
+
+
+def check(status):
+    if status != KV_OK:
+        raise PagedKVError(status, lib.kv_last_error().decode(errors="replace"))
+
+
+def _stream(stream=None, device=None):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t, name, dtype=None, device=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch.Tensor" % name)
+    if not t.is_cuda:
+        raise ValueError("%s must be on a CUDA device" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise ValueError("%s has dtype %s, expected %s" % (name, t.dtype, dtype))
+    if device is not None and t.device != device:
+        raise ValueError("%s is on %s, expected %s" % (name, t.device, device))
+
+
+def required_bytes(num_layers, num_blocks, block_size, num_kv_heads, head_dim, cache_dtype):
+    d = PoolDesc(num_layers, num_blocks, block_size, num_kv_heads, head_dim,
+                 DTYPE_CODES[cache_dtype])
+    n = ctypes.c_uint64()
+    check(lib.kv_pool_required_bytes(ctypes.byref(d), ctypes.byref(n)))
+    return n.value
+
+
+class KVPool:
+    """A block pool over one torch-allocated device buffer (held by this object)."""
+
+    def __init__(self, num_layers, num_blocks, block_size, num_kv_heads, head_dim,
+                 cache_dtype="bf16", device="cuda"):
+        self.desc = PoolDesc(num_layers, num_blocks, block_size, num_kv_heads, head_dim,
+                             DTYPE_CODES[cache_dtype])
+        self.cache_dtype = cache_dtype
+        self.device = torch.device(device)
+        nbytes = required_bytes(num_layers, num_blocks, block_size, num_kv_heads, head_dim,
+                                cache_dtype)
+        self.buffer = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        h = ctypes.c_void_p()
+        check(lib.kv_pool_create(ctypes.byref(self.desc), _ptr(self.buffer), nbytes,
+                                 ctypes.byref(h)))
+        self.handle = h
+        self.status_clear()
+
+    # geometry
+    num_layers = property(lambda s: s.desc.num_layers)
+    num_blocks = property(lambda s: s.desc.num_blocks)
+    block_size = property(lambda s: s.desc.block_size)
+    num_kv_heads = property(lambda s: s.desc.num_kv_heads)
+    head_dim = property(lambda s: s.desc.head_dim)
+    quantized = property(lambda s: s.cache_dtype in ("int8", "e5m2"))
+
+    def close(self):
+        if getattr(self, "handle", None):
+            lib.kv_pool_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def layer_ptrs(self, layer):
+        k, v, ks, vs = (ctypes.c_void_p() for _ in range(4))
+        check(lib.kv_pool_layer_ptrs(self.handle, layer, ctypes.byref(k), ctypes.byref(v),
+                                     ctypes.byref(ks), ctypes.byref(vs)))
+        return k.value, v.value, ks.value, vs.value
+
+    def _view(self, addr, nbytes, dtype, shape):
+        off = addr - self.buffer.data_ptr()
+        return self.buffer[off:off + nbytes].view(dtype).view(shape)
+
+    def layer_views(self, layer):
+        """(K, V, K_scale, V_scale) torch views of one layer's regions."""
+        k, v, ks, vs = self.layer_ptrs(layer)
+        shape = (self.num_blocks, self.num_kv_heads, self.block_size, self.head_dim)
+        dt = CACHE_TORCH[self.cache_dtype]
+        elt = 2 if self.cache_dtype in ("bf16", "fp16") else 1
+        n = self.num_blocks * self.num_kv_heads * self.block_size
+        K = self._view(k, n * self.head_dim * elt, dt, shape)
+        V = self._view(v, n * self.head_dim * elt, dt, shape)
+        if ks is None:
+            return K, V, None, None
+        sshape = shape[:3]
+        return K, V, self._view(ks, n * 4, torch.float32, sshape), \
+            self._view(vs, n * 4, torch.float32, sshape)
+
+    # status word
+    def status_clear(self, stream=None):
+        check(lib.kv_pool_status_clear(self.handle, _stream(stream, self.device)))
+
+    def status(self, stream=None):
+        v = ctypes.c_int32()
+        check(lib.kv_pool_status(self.handle, _stream(stream, self.device), ctypes.byref(v)))
+        return v.value
+
+    # allocator
+    def alloc(self, n):
+        ids = (ctypes.c_int32 * max(n, 1))()
+        check(lib.kv_alloc_blocks(self.handle, n, ids))
+        return list(ids[:n])
+
+    def free(self, ids):
+        arr = (ctypes.c_int32 * max(len(ids), 1))(*ids)
+        check(lib.kv_free_blocks(self.handle, len(ids), arr))
+
+    def share(self, ids):
+        arr = (ctypes.c_int32 * max(len(ids), 1))(*ids)
+        check(lib.kv_share_blocks(self.handle, len(ids), arr))
+
+    def cow_prepare(self, block):
+        out = ctypes.c_int32()
+        check(lib.kv_cow_prepare(self.handle, block, ctypes.byref(out)))
+        return out.value
+
+    def refcount(self, block):
+        out = ctypes.c_int32()
+        check(lib.kv_block_refcount(self.handle, block, ctypes.byref(out)))
+        return out.value
+
+    def stats(self):
+        u, f, s = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+        check(lib.kv_pool_stats(self.handle, ctypes.byref(u), ctypes.byref(f), ctypes.byref(s)))
+        return {"used": u.value, "free": f.value, "shared": s.value}
+
+
+# ------------------------------------------------------------------ ops
+
+def kv_append(pool, layer, k_new, v_new, slot_mapping, stream=None):
+    """Write k_new/v_new [T, Hkv, D] rows to their slots (int64 [T])."""
+    _need(k_new, "k_new", (torch.bfloat16, torch.float16), pool.device)
+    _need(v_new, "v_new", k_new.dtype, pool.device)
+    _need(slot_mapping, "slot_mapping", torch.int64, pool.device)
+    T = k_new.shape[0]
+    if tuple(k_new.shape) != (T, pool.num_kv_heads, pool.head_dim) or v_new.shape != k_new.shape \
+            or slot_mapping.shape != (T,):
+        raise ValueError("k_new, v_new must be [T, kv_heads, head_dim], slot_mapping [T]")
+    check(lib.kv_append(pool.handle, layer, _ptr(k_new), _ptr(v_new), TORCH_CODES[k_new.dtype],
+                        _ptr(slot_mapping), T, _stream(stream, pool.device)))
+
+
+def kv_quantize(x, kind, codes=None, scales=None, stream=None):
+    """Per-row absmax quantization of x [..., D] -> (codes [..., D], fp32 scales [...])."""
+    _need(x, "x", (torch.bfloat16, torch.float16))
+    D = x.shape[-1]
+    rows = x.numel() // D if D else 0
+    if codes is None:
+        codes = torch.empty(x.shape, dtype=CACHE_TORCH[kind], device=x.device)
+    if scales is None:
+        scales = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device)
+    _need(codes, "codes", CACHE_TORCH[kind], x.device)
+    _need(scales, "scales", torch.float32, x.device)
+    check(lib.kv_quantize(_ptr(x), TORCH_CODES[x.dtype], rows, D, DTYPE_CODES[kind],
+                          _ptr(codes), _ptr(scales), _stream(stream, x.device)))
+    return codes, scales
+
+
+def kv_block_copy(pool, pairs, stream=None):
+    """Copy whole blocks src -> dst (all layers). pairs: iterable of (src, dst)."""
+    flat = [int(v) for pr in pairs for v in pr]
+    n = len(flat) // 2
+    arr = (ctypes.c_int32 * max(len(flat), 1))(*flat)
+    check(lib.kv_block_copy(pool.handle, arr, n, _stream(stream, pool.device)))
+
+
+def workspace_bytes(pool, num_seqs, num_q_heads, max_context, partition_tokens=0):
+    n = ctypes.c_uint64()
+    check(lib.paged_attn_workspace_bytes(pool.handle, num_seqs, num_q_heads, max_context,
+                                         partition_tokens, ctypes.byref(n)))
+    return n.value
+
+
+def default_partition(pool, num_seqs, num_q_heads, max_context):
+    n = ctypes.c_int32()
+    check(lib.paged_attn_default_partition(pool.handle, num_seqs, num_q_heads, max_context,
+                                           ctypes.byref(n)))
+    return n.value
+
+
+def make_workspace(pool, num_seqs, num_q_heads, max_context, partition_tokens=0):
+    n = workspace_bytes(pool, num_seqs, num_q_heads, max_context, partition_tokens)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=pool.device)
+
+
+def _attn_args(pool, q, block_tables, context_lens, out):
+    _need(q, "q", (torch.bfloat16, torch.float16), pool.device)
+    _need(block_tables, "block_tables", torch.int32, pool.device)
+    _need(context_lens, "context_lens", torch.int32, pool.device)
+    B, Hq, D = q.shape
+    if D != pool.head_dim or block_tables.dim() != 2 or block_tables.shape[0] != B \
+            or context_lens.shape != (B,):
+        raise ValueError("q [B, Hq, D], block_tables [B, max_blocks], context_lens [B]")
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", q.dtype, pool.device)
+    if out.shape != q.shape:
+        raise ValueError("out must have q's shape")
+    return B, Hq, out
+
+
+def paged_attn_decode(pool, layer, q, block_tables, context_lens, max_context, scale,
+                      out=None, partition_tokens=0, workspace=None, stream=None):
+    """Decode attention of q [B, Hq, D] over the paged cache; returns out."""
+    B, Hq, out = _attn_args(pool, q, block_tables, context_lens, out)
+    if workspace is None:
+        workspace = make_workspace(pool, B, Hq, max_context, partition_tokens)
+    check(lib.paged_attn_decode(pool.handle, layer, _ptr(q), TORCH_CODES[q.dtype], B, Hq,
+                                _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
+                                max_context, float(scale), _ptr(out), partition_tokens,
+                                _ptr(workspace), workspace.numel(), _stream(stream, pool.device)))
+    return out
+
+
+def paged_attn_partition(pool, layer, q, block_tables, context_lens, max_context, scale,
+                         out, workspace, partition_tokens=0, stream=None):
+    B, Hq, out = _attn_args(pool, q, block_tables, context_lens, out)
+    check(lib.paged_attn_partition(pool.handle, layer, _ptr(q), TORCH_CODES[q.dtype], B, Hq,
+                                   _ptr(block_tables), block_tables.shape[1],
+                                   _ptr(context_lens), max_context, float(scale), _ptr(out),
+                                   partition_tokens, _ptr(workspace), workspace.numel(),
+                                   _stream(stream, pool.device)))
+    return out
+
+
+def paged_attn_merge(pool, context_lens, max_blocks_per_seq, max_context, out, workspace,
+                     partition_tokens=0, stream=None):
+    _need(out, "out", (torch.bfloat16, torch.float16), pool.device)
+    _need(context_lens, "context_lens", torch.int32, pool.device)
+    B, Hq, _ = out.shape
+    check(lib.paged_attn_merge(pool.handle, B, Hq, _ptr(context_lens), max_blocks_per_seq,
+                               max_context, partition_tokens, TORCH_CODES[out.dtype], _ptr(out),
+                               _ptr(workspace), workspace.numel(),
+                               _stream(stream, pool.device)))
+    return out
+
+
+def selftest_wait_timeout(status, limit_us=1000, stream=None):
+    """Run the bounded-wait self-test; status is a device int32 tensor [1]."""
+    _need(status, "status", torch.int32)
+    check(lib.kv_selftest_wait_timeout(_ptr(status), limit_us, _stream(stream, status.device)))
+
+
+def version():
+    return lib.kv_version().decode()

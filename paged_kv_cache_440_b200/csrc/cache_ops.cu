@@ -1,0 +1,376 @@
+// Append (reshape_and_cache), per-token-head quantization and copy-on-write
+// block copy.
+//
+// * Append: a decode step computes only the new token's K and V and puts them
+//   at the end of its sequence's cache [KV Cache 原理与 PagedAttention, §一;
+//   bjdmk.com.cn/news/6246348, §2.1]; in a paged cache that end is row
+//   slot % block_size of physical block slot / block_size.
+// * Quantize: symmetric absmax per (token, head) row, fp32 scale
+//   [bjdmk.com.cn/news/6246348, §5.2]; INT8 or FP8-E5M2 codes
+//   [KV Cache 原理与 PagedAttention, §四].
+// * Block copy: the copy half of copy-on-write [bjdmk.com.cn/news/6246348,
+//   §3.2]: whole blocks, every layer, K, V and scales.
+//
+// All three are pure data movement at a few hundred KB per decode step; each
+// warp handles one row (or one block) with 16-byte vector accesses.
+#include <cstring>
+#include <vector>
+
+#include "device.cuh"
+#include "internal.h"
+
+namespace pagedkv {
+namespace {
+
+using namespace dev;
+
+constexpr int kWarpsPerCta = 8;
+
+template <int IN_T>
+__device__ __forceinline__ float to_f32(uint16_t bits) {
+  if constexpr (IN_T == KV_BF16) {
+    return __uint_as_float(static_cast<uint32_t>(bits) << 16);
+  } else {
+    return __half2float(__ushort_as_half(bits));
+  }
+}
+
+// ---------------------------------------------------------------- 16-bit copy
+
+// One warp per (token, kv head): lanes [0, 16) copy the K row, [16, 32) the V
+// row, 16 bytes each (row_bytes <= 256).
+__global__ void __launch_bounds__(kWarpsPerCta * 32)
+append16_kernel(const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new,
+                const int64_t *__restrict__ slots, int num_tokens, int kv_heads,
+                int block_size, int row_chunks, int64_t num_slots, char *__restrict__ kc,
+                char *__restrict__ vc, int *status) {
+  const int warp = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (warp >= num_tokens * kv_heads) return;
+  const int t = warp / kv_heads;
+  const int h = warp - t * kv_heads;
+  const int64_t slot = slots[t];
+  if (slot < 0) return;
+  if (slot >= num_slots) {
+    if (lane == 0 && h == 0) atomicOr(status, kErrSlot);
+    return;
+  }
+  const int64_t blk = slot / block_size;
+  const int row = static_cast<int>(slot - blk * block_size);
+  const int64_t dst_row = (blk * kv_heads + h) * block_size + row;
+  const int c = lane & 15;
+  if (c >= row_chunks) return;
+  const int64_t src_row = static_cast<int64_t>(t) * kv_heads + h;
+  if (lane < 16) {
+    uint4 x = k_new[src_row * row_chunks + c];
+    reinterpret_cast<uint4 *>(kc)[dst_row * row_chunks + c] = x;
+  } else {
+    uint4 x = v_new[src_row * row_chunks + c];
+    reinterpret_cast<uint4 *>(vc)[dst_row * row_chunks + c] = x;
+  }
+}
+
+// ---------------------------------------------------------------- quantize
+
+// Quantize one row of D values held as D/32 per lane; returns the packed codes
+// of this lane (D/32 bytes, little-endian in order) and the row scale.
+template <int D, int OUT_T>
+__device__ __forceinline__ uint32_t quantize_row(const float (&x)[D / 32], float *scale_out) {
+  constexpr int E = D / 32;
+  float a = 0.f;
+#pragma unroll
+  for (int i = 0; i < E; ++i) a = fmaxf(a, fabsf(x[i]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+  constexpr float kQmax = OUT_T == KV_INT8 ? 127.0f : 57344.0f;
+  uint32_t packed = 0;
+  float scale = 0.f;
+  if (a > 0.f) {
+    scale = __fdiv_rn(a, kQmax);
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+      const float y = __fdiv_rn(x[i], scale);
+      uint32_t code;
+      if constexpr (OUT_T == KV_INT8) {
+        int q = __float2int_rn(y);
+        q = max(-127, min(127, q));
+        code = static_cast<uint32_t>(q) & 0xFFu;
+      } else {
+        code = static_cast<uint32_t>(__nv_cvt_float_to_fp8(y, __NV_SATFINITE, __NV_E5M2));
+      }
+      packed |= code << (8 * i);
+    }
+  }
+  *scale_out = scale;
+  return packed;
+}
+
+template <int D, int IN_T>
+__device__ __forceinline__ void load_row(const uint16_t *__restrict__ src, int lane,
+                                         float (&x)[D / 32]) {
+  constexpr int E = D / 32;
+  if constexpr (E == 4) {
+    uint2 v = *reinterpret_cast<const uint2 *>(src + lane * 4);
+    x[0] = to_f32<IN_T>(v.x & 0xFFFF);
+    x[1] = to_f32<IN_T>(v.x >> 16);
+    x[2] = to_f32<IN_T>(v.y & 0xFFFF);
+    x[3] = to_f32<IN_T>(v.y >> 16);
+  } else {
+    uint32_t v = *reinterpret_cast<const uint32_t *>(src + lane * 2);
+    x[0] = to_f32<IN_T>(v & 0xFFFF);
+    x[1] = to_f32<IN_T>(v >> 16);
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void store_codes(uint8_t *dst, int lane, uint32_t packed) {
+  if constexpr (D == 128) {
+    reinterpret_cast<uint32_t *>(dst)[lane] = packed;
+  } else {
+    reinterpret_cast<uint16_t *>(dst)[lane] = static_cast<uint16_t>(packed);
+  }
+}
+
+// One warp per (token, kv head): quantize the K row and the V row, store the
+// codes and scales at the slot.
+template <int D, int IN_T, int OUT_T>
+__global__ void __launch_bounds__(kWarpsPerCta * 32)
+append_quant_kernel(const uint16_t *__restrict__ k_new, const uint16_t *__restrict__ v_new,
+                    const int64_t *__restrict__ slots, int num_tokens, int kv_heads,
+                    int block_size, int64_t num_slots, uint8_t *__restrict__ kc,
+                    uint8_t *__restrict__ vc, float *__restrict__ ks, float *__restrict__ vs,
+                    int *status) {
+  const int warp = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (warp >= num_tokens * kv_heads) return;
+  const int t = warp / kv_heads;
+  const int h = warp - t * kv_heads;
+  const int64_t slot = slots[t];
+  if (slot < 0) return;
+  if (slot >= num_slots) {
+    if (lane == 0 && h == 0) atomicOr(status, kErrSlot);
+    return;
+  }
+  const int64_t blk = slot / block_size;
+  const int row = static_cast<int>(slot - blk * block_size);
+  const int64_t dst_row = (blk * kv_heads + h) * block_size + row;
+  const int64_t src_row = static_cast<int64_t>(t) * kv_heads + h;
+  float x[D / 32];
+  float scale;
+  load_row<D, IN_T>(k_new + src_row * D, lane, x);
+  uint32_t packed = quantize_row<D, OUT_T>(x, &scale);
+  store_codes<D>(kc + dst_row * D, lane, packed);
+  if (lane == 0) ks[dst_row] = scale;
+  load_row<D, IN_T>(v_new + src_row * D, lane, x);
+  packed = quantize_row<D, OUT_T>(x, &scale);
+  store_codes<D>(vc + dst_row * D, lane, packed);
+  if (lane == 0) vs[dst_row] = scale;
+}
+
+// Standalone: one warp per contiguous row.
+template <int D, int IN_T, int OUT_T>
+__global__ void __launch_bounds__(kWarpsPerCta * 32)
+quantize_kernel(const uint16_t *__restrict__ x_in, int64_t rows, uint8_t *__restrict__ codes,
+                float *__restrict__ scales) {
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * kWarpsPerCta + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  float x[D / 32];
+  float scale;
+  load_row<D, IN_T>(x_in + row * D, lane, x);
+  uint32_t packed = quantize_row<D, OUT_T>(x, &scale);
+  store_codes<D>(codes + row * D, lane, packed);
+  if (lane == 0) scales[row] = scale;
+}
+
+// ---------------------------------------------------------------- block copy
+
+constexpr int kMaxPairsPerLaunch = 1024;
+
+struct CopyPairs {
+  int32_t src[kMaxPairsPerLaunch];
+  int32_t dst[kMaxPairsPerLaunch];
+};
+
+// grid (pair, layer, region): region 0 = K, 1 = V, 2 = K scale, 3 = V scale.
+__global__ void __launch_bounds__(256)
+block_copy_kernel(const __grid_constant__ CopyPairs pairs, char *__restrict__ base,
+                  uint64_t layer_stride, uint64_t kv_stride, uint64_t sc_stride,
+                  uint32_t kv_block_bytes, uint32_t sc_block_bytes) {
+  const int i = blockIdx.x;
+  const uint64_t layer = blockIdx.y;
+  const int region = blockIdx.z;
+  char *lb = base + layer * layer_stride;
+  char *rb;
+  uint32_t bytes;
+  switch (region) {
+    case 0: rb = lb; bytes = kv_block_bytes; break;
+    case 1: rb = lb + kv_stride; bytes = kv_block_bytes; break;
+    case 2: rb = lb + 2 * kv_stride; bytes = sc_block_bytes; break;
+    default: rb = lb + 2 * kv_stride + sc_stride; bytes = sc_block_bytes; break;
+  }
+  const uint4 *src = reinterpret_cast<const uint4 *>(rb + (uint64_t)pairs.src[i] * bytes);
+  uint4 *dst = reinterpret_cast<uint4 *>(rb + (uint64_t)pairs.dst[i] * bytes);
+  const uint32_t n = bytes / 16;
+  for (uint32_t j = threadIdx.x; j < n; j += blockDim.x) dst[j] = src[j];
+}
+
+template <int D, int IN_T, int OUT_T>
+cudaError_t launch_quantize(const void *x, int64_t rows, void *codes, float *scales,
+                            cudaStream_t st) {
+  const int64_t grid = (rows + kWarpsPerCta - 1) / kWarpsPerCta;
+  quantize_kernel<D, IN_T, OUT_T><<<(unsigned)grid, kWarpsPerCta * 32, 0, st>>>(
+      static_cast<const uint16_t *>(x), rows, static_cast<uint8_t *>(codes), scales);
+  return cudaGetLastError();
+}
+
+template <int D, int IN_T, int OUT_T>
+cudaError_t launch_append_quant(kv_pool *p, int layer, const void *k, const void *v,
+                                const int64_t *slots, int T, cudaStream_t st) {
+  const int64_t warps = (int64_t)T * p->d.num_kv_heads;
+  const int64_t grid = (warps + kWarpsPerCta - 1) / kWarpsPerCta;
+  append_quant_kernel<D, IN_T, OUT_T><<<(unsigned)grid, kWarpsPerCta * 32, 0, st>>>(
+      static_cast<const uint16_t *>(k), static_cast<const uint16_t *>(v), slots, T,
+      p->d.num_kv_heads, p->d.block_size, (int64_t)p->d.num_blocks * p->d.block_size,
+      reinterpret_cast<uint8_t *>(layer_k(p, layer)), reinterpret_cast<uint8_t *>(layer_v(p, layer)),
+      layer_ks(p, layer), layer_vs(p, layer), status_word(p));
+  return cudaGetLastError();
+}
+
+template <int IN_T, int OUT_T>
+cudaError_t dispatch_append_quant_d(kv_pool *p, int layer, const void *k, const void *v,
+                                    const int64_t *slots, int T, cudaStream_t st) {
+  return p->d.head_dim == 128 ? launch_append_quant<128, IN_T, OUT_T>(p, layer, k, v, slots, T, st)
+                              : launch_append_quant<64, IN_T, OUT_T>(p, layer, k, v, slots, T, st);
+}
+
+template <int IN_T, int OUT_T>
+cudaError_t dispatch_quantize_d(int D, const void *x, int64_t rows, void *codes, float *scales,
+                                cudaStream_t st) {
+  return D == 128 ? launch_quantize<128, IN_T, OUT_T>(x, rows, codes, scales, st)
+                  : launch_quantize<64, IN_T, OUT_T>(x, rows, codes, scales, st);
+}
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+}  // namespace
+}  // namespace pagedkv
+
+using namespace pagedkv;
+
+extern "C" {
+
+kv_status kv_append(kv_pool *pool, int32_t layer, const void *k_new, const void *v_new,
+                    int32_t in_dtype, const int64_t *slot_mapping, int32_t num_tokens,
+                    kv_stream_t stream) {
+  if (!pool) return fail(KV_ERR_INVALID, "null pool");
+  if (layer < 0 || layer >= pool->d.num_layers)
+    return fail(KV_ERR_INVALID, "layer %d out of range", layer);
+  if (num_tokens < 0) return fail(KV_ERR_INVALID, "negative num_tokens");
+  if (num_tokens == 0) return ok();
+  if (!k_new || !v_new || !slot_mapping) return fail(KV_ERR_INVALID, "null input pointer");
+  if (!aligned16(k_new) || !aligned16(v_new) || (reinterpret_cast<uintptr_t>(slot_mapping) & 7))
+    return fail(KV_ERR_INVALID, "k_new / v_new must be 16-byte aligned, slot_mapping 8-byte");
+  if (in_dtype != KV_BF16 && in_dtype != KV_FP16)
+    return fail(KV_ERR_UNSUPPORTED, "in_dtype must be KV_BF16 or KV_FP16");
+  const int64_t warps = (int64_t)num_tokens * pool->d.num_kv_heads;
+  if ((warps + kWarpsPerCta - 1) / kWarpsPerCta > 0x7FFFFFFF)
+    return fail(KV_ERR_INVALID, "too many tokens");
+  cudaStream_t st = (cudaStream_t)stream;
+  const int cd = pool->d.cache_dtype;
+  cudaError_t e;
+  if (!is_quant(cd)) {
+    if (in_dtype != cd)
+      return fail(KV_ERR_UNSUPPORTED, "a 16-bit cache takes rows of its own dtype");
+    const int64_t grid = (warps + kWarpsPerCta - 1) / kWarpsPerCta;
+    append16_kernel<<<(unsigned)grid, kWarpsPerCta * 32, 0, st>>>(
+        static_cast<const uint4 *>(k_new), static_cast<const uint4 *>(v_new), slot_mapping,
+        num_tokens, pool->d.num_kv_heads, pool->d.block_size, pool->row_bytes / 16,
+        (int64_t)pool->d.num_blocks * pool->d.block_size, layer_k(pool, layer),
+        layer_v(pool, layer), status_word(pool));
+    e = cudaGetLastError();
+  } else if (cd == KV_INT8) {
+    e = in_dtype == KV_BF16
+            ? dispatch_append_quant_d<KV_BF16, KV_INT8>(pool, layer, k_new, v_new, slot_mapping, num_tokens, st)
+            : dispatch_append_quant_d<KV_FP16, KV_INT8>(pool, layer, k_new, v_new, slot_mapping, num_tokens, st);
+  } else {
+    e = in_dtype == KV_BF16
+            ? dispatch_append_quant_d<KV_BF16, KV_FP8_E5M2>(pool, layer, k_new, v_new, slot_mapping, num_tokens, st)
+            : dispatch_append_quant_d<KV_FP16, KV_FP8_E5M2>(pool, layer, k_new, v_new, slot_mapping, num_tokens, st);
+  }
+  kv_status s = cuda_check(e, "kv_append launch");
+  return s == KV_OK ? ok() : s;
+}
+
+kv_status kv_quantize(const void *x, int32_t in_dtype, int64_t rows, int32_t head_dim,
+                      int32_t out_dtype, void *codes, float *scales, kv_stream_t stream) {
+  if (rows < 0) return fail(KV_ERR_INVALID, "negative rows");
+  if (head_dim != 64 && head_dim != 128)
+    return fail(KV_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  if (in_dtype != KV_BF16 && in_dtype != KV_FP16)
+    return fail(KV_ERR_UNSUPPORTED, "in_dtype must be KV_BF16 or KV_FP16");
+  if (out_dtype != KV_INT8 && out_dtype != KV_FP8_E5M2)
+    return fail(KV_ERR_UNSUPPORTED, "out_dtype must be KV_INT8 or KV_FP8_E5M2");
+  if (rows == 0) return ok();
+  if (!x || !codes || !scales) return fail(KV_ERR_INVALID, "null pointer");
+  if (!aligned16(x) || (reinterpret_cast<uintptr_t>(codes) & 3) ||
+      (reinterpret_cast<uintptr_t>(scales) & 3))
+    return fail(KV_ERR_INVALID, "x must be 16-byte aligned, codes and scales 4-byte");
+  if ((rows + kWarpsPerCta - 1) / kWarpsPerCta > 0x7FFFFFFF)
+    return fail(KV_ERR_INVALID, "too many rows");
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e;
+  if (out_dtype == KV_INT8)
+    e = in_dtype == KV_BF16 ? dispatch_quantize_d<KV_BF16, KV_INT8>(head_dim, x, rows, codes, scales, st)
+                            : dispatch_quantize_d<KV_FP16, KV_INT8>(head_dim, x, rows, codes, scales, st);
+  else
+    e = in_dtype == KV_BF16 ? dispatch_quantize_d<KV_BF16, KV_FP8_E5M2>(head_dim, x, rows, codes, scales, st)
+                            : dispatch_quantize_d<KV_FP16, KV_FP8_E5M2>(head_dim, x, rows, codes, scales, st);
+  kv_status s = cuda_check(e, "kv_quantize launch");
+  return s == KV_OK ? ok() : s;
+}
+
+kv_status kv_block_copy(kv_pool *pool, const int32_t *host_pairs, int32_t n_pairs,
+                        kv_stream_t stream) {
+  if (!pool) return fail(KV_ERR_INVALID, "null pool");
+  if (n_pairs < 0) return fail(KV_ERR_INVALID, "negative n_pairs");
+  if (n_pairs == 0) return ok();
+  if (!host_pairs) return fail(KV_ERR_INVALID, "null host_pairs");
+  const int32_t nb = pool->d.num_blocks;
+  std::vector<uint8_t> role(nb, 0);  // 1 = src, 2 = dst
+  for (int32_t i = 0; i < n_pairs; ++i) {
+    const int32_t s = host_pairs[2 * i], d = host_pairs[2 * i + 1];
+    if (s < 0 || s >= nb || d < 0 || d >= nb)
+      return fail(KV_ERR_INVALID, "pair %d (%d -> %d) has an id outside [0, %d)", i, s, d, nb);
+    if (s == d) return fail(KV_ERR_INVALID, "pair %d copies block %d onto itself", i, s);
+    role[s] |= 1;
+  }
+  for (int32_t i = 0; i < n_pairs; ++i) {
+    const int32_t d = host_pairs[2 * i + 1];
+    if (role[d] & 2) return fail(KV_ERR_INVALID, "block %d is the destination of two pairs", d);
+    if (role[d] & 1) return fail(KV_ERR_INVALID, "block %d is both a source and a destination", d);
+    role[d] |= 2;
+  }
+  const kv_pool_desc &dd = pool->d;
+  const uint32_t kv_block = (uint32_t)dd.num_kv_heads * dd.block_size * pool->row_bytes;
+  const uint32_t sc_block = (uint32_t)dd.num_kv_heads * dd.block_size * sizeof(float);
+  const int regions = is_quant(dd.cache_dtype) ? 4 : 2;
+  cudaStream_t st = (cudaStream_t)stream;
+  for (int32_t base = 0; base < n_pairs; base += kMaxPairsPerLaunch) {
+    const int32_t n = std::min<int32_t>(kMaxPairsPerLaunch, n_pairs - base);
+    CopyPairs cp;
+    for (int32_t i = 0; i < n; ++i) {
+      cp.src[i] = host_pairs[2 * (base + i)];
+      cp.dst[i] = host_pairs[2 * (base + i) + 1];
+    }
+    dim3 grid(n, dd.num_layers, regions);
+    block_copy_kernel<<<grid, 256, 0, st>>>(cp, pool->base, pool->lay.layer_stride,
+                                            pool->lay.kv_stride, pool->lay.sc_stride, kv_block,
+                                            sc_block);
+    kv_status s = cuda_check(cudaGetLastError(), "kv_block_copy launch");
+    if (s != KV_OK) return s;
+  }
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,92 @@
+// Host-side internals shared by the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "pagedkv.h"
+
+namespace pagedkv {
+
+// Device status word bit set when a bounded wait in a kernel gives up.
+constexpr int32_t kDevErrTimeout = 8;
+
+inline int elem_bytes(int dtype) {
+  return (dtype == KV_BF16 || dtype == KV_FP16) ? 2 : 1;
+}
+inline bool is_quant(int dtype) { return dtype == KV_INT8 || dtype == KV_FP8_E5M2; }
+inline uint64_t round_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
+
+// Byte offsets of one layer's regions inside the pool buffer.
+struct Layout {
+  uint64_t kv_bytes;      // one K (or V) region
+  uint64_t kv_stride;     // kv_bytes rounded to 256
+  uint64_t sc_bytes;      // one scale region (0 for 16-bit caches)
+  uint64_t sc_stride;
+  uint64_t layer_stride;  // K + V (+ K scale + V scale), each 256-aligned
+  uint64_t status_off;    // 256-byte status region after the last layer
+  uint64_t total;
+};
+
+// Tensor maps of one layer's K and V regions (built on first use; encoding
+// needs the CUDA driver, which a GPU-less host may not have).
+struct LayerMaps {
+  CUtensorMap k;
+  CUtensorMap v;
+  bool ready = false;
+};
+
+}  // namespace pagedkv
+
+struct kv_pool {
+  kv_pool_desc d;
+  char *base = nullptr;
+  uint64_t bytes = 0;
+  pagedkv::Layout lay;
+  int elt = 2;
+  int row_bytes = 0;  // head_dim * elt
+
+  std::mutex mu;                    // guards the allocator state
+  std::vector<int32_t> ref;         // refcount per block
+  std::vector<int32_t> free_stack;  // free ids; the top is handed out next
+  int32_t shared = 0;               // blocks with refcount >= 2
+
+  std::mutex map_mu;                // guards tensor-map creation
+  std::vector<pagedkv::LayerMaps> maps;
+};
+
+namespace pagedkv {
+
+kv_status fail(kv_status s, const char *fmt, ...);
+kv_status ok();
+kv_status cuda_check(cudaError_t e, const char *what);
+
+bool compute_layout(const kv_pool_desc &d, Layout *out, std::string *why,
+                    kv_status *code);
+
+inline char *layer_k(const kv_pool *p, int layer) {
+  return p->base + (uint64_t)layer * p->lay.layer_stride;
+}
+inline char *layer_v(const kv_pool *p, int layer) {
+  return layer_k(p, layer) + p->lay.kv_stride;
+}
+inline float *layer_ks(const kv_pool *p, int layer) {
+  return p->lay.sc_bytes ? (float *)(layer_v(p, layer) + p->lay.kv_stride) : nullptr;
+}
+inline float *layer_vs(const kv_pool *p, int layer) {
+  return p->lay.sc_bytes ? (float *)((char *)layer_ks(p, layer) + p->lay.sc_stride)
+                         : nullptr;
+}
+inline int32_t *status_word(const kv_pool *p) {
+  return (int32_t *)(p->base + p->lay.status_off);
+}
+
+// Tensor maps for the layer's K and V regions; nullptr + message on failure.
+const LayerMaps *layer_maps(kv_pool *p, int layer, kv_status *code);
+
+}  // namespace pagedkv

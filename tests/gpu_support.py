@@ -1,0 +1,128 @@
+"""Helpers for the GPU parity tests.
+
+The CUDA path is driven through the package's public API; expected values are
+computed only by ``oracle/`` from the generated inputs (never from anything the
+GPU produced).
+"""
+import numpy as np
+import torch
+
+from oracle import attention, cache_ops, quant
+
+TOL = 1e-2          # max abs and max rel (floor 1e-2 on |ref|) for attention outputs
+
+
+def to_np(t, dtype=np.float32):
+    return t.detach().float().cpu().numpy().astype(dtype)
+
+
+def bits16(t):
+    return t.detach().contiguous().view(torch.int16).cpu().numpy()
+
+
+def compare(gpu_out, ref, tol=TOL, what=""):
+    """Element-wise check of a bf16/fp16 GPU output against the fp64 oracle."""
+    g = gpu_out.detach().float().cpu().numpy().astype(np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert g.shape == ref.shape, (g.shape, ref.shape)
+    assert np.all(np.isfinite(g)), "%s: non-finite GPU output" % what
+    err = np.abs(g - ref)
+    max_abs = float(err.max()) if err.size else 0.0
+    max_rel = float((err / np.maximum(np.abs(ref), 1e-2)).max()) if err.size else 0.0
+    assert max_abs <= tol and max_rel <= tol, \
+        "%s: max abs %.3g, max rel %.3g (tolerance %g)" % (what, max_abs, max_rel, tol)
+    return max_abs, max_rel
+
+
+def device_inputs(wl, device):
+    tables = torch.from_numpy(wl.block_tables).to(device)
+    lens = torch.from_numpy(wl.context_lens.astype(np.int32)).to(device)
+    return tables, lens
+
+
+def build_pool(pkv, wl, device, chunk=65536):
+    """A one-layer pool holding the workload's history, filled via the product API
+    for quantized caches (kv_append) and by a plain device copy for 16-bit ones."""
+    pool = pkv.KVPool(1, wl.num_blocks, wl.block_size, wl.kv_heads, wl.head_dim,
+                      wl.cache_dtype, device)
+    K, V, _, _ = pool.layer_views(0)
+    if wl.k_fill is not None:
+        K.copy_(wl.k_fill)
+        V.copy_(wl.v_fill)
+    else:
+        K.zero_()
+        V.zero_()
+        slots = torch.from_numpy(wl.slot_hist).to(device)
+        for s in range(0, wl.k_hist.shape[0], chunk):
+            pkv.kv_append(pool, 0, wl.k_hist[s:s + chunk].contiguous(),
+                          wl.v_hist[s:s + chunk].contiguous(), slots[s:s + chunk].contiguous())
+    return pool
+
+
+def step(pkv, pool, wl, device, partition_tokens=0, out=None):
+    """One decode step through the product API: append the new token, attend."""
+    tables, lens = device_inputs(wl, device)
+    slot_new = torch.from_numpy(wl.slot_new).to(device)
+    pkv.kv_append(pool, 0, wl.k_new, wl.v_new, slot_new)
+    max_ctx = int(wl.context_lens.max()) if wl.batch else 0
+    return pkv.paged_attn_decode(pool, 0, wl.q, tables, lens, max_ctx, wl.scale, out=out,
+                                 partition_tokens=partition_tokens)
+
+
+def oracle_cache_16(wl):
+    """Oracle's view of a 16-bit cache after this step's append (exact values:
+    float16 for fp16 caches, float32 for bf16, which numpy lacks)."""
+    dt = np.float16 if wl.cache_dtype == "fp16" else np.float32
+    k = to_np(wl.k_fill, dt)
+    v = to_np(wl.v_fill, dt)
+    cache_ops.append(k, v, to_np(wl.k_new, dt), to_np(wl.v_new, dt), wl.slot_new, wl.block_size)
+    return k, v
+
+
+def oracle_cache_quant(wl, seqs):
+    """Oracle codes/scales for the history and new token of the given sequences.
+
+    Returns the full-size code and scale arrays (other sequences' blocks left
+    zero) and, for attention, float64 dequantized caches holding only the
+    sampled sequences' blocks, with block tables renumbered to match (the
+    result does not depend on physical placement).
+    """
+    shape = (wl.num_blocks, wl.kv_heads, wl.block_size, wl.head_dim)
+    cdt = np.int8 if wl.cache_dtype == "int8" else np.uint8
+    kc, vc = np.zeros(shape, cdt), np.zeros(shape, cdt)
+    ks, vs = np.zeros(shape[:3], np.float32), np.zeros(shape[:3], np.float32)
+    starts = np.concatenate([[0], np.cumsum(np.maximum(wl.context_lens - 1, 0))])
+    used = []
+    for b in seqs:
+        lo, hi = int(starts[b]), int(starts[b + 1])
+        cache_ops.append_quantized(kc, vc, ks, vs, to_np(wl.k_hist[lo:hi]),
+                                   to_np(wl.v_hist[lo:hi]), wl.slot_hist[lo:hi],
+                                   wl.block_size, wl.cache_dtype)
+        cache_ops.append_quantized(kc, vc, ks, vs, to_np(wl.k_new[b:b + 1]),
+                                   to_np(wl.v_new[b:b + 1]), wl.slot_new[b:b + 1],
+                                   wl.block_size, wl.cache_dtype)
+        nblk = -(-int(wl.context_lens[b]) // wl.block_size)
+        used += wl.block_tables[b, :nblk].tolist()
+    used = sorted(set(used)) or [0]
+    remap = {blk: i for i, blk in enumerate(used)}
+    tables = np.full_like(wl.block_tables, -1)
+    for b in seqs:
+        nblk = -(-int(wl.context_lens[b]) // wl.block_size)
+        tables[b, :nblk] = [remap[x] for x in wl.block_tables[b, :nblk]]
+    u = np.array(used)
+    kd = quant.dequantize(kc[u], ks[u], wl.cache_dtype)
+    vd = quant.dequantize(vc[u], vs[u], wl.cache_dtype)
+    return (kc, vc, ks, vs), (kd, vd, tables)
+
+
+def oracle_outputs(wl, kcache, vcache, pairs, tables=None):
+    """Oracle decode output for the listed (b, h) pairs."""
+    q = to_np(wl.q, np.float64)
+    tables = wl.block_tables if tables is None else tables
+    return np.stack([attention.decode_one(q, kcache, vcache, tables,
+                                          wl.context_lens, wl.scale, b, h) for b, h in pairs])
+
+
+def raw_bytes(t):
+    """Host copy of a device tensor's bytes, shaped [..., last * itemsize]."""
+    return t.detach().contiguous().view(torch.uint8).cpu().numpy()

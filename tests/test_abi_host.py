@@ -1,0 +1,250 @@
+"""Host-side checks of the C ABI (no GPU): the library loads and exports every
+symbol the header declares; pool layout against the KV-bytes formula; the
+refcounted allocator against the reference model; argument validation."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import allocator as ref_alloc
+from oracle import pool as ref_pool
+from paged_kv_cache_440_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pagedkv.h")
+FAKE_BASE = 1 << 40          # never dereferenced by host-only calls
+
+
+def _declared_functions():
+    txt = open(HEADER).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:kv_status|const char \*)\s*(\w+)\s*\(", txt, re.M)))
+
+
+def test_exports_every_declared_symbol():
+    names = _declared_functions()
+    assert len(names) >= 20
+    for n in names:
+        assert hasattr(B.lib, n), n
+    assert B.version().startswith("pagedkv")
+
+
+def _make_pool(NB=64, layers=2, bs=16, hkv=2, D=64, dt="bf16"):
+    d = B.PoolDesc(layers, NB, bs, hkv, D, B.DTYPE_CODES[dt])
+    n = ctypes.c_uint64()
+    B.check(B.lib.kv_pool_required_bytes(ctypes.byref(d), ctypes.byref(n)))
+    h = ctypes.c_void_p()
+    B.check(B.lib.kv_pool_create(ctypes.byref(d), ctypes.c_void_p(FAKE_BASE), n.value,
+                                 ctypes.byref(h)))
+    return h, n.value
+
+
+def _ptrs(h, layer):
+    k, v, ks, vs = (ctypes.c_void_p() for _ in range(4))
+    B.check(B.lib.kv_pool_layer_ptrs(h, layer, ctypes.byref(k), ctypes.byref(v),
+                                     ctypes.byref(ks), ctypes.byref(vs)))
+    return k.value, v.value, ks.value, vs.value
+
+
+@pytest.mark.parametrize("dt,elt", [("bf16", 2), ("fp16", 2), ("int8", 1), ("e5m2", 1)])
+@pytest.mark.parametrize("layers,NB,bs,hkv,D", [(80, 37, 16, 8, 128), (1, 5, 32, 3, 64)])
+def test_layout_matches_kv_formula(dt, elt, layers, NB, bs, hkv, D):
+    h, total = _make_pool(NB, layers, bs, hkv, D, dt)
+    try:
+        tokens = NB * bs
+        kv = ref_pool.kv_cache_bytes(1, hkv, D, elt, tokens)       # one layer, K and V
+        prev_end = FAKE_BASE
+        for layer in range(layers):
+            k, v, ks, vs = _ptrs(h, layer)
+            assert k % 256 == 0 and v % 256 == 0 and k >= prev_end
+            assert v - k >= kv // 2                        # K region holds half the formula
+            if dt in ("int8", "e5m2"):
+                sb = ref_pool.scale_bytes(1, hkv, 4, tokens)
+                assert ks - v >= kv // 2 and vs - ks >= sb // 2
+                prev_end = vs + sb // 2
+            else:
+                assert ks is None and vs is None
+                prev_end = v + kv // 2
+        # padding between regions is below 256 bytes each, plus a 256-byte status region
+        scales = ref_pool.scale_bytes(layers, hkv, 4, tokens) if dt in ("int8", "e5m2") else 0
+        exact = ref_pool.kv_cache_bytes(layers, hkv, D, elt, tokens) + scales
+        assert exact + 256 <= total <= exact + 256 + layers * 4 * 255
+    finally:
+        B.lib.kv_pool_destroy(h)
+
+
+def test_pool_rejects_bad_descriptions():
+    n = ctypes.c_uint64()
+    for desc, code in [((1, 8, 8, 1, 64, 0), B.KV_ERR_UNSUPPORTED),
+                       ((1, 8, 16, 1, 96, 0), B.KV_ERR_UNSUPPORTED),
+                       ((1, 8, 16, 1, 64, 7), B.KV_ERR_UNSUPPORTED),
+                       ((0, 8, 16, 1, 64, 0), B.KV_ERR_INVALID),
+                       ((1, -1, 16, 1, 64, 0), B.KV_ERR_INVALID)]:
+        d = B.PoolDesc(*desc)
+        assert B.lib.kv_pool_required_bytes(ctypes.byref(d), ctypes.byref(n)) == code
+        assert B.lib.kv_last_error()
+    d = B.PoolDesc(1, 8, 16, 1, 64, 0)
+    B.check(B.lib.kv_pool_required_bytes(ctypes.byref(d), ctypes.byref(n)))
+    h = ctypes.c_void_p()
+    assert B.lib.kv_pool_create(ctypes.byref(d), ctypes.c_void_p(FAKE_BASE + 16), n.value,
+                                ctypes.byref(h)) == B.KV_ERR_INVALID          # misaligned
+    assert B.lib.kv_pool_create(ctypes.byref(d), ctypes.c_void_p(FAKE_BASE), n.value - 1,
+                                ctypes.byref(h)) == B.KV_ERR_INVALID          # too small
+
+
+def _arr(ids):
+    return (ctypes.c_int32 * max(len(ids), 1))(*ids)
+
+
+def _stats(h):
+    u, f, s = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+    B.check(B.lib.kv_pool_stats(h, ctypes.byref(u), ctypes.byref(f), ctypes.byref(s)))
+    return u.value, f.value, s.value
+
+
+def test_allocator_random_ops_match_model():
+    rng = np.random.default_rng(0)
+    NB = 40
+    h, _ = _make_pool(NB)
+    model = ref_alloc.PoolModel(NB)
+    held = []                     # references we own (one entry per reference)
+    try:
+        for step in range(3000):
+            op = rng.integers(0, 4)
+            if op == 0:
+                n = int(rng.integers(0, 6))
+                out = (ctypes.c_int32 * max(n, 1))()
+                st = B.lib.kv_alloc_blocks(h, n, out)
+                if model.free_count() < n:
+                    assert st == B.KV_ERR_OOM
+                else:
+                    assert st == B.KV_OK
+                    ids = list(out[:n])
+                    assert len(set(ids)) == n
+                    model.take(ids)
+                    held += ids
+            elif op == 1 and held:
+                k = int(rng.integers(1, min(4, len(held)) + 1))
+                pick = [held.pop(int(rng.integers(0, len(held)))) for _ in range(k)]
+                B.check(B.lib.kv_free_blocks(h, len(pick), _arr(pick)))
+                model.free(pick)
+            elif op == 2 and held:
+                i = held[int(rng.integers(0, len(held)))]
+                B.check(B.lib.kv_share_blocks(h, 1, _arr([i])))
+                model.share([i])
+                held.append(i)
+            elif op == 3 and held:
+                i = held[int(rng.integers(0, len(held)))]
+                new = ctypes.c_int32()
+                st = B.lib.kv_cow_prepare(h, i, ctypes.byref(new))
+                if not model.cow_needed(i):
+                    assert st == B.KV_OK and new.value == i
+                elif model.free_count() == 0:
+                    assert st == B.KV_ERR_OOM
+                else:
+                    assert st == B.KV_OK and new.value != i
+                    model.free([i])
+                    model.take([new.value])
+                    held.remove(i)
+                    held.append(new.value)
+            u, f, s = _stats(h)
+            assert (u, f, s) == (model.used_count(), model.free_count(), model.shared_count())
+            for i in range(NB):
+                r = ctypes.c_int32()
+                B.check(B.lib.kv_block_refcount(h, i, ctypes.byref(r)))
+                assert r.value == model.ref[i]
+    finally:
+        B.lib.kv_pool_destroy(h)
+
+
+def test_allocator_errors_change_nothing():
+    h, _ = _make_pool(8)
+    try:
+        out = (ctypes.c_int32 * 8)()
+        B.check(B.lib.kv_alloc_blocks(h, 3, out))
+        ids = list(out[:3])
+        before = _stats(h)
+        assert B.lib.kv_alloc_blocks(h, 6, out) == B.KV_ERR_OOM
+        assert B.lib.kv_free_blocks(h, 2, _arr([ids[0], 7])) == B.KV_ERR_INVALID   # 7 is free
+        assert B.lib.kv_free_blocks(h, 2, _arr([ids[0], ids[0]])) == B.KV_ERR_INVALID
+        assert B.lib.kv_share_blocks(h, 1, _arr([9])) == B.KV_ERR_INVALID
+        assert B.lib.kv_alloc_blocks(h, -1, out) == B.KV_ERR_INVALID
+        assert _stats(h) == before
+    finally:
+        B.lib.kv_pool_destroy(h)
+
+
+def test_block_copy_validation_rejects_bad_pairs_before_launch():
+    h, _ = _make_pool(16)
+    try:
+        bad = [[(3, 3)], [(1, 2), (4, 2)], [(1, 2), (2, 5)], [(0, 16)], [(-1, 3)]]
+        for pairs in bad:
+            flat = [v for p in pairs for v in p]
+            assert B.lib.kv_block_copy(h, _arr(flat), len(pairs), None) == B.KV_ERR_INVALID
+        assert B.lib.kv_block_copy(h, _arr([]), 0, None) == B.KV_OK
+    finally:
+        B.lib.kv_pool_destroy(h)
+
+
+def test_attention_argument_validation_and_workspace_size():
+    h, _ = _make_pool(64, 1, 16, 2, 64, "bf16")
+    try:
+        n = ctypes.c_uint64()
+        # Hq must be a multiple of Hkv
+        assert B.lib.paged_attn_workspace_bytes(h, 4, 3, 250, 0, ctypes.byref(n)) == B.KV_ERR_INVALID
+        # partition must be a multiple of the block size
+        assert B.lib.paged_attn_workspace_bytes(h, 4, 8, 250, 24, ctypes.byref(n)) == B.KV_ERR_INVALID
+        # one partition: no workspace
+        B.check(B.lib.paged_attn_workspace_bytes(h, 4, 8, 250, 256, ctypes.byref(n)))
+        assert n.value == 0
+        # P = ceil(250 / 64) = 4 partitions: o [4,8,4,64] + m, l [4,8,4] fp32, 256-aligned
+        B.check(B.lib.paged_attn_workspace_bytes(h, 4, 8, 250, 64, ctypes.byref(n)))
+        parts = 4 * 8 * 4
+        r256 = lambda x: -(-x // 256) * 256
+        assert n.value == r256(parts * 64 * 4) + 2 * r256(parts * 4)
+        p = ctypes.c_int32()
+        B.check(B.lib.paged_attn_default_partition(h, 4, 8, 250, ctypes.byref(p)))
+        assert p.value % 16 == 0 and p.value >= 16
+        # validation failures return before any device work
+        nul = ctypes.c_void_p(0)
+        fake = ctypes.c_void_p(FAKE_BASE)
+        args = lambda q, qdt, hq, tbl, mb, lens, mc, sc, out: (
+            h, 0, q, qdt, 4, hq, tbl, mb, lens, mc, sc, out, 0, fake, 1 << 20, None)
+        assert B.lib.paged_attn_decode(*args(nul, 0, 8, fake, 16, fake, 250, 0.125, fake)) == B.KV_ERR_INVALID
+        assert B.lib.paged_attn_decode(*args(fake, 1, 8, fake, 16, fake, 250, 0.125, fake)) == B.KV_ERR_UNSUPPORTED
+        assert B.lib.paged_attn_decode(*args(fake, 0, 5, fake, 16, fake, 250, 0.125, fake)) == B.KV_ERR_INVALID
+        assert B.lib.paged_attn_decode(*args(fake, 0, 8, fake, 0, fake, 250, 0.125, fake)) == B.KV_ERR_INVALID
+        assert B.lib.paged_attn_decode(*args(fake, 0, 8, fake, 16, fake, 250, float("nan"), fake)) == B.KV_ERR_INVALID
+        assert B.lib.paged_attn_decode(*args(fake, 0, 8, fake, 16, fake, -1, 0.125, fake)) == B.KV_ERR_INVALID
+        # too small a workspace
+        st = B.lib.paged_attn_decode(h, 0, fake, 0, 4, 8, fake, 16, fake, 250, 0.125, fake, 64,
+                                     fake, 16, None)
+        assert st == B.KV_ERR_INVALID
+        # append / quantize validation
+        assert B.lib.kv_append(h, 1, fake, fake, 0, fake, 1, None) == B.KV_ERR_INVALID   # layer
+        assert B.lib.kv_append(h, 0, fake, fake, 1, fake, 1, None) == B.KV_ERR_UNSUPPORTED
+        assert B.lib.kv_append(h, 0, fake, fake, 0, fake, -1, None) == B.KV_ERR_INVALID
+        assert B.lib.kv_append(h, 0, fake, fake, 0, fake, 0, None) == B.KV_OK
+        assert B.lib.kv_quantize(fake, 0, 4, 96, 3, fake, fake, None) == B.KV_ERR_UNSUPPORTED
+        assert B.lib.kv_quantize(fake, 0, 4, 64, 0, fake, fake, None) == B.KV_ERR_UNSUPPORTED
+        assert B.lib.kv_quantize(fake, 0, 0, 64, 3, fake, fake, None) == B.KV_OK
+    finally:
+        B.lib.kv_pool_destroy(h)
+
+
+def test_valid_call_without_a_gpu_fails_loudly():
+    """On a host with no GPU a well-formed launch reports KV_ERR_CUDA; nothing
+    falls back to a CPU path."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    h, _ = _make_pool(64, 1, 16, 2, 64, "bf16")
+    try:
+        fake = ctypes.c_void_p(FAKE_BASE)
+        st = B.lib.paged_attn_decode(h, 0, fake, 0, 4, 8, fake, 16, fake, 250, 0.125, fake, 0,
+                                     fake, 1 << 20, None)
+        assert st == B.KV_ERR_CUDA
+    finally:
+        B.lib.kv_pool_destroy(h)

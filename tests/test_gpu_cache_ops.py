@@ -1,0 +1,118 @@
+"""GPU parity of append, quantize and copy-on-write block copy: bit-exact
+against the oracle on the same generated inputs; plus the device status word
+and the bounded-wait self-test."""
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from gpu_support import bits16, raw_bytes, to_np
+from oracle import cache_ops, quant
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module")
+def pkv():
+    import paged_kv_cache_440_b200 as p
+    return p
+
+
+@pytest.mark.parametrize("make", [W.tiny, W.gqa70b, W.mha13b])
+def test_append_16bit_bit_exact(pkv, make):
+    wl = make(DEV)
+    pool = pkv.KVPool(1, wl.num_blocks, wl.block_size, wl.kv_heads, wl.head_dim,
+                      wl.cache_dtype, DEV)
+    K, V, _, _ = pool.layer_views(0)
+    K.copy_(wl.k_fill)
+    V.copy_(wl.v_fill)
+    slots = wl.slot_new.copy()
+    slots[1] = -1                                     # padding token: skipped
+    pkv.kv_append(pool, 0, wl.k_new, wl.v_new, torch.from_numpy(slots).to(DEV))
+    torch.cuda.synchronize()
+    assert pool.status() == 0
+    kb, vb = bits16(wl.k_fill), bits16(wl.v_fill)
+    cache_ops.append(kb, vb, bits16(wl.k_new), bits16(wl.v_new), slots, wl.block_size)
+    touched = np.unique(np.maximum(slots, 0) // wl.block_size)
+    if kb.size > 300_000_000:                          # large pool: touched + sampled blocks
+        rng = np.random.default_rng(0)
+        blocks = np.unique(np.concatenate([touched, rng.choice(wl.num_blocks, 256)]))
+        idx = torch.from_numpy(blocks).to(DEV)
+        assert np.array_equal(bits16(K[idx]), kb[blocks])
+        assert np.array_equal(bits16(V[idx]), vb[blocks])
+    else:
+        assert np.array_equal(bits16(K), kb)
+        assert np.array_equal(bits16(V), vb)
+
+
+def test_append_out_of_range_slot_is_reported_not_written(pkv):
+    pool = pkv.KVPool(1, 8, 16, 2, 64, "bf16", DEV)
+    K, V, _, _ = pool.layer_views(0)
+    K.zero_()
+    V.zero_()
+    x = torch.randn(2, 2, 64, device=DEV).to(torch.bfloat16)
+    pkv.kv_append(pool, 0, x, x, torch.tensor([3, 8 * 16 + 5], dtype=torch.int64, device=DEV))
+    torch.cuda.synchronize()
+    assert pool.status() & 4
+    assert torch.equal(K[0, :, 3], x[0]) and int((K != 0).sum()) == 2 * 64
+
+
+def _special_rows(D):
+    rows = [np.zeros(D), np.full(D, 1e-30), np.full(D, -3.0), np.linspace(-1, 1, D)]
+    r = np.zeros(D)
+    r[5] = 1e4
+    r[6] = -2.0 ** -20
+    rows.append(r)
+    r = np.zeros(D)
+    r[0] = 57344.0
+    r[1:] = np.linspace(-1e-3, 1e-3, D - 1)           # E5M2 subnormal codes
+    rows.append(r)
+    return np.stack(rows)
+
+
+@pytest.mark.parametrize("kind", ["int8", "e5m2"])
+@pytest.mark.parametrize("in_dt", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("D", [64, 128])
+def test_quantize_bit_exact(pkv, kind, in_dt, D):
+    g = torch.Generator(device=DEV).manual_seed(D)
+    x = torch.randn(20000, D, generator=g, device=DEV)
+    x = x * torch.exp(torch.randn(20000, 1, generator=g, device=DEV) * 3)   # wide dynamic range
+    x = torch.cat([x, torch.from_numpy(_special_rows(D)).float().to(DEV)]).to(in_dt)
+    codes, scales = pkv.kv_quantize(x, kind)
+    torch.cuda.synchronize()
+    ref_codes, ref_scales = quant.quantize_rows(to_np(x), kind)
+    assert np.array_equal(scales.cpu().numpy().view(np.uint32), ref_scales.view(np.uint32))
+    assert np.array_equal(codes.cpu().numpy(), ref_codes)
+
+
+@pytest.mark.parametrize("cache", ["bf16", "int8", "e5m2"])
+def test_block_copy_bit_exact(pkv, cache):
+    """Shared-prefix shapes: 200 copy-on-write pairs, 3 layers, random pool bytes."""
+    layers, NB, bs, hkv, D = 3, 1500, 16, 8, 128
+    pool = pkv.KVPool(layers, NB, bs, hkv, D, cache, DEV)
+    g = torch.Generator(device=DEV).manual_seed(7)
+    pool.buffer.copy_(torch.randint(0, 256, pool.buffer.shape, generator=g, device=DEV,
+                                    dtype=torch.uint8))
+    before = [[raw_bytes(t) if t is not None else None for t in pool.layer_views(l)]
+              for l in range(layers)]
+    rng = np.random.default_rng(3)
+    ids = rng.permutation(NB)[:400]
+    pairs = list(zip(ids[:200].tolist(), ids[200:].tolist()))
+    pkv.kv_block_copy(pool, pairs)
+    torch.cuda.synchronize()
+    regions = [a for lay in before for a in lay if a is not None]
+    cache_ops.block_copy(regions, pairs)
+    after = [raw_bytes(t) for l in range(layers) for t in pool.layer_views(l) if t is not None]
+    for a, r in zip(after, regions):
+        assert np.array_equal(a, r)
+
+
+def test_bounded_wait_gives_up_and_reports(pkv):
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    pkv.selftest_wait_timeout(st, limit_us=2000)
+    torch.cuda.synchronize()
+    assert int(st.item()) & 8
+    # the context is still usable afterwards
+    y = torch.ones(4, device=DEV) * 2
+    assert float(y.sum()) == 8.0

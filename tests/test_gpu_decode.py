@@ -1,0 +1,248 @@
+"""GPU parity of paged decode attention against the fp64 oracle.
+
+Each test runs one decode step (append of the step's token, then attention)
+through the C ABI and compares every output it checks, element by element, with
+the oracle on the same generated inputs. Tolerance: max abs 1e-2 and max rel
+1e-2 (relative to max(|ref|, 1e-2)). Full-size workloads run in the launch
+configuration the benchmark times (default partition size); outputs there are
+checked for all heads of every sequence, or of a seeded sample of sequences
+where the oracle would be slow.
+"""
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from gpu_support import (build_pool, compare, device_inputs, oracle_cache_16,
+                         oracle_cache_quant, oracle_outputs, step, to_np)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module")
+def pkv():
+    import paged_kv_cache_440_b200 as p
+    return p
+
+
+def _all_pairs(wl, seqs=None):
+    seqs = range(wl.batch) if seqs is None else seqs
+    return [(b, h) for b in seqs for h in range(wl.q_heads)]
+
+
+def _run_16(pkv, wl, partition_tokens=0, seqs=None):
+    pool = build_pool(pkv, wl, DEV)
+    out = step(pkv, pool, wl, DEV, partition_tokens)
+    torch.cuda.synchronize()
+    assert pool.status() == 0
+    k, v = oracle_cache_16(wl)
+    pairs = _all_pairs(wl, seqs)
+    ref = oracle_outputs(wl, k, v, pairs)
+    got = torch.stack([out[b, h] for b, h in pairs])
+    return compare(got, ref, what=wl.name)
+
+
+def test_tiny_default_partition(pkv):
+    _run_16(pkv, W.tiny(DEV))
+
+
+@pytest.mark.parametrize("S", [16, 48, 64, 128, 256, 4096])
+def test_tiny_partition_sizes_agree(pkv, S):
+    _run_16(pkv, W.tiny(DEV), partition_tokens=S)
+
+
+def test_gqa70b_every_output(pkv):
+    """LLaMA-70B-shaped GQA layer, batch 32, lengths U[512, 4096], all 2048 outputs."""
+    _run_16(pkv, W.gqa70b(DEV))
+
+
+@pytest.mark.parametrize("S", [256, 1024, 4096])
+def test_gqa70b_split_k_sizes(pkv, S):
+    _run_16(pkv, W.gqa70b(DEV), partition_tokens=S, seqs=[0, 7, 19, 31])
+
+
+def test_mha13b_every_output(pkv):
+    """13B-shaped MHA layer (40/40 heads, fp16), batch 32 x 2048, all 1280 outputs."""
+    _run_16(pkv, W.mha13b(DEV))
+
+
+@pytest.mark.parametrize("kind", ["int8", "e5m2"])
+@pytest.mark.parametrize("variant,seqs", [("a", [0, 13, 40, 63]), ("b", [0, 5])])
+def test_quantized_long_context(pkv, kind, variant, seqs):
+    """INT8 / E5M2 per-token-head KV, bs 32, (a) 64 x 4096 and (b) 8 x 32768.
+    Codes and scales of the sampled sequences are bit-exact; their outputs match
+    the oracle run on the same dequantized values."""
+    wl = W.quant_long(kind, variant, DEV)
+    pool = build_pool(pkv, wl, DEV)
+    out = step(pkv, pool, wl, DEV)
+    torch.cuda.synchronize()
+    assert pool.status() == 0
+    (kc, vc, ks, vs), (kd, vd, otab) = oracle_cache_quant(wl, seqs)
+    K, V, KS, VS = pool.layer_views(0)
+    for b in seqs:
+        nblk = -(-int(wl.context_lens[b]) // wl.block_size)
+        ids = torch.from_numpy(wl.block_tables[b, :nblk].astype(np.int64)).to(DEV)
+        idn = wl.block_tables[b, :nblk]
+        assert np.array_equal(K[ids].cpu().numpy(), kc[idn]), "K codes, seq %d" % b
+        assert np.array_equal(V[ids].cpu().numpy(), vc[idn]), "V codes, seq %d" % b
+        assert np.array_equal(KS[ids].cpu().numpy().view(np.uint32), ks[idn].view(np.uint32))
+        assert np.array_equal(VS[ids].cpu().numpy().view(np.uint32), vs[idn].view(np.uint32))
+    pairs = _all_pairs(wl, seqs)
+    ref = oracle_outputs(wl, kd, vd, pairs, otab)
+    compare(torch.stack([out[b, h] for b, h in pairs]), ref, what=wl.name)
+
+
+def test_shared_prefix_copy_on_write(pkv):
+    """200 requests share a 1500-token prompt (94 blocks of 16, the last holding
+    12 tokens). Every request copies the shared partial block before appending
+    its private suffix. The oracle builds its own cache with its own allocator
+    model and copies; outputs agree for a sample of requests."""
+    from oracle import allocator, cache_ops
+    wl = W.shared_prefix(DEV)
+    bs, hkv, D = wl.block_size, wl.kv_heads, wl.head_dim
+    P = wl.prefix_len
+    nprefix = -(-P // bs)
+
+    # ------------------------------------------------ CUDA path (product API)
+    pool = pkv.KVPool(1, wl.num_blocks, bs, hkv, D, "bf16", DEV)
+    K, V, _, _ = pool.layer_views(0)
+    K.zero_()
+    V.zero_()
+    prefix_ids = pool.alloc(nprefix)
+    slots = torch.tensor([prefix_ids[t // bs] * bs + t % bs for t in range(P)],
+                         dtype=torch.int64, device=DEV)
+    pkv.kv_append(pool, 0, wl.prefix_k, wl.prefix_v, slots)
+    tables = []
+    for b in range(wl.batch):
+        pool.share(prefix_ids)
+        tables.append(list(prefix_ids))
+    pairs = []
+    for b in range(wl.batch):
+        last = tables[b][nprefix - 1]
+        new = pool.cow_prepare(last)
+        assert new != last
+        pairs.append((last, new))
+        tables[b][nprefix - 1] = new
+    assert pool.refcount(prefix_ids[-1]) == 1 and pool.refcount(prefix_ids[0]) == 201
+    pkv.kv_block_copy(pool, pairs)
+    sl = []
+    for b in range(wl.batch):
+        L = P + int(wl.suffix_lens[b])
+        need = -(-L // bs) - len(tables[b])
+        tables[b] += pool.alloc(need)
+        sl += [tables[b][t // bs] * bs + t % bs for t in range(P, L)]
+    pkv.kv_append(pool, 0, wl.suffix_k, wl.suffix_v, torch.tensor(sl, dtype=torch.int64, device=DEV))
+    lens = P + wl.suffix_lens
+    mb = max(len(t) for t in tables)
+    tbl = np.full((wl.batch, mb), -1, np.int32)
+    for b, t in enumerate(tables):
+        tbl[b, :len(t)] = t
+    out = pkv.paged_attn_decode(pool, 0, wl.q, torch.from_numpy(tbl).to(DEV),
+                                torch.from_numpy(lens.astype(np.int32)).to(DEV),
+                                int(lens.max()), wl.scale)
+    torch.cuda.synchronize()
+    assert pool.status() == 0
+    st = pool.stats()
+    assert st["shared"] == nprefix - 1
+
+    # ------------------------------------------------ oracle (own allocation)
+    m = allocator.PoolModel(wl.num_blocks)
+    kc = np.zeros((wl.num_blocks, hkv, bs, D), np.float32)
+    vc = np.zeros_like(kc)
+    o_prefix = m.alloc(nprefix)
+    cache_ops.append(kc, vc, to_np(wl.prefix_k), to_np(wl.prefix_v),
+                     np.array([o_prefix[t // bs] * bs + t % bs for t in range(P)]), bs)
+    o_tables = []
+    for b in range(wl.batch):
+        m.share(o_prefix)
+        o_tables.append(list(o_prefix))
+    o_pairs = []
+    for b in range(wl.batch):
+        fresh = m.alloc(1)[0]
+        m.free([o_prefix[-1]])
+        o_pairs.append((o_prefix[-1], fresh))
+        o_tables[b][-1] = fresh
+    cache_ops.block_copy([kc, vc], o_pairs)
+    o_sl = []
+    for b in range(wl.batch):
+        L = P + int(wl.suffix_lens[b])
+        o_tables[b] += m.alloc(-(-L // bs) - len(o_tables[b]))
+        o_sl += [o_tables[b][t // bs] * bs + t % bs for t in range(P, L)]
+    cache_ops.append(kc, vc, to_np(wl.suffix_k), to_np(wl.suffix_v), np.array(o_sl), bs)
+    o_tbl = np.full((wl.batch, mb), -1, np.int64)
+    for b, t in enumerate(o_tables):
+        o_tbl[b, :len(t)] = t
+    from oracle import attention
+    q = to_np(wl.q, np.float64)
+    sample = [0, 1, 57, 123, 199]
+    got = torch.stack([out[b, h] for b in sample for h in range(wl.q_heads)])
+    ref = np.stack([attention.decode_one(q, kc, vc, o_tbl, lens, wl.scale, b, h)
+                    for b in sample for h in range(wl.q_heads)])
+    compare(got, ref, what="shared_prefix")
+
+
+# --------------------------------------------------------------- edge cases
+
+EDGE_LENS = [0, 1, 15, 16, 17, 63, 64, 65, 127, 128, 129, 300]
+
+
+@pytest.mark.parametrize("cache", ["bf16", "fp16", "int8", "e5m2"])
+@pytest.mark.parametrize("G", [1, 2, 4, 8, 16])
+@pytest.mark.parametrize("D,bs", [(64, 16), (128, 32)])
+def test_edge_lengths_groups_dims(pkv, cache, G, D, bs):
+    """Empty, single-token, block-boundary and partition-boundary lengths; MHA,
+    GQA groups of 2..16 heads (16 spans two head chunks); head_dim 64 / 128;
+    block size 16 / 32; all four cache types; partitions of 4 blocks."""
+    qd = "fp16" if cache == "fp16" else "bf16"
+    lens = EDGE_LENS
+    wl = W.make_decode_workload("edge", len(lens), 2 * G, 2, D, bs, qd, cache, lens,
+                                seed=G * 1000 + D + bs, device=DEV)
+    pool = build_pool(pkv, wl, DEV)
+    out = step(pkv, pool, wl, DEV, partition_tokens=4 * bs)
+    torch.cuda.synchronize()
+    assert pool.status() == 0
+    pairs = _all_pairs(wl)
+    if cache in ("bf16", "fp16"):
+        k, v = oracle_cache_16(wl)
+        tab = None
+    else:
+        _, (k, v, tab) = oracle_cache_quant(wl, list(range(wl.batch)))
+    ref = oracle_outputs(wl, k, v, pairs, tab)
+    compare(torch.stack([out[b, h] for b, h in pairs]), ref, what="edge %s G%d" % (cache, G))
+    assert torch.all(out[0] == 0)     # empty sequence
+
+
+def test_separate_phases_equal_fused_call(pkv):
+    wl = W.gqa70b(DEV, batch=8)
+    pool = build_pool(pkv, wl, DEV)
+    out = step(pkv, pool, wl, DEV, partition_tokens=512)
+    tables, lens = device_inputs(wl, DEV)
+    ws = pkv.make_workspace(pool, wl.batch, wl.q_heads, int(wl.context_lens.max()), 512)
+    out2 = torch.empty_like(out)
+    pkv.paged_attn_partition(pool, 0, wl.q, tables, lens, int(wl.context_lens.max()), wl.scale,
+                             out2, ws, partition_tokens=512)
+    pkv.paged_attn_merge(pool, lens, tables.shape[1], int(wl.context_lens.max()), out2, ws,
+                         partition_tokens=512)
+    torch.cuda.synchronize()
+    assert torch.equal(out, out2)
+
+
+def test_bad_block_id_and_length_are_reported(pkv):
+    wl = W.make_decode_workload("bad", 3, 8, 2, 64, 16, "bf16", "bf16", [40, 40, 40],
+                                seed=5, device=DEV)
+    pool = build_pool(pkv, wl, DEV)
+    tables, lens = device_inputs(wl, DEV)
+    tables[1, 1] = wl.num_blocks + 7          # outside the pool
+    lens[2] = 10_000                           # beyond the table width and max_context
+    pool.status_clear()
+    out = pkv.paged_attn_decode(pool, 0, wl.q, tables, lens, 64, wl.scale)
+    torch.cuda.synchronize()
+    st = pool.status()
+    assert st & 1 and st & 2
+    assert torch.all(torch.isfinite(out.float()))
+    assert torch.all(out[2] == 0)
+    # sequence 0 is untouched by the bad entries
+    k, v = to_np(wl.k_fill), to_np(wl.v_fill)
+    ref = oracle_outputs(wl, k, v, [(0, h) for h in range(8)])
+    compare(out[0], ref, what="good sequence")
