@@ -225,11 +225,14 @@ kv_status kv_block_copy(kv_pool *pool, const int32_t *host_pairs,
  * K_g[t] = code * k_scale and V_g[t] = code * v_scale (dequantized in-kernel).
  * [bjdmk.com.cn/news/6246348, §2.1; KV Cache 原理与 PagedAttention, §三 工作方式 4]
  *
- * Long contexts are split into partitions of partition_tokens tokens
- * (split-K). Each partition is reduced by one CTA per (sequence, KV head,
- * partition) to a running max m, a sum l and an unnormalized output o; a
- * merge combines them: out = sum_p e^(m_p - M) o_p / sum_p e^(m_p - M) l_p,
- * M = max_p m_p. Sequences with one partition are written directly.
+ * Work split (split-K): a unit is one sequence and a group of its KV heads
+ * (with their query heads); its positions are the sequence's KV blocks. The
+ * positions of all units are laid end to end and divided evenly among
+ * num_ctas persistent CTAs, so every CTA reads the same number of blocks
+ * whatever the mix of lengths. A unit that one CTA covers entirely is
+ * finished by it; a unit cut by CTA boundaries leaves a running max m, sum l
+ * and unnormalised output o per piece, which the merge combines:
+ * out = sum_i e^(m_i - M) o_i / sum_i e^(m_i - M) l_i, M = max_i m_i.
  *
  * Common arguments:
  *   q       device [num_seqs][num_q_heads][head_dim], q_dtype, 16-byte aligned.
@@ -240,58 +243,57 @@ kv_status kv_block_copy(kv_pool *pool, const int32_t *host_pairs,
  *   context_lens  device int32 [num_seqs]; each must satisfy
  *           0 <= L_b <= min(max_context, max_blocks_per_seq * block_size),
  *           else KV_DEVERR_CONTEXT is set and that sequence's output is 0.
- *   max_context   host upper bound on every L_b; sizes the workspace.
- *   partition_tokens  0 = library default, else a positive multiple of
- *           block_size.
+ *   max_context   host upper bound on every L_b.
+ *   num_ctas      CTAs the work is divided among: 0 = one per multiprocessor
+ *           of the current device (the default), else 1 .. 65535.
  *   workspace     device, 256-byte aligned, >= paged_attn_workspace_bytes
- *           bytes (may be NULL when that size is 0). Holds the per-partition
- *           (m, l, o) in fp32 between the two phases; its contents are
- *           scratch and need no initialisation.
+ *           bytes for the same num_seqs, num_q_heads and num_ctas. Holds the
+ *           per-unit bookkeeping and the split partials between the two
+ *           kernels; its contents are scratch and need no initialisation.
+ *           Concurrent calls must use separate workspaces.
  */
 
-/* Workspace bytes paged_attn_decode / paged_attn_partition / paged_attn_merge
- * need for these sizes (0 when every sequence fits one partition). */
+/* Workspace bytes for these sizes: 16 B per unit plus 2 x 64 x (head_dim + 2)
+ * fp32 per CTA, each part rounded up to 256 B. num_ctas = 0 queries the
+ * current device (KV_ERR_CUDA without one). */
 kv_status paged_attn_workspace_bytes(const kv_pool *pool, int32_t num_seqs,
-                                     int32_t num_q_heads, int32_t max_context,
-                                     int32_t partition_tokens, uint64_t *bytes);
+                                     int32_t num_q_heads, int32_t num_ctas,
+                                     uint64_t *bytes);
 
-/* The partition size the library uses for these arguments when
- * partition_tokens is 0. */
-kv_status paged_attn_default_partition(const kv_pool *pool, int32_t num_seqs,
-                                       int32_t num_q_heads, int32_t max_context,
-                                       int32_t *partition_tokens);
+/* The CTA count used when num_ctas is 0 (multiprocessors of the current
+ * device). */
+kv_status paged_attn_default_ctas(const kv_pool *pool, int32_t *num_ctas);
 
-/* Full decode attention: paged_attn_partition followed, when any sequence can
- * span more than one partition, by paged_attn_merge, on the same stream. */
+/* Full decode attention: paged_attn_partition followed by paged_attn_merge on
+ * the same stream. */
 kv_status paged_attn_decode(kv_pool *pool, int32_t layer, const void *q,
                             int32_t q_dtype, int32_t num_seqs,
                             int32_t num_q_heads, const int32_t *block_tables,
                             int32_t max_blocks_per_seq,
                             const int32_t *context_lens, int32_t max_context,
-                            float scale, void *out, int32_t partition_tokens,
+                            float scale, void *out, int32_t num_ctas,
                             void *workspace, uint64_t workspace_bytes,
                             kv_stream_t stream);
 
-/* Phase 1 alone: one CTA per (sequence, KV head, partition). Writes out[b]
- * for sequences with a single partition and the workspace partials for the
- * others. */
+/* Phase 1 alone: the persistent attention kernel. Writes out for the units it
+ * finishes and the workspace partials and bookkeeping for split units. */
 kv_status paged_attn_partition(kv_pool *pool, int32_t layer, const void *q,
                                int32_t q_dtype, int32_t num_seqs,
                                int32_t num_q_heads, const int32_t *block_tables,
                                int32_t max_blocks_per_seq,
                                const int32_t *context_lens, int32_t max_context,
-                               float scale, void *out, int32_t partition_tokens,
+                               float scale, void *out, int32_t num_ctas,
                                void *workspace, uint64_t workspace_bytes,
                                kv_stream_t stream);
 
-/* Phase 2 alone: merge the partials of sequences with more than one
- * partition into out (q_dtype). Same argument meanings as phase 1. */
-kv_status paged_attn_merge(const kv_pool *pool, int32_t num_seqs,
-                           int32_t num_q_heads, const int32_t *context_lens,
+/* Phase 2 alone: merge split units into out (out_dtype) and write zeros for
+ * empty or invalid sequences. Must follow phase 1 with the same arguments. */
+kv_status paged_attn_merge(kv_pool *pool, int32_t num_seqs, int32_t num_q_heads,
+                           const int32_t *context_lens,
                            int32_t max_blocks_per_seq, int32_t max_context,
-                           int32_t partition_tokens, int32_t out_dtype,
-                           void *out, const void *workspace,
-                           uint64_t workspace_bytes, kv_stream_t stream);
+                           int32_t num_ctas, int32_t out_dtype, void *out,
+                           void *workspace, uint64_t workspace_bytes,
+                           kv_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 

@@ -63,8 +63,8 @@ _SIGS = {
     "kv_append": [_P, _I32, _P, _P, _I32, _P, _I32, _P],
     "kv_quantize": [_P, _I32, _I64, _I32, _I32, _P, _P, _P],
     "kv_block_copy": [_P, _PI32, _I32, _P],
-    "paged_attn_workspace_bytes": [_P, _I32, _I32, _I32, _I32, _PU64],
-    "paged_attn_default_partition": [_P, _I32, _I32, _I32, _PI32],
+    "paged_attn_workspace_bytes": [_P, _I32, _I32, _I32, _PU64],
+    "paged_attn_default_ctas": [_P, _PI32],
     "paged_attn_decode": [_P, _I32, _P, _I32, _I32, _I32, _P, _I32, _P, _I32, _F, _P, _I32,
                           _P, _U64, _P],
     "paged_attn_partition": [_P, _I32, _P, _I32, _I32, _I32, _P, _I32, _P, _I32, _F, _P,
@@ -264,22 +264,21 @@ def kv_block_copy(pool, pairs, stream=None):
     check(lib.kv_block_copy(pool.handle, arr, n, _stream(stream, pool.device)))
 
 
-def workspace_bytes(pool, num_seqs, num_q_heads, max_context, partition_tokens=0):
+def workspace_bytes(pool, num_seqs, num_q_heads, num_ctas=0):
     n = ctypes.c_uint64()
-    check(lib.paged_attn_workspace_bytes(pool.handle, num_seqs, num_q_heads, max_context,
-                                         partition_tokens, ctypes.byref(n)))
+    check(lib.paged_attn_workspace_bytes(pool.handle, num_seqs, num_q_heads, num_ctas,
+                                         ctypes.byref(n)))
     return n.value
 
 
-def default_partition(pool, num_seqs, num_q_heads, max_context):
+def default_ctas(pool):
     n = ctypes.c_int32()
-    check(lib.paged_attn_default_partition(pool.handle, num_seqs, num_q_heads, max_context,
-                                           ctypes.byref(n)))
+    check(lib.paged_attn_default_ctas(pool.handle, ctypes.byref(n)))
     return n.value
 
 
-def make_workspace(pool, num_seqs, num_q_heads, max_context, partition_tokens=0):
-    n = workspace_bytes(pool, num_seqs, num_q_heads, max_context, partition_tokens)
+def make_workspace(pool, num_seqs, num_q_heads, num_ctas=0):
+    n = workspace_bytes(pool, num_seqs, num_q_heads, num_ctas)
     return torch.empty(max(n, 256), dtype=torch.uint8, device=pool.device)
 
 
@@ -300,36 +299,36 @@ def _attn_args(pool, q, block_tables, context_lens, out):
 
 
 def paged_attn_decode(pool, layer, q, block_tables, context_lens, max_context, scale,
-                      out=None, partition_tokens=0, workspace=None, stream=None):
+                      out=None, num_ctas=0, workspace=None, stream=None):
     """Decode attention of q [B, Hq, D] over the paged cache; returns out."""
     B, Hq, out = _attn_args(pool, q, block_tables, context_lens, out)
     if workspace is None:
-        workspace = make_workspace(pool, B, Hq, max_context, partition_tokens)
+        workspace = make_workspace(pool, B, Hq, num_ctas)
     check(lib.paged_attn_decode(pool.handle, layer, _ptr(q), TORCH_CODES[q.dtype], B, Hq,
                                 _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
-                                max_context, float(scale), _ptr(out), partition_tokens,
+                                max_context, float(scale), _ptr(out), num_ctas,
                                 _ptr(workspace), workspace.numel(), _stream(stream, pool.device)))
     return out
 
 
 def paged_attn_partition(pool, layer, q, block_tables, context_lens, max_context, scale,
-                         out, workspace, partition_tokens=0, stream=None):
+                         out, workspace, num_ctas=0, stream=None):
     B, Hq, out = _attn_args(pool, q, block_tables, context_lens, out)
     check(lib.paged_attn_partition(pool.handle, layer, _ptr(q), TORCH_CODES[q.dtype], B, Hq,
                                    _ptr(block_tables), block_tables.shape[1],
                                    _ptr(context_lens), max_context, float(scale), _ptr(out),
-                                   partition_tokens, _ptr(workspace), workspace.numel(),
+                                   num_ctas, _ptr(workspace), workspace.numel(),
                                    _stream(stream, pool.device)))
     return out
 
 
 def paged_attn_merge(pool, context_lens, max_blocks_per_seq, max_context, out, workspace,
-                     partition_tokens=0, stream=None):
+                     num_ctas=0, stream=None):
     _need(out, "out", (torch.bfloat16, torch.float16), pool.device)
     _need(context_lens, "context_lens", torch.int32, pool.device)
     B, Hq, _ = out.shape
     check(lib.paged_attn_merge(pool.handle, B, Hq, _ptr(context_lens), max_blocks_per_seq,
-                               max_context, partition_tokens, TORCH_CODES[out.dtype], _ptr(out),
+                               max_context, num_ctas, TORCH_CODES[out.dtype], _ptr(out),
                                _ptr(workspace), workspace.numel(),
                                _stream(stream, pool.device)))
     return out

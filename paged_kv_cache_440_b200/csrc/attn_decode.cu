@@ -12,21 +12,30 @@
 // per byte, so the kernel is bound by HBM bandwidth [KV Cache 原理与
 // PagedAttention, §四]. Design:
 //
-// * Grid: one CTA per (partition, kv head x head chunk, sequence). A partition
-//   is `part_tokens` consecutive positions (split-K); the partials are merged
-//   by a second kernel.
-// * Each of the CTA's 4 warps owns every 4th block of the partition and a
-//   private ring of R shared-memory stages. Lane 0 of the warp fills a stage
-//   with TMA: the (block, head) K tile and V tile, each a contiguous
-//   block_size x head_dim slab of the pool, land swizzled so that fragment
-//   loads are bank-conflict free; the per-token scales of a quantized cache
-//   come along with 1-D bulk copies. Completion is signalled on an mbarrier;
-//   every wait has a time limit.
+// * Work: a "unit" is one sequence and a group of HG consecutive KV heads
+//   (with all their query heads, in chunks of up to 8). Its positions are the
+//   sequence's ceil(L / block_size) blocks. All units' positions are laid end
+//   to end and split evenly over a persistent grid (by default one CTA per
+//   SM): every CTA streams the same number of positions, whatever the length
+//   mix. A CTA's range can cut a unit only at its two ends, so each CTA emits
+//   at most two partial results per head (split-K); a unit inside one CTA is
+//   finished there. A merge kernel combines the split units.
+// * Inside a CTA one producer warp streams, for each position, the K and V
+//   rows of all HG heads of that block -- contiguous in the pool -- into a
+//   ring of shared-memory stages with a few large TMA box loads (16 KB each
+//   for bf16, 128-byte swizzled so fragment loads are bank-conflict free);
+//   the per-token scales of a quantized cache come with 1-D bulk copies.
+//   Large requests matter: the copy engine spends a roughly fixed time per
+//   request, so small tiles cannot keep HBM busy. Eight consumer warps each
+//   own one (KV head, query-head chunk) of the unit and keep its online
+//   softmax state in registers across the unit's blocks; full/empty
+//   mbarriers link producer and consumers, every wait has a time limit.
 // * GQA groups (Hq / Hkv >= 2) make q K^T a dense [16 tokens x 128] x
 //   [128 x 8 heads] tile: warp-level tensor-core MMA (m16n8k16) with tokens as
 //   M and up to 8 query heads as N. P V runs as V^T P^T with head_dim as M,
 //   the probabilities turned from accumulator to operand layout by an
-//   in-register 8x8 transpose. Online softmax in fp32 (base 2) per head.
+//   in-register 8x8 transpose and fed as two 16-bit parts (hi + lo) so P V
+//   keeps fp32-level accuracy. Online softmax in fp32 (base 2) per head.
 // * MHA (one query head per KV head) is a matrix-vector product; it stays on
 //   CUDA cores: each half-warp covers one token row (16 lanes x head_dim/16
 //   values), partial dot products are reduced with a butterfly that leaves
@@ -35,7 +44,6 @@
 //   multiply the scores, per-token V scales are folded into the softmax
 //   weights through log2(scale) so the fp16 weights stay within (0, 1].
 #include <algorithm>
-#include <mutex>
 
 #include "device.cuh"
 #include "internal.h"
@@ -45,9 +53,13 @@ namespace {
 
 using namespace dev;
 
-constexpr int kNW = 4;  // warps per CTA
-constexpr int kThreads = kNW * 32;
-constexpr int kMaxPartBlocks = 512;  // partition_tokens / block_size
+constexpr int kNC = 8;                    // consumer warps (one per slot of a unit)
+constexpr int kWarps = kNC + 1;           // + one producer warp
+constexpr int kThreads = kWarps * 32;
+constexpr int kRingBytes = 200 * 1024;    // shared-memory stages per CTA
+constexpr int kMaxStageBytes = 96 * 1024; // at least two stages
+constexpr int kMaxStages = 8;
+constexpr int kChunkHeads = 8;            // query heads of one slot (MMA N)
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct AttnParams {
@@ -57,21 +69,26 @@ struct AttnParams {
   const int32_t *context_lens;
   const float *k_scale;
   const float *v_scale;
-  float *ws_o;
-  float *ws_m;
-  float *ws_l;
+  float *part_o;   // [num_ctas][2][kNC][8][D]   unnormalised outputs of split units
+  float *part_ml;  // [num_ctas][2][kNC][8][2]   their (max, sum), base 2
+  int4 *meta;      // [num_seqs * units_per_seq]: first CTA, #CTAs, first side
   int *status;
   float scale_log2;  // scale * log2(e)
   int num_seqs;
   int q_heads;
   int kv_heads;
-  int group;       // q heads per kv head
-  int chunks;      // ceil(group / 8)
-  int max_blocks;  // block-table row length
-  int num_blocks;  // physical blocks in the pool
-  int limit;       // min(max_context, max_blocks * block_size)
-  int part_tokens;
-  int max_parts;
+  int group;           // q heads per kv head
+  int chunks;          // 8-head chunks per kv head: ceil(group / 8), 1 for MHA
+  int hg;              // kv heads per unit (HG)
+  int cpg;             // chunks per unit (<= kNC)
+  int cgroups;         // chunk groups per kv head: ceil(chunks / cpg)
+  int units_per_seq;   // (kv_heads / hg) * cgroups
+  int stage_bytes;     // bytes between ring stages (load size rounded to 1024)
+  int stages;          // ring stages (R)
+  int max_blocks;      // block-table row length
+  int num_blocks;      // physical blocks in the pool
+  int limit;           // valid lengths: 0 < L <= min(max_context, max_blocks * bs)
+  int num_ctas;
 };
 
 constexpr int align_up_c(int x, int a) { return (x + a - 1) / a * a; }
@@ -87,17 +104,22 @@ struct Tile {
   static constexpr int kRowBytes = D * kElt;
   static constexpr int kSlab = kRowBytes >= 128 ? 128 : kRowBytes;  // TMA box width, bytes
   static constexpr int kSlabs = kRowBytes / kSlab;
-  static constexpr int kTileBytes = BS * kRowBytes;
   static constexpr bool kQuant = !is16<KV_T>();
-  static constexpr int kLoadBytes = 2 * kTileBytes + (kQuant ? 2 * BS * 4 : 0);
-  static constexpr int kStageBytes = align_up_c(kLoadBytes, 1024);
 
-  // Shared-memory address of 16-byte chunk c of row r of a tile, as the TMA
-  // swizzle placed it (128-byte swizzle on 128-byte slabs, 64-byte swizzle on
-  // 64-byte rows; a 256-byte row is two slabs, each its own BS x 128 block).
-  __device__ __forceinline__ static uint32_t chunk(uint32_t tile, int r, int c) {
+  // A stage holds `rows` = HG * BS rows (HG heads of one block) of K, then of
+  // V, each as kSlabs slabs of rows x kSlab bytes, then (quantized caches) the
+  // K and V scales of those rows.
+  __host__ __device__ static constexpr int load_bytes(int rows) {
+    return 2 * rows * kRowBytes + (kQuant ? 2 * rows * 4 : 0);
+  }
+
+  // Shared-memory address of 16-byte chunk c of row r of the K (or V) part of
+  // a stage, as the TMA swizzle placed it: 128-byte swizzle on 128-byte slabs,
+  // 64-byte swizzle on 64-byte rows. Rows of one head start at a multiple of
+  // BS (a multiple of 8), so the swizzle phase of a head's row r is r's.
+  __device__ __forceinline__ static uint32_t chunk(uint32_t tile, int r, int c, int rows) {
     if constexpr (kRowBytes == 256) {
-      return tile + (((c >> 3) * BS + r) << 7) + (((c & 7) ^ (r & 7)) << 4);
+      return tile + (c >> 3) * rows * 128 + (r << 7) + (((c & 7) ^ (r & 7)) << 4);
     } else if constexpr (kRowBytes == 128) {
       return tile + (r << 7) + ((c ^ (r & 7)) << 4);
     } else {
@@ -106,30 +128,28 @@ struct Tile {
   }
 };
 
-template <int D, int BS, int KV_T>
-constexpr int smem_bytes() {
-  return kNW * 3 * Tile<D, BS, KV_T>::kStageBytes + 1024;
-}
-
+// Fill one stage with block `id` of the unit's HG heads (rows row0 ..
+// row0 + rows - 1 of the pool's 2-D view); an invalid id completes the phase
+// without data.
 template <int D, int BS, int KV_T>
 __device__ __forceinline__ void issue_stage(uint8_t *stage, uint64_t *bar, const CUtensorMap *km,
-                                            const CUtensorMap *vm, int id, int g,
+                                            const CUtensorMap *vm, int id, int row0, int rows,
                                             const AttnParams &p) {
   using T = Tile<D, BS, KV_T>;
-  if (id < 0) {  // invalid block: complete the phase with no data
+  if (id < 0) {
     mbar_arrive(bar);
     return;
   }
-  mbar_arrive_expect_tx(bar, T::kLoadBytes);
-  const int y = (id * p.kv_heads + g) * BS;
+  mbar_arrive_expect_tx(bar, T::load_bytes(rows));
+  const int kv = rows * T::kRowBytes;
 #pragma unroll
   for (int s = 0; s < T::kSlabs; ++s) {
-    tma_load_2d(stage + s * BS * T::kSlab, km, bar, s * (T::kSlab / T::kElt), y);
-    tma_load_2d(stage + T::kTileBytes + s * BS * T::kSlab, vm, bar, s * (T::kSlab / T::kElt), y);
+    tma_load_2d(stage + s * rows * T::kSlab, km, bar, s * (T::kSlab / T::kElt), row0);
+    tma_load_2d(stage + kv + s * rows * T::kSlab, vm, bar, s * (T::kSlab / T::kElt), row0);
   }
   if constexpr (T::kQuant) {
-    bulk_load(stage + 2 * T::kTileBytes, p.k_scale + y, BS * 4, bar);
-    bulk_load(stage + 2 * T::kTileBytes + BS * 4, p.v_scale + y, BS * 4, bar);
+    bulk_load(stage + 2 * kv, p.k_scale + row0, rows * 4, bar);
+    bulk_load(stage + 2 * kv + rows * 4, p.v_scale + row0, rows * 4, bar);
   }
 }
 
@@ -194,176 +214,177 @@ __device__ __forceinline__ void load_vals(uint32_t addr, float (&v)[E]) {
   }
 }
 
-// Per-warp softmax state handed to the CTA-level combine (shared memory).
-struct CombineSlot {
-  float m[8];
-  float l[8];
-};
 
-// ============================================================================
-// Partition kernel
-// ============================================================================
-template <int D, int BS, int KV_T, int Q_T, bool MMA>
-__global__ void __launch_bounds__(kThreads)
-attn_partition_kernel(const __grid_constant__ CUtensorMap kmap,
-                      const __grid_constant__ CUtensorMap vmap, const AttnParams p) {
-  using T = Tile<D, BS, KV_T>;
-  constexpr int R = 3;  // stages per warp
-  constexpr bool kQuant = T::kQuant;
-  constexpr bool kBF = (KV_T == KV_BF16);  // MMA operand type (bf16, else fp16)
+// KV blocks of sequence b; 0 for an empty or invalid length.
+template <int BS>
+__device__ __forceinline__ int seq_blocks(const AttnParams &p, int b) {
+  const int L = p.context_lens[b];
+  return (L > 0 && L <= p.limit) ? (L + BS - 1) / BS : 0;
+}
 
-  extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bars[kNW * R];
-  __shared__ int32_t bt_s[kMaxPartBlocks];
-  __shared__ CombineSlot comb[kNW];
-  uint8_t *smem = reinterpret_cast<uint8_t *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+// Even split of T blocks over G CTAs: CTA c gets q + 1 blocks if c < r, else q.
+__device__ __forceinline__ long long cta_start(long long c, long long T, long long G) {
+  const long long q = T / G, r = T % G;
+  return c * q + (c < r ? c : r);
+}
+__device__ __forceinline__ int cta_of(long long x, long long T, long long G) {
+  const long long q = T / G, r = T % G;
+  if (x < r * (q + 1)) return static_cast<int>(x / (q + 1));
+  return static_cast<int>(r + (x - r * (q + 1)) / q);
+}
 
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  const int b = blockIdx.z;
-  const int g = blockIdx.y / p.chunks;
-  const int chunk = blockIdx.y - g * p.chunks;
-  const int part = blockIdx.x;
-  const int S = p.part_tokens;
+__device__ __forceinline__ long long block_sum(long long v, long long *red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  long long t = 0;
+#pragma unroll
+  for (int i = 0; i < kWarps; ++i) t += red[i];
+  __syncthreads();
+  return t;
+}
 
-  int L = p.context_lens[b];
-  if (L < 0 || L > p.limit) {
-    if (threadIdx.x == 0 && part == 0 && blockIdx.y == 0) atomicOr(p.status, kErrContext);
-    L = 0;
+// Exclusive prefix sum over the CTA's threads; *total gets the CTA's sum.
+__device__ __forceinline__ long long block_excl_scan(long long v, long long *red,
+                                                     long long *total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  long long x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
   }
-  const int nparts = L > 0 ? (L + S - 1) / S : 1;
-  if (part >= nparts) return;
-  const int tok0 = part * S;
-  const int tok1 = min(L, tok0 + S);
-  const int blk0 = tok0 / BS;
-  const int nblk = L > 0 ? (tok1 - tok0 + BS - 1) / BS : 0;
-  const int h0 = g * p.group + chunk * 8;
-  const int nh = MMA ? min(8, p.group - chunk * 8) : 1;
-
-  if (threadIdx.x == 0) {
-    prefetch_tmap(&kmap);
-    prefetch_tmap(&vmap);
-    for (int i = 0; i < kNW * R; ++i) mbar_init(&bars[i], 1);
-    fence_barrier_init();
-  }
-  // The partition's slice of the block table; ids outside the pool are
-  // reported and the block treated as empty (no load is issued for it).
-  const int32_t *bt_row = p.block_tables + static_cast<int64_t>(b) * p.max_blocks + blk0;
-  for (int i = threadIdx.x; i < nblk; i += kThreads) {
-    int id = bt_row[i];
-    if (id < 0 || id >= p.num_blocks) {
-      atomicOr(p.status, kErrBlockId);
-      id = -1;
-    }
-    bt_s[i] = id;
+  if (lane == 31) red[warp] = x;
+  __syncthreads();
+  long long before = 0, tot = 0;
+#pragma unroll
+  for (int i = 0; i < kWarps; ++i) {
+    before += i < warp ? red[i] : 0;
+    tot += red[i];
   }
   __syncthreads();
+  *total = tot;
+  return before + x - v;
+}
 
-  // ------------------------------------------------------------- per warp
-  const int n_it = warp < nblk ? (nblk - warp + kNW - 1) / kNW : 0;
-  uint8_t *wstage = smem + warp * R * T::kStageBytes;
-  uint64_t *wbar = bars + warp * R;
-  if (lane == 0) {
-    for (int it = 0; it < R && it < n_it; ++it)
-      issue_stage<D, BS, KV_T>(wstage + it * T::kStageBytes, &wbar[it], &kmap, &vmap,
-                               bt_s[warp + it * kNW], g, p);
+// Waits on a ring barrier; gives up when another warp has aborted or the time
+// limit passes (then raises the CTA's abort flag and the device status bit).
+__device__ __forceinline__ bool ring_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                          int *status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63) == 0) {
+      if (*abort) return false;
+      if (globaltimer() - t0 > kWaitLimitNs) {
+        *abort = 1;
+        atomicOr(status, kErrTimeout);
+        return false;
+      }
+    }
   }
-  __syncwarp();
+}
 
-  const int gq = lane >> 2;  // MMA fragment row group
-  const int cq = lane & 3;   // MMA fragment column pair
+// ============================================================================
+// Consumer: per-warp state and the work on one staged block.
+// ============================================================================
+template <int D, int BS, int KV_T, int Q_T, bool MMA>
+struct Consumer {
+  using T = Tile<D, BS, KV_T>;
+  static constexpr bool kQuant = T::kQuant;
+  static constexpr bool kBF = (KV_T == KV_BF16);  // MMA operand type (bf16, else fp16)
+  static constexpr int KS = D / 16;  // k-steps over head_dim
+  static constexpr int MT = BS / 16;  // 16-token tiles per block
+  static constexpr int E = D / 16;  // values per lane in a half-warp row (scalar path)
 
-  // softmax state (MMA: heads 2cq, 2cq+1; scalar: the one head)
-  float m_run[2] = {-INFINITY, -INFINITY};   // max of scores (base 2)
-  float m2_run[2] = {-INFINITY, -INFINITY};  // max of scores + log2(v scale) (quant)
-  float l_run[2] = {0.f, 0.f};
+  float m_run[2], m2_run[2], l_run[2];
+  float oacc[MMA ? D / 16 : 1][4];
+  float oacc_s[MMA ? 1 : E];
+  uint32_t qb[MMA ? KS : 1][2];
+  float qs[MMA ? 1 : E];
+  float s_fac[2];
 
-  // ---------------------------------------------------------------- MMA path
-  constexpr int KS = D / 16;  // k-steps over head_dim
-  constexpr int MT = BS / 16;  // 16-token tiles per block
-  uint32_t qb[KS][2];
-  float oacc[D / 16][4];
-  float s_fac[2] = {p.scale_log2, p.scale_log2};
-  // ------------------------------------------------------------- scalar path
-  constexpr int E = D / 16;  // values per lane in a half-warp row
-  float qs[E];
-  float oacc_s[E];
-  const int hw = lane >> 4, jl = lane & 15;
-
-  if constexpr (MMA) {
+  __device__ __forceinline__ void reset() {
+    m_run[0] = m_run[1] = m2_run[0] = m2_run[1] = -INFINITY;
+    l_run[0] = l_run[1] = 0.f;
+    if constexpr (MMA) {
 #pragma unroll
-    for (int i = 0; i < D / 16; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
-    const bool hv = gq < nh;
-    const int64_t qrow = (static_cast<int64_t>(b) * p.q_heads + h0 + gq) * D;
-    if constexpr (!kQuant) {
-      // B operand: k = head_dim index, n = head. Lane (gq, cq) holds dims
-      // 16ks + 2cq, +1 and 16ks + 8 + 2cq, +1 of head gq.
-      const uint32_t *q32 = static_cast<const uint32_t *>(p.q);
+      for (int i = 0; i < D / 16; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
+    } else {
 #pragma unroll
-      for (int ks = 0; ks < KS; ++ks) {
-        qb[ks][0] = hv ? q32[(qrow + 16 * ks + 2 * cq) >> 1] : 0u;
-        qb[ks][1] = hv ? q32[(qrow + 16 * ks + 8 + 2 * cq) >> 1] : 0u;
+      for (int e = 0; e < E; ++e) oacc_s[e] = 0.f;
+    }
+  }
+
+  // Query fragments of heads h0 .. h0 + nh - 1 of sequence b.
+  __device__ __forceinline__ void load_query(const AttnParams &p, int b, int h0, int nh, int lane) {
+    const int gq = lane >> 2, cq = lane & 3;
+    s_fac[0] = s_fac[1] = p.scale_log2;
+    if constexpr (MMA) {
+      const bool hv = gq < nh;
+      const int64_t qrow = (static_cast<int64_t>(b) * p.q_heads + h0 + gq) * D;
+      if constexpr (!kQuant) {
+        // B operand: k = head_dim index, n = head. Lane (gq, cq) holds dims
+        // 16ks + 2cq, +1 and 16ks + 8 + 2cq, +1 of head gq.
+        const uint32_t *q32 = static_cast<const uint32_t *>(p.q);
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          qb[ks][0] = hv ? q32[(qrow + 16 * ks + 2 * cq) >> 1] : 0u;
+          qb[ks][1] = hv ? q32[(qrow + 16 * ks + 8 + 2 * cq) >> 1] : 0u;
+        }
+      } else {
+        // fp16 operands: q scaled per head by a power of two so its largest
+        // magnitude is in [2^14, 2^15) (exact), the scale folded into s_fac.
+        // k-slot order matches the code fragments: lane (gq, cq) holds dims
+        // 16ks + 4cq .. 16ks + 4cq + 3.
+        float qv[KS][4];
+        float amax = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            qv[ks][e] = hv ? load_q<Q_T>(p.q, qrow + 16 * ks + 4 * cq + e) : 0.f;
+            amax = fmaxf(amax, fabsf(qv[ks][e]));
+          }
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        int ex = 0;
+        if (amax > 0.f) {
+          frexpf(amax, &ex);
+          ex = 15 - ex;  // amax * 2^ex in [2^14, 2^15)
+        }
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          qb[ks][0] = pack2<false>(ldexpf(qv[ks][0], ex), ldexpf(qv[ks][1], ex));
+          qb[ks][1] = pack2<false>(ldexpf(qv[ks][2], ex), ldexpf(qv[ks][3], ex));
+        }
+        // the score columns of this lane are heads 2cq and 2cq+1
+        const int ex0 = __shfl_sync(0xffffffffu, ex, (2 * cq) * 4);
+        const int ex1 = __shfl_sync(0xffffffffu, ex, (2 * cq + 1) * 4);
+        s_fac[0] = ldexpf(p.scale_log2, -ex0);
+        s_fac[1] = ldexpf(p.scale_log2, -ex1);
       }
     } else {
-      // fp16 operands: q scaled per head by a power of two so its largest
-      // magnitude is in [2^14, 2^15) (exact), the scale folded into s_fac.
-      // k-slot order matches the code fragments: lane (gq, cq) holds dims
-      // 16ks + 4cq .. 16ks + 4cq + 3.
-      float qv[KS][4];
-      float amax = 0.f;
+      const int jl = lane & 15;
 #pragma unroll
-      for (int ks = 0; ks < KS; ++ks)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          qv[ks][e] = hv ? load_q<Q_T>(p.q, qrow + 16 * ks + 4 * cq + e) : 0.f;
-          amax = fmaxf(amax, fabsf(qv[ks][e]));
-        }
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-      int ex = 0;
-      if (amax > 0.f) {
-        frexpf(amax, &ex);
-        ex = 15 - ex;  // amax * 2^ex in [2^14, 2^15)
-      }
-#pragma unroll
-      for (int ks = 0; ks < KS; ++ks) {
-        qb[ks][0] = pack2<false>(ldexpf(qv[ks][0], ex), ldexpf(qv[ks][1], ex));
-        qb[ks][1] = pack2<false>(ldexpf(qv[ks][2], ex), ldexpf(qv[ks][3], ex));
-      }
-      // the score columns of this lane are heads 2cq and 2cq+1
-      const int ex0 = __shfl_sync(0xffffffffu, ex, (2 * cq) * 4);
-      const int ex1 = __shfl_sync(0xffffffffu, ex, (2 * cq + 1) * 4);
-      s_fac[0] = ldexpf(p.scale_log2, -ex0);
-      s_fac[1] = ldexpf(p.scale_log2, -ex1);
-    }
-  } else {
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-      qs[e] = load_q<Q_T>(p.q, (static_cast<int64_t>(b) * p.q_heads + h0) * D + jl * E + e) *
-              p.scale_log2;
-      oacc_s[e] = 0.f;
+      for (int e = 0; e < E; ++e)
+        qs[e] = load_q<Q_T>(p.q, (static_cast<int64_t>(b) * p.q_heads + h0) * D + jl * E + e) *
+                p.scale_log2;
     }
   }
 
-  bool alive = true;
-  int it = 0;
-  for (; it < n_it; ++it) {
-    const int s = it % R;
-    uint8_t *st = wstage + s * T::kStageBytes;
-    if (!mbar_wait(&wbar[s], (it / R) & 1, p.status)) {
-      alive = false;
-      break;
-    }
-    const int j = warp + it * kNW;
-    const int id = bt_s[j];
-    const int tok_base = (blk0 + j) * BS;
-    const int valid = id >= 0 ? min(BS, tok1 - tok_base) : 0;
+  // One staged block of head `hi` of the stage's `rows`-row group: rows
+  // [0, valid) of the head's BS rows are real tokens.
+  __device__ __forceinline__ void block(const uint8_t *st, int rows, int hi, int valid, int lane) {
     const uint32_t ktile = smem_u32(st);
-    const uint32_t vtile = ktile + T::kTileBytes;
-    const float *ksc = reinterpret_cast<const float *>(st + 2 * T::kTileBytes);
-    const float *vsc = ksc + BS;
-
+    const uint32_t vtile = ktile + rows * T::kRowBytes;
+    const int r0 = hi * BS;  // the head's first row in the stage
+    const float *ksc = reinterpret_cast<const float *>(st + 2 * rows * T::kRowBytes) + r0;
+    const float *vsc = ksc + rows;
+    const int gq = lane >> 2, cq = lane & 3;
     if constexpr (MMA) {
       // ---------------------------------------------------- scores S = K q
       float sc[MT][4];
@@ -375,44 +396,43 @@ attn_partition_kernel(const __grid_constant__ CUtensorMap kmap,
 #pragma unroll
           for (int ks = 0; ks < KS; ++ks) {
             uint32_t a0, a1, a2, a3;
-            ldsm_x4(T::chunk(ktile, row, 2 * ks + (lane >> 4)), a0, a1, a2, a3);
+            ldsm_x4(T::chunk(ktile, r0 + row, 2 * ks + (lane >> 4), rows), a0, a1, a2, a3);
             mma16816<kBF>(acc, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
           }
         } else {
 #pragma unroll
           for (int kp = 0; kp < KS / 2; ++kp) {
-            uint32_t r0, r1, r2, r3;  // byte matrices: rows 0-7 / 8-15 x chunks 2kp, 2kp+1
-            ldsm_x4(T::chunk(ktile, row, 2 * kp + (lane >> 4)), r0, r1, r2, r3);
+            uint32_t q0, q1, q2, q3;  // byte matrices: rows 0-7 / 8-15 x chunks 2kp, 2kp+1
+            ldsm_x4(T::chunk(ktile, r0 + row, 2 * kp + (lane >> 4), rows), q0, q1, q2, q3);
             if constexpr (KV_T == KV_INT8) {
-              r0 ^= 0x80808080u; r1 ^= 0x80808080u; r2 ^= 0x80808080u; r3 ^= 0x80808080u;
-              mma16816<false>(acc, int8_pair<0, 1>(r0), int8_pair<0, 1>(r1),
-                              int8_pair<2, 3>(r0), int8_pair<2, 3>(r1), qb[2 * kp][0],
+              q0 ^= 0x80808080u; q1 ^= 0x80808080u; q2 ^= 0x80808080u; q3 ^= 0x80808080u;
+              mma16816<false>(acc, int8_pair<0, 1>(q0), int8_pair<0, 1>(q1),
+                              int8_pair<2, 3>(q0), int8_pair<2, 3>(q1), qb[2 * kp][0],
                               qb[2 * kp][1]);
-              mma16816<false>(acc, int8_pair<0, 1>(r2), int8_pair<0, 1>(r3),
-                              int8_pair<2, 3>(r2), int8_pair<2, 3>(r3), qb[2 * kp + 1][0],
+              mma16816<false>(acc, int8_pair<0, 1>(q2), int8_pair<0, 1>(q3),
+                              int8_pair<2, 3>(q2), int8_pair<2, 3>(q3), qb[2 * kp + 1][0],
                               qb[2 * kp + 1][1]);
             } else {
-              mma16816<false>(acc, e5m2_pair<0, 1>(r0), e5m2_pair<0, 1>(r1),
-                              e5m2_pair<2, 3>(r0), e5m2_pair<2, 3>(r1), qb[2 * kp][0],
+              mma16816<false>(acc, e5m2_pair<0, 1>(q0), e5m2_pair<0, 1>(q1),
+                              e5m2_pair<2, 3>(q0), e5m2_pair<2, 3>(q1), qb[2 * kp][0],
                               qb[2 * kp][1]);
-              mma16816<false>(acc, e5m2_pair<0, 1>(r2), e5m2_pair<0, 1>(r3),
-                              e5m2_pair<2, 3>(r2), e5m2_pair<2, 3>(r3), qb[2 * kp + 1][0],
+              mma16816<false>(acc, e5m2_pair<0, 1>(q2), e5m2_pair<0, 1>(q3),
+                              e5m2_pair<2, 3>(q2), e5m2_pair<2, 3>(q3), qb[2 * kp + 1][0],
                               qb[2 * kp + 1][1]);
             }
           }
         }
         // acc: [0],[1] = token mt*16+gq, heads 2cq, 2cq+1; [2],[3] = token +8
         const int t0 = mt * 16 + gq, t1 = t0 + 8;
-        float f0 = s_fac[0], f1 = s_fac[1];
         float k0 = 1.f, k1 = 1.f;
         if constexpr (kQuant) {
           k0 = ksc[t0];
           k1 = ksc[t1];
         }
-        sc[mt][0] = t0 < valid ? acc[0] * f0 * k0 : -INFINITY;
-        sc[mt][1] = t0 < valid ? acc[1] * f1 * k0 : -INFINITY;
-        sc[mt][2] = t1 < valid ? acc[2] * f0 * k1 : -INFINITY;
-        sc[mt][3] = t1 < valid ? acc[3] * f1 * k1 : -INFINITY;
+        sc[mt][0] = t0 < valid ? acc[0] * s_fac[0] * k0 : -INFINITY;
+        sc[mt][1] = t0 < valid ? acc[1] * s_fac[1] * k0 : -INFINITY;
+        sc[mt][2] = t1 < valid ? acc[2] * s_fac[0] * k1 : -INFINITY;
+        sc[mt][3] = t1 < valid ? acc[3] * s_fac[1] * k1 : -INFINITY;
       }
       // ---------------------------------------------------- online softmax
       float bm0 = -INFINITY, bm1 = -INFINITY;
@@ -487,12 +507,18 @@ attn_partition_kernel(const __grid_constant__ CUtensorMap kmap,
       // ---------------------------------------------------- O^T += V^T P^T
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
-        // P^T operand (k = token, n = head) from the score layout by transpose
-        const uint32_t pb0 = movmatrix_t(pack2<kBF>(w[mt][0], w[mt][1]));
-        const uint32_t pb1 = movmatrix_t(pack2<kBF>(w[mt][2], w[mt][3]));
+        // P^T operand (k = token, n = head) from the score layout by transpose,
+        // as a hi and a lo part so that the weights keep ~fp32 accuracy
+        uint32_t h0, l0, h1, l1;
+        split2<kBF>(w[mt][0], w[mt][1], h0, l0);
+        split2<kBF>(w[mt][2], w[mt][3], h1, l1);
+        const uint32_t pb0 = movmatrix_t(h0), pb1 = movmatrix_t(h1);
+        const uint32_t pl0 = movmatrix_t(l0), pl1 = movmatrix_t(l1);
         // token rows this lane's V^T fragments cover: 2cq, 2cq+1, 2cq+8, 2cq+9
         const int tb = mt * 16 + 2 * cq;
         const bool full = (mt * 16 + 16) <= valid;
+        const uint32_t m0 = (tb < valid ? 0xFFFFu : 0u) | (tb + 1 < valid ? 0xFFFF0000u : 0u);
+        const uint32_t m1 = (tb + 8 < valid ? 0xFFFFu : 0u) | (tb + 9 < valid ? 0xFFFF0000u : 0u);
         if constexpr (!kQuant) {
 #pragma unroll
           for (int dt = 0; dt < D / 16; ++dt) {
@@ -500,65 +526,62 @@ attn_partition_kernel(const __grid_constant__ CUtensorMap kmap,
             // matrices: tokens 0-7 / chunk 2dt, tokens 0-7 / 2dt+1,
             //           tokens 8-15 / 2dt, tokens 8-15 / 2dt+1
             const int vr = mt * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
-            ldsm_x4_t(T::chunk(vtile, vr, 2 * dt + ((lane >> 3) & 1)), a0, a1, a2, a3);
+            ldsm_x4_t(T::chunk(vtile, r0 + vr, 2 * dt + ((lane >> 3) & 1), rows), a0, a1, a2, a3);
             if (!full) {  // zero rows past the valid length (stale data may be NaN)
-              const uint32_t lo0 = tb < valid ? 0xFFFFu : 0u, hi0 = tb + 1 < valid ? 0xFFFF0000u : 0u;
-              const uint32_t lo1 = tb + 8 < valid ? 0xFFFFu : 0u,
-                             hi1 = tb + 9 < valid ? 0xFFFF0000u : 0u;
-              a0 &= lo0 | hi0;
-              a1 &= lo0 | hi0;
-              a2 &= lo1 | hi1;
-              a3 &= lo1 | hi1;
+              a0 &= m0;
+              a1 &= m0;
+              a2 &= m1;
+              a3 &= m1;
             }
             mma16816<kBF>(oacc[dt], a0, a1, a2, a3, pb0, pb1);
+            mma16816<kBF>(oacc[dt], a0, a1, a2, a3, pl0, pl1);
           }
         } else {
 #pragma unroll
           for (int cp = 0; cp < D / 32; ++cp) {
             // byte matrices: tokens 0-7 / chunk 2cp, tokens 8-15 / 2cp,
             //                tokens 0-7 / 2cp+1, tokens 8-15 / 2cp+1
-            uint32_t r0, r1, r2, r3;
+            uint32_t q0, q1, q2, q3;
             const int vr = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-            ldsm_x4_t(T::chunk(vtile, vr, 2 * cp + (lane >> 4)), r0, r1, r2, r3);
+            ldsm_x4_t(T::chunk(vtile, r0 + vr, 2 * cp + (lane >> 4), rows), q0, q1, q2, q3);
             // after the transpose a lane holds tokens (2cq, 2cq+1) x dims (2gq, 2gq+1)
             // of each 16-dim chunk: bytes 0,2 -> dim 2gq; bytes 1,3 -> dim 2gq+1
             uint32_t a[8];
             if constexpr (KV_T == KV_INT8) {
-              r0 ^= 0x80808080u; r1 ^= 0x80808080u; r2 ^= 0x80808080u; r3 ^= 0x80808080u;
-              a[0] = int8_pair<0, 2>(r0); a[1] = int8_pair<1, 3>(r0);
-              a[2] = int8_pair<0, 2>(r1); a[3] = int8_pair<1, 3>(r1);
-              a[4] = int8_pair<0, 2>(r2); a[5] = int8_pair<1, 3>(r2);
-              a[6] = int8_pair<0, 2>(r3); a[7] = int8_pair<1, 3>(r3);
+              q0 ^= 0x80808080u; q1 ^= 0x80808080u; q2 ^= 0x80808080u; q3 ^= 0x80808080u;
+              a[0] = int8_pair<0, 2>(q0); a[1] = int8_pair<1, 3>(q0);
+              a[2] = int8_pair<0, 2>(q1); a[3] = int8_pair<1, 3>(q1);
+              a[4] = int8_pair<0, 2>(q2); a[5] = int8_pair<1, 3>(q2);
+              a[6] = int8_pair<0, 2>(q3); a[7] = int8_pair<1, 3>(q3);
             } else {
-              a[0] = e5m2_pair<0, 2>(r0); a[1] = e5m2_pair<1, 3>(r0);
-              a[2] = e5m2_pair<0, 2>(r1); a[3] = e5m2_pair<1, 3>(r1);
-              a[4] = e5m2_pair<0, 2>(r2); a[5] = e5m2_pair<1, 3>(r2);
-              a[6] = e5m2_pair<0, 2>(r3); a[7] = e5m2_pair<1, 3>(r3);
+              a[0] = e5m2_pair<0, 2>(q0); a[1] = e5m2_pair<1, 3>(q0);
+              a[2] = e5m2_pair<0, 2>(q1); a[3] = e5m2_pair<1, 3>(q1);
+              a[4] = e5m2_pair<0, 2>(q2); a[5] = e5m2_pair<1, 3>(q2);
+              a[6] = e5m2_pair<0, 2>(q3); a[7] = e5m2_pair<1, 3>(q3);
             }
             if (!full) {
-              const uint32_t m0 = (tb < valid ? 0xFFFFu : 0u) | (tb + 1 < valid ? 0xFFFF0000u : 0u);
-              const uint32_t m1 =
-                  (tb + 8 < valid ? 0xFFFFu : 0u) | (tb + 9 < valid ? 0xFFFF0000u : 0u);
               a[0] &= m0; a[1] &= m0; a[2] &= m1; a[3] &= m1;
               a[4] &= m0; a[5] &= m0; a[6] &= m1; a[7] &= m1;
             }
             // M rows: gq -> dim 16c + 2gq, gq+8 -> dim 16c + 2gq + 1
             mma16816<false>(oacc[2 * cp], a[0], a[1], a[2], a[3], pb0, pb1);
+            mma16816<false>(oacc[2 * cp], a[0], a[1], a[2], a[3], pl0, pl1);
             mma16816<false>(oacc[2 * cp + 1], a[4], a[5], a[6], a[7], pb0, pb1);
+            mma16816<false>(oacc[2 * cp + 1], a[4], a[5], a[6], a[7], pl0, pl1);
           }
         }
       }
     } else {
       // ====================================================== scalar (MHA)
       constexpr int NV = BS / 2;  // tokens per half-warp: rows 2i + hw
+      const int hw = lane >> 4, jl = lane & 15;
       float part_s[NV];
 #pragma unroll
       for (int i = 0; i < NV; ++i) {
         const int r = 2 * i + hw;
         float kv[E];
         const uint32_t boff = jl * E * T::kElt;  // byte offset of this lane's values in the row
-        const uint32_t addr = T::chunk(ktile, r, boff >> 4) + (boff & 15);
-        load_vals<KV_T, E>(addr, kv);
+        load_vals<KV_T, E>(T::chunk(ktile, r0 + r, boff >> 4, rows) + (boff & 15), kv);
         float a = 0.f;
 #pragma unroll
         for (int e = 0; e < E; ++e) a = fmaf(qs[e], kv[e], a);
@@ -607,150 +630,384 @@ attn_partition_kernel(const __grid_constant__ CUtensorMap kmap,
           if constexpr (kQuant) pi *= vsc[rr];
           float vv[E];
           const uint32_t boff = jl * E * T::kElt;
-          const uint32_t addr = T::chunk(vtile, rr, boff >> 4) + (boff & 15);
-          load_vals<KV_T, E>(addr, vv);
+          load_vals<KV_T, E>(T::chunk(vtile, r0 + rr, boff >> 4, rows) + (boff & 15), vv);
 #pragma unroll
           for (int e = 0; e < E; ++e) oacc_s[e] = fmaf(pi, vv[e], oacc_s[e]);
         }
       }
       l_run[0] = l_run[0] * al + lsum;
     }
-    __syncwarp();
-    if (lane == 0 && it + R < n_it)
-      issue_stage<D, BS, KV_T>(st, &wbar[s], &kmap, &vmap, bt_s[warp + (it + R) * kNW], g, p);
-  }
-  if (!alive) {
-    // drain the stages still in flight (bounded) before shared memory is reused
-    for (int k = it + 1; k < n_it && k < it + R; ++k) mbar_wait(&wbar[k % R], (k / R) & 1, p.status);
-    m_run[0] = m_run[1] = m2_run[0] = m2_run[1] = -INFINITY;
-    l_run[0] = l_run[1] = 0.f;
   }
 
-  // ---------------------------------------------------- warp -> CTA combine
-  // Bring every warp's state to (m, l, O) with O relative to m.
-  __syncthreads();  // all warps done with their stages: reuse them
-  float *obuf = reinterpret_cast<float *>(smem);  // [kNW][8][D]
-  if constexpr (MMA) {
-    l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], 4);
-    l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], 8);
-    l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], 16);
-    l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], 4);
-    l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], 8);
-    l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], 16);
-    float f0 = 1.f, f1 = 1.f;
-    if constexpr (kQuant) {
-      f0 = (m2_run[0] == -INFINITY || !alive) ? 0.f : exp2f(m2_run[0] - m_run[0]);
-      f1 = (m2_run[1] == -INFINITY || !alive) ? 0.f : exp2f(m2_run[1] - m_run[1]);
-    } else if (!alive) {
-      f0 = f1 = 0.f;
-    }
-    float *ow = obuf + warp * 8 * D;
+  // End of the unit's piece in this CTA: write the normalised output of heads
+  // h0 .. h0 + nh - 1 (whole unit) or the unnormalised partial (m, l, O) to
+  // record `pbase` + head of the workspace.
+  __device__ __forceinline__ void finish(const AttnParams &p, bool whole, int b, int h0, int nh,
+                                         int64_t pbase, bool alive, int lane) {
+    const int gq = lane >> 2, cq = lane & 3;
+    if constexpr (MMA) {
 #pragma unroll
-    for (int dt = 0; dt < D / 16; ++dt) {
-      int d0, d1;
-      if constexpr (kQuant) {  // rows gq / gq+8 are dims 16c + 2gq / + 1
-        d0 = dt * 16 + 2 * gq;
-        d1 = d0 + 1;
-      } else {
-        d0 = dt * 16 + gq;
-        d1 = d0 + 8;
+      for (int i = 0; i < 2; ++i) {
+        l_run[i] += __shfl_xor_sync(0xffffffffu, l_run[i], 4);
+        l_run[i] += __shfl_xor_sync(0xffffffffu, l_run[i], 8);
+        l_run[i] += __shfl_xor_sync(0xffffffffu, l_run[i], 16);
       }
-      ow[(2 * cq) * D + d0] = oacc[dt][0] * f0;
-      ow[(2 * cq + 1) * D + d0] = oacc[dt][1] * f1;
-      ow[(2 * cq) * D + d1] = oacc[dt][2] * f0;
-      ow[(2 * cq + 1) * D + d1] = oacc[dt][3] * f1;
-    }
-    if (gq == 0) {
-      comb[warp].m[2 * cq] = m_run[0];
-      comb[warp].m[2 * cq + 1] = m_run[1];
-      comb[warp].l[2 * cq] = l_run[0];
-      comb[warp].l[2 * cq + 1] = l_run[1];
-    }
-  } else {
-    l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], 16);
-    float *ow = obuf + warp * 8 * D;
+      float f[2] = {alive ? 1.f : 0.f, alive ? 1.f : 0.f};
+      if constexpr (kQuant) {
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      float v = oacc_s[e] + __shfl_xor_sync(0xffffffffu, oacc_s[e], 16);
-      if (!alive) v = 0.f;
-      if (hw == 0) ow[jl * E + e] = v;
-    }
-    if (lane == 0) {
-      comb[warp].m[0] = m_run[0];
-      comb[warp].l[0] = l_run[0];
-    }
-  }
-  __syncthreads();
-
-  for (int idx = threadIdx.x; idx < nh * D; idx += kThreads) {
-    const int n = idx / D;
-    const int d = idx - n * D;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kNW; ++w) M = fmaxf(M, comb[w].m[n]);
-    float Ls = 0.f, O = 0.f;
-    if (M != -INFINITY) {
-#pragma unroll
-      for (int w = 0; w < kNW; ++w) {
-        const float f = exp2_rel(comb[w].m[n], M);
-        Ls += f * comb[w].l[n];
-        O += f * obuf[(w * 8 + n) * D + d];
+        for (int i = 0; i < 2; ++i)
+          f[i] = (m2_run[i] == -INFINITY || !alive) ? 0.f : exp2f(m2_run[i] - m_run[i]);
       }
-    }
-    const int h = h0 + n;
-    if (nparts == 1) {
-      const float v = Ls > 0.f ? O / Ls : 0.f;
-      store_out<Q_T>(p.out, (static_cast<int64_t>(b) * p.q_heads + h) * D + d, v);
+      if (whole) {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) f[i] = l_run[i] > 0.f ? f[i] / l_run[i] : 0.f;
+      }
+#pragma unroll
+      for (int dt = 0; dt < D / 16; ++dt) {
+        int d0, d1;
+        if constexpr (kQuant) {  // rows gq / gq+8 are dims 16c + 2gq / + 1
+          d0 = dt * 16 + 2 * gq;
+          d1 = d0 + 1;
+        } else {
+          d0 = dt * 16 + gq;
+          d1 = d0 + 8;
+        }
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int n = 2 * cq + i;
+          if (n < nh) {
+            const float v0 = oacc[dt][i] * f[i], v1 = oacc[dt][i + 2] * f[i];
+            if (whole) {
+              const int64_t o = (static_cast<int64_t>(b) * p.q_heads + h0 + n) * D;
+              store_out<Q_T>(p.out, o + d0, v0);
+              store_out<Q_T>(p.out, o + d1, v1);
+            } else {
+              float *po = p.part_o + (pbase + n) * D;
+              po[d0] = v0;
+              po[d1] = v1;
+            }
+          }
+        }
+      }
+      if (!whole && gq == 0) {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int n = 2 * cq + i;
+          if (n < nh) {
+            p.part_ml[(pbase + n) * 2] = alive ? m_run[i] : -INFINITY;
+            p.part_ml[(pbase + n) * 2 + 1] = l_run[i];
+          }
+        }
+      }
     } else {
-      const int64_t pi = (static_cast<int64_t>(b) * p.q_heads + h) * p.max_parts + part;
-      p.ws_o[pi * D + d] = O;
-      if (d == 0) {
-        p.ws_m[pi] = M;
-        p.ws_l[pi] = Ls;
+      const int hw = lane >> 4, jl = lane & 15;
+      l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], 16);
+      const float f = !alive ? 0.f : whole ? (l_run[0] > 0.f ? 1.f / l_run[0] : 0.f) : 1.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const float v = (oacc_s[e] + __shfl_xor_sync(0xffffffffu, oacc_s[e], 16)) * f;
+        if (hw == 0) {
+          if (whole)
+            store_out<Q_T>(p.out, (static_cast<int64_t>(b) * p.q_heads + h0) * D + jl * E + e, v);
+          else
+            p.part_o[pbase * D + jl * E + e] = v;
+        }
       }
+      if (!whole && lane == 0) {
+        p.part_ml[pbase * 2] = alive ? m_run[0] : -INFINITY;
+        p.part_ml[pbase * 2 + 1] = l_run[0];
+      }
+    }
+  }
+};
+
+// Position of a CTA's walk over the flattened (unit, block) list.
+struct Walk {
+  int b;         // sequence
+  int gc;        // unit within the sequence: kv head * chunks + chunk
+  int j;         // block within the unit
+  int nb;        // blocks of sequence b
+  long long pos; // flattened position of (b, gc, j)
+};
+
+template <int BS>
+__device__ __forceinline__ void walk_advance(Walk &w, int seg, const AttnParams &p) {
+  w.pos += seg;
+  w.j += seg;
+  if (w.j == w.nb) {
+    w.j = 0;
+    if (++w.gc == p.units_per_seq) {
+      w.gc = 0;
+      do {
+        ++w.b;
+        w.nb = w.b < p.num_seqs ? seq_blocks<BS>(p, w.b) : 0;
+      } while (w.b < p.num_seqs && w.nb == 0);
     }
   }
 }
 
+// ============================================================================
+// Partition kernel: persistent, one producer warp + kNC consumer warps.
+// ============================================================================
+template <int D, int BS, int KV_T, int Q_T, bool MMA>
+__global__ void __launch_bounds__(kThreads, 1)
+attn_partition_kernel(const __grid_constant__ CUtensorMap kmap,
+                      const __grid_constant__ CUtensorMap vmap, const AttnParams p) {
+  using T = Tile<D, BS, KV_T>;
+  constexpr unsigned kFull = 0xffffffffu;
+
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[kMaxStages];
+  __shared__ __align__(8) uint64_t empty_bar[kMaxStages];
+  __shared__ int stage_id[kMaxStages];
+  __shared__ long long red[kWarps];
+  __shared__ long long s_loc[2];
+  __shared__ int s_abort;
+  uint8_t *ring = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int c = blockIdx.x;
+  const int B = p.num_seqs;
+  const int UH = p.units_per_seq;
+  const long long G = p.num_ctas;
+  const int rows = p.hg * BS;           // rows of one stage's K (or V) part
+  const int stride = p.stage_bytes;     // bytes between stages (1024-aligned)
+  const int R = p.stages;
+
+  // ---------------------------------------------------------------- prologue
+  // Total positions over all units, then this CTA's even share [s0, s1).
+  long long part = 0;
+  for (int b = threadIdx.x; b < B; b += kThreads) {
+    const int L = p.context_lens[b];
+    if (L < 0 || L > p.limit) {
+      if (c == 0) atomicOr(p.status, kErrContext);
+    } else {
+      part += (L + BS - 1) / BS;
+    }
+  }
+  const long long total = block_sum(part, red) * UH;
+  const long long s0 = cta_start(c, total, G), s1 = cta_start(c + 1, total, G);
+  if (s0 >= s1) return;  // same for every thread of the CTA
+
+  if (threadIdx.x == 0) {
+    s_loc[0] = -1;
+    s_abort = 0;
+    for (int i = 0; i < R; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], kNC);
+    }
+    fence_barrier_init();
+  }
+  if (warp == kNC && lane == 0) {
+    prefetch_tmap(&kmap);
+    prefetch_tmap(&vmap);
+  }
+  __syncthreads();
+  // Sequence holding position s0 (chunked scan over the sequences).
+  long long run = 0;
+  for (int base = 0; base < B; base += kThreads) {
+    const int b = base + threadIdx.x;
+    const int nb = b < B ? seq_blocks<BS>(p, b) : 0;
+    long long tot;
+    const long long excl = run + block_excl_scan(nb, red, &tot);
+    if (nb > 0 && excl * UH <= s0 && s0 < (excl + nb) * UH) {
+      s_loc[0] = b;
+      s_loc[1] = excl;
+    }
+    run += tot;
+    __syncthreads();
+    if (s_loc[0] >= 0) break;
+  }
+  if (s_loc[0] < 0) {  // lengths changed under the kernel: nothing consistent to do
+    if (threadIdx.x == 0) atomicOr(p.status, kErrContext);
+    return;
+  }
+  Walk w0;
+  w0.b = static_cast<int>(s_loc[0]);
+  w0.nb = seq_blocks<BS>(p, w0.b);
+  {
+    const long long off = s0 - s_loc[1] * UH;
+    w0.gc = static_cast<int>(off / w0.nb);
+    w0.j = static_cast<int>(off - static_cast<long long>(w0.gc) * w0.nb);
+  }
+  w0.pos = s0;
+
+  if (warp == kNC) {
+    // ============================================================ producer
+    Walk w = w0;
+    uint32_t k = 0;
+    bool ok = true;
+    while (w.pos < s1 && ok) {
+      if (w.b >= B || w.nb <= 0) break;  // lengths changed under the kernel
+      const int seg = static_cast<int>(min(static_cast<long long>(w.nb - w.j), s1 - w.pos));
+      const int head0 = (w.gc / p.cgroups) * p.hg;  // first kv head of the unit
+      const int32_t *btrow = p.block_tables + static_cast<int64_t>(w.b) * p.max_blocks + w.j;
+      for (int i0 = 0; i0 < seg && ok; i0 += 32) {
+        const int cnt = min(32, seg - i0);
+        int myid = -1;
+        if (lane < cnt) {
+          myid = btrow[i0 + lane];
+          if (myid < 0 || myid >= p.num_blocks) {
+            atomicOr(p.status, kErrBlockId);
+            myid = -1;
+          }
+        }
+        for (int i = 0; i < cnt; ++i) {
+          const int id = __shfl_sync(kFull, myid, i);
+          const int s = k % R;
+          int okv = 1;
+          if (lane == 0 && k >= static_cast<uint32_t>(R))
+            okv = ring_wait(&empty_bar[s], ((k / R) - 1) & 1, &s_abort, p.status);
+          okv = __shfl_sync(kFull, okv, 0);
+          if (!okv) {
+            ok = false;
+            break;
+          }
+          if (lane == 0) {
+            stage_id[s] = id;
+            const int row0 = id >= 0 ? (id * p.kv_heads + head0) * BS : 0;
+            issue_stage<D, BS, KV_T>(ring + s * stride, &full_bar[s], &kmap, &vmap, id, row0,
+                                     rows, p);
+          }
+          __syncwarp();
+          ++k;
+        }
+      }
+      walk_advance<BS>(w, seg, p);
+    }
+    if (!ok && lane == 0) {
+      // aborted: let the loads still in flight land before the CTA can exit
+      for (uint32_t kk = k > static_cast<uint32_t>(R) ? k - R : 0; kk < k; ++kk)
+        mbar_wait(&full_bar[kk % R], (kk / R) & 1, nullptr, 100000000ull);
+    }
+    return;
+  }
+
+  // ============================================================== consumers
+  // Consumer warp `warp` owns slot `warp` of each unit: kv head hi = warp / cpg
+  // of the unit's group, query-head chunk cl = warp % cpg. Every consumer visits
+  // every position (an idle one only releases the stage).
+  Consumer<D, BS, KV_T, Q_T, MMA> cs;
+  Walk w = w0;
+  uint32_t k = 0;
+  bool alive = true;
+  while (w.pos < s1) {
+    if (w.b >= B || w.nb <= 0) {  // same test as the producer: both stop here
+      if (warp == 0 && lane == 0) atomicOr(p.status, kErrContext);
+      break;
+    }
+    const int seg = static_cast<int>(min(static_cast<long long>(w.nb - w.j), s1 - w.pos));
+    const int hgi = w.gc / p.cgroups;
+    const int cgi = w.gc - hgi * p.cgroups;
+    const int cpg = min(p.cpg, p.chunks - cgi * p.cpg);
+    const bool active = warp < p.hg * cpg;
+    const int hi = active ? warp / cpg : 0;
+    const int cl = warp - hi * cpg;
+    const int g = hgi * p.hg + hi;
+    const int chunk = cgi * p.cpg + cl;
+    const int h0 = g * p.group + chunk * kChunkHeads;
+    const int nh = MMA ? min(kChunkHeads, p.group - chunk * kChunkHeads) : 1;
+    const int L = p.context_lens[w.b];
+    if (active) {
+      cs.reset();
+      cs.load_query(p, w.b, h0, nh, lane);
+    }
+    for (uint32_t kk = k; kk < k + seg; ++kk) {
+      const int s = kk % R;
+      if (alive) {
+        int okv = 1;
+        if (lane == 0) okv = ring_wait(&full_bar[s], (kk / R) & 1, &s_abort, p.status);
+        okv = __shfl_sync(kFull, okv, 0);
+        if (!okv) alive = false;
+      }
+      if (alive) {
+        while (!mbar_try_wait(&full_bar[s], (kk / R) & 1)) {
+        }  // already complete: gives every lane the acquire
+        if (active) {
+          const int jb = w.j + static_cast<int>(kk - k);
+          const int id = stage_id[s];
+          const int valid = id >= 0 ? min(BS, L - jb * BS) : 0;
+          cs.block(ring + s * stride, rows, hi, valid, lane);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_bar[s]);
+      }
+    }
+    // ------------------------------------------ end of the unit's piece here
+    const bool whole = (w.j == 0 && seg == w.nb);
+    const int side = (w.pos == s0) ? 0 : 1;
+    if (active) {
+      const int64_t pbase = ((static_cast<int64_t>(c) * 2 + side) * kNC + warp) * kChunkHeads;
+      cs.finish(p, whole, w.b, h0, nh, pbase, alive, lane);
+    }
+    if (warp == 0 && lane == 0 && w.j == 0) {  // this CTA holds the unit's first block
+      const int nu = cta_of(w.pos + w.nb - 1, total, G) - c + 1;
+      p.meta[static_cast<int64_t>(w.b) * UH + w.gc] = make_int4(c, nu, side, 0);
+    }
+    k += seg;
+    walk_advance<BS>(w, seg, p);
+  }
+}
 
 // ============================================================================
-// Merge kernel: one warp per (sequence, query head) with > 1 partition.
-// out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p, M = max_p m_p (base 2).
+// Merge kernel: one warp per (sequence, query head). Writes zeros for empty or
+// invalid sequences; combines the partials of units split across CTAs:
+// out = sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i, M = max_i m_i.
 // ============================================================================
 constexpr int kMergeWarps = 8;
 
 template <int D, int OUT_T>
-__global__ void __launch_bounds__(kMergeWarps * 32)
-attn_merge_kernel(const float *__restrict__ ws_o, const float *__restrict__ ws_m,
-                  const float *__restrict__ ws_l, const int32_t *__restrict__ context_lens,
-                  void *out, int num_seqs, int q_heads, int part_tokens, int max_parts,
-                  int limit) {
+__global__ void __launch_bounds__(kMergeWarps * 32) attn_merge_kernel(const AttnParams p) {
   const int w = blockIdx.x * kMergeWarps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (w >= num_seqs * q_heads) return;
-  const int b = w / q_heads;
-  const int L = context_lens[b];
-  if (L < 0 || L > limit) return;  // written as zeros by the partition kernel
-  const int np = (L + part_tokens - 1) / part_tokens;
-  if (np <= 1) return;  // written directly by the partition kernel
-  const int64_t base = static_cast<int64_t>(w) * max_parts;
-  float M = -INFINITY;
-  for (int pp = lane; pp < np; pp += 32) M = fmaxf(M, ws_m[base + pp]);
-  M = warp_max_xor(M, 1);
+  if (w >= p.num_seqs * p.q_heads) return;
   constexpr int E = D / 32;
+  const int b = w / p.q_heads;
+  const int h = w - b * p.q_heads;
+  const int L = p.context_lens[b];
+  const int64_t orow = static_cast<int64_t>(w) * D + lane * E;
+  if (!(L > 0 && L <= p.limit)) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) store_out<OUT_T>(p.out, orow + e, 0.f);
+    return;
+  }
+  // (unit, slot, head) of query head h, as the partition kernel assigned them
+  const int g = h / p.group;
+  const int r = h - g * p.group;
+  const int chunk = r / kChunkHeads;
+  const int n = r - chunk * kChunkHeads;
+  const int hgi = g / p.hg, hi = g - hgi * p.hg;
+  const int cgi = chunk / p.cpg, cl = chunk - cgi * p.cpg;
+  const int cpg = min(p.cpg, p.chunks - cgi * p.cpg);
+  const int slot = hi * cpg + cl;
+  const int4 mt = p.meta[static_cast<int64_t>(b) * p.units_per_seq + hgi * p.cgroups + cgi];
+  const int nu = mt.y;
+  if (nu <= 1) return;  // finished by the partition kernel
+  if (mt.x < 0 || mt.x >= p.num_ctas || nu > p.num_ctas - mt.x || (mt.z & ~1)) {
+    if (lane == 0) atomicOr(p.status, kErrTimeout);  // bookkeeping not written: phase 1 aborted
+    return;
+  }
+  auto rec = [&](int i) -> int64_t {
+    return ((static_cast<int64_t>(mt.x + i) * 2 + (i == 0 ? mt.z : 0)) * kNC + slot) * kChunkHeads + n;
+  };
+  float M = -INFINITY;
+  for (int i = lane; i < nu; i += 32) M = fmaxf(M, p.part_ml[rec(i) * 2]);
+  M = warp_max_xor(M, 1);
   float acc[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) acc[e] = 0.f;
   float Ls = 0.f;
   if (M != -INFINITY) {
-    for (int p0 = 0; p0 < np; p0 += 32) {
-      const int pp = p0 + lane;
-      const float wgt = pp < np ? exp2_rel(ws_m[base + pp], M) : 0.f;
-      Ls += pp < np ? wgt * ws_l[base + pp] : 0.f;
-      const int cnt = min(32, np - p0);
-      for (int k = 0; k < cnt; ++k) {
-        const float wk = __shfl_sync(0xffffffffu, wgt, k);
-        const float *o = ws_o + (base + p0 + k) * D + lane * E;
+    for (int i0 = 0; i0 < nu; i0 += 32) {
+      const int i = i0 + lane;
+      const float wgt = i < nu ? exp2_rel(p.part_ml[rec(i) * 2], M) : 0.f;
+      Ls += i < nu ? wgt * p.part_ml[rec(i) * 2 + 1] : 0.f;
+      const int cnt = min(32, nu - i0);
+      for (int kk = 0; kk < cnt; ++kk) {
+        const float wk = __shfl_sync(0xffffffffu, wgt, kk);
+        const float *o = p.part_o + rec(i0 + kk) * D + lane * E;
         if constexpr (E == 4) {
           const float4 v = *reinterpret_cast<const float4 *>(o);
           acc[0] = fmaf(wk, v.x, acc[0]);
@@ -768,24 +1025,23 @@ attn_merge_kernel(const float *__restrict__ ws_o, const float *__restrict__ ws_m
     for (int o = 16; o > 0; o >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
   }
 #pragma unroll
-  for (int e = 0; e < E; ++e)
-    store_out<OUT_T>(out, static_cast<int64_t>(w) * D + lane * E + e, Ls > 0.f ? acc[e] / Ls : 0.f);
+  for (int e = 0; e < E; ++e) store_out<OUT_T>(p.out, orow + e, Ls > 0.f ? acc[e] / Ls : 0.f);
 }
 
 // ============================================================================
 // Host side
 // ============================================================================
-using PartFn = cudaError_t (*)(const CUtensorMap &, const CUtensorMap &, const AttnParams &, dim3,
+using PartFn = cudaError_t (*)(const CUtensorMap &, const CUtensorMap &, const AttnParams &,
                                cudaStream_t);
 
 template <int D, int BS, int KV_T, int Q_T, bool MMA>
 cudaError_t launch_part(const CUtensorMap &km, const CUtensorMap &vm, const AttnParams &p,
-                        dim3 grid, cudaStream_t st) {
-  constexpr int smem = smem_bytes<D, BS, KV_T>();
+                        cudaStream_t st) {
+  const int smem = p.stages * p.stage_bytes + 1024;
   auto kern = attn_partition_kernel<D, BS, KV_T, Q_T, MMA>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, smem, st>>>(km, vm, p);
+  kern<<<p.num_ctas, kThreads, smem, st>>>(km, vm, p);
   return cudaGetLastError();
 }
 
@@ -813,90 +1069,149 @@ PartFn pick_partition(int D, int BS, int kv, int q, bool mma) {
   return BS == 16 ? pick_dtype<64, 16>(kv, q, mma) : pick_dtype<64, 32>(kv, q, mma);
 }
 
-cudaError_t launch_merge(int D, int out_t, const float *o, const float *m, const float *l,
-                         const int32_t *lens, void *out, int B, int Hq, int S, int Pmax, int limit,
-                         cudaStream_t st) {
-  const int64_t warps = static_cast<int64_t>(B) * Hq;
+cudaError_t launch_merge(int D, int out_t, const AttnParams &p, cudaStream_t st) {
+  const int64_t warps = static_cast<int64_t>(p.num_seqs) * p.q_heads;
   const unsigned grid = static_cast<unsigned>((warps + kMergeWarps - 1) / kMergeWarps);
   const int th = kMergeWarps * 32;
   if (D == 128) {
-    if (out_t == KV_BF16)
-      attn_merge_kernel<128, KV_BF16><<<grid, th, 0, st>>>(o, m, l, lens, out, B, Hq, S, Pmax, limit);
-    else
-      attn_merge_kernel<128, KV_FP16><<<grid, th, 0, st>>>(o, m, l, lens, out, B, Hq, S, Pmax, limit);
+    if (out_t == KV_BF16) attn_merge_kernel<128, KV_BF16><<<grid, th, 0, st>>>(p);
+    else attn_merge_kernel<128, KV_FP16><<<grid, th, 0, st>>>(p);
   } else {
-    if (out_t == KV_BF16)
-      attn_merge_kernel<64, KV_BF16><<<grid, th, 0, st>>>(o, m, l, lens, out, B, Hq, S, Pmax, limit);
-    else
-      attn_merge_kernel<64, KV_FP16><<<grid, th, 0, st>>>(o, m, l, lens, out, B, Hq, S, Pmax, limit);
+    if (out_t == KV_BF16) attn_merge_kernel<64, KV_BF16><<<grid, th, 0, st>>>(p);
+    else attn_merge_kernel<64, KV_FP16><<<grid, th, 0, st>>>(p);
   }
   return cudaGetLastError();
 }
 
-// Workspace: o [B][Hq][Pmax][D], m and l [B][Hq][Pmax], fp32, 256-aligned parts.
-struct WsLayout {
-  uint64_t o_off, m_off, l_off, total;
+// How a call's heads are grouped into units (see the kernel's notes).
+struct UnitGeom {
+  int chunks, cpg, cgroups, hg, units_per_seq, rows, stage_bytes, stages;
 };
 
-WsLayout ws_layout(int B, int Hq, int Pmax, int D) {
+UnitGeom unit_geom(const kv_pool *pool, int num_q_heads) {
+  const kv_pool_desc &d = pool->d;
+  UnitGeom u{};
+  const int group = num_q_heads / d.num_kv_heads;
+  u.chunks = group >= 2 ? (group + kChunkHeads - 1) / kChunkHeads : 1;
+  u.cpg = std::min(u.chunks, kNC);
+  u.cgroups = (u.chunks + u.cpg - 1) / u.cpg;
+  const int elt = elem_bytes(d.cache_dtype);
+  const int row_bytes = d.head_dim * elt;
+  const bool quant = is_quant(d.cache_dtype);
+  auto load = [&](int hg) { return 2 * hg * d.block_size * (row_bytes + (quant ? 4 : 0)); };
+  // the largest group of kv heads (a divisor of Hkv) with one slot per consumer
+  // warp, a stage of at most kMaxStageBytes and a TMA box of at most 256 rows
+  u.hg = 1;
+  for (int hg = 1; hg <= d.num_kv_heads; ++hg) {
+    if (d.num_kv_heads % hg) continue;
+    if (hg * u.cpg > kNC || load(hg) > kMaxStageBytes || hg * d.block_size > 256) break;
+    u.hg = hg;
+  }
+  u.units_per_seq = (d.num_kv_heads / u.hg) * u.cgroups;
+  u.rows = u.hg * d.block_size;
+  u.stage_bytes = static_cast<int>(round_up(load(u.hg), 1024));
+  u.stages = std::min(kMaxStages, kRingBytes / u.stage_bytes);
+  return u;
+}
+
+// Workspace: unit metadata, then per-CTA partials (two sides x kNC slots x 8 heads).
+struct WsLayout {
+  uint64_t meta_off, ml_off, o_off, total;
+};
+
+WsLayout ws_layout(int B, int units_per_seq, int G, int D) {
   WsLayout w{};
-  if (Pmax <= 1) return w;
-  const uint64_t n = static_cast<uint64_t>(B) * Hq * Pmax;
-  w.o_off = 0;
-  w.m_off = round_up(n * D * sizeof(float), 256);
-  w.l_off = w.m_off + round_up(n * sizeof(float), 256);
-  w.total = w.l_off + round_up(n * sizeof(float), 256);
+  const uint64_t recs = static_cast<uint64_t>(G) * 2 * kNC * kChunkHeads;
+  w.meta_off = 0;
+  w.ml_off = round_up(static_cast<uint64_t>(B) * units_per_seq * 16, 256);
+  w.o_off = w.ml_off + round_up(recs * 2 * 4, 256);
+  w.total = w.o_off + round_up(recs * D * 4, 256);
   return w;
 }
 
-int heads_per_cta_chunks(int group) { return group >= 2 ? (group + 7) / 8 : 1; }
-
-int default_partition(const kv_pool *pool, int B, int Hq, int max_ctx) {
-  const int bs = pool->d.block_size;
-  const int group = Hq / pool->d.num_kv_heads;
-  const int64_t units =
-      static_cast<int64_t>(B) * pool->d.num_kv_heads * heads_per_cta_chunks(group);
-  // Enough CTAs to fill 148 SMs, two resident each, four times over; never
-  // below four blocks per partition.
-  const int64_t want = 4LL * 148 * 2;
-  int S = 512;
-  while (S > 4 * bs && units * ((max_ctx + S - 1) / S) < want) S /= 2;
-  return S;
+kv_status sm_count(int *n) {
+  int dev = 0;
+  kv_status s = cuda_check(cudaGetDevice(&dev), "cudaGetDevice");
+  if (s != KV_OK) return s;
+  return cuda_check(cudaDeviceGetAttribute(n, cudaDevAttrMultiProcessorCount, dev),
+                    "multiprocessor count");
 }
 
-// Shared argument checks of the attention entry points. Fills S and Pmax.
+// Shared checks; resolves num_ctas (0 = one per SM).
 kv_status check_attn(const kv_pool *pool, int num_seqs, int num_q_heads, int max_context,
-                     int partition_tokens, int *S, int *Pmax) {
+                     int num_ctas, int *G) {
   if (!pool) return fail(KV_ERR_INVALID, "null pool");
-  if (num_seqs < 0 || num_seqs > 65535) return fail(KV_ERR_INVALID, "num_seqs must be in [0, 65535]");
+  if (num_seqs < 0) return fail(KV_ERR_INVALID, "negative num_seqs");
   const int hkv = pool->d.num_kv_heads;
   if (num_q_heads <= 0 || num_q_heads % hkv != 0)
     return fail(KV_ERR_INVALID, "num_q_heads (%d) must be a positive multiple of num_kv_heads (%d)",
                 num_q_heads, hkv);
-  if (static_cast<int64_t>(hkv) * heads_per_cta_chunks(num_q_heads / hkv) > 65535)
-    return fail(KV_ERR_INVALID, "too many heads");
+  if (static_cast<int64_t>(num_seqs) * num_q_heads > 0x7fffffffLL / 32)
+    return fail(KV_ERR_INVALID, "num_seqs * num_q_heads too large");
   if (max_context < 0) return fail(KV_ERR_INVALID, "negative max_context");
-  const int bs = pool->d.block_size;
-  int s = partition_tokens;
-  if (s == 0) s = default_partition(pool, num_seqs, num_q_heads, max_context);
-  if (s < bs || s % bs != 0 || s / bs > kMaxPartBlocks)
-    return fail(KV_ERR_INVALID, "partition_tokens %d must be a multiple of block_size %d, at most %d",
-                partition_tokens, bs, kMaxPartBlocks * bs);
-  *S = s;
-  *Pmax = max_context > 0 ? (max_context + s - 1) / s : 1;
-  if (*Pmax > 0x7fffffff / 2) return fail(KV_ERR_INVALID, "max_context too large");
+  if (num_ctas < 0 || num_ctas > 65535) return fail(KV_ERR_INVALID, "num_ctas must be in [0, 65535]");
+  if (num_ctas == 0) {
+    kv_status s = sm_count(G);
+    if (s != KV_OK) return s;
+  } else {
+    *G = num_ctas;
+  }
+  return KV_OK;
+}
+
+kv_status fill_params(kv_pool *pool, int layer, const void *q, int num_seqs, int num_q_heads,
+                      const int32_t *block_tables, int max_blocks_per_seq,
+                      const int32_t *context_lens, int max_context, float scale, void *out,
+                      int G, void *workspace, uint64_t workspace_bytes, AttnParams *pp) {
+  const int D = pool->d.head_dim;
+  const int group = num_q_heads / pool->d.num_kv_heads;
+  const UnitGeom u = unit_geom(pool, num_q_heads);
+  const WsLayout wl = ws_layout(num_seqs, u.units_per_seq, G, D);
+  if (!workspace || workspace_bytes < wl.total)
+    return fail(KV_ERR_INVALID, "workspace of %llu bytes needed, %llu given",
+                static_cast<unsigned long long>(wl.total),
+                static_cast<unsigned long long>(workspace_bytes));
+  if (reinterpret_cast<uintptr_t>(workspace) & 255)
+    return fail(KV_ERR_INVALID, "workspace must be 256-byte aligned");
+  AttnParams &p = *pp;
+  p = AttnParams{};
+  p.q = q;
+  p.out = out;
+  p.block_tables = block_tables;
+  p.context_lens = context_lens;
+  p.k_scale = layer >= 0 ? layer_ks(pool, layer) : nullptr;
+  p.v_scale = layer >= 0 ? layer_vs(pool, layer) : nullptr;
+  char *ws = static_cast<char *>(workspace);
+  p.meta = reinterpret_cast<int4 *>(ws + wl.meta_off);
+  p.part_ml = reinterpret_cast<float *>(ws + wl.ml_off);
+  p.part_o = reinterpret_cast<float *>(ws + wl.o_off);
+  p.status = status_word(pool);
+  p.scale_log2 = scale * kLog2e;
+  p.num_seqs = num_seqs;
+  p.q_heads = num_q_heads;
+  p.kv_heads = pool->d.num_kv_heads;
+  p.group = group;
+  p.chunks = u.chunks;
+  p.hg = u.hg;
+  p.cpg = u.cpg;
+  p.cgroups = u.cgroups;
+  p.units_per_seq = u.units_per_seq;
+  p.stage_bytes = u.stage_bytes;
+  p.stages = u.stages;
+  p.max_blocks = max_blocks_per_seq;
+  p.num_blocks = pool->d.num_blocks;
+  const int64_t tbl_cap = static_cast<int64_t>(max_blocks_per_seq) * pool->d.block_size;
+  p.limit = static_cast<int>(std::min<int64_t>(max_context, tbl_cap));
+  p.num_ctas = G;
   return KV_OK;
 }
 
 kv_status run_partition(kv_pool *pool, int32_t layer, const void *q, int32_t q_dtype,
                         int32_t num_seqs, int32_t num_q_heads, const int32_t *block_tables,
                         int32_t max_blocks_per_seq, const int32_t *context_lens,
-                        int32_t max_context, float scale, void *out, int32_t partition_tokens,
-                        void *workspace, uint64_t workspace_bytes, cudaStream_t st,
-                        int *S_out, int *Pmax_out) {
-  int S = 0, Pmax = 0;
-  kv_status s = check_attn(pool, num_seqs, num_q_heads, max_context, partition_tokens, &S, &Pmax);
-  if (s != KV_OK) return s;
+                        int32_t max_context, float scale, void *out, int32_t num_ctas,
+                        void *workspace, uint64_t workspace_bytes, cudaStream_t st) {
+  if (!pool) return fail(KV_ERR_INVALID, "null pool");
   if (layer < 0 || layer >= pool->d.num_layers) return fail(KV_ERR_INVALID, "layer %d out of range", layer);
   const int cd = pool->d.cache_dtype;
   if (q_dtype != KV_BF16 && q_dtype != KV_FP16)
@@ -906,83 +1221,46 @@ kv_status run_partition(kv_pool *pool, int32_t layer, const void *q, int32_t q_d
   if (!(scale == scale) || scale == INFINITY || scale == -INFINITY)
     return fail(KV_ERR_INVALID, "scale must be finite");
   if (max_blocks_per_seq <= 0) return fail(KV_ERR_INVALID, "max_blocks_per_seq must be > 0");
-  *S_out = S;
-  *Pmax_out = Pmax;
-  if (num_seqs == 0) return KV_OK;
-  if (!q || !out || !block_tables || !context_lens) return fail(KV_ERR_INVALID, "null pointer");
+  if (num_seqs < 0) return fail(KV_ERR_INVALID, "negative num_seqs");
+  if (num_seqs > 0 && (!q || !out || !block_tables || !context_lens))
+    return fail(KV_ERR_INVALID, "null pointer");
   if ((reinterpret_cast<uintptr_t>(q) & 15) || (reinterpret_cast<uintptr_t>(out) & 15) ||
       (reinterpret_cast<uintptr_t>(block_tables) & 3) || (reinterpret_cast<uintptr_t>(context_lens) & 3))
     return fail(KV_ERR_INVALID, "q and out must be 16-byte aligned, tables and lengths 4-byte");
-  const int D = pool->d.head_dim;
-  const WsLayout wl = ws_layout(num_seqs, num_q_heads, Pmax, D);
-  if (wl.total > 0) {
-    if (!workspace || workspace_bytes < wl.total)
-      return fail(KV_ERR_INVALID, "workspace of %llu bytes needed, %llu given",
-                  static_cast<unsigned long long>(wl.total), static_cast<unsigned long long>(workspace_bytes));
-    if (reinterpret_cast<uintptr_t>(workspace) & 255)
-      return fail(KV_ERR_INVALID, "workspace must be 256-byte aligned");
-  }
+  int G = 0;
+  kv_status s = check_attn(pool, num_seqs, num_q_heads, max_context, num_ctas, &G);
+  if (s != KV_OK) return s;
+  AttnParams p;
+  s = fill_params(pool, layer, q, num_seqs, num_q_heads, block_tables, max_blocks_per_seq,
+                  context_lens, max_context, scale, out, G, workspace, workspace_bytes, &p);
+  if (s != KV_OK) return s;
+  if (num_seqs == 0) return KV_OK;
   kv_status code;
-  const LayerMaps *maps = layer_maps(pool, layer, &code);
+  const LayerMaps *maps = layer_maps(pool, layer, p.hg * pool->d.block_size, &code);
   if (!maps) return code;
-  const int group = num_q_heads / pool->d.num_kv_heads;
-  const bool mma = group >= 2;
-  AttnParams p{};
-  p.q = q;
-  p.out = out;
-  p.block_tables = block_tables;
-  p.context_lens = context_lens;
-  p.k_scale = layer_ks(pool, layer);
-  p.v_scale = layer_vs(pool, layer);
-  char *ws = static_cast<char *>(workspace);
-  p.ws_o = wl.total ? reinterpret_cast<float *>(ws + wl.o_off) : nullptr;
-  p.ws_m = wl.total ? reinterpret_cast<float *>(ws + wl.m_off) : nullptr;
-  p.ws_l = wl.total ? reinterpret_cast<float *>(ws + wl.l_off) : nullptr;
-  p.status = status_word(pool);
-  p.scale_log2 = scale * kLog2e;
-  p.num_seqs = num_seqs;
-  p.q_heads = num_q_heads;
-  p.kv_heads = pool->d.num_kv_heads;
-  p.group = group;
-  p.chunks = heads_per_cta_chunks(group);
-  p.max_blocks = max_blocks_per_seq;
-  p.num_blocks = pool->d.num_blocks;
-  const int64_t tbl_cap = static_cast<int64_t>(max_blocks_per_seq) * pool->d.block_size;
-  p.limit = static_cast<int>(std::min<int64_t>(max_context, tbl_cap));
-  p.part_tokens = S;
-  p.max_parts = Pmax;
-  PartFn fn = pick_partition(D, pool->d.block_size, cd, q_dtype, mma);
-  dim3 grid(Pmax, p.kv_heads * p.chunks, num_seqs);
-  return cuda_check(fn(maps->k, maps->v, p, grid, st), "paged attention launch");
+  PartFn fn = pick_partition(pool->d.head_dim, pool->d.block_size, cd, q_dtype, p.group >= 2);
+  return cuda_check(fn(maps->k, maps->v, p, st), "paged attention launch");
 }
 
-kv_status run_merge(const kv_pool *pool, int32_t num_seqs, int32_t num_q_heads,
-                    const int32_t *context_lens, int32_t max_blocks_per_seq,
-                    int32_t max_context, int32_t partition_tokens,
-                    int32_t out_dtype, void *out, const void *workspace, uint64_t workspace_bytes,
-                    cudaStream_t st) {
-  int S = 0, Pmax = 0;
-  kv_status s = check_attn(pool, num_seqs, num_q_heads, max_context, partition_tokens, &S, &Pmax);
-  if (s != KV_OK) return s;
+kv_status run_merge(kv_pool *pool, int32_t num_seqs, int32_t num_q_heads,
+                    const int32_t *context_lens, int32_t max_blocks_per_seq, int32_t max_context,
+                    int32_t num_ctas, int32_t out_dtype, void *out, void *workspace,
+                    uint64_t workspace_bytes, cudaStream_t st) {
+  if (!pool) return fail(KV_ERR_INVALID, "null pool");
   if (out_dtype != KV_BF16 && out_dtype != KV_FP16)
     return fail(KV_ERR_UNSUPPORTED, "out_dtype must be KV_BF16 or KV_FP16");
   if (max_blocks_per_seq <= 0) return fail(KV_ERR_INVALID, "max_blocks_per_seq must be > 0");
-  if (num_seqs == 0 || Pmax <= 1) return KV_OK;
+  int G = 0;
+  kv_status s = check_attn(pool, num_seqs, num_q_heads, max_context, num_ctas, &G);
+  if (s != KV_OK) return s;
+  if (num_seqs == 0) return KV_OK;
   if (!out || !context_lens) return fail(KV_ERR_INVALID, "null pointer");
-  const int D = pool->d.head_dim;
-  const WsLayout wl = ws_layout(num_seqs, num_q_heads, Pmax, D);
-  if (!workspace || workspace_bytes < wl.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
-    return fail(KV_ERR_INVALID, "workspace missing, too small or misaligned");
-  const char *ws = static_cast<const char *>(workspace);
-  // same validity limit on lengths as phase 1 (invalid lengths were zeroed there)
-  const int64_t tbl_cap = static_cast<int64_t>(max_blocks_per_seq) * pool->d.block_size;
-  const int limit = static_cast<int>(std::min<int64_t>(max_context, tbl_cap));
-  return cuda_check(
-      launch_merge(D, out_dtype, reinterpret_cast<const float *>(ws + wl.o_off),
-                   reinterpret_cast<const float *>(ws + wl.m_off),
-                   reinterpret_cast<const float *>(ws + wl.l_off), context_lens, out, num_seqs,
-                   num_q_heads, S, Pmax, limit, st),
-      "merge launch");
+  if ((reinterpret_cast<uintptr_t>(out) & 15)) return fail(KV_ERR_INVALID, "out must be 16-byte aligned");
+  AttnParams p;
+  s = fill_params(pool, -1, nullptr, num_seqs, num_q_heads, nullptr, max_blocks_per_seq,
+                  context_lens, max_context, 1.f, out, G, workspace, workspace_bytes, &p);
+  if (s != KV_OK) return s;
+  return cuda_check(launch_merge(pool->d.head_dim, out_dtype, p, st), "merge launch");
 }
 
 }  // namespace
@@ -993,65 +1271,58 @@ using namespace pagedkv;
 extern "C" {
 
 kv_status paged_attn_workspace_bytes(const kv_pool *pool, int32_t num_seqs, int32_t num_q_heads,
-                                     int32_t max_context, int32_t partition_tokens,
-                                     uint64_t *bytes) {
+                                     int32_t num_ctas, uint64_t *bytes) {
   if (!bytes) return fail(KV_ERR_INVALID, "null bytes");
-  int S = 0, Pmax = 0;
-  kv_status s = check_attn(pool, num_seqs, num_q_heads, max_context, partition_tokens, &S, &Pmax);
+  int G = 0;
+  kv_status s = check_attn(pool, num_seqs, num_q_heads, 0, num_ctas, &G);
   if (s != KV_OK) return s;
-  *bytes = ws_layout(num_seqs, num_q_heads, Pmax, pool->d.head_dim).total;
+  const UnitGeom u = unit_geom(pool, num_q_heads);
+  *bytes = ws_layout(num_seqs, u.units_per_seq, G, pool->d.head_dim).total;
   return ok();
 }
 
-kv_status paged_attn_default_partition(const kv_pool *pool, int32_t num_seqs, int32_t num_q_heads,
-                                       int32_t max_context, int32_t *partition_tokens) {
-  if (!partition_tokens) return fail(KV_ERR_INVALID, "null partition_tokens");
-  int S = 0, Pmax = 0;
-  kv_status s = check_attn(pool, num_seqs, num_q_heads, max_context, 0, &S, &Pmax);
+kv_status paged_attn_default_ctas(const kv_pool *pool, int32_t *num_ctas) {
+  if (!pool || !num_ctas) return fail(KV_ERR_INVALID, "null argument");
+  int n = 0;
+  kv_status s = sm_count(&n);
   if (s != KV_OK) return s;
-  *partition_tokens = S;
+  *num_ctas = n;
   return ok();
 }
 
 kv_status paged_attn_partition(kv_pool *pool, int32_t layer, const void *q, int32_t q_dtype,
                                int32_t num_seqs, int32_t num_q_heads, const int32_t *block_tables,
                                int32_t max_blocks_per_seq, const int32_t *context_lens,
-                               int32_t max_context, float scale, void *out,
-                               int32_t partition_tokens, void *workspace, uint64_t workspace_bytes,
-                               kv_stream_t stream) {
-  int S, Pmax;
+                               int32_t max_context, float scale, void *out, int32_t num_ctas,
+                               void *workspace, uint64_t workspace_bytes, kv_stream_t stream) {
   kv_status s = run_partition(pool, layer, q, q_dtype, num_seqs, num_q_heads, block_tables,
-                              max_blocks_per_seq, context_lens, max_context, scale, out,
-                              partition_tokens, workspace, workspace_bytes,
-                              (cudaStream_t)stream, &S, &Pmax);
+                              max_blocks_per_seq, context_lens, max_context, scale, out, num_ctas,
+                              workspace, workspace_bytes, (cudaStream_t)stream);
   return s == KV_OK ? ok() : s;
 }
 
-kv_status paged_attn_merge(const kv_pool *pool, int32_t num_seqs, int32_t num_q_heads,
+kv_status paged_attn_merge(kv_pool *pool, int32_t num_seqs, int32_t num_q_heads,
                            const int32_t *context_lens, int32_t max_blocks_per_seq,
-                           int32_t max_context, int32_t partition_tokens, int32_t out_dtype,
-                           void *out, const void *workspace, uint64_t workspace_bytes,
-                           kv_stream_t stream) {
+                           int32_t max_context, int32_t num_ctas, int32_t out_dtype, void *out,
+                           void *workspace, uint64_t workspace_bytes, kv_stream_t stream) {
   kv_status s = run_merge(pool, num_seqs, num_q_heads, context_lens, max_blocks_per_seq,
-                          max_context, partition_tokens, out_dtype, out, workspace,
-                          workspace_bytes, (cudaStream_t)stream);
+                          max_context, num_ctas, out_dtype, out, workspace, workspace_bytes,
+                          (cudaStream_t)stream);
   return s == KV_OK ? ok() : s;
 }
 
 kv_status paged_attn_decode(kv_pool *pool, int32_t layer, const void *q, int32_t q_dtype,
                             int32_t num_seqs, int32_t num_q_heads, const int32_t *block_tables,
                             int32_t max_blocks_per_seq, const int32_t *context_lens,
-                            int32_t max_context, float scale, void *out, int32_t partition_tokens,
+                            int32_t max_context, float scale, void *out, int32_t num_ctas,
                             void *workspace, uint64_t workspace_bytes, kv_stream_t stream) {
-  int S, Pmax;
   kv_status s = run_partition(pool, layer, q, q_dtype, num_seqs, num_q_heads, block_tables,
-                              max_blocks_per_seq, context_lens, max_context, scale, out,
-                              partition_tokens, workspace, workspace_bytes,
-                              (cudaStream_t)stream, &S, &Pmax);
+                              max_blocks_per_seq, context_lens, max_context, scale, out, num_ctas,
+                              workspace, workspace_bytes, (cudaStream_t)stream);
   if (s != KV_OK) return s;
-  if (num_seqs > 0 && Pmax > 1) {
-    s = run_merge(pool, num_seqs, num_q_heads, context_lens, max_blocks_per_seq, max_context, S,
-                  q_dtype, out, workspace, workspace_bytes, (cudaStream_t)stream);
+  if (num_seqs > 0) {
+    s = run_merge(pool, num_seqs, num_q_heads, context_lens, max_blocks_per_seq, max_context,
+                  num_ctas, q_dtype, out, workspace, workspace_bytes, (cudaStream_t)stream);
     if (s != KV_OK) return s;
   }
   return ok();

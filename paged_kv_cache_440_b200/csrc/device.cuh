@@ -169,6 +169,23 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   }
 }
 
+// Split two floats into 16-bit pairs hi + lo with hi = round(x) and
+// lo = round(x - hi): hi + lo carries x to about 2^-17 (bf16) or 2^-22 (fp16)
+// relative, so an MMA on both parts loses almost nothing to operand rounding.
+template <bool BF16>
+__device__ __forceinline__ void split2(float a, float b, uint32_t &hi, uint32_t &lo) {
+  hi = pack2<BF16>(a, b);
+  float ha, hb;
+  if constexpr (BF16) {
+    ha = __uint_as_float(hi << 16);
+    hb = __uint_as_float(hi & 0xFFFF0000u);
+  } else {
+    ha = __half2float(__ushort_as_half(static_cast<unsigned short>(hi & 0xFFFFu)));
+    hb = __half2float(__ushort_as_half(static_cast<unsigned short>(hi >> 16)));
+  }
+  lo = pack2<BF16>(a - ha, b - hb);
+}
+
 // -------------------------------------------------- 1-byte codes -> fp16 pairs
 //
 // An E5M2 byte is the high byte of the fp16 with the same value (same sign,

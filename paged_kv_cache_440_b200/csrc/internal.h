@@ -38,7 +38,7 @@ struct Layout {
 struct LayerMaps {
   CUtensorMap k;
   CUtensorMap v;
-  bool ready = false;
+  int box_rows = 0;  // rows per box the maps were encoded for (0 = none yet)
 };
 
 }  // namespace pagedkv
@@ -86,7 +86,8 @@ inline int32_t *status_word(const kv_pool *p) {
   return (int32_t *)(p->base + p->lay.status_off);
 }
 
-// Tensor maps for the layer's K and V regions; nullptr + message on failure.
-const LayerMaps *layer_maps(kv_pool *p, int layer, kv_status *code);
+// Tensor maps for the layer's K and V regions with boxes of box_rows rows;
+// nullptr + message on failure.
+const LayerMaps *layer_maps(kv_pool *p, int layer, int box_rows, kv_status *code);
 
 }  // namespace pagedkv

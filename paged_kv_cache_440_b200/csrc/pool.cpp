@@ -86,7 +86,8 @@ bool compute_layout(const kv_pool_desc &d, Layout *out, std::string *why,
 // --------------------------------------------------------------------------
 // Tensor maps: one 2-D map per K / V region, rows = (block, head, token),
 // columns = head_dim elements. The box is one 128-byte (or 64-byte) column
-// slab of a whole (block, head) tile: block_size rows. Tiles land in shared
+// slab of box_rows consecutive rows: the block_size rows of each of a group of
+// heads of one block, which are contiguous in the pool. Boxes land in shared
 // memory with the hardware swizzle so that the 8-row fragment loads the
 // attention kernel issues are bank-conflict free.
 // --------------------------------------------------------------------------
@@ -112,7 +113,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn(std::string *why) {
   return fn;
 }
 
-static bool encode_region(const kv_pool *p, void *base, CUtensorMap *map,
+static bool encode_region(const kv_pool *p, void *base, int box_rows, CUtensorMap *map,
                           std::string *why) {
   auto fn = encode_fn(why);
   if (!fn) return false;
@@ -129,7 +130,7 @@ static bool encode_region(const kv_pool *p, void *base, CUtensorMap *map,
   cuuint64_t gdim[2] = {(cuuint64_t)d.head_dim,
                         (cuuint64_t)d.num_blocks * d.num_kv_heads * d.block_size};
   cuuint64_t gstride[1] = {(cuuint64_t)row_bytes};
-  cuuint32_t box[2] = {(cuuint32_t)(slab_bytes / elt), (cuuint32_t)d.block_size};
+  cuuint32_t box[2] = {(cuuint32_t)(slab_bytes / elt), (cuuint32_t)box_rows};
   cuuint32_t estride[2] = {1, 1};
   CUtensorMapSwizzle swz =
       slab_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
@@ -145,17 +146,18 @@ static bool encode_region(const kv_pool *p, void *base, CUtensorMap *map,
   return true;
 }
 
-const LayerMaps *layer_maps(kv_pool *p, int layer, kv_status *code) {
+const LayerMaps *layer_maps(kv_pool *p, int layer, int box_rows, kv_status *code) {
   std::lock_guard<std::mutex> g(p->map_mu);
   LayerMaps &m = p->maps[layer];
-  if (!m.ready) {
+  if (m.box_rows != box_rows) {
     std::string why;
-    if (!encode_region(p, layer_k(p, layer), &m.k, &why) ||
-        !encode_region(p, layer_v(p, layer), &m.v, &why)) {
+    m.box_rows = 0;
+    if (!encode_region(p, layer_k(p, layer), box_rows, &m.k, &why) ||
+        !encode_region(p, layer_v(p, layer), box_rows, &m.v, &why)) {
       *code = fail(KV_ERR_CUDA, "tensor map for layer %d: %s", layer, why.c_str());
       return nullptr;
     }
-    m.ready = true;
+    m.box_rows = box_rows;
   }
   *code = KV_OK;
   return &m;

@@ -59,14 +59,14 @@ def build_pool(pkv, wl, device, chunk=65536):
     return pool
 
 
-def step(pkv, pool, wl, device, partition_tokens=0, out=None):
+def step(pkv, pool, wl, device, num_ctas=0, out=None):
     """One decode step through the product API: append the new token, attend."""
     tables, lens = device_inputs(wl, device)
     slot_new = torch.from_numpy(wl.slot_new).to(device)
     pkv.kv_append(pool, 0, wl.k_new, wl.v_new, slot_new)
     max_ctx = int(wl.context_lens.max()) if wl.batch else 0
     return pkv.paged_attn_decode(pool, 0, wl.q, tables, lens, max_ctx, wl.scale, out=out,
-                                 partition_tokens=partition_tokens)
+                                 num_ctas=num_ctas)
 
 
 def oracle_cache_16(wl):

@@ -193,33 +193,31 @@ def test_attention_argument_validation_and_workspace_size():
     try:
         n = ctypes.c_uint64()
         # Hq must be a multiple of Hkv
-        assert B.lib.paged_attn_workspace_bytes(h, 4, 3, 250, 0, ctypes.byref(n)) == B.KV_ERR_INVALID
-        # partition must be a multiple of the block size
-        assert B.lib.paged_attn_workspace_bytes(h, 4, 8, 250, 24, ctypes.byref(n)) == B.KV_ERR_INVALID
-        # one partition: no workspace
-        B.check(B.lib.paged_attn_workspace_bytes(h, 4, 8, 250, 256, ctypes.byref(n)))
-        assert n.value == 0
-        # P = ceil(250 / 64) = 4 partitions: o [4,8,4,64] + m, l [4,8,4] fp32, 256-aligned
-        B.check(B.lib.paged_attn_workspace_bytes(h, 4, 8, 250, 64, ctypes.byref(n)))
-        parts = 4 * 8 * 4
+        assert B.lib.paged_attn_workspace_bytes(h, 4, 3, 10, ctypes.byref(n)) == B.KV_ERR_INVALID
+        assert B.lib.paged_attn_workspace_bytes(h, 4, 8, -1, ctypes.byref(n)) == B.KV_ERR_INVALID
+        # 16 B per unit (here one unit per sequence: both kv heads in one group)
+        # plus 10 CTAs x 2 sides x 8 slots x 8 heads x (64 + 2) fp32, 256-aligned parts
+        B.check(B.lib.paged_attn_workspace_bytes(h, 4, 8, 10, ctypes.byref(n)))
         r256 = lambda x: -(-x // 256) * 256
-        assert n.value == r256(parts * 64 * 4) + 2 * r256(parts * 4)
-        p = ctypes.c_int32()
-        B.check(B.lib.paged_attn_default_partition(h, 4, 8, 250, ctypes.byref(p)))
-        assert p.value % 16 == 0 and p.value >= 16
+        recs = 10 * 2 * 8 * 8
+        assert n.value == r256(4 * 1 * 16) + r256(recs * 2 * 4) + r256(recs * 64 * 4)
+        # 16 query heads per kv head (two 8-head chunks): still one unit per sequence
+        B.check(B.lib.paged_attn_workspace_bytes(h, 4, 32, 10, ctypes.byref(n)))
+        assert n.value == r256(4 * 1 * 16) + r256(recs * 2 * 4) + r256(recs * 64 * 4)
         # validation failures return before any device work
         nul = ctypes.c_void_p(0)
         fake = ctypes.c_void_p(FAKE_BASE)
-        args = lambda q, qdt, hq, tbl, mb, lens, mc, sc, out: (
-            h, 0, q, qdt, 4, hq, tbl, mb, lens, mc, sc, out, 0, fake, 1 << 20, None)
-        assert B.lib.paged_attn_decode(*args(nul, 0, 8, fake, 16, fake, 250, 0.125, fake)) == B.KV_ERR_INVALID
-        assert B.lib.paged_attn_decode(*args(fake, 1, 8, fake, 16, fake, 250, 0.125, fake)) == B.KV_ERR_UNSUPPORTED
-        assert B.lib.paged_attn_decode(*args(fake, 0, 5, fake, 16, fake, 250, 0.125, fake)) == B.KV_ERR_INVALID
-        assert B.lib.paged_attn_decode(*args(fake, 0, 8, fake, 0, fake, 250, 0.125, fake)) == B.KV_ERR_INVALID
-        assert B.lib.paged_attn_decode(*args(fake, 0, 8, fake, 16, fake, 250, float("nan"), fake)) == B.KV_ERR_INVALID
-        assert B.lib.paged_attn_decode(*args(fake, 0, 8, fake, 16, fake, -1, 0.125, fake)) == B.KV_ERR_INVALID
+        big = 1 << 20
+        args = lambda q, qdt, hq, mb, mc, sc: (h, 0, q, qdt, 4, hq, fake, mb, fake, mc, sc, fake,
+                                               10, fake, big, None)
+        assert B.lib.paged_attn_decode(*args(nul, 0, 8, 16, 250, 0.125)) == B.KV_ERR_INVALID
+        assert B.lib.paged_attn_decode(*args(fake, 1, 8, 16, 250, 0.125)) == B.KV_ERR_UNSUPPORTED
+        assert B.lib.paged_attn_decode(*args(fake, 0, 5, 16, 250, 0.125)) == B.KV_ERR_INVALID
+        assert B.lib.paged_attn_decode(*args(fake, 0, 8, 0, 250, 0.125)) == B.KV_ERR_INVALID
+        assert B.lib.paged_attn_decode(*args(fake, 0, 8, 16, 250, float("nan"))) == B.KV_ERR_INVALID
+        assert B.lib.paged_attn_decode(*args(fake, 0, 8, 16, -1, 0.125)) == B.KV_ERR_INVALID
         # too small a workspace
-        st = B.lib.paged_attn_decode(h, 0, fake, 0, 4, 8, fake, 16, fake, 250, 0.125, fake, 64,
+        st = B.lib.paged_attn_decode(h, 0, fake, 0, 4, 8, fake, 16, fake, 250, 0.125, fake, 10,
                                      fake, 16, None)
         assert st == B.KV_ERR_INVALID
         # append / quantize validation
@@ -243,8 +241,10 @@ def test_valid_call_without_a_gpu_fails_loudly():
     h, _ = _make_pool(64, 1, 16, 2, 64, "bf16")
     try:
         fake = ctypes.c_void_p(FAKE_BASE)
-        st = B.lib.paged_attn_decode(h, 0, fake, 0, 4, 8, fake, 16, fake, 250, 0.125, fake, 0,
+        st = B.lib.paged_attn_decode(h, 0, fake, 0, 4, 8, fake, 16, fake, 250, 0.125, fake, 10,
                                      fake, 1 << 20, None)
         assert st == B.KV_ERR_CUDA
+        n = ctypes.c_uint64()
+        assert B.lib.paged_attn_workspace_bytes(h, 4, 8, 0, ctypes.byref(n)) == B.KV_ERR_CUDA
     finally:
         B.lib.kv_pool_destroy(h)

@@ -78,7 +78,9 @@ def test_quantize_bit_exact(pkv, kind, in_dt, D):
     g = torch.Generator(device=DEV).manual_seed(D)
     x = torch.randn(20000, D, generator=g, device=DEV)
     x = x * torch.exp(torch.randn(20000, 1, generator=g, device=DEV) * 3)   # wide dynamic range
+    x = x.clamp(-6e4, 6e4)                                                  # finite in fp16
     x = torch.cat([x, torch.from_numpy(_special_rows(D)).float().to(DEV)]).to(in_dt)
+    assert torch.isfinite(x.float()).all()
     codes, scales = pkv.kv_quantize(x, kind)
     torch.cuda.synchronize()
     ref_codes, ref_scales = quant.quantize_rows(to_np(x), kind)

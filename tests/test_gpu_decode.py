@@ -31,9 +31,9 @@ def _all_pairs(wl, seqs=None):
     return [(b, h) for b in seqs for h in range(wl.q_heads)]
 
 
-def _run_16(pkv, wl, partition_tokens=0, seqs=None):
+def _run_16(pkv, wl, num_ctas=0, seqs=None):
     pool = build_pool(pkv, wl, DEV)
-    out = step(pkv, pool, wl, DEV, partition_tokens)
+    out = step(pkv, pool, wl, DEV, num_ctas)
     torch.cuda.synchronize()
     assert pool.status() == 0
     k, v = oracle_cache_16(wl)
@@ -43,13 +43,15 @@ def _run_16(pkv, wl, partition_tokens=0, seqs=None):
     return compare(got, ref, what=wl.name)
 
 
-def test_tiny_default_partition(pkv):
+def test_tiny_default_split(pkv):
     _run_16(pkv, W.tiny(DEV))
 
 
-@pytest.mark.parametrize("S", [16, 48, 64, 128, 256, 4096])
-def test_tiny_partition_sizes_agree(pkv, S):
-    _run_16(pkv, W.tiny(DEV), partition_tokens=S)
+@pytest.mark.parametrize("G", [1, 2, 3, 5, 13, 56, 57, 200])
+def test_tiny_split_counts_agree(pkv, G):
+    """The tiny case has 56 (sequence, kv head) blocks: from one CTA doing
+    everything to more CTAs than blocks (idle CTAs), splits fall everywhere."""
+    _run_16(pkv, W.tiny(DEV), num_ctas=G)
 
 
 def test_gqa70b_every_output(pkv):
@@ -57,9 +59,9 @@ def test_gqa70b_every_output(pkv):
     _run_16(pkv, W.gqa70b(DEV))
 
 
-@pytest.mark.parametrize("S", [256, 1024, 4096])
-def test_gqa70b_split_k_sizes(pkv, S):
-    _run_16(pkv, W.gqa70b(DEV), partition_tokens=S, seqs=[0, 7, 19, 31])
+@pytest.mark.parametrize("G", [7, 300, 2000])
+def test_gqa70b_split_counts(pkv, G):
+    _run_16(pkv, W.gqa70b(DEV), num_ctas=G, seqs=[0, 7, 19, 31])
 
 
 def test_mha13b_every_output(pkv):
@@ -191,15 +193,15 @@ EDGE_LENS = [0, 1, 15, 16, 17, 63, 64, 65, 127, 128, 129, 300]
 @pytest.mark.parametrize("G", [1, 2, 4, 8, 16])
 @pytest.mark.parametrize("D,bs", [(64, 16), (128, 32)])
 def test_edge_lengths_groups_dims(pkv, cache, G, D, bs):
-    """Empty, single-token, block-boundary and partition-boundary lengths; MHA,
-    GQA groups of 2..16 heads (16 spans two head chunks); head_dim 64 / 128;
-    block size 16 / 32; all four cache types; partitions of 4 blocks."""
+    """Empty, single-token and block-boundary lengths; MHA, GQA groups of 2..16
+    heads (16 spans two head units); head_dim 64 / 128; block size 16 / 32; all
+    four cache types; 13 CTAs, so units are split at assorted places."""
     qd = "fp16" if cache == "fp16" else "bf16"
     lens = EDGE_LENS
     wl = W.make_decode_workload("edge", len(lens), 2 * G, 2, D, bs, qd, cache, lens,
                                 seed=G * 1000 + D + bs, device=DEV)
     pool = build_pool(pkv, wl, DEV)
-    out = step(pkv, pool, wl, DEV, partition_tokens=4 * bs)
+    out = step(pkv, pool, wl, DEV, num_ctas=13)
     torch.cuda.synchronize()
     assert pool.status() == 0
     pairs = _all_pairs(wl)
@@ -216,14 +218,14 @@ def test_edge_lengths_groups_dims(pkv, cache, G, D, bs):
 def test_separate_phases_equal_fused_call(pkv):
     wl = W.gqa70b(DEV, batch=8)
     pool = build_pool(pkv, wl, DEV)
-    out = step(pkv, pool, wl, DEV, partition_tokens=512)
+    out = step(pkv, pool, wl, DEV, num_ctas=37)
     tables, lens = device_inputs(wl, DEV)
-    ws = pkv.make_workspace(pool, wl.batch, wl.q_heads, int(wl.context_lens.max()), 512)
+    ws = pkv.make_workspace(pool, wl.batch, wl.q_heads, 37)
     out2 = torch.empty_like(out)
     pkv.paged_attn_partition(pool, 0, wl.q, tables, lens, int(wl.context_lens.max()), wl.scale,
-                             out2, ws, partition_tokens=512)
+                             out2, ws, num_ctas=37)
     pkv.paged_attn_merge(pool, lens, tables.shape[1], int(wl.context_lens.max()), out2, ws,
-                         partition_tokens=512)
+                         num_ctas=37)
     torch.cuda.synchronize()
     assert torch.equal(out, out2)
 
