@@ -275,6 +275,29 @@ kv_status paged_attn_decode(kv_pool *pool, int32_t layer, const void *q,
                             void *workspace, uint64_t workspace_bytes,
                             kv_stream_t stream);
 
+/* paged_attn_decode for callers that cannot allocate a workspace -- for
+ * example a serving process that has given all free GPU memory to its KV pool
+ * and admits no further allocation, or an application reaching this library
+ * through a plugin or foreign-function layer with no device allocator. The
+ * pages have no counterpart; this is a convenience of this library.
+ * The split-K scratch lives in a 16 MiB array inside the library's own device
+ * memory (every GPU that loads the library holds it until the process exits).
+ * The first call on each device looks up that array's device address with the
+ * device current; make that first call before any stream capture. Calls whose
+ * scratch would exceed 16 MiB (paged_attn_workspace_bytes for the same
+ * num_seqs, num_q_heads, num_ctas) return KV_ERR_INVALID and queue nothing.
+ * Every call uses the same array, so calls that overlap on the GPU (on
+ * different streams, or on one device from several threads without ordering)
+ * race and corrupt each other's results; serialize them. No call allocates.
+ * Other arguments and results are those of paged_attn_decode. */
+kv_status paged_attn_decode_static(kv_pool *pool, int32_t layer, const void *q,
+                                   int32_t q_dtype, int32_t num_seqs,
+                                   int32_t num_q_heads, const int32_t *block_tables,
+                                   int32_t max_blocks_per_seq,
+                                   const int32_t *context_lens,
+                                   int32_t max_context, float scale, void *out,
+                                   int32_t num_ctas, kv_stream_t stream);
+
 /* Phase 1 alone: the persistent attention kernel. Writes out for the units it
  * finishes and the workspace partials and bookkeeping for split units. */
 kv_status paged_attn_partition(kv_pool *pool, int32_t layer, const void *q,

@@ -71,6 +71,8 @@ _SIGS = {
                              _I32, _P, _U64, _P],
     "paged_attn_merge": [_P, _I32, _I32, _P, _I32, _I32, _I32, _I32, _P, _P, _U64, _P],
     "kv_selftest_wait_timeout": [_P, ctypes.c_uint32, _P],
+    "paged_attn_decode_static": [_P, _I32, _P, _I32, _I32, _I32, _P, _I32, _P, _I32, _F, _P,
+                                 _I32, _P],
 }
 for _name, _args in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -308,6 +310,19 @@ def paged_attn_decode(pool, layer, q, block_tables, context_lens, max_context, s
                                 _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
                                 max_context, float(scale), _ptr(out), num_ctas,
                                 _ptr(workspace), workspace.numel(), _stream(stream, pool.device)))
+    return out
+
+
+def paged_attn_decode_static(pool, layer, q, block_tables, context_lens, max_context, scale,
+                             out=None, num_ctas=0, stream=None):
+    """paged_attn_decode without a workspace argument: the library's built-in
+    16 MiB scratch is used instead (see include/pagedkv.h). For callers that
+    cannot allocate device memory; calls must not overlap on the GPU."""
+    B, Hq, out = _attn_args(pool, q, block_tables, context_lens, out)
+    check(lib.paged_attn_decode_static(pool.handle, layer, _ptr(q), TORCH_CODES[q.dtype], B, Hq,
+                                       _ptr(block_tables), block_tables.shape[1],
+                                       _ptr(context_lens), max_context, float(scale), _ptr(out),
+                                       num_ctas, _stream(stream, pool.device)))
     return out
 
 

@@ -1329,3 +1329,77 @@ kv_status paged_attn_decode(kv_pool *pool, int32_t layer, const void *q, int32_t
 }
 
 }  // extern "C"
+
+// ============================================================================
+// Decode attention for callers that cannot allocate a workspace.
+//
+// Some callers cannot hand this library a workspace: a serving process that
+// has already given all of the GPU's free memory to its KV pool and admits no
+// further allocation, or a host application that reaches this library through
+// a plugin or foreign-function interface with no access to a device
+// allocator. For them, paged_attn_decode_static keeps the split-K scratch in a
+// fixed array compiled into this library instead. Every GPU that loads the
+// library holds that array until the process exits.
+// ============================================================================
+
+// The scratch: unit bookkeeping and split partials, as for a caller workspace.
+static __device__ __align__(256) unsigned char g_decode_scratch[16u << 20];
+
+namespace pagedkv {
+namespace {
+
+constexpr uint64_t kStaticScratchBytes = 16ull << 20;
+constexpr int kMaxScratchDevices = 64;
+std::mutex g_scratch_mu;
+void *g_scratch_ptr[kMaxScratchDevices];  // device address of the array, per device
+
+// Device address of the scratch array on the current device. Host code cannot
+// use the array's name as a device pointer (it is a host-side stand-in), so the
+// address is looked up once per device, with that device current.
+kv_status scratch_address(void **out) {
+  int dev = 0;
+  kv_status s = cuda_check(cudaGetDevice(&dev), "cudaGetDevice");
+  if (s != KV_OK) return s;
+  if (dev < 0 || dev >= kMaxScratchDevices)
+    return fail(KV_ERR_UNSUPPORTED, "device %d: at most %d devices", dev, kMaxScratchDevices);
+  std::lock_guard<std::mutex> g(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void *ptr = nullptr;
+    s = cuda_check(cudaGetSymbolAddress(&ptr, g_decode_scratch), "scratch address");
+    if (s != KV_OK) return s;
+    g_scratch_ptr[dev] = ptr;
+  }
+  *out = g_scratch_ptr[dev];
+  return KV_OK;
+}
+
+}  // namespace
+}  // namespace pagedkv
+
+extern "C" kv_status paged_attn_decode_static(kv_pool *pool, int32_t layer, const void *q,
+                                              int32_t q_dtype, int32_t num_seqs,
+                                              int32_t num_q_heads, const int32_t *block_tables,
+                                              int32_t max_blocks_per_seq,
+                                              const int32_t *context_lens, int32_t max_context,
+                                              float scale, void *out, int32_t num_ctas,
+                                              kv_stream_t stream) {
+  int G = 0;
+  kv_status s = check_attn(pool, num_seqs, num_q_heads, max_context, num_ctas, &G);
+  if (s != KV_OK) return s;
+  const UnitGeom u = unit_geom(pool, num_q_heads);
+  const uint64_t need = ws_layout(num_seqs, u.units_per_seq, G, pool->d.head_dim).total;
+  if (need > kStaticScratchBytes)
+    return fail(KV_ERR_INVALID,
+                "these sizes need %llu bytes of scratch; the built-in scratch holds %llu "
+                "(use fewer sequences or CTAs, or paged_attn_decode with a workspace)",
+                static_cast<unsigned long long>(need),
+                static_cast<unsigned long long>(kStaticScratchBytes));
+  void *ws = nullptr;
+  s = scratch_address(&ws);
+  if (s != KV_OK) return s;
+  // Nothing in the scratch needs to start at zero: the partition kernel writes
+  // every bookkeeping entry and partial that the merge kernel then reads.
+  return paged_attn_decode(pool, layer, q, q_dtype, num_seqs, num_q_heads, block_tables,
+                           max_blocks_per_seq, context_lens, max_context, scale, out, num_ctas,
+                           ws, kStaticScratchBytes, stream);
+}
