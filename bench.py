@@ -218,19 +218,11 @@ def run_ours(args, rank, world, device):
     def flush_l2():
         torch.sum(flush, 0, out=flush_sink)
 
-    def one_step(ev=None):
-        if ev:
-            ev[0].record(stream)
+    def one_step():
         pkv.kv_append(pool, 0, wl.k_new, wl.v_new, slot_new)
-        if ev:
-            ev[1].record(stream)
         pkv.paged_attn_partition(pool, 0, wl.q, tables, lens, max_ctx, wl.scale, out, ws,
                                  num_ctas=G)
-        if ev:
-            ev[2].record(stream)
         pkv.paged_attn_merge(pool, lens, tables.shape[1], max_ctx, out, ws, num_ctas=G)
-        if ev:
-            ev[3].record(stream)
 
     for _ in range(args.warmup):
         flush_l2()
@@ -238,30 +230,48 @@ def run_ours(args, rank, world, device):
     torch.cuda.synchronize(device)
     pool.status_clear()
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    # Timed region: K steps, each bracketed by events with nothing between its
+    # three kernels (so each may launch while its predecessor finishes); the L2
+    # flush before each step is outside the events.
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
     sampler = ClockSampler(device.index if device.index is not None else 0).start()
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(device)
     t0 = time.time()
     for i in range(args.steps):
-        flush_l2()                              # evict L2 outside the timed events
-        one_step(evs[i])
+        flush_l2()
+        evs[i][0].record(stream)
+        one_step()
+        evs[i][1].record(stream)
     torch.cuda.synchronize(device)
     t1 = time.time()
     if world > 1:
         torch.distributed.barrier()
+    # The attention kernel alone, same conditions (L2 flushed before each launch),
+    # for its roofline fraction.
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush_l2()
+        kev[i][0].record(stream)
+        pkv.paged_attn_partition(pool, 0, wl.q, tables, lens, max_ctx, wl.scale, out, ws,
+                                 num_ctas=G)
+        kev[i][1].record(stream)
+    torch.cuda.synchronize(device)
+    t2 = time.time()
     sampler.stop()
     status = pool.status()
-    step_ms = np.array([e[0].elapsed_time(e[3]) for e in evs])
-    part_ms = np.array([e[1].elapsed_time(e[2]) for e in evs])
+    step_ms = np.array([a.elapsed_time(b) for a, b in evs])
+    part_ms = np.array([a.elapsed_time(b) for a, b in kev])
     step_s = float(step_ms.mean()) / 1e3
     part_s = float(part_ms.mean()) / 1e3
     if world > 1:
         t = torch.tensor([step_s, part_s], device=device, dtype=torch.float64)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         step_s, part_s = float(t[0]), float(t[1])
-    clocks = sampler.summary(t0, t1)
+    clocks = sampler.summary(t0, t2)
 
     # ---------------------------------------------------------- end to end
     e2e = None

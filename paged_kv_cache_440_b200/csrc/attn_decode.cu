@@ -777,6 +777,8 @@ attn_partition_kernel(const __grid_constant__ CUtensorMap kmap,
   const int R = p.stages;
 
   // ---------------------------------------------------------------- prologue
+  launch_dependents();      // let the merge kernel be scheduled early
+  grid_dependency_wait();   // inputs may come from the previous kernel
   // Total positions over all units, then this CTA's even share [s0, s1).
   long long part = 0;
   for (int b = threadIdx.x; b < B; b += kThreads) {
@@ -960,6 +962,8 @@ constexpr int kMergeWarps = 8;
 
 template <int D, int OUT_T>
 __global__ void __launch_bounds__(kMergeWarps * 32) attn_merge_kernel(const AttnParams p) {
+  launch_dependents();
+  grid_dependency_wait();  // the partials come from the partition kernel
   const int w = blockIdx.x * kMergeWarps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (w >= p.num_seqs * p.q_heads) return;
@@ -1041,7 +1045,8 @@ cudaError_t launch_part(const CUtensorMap &km, const CUtensorMap &vm, const Attn
   auto kern = attn_partition_kernel<D, BS, KV_T, Q_T, MMA>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  kern<<<p.num_ctas, kThreads, smem, st>>>(km, vm, p);
+  e = launch_pdl(kern, dim3(p.num_ctas), dim3(kThreads), smem, st, km, vm, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -1073,13 +1078,15 @@ cudaError_t launch_merge(int D, int out_t, const AttnParams &p, cudaStream_t st)
   const int64_t warps = static_cast<int64_t>(p.num_seqs) * p.q_heads;
   const unsigned grid = static_cast<unsigned>((warps + kMergeWarps - 1) / kMergeWarps);
   const int th = kMergeWarps * 32;
+  cudaError_t e;
   if (D == 128) {
-    if (out_t == KV_BF16) attn_merge_kernel<128, KV_BF16><<<grid, th, 0, st>>>(p);
-    else attn_merge_kernel<128, KV_FP16><<<grid, th, 0, st>>>(p);
+    e = out_t == KV_BF16 ? launch_pdl(attn_merge_kernel<128, KV_BF16>, dim3(grid), dim3(th), 0, st, p)
+                         : launch_pdl(attn_merge_kernel<128, KV_FP16>, dim3(grid), dim3(th), 0, st, p);
   } else {
-    if (out_t == KV_BF16) attn_merge_kernel<64, KV_BF16><<<grid, th, 0, st>>>(p);
-    else attn_merge_kernel<64, KV_FP16><<<grid, th, 0, st>>>(p);
+    e = out_t == KV_BF16 ? launch_pdl(attn_merge_kernel<64, KV_BF16>, dim3(grid), dim3(th), 0, st, p)
+                         : launch_pdl(attn_merge_kernel<64, KV_FP16>, dim3(grid), dim3(th), 0, st, p);
   }
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

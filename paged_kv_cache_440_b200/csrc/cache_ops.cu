@@ -44,6 +44,8 @@ append16_kernel(const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new
                 const int64_t *__restrict__ slots, int num_tokens, int kv_heads,
                 int block_size, int row_chunks, int64_t num_slots, char *__restrict__ kc,
                 char *__restrict__ vc, int *status) {
+  launch_dependents();
+  grid_dependency_wait();
   const int warp = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (warp >= num_tokens * kv_heads) return;
@@ -140,6 +142,8 @@ append_quant_kernel(const uint16_t *__restrict__ k_new, const uint16_t *__restri
                     int block_size, int64_t num_slots, uint8_t *__restrict__ kc,
                     uint8_t *__restrict__ vc, float *__restrict__ ks, float *__restrict__ vs,
                     int *status) {
+  launch_dependents();
+  grid_dependency_wait();
   const int warp = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (warp >= num_tokens * kv_heads) return;
@@ -229,11 +233,13 @@ cudaError_t launch_append_quant(kv_pool *p, int layer, const void *k, const void
                                 const int64_t *slots, int T, cudaStream_t st) {
   const int64_t warps = (int64_t)T * p->d.num_kv_heads;
   const int64_t grid = (warps + kWarpsPerCta - 1) / kWarpsPerCta;
-  append_quant_kernel<D, IN_T, OUT_T><<<(unsigned)grid, kWarpsPerCta * 32, 0, st>>>(
+  cudaError_t e = launch_pdl(
+      append_quant_kernel<D, IN_T, OUT_T>, dim3((unsigned)grid), dim3(kWarpsPerCta * 32), 0, st,
       static_cast<const uint16_t *>(k), static_cast<const uint16_t *>(v), slots, T,
       p->d.num_kv_heads, p->d.block_size, (int64_t)p->d.num_blocks * p->d.block_size,
       reinterpret_cast<uint8_t *>(layer_k(p, layer)), reinterpret_cast<uint8_t *>(layer_v(p, layer)),
       layer_ks(p, layer), layer_vs(p, layer), status_word(p));
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -283,12 +289,12 @@ kv_status kv_append(kv_pool *pool, int32_t layer, const void *k_new, const void 
     if (in_dtype != cd)
       return fail(KV_ERR_UNSUPPORTED, "a 16-bit cache takes rows of its own dtype");
     const int64_t grid = (warps + kWarpsPerCta - 1) / kWarpsPerCta;
-    append16_kernel<<<(unsigned)grid, kWarpsPerCta * 32, 0, st>>>(
-        static_cast<const uint4 *>(k_new), static_cast<const uint4 *>(v_new), slot_mapping,
-        num_tokens, pool->d.num_kv_heads, pool->d.block_size, pool->row_bytes / 16,
-        (int64_t)pool->d.num_blocks * pool->d.block_size, layer_k(pool, layer),
-        layer_v(pool, layer), status_word(pool));
-    e = cudaGetLastError();
+    e = launch_pdl(append16_kernel, dim3((unsigned)grid), dim3(kWarpsPerCta * 32), 0, st,
+                   static_cast<const uint4 *>(k_new), static_cast<const uint4 *>(v_new),
+                   slot_mapping, num_tokens, pool->d.num_kv_heads, pool->d.block_size,
+                   pool->row_bytes / 16, (int64_t)pool->d.num_blocks * pool->d.block_size,
+                   layer_k(pool, layer), layer_v(pool, layer), status_word(pool));
+    if (e == cudaSuccess) e = cudaGetLastError();
   } else if (cd == KV_INT8) {
     e = in_dtype == KV_BF16
             ? dispatch_append_quant_d<KV_BF16, KV_INT8>(pool, layer, k_new, v_new, slot_mapping, num_tokens, st)

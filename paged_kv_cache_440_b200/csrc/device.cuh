@@ -32,6 +32,20 @@ __device__ __forceinline__ uint64_t globaltimer() {
   return t;
 }
 
+// ------------------------------------------------- programmatic dependent launch
+// Kernels of this library are launched so that the next kernel in the stream
+// may be scheduled before they finish (launch_dependents). Each kernel waits
+// for the previous grid to complete, with its memory visible, before it reads
+// any input (grid_dependency_wait); without such a launch both are no-ops.
+
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {

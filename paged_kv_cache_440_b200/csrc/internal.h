@@ -7,6 +7,7 @@
 #include <cstdint>
 #include <mutex>
 #include <string>
+#include <utility>
 #include <vector>
 
 #include "pagedkv.h"
@@ -84,6 +85,25 @@ inline float *layer_vs(const kv_pool *p, int layer) {
 }
 inline int32_t *status_word(const kv_pool *p) {
   return (int32_t *)(p->base + p->lay.status_off);
+}
+
+// Launch `kern` on `st` so that it may be scheduled while the previous kernel
+// in the stream is still running (programmatic stream serialization). The
+// kernel must call grid_dependency_wait() before reading its inputs.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 // Tensor maps for the layer's K and V regions with boxes of box_rows rows;
