@@ -970,13 +970,6 @@ __global__ void __launch_bounds__(kMergeWarps * 32) attn_merge_kernel(const Attn
   constexpr int E = D / 32;
   const int b = w / p.q_heads;
   const int h = w - b * p.q_heads;
-  const int L = p.context_lens[b];
-  const int64_t orow = static_cast<int64_t>(w) * D + lane * E;
-  if (!(L > 0 && L <= p.limit)) {
-#pragma unroll
-    for (int e = 0; e < E; ++e) store_out<OUT_T>(p.out, orow + e, 0.f);
-    return;
-  }
   // (unit, slot, head) of query head h, as the partition kernel assigned them
   const int g = h / p.group;
   const int r = h - g * p.group;
@@ -986,7 +979,16 @@ __global__ void __launch_bounds__(kMergeWarps * 32) attn_merge_kernel(const Attn
   const int cgi = chunk / p.cpg, cl = chunk - cgi * p.cpg;
   const int cpg = min(p.cpg, p.chunks - cgi * p.cpg);
   const int slot = hi * cpg + cl;
+  // length and bookkeeping in one round trip (the bookkeeping is used only
+  // for a valid, non-empty length: it is rewritten for such units every call)
+  const int L = p.context_lens[b];
   const int4 mt = p.meta[static_cast<int64_t>(b) * p.units_per_seq + hgi * p.cgroups + cgi];
+  const int64_t orow = static_cast<int64_t>(w) * D + lane * E;
+  if (!(L > 0 && L <= p.limit)) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) store_out<OUT_T>(p.out, orow + e, 0.f);
+    return;
+  }
   const int nu = mt.y;
   if (nu <= 1) return;  // finished by the partition kernel
   if (mt.x < 0 || mt.x >= p.num_ctas || nu > p.num_ctas - mt.x || (mt.z & ~1)) {
@@ -996,40 +998,47 @@ __global__ void __launch_bounds__(kMergeWarps * 32) attn_merge_kernel(const Attn
   auto rec = [&](int i) -> int64_t {
     return ((static_cast<int64_t>(mt.x + i) * 2 + (i == 0 ? mt.z : 0)) * kNC + slot) * kChunkHeads + n;
   };
-  float M = -INFINITY;
-  for (int i = lane; i < nu; i += 32) M = fmaxf(M, p.part_ml[rec(i) * 2]);
-  M = warp_max_xor(M, 1);
-  float acc[E];
+  auto load_o = [&](int i, float (&v)[E]) {
+    const float *o = p.part_o + rec(i) * D + lane * E;
+    if constexpr (E == 4) {
+      const float4 x = *reinterpret_cast<const float4 *>(o);
+      v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+    } else {
+      const float2 x = *reinterpret_cast<const float2 *>(o);
+      v[0] = x.x; v[1] = x.y;
+    }
+  };
+  // one online pass: running max M, sum Ls and output acc; piece i + 1 is
+  // loaded while piece i is combined
+  float M = -INFINITY, Ls = 0.f;
+  float acc[E], o[E], o_n[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) acc[e] = 0.f;
-  float Ls = 0.f;
-  if (M != -INFINITY) {
-    for (int i0 = 0; i0 < nu; i0 += 32) {
-      const int i = i0 + lane;
-      const float wgt = i < nu ? exp2_rel(p.part_ml[rec(i) * 2], M) : 0.f;
-      Ls += i < nu ? wgt * p.part_ml[rec(i) * 2 + 1] : 0.f;
-      const int cnt = min(32, nu - i0);
-      for (int kk = 0; kk < cnt; ++kk) {
-        const float wk = __shfl_sync(0xffffffffu, wgt, kk);
-        const float *o = p.part_o + rec(i0 + kk) * D + lane * E;
-        if constexpr (E == 4) {
-          const float4 v = *reinterpret_cast<const float4 *>(o);
-          acc[0] = fmaf(wk, v.x, acc[0]);
-          acc[1] = fmaf(wk, v.y, acc[1]);
-          acc[2] = fmaf(wk, v.z, acc[2]);
-          acc[3] = fmaf(wk, v.w, acc[3]);
-        } else {
-          const float2 v = *reinterpret_cast<const float2 *>(o);
-          acc[0] = fmaf(wk, v.x, acc[0]);
-          acc[1] = fmaf(wk, v.y, acc[1]);
-        }
-      }
+  float2 ml = *reinterpret_cast<const float2 *>(p.part_ml + rec(0) * 2);
+  load_o(0, o);
+  for (int i = 0; i < nu; ++i) {
+    float2 ml_n = ml;
+    if (i + 1 < nu) {
+      ml_n = *reinterpret_cast<const float2 *>(p.part_ml + rec(i + 1) * 2);
+      load_o(i + 1, o_n);
     }
+    const float Mn = fmaxf(M, ml.x);
+    if (Mn != -INFINITY) {
+      const float a = exp2_rel(M, Mn), wt = exp2_rel(ml.x, Mn);
+      Ls = Ls * a + ml.y * wt;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
+      for (int e = 0; e < E; ++e) acc[e] = acc[e] * a + o[e] * wt;
+      M = Mn;
+    }
+    if (i + 1 < nu) {
+      ml = ml_n;
+#pragma unroll
+      for (int e = 0; e < E; ++e) o[e] = o_n[e];
+    }
   }
+  const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
 #pragma unroll
-  for (int e = 0; e < E; ++e) store_out<OUT_T>(p.out, orow + e, Ls > 0.f ? acc[e] / Ls : 0.f);
+  for (int e = 0; e < E; ++e) store_out<OUT_T>(p.out, orow + e, acc[e] * inv);
 }
 
 // ============================================================================
