@@ -3,9 +3,11 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload gqa70b|mha13b|quant_a_int8|...] [--ctas G]
 
-A step is the whole hot path for one batch: append of each sequence's new K/V
-token into the paged cache (kv_append), then paged decode attention
-(persistent partition kernel + merge kernel), all through the library's C ABI.
+A step is the whole hot path for one batch: the append of each sequence's new
+K/V token into the paged cache and the paged decode attention over the cache
+including it, through the library's C ABI: paged_attn_decode_append (the
+append folded into the persistent attention kernel) and its split-K merge
+kernel; with --separate-append, kv_append + paged_attn_decode instead.
 
 Workload (default): batch 32, 64 query / 8 KV heads, head_dim 128, bf16,
 16-token blocks, context lengths uniform on [512, 4096] (seed 0), pool 1.2x
@@ -218,11 +220,16 @@ def run_ours(args, rank, world, device):
     def flush_l2():
         torch.sum(flush, 0, out=flush_sink)
 
+    fused = not args.separate_append and wl.group <= 8
+
     def one_step():
-        pkv.kv_append(pool, 0, wl.k_new, wl.v_new, slot_new)
-        pkv.paged_attn_partition(pool, 0, wl.q, tables, lens, max_ctx, wl.scale, out, ws,
-                                 num_ctas=G)
-        pkv.paged_attn_merge(pool, lens, tables.shape[1], max_ctx, out, ws, num_ctas=G)
+        if fused:   # append folded into the attention kernel, then the merge
+            pkv.paged_attn_decode_append(pool, 0, wl.q, wl.k_new, wl.v_new, tables, lens,
+                                         max_ctx, wl.scale, out=out, num_ctas=G, workspace=ws)
+        else:
+            pkv.kv_append(pool, 0, wl.k_new, wl.v_new, slot_new)
+            pkv.paged_attn_decode(pool, 0, wl.q, tables, lens, max_ctx, wl.scale, out=out,
+                                  num_ctas=G, workspace=ws)
 
     for _ in range(args.warmup):
         flush_l2()
@@ -231,8 +238,8 @@ def run_ours(args, rank, world, device):
     pool.status_clear()
 
     # Timed region: K steps, each bracketed by events with nothing between its
-    # three kernels (so each may launch while its predecessor finishes); the L2
-    # flush before each step is outside the events.
+    # kernels (so each may launch while its predecessor finishes); the L2 flush
+    # before each step is outside the events.
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
     sampler = ClockSampler(device.index if device.index is not None else 0).start()
@@ -256,8 +263,12 @@ def run_ours(args, rank, world, device):
     for i in range(args.steps):
         flush_l2()
         kev[i][0].record(stream)
-        pkv.paged_attn_partition(pool, 0, wl.q, tables, lens, max_ctx, wl.scale, out, ws,
-                                 num_ctas=G)
+        if fused:
+            pkv.paged_attn_partition_append(pool, 0, wl.q, wl.k_new, wl.v_new, tables, lens,
+                                            max_ctx, wl.scale, out, ws, num_ctas=G)
+        else:
+            pkv.paged_attn_partition(pool, 0, wl.q, tables, lens, max_ctx, wl.scale, out, ws,
+                                     num_ctas=G)
         kev[i][1].record(stream)
     torch.cuda.synchronize(device)
     t2 = time.time()
@@ -295,9 +306,13 @@ def run_ours(args, rank, world, device):
             for d, h in ((d_q, h_q), (d_kn, h_kn), (d_vn, h_vn), (d_slot, h_slot),
                          (d_tab, h_tab), (d_len, h_len)):
                 d.copy_(h, non_blocking=True)
-            pkv.kv_append(pool, 0, d_kn, d_vn, d_slot)
-            pkv.paged_attn_decode(pool, 0, d_q, d_tab, d_len, max_ctx, wl.scale, out=d_out,
-                                  num_ctas=G, workspace=ws)
+            if fused:
+                pkv.paged_attn_decode_append(pool, 0, d_q, d_kn, d_vn, d_tab, d_len, max_ctx,
+                                             wl.scale, out=d_out, num_ctas=G, workspace=ws)
+            else:
+                pkv.kv_append(pool, 0, d_kn, d_vn, d_slot)
+                pkv.paged_attn_decode(pool, 0, d_q, d_tab, d_len, max_ctx, wl.scale, out=d_out,
+                                      num_ctas=G, workspace=ws)
             h_out.copy_(d_out, non_blocking=True)
             b_.record(stream)
             b_.synchronize()
@@ -312,8 +327,8 @@ def run_ours(args, rank, world, device):
 
     dec_bytes, app_bytes = step_bytes(wl)
     res = {"wl": wl, "desc": desc, "G": G, "step_s": step_s, "part_s": part_s,
-           "dec_bytes": dec_bytes, "app_bytes": app_bytes, "clocks": clocks,
-           "status": status, "e2e": e2e, "launches": args.steps * 3,
+           "dec_bytes": dec_bytes, "app_bytes": app_bytes, "clocks": clocks, "fused": fused,
+           "status": status, "e2e": e2e, "launches": args.steps * (2 if fused else 3),
            "wall": t1 - t0}
     return res
 
@@ -327,6 +342,8 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="gqa70b")
     ap.add_argument("--ctas", type=int, default=0, help="CTAs of the attention kernel (0 = one per SM)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--separate-append", action="store_true",
+                    help="kv_append + paged_attn_decode instead of paged_attn_decode_append")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     args = ap.parse_args()
@@ -372,7 +389,10 @@ def main():
     total_bytes = (r["dec_bytes"] + r["app_bytes"]) * world
     gbs = total_bytes / r["step_s"] / 1e9
     peak, peak_kind = measured_peak()
-    achieved = r["dec_bytes"] / r["part_s"] / 1e9
+    # the timed kernel's algorithmic bytes: the KV stream, q and out, plus the
+    # new rows when the append is folded into it
+    kern_bytes = r["dec_bytes"] + (r["app_bytes"] if r.get("fused") else 0)
+    achieved = kern_bytes / r["part_s"] / 1e9
     traffic = None
     try:
         with open(TRAFFIC_FILE) as f:
@@ -405,7 +425,9 @@ def main():
             "decode_tokens_per_s": round(wl.batch * world / r["step_s"], 1),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
                          "unit": "GB/s", "frac": round(achieved / peak, 4),
-                         "traffic": traffic, "kernel": "attn_partition_kernel",
+                         "traffic": traffic,
+                         "kernel": "attn_partition_kernel" + (" (append fused)" if r.get("fused")
+                                                              else ""),
                          "peak_source": peak_kind + " (MEASURED_PEAKS.json hbm_gbs)"
                          if peak_kind == "measured" else "fallback 6650 GB/s",
                          "kernel_ms": round(r["part_s"] * 1e3, 5)},

@@ -298,6 +298,29 @@ kv_status paged_attn_decode_static(kv_pool *pool, int32_t layer, const void *q,
                                    int32_t max_context, float scale, void *out,
                                    int32_t num_ctas, kv_stream_t stream);
 
+/* A decode step with the append folded into the attention kernel: for every
+ * sequence b with a valid length L_b > 0, the new token's rows k_new[b] and
+ * v_new[b] are written at position L_b - 1, i.e. row (L_b - 1) % block_size of
+ * block block_tables[b][(L_b - 1) / block_size] (quantized exactly as
+ * kv_append does for INT8 / E5M2 caches), and the attention over positions
+ * 0 .. L_b - 1 uses them. The same results as kv_append with those slots
+ * followed by paged_attn_decode, with one kernel fewer. Only the new token's
+ * K and V are computed each step and put at the cache end
+ * [KV Cache 原理与 PagedAttention, §一].
+ * k_new, v_new: device [num_seqs][num_kv_heads][head_dim] of q_dtype (for a
+ *   16-bit cache, its own dtype: rows are copied bit for bit), 16-byte aligned.
+ * Needs num_q_heads / num_kv_heads <= 8 (else KV_ERR_UNSUPPORTED: use
+ * kv_append and paged_attn_decode). Other arguments as paged_attn_decode. */
+kv_status paged_attn_decode_append(kv_pool *pool, int32_t layer, const void *q,
+                                   const void *k_new, const void *v_new,
+                                   int32_t q_dtype, int32_t num_seqs,
+                                   int32_t num_q_heads, const int32_t *block_tables,
+                                   int32_t max_blocks_per_seq,
+                                   const int32_t *context_lens,
+                                   int32_t max_context, float scale, void *out,
+                                   int32_t num_ctas, void *workspace,
+                                   uint64_t workspace_bytes, kv_stream_t stream);
+
 /* Phase 1 alone: the persistent attention kernel. Writes out for the units it
  * finishes and the workspace partials and bookkeeping for split units. */
 kv_status paged_attn_partition(kv_pool *pool, int32_t layer, const void *q,
@@ -308,6 +331,20 @@ kv_status paged_attn_partition(kv_pool *pool, int32_t layer, const void *q,
                                float scale, void *out, int32_t num_ctas,
                                void *workspace, uint64_t workspace_bytes,
                                kv_stream_t stream);
+
+/* Phase 1 of paged_attn_decode_append alone: the attention kernel with the
+ * new token's rows written as it streams the cache. Arguments as
+ * paged_attn_decode_append; paged_attn_merge completes it. */
+kv_status paged_attn_partition_append(kv_pool *pool, int32_t layer, const void *q,
+                                      const void *k_new, const void *v_new,
+                                      int32_t q_dtype, int32_t num_seqs,
+                                      int32_t num_q_heads,
+                                      const int32_t *block_tables,
+                                      int32_t max_blocks_per_seq,
+                                      const int32_t *context_lens,
+                                      int32_t max_context, float scale, void *out,
+                                      int32_t num_ctas, void *workspace,
+                                      uint64_t workspace_bytes, kv_stream_t stream);
 
 /* Phase 2 alone: merge split units into out (out_dtype) and write zeros for
  * empty or invalid sequences. Must follow phase 1 with the same arguments. */

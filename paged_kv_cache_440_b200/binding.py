@@ -69,6 +69,10 @@ _SIGS = {
                           _P, _U64, _P],
     "paged_attn_partition": [_P, _I32, _P, _I32, _I32, _I32, _P, _I32, _P, _I32, _F, _P,
                              _I32, _P, _U64, _P],
+    "paged_attn_decode_append": [_P, _I32, _P, _P, _P, _I32, _I32, _I32, _P, _I32, _P, _I32, _F,
+                                 _P, _I32, _P, _U64, _P],
+    "paged_attn_partition_append": [_P, _I32, _P, _P, _P, _I32, _I32, _I32, _P, _I32, _P, _I32,
+                                    _F, _P, _I32, _P, _U64, _P],
     "paged_attn_merge": [_P, _I32, _I32, _P, _I32, _I32, _I32, _I32, _P, _P, _U64, _P],
     "kv_selftest_wait_timeout": [_P, ctypes.c_uint32, _P],
     "paged_attn_decode_static": [_P, _I32, _P, _I32, _I32, _I32, _P, _I32, _P, _I32, _F, _P,
@@ -326,6 +330,26 @@ def paged_attn_decode_static(pool, layer, q, block_tables, context_lens, max_con
     return out
 
 
+def paged_attn_decode_append(pool, layer, q, k_new, v_new, block_tables, context_lens,
+                             max_context, scale, out=None, num_ctas=0, workspace=None,
+                             stream=None):
+    """Write each sequence's new token (k_new, v_new [B, Hkv, D]) at position
+    L - 1 and attend q over the cache including it, in one attention kernel."""
+    B, Hq, out = _attn_args(pool, q, block_tables, context_lens, out)
+    _need(k_new, "k_new", q.dtype, pool.device)
+    _need(v_new, "v_new", q.dtype, pool.device)
+    if tuple(k_new.shape) != (B, pool.num_kv_heads, pool.head_dim) or v_new.shape != k_new.shape:
+        raise ValueError("k_new, v_new must be [B, kv_heads, head_dim]")
+    if workspace is None:
+        workspace = make_workspace(pool, B, Hq, num_ctas)
+    check(lib.paged_attn_decode_append(pool.handle, layer, _ptr(q), _ptr(k_new), _ptr(v_new),
+                                       TORCH_CODES[q.dtype], B, Hq, _ptr(block_tables),
+                                       block_tables.shape[1], _ptr(context_lens), max_context,
+                                       float(scale), _ptr(out), num_ctas, _ptr(workspace),
+                                       workspace.numel(), _stream(stream, pool.device)))
+    return out
+
+
 def paged_attn_partition(pool, layer, q, block_tables, context_lens, max_context, scale,
                          out, workspace, num_ctas=0, stream=None):
     B, Hq, out = _attn_args(pool, q, block_tables, context_lens, out)
@@ -334,6 +358,21 @@ def paged_attn_partition(pool, layer, q, block_tables, context_lens, max_context
                                    _ptr(context_lens), max_context, float(scale), _ptr(out),
                                    num_ctas, _ptr(workspace), workspace.numel(),
                                    _stream(stream, pool.device)))
+    return out
+
+
+def paged_attn_partition_append(pool, layer, q, k_new, v_new, block_tables, context_lens,
+                                max_context, scale, out, workspace, num_ctas=0, stream=None):
+    B, Hq, out = _attn_args(pool, q, block_tables, context_lens, out)
+    _need(k_new, "k_new", q.dtype, pool.device)
+    _need(v_new, "v_new", q.dtype, pool.device)
+    if tuple(k_new.shape) != (B, pool.num_kv_heads, pool.head_dim) or v_new.shape != k_new.shape:
+        raise ValueError("k_new, v_new must be [B, kv_heads, head_dim]")
+    check(lib.paged_attn_partition_append(pool.handle, layer, _ptr(q), _ptr(k_new), _ptr(v_new),
+                                          TORCH_CODES[q.dtype], B, Hq, _ptr(block_tables),
+                                          block_tables.shape[1], _ptr(context_lens), max_context,
+                                          float(scale), _ptr(out), num_ctas, _ptr(workspace),
+                                          workspace.numel(), _stream(stream, pool.device)))
     return out
 
 

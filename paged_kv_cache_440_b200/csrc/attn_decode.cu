@@ -73,6 +73,14 @@ struct AttnParams {
   float *part_ml;  // [num_ctas][2][kNC][8][2]   their (max, sum), base 2
   int4 *meta;      // [num_seqs * units_per_seq]: first CTA, #CTAs, first side
   int *status;
+  // fused append (paged_attn_decode_append): each sequence's new token, written
+  // at position L - 1 before it is attended; null when not fused
+  const void *k_new;  // [num_seqs][kv_heads][D], the query dtype
+  const void *v_new;
+  char *k_cache;      // the layer's K / V regions and scales, for the writes
+  char *v_cache;
+  float *k_scale_w;
+  float *v_scale_w;
   float scale_log2;  // scale * log2(e)
   int num_seqs;
   int q_heads;
@@ -721,6 +729,81 @@ struct Consumer {
   }
 };
 
+// The new token's K and V rows for one kv head, as this lane's share: lane l
+// holds elements l * D/32 .. of the row (16-bit bits, or codes and scales).
+template <int D, int BS, int KV_T, int Q_T>
+struct NewRow {
+  static constexpr int E = D / 32;
+  static constexpr bool kQuant = !is16<KV_T>();
+  uint32_t k[2], v[2];  // 16-bit: E * 2 bytes; 1-byte: E codes in k[0] / v[0]
+  float ks, vs;
+
+  __device__ __forceinline__ void load(const AttnParams &p, int b, int g, int lane) {
+    const int64_t row = (static_cast<int64_t>(b) * p.kv_heads + g) * D;
+    const uint16_t *kn = static_cast<const uint16_t *>(p.k_new) + row;
+    const uint16_t *vn = static_cast<const uint16_t *>(p.v_new) + row;
+    if constexpr (!kQuant) {
+      if constexpr (E == 4) {
+        const uint2 a = *reinterpret_cast<const uint2 *>(kn + lane * 4);
+        const uint2 c = *reinterpret_cast<const uint2 *>(vn + lane * 4);
+        k[0] = a.x; k[1] = a.y; v[0] = c.x; v[1] = c.y;
+      } else {
+        k[0] = *reinterpret_cast<const uint32_t *>(kn + lane * 2);
+        v[0] = *reinterpret_cast<const uint32_t *>(vn + lane * 2);
+        k[1] = v[1] = 0u;
+      }
+    } else {
+      float x[E];
+      load_row<D, Q_T>(kn, lane, x);
+      k[0] = quantize_row<D, KV_T>(x, &ks);
+      load_row<D, Q_T>(vn, lane, x);
+      v[0] = quantize_row<D, KV_T>(x, &vs);
+      k[1] = v[1] = 0u;
+    }
+  }
+
+  // Put the row in the stage (row r0 + rl of the stage's K / V parts, where the
+  // load brought whatever the pool held) and in the pool (block id, head g).
+  __device__ __forceinline__ void store(const AttnParams &p, uint8_t *st, int rows, int r, int id,
+                                        int g, int rl, int lane) const {
+    using T = Tile<D, BS, KV_T>;
+    const uint32_t ktile = smem_u32(st);
+    const uint32_t vtile = ktile + rows * T::kRowBytes;
+    const uint32_t off = lane * E * T::kElt;  // this lane's bytes within the row
+    const uint32_t ka = T::chunk(ktile, r, off >> 4, rows) + (off & 15);
+    const uint32_t va = T::chunk(vtile, r, off >> 4, rows) + (off & 15);
+    const int64_t grow = (static_cast<int64_t>(id) * p.kv_heads + g) * BS + rl;
+    char *kg = p.k_cache + grow * T::kRowBytes + off;
+    char *vg = p.v_cache + grow * T::kRowBytes + off;
+    constexpr int kBytes = E * T::kElt;
+    if constexpr (kBytes == 8) {
+      asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(ka), "r"(k[0]), "r"(k[1]) : "memory");
+      asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(va), "r"(v[0]), "r"(v[1]) : "memory");
+      *reinterpret_cast<uint2 *>(kg) = make_uint2(k[0], k[1]);
+      *reinterpret_cast<uint2 *>(vg) = make_uint2(v[0], v[1]);
+    } else if constexpr (kBytes == 4) {
+      asm volatile("st.shared.u32 [%0], %1;" ::"r"(ka), "r"(k[0]) : "memory");
+      asm volatile("st.shared.u32 [%0], %1;" ::"r"(va), "r"(v[0]) : "memory");
+      *reinterpret_cast<uint32_t *>(kg) = k[0];
+      *reinterpret_cast<uint32_t *>(vg) = v[0];
+    } else {
+      asm volatile("st.shared.u16 [%0], %1;" ::"r"(ka), "h"(static_cast<uint16_t>(k[0])) : "memory");
+      asm volatile("st.shared.u16 [%0], %1;" ::"r"(va), "h"(static_cast<uint16_t>(v[0])) : "memory");
+      *reinterpret_cast<uint16_t *>(kg) = static_cast<uint16_t>(k[0]);
+      *reinterpret_cast<uint16_t *>(vg) = static_cast<uint16_t>(v[0]);
+    }
+    if constexpr (kQuant) {
+      if (lane == 0) {
+        float *sc = reinterpret_cast<float *>(st + 2 * rows * T::kRowBytes);
+        sc[r] = ks;
+        sc[rows + r] = vs;
+        p.k_scale_w[grow] = ks;
+        p.v_scale_w[grow] = vs;
+      }
+    }
+  }
+};
+
 // Position of a CTA's walk over the flattened (unit, block) list.
 struct Walk {
   int b;         // sequence
@@ -912,6 +995,13 @@ attn_partition_kernel(const __grid_constant__ CUtensorMap kmap,
     const int h0 = g * p.group + chunk * kChunkHeads;
     const int nh = MMA ? min(kChunkHeads, p.group - chunk * kChunkHeads) : 1;
     const int L = p.context_lens[w.b];
+    // fused append: the new token (position L - 1) is in block jl of the unit;
+    // with one query-head chunk per kv head this warp alone uses its rows
+    const int jl = (L - 1) / BS;
+    const bool has_new =
+        p.k_new != nullptr && active && L > 0 && jl >= w.j && jl < w.j + seg;
+    NewRow<D, BS, KV_T, Q_T> nr;
+    if (has_new) nr.load(p, w.b, g, lane);
     if (active) {
       cs.reset();
       cs.load_query(p, w.b, h0, nh, lane);
@@ -931,6 +1021,13 @@ attn_partition_kernel(const __grid_constant__ CUtensorMap kmap,
           const int jb = w.j + static_cast<int>(kk - k);
           const int id = stage_id[s];
           const int valid = id >= 0 ? min(BS, L - jb * BS) : 0;
+          if (has_new && jb == jl && id >= 0) {
+            const int rl = (L - 1) - jl * BS;
+            nr.store(p, ring + s * stride, rows, hi * BS + rl, id, g, rl, lane);
+            // the producer's next TMA into this stage must come after these writes
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+          }
           cs.block(ring + s * stride, rows, hi, valid, lane);
         }
         __syncwarp();
@@ -1226,7 +1323,8 @@ kv_status run_partition(kv_pool *pool, int32_t layer, const void *q, int32_t q_d
                         int32_t num_seqs, int32_t num_q_heads, const int32_t *block_tables,
                         int32_t max_blocks_per_seq, const int32_t *context_lens,
                         int32_t max_context, float scale, void *out, int32_t num_ctas,
-                        void *workspace, uint64_t workspace_bytes, cudaStream_t st) {
+                        void *workspace, uint64_t workspace_bytes, const void *k_new,
+                        const void *v_new, cudaStream_t st) {
   if (!pool) return fail(KV_ERR_INVALID, "null pool");
   if (layer < 0 || layer >= pool->d.num_layers) return fail(KV_ERR_INVALID, "layer %d out of range", layer);
   const int cd = pool->d.cache_dtype;
@@ -1250,6 +1348,21 @@ kv_status run_partition(kv_pool *pool, int32_t layer, const void *q, int32_t q_d
   s = fill_params(pool, layer, q, num_seqs, num_q_heads, block_tables, max_blocks_per_seq,
                   context_lens, max_context, scale, out, G, workspace, workspace_bytes, &p);
   if (s != KV_OK) return s;
+  if (k_new || v_new) {
+    if (!k_new || !v_new) return fail(KV_ERR_INVALID, "k_new and v_new go together");
+    if ((reinterpret_cast<uintptr_t>(k_new) & 15) || (reinterpret_cast<uintptr_t>(v_new) & 15))
+      return fail(KV_ERR_INVALID, "k_new and v_new must be 16-byte aligned");
+    if (p.cpg != 1)
+      return fail(KV_ERR_UNSUPPORTED,
+                  "the fused append supports up to 8 query heads per kv head; use kv_append "
+                  "and paged_attn_decode");
+    p.k_new = k_new;
+    p.v_new = v_new;
+    p.k_cache = layer_k(pool, layer);
+    p.v_cache = layer_v(pool, layer);
+    p.k_scale_w = layer_ks(pool, layer);
+    p.v_scale_w = layer_vs(pool, layer);
+  }
   if (num_seqs == 0) return KV_OK;
   kv_status code;
   const LayerMaps *maps = layer_maps(pool, layer, p.hg * pool->d.block_size, &code);
@@ -1313,7 +1426,21 @@ kv_status paged_attn_partition(kv_pool *pool, int32_t layer, const void *q, int3
                                void *workspace, uint64_t workspace_bytes, kv_stream_t stream) {
   kv_status s = run_partition(pool, layer, q, q_dtype, num_seqs, num_q_heads, block_tables,
                               max_blocks_per_seq, context_lens, max_context, scale, out, num_ctas,
-                              workspace, workspace_bytes, (cudaStream_t)stream);
+                              workspace, workspace_bytes, nullptr, nullptr, (cudaStream_t)stream);
+  return s == KV_OK ? ok() : s;
+}
+
+kv_status paged_attn_partition_append(kv_pool *pool, int32_t layer, const void *q,
+                                      const void *k_new, const void *v_new, int32_t q_dtype,
+                                      int32_t num_seqs, int32_t num_q_heads,
+                                      const int32_t *block_tables, int32_t max_blocks_per_seq,
+                                      const int32_t *context_lens, int32_t max_context,
+                                      float scale, void *out, int32_t num_ctas, void *workspace,
+                                      uint64_t workspace_bytes, kv_stream_t stream) {
+  if (num_seqs > 0 && (!k_new || !v_new)) return fail(KV_ERR_INVALID, "null k_new / v_new");
+  kv_status s = run_partition(pool, layer, q, q_dtype, num_seqs, num_q_heads, block_tables,
+                              max_blocks_per_seq, context_lens, max_context, scale, out, num_ctas,
+                              workspace, workspace_bytes, k_new, v_new, (cudaStream_t)stream);
   return s == KV_OK ? ok() : s;
 }
 
@@ -1334,7 +1461,27 @@ kv_status paged_attn_decode(kv_pool *pool, int32_t layer, const void *q, int32_t
                             void *workspace, uint64_t workspace_bytes, kv_stream_t stream) {
   kv_status s = run_partition(pool, layer, q, q_dtype, num_seqs, num_q_heads, block_tables,
                               max_blocks_per_seq, context_lens, max_context, scale, out, num_ctas,
-                              workspace, workspace_bytes, (cudaStream_t)stream);
+                              workspace, workspace_bytes, nullptr, nullptr, (cudaStream_t)stream);
+  if (s != KV_OK) return s;
+  if (num_seqs > 0) {
+    s = run_merge(pool, num_seqs, num_q_heads, context_lens, max_blocks_per_seq, max_context,
+                  num_ctas, q_dtype, out, workspace, workspace_bytes, (cudaStream_t)stream);
+    if (s != KV_OK) return s;
+  }
+  return ok();
+}
+
+kv_status paged_attn_decode_append(kv_pool *pool, int32_t layer, const void *q,
+                                   const void *k_new, const void *v_new, int32_t q_dtype,
+                                   int32_t num_seqs, int32_t num_q_heads,
+                                   const int32_t *block_tables, int32_t max_blocks_per_seq,
+                                   const int32_t *context_lens, int32_t max_context, float scale,
+                                   void *out, int32_t num_ctas, void *workspace,
+                                   uint64_t workspace_bytes, kv_stream_t stream) {
+  if (num_seqs > 0 && (!k_new || !v_new)) return fail(KV_ERR_INVALID, "null k_new / v_new");
+  kv_status s = run_partition(pool, layer, q, q_dtype, num_seqs, num_q_heads, block_tables,
+                              max_blocks_per_seq, context_lens, max_context, scale, out, num_ctas,
+                              workspace, workspace_bytes, k_new, v_new, (cudaStream_t)stream);
   if (s != KV_OK) return s;
   if (num_seqs > 0) {
     s = run_merge(pool, num_seqs, num_q_heads, context_lens, max_blocks_per_seq, max_context,

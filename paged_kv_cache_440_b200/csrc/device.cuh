@@ -10,6 +10,8 @@
 #include <cuda_fp8.h>
 #include <cstdint>
 
+#include "pagedkv.h"
+
 namespace pagedkv {
 namespace dev {
 
@@ -226,6 +228,79 @@ __device__ __forceinline__ uint32_t int8_pair(uint32_t src_biased) {
   const __half2 bias = __halves2half2(__ushort_as_half(0x6480), __ushort_as_half(0x6480));
   v = __hsub2(v, bias);
   return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// ------------------------------------------------ per-row KV quantization
+// One warp handles one row of D values, lane l holding elements
+// l * D/32 .. l * D/32 + D/32 - 1 (used by the append kernel and by the
+// attention kernel's fused append, so both produce the same bytes).
+
+template <int IN_T>
+__device__ __forceinline__ float to_f32(uint16_t bits) {
+  if constexpr (IN_T == KV_BF16) {
+    return __uint_as_float(static_cast<uint32_t>(bits) << 16);
+  } else {
+    return __half2float(__ushort_as_half(bits));
+  }
+}
+
+// Quantize one row of D values held as D/32 per lane; returns the packed codes
+// of this lane (D/32 bytes, little-endian in order) and the row scale.
+template <int D, int OUT_T>
+__device__ __forceinline__ uint32_t quantize_row(const float (&x)[D / 32], float *scale_out) {
+  constexpr int E = D / 32;
+  float a = 0.f;
+#pragma unroll
+  for (int i = 0; i < E; ++i) a = fmaxf(a, fabsf(x[i]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+  constexpr float kQmax = OUT_T == KV_INT8 ? 127.0f : 57344.0f;
+  uint32_t packed = 0;
+  float scale = 0.f;
+  if (a > 0.f) {
+    scale = __fdiv_rn(a, kQmax);
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+      const float y = __fdiv_rn(x[i], scale);
+      uint32_t code;
+      if constexpr (OUT_T == KV_INT8) {
+        int q = __float2int_rn(y);
+        q = max(-127, min(127, q));
+        code = static_cast<uint32_t>(q) & 0xFFu;
+      } else {
+        code = static_cast<uint32_t>(__nv_cvt_float_to_fp8(y, __NV_SATFINITE, __NV_E5M2));
+      }
+      packed |= code << (8 * i);
+    }
+  }
+  *scale_out = scale;
+  return packed;
+}
+
+template <int D, int IN_T>
+__device__ __forceinline__ void load_row(const uint16_t *__restrict__ src, int lane,
+                                         float (&x)[D / 32]) {
+  constexpr int E = D / 32;
+  if constexpr (E == 4) {
+    uint2 v = *reinterpret_cast<const uint2 *>(src + lane * 4);
+    x[0] = to_f32<IN_T>(v.x & 0xFFFF);
+    x[1] = to_f32<IN_T>(v.x >> 16);
+    x[2] = to_f32<IN_T>(v.y & 0xFFFF);
+    x[3] = to_f32<IN_T>(v.y >> 16);
+  } else {
+    uint32_t v = *reinterpret_cast<const uint32_t *>(src + lane * 2);
+    x[0] = to_f32<IN_T>(v & 0xFFFF);
+    x[1] = to_f32<IN_T>(v >> 16);
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void store_codes(uint8_t *dst, int lane, uint32_t packed) {
+  if constexpr (D == 128) {
+    reinterpret_cast<uint32_t *>(dst)[lane] = packed;
+  } else {
+    reinterpret_cast<uint16_t *>(dst)[lane] = static_cast<uint16_t>(packed);
+  }
 }
 
 }  // namespace dev

@@ -45,13 +45,14 @@ def build_pool(pkv, wl, device, chunk=65536):
     for quantized caches (kv_append) and by a plain device copy for 16-bit ones."""
     pool = pkv.KVPool(1, wl.num_blocks, wl.block_size, wl.kv_heads, wl.head_dim,
                       wl.cache_dtype, device)
-    K, V, _, _ = pool.layer_views(0)
+    K, V, KS, VS = pool.layer_views(0)
     if wl.k_fill is not None:
         K.copy_(wl.k_fill)
         V.copy_(wl.v_fill)
     else:
-        K.zero_()
-        V.zero_()
+        # rows no append writes compare against the oracle's zeros
+        for t in (K, V, KS, VS):
+            t.zero_()
         slots = torch.from_numpy(wl.slot_hist).to(device)
         for s in range(0, wl.k_hist.shape[0], chunk):
             pkv.kv_append(pool, 0, wl.k_hist[s:s + chunk].contiguous(),

@@ -13,8 +13,9 @@ import pytest
 import torch
 
 import workloads as W
-from gpu_support import (build_pool, compare, device_inputs, oracle_cache_16,
+from gpu_support import (bits16, build_pool, compare, device_inputs, oracle_cache_16,
                          oracle_cache_quant, oracle_outputs, step, to_np)
+from oracle import cache_ops
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
@@ -248,3 +249,87 @@ def test_bad_block_id_and_length_are_reported(pkv):
     k, v = to_np(wl.k_fill), to_np(wl.v_fill)
     ref = oracle_outputs(wl, k, v, [(0, h) for h in range(8)])
     compare(out[0], ref, what="good sequence")
+
+
+# --------------------------------------------------------------- fused append
+
+def _fused_workloads():
+    return [
+        ("tiny", lambda: W.tiny(DEV)),
+        ("gqa70b-8", lambda: W.gqa70b(DEV, batch=8)),
+        ("mha-fp16", lambda: W.make_decode_workload("mha", 6, 4, 4, 128, 16, "fp16", "fp16",
+                                                    [1, 16, 17, 200, 31, 64], seed=3, device=DEV)),
+        ("g4-d64-bs32", lambda: W.make_decode_workload("g4", 5, 8, 2, 64, 32, "bf16", "bf16",
+                                                       [0, 1, 32, 33, 150], seed=4, device=DEV)),
+        ("int8", lambda: W.make_decode_workload("q8", 4, 16, 2, 128, 32, "bf16", "int8",
+                                                [1, 31, 32, 300], seed=5, device=DEV)),
+        ("e5m2", lambda: W.make_decode_workload("e5", 4, 16, 2, 128, 16, "bf16", "e5m2",
+                                                [2, 17, 64, 129], seed=6, device=DEV)),
+    ]
+
+
+@pytest.mark.parametrize("name,make", _fused_workloads())
+@pytest.mark.parametrize("num_ctas", [0, 7])
+def test_fused_append_matches_oracle(pkv, name, make, num_ctas):
+    """paged_attn_decode_append writes the step's token at position L - 1 (bit-
+    exact with the oracle's append / quantize) and attends over it."""
+    wl = make()
+    pool = build_pool(pkv, wl, DEV)
+    tables, lens = device_inputs(wl, DEV)
+    max_ctx = max(int(wl.context_lens.max()), 1)
+    out = pkv.paged_attn_decode_append(pool, 0, wl.q, wl.k_new, wl.v_new, tables, lens, max_ctx,
+                                       wl.scale, num_ctas=num_ctas)
+    torch.cuda.synchronize()
+    assert pool.status() == 0
+    pairs = _all_pairs(wl)
+    K, V, KS, VS = pool.layer_views(0)
+    if wl.cache_dtype in ("bf16", "fp16"):
+        k, v = oracle_cache_16(wl)
+        tab = None
+        kb, vb = bits16(wl.k_fill), bits16(wl.v_fill)
+        cache_ops.append(kb, vb, bits16(wl.k_new), bits16(wl.v_new), wl.slot_new, wl.block_size)
+        assert np.array_equal(bits16(K), kb) and np.array_equal(bits16(V), vb)
+    else:
+        (kc, vc, ks, vs), (k, v, tab) = oracle_cache_quant(wl, list(range(wl.batch)))
+        used = sorted({int(x) for b in range(wl.batch)
+                       for x in wl.block_tables[b, :-(-int(wl.context_lens[b]) // wl.block_size)]})
+        assert np.array_equal(K[used].cpu().numpy(), kc[used])
+        assert np.array_equal(V[used].cpu().numpy(), vc[used])
+        assert np.array_equal(KS[used].cpu().numpy().view(np.uint32), ks[used].view(np.uint32))
+        assert np.array_equal(VS[used].cpu().numpy().view(np.uint32), vs[used].view(np.uint32))
+    ref = oracle_outputs(wl, k, v, pairs, tab)
+    compare(torch.stack([out[b, h] for b, h in pairs]), ref, what="fused append " + name)
+
+
+def test_fused_append_rejects_more_than_8_heads_per_kv_head(pkv):
+    wl = W.make_decode_workload("g16", 2, 32, 2, 64, 16, "bf16", "bf16", [5, 9], seed=7,
+                                device=DEV)
+    pool = build_pool(pkv, wl, DEV)
+    tables, lens = device_inputs(wl, DEV)
+    with pytest.raises(pkv.PagedKVError) as e:
+        pkv.paged_attn_decode_append(pool, 0, wl.q, wl.k_new, wl.v_new, tables, lens, 9, wl.scale)
+    assert e.value.status == 4
+
+
+def test_fused_append_phases_equal_one_call(pkv):
+    """paged_attn_partition_append + paged_attn_merge gives the bits of
+    paged_attn_decode_append."""
+    wl = W.gqa70b(DEV, batch=6)
+    tables, lens = device_inputs(wl, DEV)
+    max_ctx = int(wl.context_lens.max())
+    outs = []
+    for phases in (False, True):
+        pool = build_pool(pkv, wl, DEV)
+        if phases:
+            ws = pkv.make_workspace(pool, wl.batch, wl.q_heads, 11)
+            out = torch.empty_like(wl.q)
+            pkv.paged_attn_partition_append(pool, 0, wl.q, wl.k_new, wl.v_new, tables, lens,
+                                            max_ctx, wl.scale, out, ws, num_ctas=11)
+            pkv.paged_attn_merge(pool, lens, tables.shape[1], max_ctx, out, ws, num_ctas=11)
+        else:
+            out = pkv.paged_attn_decode_append(pool, 0, wl.q, wl.k_new, wl.v_new, tables, lens,
+                                               max_ctx, wl.scale, num_ctas=11)
+        torch.cuda.synchronize()
+        outs.append((bits16(out), bits16(pool.layer_views(0)[0]), bits16(pool.layer_views(0)[1])))
+    for a, b in zip(*outs):
+        assert np.array_equal(a, b)
