@@ -77,6 +77,21 @@ def elt_bytes(cache):
     return 2 if cache in ("bf16", "fp16") else 1
 
 
+def max_over_ranks(values, world, device):
+    """Per-rank times -> the slowest rank's (every rank gets the same list)."""
+    if world == 1:
+        return list(values)
+    t = torch.tensor(values, device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
+def job_throughput(bytes_per_step, world, step_s):
+    """Whole-job GB/s: every rank (replica) moves bytes_per_step per step; the
+    job's step takes the slowest rank's time."""
+    return bytes_per_step * world / step_s / 1e9
+
+
 def step_bytes(wl):
     """Algorithmic bytes of one step: (decode kernel bytes, append bytes)."""
     e = elt_bytes(wl.cache_dtype)
@@ -278,10 +293,7 @@ def run_ours(args, rank, world, device):
     part_ms = np.array([a.elapsed_time(b) for a, b in kev])
     step_s = float(step_ms.mean()) / 1e3
     part_s = float(part_ms.mean()) / 1e3
-    if world > 1:
-        t = torch.tensor([step_s, part_s], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        step_s, part_s = float(t[0]), float(t[1])
+    step_s, part_s = max_over_ranks([step_s, part_s], world, device)
     clocks = sampler.summary(t0, t2)
 
     # ---------------------------------------------------------- end to end
@@ -319,10 +331,7 @@ def run_ours(args, rank, world, device):
             if i >= args.warmup:
                 times.append(a.elapsed_time(b_) / 1e3)
         e2e_s = float(np.mean(times))
-        if world > 1:
-            t = torch.tensor([e2e_s], device=device, dtype=torch.float64)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e2e_s = float(t[0])
+        e2e_s, = max_over_ranks([e2e_s], world, device)
         e2e = (e2e_s, h2d, d2h)
 
     dec_bytes, app_bytes = step_bytes(wl)
@@ -387,7 +396,7 @@ def main():
     r = run_ours(args, rank, world, device)
     wl = r["wl"]
     total_bytes = (r["dec_bytes"] + r["app_bytes"]) * world
-    gbs = total_bytes / r["step_s"] / 1e9
+    gbs = job_throughput(r["dec_bytes"] + r["app_bytes"], world, r["step_s"])
     peak, peak_kind = measured_peak()
     # the timed kernel's algorithmic bytes: the KV stream, q and out, plus the
     # new rows when the append is folded into it

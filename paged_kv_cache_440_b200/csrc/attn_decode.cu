@@ -1055,7 +1055,7 @@ attn_partition_kernel(const __grid_constant__ CUtensorMap kmap,
 // invalid sequences; combines the partials of units split across CTAs:
 // out = sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i, M = max_i m_i.
 // ============================================================================
-constexpr int kMergeWarps = 8;
+constexpr int kMergeWarps = 4;  // small CTAs: one fits beside a partition CTA
 
 template <int D, int OUT_T>
 __global__ void __launch_bounds__(kMergeWarps * 32) attn_merge_kernel(const AttnParams p) {
@@ -1105,32 +1105,36 @@ __global__ void __launch_bounds__(kMergeWarps * 32) attn_merge_kernel(const Attn
       v[0] = x.x; v[1] = x.y;
     }
   };
-  // one online pass: running max M, sum Ls and output acc; piece i + 1 is
-  // loaded while piece i is combined
+  // One online pass over the pieces in order: running max M, sum Ls and
+  // output acc. The loads of up to kBatch pieces are issued together, so a
+  // unit costs one round trip per kBatch pieces rather than one per piece.
+  constexpr int kBatch = 8;
   float M = -INFINITY, Ls = 0.f;
-  float acc[E], o[E], o_n[E];
+  float acc[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) acc[e] = 0.f;
-  float2 ml = *reinterpret_cast<const float2 *>(p.part_ml + rec(0) * 2);
-  load_o(0, o);
-  for (int i = 0; i < nu; ++i) {
-    float2 ml_n = ml;
-    if (i + 1 < nu) {
-      ml_n = *reinterpret_cast<const float2 *>(p.part_ml + rec(i + 1) * 2);
-      load_o(i + 1, o_n);
-    }
-    const float Mn = fmaxf(M, ml.x);
-    if (Mn != -INFINITY) {
-      const float a = exp2_rel(M, Mn), wt = exp2_rel(ml.x, Mn);
-      Ls = Ls * a + ml.y * wt;
+  for (int i0 = 0; i0 < nu; i0 += kBatch) {
+    float2 ml[kBatch];
+    float o[kBatch][E];
 #pragma unroll
-      for (int e = 0; e < E; ++e) acc[e] = acc[e] * a + o[e] * wt;
-      M = Mn;
+    for (int k = 0; k < kBatch; ++k) {
+      if (i0 + k < nu) {
+        ml[k] = *reinterpret_cast<const float2 *>(p.part_ml + rec(i0 + k) * 2);
+        load_o(i0 + k, o[k]);
+      }
     }
-    if (i + 1 < nu) {
-      ml = ml_n;
 #pragma unroll
-      for (int e = 0; e < E; ++e) o[e] = o_n[e];
+    for (int k = 0; k < kBatch; ++k) {
+      if (i0 + k < nu) {
+        const float Mn = fmaxf(M, ml[k].x);
+        if (Mn != -INFINITY) {
+          const float a = exp2_rel(M, Mn), wt = exp2_rel(ml[k].x, Mn);
+          Ls = Ls * a + ml[k].y * wt;
+#pragma unroll
+          for (int e = 0; e < E; ++e) acc[e] = acc[e] * a + o[k][e] * wt;
+          M = Mn;
+        }
+      }
     }
   }
   const float inv = Ls > 0.f ? 1.f / Ls : 0.f;

@@ -333,3 +333,34 @@ def test_fused_append_phases_equal_one_call(pkv):
         outs.append((bits16(out), bits16(pool.layer_views(0)[0]), bits16(pool.layer_views(0)[1])))
     for a, b in zip(*outs):
         assert np.array_equal(a, b)
+
+
+@pytest.mark.parametrize("name,make", _fused_workloads())
+@pytest.mark.parametrize("G", [3, 37, 0, 300])
+def test_decode_whatever_the_workspace_held(pkv, name, make, G):
+    """The split-K workspace needs no initialisation: paged_attn_decode gives
+    the bits of a first partition + merge whatever the workspace held before
+    (zeros, all ones, random bytes), and again on a second call with the same
+    workspace."""
+    wl = make()
+    pool = build_pool(pkv, wl, DEV)
+    tables, lens = device_inputs(wl, DEV)
+    pkv.kv_append(pool, 0, wl.k_new, wl.v_new, torch.from_numpy(wl.slot_new).to(DEV))
+    max_ctx = max(int(wl.context_lens.max()), 1)
+    ws = pkv.make_workspace(pool, wl.batch, wl.q_heads, G)
+    ref = torch.empty_like(wl.q)
+    pkv.paged_attn_partition(pool, 0, wl.q, tables, lens, max_ctx, wl.scale, ref, ws, num_ctas=G)
+    pkv.paged_attn_merge(pool, lens, tables.shape[1], max_ctx, ref, ws, num_ctas=G)
+    gen = torch.Generator(device=DEV).manual_seed(G + 1)
+    fills = [lambda: ws.zero_(), lambda: ws.fill_(255),
+             lambda: ws.copy_(torch.randint(0, 256, ws.shape, generator=gen, device=DEV,
+                                            dtype=torch.int32).to(torch.uint8))]
+    for fill in fills:
+        fill()
+        for _ in range(2):
+            out = torch.full_like(wl.q, float("nan"))
+            pkv.paged_attn_decode(pool, 0, wl.q, tables, lens, max_ctx, wl.scale, out=out,
+                                  num_ctas=G, workspace=ws)
+            torch.cuda.synchronize()
+            assert np.array_equal(bits16(out), bits16(ref)), name
+    assert pool.status() == 0
