@@ -30,16 +30,14 @@
 //   own one (KV head, query-head chunk) of the unit and keep its online
 //   softmax state in registers across the unit's blocks; full/empty
 //   mbarriers link producer and consumers, every wait has a time limit.
-// * GQA groups (Hq / Hkv >= 2) make q K^T a dense [16 tokens x 128] x
-//   [128 x 8 heads] tile: warp-level tensor-core MMA (m16n8k16) with tokens as
-//   M and up to 8 query heads as N. P V runs as V^T P^T with head_dim as M,
-//   the probabilities turned from accumulator to operand layout by an
+// * q K^T for the query heads of one KV head is a [16 tokens x head_dim] x
+//   [head_dim x 8 heads] tile: warp-level tensor-core MMA (m16n8k16) with
+//   tokens as M and up to 8 query heads as N (MHA uses one of the 8 columns:
+//   the tensor pipe is otherwise idle, and one MMA replaces the CUDA-core
+//   dot products and their reductions). P V runs as V^T P^T with head_dim as
+//   M, the probabilities turned from accumulator to operand layout by an
 //   in-register 8x8 transpose and fed as two 16-bit parts (hi + lo) so P V
 //   keeps fp32-level accuracy. Online softmax in fp32 (base 2) per head.
-// * MHA (one query head per KV head) is a matrix-vector product; it stays on
-//   CUDA cores: each half-warp covers one token row (16 lanes x head_dim/16
-//   values), partial dot products are reduced with a butterfly that leaves
-//   one token's score per lane.
 // * INT8 / E5M2 codes convert exactly to fp16 in registers; per-token K scales
 //   multiply the scores, per-token V scales are folded into the softmax
 //   weights through log2(scale) so the fp16 weights stay within (0, 1].
@@ -188,41 +186,6 @@ __device__ __forceinline__ void store_out(void *out, int64_t idx, float v) {
   else static_cast<__half *>(out)[idx] = __float2half_rn(v);
 }
 
-// Load E consecutive cache values from shared memory (address in the shared
-// window) and widen them to fp32. 1-byte codes are returned as their values
-// (the per-token scale is applied by the caller).
-template <int KV_T, int E>
-__device__ __forceinline__ void load_vals(uint32_t addr, float (&v)[E]) {
-  constexpr int kBytes = E * (is16<KV_T>() ? 2 : 1);
-  uint32_t w[4] = {0u, 0u, 0u, 0u};
-  if constexpr (kBytes == 16) {
-    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
-                 : "r"(addr));
-  } else if constexpr (kBytes == 8) {
-    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(w[0]), "=r"(w[1]) : "r"(addr));
-  } else {
-    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w[0]) : "r"(addr));
-  }
-#pragma unroll
-  for (int e = 0; e < E; ++e) {
-    if constexpr (KV_T == KV_BF16) {
-      const uint32_t x = w[e >> 1];
-      v[e] = __uint_as_float((e & 1) ? (x & 0xFFFF0000u) : (x << 16));
-    } else if constexpr (KV_T == KV_FP16) {
-      const uint32_t x = w[e >> 1];
-      v[e] = __half2float(__ushort_as_half(static_cast<uint16_t>((e & 1) ? (x >> 16) : x)));
-    } else if constexpr (KV_T == KV_INT8) {
-      const int32_t x = static_cast<int32_t>(w[e >> 2]);
-      v[e] = static_cast<float>((x << (24 - 8 * (e & 3))) >> 24);
-    } else {
-      const uint32_t byte = (w[e >> 2] >> (8 * (e & 3))) & 0xFFu;
-      v[e] = __half2float(__ushort_as_half(static_cast<uint16_t>(byte << 8)));
-    }
-  }
-}
-
-
 // KV blocks of sequence b; 0 for an empty or invalid length.
 template <int BS>
 __device__ __forceinline__ int seq_blocks(const AttnParams &p, int b) {
@@ -299,88 +262,72 @@ __device__ __forceinline__ bool ring_wait(uint64_t *bar, uint32_t parity, volati
 // ============================================================================
 // Consumer: per-warp state and the work on one staged block.
 // ============================================================================
-template <int D, int BS, int KV_T, int Q_T, bool MMA>
+template <int D, int BS, int KV_T, int Q_T>
 struct Consumer {
   using T = Tile<D, BS, KV_T>;
   static constexpr bool kQuant = T::kQuant;
   static constexpr bool kBF = (KV_T == KV_BF16);  // MMA operand type (bf16, else fp16)
   static constexpr int KS = D / 16;  // k-steps over head_dim
   static constexpr int MT = BS / 16;  // 16-token tiles per block
-  static constexpr int E = D / 16;  // values per lane in a half-warp row (scalar path)
 
   float m_run[2], m2_run[2], l_run[2];
-  float oacc[MMA ? D / 16 : 1][4];
-  float oacc_s[MMA ? 1 : E];
-  uint32_t qb[MMA ? KS : 1][2];
-  float qs[MMA ? 1 : E];
+  float oacc[D / 16][4];
+  uint32_t qb[KS][2];
   float s_fac[2];
 
   __device__ __forceinline__ void reset() {
     m_run[0] = m_run[1] = m2_run[0] = m2_run[1] = -INFINITY;
     l_run[0] = l_run[1] = 0.f;
-    if constexpr (MMA) {
 #pragma unroll
-      for (int i = 0; i < D / 16; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
-    } else {
-#pragma unroll
-      for (int e = 0; e < E; ++e) oacc_s[e] = 0.f;
-    }
+    for (int i = 0; i < D / 16; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
   }
 
   // Query fragments of heads h0 .. h0 + nh - 1 of sequence b.
   __device__ __forceinline__ void load_query(const AttnParams &p, int b, int h0, int nh, int lane) {
     const int gq = lane >> 2, cq = lane & 3;
     s_fac[0] = s_fac[1] = p.scale_log2;
-    if constexpr (MMA) {
-      const bool hv = gq < nh;
-      const int64_t qrow = (static_cast<int64_t>(b) * p.q_heads + h0 + gq) * D;
-      if constexpr (!kQuant) {
-        // B operand: k = head_dim index, n = head. Lane (gq, cq) holds dims
-        // 16ks + 2cq, +1 and 16ks + 8 + 2cq, +1 of head gq.
-        const uint32_t *q32 = static_cast<const uint32_t *>(p.q);
+    const bool hv = gq < nh;
+    const int64_t qrow = (static_cast<int64_t>(b) * p.q_heads + h0 + gq) * D;
+    if constexpr (!kQuant) {
+      // B operand: k = head_dim index, n = head. Lane (gq, cq) holds dims
+      // 16ks + 2cq, +1 and 16ks + 8 + 2cq, +1 of head gq.
+      const uint32_t *q32 = static_cast<const uint32_t *>(p.q);
 #pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-          qb[ks][0] = hv ? q32[(qrow + 16 * ks + 2 * cq) >> 1] : 0u;
-          qb[ks][1] = hv ? q32[(qrow + 16 * ks + 8 + 2 * cq) >> 1] : 0u;
-        }
-      } else {
-        // fp16 operands: q scaled per head by a power of two so its largest
-        // magnitude is in [2^14, 2^15) (exact), the scale folded into s_fac.
-        // k-slot order matches the code fragments: lane (gq, cq) holds dims
-        // 16ks + 4cq .. 16ks + 4cq + 3.
-        float qv[KS][4];
-        float amax = 0.f;
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            qv[ks][e] = hv ? load_q<Q_T>(p.q, qrow + 16 * ks + 4 * cq + e) : 0.f;
-            amax = fmaxf(amax, fabsf(qv[ks][e]));
-          }
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-        int ex = 0;
-        if (amax > 0.f) {
-          frexpf(amax, &ex);
-          ex = 15 - ex;  // amax * 2^ex in [2^14, 2^15)
-        }
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-          qb[ks][0] = pack2<false>(ldexpf(qv[ks][0], ex), ldexpf(qv[ks][1], ex));
-          qb[ks][1] = pack2<false>(ldexpf(qv[ks][2], ex), ldexpf(qv[ks][3], ex));
-        }
-        // the score columns of this lane are heads 2cq and 2cq+1
-        const int ex0 = __shfl_sync(0xffffffffu, ex, (2 * cq) * 4);
-        const int ex1 = __shfl_sync(0xffffffffu, ex, (2 * cq + 1) * 4);
-        s_fac[0] = ldexpf(p.scale_log2, -ex0);
-        s_fac[1] = ldexpf(p.scale_log2, -ex1);
+      for (int ks = 0; ks < KS; ++ks) {
+        qb[ks][0] = hv ? q32[(qrow + 16 * ks + 2 * cq) >> 1] : 0u;
+        qb[ks][1] = hv ? q32[(qrow + 16 * ks + 8 + 2 * cq) >> 1] : 0u;
       }
     } else {
-      const int jl = lane & 15;
+      // fp16 operands: q scaled per head by a power of two so its largest
+      // magnitude is in [2^14, 2^15) (exact), the scale folded into s_fac.
+      // k-slot order matches the code fragments: lane (gq, cq) holds dims
+      // 16ks + 4cq .. 16ks + 4cq + 3.
+      float qv[KS][4];
+      float amax = 0.f;
 #pragma unroll
-      for (int e = 0; e < E; ++e)
-        qs[e] = load_q<Q_T>(p.q, (static_cast<int64_t>(b) * p.q_heads + h0) * D + jl * E + e) *
-                p.scale_log2;
+      for (int ks = 0; ks < KS; ++ks)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          qv[ks][e] = hv ? load_q<Q_T>(p.q, qrow + 16 * ks + 4 * cq + e) : 0.f;
+          amax = fmaxf(amax, fabsf(qv[ks][e]));
+        }
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+      int ex = 0;
+      if (amax > 0.f) {
+        frexpf(amax, &ex);
+        ex = 15 - ex;  // amax * 2^ex in [2^14, 2^15)
+      }
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        qb[ks][0] = pack2<false>(ldexpf(qv[ks][0], ex), ldexpf(qv[ks][1], ex));
+        qb[ks][1] = pack2<false>(ldexpf(qv[ks][2], ex), ldexpf(qv[ks][3], ex));
+      }
+      // the score columns of this lane are heads 2cq and 2cq+1
+      const int ex0 = __shfl_sync(0xffffffffu, ex, (2 * cq) * 4);
+      const int ex1 = __shfl_sync(0xffffffffu, ex, (2 * cq + 1) * 4);
+      s_fac[0] = ldexpf(p.scale_log2, -ex0);
+      s_fac[1] = ldexpf(p.scale_log2, -ex1);
     }
   }
 
@@ -393,257 +340,190 @@ struct Consumer {
     const float *ksc = reinterpret_cast<const float *>(st + 2 * rows * T::kRowBytes) + r0;
     const float *vsc = ksc + rows;
     const int gq = lane >> 2, cq = lane & 3;
-    if constexpr (MMA) {
-      // ---------------------------------------------------- scores S = K q
-      float sc[MT][4];
+    // ---------------------------------------------------- scores S = K q
+    float sc[MT][4];
 #pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        const int row = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-        if constexpr (!kQuant) {
-#pragma unroll
-          for (int ks = 0; ks < KS; ++ks) {
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4(T::chunk(ktile, r0 + row, 2 * ks + (lane >> 4), rows), a0, a1, a2, a3);
-            mma16816<kBF>(acc, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
-          }
-        } else {
-#pragma unroll
-          for (int kp = 0; kp < KS / 2; ++kp) {
-            uint32_t q0, q1, q2, q3;  // byte matrices: rows 0-7 / 8-15 x chunks 2kp, 2kp+1
-            ldsm_x4(T::chunk(ktile, r0 + row, 2 * kp + (lane >> 4), rows), q0, q1, q2, q3);
-            if constexpr (KV_T == KV_INT8) {
-              q0 ^= 0x80808080u; q1 ^= 0x80808080u; q2 ^= 0x80808080u; q3 ^= 0x80808080u;
-              mma16816<false>(acc, int8_pair<0, 1>(q0), int8_pair<0, 1>(q1),
-                              int8_pair<2, 3>(q0), int8_pair<2, 3>(q1), qb[2 * kp][0],
-                              qb[2 * kp][1]);
-              mma16816<false>(acc, int8_pair<0, 1>(q2), int8_pair<0, 1>(q3),
-                              int8_pair<2, 3>(q2), int8_pair<2, 3>(q3), qb[2 * kp + 1][0],
-                              qb[2 * kp + 1][1]);
-            } else {
-              mma16816<false>(acc, e5m2_pair<0, 1>(q0), e5m2_pair<0, 1>(q1),
-                              e5m2_pair<2, 3>(q0), e5m2_pair<2, 3>(q1), qb[2 * kp][0],
-                              qb[2 * kp][1]);
-              mma16816<false>(acc, e5m2_pair<0, 1>(q2), e5m2_pair<0, 1>(q3),
-                              e5m2_pair<2, 3>(q2), e5m2_pair<2, 3>(q3), qb[2 * kp + 1][0],
-                              qb[2 * kp + 1][1]);
-            }
-          }
-        }
-        // acc: [0],[1] = token mt*16+gq, heads 2cq, 2cq+1; [2],[3] = token +8
-        const int t0 = mt * 16 + gq, t1 = t0 + 8;
-        float k0 = 1.f, k1 = 1.f;
-        if constexpr (kQuant) {
-          k0 = ksc[t0];
-          k1 = ksc[t1];
-        }
-        sc[mt][0] = t0 < valid ? acc[0] * s_fac[0] * k0 : -INFINITY;
-        sc[mt][1] = t0 < valid ? acc[1] * s_fac[1] * k0 : -INFINITY;
-        sc[mt][2] = t1 < valid ? acc[2] * s_fac[0] * k1 : -INFINITY;
-        sc[mt][3] = t1 < valid ? acc[3] * s_fac[1] * k1 : -INFINITY;
-      }
-      // ---------------------------------------------------- online softmax
-      float bm0 = -INFINITY, bm1 = -INFINITY;
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        bm0 = fmaxf(bm0, fmaxf(sc[mt][0], sc[mt][2]));
-        bm1 = fmaxf(bm1, fmaxf(sc[mt][1], sc[mt][3]));
-      }
-      bm0 = warp_max_xor(bm0, 4);
-      bm1 = warp_max_xor(bm1, 4);
-      const float mn0 = fmaxf(m_run[0], bm0), mn1 = fmaxf(m_run[1], bm1);
-      const float al0 = rescale(m_run[0], mn0), al1 = rescale(m_run[1], mn1);
-      m_run[0] = mn0;
-      m_run[1] = mn1;
-      float ls0 = 0.f, ls1 = 0.f;
-      // weights for P V: exp2(s - m) (16-bit), exp2(s + log2 sv - m2) (quant)
-      float w[MT][4];
-      float be0 = 1.f, be1 = 1.f;  // O rescale factors
+    for (int mt = 0; mt < MT; ++mt) {
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      const int row = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
       if constexpr (!kQuant) {
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          w[mt][0] = exp2_rel(sc[mt][0], mn0);
-          w[mt][1] = exp2_rel(sc[mt][1], mn1);
-          w[mt][2] = exp2_rel(sc[mt][2], mn0);
-          w[mt][3] = exp2_rel(sc[mt][3], mn1);
-          ls0 += w[mt][0] + w[mt][2];
-          ls1 += w[mt][1] + w[mt][3];
+        for (int ks = 0; ks < KS; ++ks) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(T::chunk(ktile, r0 + row, 2 * ks + (lane >> 4), rows), a0, a1, a2, a3);
+          mma16816<kBF>(acc, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
         }
-        be0 = al0;
-        be1 = al1;
       } else {
-        float y[MT][4];
-        float bn0 = -INFINITY, bn1 = -INFINITY;
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          const int t0 = mt * 16 + gq, t1 = t0 + 8;
-          const float lv0 = t0 < valid ? log2f(vsc[t0]) : -INFINITY;
-          const float lv1 = t1 < valid ? log2f(vsc[t1]) : -INFINITY;
-          y[mt][0] = sc[mt][0] + lv0;
-          y[mt][1] = sc[mt][1] + lv0;
-          y[mt][2] = sc[mt][2] + lv1;
-          y[mt][3] = sc[mt][3] + lv1;
-          bn0 = fmaxf(bn0, fmaxf(y[mt][0], y[mt][2]));
-          bn1 = fmaxf(bn1, fmaxf(y[mt][1], y[mt][3]));
-          ls0 += exp2_rel(sc[mt][0], mn0) + exp2_rel(sc[mt][2], mn0);
-          ls1 += exp2_rel(sc[mt][1], mn1) + exp2_rel(sc[mt][3], mn1);
-        }
-        bn0 = warp_max_xor(bn0, 4);
-        bn1 = warp_max_xor(bn1, 4);
-        const float n0 = fmaxf(m2_run[0], bn0), n1 = fmaxf(m2_run[1], bn1);
-        be0 = rescale(m2_run[0], n0);
-        be1 = rescale(m2_run[1], n1);
-        m2_run[0] = n0;
-        m2_run[1] = n1;
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          w[mt][0] = exp2_rel(y[mt][0], n0);
-          w[mt][1] = exp2_rel(y[mt][1], n1);
-          w[mt][2] = exp2_rel(y[mt][2], n0);
-          w[mt][3] = exp2_rel(y[mt][3], n1);
+        for (int kp = 0; kp < KS / 2; ++kp) {
+          uint32_t q0, q1, q2, q3;  // byte matrices: rows 0-7 / 8-15 x chunks 2kp, 2kp+1
+          ldsm_x4(T::chunk(ktile, r0 + row, 2 * kp + (lane >> 4), rows), q0, q1, q2, q3);
+          if constexpr (KV_T == KV_INT8) {
+            q0 ^= 0x80808080u; q1 ^= 0x80808080u; q2 ^= 0x80808080u; q3 ^= 0x80808080u;
+            mma16816<false>(acc, int8_pair<0, 1>(q0), int8_pair<0, 1>(q1),
+                            int8_pair<2, 3>(q0), int8_pair<2, 3>(q1), qb[2 * kp][0],
+                            qb[2 * kp][1]);
+            mma16816<false>(acc, int8_pair<0, 1>(q2), int8_pair<0, 1>(q3),
+                            int8_pair<2, 3>(q2), int8_pair<2, 3>(q3), qb[2 * kp + 1][0],
+                            qb[2 * kp + 1][1]);
+          } else {
+            mma16816<false>(acc, e5m2_pair<0, 1>(q0), e5m2_pair<0, 1>(q1),
+                            e5m2_pair<2, 3>(q0), e5m2_pair<2, 3>(q1), qb[2 * kp][0],
+                            qb[2 * kp][1]);
+            mma16816<false>(acc, e5m2_pair<0, 1>(q2), e5m2_pair<0, 1>(q3),
+                            e5m2_pair<2, 3>(q2), e5m2_pair<2, 3>(q3), qb[2 * kp + 1][0],
+                            qb[2 * kp + 1][1]);
+          }
         }
       }
-      l_run[0] = l_run[0] * al0 + ls0;
-      l_run[1] = l_run[1] * al1 + ls1;
-#pragma unroll
-      for (int dt = 0; dt < D / 16; ++dt) {
-        oacc[dt][0] *= be0;
-        oacc[dt][1] *= be1;
-        oacc[dt][2] *= be0;
-        oacc[dt][3] *= be1;
+      // acc: [0],[1] = token mt*16+gq, heads 2cq, 2cq+1; [2],[3] = token +8
+      const int t0 = mt * 16 + gq, t1 = t0 + 8;
+      float k0 = 1.f, k1 = 1.f;
+      if constexpr (kQuant) {
+        k0 = ksc[t0];
+        k1 = ksc[t1];
       }
-      // ---------------------------------------------------- O^T += V^T P^T
+      sc[mt][0] = t0 < valid ? acc[0] * s_fac[0] * k0 : -INFINITY;
+      sc[mt][1] = t0 < valid ? acc[1] * s_fac[1] * k0 : -INFINITY;
+      sc[mt][2] = t1 < valid ? acc[2] * s_fac[0] * k1 : -INFINITY;
+      sc[mt][3] = t1 < valid ? acc[3] * s_fac[1] * k1 : -INFINITY;
+    }
+    // ---------------------------------------------------- online softmax
+    float bm0 = -INFINITY, bm1 = -INFINITY;
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      bm0 = fmaxf(bm0, fmaxf(sc[mt][0], sc[mt][2]));
+      bm1 = fmaxf(bm1, fmaxf(sc[mt][1], sc[mt][3]));
+    }
+    bm0 = warp_max_xor(bm0, 4);
+    bm1 = warp_max_xor(bm1, 4);
+    const float mn0 = fmaxf(m_run[0], bm0), mn1 = fmaxf(m_run[1], bm1);
+    const float al0 = rescale(m_run[0], mn0), al1 = rescale(m_run[1], mn1);
+    m_run[0] = mn0;
+    m_run[1] = mn1;
+    float ls0 = 0.f, ls1 = 0.f;
+    // weights for P V: exp2(s - m) (16-bit), exp2(s + log2 sv - m2) (quant)
+    float w[MT][4];
+    float be0 = 1.f, be1 = 1.f;  // O rescale factors
+    if constexpr (!kQuant) {
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
-        // P^T operand (k = token, n = head) from the score layout by transpose,
-        // as a hi and a lo part so that the weights keep ~fp32 accuracy
-        uint32_t h0, l0, h1, l1;
-        split2<kBF>(w[mt][0], w[mt][1], h0, l0);
-        split2<kBF>(w[mt][2], w[mt][3], h1, l1);
-        const uint32_t pb0 = movmatrix_t(h0), pb1 = movmatrix_t(h1);
-        const uint32_t pl0 = movmatrix_t(l0), pl1 = movmatrix_t(l1);
-        // token rows this lane's V^T fragments cover: 2cq, 2cq+1, 2cq+8, 2cq+9
-        const int tb = mt * 16 + 2 * cq;
-        const bool full = (mt * 16 + 16) <= valid;
-        const uint32_t m0 = (tb < valid ? 0xFFFFu : 0u) | (tb + 1 < valid ? 0xFFFF0000u : 0u);
-        const uint32_t m1 = (tb + 8 < valid ? 0xFFFFu : 0u) | (tb + 9 < valid ? 0xFFFF0000u : 0u);
-        if constexpr (!kQuant) {
-#pragma unroll
-          for (int dt = 0; dt < D / 16; ++dt) {
-            uint32_t a0, a1, a2, a3;
-            // matrices: tokens 0-7 / chunk 2dt, tokens 0-7 / 2dt+1,
-            //           tokens 8-15 / 2dt, tokens 8-15 / 2dt+1
-            const int vr = mt * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
-            ldsm_x4_t(T::chunk(vtile, r0 + vr, 2 * dt + ((lane >> 3) & 1), rows), a0, a1, a2, a3);
-            if (!full) {  // zero rows past the valid length (stale data may be NaN)
-              a0 &= m0;
-              a1 &= m0;
-              a2 &= m1;
-              a3 &= m1;
-            }
-            mma16816<kBF>(oacc[dt], a0, a1, a2, a3, pb0, pb1);
-            mma16816<kBF>(oacc[dt], a0, a1, a2, a3, pl0, pl1);
-          }
-        } else {
-#pragma unroll
-          for (int cp = 0; cp < D / 32; ++cp) {
-            // byte matrices: tokens 0-7 / chunk 2cp, tokens 8-15 / 2cp,
-            //                tokens 0-7 / 2cp+1, tokens 8-15 / 2cp+1
-            uint32_t q0, q1, q2, q3;
-            const int vr = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-            ldsm_x4_t(T::chunk(vtile, r0 + vr, 2 * cp + (lane >> 4), rows), q0, q1, q2, q3);
-            // after the transpose a lane holds tokens (2cq, 2cq+1) x dims (2gq, 2gq+1)
-            // of each 16-dim chunk: bytes 0,2 -> dim 2gq; bytes 1,3 -> dim 2gq+1
-            uint32_t a[8];
-            if constexpr (KV_T == KV_INT8) {
-              q0 ^= 0x80808080u; q1 ^= 0x80808080u; q2 ^= 0x80808080u; q3 ^= 0x80808080u;
-              a[0] = int8_pair<0, 2>(q0); a[1] = int8_pair<1, 3>(q0);
-              a[2] = int8_pair<0, 2>(q1); a[3] = int8_pair<1, 3>(q1);
-              a[4] = int8_pair<0, 2>(q2); a[5] = int8_pair<1, 3>(q2);
-              a[6] = int8_pair<0, 2>(q3); a[7] = int8_pair<1, 3>(q3);
-            } else {
-              a[0] = e5m2_pair<0, 2>(q0); a[1] = e5m2_pair<1, 3>(q0);
-              a[2] = e5m2_pair<0, 2>(q1); a[3] = e5m2_pair<1, 3>(q1);
-              a[4] = e5m2_pair<0, 2>(q2); a[5] = e5m2_pair<1, 3>(q2);
-              a[6] = e5m2_pair<0, 2>(q3); a[7] = e5m2_pair<1, 3>(q3);
-            }
-            if (!full) {
-              a[0] &= m0; a[1] &= m0; a[2] &= m1; a[3] &= m1;
-              a[4] &= m0; a[5] &= m0; a[6] &= m1; a[7] &= m1;
-            }
-            // M rows: gq -> dim 16c + 2gq, gq+8 -> dim 16c + 2gq + 1
-            mma16816<false>(oacc[2 * cp], a[0], a[1], a[2], a[3], pb0, pb1);
-            mma16816<false>(oacc[2 * cp], a[0], a[1], a[2], a[3], pl0, pl1);
-            mma16816<false>(oacc[2 * cp + 1], a[4], a[5], a[6], a[7], pb0, pb1);
-            mma16816<false>(oacc[2 * cp + 1], a[4], a[5], a[6], a[7], pl0, pl1);
-          }
-        }
+        w[mt][0] = exp2_rel(sc[mt][0], mn0);
+        w[mt][1] = exp2_rel(sc[mt][1], mn1);
+        w[mt][2] = exp2_rel(sc[mt][2], mn0);
+        w[mt][3] = exp2_rel(sc[mt][3], mn1);
+        ls0 += w[mt][0] + w[mt][2];
+        ls1 += w[mt][1] + w[mt][3];
       }
+      be0 = al0;
+      be1 = al1;
     } else {
-      // ====================================================== scalar (MHA)
-      constexpr int NV = BS / 2;  // tokens per half-warp: rows 2i + hw
-      const int hw = lane >> 4, jl = lane & 15;
-      float part_s[NV];
+      float y[MT][4];
+      float bn0 = -INFINITY, bn1 = -INFINITY;
 #pragma unroll
-      for (int i = 0; i < NV; ++i) {
-        const int r = 2 * i + hw;
-        float kv[E];
-        const uint32_t boff = jl * E * T::kElt;  // byte offset of this lane's values in the row
-        load_vals<KV_T, E>(T::chunk(ktile, r0 + r, boff >> 4, rows) + (boff & 15), kv);
-        float a = 0.f;
-#pragma unroll
-        for (int e = 0; e < E; ++e) a = fmaf(qs[e], kv[e], a);
-        part_s[i] = a;
+      for (int mt = 0; mt < MT; ++mt) {
+        const int t0 = mt * 16 + gq, t1 = t0 + 8;
+        const float lv0 = t0 < valid ? log2f(vsc[t0]) : -INFINITY;
+        const float lv1 = t1 < valid ? log2f(vsc[t1]) : -INFINITY;
+        y[mt][0] = sc[mt][0] + lv0;
+        y[mt][1] = sc[mt][1] + lv0;
+        y[mt][2] = sc[mt][2] + lv1;
+        y[mt][3] = sc[mt][3] + lv1;
+        bn0 = fmaxf(bn0, fmaxf(y[mt][0], y[mt][2]));
+        bn1 = fmaxf(bn1, fmaxf(y[mt][1], y[mt][3]));
+        ls0 += exp2_rel(sc[mt][0], mn0) + exp2_rel(sc[mt][2], mn0);
+        ls1 += exp2_rel(sc[mt][1], mn1) + exp2_rel(sc[mt][3], mn1);
       }
-      // butterfly reduce-scatter over the 16 lanes of the half-warp
-      int nv = NV;
+      bn0 = warp_max_xor(bn0, 4);
+      bn1 = warp_max_xor(bn1, 4);
+      const float n0 = fmaxf(m2_run[0], bn0), n1 = fmaxf(m2_run[1], bn1);
+      be0 = rescale(m2_run[0], n0);
+      be1 = rescale(m2_run[1], n1);
+      m2_run[0] = n0;
+      m2_run[1] = n1;
 #pragma unroll
-      for (int o = 8; o >= 1; o >>= 1) {
-        if (nv > 1) {
-          const bool up = (jl & o) != 0;
+      for (int mt = 0; mt < MT; ++mt) {
+        w[mt][0] = exp2_rel(y[mt][0], n0);
+        w[mt][1] = exp2_rel(y[mt][1], n1);
+        w[mt][2] = exp2_rel(y[mt][2], n0);
+        w[mt][3] = exp2_rel(y[mt][3], n1);
+      }
+    }
+    l_run[0] = l_run[0] * al0 + ls0;
+    l_run[1] = l_run[1] * al1 + ls1;
 #pragma unroll
-          for (int k = 0; k < NV / 2; ++k) {
-            if (k < nv / 2) {
-              const float send = up ? part_s[k] : part_s[k + nv / 2];
-              const float keep = up ? part_s[k + nv / 2] : part_s[k];
-              part_s[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-            }
+    for (int dt = 0; dt < D / 16; ++dt) {
+      oacc[dt][0] *= be0;
+      oacc[dt][1] *= be1;
+      oacc[dt][2] *= be0;
+      oacc[dt][3] *= be1;
+    }
+    // ---------------------------------------------------- O^T += V^T P^T
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      // P^T operand (k = token, n = head) from the score layout by transpose,
+      // as a hi and a lo part so that the weights keep ~fp32 accuracy
+      uint32_t h0, l0, h1, l1;
+      split2<kBF>(w[mt][0], w[mt][1], h0, l0);
+      split2<kBF>(w[mt][2], w[mt][3], h1, l1);
+      const uint32_t pb0 = movmatrix_t(h0), pb1 = movmatrix_t(h1);
+      const uint32_t pl0 = movmatrix_t(l0), pl1 = movmatrix_t(l1);
+      // token rows this lane's V^T fragments cover: 2cq, 2cq+1, 2cq+8, 2cq+9
+      const int tb = mt * 16 + 2 * cq;
+      const bool full = (mt * 16 + 16) <= valid;
+      const uint32_t m0 = (tb < valid ? 0xFFFFu : 0u) | (tb + 1 < valid ? 0xFFFF0000u : 0u);
+      const uint32_t m1 = (tb + 8 < valid ? 0xFFFFu : 0u) | (tb + 9 < valid ? 0xFFFF0000u : 0u);
+      if constexpr (!kQuant) {
+#pragma unroll
+        for (int dt = 0; dt < D / 16; ++dt) {
+          uint32_t a0, a1, a2, a3;
+          // matrices: tokens 0-7 / chunk 2dt, tokens 0-7 / 2dt+1,
+          //           tokens 8-15 / 2dt, tokens 8-15 / 2dt+1
+          const int vr = mt * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
+          ldsm_x4_t(T::chunk(vtile, r0 + vr, 2 * dt + ((lane >> 3) & 1), rows), a0, a1, a2, a3);
+          if (!full) {  // zero rows past the valid length (stale data may be NaN)
+            a0 &= m0;
+            a1 &= m0;
+            a2 &= m1;
+            a3 &= m1;
           }
-          nv >>= 1;
-        } else {
-          part_s[0] += __shfl_xor_sync(0xffffffffu, part_s[0], o);
+          mma16816<kBF>(oacc[dt], a0, a1, a2, a3, pb0, pb1);
+          mma16816<kBF>(oacc[dt], a0, a1, a2, a3, pl0, pl1);
+        }
+      } else {
+#pragma unroll
+        for (int cp = 0; cp < D / 32; ++cp) {
+          // byte matrices: tokens 0-7 / chunk 2cp, tokens 8-15 / 2cp,
+          //                tokens 0-7 / 2cp+1, tokens 8-15 / 2cp+1
+          uint32_t q0, q1, q2, q3;
+          const int vr = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+          ldsm_x4_t(T::chunk(vtile, r0 + vr, 2 * cp + (lane >> 4), rows), q0, q1, q2, q3);
+          // after the transpose a lane holds tokens (2cq, 2cq+1) x dims (2gq, 2gq+1)
+          // of each 16-dim chunk: bytes 0,2 -> dim 2gq; bytes 1,3 -> dim 2gq+1
+          uint32_t a[8];
+          if constexpr (KV_T == KV_INT8) {
+            q0 ^= 0x80808080u; q1 ^= 0x80808080u; q2 ^= 0x80808080u; q3 ^= 0x80808080u;
+            a[0] = int8_pair<0, 2>(q0); a[1] = int8_pair<1, 3>(q0);
+            a[2] = int8_pair<0, 2>(q1); a[3] = int8_pair<1, 3>(q1);
+            a[4] = int8_pair<0, 2>(q2); a[5] = int8_pair<1, 3>(q2);
+            a[6] = int8_pair<0, 2>(q3); a[7] = int8_pair<1, 3>(q3);
+          } else {
+            a[0] = e5m2_pair<0, 2>(q0); a[1] = e5m2_pair<1, 3>(q0);
+            a[2] = e5m2_pair<0, 2>(q1); a[3] = e5m2_pair<1, 3>(q1);
+            a[4] = e5m2_pair<0, 2>(q2); a[5] = e5m2_pair<1, 3>(q2);
+            a[6] = e5m2_pair<0, 2>(q3); a[7] = e5m2_pair<1, 3>(q3);
+          }
+          if (!full) {
+            a[0] &= m0; a[1] &= m0; a[2] &= m1; a[3] &= m1;
+            a[4] &= m0; a[5] &= m0; a[6] &= m1; a[7] &= m1;
+          }
+          // M rows: gq -> dim 16c + 2gq, gq+8 -> dim 16c + 2gq + 1
+          mma16816<false>(oacc[2 * cp], a[0], a[1], a[2], a[3], pb0, pb1);
+          mma16816<false>(oacc[2 * cp], a[0], a[1], a[2], a[3], pl0, pl1);
+          mma16816<false>(oacc[2 * cp + 1], a[4], a[5], a[6], a[7], pb0, pb1);
+          mma16816<false>(oacc[2 * cp + 1], a[4], a[5], a[6], a[7], pl0, pl1);
         }
       }
-      // this lane now holds row 2*idx + hw, idx = jl (16 rows) or jl >> 1 (8 rows)
-      const int idx = NV == 16 ? jl : (jl >> 1);
-      const int r = 2 * idx + hw;
-      float kscale = 1.f;
-      if constexpr (kQuant) kscale = ksc[r];
-      const float sv = r < valid ? part_s[0] * kscale : -INFINITY;
-      const float bm = warp_max_xor(sv, 1);
-      const float mn = fmaxf(m_run[0], bm);
-      const float al = rescale(m_run[0], mn);
-      m_run[0] = mn;
-      const float pw = exp2_rel(sv, mn);
-      float lsum = 0.f;
-#pragma unroll
-      for (int e = 0; e < E; ++e) oacc_s[e] *= al;
-#pragma unroll
-      for (int i = 0; i < NV; ++i) {
-        const int src = hw * 16 + (NV == 16 ? i : 2 * i);
-        float pi = __shfl_sync(0xffffffffu, pw, src);
-        const int rr = 2 * i + hw;
-        lsum += pi;
-        if (rr < valid) {
-          if constexpr (kQuant) pi *= vsc[rr];
-          float vv[E];
-          const uint32_t boff = jl * E * T::kElt;
-          load_vals<KV_T, E>(T::chunk(vtile, r0 + rr, boff >> 4, rows) + (boff & 15), vv);
-#pragma unroll
-          for (int e = 0; e < E; ++e) oacc_s[e] = fmaf(pi, vv[e], oacc_s[e]);
-        }
-      }
-      l_run[0] = l_run[0] * al + lsum;
     }
   }
 
@@ -653,77 +533,57 @@ struct Consumer {
   __device__ __forceinline__ void finish(const AttnParams &p, bool whole, int b, int h0, int nh,
                                          int64_t pbase, bool alive, int lane) {
     const int gq = lane >> 2, cq = lane & 3;
-    if constexpr (MMA) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      l_run[i] += __shfl_xor_sync(0xffffffffu, l_run[i], 4);
+      l_run[i] += __shfl_xor_sync(0xffffffffu, l_run[i], 8);
+      l_run[i] += __shfl_xor_sync(0xffffffffu, l_run[i], 16);
+    }
+    float f[2] = {alive ? 1.f : 0.f, alive ? 1.f : 0.f};
+    if constexpr (kQuant) {
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+        f[i] = (m2_run[i] == -INFINITY || !alive) ? 0.f : exp2f(m2_run[i] - m_run[i]);
+    }
+    if (whole) {
+#pragma unroll
+      for (int i = 0; i < 2; ++i) f[i] = l_run[i] > 0.f ? f[i] / l_run[i] : 0.f;
+    }
+#pragma unroll
+    for (int dt = 0; dt < D / 16; ++dt) {
+      int d0, d1;
+      if constexpr (kQuant) {  // rows gq / gq+8 are dims 16c + 2gq / + 1
+        d0 = dt * 16 + 2 * gq;
+        d1 = d0 + 1;
+      } else {
+        d0 = dt * 16 + gq;
+        d1 = d0 + 8;
+      }
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
-        l_run[i] += __shfl_xor_sync(0xffffffffu, l_run[i], 4);
-        l_run[i] += __shfl_xor_sync(0xffffffffu, l_run[i], 8);
-        l_run[i] += __shfl_xor_sync(0xffffffffu, l_run[i], 16);
-      }
-      float f[2] = {alive ? 1.f : 0.f, alive ? 1.f : 0.f};
-      if constexpr (kQuant) {
-#pragma unroll
-        for (int i = 0; i < 2; ++i)
-          f[i] = (m2_run[i] == -INFINITY || !alive) ? 0.f : exp2f(m2_run[i] - m_run[i]);
-      }
-      if (whole) {
-#pragma unroll
-        for (int i = 0; i < 2; ++i) f[i] = l_run[i] > 0.f ? f[i] / l_run[i] : 0.f;
-      }
-#pragma unroll
-      for (int dt = 0; dt < D / 16; ++dt) {
-        int d0, d1;
-        if constexpr (kQuant) {  // rows gq / gq+8 are dims 16c + 2gq / + 1
-          d0 = dt * 16 + 2 * gq;
-          d1 = d0 + 1;
-        } else {
-          d0 = dt * 16 + gq;
-          d1 = d0 + 8;
-        }
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int n = 2 * cq + i;
-          if (n < nh) {
-            const float v0 = oacc[dt][i] * f[i], v1 = oacc[dt][i + 2] * f[i];
-            if (whole) {
-              const int64_t o = (static_cast<int64_t>(b) * p.q_heads + h0 + n) * D;
-              store_out<Q_T>(p.out, o + d0, v0);
-              store_out<Q_T>(p.out, o + d1, v1);
-            } else {
-              float *po = p.part_o + (pbase + n) * D;
-              po[d0] = v0;
-              po[d1] = v1;
-            }
+        const int n = 2 * cq + i;
+        if (n < nh) {
+          const float v0 = oacc[dt][i] * f[i], v1 = oacc[dt][i + 2] * f[i];
+          if (whole) {
+            const int64_t o = (static_cast<int64_t>(b) * p.q_heads + h0 + n) * D;
+            store_out<Q_T>(p.out, o + d0, v0);
+            store_out<Q_T>(p.out, o + d1, v1);
+          } else {
+            float *po = p.part_o + (pbase + n) * D;
+            po[d0] = v0;
+            po[d1] = v1;
           }
         }
       }
-      if (!whole && gq == 0) {
+    }
+    if (!whole && gq == 0) {
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int n = 2 * cq + i;
-          if (n < nh) {
-            p.part_ml[(pbase + n) * 2] = alive ? m_run[i] : -INFINITY;
-            p.part_ml[(pbase + n) * 2 + 1] = l_run[i];
-          }
+      for (int i = 0; i < 2; ++i) {
+        const int n = 2 * cq + i;
+        if (n < nh) {
+          p.part_ml[(pbase + n) * 2] = alive ? m_run[i] : -INFINITY;
+          p.part_ml[(pbase + n) * 2 + 1] = l_run[i];
         }
-      }
-    } else {
-      const int hw = lane >> 4, jl = lane & 15;
-      l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], 16);
-      const float f = !alive ? 0.f : whole ? (l_run[0] > 0.f ? 1.f / l_run[0] : 0.f) : 1.f;
-#pragma unroll
-      for (int e = 0; e < E; ++e) {
-        const float v = (oacc_s[e] + __shfl_xor_sync(0xffffffffu, oacc_s[e], 16)) * f;
-        if (hw == 0) {
-          if (whole)
-            store_out<Q_T>(p.out, (static_cast<int64_t>(b) * p.q_heads + h0) * D + jl * E + e, v);
-          else
-            p.part_o[pbase * D + jl * E + e] = v;
-        }
-      }
-      if (!whole && lane == 0) {
-        p.part_ml[pbase * 2] = alive ? m_run[0] : -INFINITY;
-        p.part_ml[pbase * 2 + 1] = l_run[0];
       }
     }
   }
@@ -832,7 +692,7 @@ __device__ __forceinline__ void walk_advance(Walk &w, int seg, const AttnParams 
 // ============================================================================
 // Partition kernel: persistent, one producer warp + kNC consumer warps.
 // ============================================================================
-template <int D, int BS, int KV_T, int Q_T, bool MMA>
+template <int D, int BS, int KV_T, int Q_T>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_partition_kernel(const __grid_constant__ CUtensorMap kmap,
                       const __grid_constant__ CUtensorMap vmap, const AttnParams p) {
@@ -974,7 +834,7 @@ attn_partition_kernel(const __grid_constant__ CUtensorMap kmap,
   // Consumer warp `warp` owns slot `warp` of each unit: kv head hi = warp / cpg
   // of the unit's group, query-head chunk cl = warp % cpg. Every consumer visits
   // every position (an idle one only releases the stage).
-  Consumer<D, BS, KV_T, Q_T, MMA> cs;
+  Consumer<D, BS, KV_T, Q_T> cs;
   Walk w = w0;
   uint32_t k = 0;
   bool alive = true;
@@ -993,7 +853,7 @@ attn_partition_kernel(const __grid_constant__ CUtensorMap kmap,
     const int g = hgi * p.hg + hi;
     const int chunk = cgi * p.cpg + cl;
     const int h0 = g * p.group + chunk * kChunkHeads;
-    const int nh = MMA ? min(kChunkHeads, p.group - chunk * kChunkHeads) : 1;
+    const int nh = min(kChunkHeads, p.group - chunk * kChunkHeads);
     const int L = p.context_lens[w.b];
     // fused append: the new token (position L - 1) is in block jl of the unit;
     // with one query-head chunk per kv head this warp alone uses its rows
@@ -1148,11 +1008,11 @@ __global__ void __launch_bounds__(kMergeWarps * 32) attn_merge_kernel(const Attn
 using PartFn = cudaError_t (*)(const CUtensorMap &, const CUtensorMap &, const AttnParams &,
                                cudaStream_t);
 
-template <int D, int BS, int KV_T, int Q_T, bool MMA>
+template <int D, int BS, int KV_T, int Q_T>
 cudaError_t launch_part(const CUtensorMap &km, const CUtensorMap &vm, const AttnParams &p,
                         cudaStream_t st) {
   const int smem = p.stages * p.stage_bytes + 1024;
-  auto kern = attn_partition_kernel<D, BS, KV_T, Q_T, MMA>;
+  auto kern = attn_partition_kernel<D, BS, KV_T, Q_T>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   e = launch_pdl(kern, dim3(p.num_ctas), dim3(kThreads), smem, st, km, vm, p);
@@ -1160,28 +1020,22 @@ cudaError_t launch_part(const CUtensorMap &km, const CUtensorMap &vm, const Attn
   return cudaGetLastError();
 }
 
-template <int D, int BS, int KV_T, int Q_T>
-PartFn pick_path(bool mma) {
-  return mma ? launch_part<D, BS, KV_T, Q_T, true> : launch_part<D, BS, KV_T, Q_T, false>;
-}
-
 template <int D, int BS>
-PartFn pick_dtype(int kv, int q, bool mma) {
+PartFn pick_dtype(int kv, int q) {
   switch (kv) {
-    case KV_BF16: return pick_path<D, BS, KV_BF16, KV_BF16>(mma);
-    case KV_FP16: return pick_path<D, BS, KV_FP16, KV_FP16>(mma);
+    case KV_BF16: return launch_part<D, BS, KV_BF16, KV_BF16>;
+    case KV_FP16: return launch_part<D, BS, KV_FP16, KV_FP16>;
     case KV_INT8:
-      return q == KV_BF16 ? pick_path<D, BS, KV_INT8, KV_BF16>(mma)
-                          : pick_path<D, BS, KV_INT8, KV_FP16>(mma);
+      return q == KV_BF16 ? launch_part<D, BS, KV_INT8, KV_BF16> : launch_part<D, BS, KV_INT8, KV_FP16>;
     default:
-      return q == KV_BF16 ? pick_path<D, BS, KV_FP8_E5M2, KV_BF16>(mma)
-                          : pick_path<D, BS, KV_FP8_E5M2, KV_FP16>(mma);
+      return q == KV_BF16 ? launch_part<D, BS, KV_FP8_E5M2, KV_BF16>
+                          : launch_part<D, BS, KV_FP8_E5M2, KV_FP16>;
   }
 }
 
-PartFn pick_partition(int D, int BS, int kv, int q, bool mma) {
-  if (D == 128) return BS == 16 ? pick_dtype<128, 16>(kv, q, mma) : pick_dtype<128, 32>(kv, q, mma);
-  return BS == 16 ? pick_dtype<64, 16>(kv, q, mma) : pick_dtype<64, 32>(kv, q, mma);
+PartFn pick_partition(int D, int BS, int kv, int q) {
+  if (D == 128) return BS == 16 ? pick_dtype<128, 16>(kv, q) : pick_dtype<128, 32>(kv, q);
+  return BS == 16 ? pick_dtype<64, 16>(kv, q) : pick_dtype<64, 32>(kv, q);
 }
 
 cudaError_t launch_merge(int D, int out_t, const AttnParams &p, cudaStream_t st) {
@@ -1209,7 +1063,7 @@ UnitGeom unit_geom(const kv_pool *pool, int num_q_heads) {
   const kv_pool_desc &d = pool->d;
   UnitGeom u{};
   const int group = num_q_heads / d.num_kv_heads;
-  u.chunks = group >= 2 ? (group + kChunkHeads - 1) / kChunkHeads : 1;
+  u.chunks = (group + kChunkHeads - 1) / kChunkHeads;
   u.cpg = std::min(u.chunks, kNC);
   u.cgroups = (u.chunks + u.cpg - 1) / u.cpg;
   const int elt = elem_bytes(d.cache_dtype);
@@ -1371,7 +1225,7 @@ kv_status run_partition(kv_pool *pool, int32_t layer, const void *q, int32_t q_d
   kv_status code;
   const LayerMaps *maps = layer_maps(pool, layer, p.hg * pool->d.block_size, &code);
   if (!maps) return code;
-  PartFn fn = pick_partition(pool->d.head_dim, pool->d.block_size, cd, q_dtype, p.group >= 2);
+  PartFn fn = pick_partition(pool->d.head_dim, pool->d.block_size, cd, q_dtype);
   return cuda_check(fn(maps->k, maps->v, p, st), "paged attention launch");
 }
 
