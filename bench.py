@@ -299,14 +299,26 @@ def run_ours(args, rank, world, device):
     # ---------------------------------------------------------- end to end
     e2e = None
     if not args.no_e2e:
-        pin = lambda t: t.cpu().pin_memory()
-        h_q, h_kn, h_vn = pin(wl.q), pin(wl.k_new), pin(wl.v_new)
-        h_slot, h_tab, h_len = pin(slot_new), pin(tables), pin(lens)
+        # The step's inputs travel in one pinned host buffer and one copy: q,
+        # the new K/V rows, block tables, lengths (and slots when the append is
+        # a separate kernel), each at a 256-byte offset.
+        parts = [wl.q, wl.k_new, wl.v_new, tables, lens] + ([] if fused else [slot_new])
+        offs, n = [], 0
+        for t in parts:
+            offs.append(n)
+            n += -(-t.numel() * t.element_size() // 256) * 256
+        h_in = torch.empty(n, dtype=torch.uint8).pin_memory()
+        d_in = torch.empty(n, dtype=torch.uint8, device=device)
+        views = []
+        for t, o in zip(parts, offs):
+            nb = t.numel() * t.element_size()
+            h_in[o:o + nb].copy_(t.contiguous().view(torch.uint8).reshape(-1).cpu())
+            views.append(d_in[o:o + nb].view(t.dtype).view(t.shape))
+        d_q, d_kn, d_vn, d_tab, d_len = views[:5]
+        d_slot = None if fused else views[5]
         h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        d_q, d_kn, d_vn = torch.empty_like(wl.q), torch.empty_like(wl.k_new), torch.empty_like(wl.v_new)
-        d_slot, d_tab, d_len = torch.empty_like(slot_new), torch.empty_like(tables), torch.empty_like(lens)
         d_out = torch.empty_like(out)
-        h2d = sum(t.numel() * t.element_size() for t in (h_q, h_kn, h_vn, h_slot, h_tab, h_len))
+        h2d = sum(t.numel() * t.element_size() for t in parts)
         d2h = h_out.numel() * h_out.element_size()
         n_e2e = max(10, args.steps // 10)
         times = []
@@ -315,9 +327,7 @@ def run_ours(args, rank, world, device):
             torch.cuda.synchronize(device)
             a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
-            for d, h in ((d_q, h_q), (d_kn, h_kn), (d_vn, h_vn), (d_slot, h_slot),
-                         (d_tab, h_tab), (d_len, h_len)):
-                d.copy_(h, non_blocking=True)
+            d_in.copy_(h_in, non_blocking=True)
             if fused:
                 pkv.paged_attn_decode_append(pool, 0, d_q, d_kn, d_vn, d_tab, d_len, max_ctx,
                                              wl.scale, out=d_out, num_ctas=G, workspace=ws)

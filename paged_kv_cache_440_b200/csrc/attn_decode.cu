@@ -42,6 +42,7 @@
 //   multiply the scores, per-token V scales are folded into the softmax
 //   weights through log2(scale) so the fp16 weights stay within (0, 1].
 #include <algorithm>
+#include <cfloat>
 
 #include "device.cuh"
 #include "internal.h"
@@ -171,6 +172,20 @@ __device__ __forceinline__ float exp2_rel(float x, float m) {
 // Rescale factor exp2(m_old - m_new), 1 while nothing has been seen.
 __device__ __forceinline__ float rescale(float m_old, float m_new) {
   return m_new == -INFINITY ? 1.f : exp2f(m_old - m_new);
+}
+
+// The SFU's base-2 exponential and logarithm (relative error about 2^-22,
+// ample for softmax weights that are rounded to 16 bits for the MMA).
+// ex2(-inf) = 0 and lg2(0) = -inf; subnormal inputs and results are zero.
+__device__ __forceinline__ float ex2_sfu(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float lg2_sfu(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 template <int Q_T>
@@ -334,6 +349,7 @@ struct Consumer {
   // One staged block of head `hi` of the stage's `rows`-row group: rows
   // [0, valid) of the head's BS rows are real tokens.
   __device__ __forceinline__ void block(const uint8_t *st, int rows, int hi, int valid, int lane) {
+    if (valid <= 0) return;  // no token (an invalid block id): nothing to add
     const uint32_t ktile = smem_u32(st);
     const uint32_t vtile = ktile + rows * T::kRowBytes;
     const int r0 = hi * BS;  // the head's first row in the stage
@@ -397,8 +413,11 @@ struct Consumer {
     }
     bm0 = warp_max_xor(bm0, 4);
     bm1 = warp_max_xor(bm1, 4);
+    // a block holds at least one valid token, so the new maxima are finite;
+    // a factor is exactly 1 when its maximum did not move
     const float mn0 = fmaxf(m_run[0], bm0), mn1 = fmaxf(m_run[1], bm1);
-    const float al0 = rescale(m_run[0], mn0), al1 = rescale(m_run[1], mn1);
+    const float al0 = mn0 == m_run[0] ? 1.f : ex2_sfu(m_run[0] - mn0);
+    const float al1 = mn1 == m_run[1] ? 1.f : ex2_sfu(m_run[1] - mn1);
     m_run[0] = mn0;
     m_run[1] = mn1;
     float ls0 = 0.f, ls1 = 0.f;
@@ -408,10 +427,10 @@ struct Consumer {
     if constexpr (!kQuant) {
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
-        w[mt][0] = exp2_rel(sc[mt][0], mn0);
-        w[mt][1] = exp2_rel(sc[mt][1], mn1);
-        w[mt][2] = exp2_rel(sc[mt][2], mn0);
-        w[mt][3] = exp2_rel(sc[mt][3], mn1);
+        w[mt][0] = ex2_sfu(sc[mt][0] - mn0);
+        w[mt][1] = ex2_sfu(sc[mt][1] - mn1);
+        w[mt][2] = ex2_sfu(sc[mt][2] - mn0);
+        w[mt][3] = ex2_sfu(sc[mt][3] - mn1);
         ls0 += w[mt][0] + w[mt][2];
         ls1 += w[mt][1] + w[mt][3];
       }
@@ -423,40 +442,47 @@ struct Consumer {
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
         const int t0 = mt * 16 + gq, t1 = t0 + 8;
-        const float lv0 = t0 < valid ? log2f(vsc[t0]) : -INFINITY;
-        const float lv1 = t1 < valid ? log2f(vsc[t1]) : -INFINITY;
+        const float lv0 = t0 < valid ? lg2_sfu(vsc[t0]) : -INFINITY;
+        const float lv1 = t1 < valid ? lg2_sfu(vsc[t1]) : -INFINITY;
         y[mt][0] = sc[mt][0] + lv0;
         y[mt][1] = sc[mt][1] + lv0;
         y[mt][2] = sc[mt][2] + lv1;
         y[mt][3] = sc[mt][3] + lv1;
         bn0 = fmaxf(bn0, fmaxf(y[mt][0], y[mt][2]));
         bn1 = fmaxf(bn1, fmaxf(y[mt][1], y[mt][3]));
-        ls0 += exp2_rel(sc[mt][0], mn0) + exp2_rel(sc[mt][2], mn0);
-        ls1 += exp2_rel(sc[mt][1], mn1) + exp2_rel(sc[mt][3], mn1);
+        ls0 += ex2_sfu(sc[mt][0] - mn0) + ex2_sfu(sc[mt][2] - mn0);
+        ls1 += ex2_sfu(sc[mt][1] - mn1) + ex2_sfu(sc[mt][3] - mn1);
       }
       bn0 = warp_max_xor(bn0, 4);
       bn1 = warp_max_xor(bn1, 4);
+      // the second maxima stay -inf while every V scale seen is 0; a finite
+      // stand-in keeps y - n from becoming NaN (all such y are -inf)
       const float n0 = fmaxf(m2_run[0], bn0), n1 = fmaxf(m2_run[1], bn1);
-      be0 = rescale(m2_run[0], n0);
-      be1 = rescale(m2_run[1], n1);
+      const float f0 = fmaxf(n0, -FLT_MAX), f1 = fmaxf(n1, -FLT_MAX);
+      be0 = n0 == m2_run[0] ? 1.f : ex2_sfu(m2_run[0] - f0);
+      be1 = n1 == m2_run[1] ? 1.f : ex2_sfu(m2_run[1] - f1);
       m2_run[0] = n0;
       m2_run[1] = n1;
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
-        w[mt][0] = exp2_rel(y[mt][0], n0);
-        w[mt][1] = exp2_rel(y[mt][1], n1);
-        w[mt][2] = exp2_rel(y[mt][2], n0);
-        w[mt][3] = exp2_rel(y[mt][3], n1);
+        w[mt][0] = ex2_sfu(y[mt][0] - f0);
+        w[mt][1] = ex2_sfu(y[mt][1] - f1);
+        w[mt][2] = ex2_sfu(y[mt][2] - f0);
+        w[mt][3] = ex2_sfu(y[mt][3] - f1);
       }
     }
     l_run[0] = l_run[0] * al0 + ls0;
     l_run[1] = l_run[1] * al1 + ls1;
+    // once the running maxima settle, most blocks move none of them: the whole
+    // warp then skips the O rescale
+    if (__any_sync(0xffffffffu, be0 != 1.f || be1 != 1.f)) {
 #pragma unroll
-    for (int dt = 0; dt < D / 16; ++dt) {
-      oacc[dt][0] *= be0;
-      oacc[dt][1] *= be1;
-      oacc[dt][2] *= be0;
-      oacc[dt][3] *= be1;
+      for (int dt = 0; dt < D / 16; ++dt) {
+        oacc[dt][0] *= be0;
+        oacc[dt][1] *= be1;
+        oacc[dt][2] *= be0;
+        oacc[dt][3] *= be1;
+      }
     }
     // ---------------------------------------------------- O^T += V^T P^T
 #pragma unroll
