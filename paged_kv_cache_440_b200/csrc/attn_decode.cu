@@ -289,6 +289,7 @@ struct Consumer {
   float oacc[D / 16][4];
   uint32_t qb[KS][2];
   float s_fac[2];
+  float qcorr[2];  // INT8 keys enter the MMA as 1152 + code: 1152 * sum(q) per head
 
   __device__ __forceinline__ void reset() {
     m_run[0] = m_run[1] = m2_run[0] = m2_run[1] = -INFINITY;
@@ -343,6 +344,20 @@ struct Consumer {
       const int ex1 = __shfl_sync(0xffffffffu, ex, (2 * cq + 1) * 4);
       s_fac[0] = ldexpf(p.scale_log2, -ex0);
       s_fac[1] = ldexpf(p.scale_log2, -ex1);
+      if constexpr (KV_T == KV_INT8) {
+        // sum of the fp16 query operands of head gq (as the MMA sees them)
+        float qsum = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          const __half2 a = *reinterpret_cast<const __half2 *>(&qb[ks][0]);
+          const __half2 c = *reinterpret_cast<const __half2 *>(&qb[ks][1]);
+          qsum += (__low2float(a) + __high2float(a)) + (__low2float(c) + __high2float(c));
+        }
+        qsum += __shfl_xor_sync(0xffffffffu, qsum, 1);
+        qsum += __shfl_xor_sync(0xffffffffu, qsum, 2);
+        qcorr[0] = 1152.f * __shfl_sync(0xffffffffu, qsum, (2 * cq) * 4);
+        qcorr[1] = 1152.f * __shfl_sync(0xffffffffu, qsum, (2 * cq + 1) * 4);
+      }
     }
   }
 
@@ -375,13 +390,15 @@ struct Consumer {
           uint32_t q0, q1, q2, q3;  // byte matrices: rows 0-7 / 8-15 x chunks 2kp, 2kp+1
           ldsm_x4(T::chunk(ktile, r0 + row, 2 * kp + (lane >> 4), rows), q0, q1, q2, q3);
           if constexpr (KV_T == KV_INT8) {
+            // keys as 1152 + code (exact in fp16); the bias is removed per
+            // score below with the query sums
             q0 ^= 0x80808080u; q1 ^= 0x80808080u; q2 ^= 0x80808080u; q3 ^= 0x80808080u;
-            mma16816<false>(acc, int8_pair<0, 1>(q0), int8_pair<0, 1>(q1),
-                            int8_pair<2, 3>(q0), int8_pair<2, 3>(q1), qb[2 * kp][0],
-                            qb[2 * kp][1]);
-            mma16816<false>(acc, int8_pair<0, 1>(q2), int8_pair<0, 1>(q3),
-                            int8_pair<2, 3>(q2), int8_pair<2, 3>(q3), qb[2 * kp + 1][0],
-                            qb[2 * kp + 1][1]);
+            mma16816<false>(acc, int8_pair_biased<0, 1>(q0), int8_pair_biased<0, 1>(q1),
+                            int8_pair_biased<2, 3>(q0), int8_pair_biased<2, 3>(q1),
+                            qb[2 * kp][0], qb[2 * kp][1]);
+            mma16816<false>(acc, int8_pair_biased<0, 1>(q2), int8_pair_biased<0, 1>(q3),
+                            int8_pair_biased<2, 3>(q2), int8_pair_biased<2, 3>(q3),
+                            qb[2 * kp + 1][0], qb[2 * kp + 1][1]);
           } else {
             mma16816<false>(acc, e5m2_pair<0, 1>(q0), e5m2_pair<0, 1>(q1),
                             e5m2_pair<2, 3>(q0), e5m2_pair<2, 3>(q1), qb[2 * kp][0],
@@ -398,6 +415,12 @@ struct Consumer {
       if constexpr (kQuant) {
         k0 = ksc[t0];
         k1 = ksc[t1];
+      }
+      if constexpr (KV_T == KV_INT8) {
+        acc[0] -= qcorr[0];
+        acc[1] -= qcorr[1];
+        acc[2] -= qcorr[0];
+        acc[3] -= qcorr[1];
       }
       sc[mt][0] = t0 < valid ? acc[0] * s_fac[0] * k0 : -INFINITY;
       sc[mt][1] = t0 < valid ? acc[1] * s_fac[1] * k0 : -INFINITY;

@@ -220,6 +220,14 @@ __device__ __forceinline__ uint32_t e5m2_pair(uint32_t src) {
   return prmt(src, 0u, (B << 12) | (4 << 8) | (A << 4) | 4);
 }
 
+// Two INT8 codes (sign bit flipped by the caller) as fp16 1152 + code, exact:
+// the bias stays in and is removed from the dot product by the caller.
+template <int A, int B>
+__device__ __forceinline__ uint32_t int8_pair_biased(uint32_t src_biased) {
+  // result bytes: [0] = u[A], [1] = 0x64, [2] = u[B], [3] = 0x64 -> 1024 + u
+  return prmt(src_biased, 0x64646464u, (4 << 12) | (B << 8) | (4 << 4) | A);
+}
+
 template <int A, int B>
 __device__ __forceinline__ uint32_t int8_pair(uint32_t src_biased) {
   // result bytes: [0] = u[A], [1] = 0x64, [2] = u[B], [3] = 0x64
