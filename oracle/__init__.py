@@ -16,6 +16,8 @@ in exact bit/byte arithmetic where the operation is a copy or an encoding):
   an fp32 scale, and the matching dequantization.
 * ``pool``       -- the pages' KV-bytes formula and block arithmetic.
 * ``allocator``  -- a reference model of a refcounted block pool.
+* ``prefix_cache`` -- a reference model of the prefix cache: cached full-block
+  prefixes as a dict, longest-prefix match by brute force, LRU leaf eviction.
 
 Pinned by ``tests/test_oracle_*.py`` against the pages' worked numbers,
 closed forms, invariants, brute force and independent library routines.
