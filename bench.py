@@ -62,6 +62,10 @@ WORKLOADS = {
                      lambda dev: W.quant_long("int8", "b", dev)),
     "quant_b_e5m2": ("FP8-E5M2 per-token-head KV: 64/8 heads, head_dim 128, block 32, 8 x 32768",
                      lambda dev: W.quant_long("e5m2", "b", dev)),
+    "shared_prefix": ("Shared prompt: 200 requests, 1500-token prefix in 94 shared blocks (the last "
+                      "copied on write per request), suffixes U[1,512], 64/8 heads, D 128, bf16, "
+                      "block 16; GB/s counts logical bytes (the shared prefix is read from L2)",
+                      lambda dev: SharedPrefixStep(dev)),
 }
 
 
@@ -204,6 +208,67 @@ def oracle_sample(wl, budget_s=15.0):
     return nbytes / t_total / 1e9, t_total, done, threads
 
 
+# ------------------------------------------------------------------ shared prefix
+
+class SharedPrefixStep:
+    """The shared-prompt workload as a decode step: 200 requests share a
+    1500-token prompt (94 blocks of 16, the last holding 12 tokens). Setup goes
+    through the library's allocator: each request shares the prompt blocks,
+    copies the partial one on write, and appends its suffix except the last
+    token, which is the step's append."""
+
+    def __init__(self, device):
+        self.sp = sp = W.shared_prefix(device)
+        self.batch, self.q_heads, self.kv_heads = sp.batch, sp.q_heads, sp.kv_heads
+        self.head_dim, self.block_size, self.cache_dtype = sp.head_dim, sp.block_size, "bf16"
+        self.group = sp.q_heads // sp.kv_heads
+        self.scale, self.q, self.num_blocks = sp.scale, sp.q, sp.num_blocks
+        self.k_fill = None
+        self.context_lens = (sp.prefix_len + sp.suffix_lens).astype(np.int32)
+        ends = np.cumsum(sp.suffix_lens) - 1          # each request's last suffix row
+        idx = torch.from_numpy(ends.astype(np.int64)).to(sp.suffix_k.device)
+        self.k_new = sp.suffix_k.index_select(0, idx).contiguous()
+        self.v_new = sp.suffix_v.index_select(0, idx).contiguous()
+
+    def setup(self, pool, pkv):
+        sp, bs = self.sp, self.block_size
+        dev = sp.q.device
+        P = sp.prefix_len
+        nprefix = -(-P // bs)
+        prefix_ids = pool.alloc(nprefix)
+        slots = torch.tensor([prefix_ids[t // bs] * bs + t % bs for t in range(P)],
+                             dtype=torch.int64, device=dev)
+        pkv.kv_append(pool, 0, sp.prefix_k, sp.prefix_v, slots)
+        tables, pairs = [], []
+        for _ in range(self.batch):
+            pool.share(prefix_ids)
+            tables.append(list(prefix_ids))
+        for t in tables:                      # copy-on-write of the partial block
+            new = pool.cow_prepare(t[-1])
+            pairs.append((t[-1], new))
+            t[-1] = new
+        pkv.kv_block_copy(pool, pairs)
+        sl, rows, off = [], [], 0
+        for b, t in enumerate(tables):
+            L = int(self.context_lens[b])
+            t += pool.alloc(-(-L // bs) - len(t))
+            sl += [t[p // bs] * bs + p % bs for p in range(P, L - 1)]
+            rows += list(range(off, off + int(sp.suffix_lens[b]) - 1))
+            off += int(sp.suffix_lens[b])
+        if sl:
+            ri = torch.tensor(rows, dtype=torch.int64, device=dev)
+            pkv.kv_append(pool, 0, sp.suffix_k.index_select(0, ri).contiguous(),
+                          sp.suffix_v.index_select(0, ri).contiguous(),
+                          torch.tensor(sl, dtype=torch.int64, device=dev))
+        mb = max(len(t) for t in tables)
+        self.block_tables = np.full((self.batch, mb), -1, np.int32)
+        for b, t in enumerate(tables):
+            self.block_tables[b, :len(t)] = t
+        L = self.context_lens
+        self.slot_new = np.array([tables[b][(L[b] - 1) // bs] * bs + (L[b] - 1) % bs
+                                  for b in range(self.batch)], np.int64)
+
+
 # ------------------------------------------------------------------ ours
 
 def run_ours(args, rank, world, device):
@@ -213,7 +278,9 @@ def run_ours(args, rank, world, device):
     pool = pkv.KVPool(1, wl.num_blocks, wl.block_size, wl.kv_heads, wl.head_dim,
                       wl.cache_dtype, device)
     K, V, _, _ = pool.layer_views(0)
-    if wl.k_fill is not None:
+    if getattr(wl, "setup", None) is not None:
+        wl.setup(pool, pkv)        # builds the cache through the allocator and CoW
+    elif wl.k_fill is not None:
         K.copy_(wl.k_fill)
         V.copy_(wl.v_fill)
     else:
@@ -438,7 +505,8 @@ def main():
                        "kv_heads": wl.kv_heads, "head_dim": wl.head_dim,
                        "block_size": wl.block_size, "cached_tokens": int(wl.context_lens.sum()),
                        "num_ctas": r["G"], "parallelism": "replicas" if world > 1 else "1 gpu",
-                       "l2": "K/V 2.3x L2; L2 flushed before each timed step by reading 256 MiB",
+                       "l2": "K/V %.1fx L2 (126 MB); L2 flushed before each timed step by "
+                             "reading 256 MiB" % (r["dec_bytes"] / 126e6),
                        "bytes_per_step": r["dec_bytes"] + r["app_bytes"]},
             "pct_of_8tbs": round(100 * gbs / world / NOMINAL_HBM_GBS, 2),
             "decode_tokens_per_s": round(wl.batch * world / r["step_s"], 1),

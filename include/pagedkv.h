@@ -357,6 +357,73 @@ kv_status paged_attn_merge(kv_pool *pool, int32_t num_seqs, int32_t num_q_heads,
 
 /* ------------------------------------------------------------------------ */
 
+/* ------------------------------------------------------------------------ */
+/* Prefix cache (host only)                                                  */
+/*                                                                           */
+/* Requests whose prompts begin with the same tokens reuse the KV blocks      */
+/* already computed for that prefix instead of prefilling it again: a radix   */
+/* tree over token sequences, longest-prefix match (including part of a       */
+/* block), least-recently-used leaves evicted first so a hot shared prefix    */
+/* outlives the private tails below it [bjdmk.com.cn/news/6246348, §4.1,      */
+/* §4.2; KV Cache 原理与 PagedAttention, §五]. KV depends on token and        */
+/* position, so only exact prefixes match (§4.3).                             */
+/*                                                                           */
+/* The cache borrows the pool's refcounted allocator: it holds one reference  */
+/* per cached block, and each block a lookup returns carries one more,        */
+/* owned by the caller (release it with kv_free_blocks). Destroy the cache    */
+/* before its pool. Calls on one cache are serialised internally.             */
+/* ------------------------------------------------------------------------ */
+
+typedef struct kv_prefix_cache kv_prefix_cache;
+
+typedef struct {
+  int64_t nodes;          /* radix-tree nodes (edges) */
+  int64_t cached_blocks;  /* blocks the cache holds a reference on */
+  int64_t lookups;        /* kv_prefix_match calls */
+  int64_t hits;           /* lookups that matched at least one token */
+  int64_t hit_tokens;     /* tokens matched over all lookups */
+} kv_prefix_cache_stats;
+
+kv_status kv_prefix_cache_create(kv_pool *pool, kv_prefix_cache **out);
+
+/* Drops the cache's references (blocks held only by it become free). */
+kv_status kv_prefix_cache_destroy(kv_prefix_cache *cache);
+
+/* Longest cached prefix of tokens[0..n): *num_blocks ids in block_ids (host,
+ * capacity max_blocks >= ceil(n / block_size), else KV_ERR_INVALID) covering
+ * *matched_tokens tokens. Whole blocks come first; when the match continues
+ * into part of one more cached block (at least one token), that block is the
+ * last id: copy it (kv_cow_prepare + kv_block_copy) before appending at
+ * position *matched_tokens. Ties between partial blocks go to the smallest
+ * id. Each returned id carries a new reference for the caller. To keep the
+ * last prompt token for the prefill to compute, pass n - 1. */
+kv_status kv_prefix_match(kv_prefix_cache *cache, const int32_t *tokens, int32_t n,
+                          int32_t max_blocks, int32_t *block_ids,
+                          int32_t *num_blocks, int32_t *matched_tokens);
+
+/* Record that the KV of tokens[0..n) lives in block_ids (host, one id per
+ * whole block: n / block_size of them; a trailing partial block is not
+ * cached). Prefixes already cached keep their blocks; the cache takes a
+ * reference on each block it adds and reports their count in *newly_cached
+ * (may be null). KV_ERR_INVALID, nothing changed, if an id is not allocated. */
+kv_status kv_prefix_insert(kv_prefix_cache *cache, const int32_t *tokens, int32_t n,
+                           const int32_t *block_ids, int32_t num_blocks,
+                           int32_t *newly_cached);
+
+/* Free up to `want` blocks, each time the least recently used leaf block
+ * (ties: smallest id) that only the cache holds (refcount 1); blocks a
+ * request still uses are skipped, and so are their ancestors. The freed ids,
+ * in order, go to freed_ids (host, capacity want). */
+kv_status kv_prefix_evict(kv_prefix_cache *cache, int32_t want, int32_t *freed_ids,
+                          int32_t *num_freed);
+
+/* Forget every cached prefix, e.g. after the model's weights change. */
+kv_status kv_prefix_clear(kv_prefix_cache *cache);
+
+kv_status kv_prefix_stats(kv_prefix_cache *cache, kv_prefix_cache_stats *out);
+
+/* ------------------------------------------------------------------------ */
+
 /* Failure-path self-test: launch one thread that waits on a shared-memory
  * barrier nothing completes, using the same bounded wait as the attention
  * kernel. After limit_us microseconds (1 .. 1e6) it gives up, ORs

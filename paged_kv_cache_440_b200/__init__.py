@@ -6,7 +6,7 @@ The compute runs in ``libpagedkv.so`` (C ABI in ``include/pagedkv.h``);
 been built (``python -m paged_kv_cache_440_b200.build``). There is no fallback.
 """
 _EXPORTS = (
-    "KVPool", "PagedKVError", "default_ctas", "kv_append", "kv_block_copy",
+    "KVPool", "PagedKVError", "PrefixCache", "default_ctas", "kv_append", "kv_block_copy",
     "kv_quantize", "make_workspace", "paged_attn_decode", "paged_attn_decode_append",
     "paged_attn_decode_static", "paged_attn_partition_append",
     "paged_attn_merge",

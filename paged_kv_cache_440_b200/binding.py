@@ -45,7 +45,22 @@ _PI32 = ctypes.POINTER(ctypes.c_int32)
 _PU64 = ctypes.POINTER(ctypes.c_uint64)
 _F = ctypes.c_float
 
+class PrefixCacheStats(ctypes.Structure):
+    _fields_ = [("nodes", ctypes.c_int64), ("cached_blocks", ctypes.c_int64),
+                ("lookups", ctypes.c_int64), ("hits", ctypes.c_int64),
+                ("hit_tokens", ctypes.c_int64)]
+
+
+_PI32 = ctypes.POINTER(ctypes.c_int32)
+
 _SIGS = {
+    "kv_prefix_cache_create": [_P, ctypes.POINTER(_P)],
+    "kv_prefix_cache_destroy": [_P],
+    "kv_prefix_match": [_P, _PI32, _I32, _I32, _PI32, _PI32, _PI32],
+    "kv_prefix_insert": [_P, _PI32, _I32, _PI32, _I32, _PI32],
+    "kv_prefix_evict": [_P, _I32, _PI32, _PI32],
+    "kv_prefix_clear": [_P],
+    "kv_prefix_stats": [_P, ctypes.POINTER(PrefixCacheStats)],
     "kv_pool_required_bytes": [ctypes.POINTER(PoolDesc), _PU64],
     "kv_pool_create": [ctypes.POINTER(PoolDesc), _P, _U64, ctypes.POINTER(_P)],
     "kv_pool_destroy": [_P],
@@ -229,6 +244,64 @@ class KVPool:
         u, f, s = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
         check(lib.kv_pool_stats(self.handle, ctypes.byref(u), ctypes.byref(f), ctypes.byref(s)))
         return {"used": u.value, "free": f.value, "shared": s.value}
+
+
+class PrefixCache:
+    """Host-side prefix cache over a pool's blocks (C ABI kv_prefix_*): a radix
+    tree of token sequences with longest-prefix match and LRU leaf eviction."""
+
+    def __init__(self, pool):
+        self.pool = pool
+        h = ctypes.c_void_p()
+        check(lib.kv_prefix_cache_create(pool.handle, ctypes.byref(h)))
+        self.handle = h
+
+    @staticmethod
+    def _arr(xs):
+        xs = list(xs)
+        return (ctypes.c_int32 * max(len(xs), 1))(*xs), len(xs)
+
+    def match(self, tokens):
+        """(block ids, matched tokens); the caller owns one reference per id."""
+        arr, n = self._arr(tokens)
+        cap = max(-(-n // self.pool.block_size), 1)
+        out = (ctypes.c_int32 * cap)()
+        nb, mt = ctypes.c_int32(), ctypes.c_int32()
+        check(lib.kv_prefix_match(self.handle, arr, n, cap, out, ctypes.byref(nb),
+                                  ctypes.byref(mt)))
+        return list(out[:nb.value]), mt.value
+
+    def insert(self, tokens, block_ids):
+        arr, n = self._arr(tokens)
+        ids, nb = self._arr(block_ids)
+        new = ctypes.c_int32()
+        check(lib.kv_prefix_insert(self.handle, arr, n, ids, nb, ctypes.byref(new)))
+        return new.value
+
+    def evict(self, want):
+        out = (ctypes.c_int32 * max(want, 1))()
+        k = ctypes.c_int32()
+        check(lib.kv_prefix_evict(self.handle, want, out, ctypes.byref(k)))
+        return list(out[:k.value])
+
+    def clear(self):
+        check(lib.kv_prefix_clear(self.handle))
+
+    def stats(self):
+        st = PrefixCacheStats()
+        check(lib.kv_prefix_stats(self.handle, ctypes.byref(st)))
+        return {f: getattr(st, f) for f, _ in PrefixCacheStats._fields_}
+
+    def close(self):
+        if getattr(self, "handle", None):
+            lib.kv_prefix_cache_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 # ------------------------------------------------------------------ ops
