@@ -9,7 +9,8 @@ Every routine is the plainest statement of what the pages define, in float64 (or
 in exact bit/byte arithmetic where the operation is a copy or an encoding):
 
 * ``attention``  -- softmax(q K^T * scale) V over the logically contiguous
-  sequence gathered through the block table (no split, no online softmax).
+  sequence gathered through the block table (no split, no online softmax);
+  chunked prefill: every new token attends to the positions up to its own.
 * ``cache_ops``  -- append of a step's K/V into the slot it maps to, copy of
   whole physical blocks (copy-on-write), both as byte copies.
 * ``quant``      -- per-token-head absmax quantization to INT8 and FP8-E5M2 with

@@ -70,3 +70,37 @@ def paged_decode(q, k_cache, v_cache, block_tables, context_lens, scale):
         for h in range(Hq):
             out[b, h] = decode_one(q, k_cache, v_cache, block_tables, context_lens, scale, b, h)
     return out
+
+
+def prefill_one(q_vec, k_cache, v_cache, table_row, pos, kv_head, scale):
+    """Output for one query at position `pos` of a sequence: it attends to
+    positions 0..pos, each token seeing every token before it and itself
+    [KV Cache 原理与 PagedAttention, §一: token t attends to tokens 1..t]."""
+    bs = k_cache.shape[2]
+    K = gather_sequence(k_cache, table_row, pos + 1, kv_head, bs)
+    V = gather_sequence(v_cache, table_row, pos + 1, kv_head, bs)
+    return attend(q_vec, K, V, scale)
+
+
+def paged_prefill(q, cu_q, k_cache, v_cache, block_tables, context_lens, scale):
+    """Chunked prefill over the paged cache: sequence b's new tokens are the
+    last c_b = cu_q[b+1] - cu_q[b] of its context_lens[b] positions (their K/V
+    already in the cache, behind a prefix that may come from a prefix cache
+    [bjdmk.com.cn/news/6246348, §4.1: the cached prefix's prefill is
+    skipped]); new token i sits at position context_lens[b] - c_b + i.
+
+    q [T, Hq, D] with T = cu_q[-1] (sequence-major); returns float64 [T, Hq, D].
+    """
+    T, Hq, D = q.shape
+    Hkv = k_cache.shape[1]
+    G = Hq // Hkv
+    out = np.zeros((T, Hq, D), dtype=np.float64)
+    for b in range(len(cu_q) - 1):
+        c = int(cu_q[b + 1] - cu_q[b])
+        L = int(context_lens[b])
+        for i in range(c):
+            pos = L - c + i
+            for h in range(Hq):
+                out[cu_q[b] + i, h] = prefill_one(q[cu_q[b] + i, h], k_cache, v_cache,
+                                                  block_tables[b], pos, h // G, scale)
+    return out

@@ -1272,10 +1272,10 @@ kv_status run_partition(kv_pool *pool, int32_t layer, const void *q, int32_t q_d
   }
   if (num_seqs == 0) return KV_OK;
   kv_status code;
-  const LayerMaps *maps = layer_maps(pool, layer, p.hg * pool->d.block_size, &code);
-  if (!maps) return code;
+  LayerMaps maps;
+  if (!layer_maps(pool, layer, p.hg * pool->d.block_size, &maps, &code)) return code;
   PartFn fn = pick_partition(pool->d.head_dim, pool->d.block_size, cd, q_dtype);
-  return cuda_check(fn(maps->k, maps->v, p, st), "paged attention launch");
+  return cuda_check(fn(maps.k, maps.v, p, st), "paged attention launch");
 }
 
 kv_status run_merge(kv_pool *pool, int32_t num_seqs, int32_t num_q_heads,

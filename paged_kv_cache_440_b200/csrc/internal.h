@@ -57,8 +57,8 @@ struct kv_pool {
   std::vector<int32_t> free_stack;  // free ids; the top is handed out next
   int32_t shared = 0;               // blocks with refcount >= 2
 
-  std::mutex map_mu;                // guards tensor-map creation
-  std::vector<pagedkv::LayerMaps> maps;
+  std::mutex map_mu;                // guards the tensor-map cache
+  std::vector<std::vector<pagedkv::LayerMaps>> maps;  // per layer, one per box height
 };
 
 namespace pagedkv {
@@ -106,8 +106,9 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
-// Tensor maps for the layer's K and V regions with boxes of box_rows rows;
-// nullptr + message on failure.
-const LayerMaps *layer_maps(kv_pool *p, int layer, int box_rows, kv_status *code);
+// Tensor maps for the layer's K and V regions with boxes of box_rows rows,
+// copied to *out (encoded on first use, then cached per box height); false +
+// message on failure.
+bool layer_maps(kv_pool *p, int layer, int box_rows, LayerMaps *out, kv_status *code);
 
 }  // namespace pagedkv

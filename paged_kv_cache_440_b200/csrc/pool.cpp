@@ -146,21 +146,28 @@ static bool encode_region(const kv_pool *p, void *base, int box_rows, CUtensorMa
   return true;
 }
 
-const LayerMaps *layer_maps(kv_pool *p, int layer, int box_rows, kv_status *code) {
+bool layer_maps(kv_pool *p, int layer, int box_rows, LayerMaps *out, kv_status *code) {
   std::lock_guard<std::mutex> g(p->map_mu);
-  LayerMaps &m = p->maps[layer];
-  if (m.box_rows != box_rows) {
-    std::string why;
-    m.box_rows = 0;
-    if (!encode_region(p, layer_k(p, layer), box_rows, &m.k, &why) ||
-        !encode_region(p, layer_v(p, layer), box_rows, &m.v, &why)) {
-      *code = fail(KV_ERR_CUDA, "tensor map for layer %d: %s", layer, why.c_str());
-      return nullptr;
+  std::vector<LayerMaps> &v = p->maps[layer];
+  for (const LayerMaps &m : v) {
+    if (m.box_rows == box_rows) {
+      *out = m;
+      *code = KV_OK;
+      return true;
     }
-    m.box_rows = box_rows;
   }
+  LayerMaps m;
+  std::string why;
+  if (!encode_region(p, layer_k(p, layer), box_rows, &m.k, &why) ||
+      !encode_region(p, layer_v(p, layer), box_rows, &m.v, &why)) {
+    *code = fail(KV_ERR_CUDA, "tensor map for layer %d: %s", layer, why.c_str());
+    return false;
+  }
+  m.box_rows = box_rows;
+  v.push_back(m);
+  *out = m;
   *code = KV_OK;
-  return &m;
+  return true;
 }
 
 }  // namespace pagedkv
