@@ -357,6 +357,32 @@ kv_status paged_attn_merge(kv_pool *pool, int32_t num_seqs, int32_t num_q_heads,
 
 /* ------------------------------------------------------------------------ */
 
+/* Chunked prefill over the paged cache. Sequence b's c_b = cu_q_lens[b+1] -
+ * cu_q_lens[b] new tokens are the last c_b of its context_lens[b] positions;
+ * their K/V rows must already be in the pool (kv_append at their slots),
+ * behind a prefix that may have come from the prefix cache. New token i of
+ * sequence b, at position context_lens[b] - c_b + i, attends to positions
+ * 0 .. context_lens[b] - c_b + i: every token sees the tokens before it and
+ * itself [KV Cache 原理与 PagedAttention, §一; bjdmk.com.cn/news/6246348, §4.1:
+ * a cached prefix's prefill is skipped].
+ *   q, out     device [total_q][num_q_heads][head_dim], the cache dtype
+ *              (16-bit caches only, else KV_ERR_UNSUPPORTED), 16-byte aligned,
+ *              sequences one after another (row cu_q_lens[b] + i).
+ *   cu_q_lens  device int32 [num_seqs + 1], non-decreasing, cu_q_lens[0] = 0,
+ *              cu_q_lens[num_seqs] = total_q; max_q_len >= every c_b (host).
+ *   Other arguments as paged_attn_decode. Up to 128 query heads per kv head.
+ * A sequence with c_b > context_lens[b], a length beyond the table, or rows
+ * outside [0, total_q) sets KV_DEVERR_CONTEXT and its rows are not written;
+ * an invalid block id sets KV_DEVERR_BLOCK_ID and its positions are skipped.
+ * One kernel launch; no workspace. */
+kv_status paged_attn_prefill(kv_pool *pool, int32_t layer, const void *q,
+                             int32_t q_dtype, int32_t num_seqs, int32_t num_q_heads,
+                             const int32_t *cu_q_lens, int32_t total_q,
+                             int32_t max_q_len, const int32_t *block_tables,
+                             int32_t max_blocks_per_seq, const int32_t *context_lens,
+                             int32_t max_context, float scale, void *out,
+                             kv_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Prefix cache (host only)                                                  */
 /*                                                                           */

@@ -9,7 +9,7 @@ _EXPORTS = (
     "KVPool", "PagedKVError", "PrefixCache", "default_ctas", "kv_append", "kv_block_copy",
     "kv_quantize", "make_workspace", "paged_attn_decode", "paged_attn_decode_append",
     "paged_attn_decode_static", "paged_attn_partition_append",
-    "paged_attn_merge",
+    "paged_attn_merge", "paged_attn_prefill",
     "paged_attn_partition", "required_bytes", "selftest_wait_timeout", "version",
     "workspace_bytes",
 )

@@ -54,6 +54,8 @@ class PrefixCacheStats(ctypes.Structure):
 _PI32 = ctypes.POINTER(ctypes.c_int32)
 
 _SIGS = {
+    "paged_attn_prefill": [_P, _I32, _P, _I32, _I32, _I32, _P, _I32, _I32, _P, _I32, _P, _I32,
+                           _F, _P, _P],
     "kv_prefix_cache_create": [_P, ctypes.POINTER(_P)],
     "kv_prefix_cache_destroy": [_P],
     "kv_prefix_match": [_P, _PI32, _I32, _I32, _PI32, _PI32, _PI32],
@@ -431,6 +433,28 @@ def paged_attn_partition(pool, layer, q, block_tables, context_lens, max_context
                                    _ptr(context_lens), max_context, float(scale), _ptr(out),
                                    num_ctas, _ptr(workspace), workspace.numel(),
                                    _stream(stream, pool.device)))
+    return out
+
+
+def paged_attn_prefill(pool, layer, q, cu_q_lens, max_q_len, block_tables, context_lens,
+                       max_context, scale, out=None, stream=None):
+    """Chunked prefill: q [T, Hq, D] (sequence-major rows, cu_q_lens [B+1]
+    int32 on the device); each new token attends to the positions up to its
+    own. The new tokens' K/V must already be in the pool."""
+    _need(q, "q", (torch.bfloat16, torch.float16), pool.device)
+    _need(cu_q_lens, "cu_q_lens", torch.int32, pool.device)
+    _need(block_tables, "block_tables", torch.int32, pool.device)
+    _need(context_lens, "context_lens", torch.int32, pool.device)
+    T, Hq, D = q.shape
+    B = context_lens.shape[0]
+    if cu_q_lens.shape[0] != B + 1 or block_tables.shape[0] != B:
+        raise ValueError("cu_q_lens must be [B+1] and block_tables [B, max_blocks]")
+    if out is None:
+        out = torch.empty_like(q)
+    check(lib.paged_attn_prefill(pool.handle, layer, _ptr(q), TORCH_CODES[q.dtype], B, Hq,
+                                 _ptr(cu_q_lens), T, max_q_len, _ptr(block_tables),
+                                 block_tables.shape[1], _ptr(context_lens), max_context,
+                                 float(scale), _ptr(out), _stream(stream, pool.device)))
     return out
 
 

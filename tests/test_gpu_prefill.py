@@ -1,0 +1,109 @@
+"""Chunked prefill on the GPU against the oracle (every output row)."""
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from gpu_support import bits16, build_pool, compare, device_inputs, oracle_cache_16, to_np
+from oracle import attention
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module")
+def pkv():
+    import paged_kv_cache_440_b200 as m
+    return m
+
+
+def _cache_16(wl):
+    dt = np.float16 if wl.cache_dtype == "fp16" else np.float32
+    return to_np(wl.k_fill, dt), to_np(wl.v_fill, dt)
+
+
+def _run(pkv, pw):
+    wl = pw.cache
+    pool = build_pool(pkv, wl, DEV)
+    tables, lens = device_inputs(wl, DEV)
+    cu = torch.from_numpy(pw.cu_q).to(DEV)
+    out = pkv.paged_attn_prefill(pool, 0, pw.q, cu, int(max(pw.chunk_lens.max(), 1)), tables,
+                                 lens, int(max(wl.context_lens.max(), 1)), wl.scale)
+    torch.cuda.synchronize()
+    return pool, out
+
+
+CASES = [
+    # name, Hq, Hkv, D, bs, dtype, lens, chunks
+    ("gqa-g8-d128-bs16", 16, 2, 128, 16, "bf16", [37, 300, 129, 64, 5], [37, 100, 1, 64, 2]),
+    ("mha-fp16-d64-bs32", 4, 4, 64, 32, "fp16", [50, 200, 33], [50, 17, 33]),
+    ("g8-d128-bs32-long", 8, 1, 128, 32, "bf16", [1000, 65], [300, 65]),
+    ("g16-d64-bs16", 32, 2, 64, 16, "bf16", [90, 17], [41, 17]),
+    ("g3-d128-bs16", 6, 2, 128, 16, "fp16", [70, 140], [70, 60]),
+    ("g64-d128-bs16", 64, 1, 128, 16, "bf16", [40, 3], [9, 3]),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
+def test_prefill_matches_oracle(pkv, case):
+    name, hq, hkv, D, bs, dt, lens, chunks = case
+    pw = W.make_prefill_workload(name, hq, hkv, D, bs, dt, lens, chunks, seed=11, device=DEV)
+    pool, out = _run(pkv, pw)
+    assert pool.status() == 0
+    k, v = _cache_16(pw.cache)
+    ref = attention.paged_prefill(to_np(pw.q, np.float64), pw.cu_q, k, v, pw.cache.block_tables,
+                                  pw.cache.context_lens, pw.cache.scale)
+    compare(out, ref, what=name)
+
+
+def test_prefill_last_token_agrees_with_decode(pkv):
+    """A one-token chunk is a decode step: both paths give the same output
+    within the tolerance (different kernels, different orders)."""
+    pw = W.make_prefill_workload("one", 16, 2, 128, 16, "bf16", [300, 45, 129], [1, 1, 1],
+                                 seed=12, device=DEV)
+    pool, out = _run(pkv, pw)
+    wl = pw.cache
+    tables, lens = device_inputs(wl, DEV)
+    dec = pkv.paged_attn_decode(pool, 0, pw.q.contiguous(), tables, lens,
+                                int(wl.context_lens.max()), wl.scale)
+    torch.cuda.synchronize()
+    diff = (out.float() - dec.float()).abs().max().item()
+    assert diff <= 1e-2
+
+
+def test_prefill_70b_shape_sampled(pkv):
+    """The 70B-shaped chunked-prefill workload (8 requests, 512 new tokens
+    behind a 1536-token prefix): sampled rows against the oracle."""
+    pw = W.prefill70b(DEV)
+    pool, out = _run(pkv, pw)
+    assert pool.status() == 0
+    wl = pw.cache
+    k, v = _cache_16(wl)
+    rows = [(b, i) for b in (0, 5, 7) for i in (0, 1, 15, 16, 255, 511)]
+    got = torch.stack([out[pw.cu_q[b] + i] for b, i in rows])
+    ref = np.stack([np.stack([attention.prefill_one(to_np(pw.q[pw.cu_q[b] + i, h], np.float64), k, v,
+                                                    wl.block_tables[b],
+                                                    int(wl.context_lens[b] - pw.chunk_lens[b] + i),
+                                                    h // 8, wl.scale)
+                              for h in range(64)]) for b, i in rows])
+    compare(got, ref, what="prefill70b")
+
+
+def test_prefill_bad_chunk_is_reported(pkv):
+    pw = W.make_prefill_workload("bad", 8, 2, 64, 16, "bf16", [40, 30], [10, 12], seed=13,
+                                 device=DEV)
+    wl = pw.cache
+    pool = build_pool(pkv, wl, DEV)
+    tables, lens = device_inputs(wl, DEV)
+    lens[1] = 5                                   # fewer positions than new tokens
+    cu = torch.from_numpy(pw.cu_q).to(DEV)
+    out = torch.full_like(pw.q, 7.0)
+    pool.status_clear()
+    pkv.paged_attn_prefill(pool, 0, pw.q, cu, 12, tables, lens, 40, wl.scale, out=out)
+    torch.cuda.synchronize()
+    assert pool.status() & 2
+    assert torch.all(out[10:] == 7.0)             # the bad sequence's rows are left alone
+    k, v = _cache_16(wl)
+    ref = attention.paged_prefill(to_np(pw.q[:10], np.float64), pw.cu_q[:2], k, v,
+                                  wl.block_tables[:1], wl.context_lens[:1], wl.scale)
+    compare(out[:10], ref, what="good sequence")

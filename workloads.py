@@ -245,3 +245,37 @@ CONFIGS = {
     "gqa70b": gqa70b,
     "mha13b": mha13b,
 }
+
+
+# ---------------------------------------------------------------------------
+# Chunked prefill: a decode-shaped 16-bit cache whose last c_b positions of
+# each sequence are that step's new tokens, plus their queries.
+# ---------------------------------------------------------------------------
+
+@dataclass
+class PrefillWorkload:
+    cache: DecodeWorkload        # k_fill / v_fill hold every position (new tokens included)
+    chunk_lens: np.ndarray       # int32 [B]: new tokens per sequence (<= context length)
+    cu_q: np.ndarray             # int32 [B + 1]
+    q: torch.Tensor              # [sum(chunk_lens), Hq, D], sequence-major
+
+
+def make_prefill_workload(name, q_heads, kv_heads, head_dim, block_size, dtype, lens, chunks,
+                          seed=0, device="cpu"):
+    cache = make_decode_workload(name, len(lens), q_heads, kv_heads, head_dim, block_size,
+                                 dtype, dtype, lens, seed=seed, device=device)
+    chunks = np.asarray(chunks, dtype=np.int32)
+    cu = np.concatenate([[0], np.cumsum(chunks)]).astype(np.int32)
+    gen = torch.Generator(device=device).manual_seed(seed + 7919)
+    q = torch.randn(int(cu[-1]), q_heads, head_dim, generator=gen, device=device,
+                    dtype=torch.float32).to(_TORCH_DT[dtype])
+    return PrefillWorkload(cache, chunks, cu, q)
+
+
+def prefill70b(device="cpu", seed=0, batch=8, prefix=1536, chunk=512):
+    """LLaMA-70B-shaped GQA layer (64/8 heads, D 128, bf16, bs 16): `batch`
+    requests each prefilling a `chunk`-token piece of the prompt behind a
+    `prefix`-token cached prefix (chunked prefill after a prefix-cache hit)."""
+    lens = [prefix + chunk] * batch
+    return make_prefill_workload("prefill70b", 64, 8, 128, 16, "bf16", lens, [chunk] * batch,
+                                 seed=seed, device=device)
