@@ -269,6 +269,162 @@ class SharedPrefixStep:
                                   for b in range(self.batch)], np.int64)
 
 
+# ------------------------------------------------------------------ prefill
+
+PREFILL_WORKLOADS = {
+    "prefill70b": ("LLaMA-70B-shaped GQA layer (64/8 heads, D 128, bf16, block 16): 8 requests "
+                   "each prefilling 512 new tokens behind a 1536-token cached prefix",
+                   lambda dev: W.prefill70b(dev)),
+}
+
+
+def prefill_flops(pw):
+    """Algorithmic FLOPs: each new token at position p and each query head does
+    q.K over p + 1 positions and P.V over them (2 FLOPs per multiply-add)."""
+    wl = pw.cache
+    tot = 0
+    for b in range(wl.batch):
+        L, c = int(wl.context_lens[b]), int(pw.chunk_lens[b])
+        tot += sum(L - c + i + 1 for i in range(c))
+    return 4 * wl.head_dim * wl.q_heads * tot
+
+
+def run_prefill(args, rank, world, device):
+    import paged_kv_cache_440_b200 as pkv
+    desc, make = PREFILL_WORKLOADS[args.workload]
+    pw = make(device)
+    wl = pw.cache
+    pool = pkv.KVPool(1, wl.num_blocks, wl.block_size, wl.kv_heads, wl.head_dim,
+                      wl.cache_dtype, device)
+    K, V, _, _ = pool.layer_views(0)
+    K.copy_(wl.k_fill)
+    V.copy_(wl.v_fill)
+    tables = torch.from_numpy(wl.block_tables).to(device)
+    lens = torch.from_numpy(wl.context_lens.astype(np.int32)).to(device)
+    cu = torch.from_numpy(pw.cu_q).to(device)
+    max_q, max_ctx = int(pw.chunk_lens.max()), int(wl.context_lens.max())
+    out = torch.empty_like(pw.q)
+    flush = torch.ones(64 << 20, dtype=torch.float32, device=device)
+    sink = torch.empty((), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(q=pw.q, tb=tables, ln=lens, c=cu, o=out):
+        pkv.paged_attn_prefill(pool, 0, q, c, max_q, tb, ln, max_ctx, wl.scale, out=o)
+
+    for _ in range(args.warmup):
+        torch.sum(flush, 0, out=sink)
+        step()
+    torch.cuda.synchronize(device)
+    pool.status_clear()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    sampler = ClockSampler(device.index if device.index is not None else 0).start()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    t0 = time.time()
+    for i in range(args.steps):
+        torch.sum(flush, 0, out=sink)
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize(device)
+    t1 = time.time()
+    sampler.stop()
+    step_s = float(np.mean([a.elapsed_time(b_) for a, b_ in evs])) / 1e3
+    step_s, = max_over_ranks([step_s], world, device)
+    e2e = None
+    if not args.no_e2e:
+        h_q = pw.q.cpu().pin_memory()
+        h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        d_q = torch.empty_like(pw.q)
+        times = []
+        for i in range(args.warmup + max(10, args.steps // 10)):
+            torch.sum(flush, 0, out=sink)
+            torch.cuda.synchronize(device)
+            a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            d_q.copy_(h_q, non_blocking=True)
+            step(q=d_q)
+            h_out.copy_(out, non_blocking=True)
+            b_.record(stream)
+            b_.synchronize()
+            if i >= args.warmup:
+                times.append(a.elapsed_time(b_) / 1e3)
+        e2e_s, = max_over_ranks([float(np.mean(times))], world, device)
+        e2e = (e2e_s, h_q.numel() * 2, h_out.numel() * 2)
+    return {"pw": pw, "desc": desc, "step_s": step_s, "clocks": sampler.summary(t0, t1),
+            "status": pool.status(), "e2e": e2e, "launches": args.steps}
+
+
+def prefill_oracle_sample(pw, budget_s):
+    """TFLOP/s of the fp64 oracle on a bounded sample of the prefill rows."""
+    from threadpoolctl import threadpool_info
+    from oracle import attention
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    wl = pw.cache
+    k = wl.k_fill.float().cpu().numpy()
+    v = wl.v_fill.float().cpu().numpy()
+    q = pw.q.float().cpu().numpy().astype(np.float64)
+    G = wl.q_heads // wl.kv_heads
+    flops, t, rows = 0, 0.0, 0
+    for b in range(wl.batch):
+        L, c = int(wl.context_lens[b]), int(pw.chunk_lens[b])
+        for i in range(0, c, 37):                     # a spread of positions
+            pos = L - c + i
+            t0 = time.perf_counter()
+            for h in range(wl.q_heads):
+                attention.prefill_one(q[pw.cu_q[b] + i, h], k, v, wl.block_tables[b], pos,
+                                      h // G, wl.scale)
+            t += time.perf_counter() - t0
+            flops += 4 * wl.head_dim * wl.q_heads * (pos + 1)
+            rows += 1
+            if t >= budget_s:
+                return flops / t / 1e12, t, rows, threads
+    return flops / t / 1e12, t, rows, threads
+
+
+def prefill_main(args, rank, world, device):
+    r = run_prefill(args, rank, world, device)
+    pw = r["pw"]
+    wl = pw.cache
+    flops = prefill_flops(pw) * world
+    tflops = flops / r["step_s"] / 1e12
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peak, kind = float(json.load(f)["bf16_tflops"]), "measured (MEASURED_PEAKS.json bf16_tflops, cuBLAS burst)"
+    except Exception:
+        peak, kind = 1590.0, "fallback 1590 TFLOP/s"
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, secs, rows, threads = prefill_oracle_sample(pw, args.cpu_budget)
+        cpu = {"value": round(v, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": "%d new-token rows (all 64 heads each), %.1f s of fp64 numpy" % (rows, secs)}
+    if rank == 0:
+        line = {
+            "metric": "chunked prefill attention TFLOP/s", "value": round(tflops, 2),
+            "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(r["step_s"] * 1e3, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": wl.cache_dtype, "data": "synthetic",
+            "config": {"workload": r["desc"], "batch": wl.batch, "new_tokens": int(pw.cu_q[-1]),
+                       "cached_tokens": int(wl.context_lens.sum()), "q_heads": wl.q_heads,
+                       "kv_heads": wl.kv_heads, "head_dim": wl.head_dim,
+                       "block_size": wl.block_size,
+                       "parallelism": "replicas" if world > 1 else "1 gpu",
+                       "l2": "L2 flushed before each timed step by reading 256 MiB"},
+            "roofline": {"bound": "tensor", "achieved": round(tflops / world, 2), "peak": peak,
+                         "unit": "TFLOP/s", "frac": round(tflops / world / peak, 4),
+                         "traffic": None, "kernel": "attn_prefill_kernel", "peak_source": kind,
+                         "kernel_ms": round(r["step_s"] * 1e3, 5)},
+            "cpu_baseline": cpu,
+            "e2e": None if r["e2e"] is None else {
+                "value": round(flops / r["e2e"][0] / 1e12, 2), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": r["e2e"][1], "d2h_bytes_per_step": r["e2e"][2]},
+            "gpu_launches": r["launches"], "clocks": r["clocks"], "device_status": r["status"],
+        }
+        print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------------------ ours
 
 def run_ours(args, rank, world, device):
@@ -425,7 +581,8 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="gqa70b")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(PREFILL_WORKLOADS),
+                    default="gqa70b")
     ap.add_argument("--ctas", type=int, default=0, help="CTAs of the attention kernel (0 = one per SM)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--separate-append", action="store_true",
@@ -443,7 +600,26 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
 
-    desc, make = WORKLOADS[args.workload]
+    if args.impl == "reference" and args.workload in PREFILL_WORKLOADS:
+        if rank == 0:
+            desc, make = PREFILL_WORKLOADS[args.workload]
+            pw = make("cpu")
+            v, secs, rows, threads = prefill_oracle_sample(pw, args.cpu_budget)
+            print(json.dumps({
+                "impl": "reference", "metric": "chunked prefill attention TFLOP/s",
+                "value": round(v, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": round(prefill_flops(pw) / (v * 1e12) * 1e3, 3),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": {"workload": desc, "batch": pw.cache.batch},
+                "cpu_baseline": {"value": round(v, 6), "unit": "TFLOP/s", "cores": threads,
+                                 "kind": "oracle",
+                                 "sample": "%d new-token rows, %.1f s" % (rows, secs)},
+                "e2e": {"value": round(v, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}), flush=True)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+    desc, make = WORKLOADS.get(args.workload, (None, None))
     if args.impl == "reference":
         if rank == 0:
             wl = make("cpu")
@@ -470,6 +646,12 @@ def main():
 
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
+    if args.workload in PREFILL_WORKLOADS:
+        prefill_main(args, rank, world, device)
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+        return
     r = run_ours(args, rank, world, device)
     wl = r["wl"]
     total_bytes = (r["dec_bytes"] + r["app_bytes"]) * world
