@@ -62,6 +62,8 @@ WORKLOADS = {
                      lambda dev: W.quant_long("int8", "b", dev)),
     "quant_b_e5m2": ("FP8-E5M2 per-token-head KV: 64/8 heads, head_dim 128, block 32, 8 x 32768",
                      lambda dev: W.quant_long("e5m2", "b", dev)),
+    "quant_a_e5m2_cast": ("FP8-E5M2 KV cast with no scale: 64/8 heads, head_dim 128, block 32, "
+                          "64 x 4096", lambda dev: W.quant_long("e5m2_cast", "a", dev)),
     "shared_prefix": ("Shared prompt: 200 requests, 1500-token prefix in 94 shared blocks (the last "
                       "copied on write per request), suffixes U[1,512], 64/8 heads, D 128, bf16, "
                       "block 16; GB/s counts logical bytes (the shared prefix is read from L2)",
@@ -101,12 +103,13 @@ def step_bytes(wl):
     e = elt_bytes(wl.cache_dtype)
     tokens = int(wl.context_lens.sum())
     kv = tokens * wl.kv_heads * wl.head_dim * 2 * e
-    if e == 1:
+    if wl.cache_dtype in ("int8", "e5m2"):
         kv += tokens * wl.kv_heads * 2 * 4                   # per-token-head scales
     q_out = 2 * wl.batch * wl.q_heads * wl.head_dim * 2
     rows = wl.batch * wl.kv_heads
     append = rows * wl.head_dim * 2 * 2 + wl.batch * 8        # read new K, V and slots
-    append += rows * wl.head_dim * 2 * e + (rows * 2 * 4 if e == 1 else 0)   # write rows
+    append += rows * wl.head_dim * 2 * e + \
+        (rows * 2 * 4 if wl.cache_dtype in ("int8", "e5m2") else 0)           # write rows
     return kv + q_out, append
 
 

@@ -65,7 +65,8 @@ typedef enum {
   KV_BF16 = 0,
   KV_FP16 = 1,
   KV_FP8_E5M2 = 2,         /* 1 sign, 5 exponent (bias 15), 2 mantissa bits     */
-  KV_INT8 = 3              /* two's complement, codes in [-127, 127]            */
+  KV_INT8 = 3,             /* two's complement, codes in [-127, 127]            */
+  KV_FP8_E5M2_CAST = 4     /* E5M2 codes cast from the values with no scale     */
 } kv_dtype;
 
 /* Bits of the device status word. */

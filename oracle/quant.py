@@ -100,10 +100,16 @@ def quantize_rows(x, kind):
 
     x: float32-representable values, shape [..., D]; each row of D values is one
        (token, kv head) of K or V.
-    kind: "int8" or "e5m2".
+    kind: "int8", "e5m2" or "e5m2_cast" (no scale).
     Returns (codes [..., D] int8|uint8, scales [...] float32).
     """
     x = np.asarray(x, dtype=np.float32)
+    if kind == "e5m2_cast":
+        # FP8 storage with no scale: each value cast to E5M2 (round to nearest
+        # even, saturating), dequantized as the code's value [KV Cache 原理与
+        # PagedAttention, §四: FP8 KV stored in FP8 and converted back before
+        # use; the vLLM example's fp8_e5m2 KV dtype]. Scales are reported as 1.
+        return e5m2_encode(x), np.ones(x.shape[:-1], dtype=np.float32)
     qmax = QMAX_INT8 if kind == "int8" else QMAX_E5M2
     a = np.max(np.abs(x), axis=-1)                            # exact in fp32
     scale = np.divide(a, qmax, dtype=np.float32)               # fl32(a / QMAX)
@@ -126,7 +132,7 @@ def dequantize(codes, scales, kind):
     """codes [..., D], scales [...] -> float64 values code * scale (exact in fp64)."""
     if kind == "int8":
         v = np.asarray(codes, dtype=np.int8).astype(np.float64)
-    elif kind == "e5m2":
+    elif kind in ("e5m2", "e5m2_cast"):
         v = e5m2_decode(codes)
     else:
         raise ValueError(kind)

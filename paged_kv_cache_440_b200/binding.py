@@ -22,13 +22,14 @@ lib = ctypes.CDLL(LIB_PATH)
 
 # ----------------------------------------------------------------- constants
 KV_OK, KV_ERR_INVALID, KV_ERR_OOM, KV_ERR_CUDA, KV_ERR_UNSUPPORTED = 0, 1, 2, 3, 4
-KV_BF16, KV_FP16, KV_FP8_E5M2, KV_INT8 = 0, 1, 2, 3
+KV_BF16, KV_FP16, KV_FP8_E5M2, KV_INT8, KV_FP8_E5M2_CAST = 0, 1, 2, 3, 4
 KV_DEVERR_BLOCK_ID, KV_DEVERR_CONTEXT, KV_DEVERR_SLOT, KV_DEVERR_TIMEOUT = 1, 2, 4, 8
 
-DTYPE_CODES = {"bf16": KV_BF16, "fp16": KV_FP16, "e5m2": KV_FP8_E5M2, "int8": KV_INT8}
+DTYPE_CODES = {"bf16": KV_BF16, "fp16": KV_FP16, "e5m2": KV_FP8_E5M2, "int8": KV_INT8,
+               "e5m2_cast": KV_FP8_E5M2_CAST}
 TORCH_CODES = {torch.bfloat16: KV_BF16, torch.float16: KV_FP16}
 CACHE_TORCH = {"bf16": torch.bfloat16, "fp16": torch.float16, "e5m2": torch.uint8,
-               "int8": torch.int8}
+               "int8": torch.int8, "e5m2_cast": torch.uint8}
 
 
 class PoolDesc(ctypes.Structure):
@@ -171,7 +172,7 @@ class KVPool:
     block_size = property(lambda s: s.desc.block_size)
     num_kv_heads = property(lambda s: s.desc.num_kv_heads)
     head_dim = property(lambda s: s.desc.head_dim)
-    quantized = property(lambda s: s.cache_dtype in ("int8", "e5m2"))
+    quantized = property(lambda s: s.cache_dtype in ("int8", "e5m2", "e5m2_cast"))
 
     def close(self):
         if getattr(self, "handle", None):

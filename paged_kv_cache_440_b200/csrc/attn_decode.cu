@@ -111,13 +111,14 @@ struct Tile {
   static constexpr int kRowBytes = D * kElt;
   static constexpr int kSlab = kRowBytes >= 128 ? 128 : kRowBytes;  // TMA box width, bytes
   static constexpr int kSlabs = kRowBytes / kSlab;
-  static constexpr bool kQuant = !is16<KV_T>();
+  static constexpr bool kQuant = !is16<KV_T>();                 // 1-byte codes
+  static constexpr bool kScaled = kQuant && KV_T != KV_FP8_E5M2_CAST;  // with fp32 scales
 
   // A stage holds `rows` = HG * BS rows (HG heads of one block) of K, then of
   // V, each as kSlabs slabs of rows x kSlab bytes, then (quantized caches) the
   // K and V scales of those rows.
   __host__ __device__ static constexpr int load_bytes(int rows) {
-    return 2 * rows * kRowBytes + (kQuant ? 2 * rows * 4 : 0);
+    return 2 * rows * kRowBytes + (kScaled ? 2 * rows * 4 : 0);
   }
 
   // Shared-memory address of 16-byte chunk c of row r of the K (or V) part of
@@ -154,7 +155,7 @@ __device__ __forceinline__ void issue_stage(uint8_t *stage, uint64_t *bar, const
     tma_load_2d(stage + s * rows * T::kSlab, km, bar, s * (T::kSlab / T::kElt), row0);
     tma_load_2d(stage + kv + s * rows * T::kSlab, vm, bar, s * (T::kSlab / T::kElt), row0);
   }
-  if constexpr (T::kQuant) {
+  if constexpr (T::kScaled) {
     bulk_load(stage + 2 * kv, p.k_scale + row0, rows * 4, bar);
     bulk_load(stage + 2 * kv + rows * 4, p.v_scale + row0, rows * 4, bar);
   }
@@ -280,7 +281,8 @@ __device__ __forceinline__ bool ring_wait(uint64_t *bar, uint32_t parity, volati
 template <int D, int BS, int KV_T, int Q_T>
 struct Consumer {
   using T = Tile<D, BS, KV_T>;
-  static constexpr bool kQuant = T::kQuant;
+  static constexpr bool kQuant = T::kQuant;    // 1-byte codes (fp16 MMA, scaled q)
+  static constexpr bool kScaled = T::kScaled;  // per-token-head scales
   static constexpr bool kBF = (KV_T == KV_BF16);  // MMA operand type (bf16, else fp16)
   static constexpr int KS = D / 16;  // k-steps over head_dim
   static constexpr int MT = BS / 16;  // 16-token tiles per block
@@ -412,7 +414,7 @@ struct Consumer {
       // acc: [0],[1] = token mt*16+gq, heads 2cq, 2cq+1; [2],[3] = token +8
       const int t0 = mt * 16 + gq, t1 = t0 + 8;
       float k0 = 1.f, k1 = 1.f;
-      if constexpr (kQuant) {
+      if constexpr (kScaled) {
         k0 = ksc[t0];
         k1 = ksc[t1];
       }
@@ -447,7 +449,7 @@ struct Consumer {
     // weights for P V: exp2(s - m) (16-bit), exp2(s + log2 sv - m2) (quant)
     float w[MT][4];
     float be0 = 1.f, be1 = 1.f;  // O rescale factors
-    if constexpr (!kQuant) {
+    if constexpr (!kScaled) {
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
         w[mt][0] = ex2_sfu(sc[mt][0] - mn0);
@@ -589,7 +591,7 @@ struct Consumer {
       l_run[i] += __shfl_xor_sync(0xffffffffu, l_run[i], 16);
     }
     float f[2] = {alive ? 1.f : 0.f, alive ? 1.f : 0.f};
-    if constexpr (kQuant) {
+    if constexpr (kScaled) {
 #pragma unroll
       for (int i = 0; i < 2; ++i)
         f[i] = (m2_run[i] == -INFINITY || !alive) ? 0.f : exp2f(m2_run[i] - m_run[i]);
@@ -644,6 +646,7 @@ template <int D, int BS, int KV_T, int Q_T>
 struct NewRow {
   static constexpr int E = D / 32;
   static constexpr bool kQuant = !is16<KV_T>();
+  static constexpr bool kScaled = Tile<D, BS, KV_T>::kScaled;
   uint32_t k[2], v[2];  // 16-bit: E * 2 bytes; 1-byte: E codes in k[0] / v[0]
   float ks, vs;
 
@@ -701,7 +704,7 @@ struct NewRow {
       *reinterpret_cast<uint16_t *>(kg) = static_cast<uint16_t>(k[0]);
       *reinterpret_cast<uint16_t *>(vg) = static_cast<uint16_t>(v[0]);
     }
-    if constexpr (kQuant) {
+    if constexpr (kScaled) {
       if (lane == 0) {
         float *sc = reinterpret_cast<float *>(st + 2 * rows * T::kRowBytes);
         sc[r] = ks;
@@ -1076,9 +1079,12 @@ PartFn pick_dtype(int kv, int q) {
     case KV_FP16: return launch_part<D, BS, KV_FP16, KV_FP16>;
     case KV_INT8:
       return q == KV_BF16 ? launch_part<D, BS, KV_INT8, KV_BF16> : launch_part<D, BS, KV_INT8, KV_FP16>;
-    default:
+    case KV_FP8_E5M2:
       return q == KV_BF16 ? launch_part<D, BS, KV_FP8_E5M2, KV_BF16>
                           : launch_part<D, BS, KV_FP8_E5M2, KV_FP16>;
+    default:
+      return q == KV_BF16 ? launch_part<D, BS, KV_FP8_E5M2_CAST, KV_BF16>
+                          : launch_part<D, BS, KV_FP8_E5M2_CAST, KV_FP16>;
   }
 }
 
@@ -1117,7 +1123,7 @@ UnitGeom unit_geom(const kv_pool *pool, int num_q_heads) {
   u.cgroups = (u.chunks + u.cpg - 1) / u.cpg;
   const int elt = elem_bytes(d.cache_dtype);
   const int row_bytes = d.head_dim * elt;
-  const bool quant = is_quant(d.cache_dtype);
+  const bool quant = has_scales(d.cache_dtype);  // scale rows ride with the stage
   auto load = [&](int hg) { return 2 * hg * d.block_size * (row_bytes + (quant ? 4 : 0)); };
   // the largest group of kv heads (a divisor of Hkv) with one slot per consumer
   // warp, a stage of at most kMaxStageBytes and a TMA box of at most 256 rows

@@ -96,11 +96,11 @@ append_quant_kernel(const uint16_t *__restrict__ k_new, const uint16_t *__restri
   load_row<D, IN_T>(k_new + src_row * D, lane, x);
   uint32_t packed = quantize_row<D, OUT_T>(x, &scale);
   store_codes<D>(kc + dst_row * D, lane, packed);
-  if (lane == 0) ks[dst_row] = scale;
+  if (OUT_T != KV_FP8_E5M2_CAST && lane == 0) ks[dst_row] = scale;
   load_row<D, IN_T>(v_new + src_row * D, lane, x);
   packed = quantize_row<D, OUT_T>(x, &scale);
   store_codes<D>(vc + dst_row * D, lane, packed);
-  if (lane == 0) vs[dst_row] = scale;
+  if (OUT_T != KV_FP8_E5M2_CAST && lane == 0) vs[dst_row] = scale;
 }
 
 // Standalone: one warp per contiguous row.
@@ -231,10 +231,14 @@ kv_status kv_append(kv_pool *pool, int32_t layer, const void *k_new, const void 
     e = in_dtype == KV_BF16
             ? dispatch_append_quant_d<KV_BF16, KV_INT8>(pool, layer, k_new, v_new, slot_mapping, num_tokens, st)
             : dispatch_append_quant_d<KV_FP16, KV_INT8>(pool, layer, k_new, v_new, slot_mapping, num_tokens, st);
-  } else {
+  } else if (cd == KV_FP8_E5M2) {
     e = in_dtype == KV_BF16
             ? dispatch_append_quant_d<KV_BF16, KV_FP8_E5M2>(pool, layer, k_new, v_new, slot_mapping, num_tokens, st)
             : dispatch_append_quant_d<KV_FP16, KV_FP8_E5M2>(pool, layer, k_new, v_new, slot_mapping, num_tokens, st);
+  } else {  // scale-less cast
+    e = in_dtype == KV_BF16
+            ? dispatch_append_quant_d<KV_BF16, KV_FP8_E5M2_CAST>(pool, layer, k_new, v_new, slot_mapping, num_tokens, st)
+            : dispatch_append_quant_d<KV_FP16, KV_FP8_E5M2_CAST>(pool, layer, k_new, v_new, slot_mapping, num_tokens, st);
   }
   kv_status s = cuda_check(e, "kv_append launch");
   return s == KV_OK ? ok() : s;
@@ -292,7 +296,7 @@ kv_status kv_block_copy(kv_pool *pool, const int32_t *host_pairs, int32_t n_pair
   const kv_pool_desc &dd = pool->d;
   const uint32_t kv_block = (uint32_t)dd.num_kv_heads * dd.block_size * pool->row_bytes;
   const uint32_t sc_block = (uint32_t)dd.num_kv_heads * dd.block_size * sizeof(float);
-  const int regions = is_quant(dd.cache_dtype) ? 4 : 2;
+  const int regions = has_scales(dd.cache_dtype) ? 4 : 2;
   cudaStream_t st = (cudaStream_t)stream;
   for (int32_t base = 0; base < n_pairs; base += kMaxPairsPerLaunch) {
     const int32_t n = std::min<int32_t>(kMaxPairsPerLaunch, n_pairs - base);

@@ -257,6 +257,15 @@ __device__ __forceinline__ float to_f32(uint16_t bits) {
 template <int D, int OUT_T>
 __device__ __forceinline__ uint32_t quantize_row(const float (&x)[D / 32], float *scale_out) {
   constexpr int E = D / 32;
+  if constexpr (OUT_T == KV_FP8_E5M2_CAST) {  // plain cast: no scale, saturating RNE
+    uint32_t packed = 0;
+#pragma unroll
+    for (int i = 0; i < E; ++i)
+      packed |= static_cast<uint32_t>(__nv_cvt_float_to_fp8(x[i], __NV_SATFINITE, __NV_E5M2))
+                << (8 * i);
+    *scale_out = 1.f;
+    return packed;
+  }
   float a = 0.f;
 #pragma unroll
   for (int i = 0; i < E; ++i) a = fmaxf(a, fabsf(x[i]));

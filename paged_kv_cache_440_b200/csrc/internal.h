@@ -20,7 +20,12 @@ constexpr int32_t kDevErrTimeout = 8;
 inline int elem_bytes(int dtype) {
   return (dtype == KV_BF16 || dtype == KV_FP16) ? 2 : 1;
 }
-inline bool is_quant(int dtype) { return dtype == KV_INT8 || dtype == KV_FP8_E5M2; }
+// 1-byte codes (read through the code paths of the kernels)
+inline bool is_quant(int dtype) {
+  return dtype == KV_INT8 || dtype == KV_FP8_E5M2 || dtype == KV_FP8_E5M2_CAST;
+}
+// codes with a per-token-head fp32 scale (scale regions in the pool)
+inline bool has_scales(int dtype) { return dtype == KV_INT8 || dtype == KV_FP8_E5M2; }
 inline uint64_t round_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
 
 // Byte offsets of one layer's regions inside the pool buffer.

@@ -60,8 +60,8 @@ bool compute_layout(const kv_pool_desc &d, Layout *out, std::string *why,
     *why = "head_dim must be 64 or 128";
     return false;
   }
-  if (d.cache_dtype < KV_BF16 || d.cache_dtype > KV_INT8) {
-    *why = "cache_dtype must be KV_BF16, KV_FP16, KV_FP8_E5M2 or KV_INT8";
+  if (d.cache_dtype < KV_BF16 || d.cache_dtype > KV_FP8_E5M2_CAST) {
+    *why = "cache_dtype must be KV_BF16, KV_FP16, KV_FP8_E5M2, KV_INT8 or KV_FP8_E5M2_CAST";
     return false;
   }
   const uint64_t rows = (uint64_t)d.num_blocks * d.num_kv_heads * d.block_size;
@@ -73,7 +73,7 @@ bool compute_layout(const kv_pool_desc &d, Layout *out, std::string *why,
   Layout L;
   L.kv_bytes = rows * d.head_dim * elem_bytes(d.cache_dtype);
   L.kv_stride = round_up(L.kv_bytes, 256);
-  L.sc_bytes = is_quant(d.cache_dtype) ? rows * sizeof(float) : 0;
+  L.sc_bytes = has_scales(d.cache_dtype) ? rows * sizeof(float) : 0;
   L.sc_stride = round_up(L.sc_bytes, 256);
   L.layer_stride = 2 * L.kv_stride + 2 * L.sc_stride;
   L.status_off = L.layer_stride * (uint64_t)d.num_layers;

@@ -52,7 +52,8 @@ def build_pool(pkv, wl, device, chunk=65536):
     else:
         # rows no append writes compare against the oracle's zeros
         for t in (K, V, KS, VS):
-            t.zero_()
+            if t is not None:                     # the scale-less cast has no scales
+                t.zero_()
         slots = torch.from_numpy(wl.slot_hist).to(device)
         for s in range(0, wl.k_hist.shape[0], chunk):
             pkv.kv_append(pool, 0, wl.k_hist[s:s + chunk].contiguous(),

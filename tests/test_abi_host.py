@@ -48,7 +48,8 @@ def _ptrs(h, layer):
     return k.value, v.value, ks.value, vs.value
 
 
-@pytest.mark.parametrize("dt,elt", [("bf16", 2), ("fp16", 2), ("int8", 1), ("e5m2", 1)])
+@pytest.mark.parametrize("dt,elt", [("bf16", 2), ("fp16", 2), ("int8", 1), ("e5m2", 1),
+                                    ("e5m2_cast", 1)])
 @pytest.mark.parametrize("layers,NB,bs,hkv,D", [(80, 37, 16, 8, 128), (1, 5, 32, 3, 64)])
 def test_layout_matches_kv_formula(dt, elt, layers, NB, bs, hkv, D):
     h, total = _make_pool(NB, layers, bs, hkv, D, dt)

@@ -88,7 +88,7 @@ def test_quantize_bit_exact(pkv, kind, in_dt, D):
     assert np.array_equal(codes.cpu().numpy(), ref_codes)
 
 
-@pytest.mark.parametrize("cache", ["bf16", "int8", "e5m2"])
+@pytest.mark.parametrize("cache", ["bf16", "int8", "e5m2", "e5m2_cast"])
 def test_block_copy_bit_exact(pkv, cache):
     """Shared-prefix shapes: 200 copy-on-write pairs, 3 layers, random pool bytes."""
     layers, NB, bs, hkv, D = 3, 1500, 16, 8, 128
@@ -118,3 +118,29 @@ def test_bounded_wait_gives_up_and_reports(pkv):
     # the context is still usable afterwards
     y = torch.ones(4, device=DEV) * 2
     assert float(y.sum()) == 8.0
+
+
+@pytest.mark.parametrize("in_dt", [torch.bfloat16, torch.float16])
+def test_append_scale_less_e5m2_bit_exact(pkv, in_dt):
+    """FP8 storage without a scale: each value's own E5M2 code (saturating RNE)
+    lands in its slot, and the pool has no scale regions."""
+    NB, bs, hkv, D, T = 64, 16, 4, 128, 300
+    pool = pkv.KVPool(1, NB, bs, hkv, D, "e5m2_cast", DEV)
+    K, V, KS, VS = pool.layer_views(0)
+    assert KS is None and VS is None
+    K.zero_()
+    V.zero_()
+    g = torch.Generator(device=DEV).manual_seed(5)
+    k = (torch.randn(T, hkv, D, generator=g, device=DEV) * 30).clamp(-6e4, 6e4).to(in_dt)
+    v = (torch.randn(T, hkv, D, generator=g, device=DEV) * 1e-3).to(in_dt)
+    slots = torch.randperm(NB * bs, generator=torch.Generator().manual_seed(6))[:T].to(DEV)
+    pkv.kv_append(pool, 0, k, v, slots)
+    torch.cuda.synchronize()
+    kc = np.zeros((NB, hkv, bs, D), np.uint8)
+    vc = np.zeros_like(kc)
+    ks = np.zeros((NB, hkv, bs), np.float32)
+    vs = np.zeros_like(ks)
+    cache_ops.append_quantized(kc, vc, ks, vs, to_np(k), to_np(v), slots.cpu().numpy(), bs,
+                               "e5m2_cast")
+    assert np.array_equal(K.cpu().numpy(), kc)
+    assert np.array_equal(V.cpu().numpy(), vc)

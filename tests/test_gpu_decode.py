@@ -190,7 +190,7 @@ def test_shared_prefix_copy_on_write(pkv):
 EDGE_LENS = [0, 1, 15, 16, 17, 63, 64, 65, 127, 128, 129, 300]
 
 
-@pytest.mark.parametrize("cache", ["bf16", "fp16", "int8", "e5m2"])
+@pytest.mark.parametrize("cache", ["bf16", "fp16", "int8", "e5m2", "e5m2_cast"])
 @pytest.mark.parametrize("G", [1, 2, 4, 8, 16])
 @pytest.mark.parametrize("D,bs", [(64, 16), (128, 32)])
 def test_edge_lengths_groups_dims(pkv, cache, G, D, bs):
@@ -265,6 +265,8 @@ def _fused_workloads():
                                                 [1, 31, 32, 300], seed=5, device=DEV)),
         ("e5m2", lambda: W.make_decode_workload("e5", 4, 16, 2, 128, 16, "bf16", "e5m2",
                                                 [2, 17, 64, 129], seed=6, device=DEV)),
+        ("e5m2-cast", lambda: W.make_decode_workload("e5c", 4, 16, 2, 64, 32, "fp16", "e5m2_cast",
+                                                     [3, 32, 33, 200], seed=8, device=DEV)),
     ]
 
 
@@ -295,8 +297,9 @@ def test_fused_append_matches_oracle(pkv, name, make, num_ctas):
                        for x in wl.block_tables[b, :-(-int(wl.context_lens[b]) // wl.block_size)]})
         assert np.array_equal(K[used].cpu().numpy(), kc[used])
         assert np.array_equal(V[used].cpu().numpy(), vc[used])
-        assert np.array_equal(KS[used].cpu().numpy().view(np.uint32), ks[used].view(np.uint32))
-        assert np.array_equal(VS[used].cpu().numpy().view(np.uint32), vs[used].view(np.uint32))
+        if KS is not None:                       # the scale-less cast keeps no scales
+            assert np.array_equal(KS[used].cpu().numpy().view(np.uint32), ks[used].view(np.uint32))
+            assert np.array_equal(VS[used].cpu().numpy().view(np.uint32), vs[used].view(np.uint32))
     ref = oracle_outputs(wl, k, v, pairs, tab)
     compare(torch.stack([out[b, h] for b, h in pairs]), ref, what="fused append " + name)
 

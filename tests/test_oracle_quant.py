@@ -140,3 +140,19 @@ def test_zero_row_and_dequantize_exact():
         # the row's absmax maps to -QMAX; its dequantized value is -QMAX * scale
         assert deq[1, 3] == -qmax * float(scale[1])
         assert abs(deq[1, 3] + 2.5) <= 2.5 * 2.0 ** -23
+
+
+def test_scale_less_e5m2_cast_is_the_plain_encoding():
+    """The scale-less FP8 variant stores each value's own E5M2 code: codes of
+    exactly representable values decode to themselves, larger values saturate
+    to the largest finite code, and the scale is 1."""
+    exact = np.array([[1.0, -1.25, 57344.0, 2.0 ** -16, 0.0, -3.0 * 2.0 ** -15, 1.5, -96.0]],
+                     dtype=np.float32)
+    codes, scales = quant.quantize_rows(exact, "e5m2_cast")
+    assert scales.tolist() == [1.0]
+    np.testing.assert_array_equal(quant.dequantize(codes, scales, "e5m2_cast"), exact)
+    big, _ = quant.quantize_rows(np.array([[1e6, -7e4, 60000.0, 0.1]], np.float32), "e5m2_cast")
+    assert big[0, :3].tolist() == [0x7B, 0xFB, 0x7B]
+    # 0.1 lies between 0.09375 (0x2E) and 0.109375 (0x2F): 0.00625 above the
+    # first, 0.009375 below the second
+    assert big[0, 3] == 0x2E
