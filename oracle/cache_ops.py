@@ -40,11 +40,14 @@ def append_quantized(k_codes, v_codes, k_scales, v_scales, k_new, v_new,
                      slot_mapping, block_size, kind):
     """Quantize each new (token, head) row, then place codes and scales by slot.
 
-    k_codes, v_codes [NB, Hkv, bs, D]; k_scales, v_scales [NB, Hkv, bs] float32;
+    k_codes, v_codes [NB, Hkv, bs, D] ([..., D/2] packed bytes for INT4);
+    k_scales, v_scales [NB, Hkv, bs] float32;
     k_new, v_new [T, Hkv, D] float32-representable values.
     """
     kc, ks = quant.quantize_rows(k_new, kind)
     vc, vs = quant.quantize_rows(v_new, kind)
+    if kind == "int4":                    # the cache holds two codes per byte
+        kc, vc = quant.pack_int4(kc), quant.pack_int4(vc)
     for i, slot in enumerate(np.asarray(slot_mapping).tolist()):
         if slot < 0:
             continue

@@ -27,6 +27,7 @@ Inf/NaN), working on the raw fp32 bits.
 import numpy as np
 
 QMAX_INT8 = np.float32(127.0)
+QMAX_INT4 = np.float32(7.0)
 QMAX_E5M2 = np.float32(57344.0)       # (1 + 3/4) * 2**15
 E5M2_MAX_CODE = 0x7B                  # exponent field 30, mantissa 3
 
@@ -95,12 +96,39 @@ def int8_encode(y):
     return np.clip(r, -127, 127).astype(np.int8)
 
 
+def int4_encode(y):
+    """float32 value(s) -> 4-bit codes (held in int8): round half to even,
+    clamp to [-7, 7] (symmetric; -8 is not used)."""
+    y = np.asarray(y, dtype=np.float32)
+    return np.clip(np.rint(y.astype(np.float64)), -7, 7).astype(np.int8)
+
+
+def pack_int4(codes):
+    """[..., D] codes in [-8, 7] -> [..., D/2] bytes: element 2i in the low
+    nibble of byte i, element 2i+1 in the high nibble (two's complement)."""
+    c = np.asarray(codes, dtype=np.int64) & 0xF
+    return (c[..., 0::2] | (c[..., 1::2] << 4)).astype(np.uint8)
+
+
+def unpack_int4(packed):
+    """Inverse of pack_int4: [..., D/2] bytes -> [..., D] int8 codes."""
+    b = np.asarray(packed, dtype=np.uint8).astype(np.int64)
+    lo, hi = b & 0xF, b >> 4
+    lo = np.where(lo >= 8, lo - 16, lo)
+    hi = np.where(hi >= 8, hi - 16, hi)
+    out = np.empty(b.shape[:-1] + (2 * b.shape[-1],), dtype=np.int8)
+    out[..., 0::2] = lo
+    out[..., 1::2] = hi
+    return out
+
+
 def quantize_rows(x, kind):
     """Per-row symmetric absmax quantization.
 
     x: float32-representable values, shape [..., D]; each row of D values is one
        (token, kv head) of K or V.
-    kind: "int8", "e5m2" or "e5m2_cast" (no scale).
+    kind: "int8", "int4" (codes unpacked, one per int8), "e5m2" or
+    "e5m2_cast" (no scale).
     Returns (codes [..., D] int8|uint8, scales [...] float32).
     """
     x = np.asarray(x, dtype=np.float32)
@@ -110,7 +138,10 @@ def quantize_rows(x, kind):
         # PagedAttention, §四: FP8 KV stored in FP8 and converted back before
         # use; the vLLM example's fp8_e5m2 KV dtype]. Scales are reported as 1.
         return e5m2_encode(x), np.ones(x.shape[:-1], dtype=np.float32)
-    qmax = QMAX_INT8 if kind == "int8" else QMAX_E5M2
+    # INT4 KV (the pages' most aggressive row, 1/4 of the memory [KV Cache
+    # 原理与 PagedAttention, §四 table]): the same per-token-head absmax form
+    # with QMAX 7; the pages' calibration needs data and is not modelled.
+    qmax = {"int8": QMAX_INT8, "int4": QMAX_INT4}.get(kind, QMAX_E5M2)
     a = np.max(np.abs(x), axis=-1)                            # exact in fp32
     scale = np.divide(a, qmax, dtype=np.float32)               # fl32(a / QMAX)
     nz = scale > 0
@@ -118,6 +149,9 @@ def quantize_rows(x, kind):
     y = np.divide(x, safe[..., None], dtype=np.float32)        # fl32(x / scale)
     if kind == "int8":
         codes = int8_encode(y)
+        codes = np.where(nz[..., None], codes, np.int8(0)).astype(np.int8)
+    elif kind == "int4":
+        codes = int4_encode(y)
         codes = np.where(nz[..., None], codes, np.int8(0)).astype(np.int8)
     elif kind == "e5m2":
         codes = e5m2_encode(y)
@@ -130,7 +164,7 @@ def quantize_rows(x, kind):
 
 def dequantize(codes, scales, kind):
     """codes [..., D], scales [...] -> float64 values code * scale (exact in fp64)."""
-    if kind == "int8":
+    if kind in ("int8", "int4"):
         v = np.asarray(codes, dtype=np.int8).astype(np.float64)
     elif kind in ("e5m2", "e5m2_cast"):
         v = e5m2_decode(codes)

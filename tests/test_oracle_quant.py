@@ -94,13 +94,15 @@ def test_int8_round_half_even_definition():
 def test_hand_derived_rows():
     with open(GOLDEN) as f:
         g = json.load(f)
-    for kind in ("int8", "e5m2"):
+    for kind in ("int8", "e5m2", "int4"):
         for case in g[kind]:
             x = np.array(case["x"], dtype=np.float32)[None, :]
             codes, scale = quant.quantize_rows(x, kind)
             assert scale[0] == np.float32(case["scale"]), case["why"]
-            got = codes[0].astype(np.int64) if kind == "int8" else codes[0].astype(np.int64)
+            got = codes[0].astype(np.int64)
             assert list(got) == case["codes"], case["why"]
+            if kind == "int4":
+                assert list(quant.pack_int4(codes)[0]) == case["packed"], case["why"]
 
 
 def test_quantize_rows_bounds():
@@ -156,3 +158,21 @@ def test_scale_less_e5m2_cast_is_the_plain_encoding():
     # 0.1 lies between 0.09375 (0x2E) and 0.109375 (0x2F): 0.00625 above the
     # first, 0.009375 below the second
     assert big[0, 3] == 0x2E
+
+
+def test_int4_bounds_and_packing():
+    rng = np.random.default_rng(14)
+    x = (rng.standard_normal((4096, 128)) * rng.uniform(0.01, 100, (4096, 1))).astype(np.float32)
+    codes, scale = quant.quantize_rows(x, "int4")
+    a = np.abs(x).max(axis=1)
+    assert np.array_equal(scale, (a / np.float32(7.0)).astype(np.float32))
+    assert codes.min() >= -7 and codes.max() <= 7
+    # the row's largest magnitude maps to +-7; everything within half a step
+    idx = np.abs(x).argmax(axis=1)
+    assert np.all(np.abs(codes[np.arange(4096), idx].astype(int)) == 7)
+    err = np.abs(quant.dequantize(codes, scale, "int4") - x.astype(np.float64))
+    assert np.all(err <= scale[:, None].astype(np.float64) * (0.5 + 7 * 2.0 ** -23))
+    # packing round-trips every code pair, including -8
+    allc = np.array([[a, b] for a in range(-8, 8) for b in range(-8, 8)], dtype=np.int8)
+    assert np.array_equal(quant.unpack_int4(quant.pack_int4(allc)), allc)
+    assert quant.pack_int4(allc).shape == (256, 1) and len(set(quant.pack_int4(allc)[:, 0])) == 256
