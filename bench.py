@@ -62,6 +62,8 @@ WORKLOADS = {
                      lambda dev: W.quant_long("int8", "b", dev)),
     "quant_b_e5m2": ("FP8-E5M2 per-token-head KV: 64/8 heads, head_dim 128, block 32, 8 x 32768",
                      lambda dev: W.quant_long("e5m2", "b", dev)),
+    "quant_a_int4": ("INT4 per-token-head KV (two codes per byte): 64/8 heads, head_dim 128, "
+                     "block 32, 64 x 4096", lambda dev: W.quant_long("int4", "a", dev)),
     "quant_a_e5m2_cast": ("FP8-E5M2 KV cast with no scale: 64/8 heads, head_dim 128, block 32, "
                           "64 x 4096", lambda dev: W.quant_long("e5m2_cast", "a", dev)),
     "shared_prefix": ("Shared prompt: 200 requests, 1500-token prefix in 94 shared blocks (the last "
@@ -80,7 +82,7 @@ def measured_peak():
 
 
 def elt_bytes(cache):
-    return 2 if cache in ("bf16", "fp16") else 1
+    return 2 if cache in ("bf16", "fp16") else 0.5 if cache == "int4" else 1
 
 
 def max_over_ranks(values, world, device):
@@ -103,14 +105,14 @@ def step_bytes(wl):
     e = elt_bytes(wl.cache_dtype)
     tokens = int(wl.context_lens.sum())
     kv = tokens * wl.kv_heads * wl.head_dim * 2 * e
-    if wl.cache_dtype in ("int8", "e5m2"):
+    if wl.cache_dtype in ("int8", "e5m2", "int4"):
         kv += tokens * wl.kv_heads * 2 * 4                   # per-token-head scales
     q_out = 2 * wl.batch * wl.q_heads * wl.head_dim * 2
     rows = wl.batch * wl.kv_heads
     append = rows * wl.head_dim * 2 * 2 + wl.batch * 8        # read new K, V and slots
     append += rows * wl.head_dim * 2 * e + \
-        (rows * 2 * 4 if wl.cache_dtype in ("int8", "e5m2") else 0)           # write rows
-    return kv + q_out, append
+        (rows * 2 * 4 if wl.cache_dtype in ("int8", "e5m2", "int4") else 0)   # write rows
+    return int(kv + q_out), int(append)
 
 
 # ------------------------------------------------------------------ clocks

@@ -66,7 +66,9 @@ typedef enum {
   KV_FP16 = 1,
   KV_FP8_E5M2 = 2,         /* 1 sign, 5 exponent (bias 15), 2 mantissa bits     */
   KV_INT8 = 3,             /* two's complement, codes in [-127, 127]            */
-  KV_FP8_E5M2_CAST = 4     /* E5M2 codes cast from the values with no scale     */
+  KV_FP8_E5M2_CAST = 4,    /* E5M2 codes cast from the values with no scale     */
+  KV_INT4 = 5              /* 4-bit codes in [-7, 7], two per byte (element 2i  */
+                           /* in the low nibble), head_dim 128 only             */
 } kv_dtype;
 
 /* Bits of the device status word. */
@@ -182,8 +184,10 @@ kv_status kv_pool_stats(const kv_pool *pool, int32_t *used, int32_t *free_,
  *   skips it and sets KV_DEVERR_SLOT. Slots must be distinct (duplicates race).
  * 16-bit caches: in_dtype must equal the cache dtype; the rows are copied
  *   bit for bit.
- * INT8 / E5M2 caches: each (token, head) row x of head_dim values is
+ * INT8 / E5M2 / INT4 caches: each (token, head) row x of head_dim values is
  *   quantized as kv_quantize does and its code row and fp32 scale are stored.
+ * E5M2_CAST caches: each value is cast to E5M2 (saturating round to nearest
+ *   even) and stored; no scale.
  * Errors: KV_ERR_INVALID (bad layer, null, misaligned, num_tokens < 0),
  *   KV_ERR_UNSUPPORTED (dtype combination), KV_ERR_CUDA. */
 kv_status kv_append(kv_pool *pool, int32_t layer, const void *k_new,
@@ -195,11 +199,13 @@ kv_status kv_append(kv_pool *pool, int32_t layer, const void *k_new,
  * one scale per token per head]:
  *   a = max|x|; scale = fl32(a / QMAX) (QMAX 127 for INT8, 57344 for E5M2);
  *   code = round-half-even(fl32(x / scale)), clamped to [-127, 127] (INT8) or
- *   rounded to E5M2 with saturation to +-57344; a == 0 gives scale 0, codes 0.
+ *   [-7, 7] (INT4, QMAX 7: the pages' most aggressive KV row), or rounded to
+ *   E5M2 with saturation to +-57344; a == 0 gives scale 0, codes 0.
  *   Both divisions are IEEE fp32 divisions, so results are bit-reproducible.
  * x: device [rows][head_dim] of in_dtype (BF16 / FP16), 16-byte aligned.
- * codes: device [rows][head_dim] bytes; scales: device fp32 [rows].
- * head_dim: 64 or 128. out_dtype: KV_INT8 or KV_FP8_E5M2. */
+ * codes: device [rows][head_dim] bytes ([rows][head_dim / 2] for INT4: element
+ *   2i in the low nibble of byte i); scales: device fp32 [rows].
+ * head_dim: 64 or 128 (128 for INT4). out_dtype: KV_INT8, KV_FP8_E5M2 or KV_INT4. */
 kv_status kv_quantize(const void *x, int32_t in_dtype, int64_t rows,
                       int32_t head_dim, int32_t out_dtype, void *codes,
                       float *scales, kv_stream_t stream);

@@ -22,14 +22,19 @@ lib = ctypes.CDLL(LIB_PATH)
 
 # ----------------------------------------------------------------- constants
 KV_OK, KV_ERR_INVALID, KV_ERR_OOM, KV_ERR_CUDA, KV_ERR_UNSUPPORTED = 0, 1, 2, 3, 4
-KV_BF16, KV_FP16, KV_FP8_E5M2, KV_INT8, KV_FP8_E5M2_CAST = 0, 1, 2, 3, 4
+KV_BF16, KV_FP16, KV_FP8_E5M2, KV_INT8, KV_FP8_E5M2_CAST, KV_INT4 = 0, 1, 2, 3, 4, 5
 KV_DEVERR_BLOCK_ID, KV_DEVERR_CONTEXT, KV_DEVERR_SLOT, KV_DEVERR_TIMEOUT = 1, 2, 4, 8
 
 DTYPE_CODES = {"bf16": KV_BF16, "fp16": KV_FP16, "e5m2": KV_FP8_E5M2, "int8": KV_INT8,
-               "e5m2_cast": KV_FP8_E5M2_CAST}
+               "e5m2_cast": KV_FP8_E5M2_CAST, "int4": KV_INT4}
 TORCH_CODES = {torch.bfloat16: KV_BF16, torch.float16: KV_FP16}
 CACHE_TORCH = {"bf16": torch.bfloat16, "fp16": torch.float16, "e5m2": torch.uint8,
-               "int8": torch.int8, "e5m2_cast": torch.uint8}
+               "int8": torch.int8, "e5m2_cast": torch.uint8, "int4": torch.uint8}
+
+
+def code_row(kind, head_dim):
+    """Stored elements of one (token, head) row: INT4 packs two codes per byte."""
+    return head_dim // 2 if kind == "int4" else head_dim
 
 
 class PoolDesc(ctypes.Structure):
@@ -172,7 +177,7 @@ class KVPool:
     block_size = property(lambda s: s.desc.block_size)
     num_kv_heads = property(lambda s: s.desc.num_kv_heads)
     head_dim = property(lambda s: s.desc.head_dim)
-    quantized = property(lambda s: s.cache_dtype in ("int8", "e5m2", "e5m2_cast"))
+    quantized = property(lambda s: s.cache_dtype in ("int8", "e5m2", "e5m2_cast", "int4"))
 
     def close(self):
         if getattr(self, "handle", None):
@@ -198,12 +203,13 @@ class KVPool:
     def layer_views(self, layer):
         """(K, V, K_scale, V_scale) torch views of one layer's regions."""
         k, v, ks, vs = self.layer_ptrs(layer)
-        shape = (self.num_blocks, self.num_kv_heads, self.block_size, self.head_dim)
+        row = code_row(self.cache_dtype, self.head_dim)   # elements per (token, head) row
+        shape = (self.num_blocks, self.num_kv_heads, self.block_size, row)
         dt = CACHE_TORCH[self.cache_dtype]
         elt = 2 if self.cache_dtype in ("bf16", "fp16") else 1
         n = self.num_blocks * self.num_kv_heads * self.block_size
-        K = self._view(k, n * self.head_dim * elt, dt, shape)
-        V = self._view(v, n * self.head_dim * elt, dt, shape)
+        K = self._view(k, n * row * elt, dt, shape)
+        V = self._view(v, n * row * elt, dt, shape)
         if ks is None:
             return K, V, None, None
         sshape = shape[:3]
@@ -328,7 +334,8 @@ def kv_quantize(x, kind, codes=None, scales=None, stream=None):
     D = x.shape[-1]
     rows = x.numel() // D if D else 0
     if codes is None:
-        codes = torch.empty(x.shape, dtype=CACHE_TORCH[kind], device=x.device)
+        codes = torch.empty(x.shape[:-1] + (code_row(kind, D),), dtype=CACHE_TORCH[kind],
+                            device=x.device)
     if scales is None:
         scales = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device)
     _need(codes, "codes", CACHE_TORCH[kind], x.device)

@@ -107,8 +107,8 @@ constexpr bool is16() {
 
 template <int D, int BS, int KV_T>
 struct Tile {
-  static constexpr int kElt = is16<KV_T>() ? 2 : 1;
-  static constexpr int kRowBytes = D * kElt;
+  static constexpr int kElt = is16<KV_T>() ? 2 : 1;  // tensor-map element bytes
+  static constexpr int kRowBytes = KV_T == KV_INT4 ? D / 2 : D * kElt;
   static constexpr int kSlab = kRowBytes >= 128 ? 128 : kRowBytes;  // TMA box width, bytes
   static constexpr int kSlabs = kRowBytes / kSlab;
   static constexpr bool kQuant = !is16<KV_T>();                 // 1-byte codes
@@ -320,13 +320,18 @@ struct Consumer {
       // magnitude is in [2^14, 2^15) (exact), the scale folded into s_fac.
       // k-slot order matches the code fragments: lane (gq, cq) holds dims
       // 16ks + 4cq .. 16ks + 4cq + 3.
+      // INT4 codes unpack in another order: k-step ks = 2c + s takes dims
+      // 32c + 8cq + 2s + {0, 4} (first pair) and {1, 5} (second pair).
       float qv[KS][4];
       float amax = 0.f;
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          qv[ks][e] = hv ? load_q<Q_T>(p.q, qrow + 16 * ks + 4 * cq + e) : 0.f;
+          const int dim = KV_T == KV_INT4
+                              ? (ks >> 1) * 32 + 8 * cq + 2 * (ks & 1) + ((e & 1) << 2) + (e >> 1)
+                              : 16 * ks + 4 * cq + e;
+          qv[ks][e] = hv ? load_q<Q_T>(p.q, qrow + dim) : 0.f;
           amax = fmaxf(amax, fabsf(qv[ks][e]));
         }
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
@@ -346,7 +351,7 @@ struct Consumer {
       const int ex1 = __shfl_sync(0xffffffffu, ex, (2 * cq + 1) * 4);
       s_fac[0] = ldexpf(p.scale_log2, -ex0);
       s_fac[1] = ldexpf(p.scale_log2, -ex1);
-      if constexpr (KV_T == KV_INT8) {
+      if constexpr (KV_T == KV_INT8 || KV_T == KV_INT4) {
         // sum of the fp16 query operands of head gq (as the MMA sees them)
         float qsum = 0.f;
 #pragma unroll
@@ -357,8 +362,9 @@ struct Consumer {
         }
         qsum += __shfl_xor_sync(0xffffffffu, qsum, 1);
         qsum += __shfl_xor_sync(0xffffffffu, qsum, 2);
-        qcorr[0] = 1152.f * __shfl_sync(0xffffffffu, qsum, (2 * cq) * 4);
-        qcorr[1] = 1152.f * __shfl_sync(0xffffffffu, qsum, (2 * cq + 1) * 4);
+        constexpr float kBias = KV_T == KV_INT8 ? 1152.f : 1032.f;
+        qcorr[0] = kBias * __shfl_sync(0xffffffffu, qsum, (2 * cq) * 4);
+        qcorr[1] = kBias * __shfl_sync(0xffffffffu, qsum, (2 * cq + 1) * 4);
       }
     }
   }
@@ -385,6 +391,27 @@ struct Consumer {
           uint32_t a0, a1, a2, a3;
           ldsm_x4(T::chunk(ktile, r0 + row, 2 * ks + (lane >> 4), rows), a0, a1, a2, a3);
           mma16816<kBF>(acc, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
+        }
+      } else if constexpr (KV_T == KV_INT4) {
+        // 16-byte chunk c of a row = dims 32c .. 32c + 31; a lane's word holds
+        // dims 32c + 8cq .. + 7 of its token (nibble k = dim 8cq + k)
+#pragma unroll
+        for (int cpair = 0; cpair < 2; ++cpair) {
+          uint32_t w0, w1, w2, w3;  // rows 0-7 / 8-15 x chunks 2cpair, 2cpair+1
+          ldsm_x4(T::chunk(ktile, r0 + row, 2 * cpair + (lane >> 4), rows), w0, w1, w2, w3);
+          w0 ^= 0x88888888u; w1 ^= 0x88888888u; w2 ^= 0x88888888u; w3 ^= 0x88888888u;
+          const int kc = 4 * cpair;  // k-steps 4cpair .. 4cpair + 3
+          mma16816<false>(acc, int4_pair_biased<0>(w0), int4_pair_biased<0>(w1),
+                          int4_pair_biased<1>(w0), int4_pair_biased<1>(w1), qb[kc][0], qb[kc][1]);
+          mma16816<false>(acc, int4_pair_biased<2>(w0), int4_pair_biased<2>(w1),
+                          int4_pair_biased<3>(w0), int4_pair_biased<3>(w1), qb[kc + 1][0],
+                          qb[kc + 1][1]);
+          mma16816<false>(acc, int4_pair_biased<0>(w2), int4_pair_biased<0>(w3),
+                          int4_pair_biased<1>(w2), int4_pair_biased<1>(w3), qb[kc + 2][0],
+                          qb[kc + 2][1]);
+          mma16816<false>(acc, int4_pair_biased<2>(w2), int4_pair_biased<2>(w3),
+                          int4_pair_biased<3>(w2), int4_pair_biased<3>(w3), qb[kc + 3][0],
+                          qb[kc + 3][1]);
         }
       } else {
 #pragma unroll
@@ -418,7 +445,7 @@ struct Consumer {
         k0 = ksc[t0];
         k1 = ksc[t1];
       }
-      if constexpr (KV_T == KV_INT8) {
+      if constexpr (KV_T == KV_INT8 || KV_T == KV_INT4) {
         acc[0] -= qcorr[0];
         acc[1] -= qcorr[1];
         acc[2] -= qcorr[0];
@@ -541,6 +568,35 @@ struct Consumer {
           mma16816<kBF>(oacc[dt], a0, a1, a2, a3, pb0, pb1);
           mma16816<kBF>(oacc[dt], a0, a1, a2, a3, pl0, pl1);
         }
+      } else if constexpr (KV_T == KV_INT4) {
+        // after the transpose a lane holds, for tokens 2cq and 2cq+1 (low /
+        // high half), the 4 nibbles of dims 32c + 4gq .. + 3; m-tile 2c + t
+        // takes dims 32c + 4gq + 2t (rows gq) and + 1 (rows gq + 8)
+#pragma unroll
+        for (int cp = 0; cp < D / 64; ++cp) {
+          uint32_t w0, w1, w2, w3;  // tokens 0-7 / 8-15 x chunks 2cp, 2cp+1
+          const int vr = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+          ldsm_x4_t(T::chunk(vtile, r0 + vr, 2 * cp + (lane >> 4), rows), w0, w1, w2, w3);
+          w0 ^= 0x88888888u; w1 ^= 0x88888888u; w2 ^= 0x88888888u; w3 ^= 0x88888888u;
+          uint32_t a[16];
+          a[0] = int4_pair<0>(w0); a[1] = int4_pair<1>(w0); a[2] = int4_pair<0>(w1); a[3] = int4_pair<1>(w1);
+          a[4] = int4_pair<2>(w0); a[5] = int4_pair<3>(w0); a[6] = int4_pair<2>(w1); a[7] = int4_pair<3>(w1);
+          a[8] = int4_pair<0>(w2); a[9] = int4_pair<1>(w2); a[10] = int4_pair<0>(w3); a[11] = int4_pair<1>(w3);
+          a[12] = int4_pair<2>(w2); a[13] = int4_pair<3>(w2); a[14] = int4_pair<2>(w3); a[15] = int4_pair<3>(w3);
+          if (!full) {
+#pragma unroll
+            for (int i = 0; i < 16; i += 4) {
+              a[i] &= m0; a[i + 1] &= m0; a[i + 2] &= m1; a[i + 3] &= m1;
+            }
+          }
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {  // m-tiles 4cp + t
+            mma16816<false>(oacc[4 * cp + t], a[4 * t], a[4 * t + 1], a[4 * t + 2], a[4 * t + 3],
+                            pb0, pb1);
+            mma16816<false>(oacc[4 * cp + t], a[4 * t], a[4 * t + 1], a[4 * t + 2], a[4 * t + 3],
+                            pl0, pl1);
+          }
+        }
       } else {
 #pragma unroll
         for (int cp = 0; cp < D / 32; ++cp) {
@@ -603,7 +659,10 @@ struct Consumer {
 #pragma unroll
     for (int dt = 0; dt < D / 16; ++dt) {
       int d0, d1;
-      if constexpr (kQuant) {  // rows gq / gq+8 are dims 16c + 2gq / + 1
+      if constexpr (KV_T == KV_INT4) {  // rows gq / gq+8: dims 32c + 4gq + 2t / + 1
+        d0 = (dt >> 1) * 32 + 4 * gq + 2 * (dt & 1);
+        d1 = d0 + 1;
+      } else if constexpr (kQuant) {  // rows gq / gq+8 are dims 16c + 2gq / + 1
         d0 = dt * 16 + 2 * gq;
         d1 = d0 + 1;
       } else {
@@ -681,13 +740,14 @@ struct NewRow {
     using T = Tile<D, BS, KV_T>;
     const uint32_t ktile = smem_u32(st);
     const uint32_t vtile = ktile + rows * T::kRowBytes;
-    const uint32_t off = lane * E * T::kElt;  // this lane's bytes within the row
+    // this lane's bytes within the row (INT4: two codes per byte)
+    const uint32_t off = lane * (KV_T == KV_INT4 ? E / 2 : E * T::kElt);
     const uint32_t ka = T::chunk(ktile, r, off >> 4, rows) + (off & 15);
     const uint32_t va = T::chunk(vtile, r, off >> 4, rows) + (off & 15);
     const int64_t grow = (static_cast<int64_t>(id) * p.kv_heads + g) * BS + rl;
     char *kg = p.k_cache + grow * T::kRowBytes + off;
     char *vg = p.v_cache + grow * T::kRowBytes + off;
-    constexpr int kBytes = E * T::kElt;
+    constexpr int kBytes = KV_T == KV_INT4 ? E / 2 : E * T::kElt;
     if constexpr (kBytes == 8) {
       asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(ka), "r"(k[0]), "r"(k[1]) : "memory");
       asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(va), "r"(v[0]), "r"(v[1]) : "memory");
@@ -1082,6 +1142,11 @@ PartFn pick_dtype(int kv, int q) {
     case KV_FP8_E5M2:
       return q == KV_BF16 ? launch_part<D, BS, KV_FP8_E5M2, KV_BF16>
                           : launch_part<D, BS, KV_FP8_E5M2, KV_FP16>;
+    case KV_INT4:  // pools reject INT4 unless head_dim is 128
+      if constexpr (D == 128)
+        return q == KV_BF16 ? launch_part<D, BS, KV_INT4, KV_BF16> : launch_part<D, BS, KV_INT4, KV_FP16>;
+      else
+        return nullptr;
     default:
       return q == KV_BF16 ? launch_part<D, BS, KV_FP8_E5M2_CAST, KV_BF16>
                           : launch_part<D, BS, KV_FP8_E5M2_CAST, KV_FP16>;
@@ -1121,8 +1186,7 @@ UnitGeom unit_geom(const kv_pool *pool, int num_q_heads) {
   u.chunks = (group + kChunkHeads - 1) / kChunkHeads;
   u.cpg = std::min(u.chunks, kNC);
   u.cgroups = (u.chunks + u.cpg - 1) / u.cpg;
-  const int elt = elem_bytes(d.cache_dtype);
-  const int row_bytes = d.head_dim * elt;
+  const int row_bytes = row_bytes_of(d.cache_dtype, d.head_dim);
   const bool quant = has_scales(d.cache_dtype);  // scale rows ride with the stage
   auto load = [&](int hg) { return 2 * hg * d.block_size * (row_bytes + (quant ? 4 : 0)); };
   // the largest group of kv heads (a divisor of Hkv) with one slot per consumer
@@ -1281,6 +1345,7 @@ kv_status run_partition(kv_pool *pool, int32_t layer, const void *q, int32_t q_d
   LayerMaps maps;
   if (!layer_maps(pool, layer, p.hg * pool->d.block_size, &maps, &code)) return code;
   PartFn fn = pick_partition(pool->d.head_dim, pool->d.block_size, cd, q_dtype);
+  if (!fn) return fail(KV_ERR_UNSUPPORTED, "no attention kernel for this cache shape");
   return cuda_check(fn(maps.k, maps.v, p, st), "paged attention launch");
 }
 

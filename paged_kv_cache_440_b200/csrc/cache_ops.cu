@@ -95,11 +95,12 @@ append_quant_kernel(const uint16_t *__restrict__ k_new, const uint16_t *__restri
   float scale;
   load_row<D, IN_T>(k_new + src_row * D, lane, x);
   uint32_t packed = quantize_row<D, OUT_T>(x, &scale);
-  store_codes<D>(kc + dst_row * D, lane, packed);
+  constexpr int kRow = OUT_T == KV_INT4 ? D / 2 : D;  // bytes per row
+  store_codes<D, OUT_T>(kc + dst_row * kRow, lane, packed);
   if (OUT_T != KV_FP8_E5M2_CAST && lane == 0) ks[dst_row] = scale;
   load_row<D, IN_T>(v_new + src_row * D, lane, x);
   packed = quantize_row<D, OUT_T>(x, &scale);
-  store_codes<D>(vc + dst_row * D, lane, packed);
+  store_codes<D, OUT_T>(vc + dst_row * kRow, lane, packed);
   if (OUT_T != KV_FP8_E5M2_CAST && lane == 0) vs[dst_row] = scale;
 }
 
@@ -115,7 +116,7 @@ quantize_kernel(const uint16_t *__restrict__ x_in, int64_t rows, uint8_t *__rest
   float scale;
   load_row<D, IN_T>(x_in + row * D, lane, x);
   uint32_t packed = quantize_row<D, OUT_T>(x, &scale);
-  store_codes<D>(codes + row * D, lane, packed);
+  store_codes<D, OUT_T>(codes + row * (OUT_T == KV_INT4 ? D / 2 : D), lane, packed);
   if (lane == 0) scales[row] = scale;
 }
 
@@ -231,6 +232,10 @@ kv_status kv_append(kv_pool *pool, int32_t layer, const void *k_new, const void 
     e = in_dtype == KV_BF16
             ? dispatch_append_quant_d<KV_BF16, KV_INT8>(pool, layer, k_new, v_new, slot_mapping, num_tokens, st)
             : dispatch_append_quant_d<KV_FP16, KV_INT8>(pool, layer, k_new, v_new, slot_mapping, num_tokens, st);
+  } else if (cd == KV_INT4) {
+    e = in_dtype == KV_BF16
+            ? launch_append_quant<128, KV_BF16, KV_INT4>(pool, layer, k_new, v_new, slot_mapping, num_tokens, st)
+            : launch_append_quant<128, KV_FP16, KV_INT4>(pool, layer, k_new, v_new, slot_mapping, num_tokens, st);
   } else if (cd == KV_FP8_E5M2) {
     e = in_dtype == KV_BF16
             ? dispatch_append_quant_d<KV_BF16, KV_FP8_E5M2>(pool, layer, k_new, v_new, slot_mapping, num_tokens, st)
@@ -251,8 +256,10 @@ kv_status kv_quantize(const void *x, int32_t in_dtype, int64_t rows, int32_t hea
     return fail(KV_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
   if (in_dtype != KV_BF16 && in_dtype != KV_FP16)
     return fail(KV_ERR_UNSUPPORTED, "in_dtype must be KV_BF16 or KV_FP16");
-  if (out_dtype != KV_INT8 && out_dtype != KV_FP8_E5M2)
-    return fail(KV_ERR_UNSUPPORTED, "out_dtype must be KV_INT8 or KV_FP8_E5M2");
+  if (out_dtype != KV_INT8 && out_dtype != KV_FP8_E5M2 && out_dtype != KV_INT4)
+    return fail(KV_ERR_UNSUPPORTED, "out_dtype must be KV_INT8, KV_FP8_E5M2 or KV_INT4");
+  if (out_dtype == KV_INT4 && head_dim != 128)
+    return fail(KV_ERR_UNSUPPORTED, "KV_INT4 rows need head_dim 128");
   if (rows == 0) return ok();
   if (!x || !codes || !scales) return fail(KV_ERR_INVALID, "null pointer");
   if (!aligned16(x) || (reinterpret_cast<uintptr_t>(codes) & 3) ||
@@ -265,6 +272,9 @@ kv_status kv_quantize(const void *x, int32_t in_dtype, int64_t rows, int32_t hea
   if (out_dtype == KV_INT8)
     e = in_dtype == KV_BF16 ? dispatch_quantize_d<KV_BF16, KV_INT8>(head_dim, x, rows, codes, scales, st)
                             : dispatch_quantize_d<KV_FP16, KV_INT8>(head_dim, x, rows, codes, scales, st);
+  else if (out_dtype == KV_INT4)
+    e = in_dtype == KV_BF16 ? launch_quantize<128, KV_BF16, KV_INT4>(x, rows, codes, scales, st)
+                            : launch_quantize<128, KV_FP16, KV_INT4>(x, rows, codes, scales, st);
   else
     e = in_dtype == KV_BF16 ? dispatch_quantize_d<KV_BF16, KV_FP8_E5M2>(head_dim, x, rows, codes, scales, st)
                             : dispatch_quantize_d<KV_FP16, KV_FP8_E5M2>(head_dim, x, rows, codes, scales, st);

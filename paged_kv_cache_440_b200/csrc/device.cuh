@@ -202,6 +202,25 @@ __device__ __forceinline__ void split2(float a, float b, uint32_t &hi, uint32_t 
   lo = pack2<BF16>(a - ha, b - hb);
 }
 
+// -------------------------------------------------- 4-bit codes -> fp16 pairs
+//
+// INT4 codes (two's complement nibbles) become offset binary u = code + 8 when
+// the caller xors the word with 0x88888888. Nibbles K and K + 4 of a 32-bit
+// word, placed under the fp16 exponent byte 0x64, are 1024 + u: an exact pair,
+// 1032 above the codes.
+template <int K>
+__device__ __forceinline__ uint32_t int4_pair_biased(uint32_t w_biased) {
+  return ((w_biased >> (4 * K)) & 0x000F000Fu) | 0x64006400u;
+}
+template <int K>
+__device__ __forceinline__ uint32_t int4_pair(uint32_t w_biased) {
+  uint32_t h = int4_pair_biased<K>(w_biased);
+  __half2 v = *reinterpret_cast<__half2 *>(&h);
+  const __half2 bias = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));
+  v = __hsub2(v, bias);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+
 // -------------------------------------------------- 1-byte codes -> fp16 pairs
 //
 // An E5M2 byte is the high byte of the fp16 with the same value (same sign,
@@ -271,7 +290,7 @@ __device__ __forceinline__ uint32_t quantize_row(const float (&x)[D / 32], float
   for (int i = 0; i < E; ++i) a = fmaxf(a, fabsf(x[i]));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-  constexpr float kQmax = OUT_T == KV_INT8 ? 127.0f : 57344.0f;
+  constexpr float kQmax = OUT_T == KV_INT8 ? 127.0f : OUT_T == KV_INT4 ? 7.0f : 57344.0f;
   uint32_t packed = 0;
   float scale = 0.f;
   if (a > 0.f) {
@@ -284,6 +303,12 @@ __device__ __forceinline__ uint32_t quantize_row(const float (&x)[D / 32], float
         int q = __float2int_rn(y);
         q = max(-127, min(127, q));
         code = static_cast<uint32_t>(q) & 0xFFu;
+      } else if constexpr (OUT_T == KV_INT4) {
+        int q = __float2int_rn(y);
+        q = max(-7, min(7, q));
+        code = static_cast<uint32_t>(q) & 0xFu;
+        packed |= code << (4 * i);  // two codes per byte, element 2i low
+        continue;
       } else {
         code = static_cast<uint32_t>(__nv_cvt_float_to_fp8(y, __NV_SATFINITE, __NV_E5M2));
       }
@@ -311,9 +336,14 @@ __device__ __forceinline__ void load_row(const uint16_t *__restrict__ src, int l
   }
 }
 
-template <int D>
+// Store this lane's codes of one row (row base `dst`): D/32 bytes, or D/64
+// for INT4 (4 bits per code).
+template <int D, int OUT_T = KV_INT8>
 __device__ __forceinline__ void store_codes(uint8_t *dst, int lane, uint32_t packed) {
-  if constexpr (D == 128) {
+  if constexpr (OUT_T == KV_INT4) {
+    static_assert(D == 128, "INT4 rows need head_dim 128");
+    reinterpret_cast<uint16_t *>(dst)[lane] = static_cast<uint16_t>(packed);
+  } else if constexpr (D == 128) {
     reinterpret_cast<uint32_t *>(dst)[lane] = packed;
   } else {
     reinterpret_cast<uint16_t *>(dst)[lane] = static_cast<uint16_t>(packed);

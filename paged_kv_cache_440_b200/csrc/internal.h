@@ -17,15 +17,23 @@ namespace pagedkv {
 // Device status word bit set when a bounded wait in a kernel gives up.
 constexpr int32_t kDevErrTimeout = 8;
 
+// Element size of the tensor maps (INT4 rows are addressed as bytes).
 inline int elem_bytes(int dtype) {
   return (dtype == KV_BF16 || dtype == KV_FP16) ? 2 : 1;
 }
+// Bytes of one (token, head) row of head_dim values.
+inline int row_bytes_of(int dtype, int head_dim) {
+  return dtype == KV_INT4 ? head_dim / 2 : head_dim * elem_bytes(dtype);
+}
 // 1-byte codes (read through the code paths of the kernels)
 inline bool is_quant(int dtype) {
-  return dtype == KV_INT8 || dtype == KV_FP8_E5M2 || dtype == KV_FP8_E5M2_CAST;
+  return dtype == KV_INT8 || dtype == KV_FP8_E5M2 || dtype == KV_FP8_E5M2_CAST ||
+         dtype == KV_INT4;
 }
 // codes with a per-token-head fp32 scale (scale regions in the pool)
-inline bool has_scales(int dtype) { return dtype == KV_INT8 || dtype == KV_FP8_E5M2; }
+inline bool has_scales(int dtype) {
+  return dtype == KV_INT8 || dtype == KV_FP8_E5M2 || dtype == KV_INT4;
+}
 inline uint64_t round_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
 
 // Byte offsets of one layer's regions inside the pool buffer.
@@ -55,7 +63,7 @@ struct kv_pool {
   uint64_t bytes = 0;
   pagedkv::Layout lay;
   int elt = 2;
-  int row_bytes = 0;  // head_dim * elt
+  int row_bytes = 0;  // bytes of one (token, head) row
 
   std::mutex mu;                    // guards the allocator state
   std::vector<int32_t> ref;         // refcount per block

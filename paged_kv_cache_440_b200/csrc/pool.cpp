@@ -60,8 +60,12 @@ bool compute_layout(const kv_pool_desc &d, Layout *out, std::string *why,
     *why = "head_dim must be 64 or 128";
     return false;
   }
-  if (d.cache_dtype < KV_BF16 || d.cache_dtype > KV_FP8_E5M2_CAST) {
-    *why = "cache_dtype must be KV_BF16, KV_FP16, KV_FP8_E5M2, KV_INT8 or KV_FP8_E5M2_CAST";
+  if (d.cache_dtype < KV_BF16 || d.cache_dtype > KV_INT4) {
+    *why = "cache_dtype must be KV_BF16, KV_FP16, KV_FP8_E5M2, KV_INT8, KV_FP8_E5M2_CAST or KV_INT4";
+    return false;
+  }
+  if (d.cache_dtype == KV_INT4 && d.head_dim != 128) {
+    *why = "KV_INT4 caches need head_dim 128";
     return false;
   }
   const uint64_t rows = (uint64_t)d.num_blocks * d.num_kv_heads * d.block_size;
@@ -71,7 +75,7 @@ bool compute_layout(const kv_pool_desc &d, Layout *out, std::string *why,
     return false;
   }
   Layout L;
-  L.kv_bytes = rows * d.head_dim * elem_bytes(d.cache_dtype);
+  L.kv_bytes = rows * row_bytes_of(d.cache_dtype, d.head_dim);
   L.kv_stride = round_up(L.kv_bytes, 256);
   L.sc_bytes = has_scales(d.cache_dtype) ? rows * sizeof(float) : 0;
   L.sc_stride = round_up(L.sc_bytes, 256);
@@ -127,7 +131,7 @@ static bool encode_region(const kv_pool *p, void *base, int box_rows, CUtensorMa
   const int elt = p->elt;
   const int row_bytes = p->row_bytes;
   const int slab_bytes = row_bytes >= 128 ? 128 : row_bytes;  // 128 or 64
-  cuuint64_t gdim[2] = {(cuuint64_t)d.head_dim,
+  cuuint64_t gdim[2] = {(cuuint64_t)(row_bytes / elt),
                         (cuuint64_t)d.num_blocks * d.num_kv_heads * d.block_size};
   cuuint64_t gstride[1] = {(cuuint64_t)row_bytes};
   cuuint32_t box[2] = {(cuuint32_t)(slab_bytes / elt), (cuuint32_t)box_rows};
@@ -210,7 +214,7 @@ kv_status kv_pool_create(const kv_pool_desc *desc, void *device_base, uint64_t b
   p->bytes = bytes;
   p->lay = L;
   p->elt = elem_bytes(desc->cache_dtype);
-  p->row_bytes = desc->head_dim * p->elt;
+  p->row_bytes = row_bytes_of(desc->cache_dtype, desc->head_dim);
   p->ref.assign(desc->num_blocks, 0);
   p->free_stack.resize(desc->num_blocks);
   for (int32_t i = 0; i < desc->num_blocks; ++i)

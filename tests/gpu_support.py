@@ -89,7 +89,8 @@ def oracle_cache_quant(wl, seqs):
     sampled sequences' blocks, with block tables renumbered to match (the
     result does not depend on physical placement).
     """
-    shape = (wl.num_blocks, wl.kv_heads, wl.block_size, wl.head_dim)
+    row = wl.head_dim // 2 if wl.cache_dtype == "int4" else wl.head_dim
+    shape = (wl.num_blocks, wl.kv_heads, wl.block_size, row)
     cdt = np.int8 if wl.cache_dtype == "int8" else np.uint8
     kc, vc = np.zeros(shape, cdt), np.zeros(shape, cdt)
     ks, vs = np.zeros(shape[:3], np.float32), np.zeros(shape[:3], np.float32)
@@ -112,8 +113,9 @@ def oracle_cache_quant(wl, seqs):
         nblk = -(-int(wl.context_lens[b]) // wl.block_size)
         tables[b, :nblk] = [remap[x] for x in wl.block_tables[b, :nblk]]
     u = np.array(used)
-    kd = quant.dequantize(kc[u], ks[u], wl.cache_dtype)
-    vd = quant.dequantize(vc[u], vs[u], wl.cache_dtype)
+    unpack = quant.unpack_int4 if wl.cache_dtype == "int4" else (lambda c: c)
+    kd = quant.dequantize(unpack(kc[u]), ks[u], wl.cache_dtype)
+    vd = quant.dequantize(unpack(vc[u]), vs[u], wl.cache_dtype)
     return (kc, vc, ks, vs), (kd, vd, tables)
 
 

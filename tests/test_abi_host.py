@@ -249,3 +249,23 @@ def test_valid_call_without_a_gpu_fails_loudly():
         assert B.lib.paged_attn_workspace_bytes(h, 4, 8, 0, ctypes.byref(n)) == B.KV_ERR_CUDA
     finally:
         B.lib.kv_pool_destroy(h)
+
+
+def test_int4_layout_and_head_dim():
+    """INT4 rows are head_dim / 2 bytes (two codes per byte) with fp32 scales;
+    head_dim 64 is rejected."""
+    NB, layers, bs, hkv, D = 37, 2, 16, 8, 128
+    h, total = _make_pool(NB, layers, bs, hkv, D, "int4")
+    try:
+        tokens = NB * bs
+        kv = ref_pool.kv_cache_bytes(1, hkv, D, 0.5, tokens)      # K and V, half a byte per value
+        k, v, ks, vs = _ptrs(h, 0)
+        assert v - k >= kv // 2 and ks - v >= kv // 2 and vs is not None
+        exact = ref_pool.kv_cache_bytes(layers, hkv, D, 0.5, tokens) + \
+            ref_pool.scale_bytes(layers, hkv, 4, tokens)
+        assert exact + 256 <= total <= exact + 256 + layers * 4 * 255
+    finally:
+        B.lib.kv_pool_destroy(h)
+    d = B.PoolDesc(1, 8, 16, 2, 64, B.DTYPE_CODES["int4"])
+    n = ctypes.c_uint64()
+    assert B.lib.kv_pool_required_bytes(ctypes.byref(d), ctypes.byref(n)) == B.KV_ERR_UNSUPPORTED

@@ -71,10 +71,12 @@ def _special_rows(D):
     return np.stack(rows)
 
 
-@pytest.mark.parametrize("kind", ["int8", "e5m2"])
+@pytest.mark.parametrize("kind", ["int8", "e5m2", "int4"])
 @pytest.mark.parametrize("in_dt", [torch.bfloat16, torch.float16])
 @pytest.mark.parametrize("D", [64, 128])
 def test_quantize_bit_exact(pkv, kind, in_dt, D):
+    if kind == "int4" and D != 128:
+        pytest.skip("INT4 rows need head_dim 128")
     g = torch.Generator(device=DEV).manual_seed(D)
     x = torch.randn(20000, D, generator=g, device=DEV)
     x = x * torch.exp(torch.randn(20000, 1, generator=g, device=DEV) * 3)   # wide dynamic range
@@ -84,11 +86,13 @@ def test_quantize_bit_exact(pkv, kind, in_dt, D):
     codes, scales = pkv.kv_quantize(x, kind)
     torch.cuda.synchronize()
     ref_codes, ref_scales = quant.quantize_rows(to_np(x), kind)
+    if kind == "int4":
+        ref_codes = quant.pack_int4(ref_codes)
     assert np.array_equal(scales.cpu().numpy().view(np.uint32), ref_scales.view(np.uint32))
     assert np.array_equal(codes.cpu().numpy(), ref_codes)
 
 
-@pytest.mark.parametrize("cache", ["bf16", "int8", "e5m2", "e5m2_cast"])
+@pytest.mark.parametrize("cache", ["bf16", "int8", "e5m2", "e5m2_cast", "int4"])
 def test_block_copy_bit_exact(pkv, cache):
     """Shared-prefix shapes: 200 copy-on-write pairs, 3 layers, random pool bytes."""
     layers, NB, bs, hkv, D = 3, 1500, 16, 8, 128

@@ -70,7 +70,7 @@ def test_mha13b_every_output(pkv):
     _run_16(pkv, W.mha13b(DEV))
 
 
-@pytest.mark.parametrize("kind", ["int8", "e5m2"])
+@pytest.mark.parametrize("kind", ["int8", "e5m2", "int4"])
 @pytest.mark.parametrize("variant,seqs", [("a", [0, 13, 40, 63]), ("b", [0, 5])])
 def test_quantized_long_context(pkv, kind, variant, seqs):
     """INT8 / E5M2 per-token-head KV, bs 32, (a) 64 x 4096 and (b) 8 x 32768.
@@ -190,13 +190,15 @@ def test_shared_prefix_copy_on_write(pkv):
 EDGE_LENS = [0, 1, 15, 16, 17, 63, 64, 65, 127, 128, 129, 300]
 
 
-@pytest.mark.parametrize("cache", ["bf16", "fp16", "int8", "e5m2", "e5m2_cast"])
+@pytest.mark.parametrize("cache", ["bf16", "fp16", "int8", "e5m2", "e5m2_cast", "int4"])
 @pytest.mark.parametrize("G", [1, 2, 4, 8, 16])
 @pytest.mark.parametrize("D,bs", [(64, 16), (128, 32)])
 def test_edge_lengths_groups_dims(pkv, cache, G, D, bs):
     """Empty, single-token and block-boundary lengths; MHA, GQA groups of 2..16
     heads (16 spans two head units); head_dim 64 / 128; block size 16 / 32; all
     four cache types; 13 CTAs, so units are split at assorted places."""
+    if cache == "int4" and D != 128:
+        pytest.skip("INT4 rows need head_dim 128")
     qd = "fp16" if cache == "fp16" else "bf16"
     lens = EDGE_LENS
     wl = W.make_decode_workload("edge", len(lens), 2 * G, 2, D, bs, qd, cache, lens,
@@ -267,6 +269,8 @@ def _fused_workloads():
                                                 [2, 17, 64, 129], seed=6, device=DEV)),
         ("e5m2-cast", lambda: W.make_decode_workload("e5c", 4, 16, 2, 64, 32, "fp16", "e5m2_cast",
                                                      [3, 32, 33, 200], seed=8, device=DEV)),
+        ("int4", lambda: W.make_decode_workload("i4", 5, 16, 2, 128, 16, "bf16", "int4",
+                                                [1, 15, 16, 17, 300], seed=9, device=DEV)),
     ]
 
 
