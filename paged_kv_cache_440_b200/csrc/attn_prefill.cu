@@ -7,19 +7,38 @@
 // L_b - c_b + i and attends to positions 0 .. L_b - c_b + i: each token sees
 // every token before it and itself [KV Cache 原理与 PagedAttention, §一].
 //
-// Design (sm_100a):
-// * One CTA per (tile of new tokens, KV head, sequence). The tile's rows are
-//   (token, query head of the KV head's group) pairs, head fastest: 128 rows
-//   = 128 / G tokens x G heads, 16 rows per consumer warp.
-// * One producer warp streams the KV head's cached blocks, 64 positions per
+// Design (sm_100a, fifth-generation tensor cores):
+// * One CTA per (tile of new tokens, KV head, sequence). The tile's 128 rows
+//   are (token, query head of the KV head's group) pairs, head fastest:
+//   128 / G tokens x G heads. Row r lives in TMEM lane r.
+// * The producer warp streams the KV head's cached blocks, 64 positions per
 //   stage (K then V, 128-byte swizzled TMA boxes of one block-head slab), into
-//   a 4-stage ring; full/empty mbarriers, every wait bounded.
-// * Eight consumer warps hold their Q rows as MMA A fragments and, per 32
-//   positions, compute S = Q K^T with m16n8k16 tensor-core MMAs (K read by
-//   ldmatrix), the online softmax in fp32 (base 2) with the causal mask, and
-//   O += P V (P from the score accumulators, as hi + lo 16-bit parts; V by
-//   transposed ldmatrix). This is the dense tile of prefill: every staged K/V
-//   byte serves 128 query rows.
+//   a 4-stage ring.
+// * The MMA warp (one thread) issues tcgen05 MMAs: S_j = Q K_j^T (M 128,
+//   N 64, K head_dim; Q and K both K-major in shared memory) into one of two
+//   TMEM score buffers, and O += P_j V_j (M 128, N head_dim, K 64; P K-major,
+//   V MN-major straight from the TMA stage) into a TMEM accumulator that stays
+//   resident for the whole key range. Order: S_0, S_1, then per stage j
+//   O += P_j V_j followed by S_{j+2}, so the tensor core computes the next
+//   scores while the softmax warps work on the current ones.
+// * 16 softmax warps: warp w reads TMEM lanes 32 (w mod 4) .. + 31 (the
+//   lanes a warp may access) and columns of group w / 4, so four threads share
+//   a row, 16 scores each per stage; the row maximum is combined through
+//   shared memory once per stage. Scale, causal and tail masks and the online
+//   softmax run in fp32 (base 2). The running maximum is only raised (and O,
+//   l rescaled in TMEM) when a new score exceeds it by more than 2^8;
+//   otherwise the stale maximum stays in use, which keeps every P value below
+//   256 and leaves the result unchanged up to rounding.
+// * P_j goes to shared memory in the 128-byte swizzled K-major layout the MMA
+//   reads, as two 16-bit parts hi + lo; O accumulates P_hi V + P_lo V, so
+//   rounding P to 16 bits costs nothing measurable (bf16: hi and lo by
+//   truncation, bit masks only; fp16: by rounding conversions).
+// * Synchronisation is by mbarriers: TMA -> MMA (full), MMA -> producer
+//   (stage free, by tcgen05.commit after P_j V_j), MMA -> softmax (S_j ready),
+//   softmax -> MMA (P_j written), MMA -> softmax (P_j V_j done, needed only to
+//   rescale O and for the final read). Every wait is bounded; after a timeout
+//   every role runs to the end without waiting, the output is not written and
+//   the CTA frees its TMEM.
 #include <algorithm>
 #include <cfloat>
 
@@ -31,11 +50,18 @@ namespace {
 
 using namespace dev;
 
-constexpr int kPfC = 8;                 // consumer warps
-constexpr int kPfThreads = (kPfC + 1) * 32;
-constexpr int kPfRows = kPfC * 16;      // query rows per CTA
+constexpr int kPfRows = 128;            // query rows per CTA (TMEM lanes)
+constexpr int kPfGroups = 4;            // softmax threads per row (column groups)
+constexpr int kPfSoftmax = 128 * kPfGroups;
+constexpr int kPfProducerWarp = kPfSoftmax / 32;
+constexpr int kPfMmaWarp = kPfProducerWarp + 1;
+constexpr int kPfThreads = kPfSoftmax + 64;
 constexpr int kPfKeys = 64;             // positions per stage
-constexpr int kPfStages = 4;
+// Ring depth: 3 stages of 32 KB for head_dim 128 (shared memory then holds
+// the ring, Q, and two hi + lo P buffers: 193 KB), 4 of 16 KB for 64.
+__host__ __device__ constexpr int pf_stages(int D) { return D == 128 ? 3 : 4; }
+constexpr uint32_t kPfTmemCols = 256;   // S: 2 x 64 columns, O: head_dim columns
+constexpr float kPfRescaleLog2 = 8.f;   // raise the running max only beyond 2^8
 
 struct PrefillParams {
   const void *q;              // [T][Hq][D]
@@ -55,11 +81,12 @@ __device__ __forceinline__ float ex2f(float x) {
   return y;
 }
 
-// Bounded wait on a ring barrier; gives up (false) when another warp has
+// Bounded wait on a pipeline barrier; gives up (false) when another role has
 // given up or after the time limit, recording KV_DEVERR_TIMEOUT.
 __device__ __forceinline__ bool ring_wait_pf(uint64_t *bar, uint32_t parity, volatile int *abort,
                                              int *status) {
   if (mbar_try_wait(bar, parity)) return true;
+  if (*abort) return false;
   const uint64_t t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -74,10 +101,26 @@ __device__ __forceinline__ bool ring_wait_pf(uint64_t *bar, uint32_t parity, vol
   }
 }
 
-// Shared address of 16-byte chunk c of row r in a stage part of `rows` rows
-// stored as 128-byte slabs (slab-major), 128-byte swizzled.
-__device__ __forceinline__ uint32_t pf_chunk(uint32_t base, int r, int c, int rows) {
-  return base + (c >> 3) * rows * 128 + (r << 7) + (((c & 7) ^ (r & 7)) << 4);
+// Byte offset of 16-byte chunk c of row r in a tile of `rows` rows stored as
+// 128-byte slabs (slab-major), 128-byte swizzled.
+__device__ __forceinline__ uint32_t pf_chunk(int r, int c, int rows) {
+  return (c >> 3) * rows * 128 + (r << 7) + (((c & 7) ^ (r & 7)) << 4);
+}
+
+// Two P values -> 16-bit pairs hi + lo (low half = first value).
+template <bool BF16>
+__device__ __forceinline__ void split_p(float a, float b, uint32_t &hi, uint32_t &lo) {
+  if constexpr (BF16) {
+    // bf16 is the upper half of fp32: truncate for hi, the exact remainder
+    // truncated again for lo (hi + lo within 2^-14 relative of the value)
+    const uint32_t ua = __float_as_uint(a), ub = __float_as_uint(b);
+    const float ra = a - __uint_as_float(ua & 0xFFFF0000u);
+    const float rb = b - __uint_as_float(ub & 0xFFFF0000u);
+    hi = prmt(ua, ub, 0x7632);
+    lo = prmt(__float_as_uint(ra), __float_as_uint(rb), 0x7632);
+  } else {
+    split2<false>(a, b, hi, lo);
+  }
 }
 
 template <int D, int BS, int KV_T>
@@ -85,20 +128,36 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
                     const __grid_constant__ CUtensorMap vmap, const PrefillParams p) {
   constexpr bool kBF = (KV_T == KV_BF16);
+  constexpr int kStages = pf_stages(D);
   constexpr int kSlabs = D / 64;                     // 128-byte slabs per row
   constexpr int kPartBytes = kPfKeys * D * 2;        // K (or V) of one stage
   constexpr int kStageBytes = 2 * kPartBytes;
+  constexpr int kQBytes = kPfRows * D * 2;
+  constexpr int kPBytes = kPfRows * kPfKeys * 2;     // one part (hi or lo) of P
   constexpr int kBlocksPerStage = kPfKeys / BS;
-  constexpr int KSD = D / 16;                        // k-steps over head_dim
+  constexpr uint32_t kAllBlocks = (1u << kBlocksPerStage) - 1u;
+  constexpr uint32_t kOCol = 2 * kPfKeys;            // first TMEM column of O
+  constexpr int kSCols = kPfKeys / kPfGroups;        // scores per thread per stage
+  constexpr int kOCols = D / kPfGroups;              // O columns per thread
   constexpr unsigned kFull = 0xffffffffu;
+  static_assert(kOCol + D <= kPfTmemCols, "TMEM budget");
+  static_assert(kSCols % 8 == 0 && (kOCols == 16 || kOCols == 32), "column split");
 
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full_bar[kPfStages];
-  __shared__ __align__(8) uint64_t empty_bar[kPfStages];
-  __shared__ uint32_t stage_mask[kPfStages];         // valid blocks of the stage
+  __shared__ __align__(8) uint64_t full_bar[kStages];
+  __shared__ __align__(8) uint64_t empty_bar[kStages];
+  __shared__ __align__(8) uint64_t s_full[2];
+  __shared__ __align__(8) uint64_t p_full[2];
+  __shared__ __align__(8) uint64_t o_done[2];
+  __shared__ __align__(8) uint64_t mma_idle;
+  __shared__ uint32_t stage_mask[kStages];         // valid blocks of the stage
+  __shared__ float red[2][kPfGroups][kPfRows];       // row maxima, then row sums
+  __shared__ uint32_t tmem_slot;
   __shared__ int s_abort;
   uint8_t *ring = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *qs = ring + kStages * kStageBytes;
+  uint8_t *ps = qs + kQBytes;
 
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -120,39 +179,68 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
 
   if (threadIdx.x == 0) {
     s_abort = 0;
-    for (int i = 0; i < kPfStages; ++i) {
+    for (int i = 0; i < kStages; ++i) {
       mbar_init(&full_bar[i], 1);
-      mbar_init(&empty_bar[i], kPfC);
+      mbar_init(&empty_bar[i], 1);
     }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], kPfSoftmax);
+      mbar_init(&o_done[i], 1);
+    }
+    mbar_init(&mma_idle, 1);
     fence_barrier_init();
   }
-  __syncthreads();
+  if (warp == kPfMmaWarp) tmem_alloc(&tmem_slot, kPfTmemCols);
 
-  if (warp == kPfC) {
+  // softmax threads: row and column group
+  const int row = (warp & 3) * 32 + lane;
+  const int cg = warp >> 2;
+  bool rvalid = false;
+  int rpos = 0x7fffffff;
+  int64_t rq = 0;
+  if (warp < kPfProducerWarp) {
+    const int tl = row / p.group, hl = row - tl * p.group;
+    rvalid = tl < p.tile_tokens && t0 + tl < cb;
+    if (rvalid) rpos = L - cb + t0 + tl;
+    rq = (static_cast<int64_t>(q0 + t0 + tl) * p.q_heads + g * p.group + hl) * D;
+    // this thread's share of the Q row -> shared memory, K-major, 128-byte
+    // swizzled (zeros past the tile)
+    const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(p.q) + rq);
+    constexpr int kQc = D / 8 / kPfGroups;
+#pragma unroll
+    for (int i = 0; i < kQc; ++i) {
+      const int c = cg * kQc + i;
+      const uint4 v = rvalid ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+      *reinterpret_cast<uint4 *>(qs + pf_chunk(row, c, kPfRows)) = v;
+    }
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tm = tmem_slot;
+
+  if (warp == kPfProducerWarp) {
     // ============================================================ producer
     if (lane == 0) {
       prefetch_tmap(&kmap);
       prefetch_tmap(&vmap);
     }
-    const int32_t *row = p.block_tables + static_cast<int64_t>(b) * p.max_blocks;
-    bool ok = true;
+    const int32_t *btab = p.block_tables + static_cast<int64_t>(b) * p.max_blocks;
     int issued = 0;
-    for (int st = 0; st < nstages && ok; ++st) {
-      const int s = st % kPfStages;
+    for (int st = 0; st < nstages; ++st) {
+      const int s = st % kStages;
       int okv = 1;
-      if (lane == 0 && st >= kPfStages)
-        okv = ring_wait_pf(&empty_bar[s], ((st / kPfStages) - 1) & 1, &s_abort, p.status);
+      if (lane == 0 && st >= kStages)
+        okv = ring_wait_pf(&empty_bar[s], ((st / kStages) - 1) & 1, &s_abort, p.status);
       okv = __shfl_sync(kFull, okv, 0);
-      if (!okv) {
-        ok = false;
-        break;
-      }
-      // block ids of the stage (lanes 0 .. kBlocksPerStage-1)
+      if (!okv) break;
       const int j0 = st * kBlocksPerStage;
       const int nblk = min(kBlocksPerStage, (nkeys - st * kPfKeys + BS - 1) / BS);
       int id = -1;
       if (lane < nblk) {
-        id = row[j0 + lane];
+        id = btab[j0 + lane];
         if (id < 0 || id >= p.num_blocks) {
           atomicOr(p.status, kErrBlockId);
           id = -1;
@@ -180,196 +268,204 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
       __syncwarp();
       ++issued;
     }
-    if (!ok && lane == 0) {
-      // aborted: let the loads still in flight land before the CTA can exit
-      for (int st = max(0, issued - kPfStages); st < issued; ++st)
-        mbar_wait(&full_bar[st % kPfStages], (st / kPfStages) & 1, nullptr, 100000000ull);
+    if (lane == 0) {
+      // let the loads still in flight land before the CTA can exit
+      for (int st = max(0, issued - kStages); st < issued; ++st)
+        mbar_wait(&full_bar[st % kStages], (st / kStages) & 1, nullptr, 100000000ull);
     }
-    return;
-  }
-
-  // ============================================================== consumers
-  const int gq = lane >> 2, cq = lane & 3;
-  // rows of this lane: gq and gq + 8 of the warp's 16
-  int rpos[2];
-  bool rvalid[2];
-  int64_t rq[2];
+    __syncwarp();
+  } else if (warp == kPfMmaWarp) {
+    // ============================================================ MMA issue
+    if (lane == 0) {
+      const uint32_t idesc_s = umma_idesc_f16<kBF>(kPfRows, kPfKeys, false);
+      const uint32_t idesc_o = umma_idesc_f16<kBF>(kPfRows, D, true);
+      const uint32_t q_addr = smem_u32(qs), p_addr = smem_u32(ps);
+      const uint32_t ring_addr = smem_u32(ring);
+      bool ok = true;
+      auto issue_s = [&](int j) {
+        const int s = j % kStages;
+        if (!ring_wait_pf(&full_bar[s], (j / kStages) & 1, &s_abort, p.status)) return false;
+        tc_fence_after();
+        const uint32_t kst = ring_addr + s * kStageBytes;
 #pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const int R = warp * 16 + gq + 8 * i;
-    const int tl = R / p.group, hl = R - tl * p.group;
-    rvalid[i] = tl < p.tile_tokens && t0 + tl < cb;
-    rpos[i] = rvalid[i] ? L - cb + t0 + tl : 0x7fffffff;
-    rq[i] = (static_cast<int64_t>(q0 + t0 + tl) * p.q_heads + g * p.group + hl) * D;
-  }
-  // Q as A fragments: a0 (row gq, dims 16k+2cq..), a1 (row gq+8), a2, a3 (+8 dims)
-  uint32_t qa[KSD][4];
-  {
-    const uint32_t *q32 = static_cast<const uint32_t *>(p.q);
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t koff = (ks & 3) * 32;
+          const uint64_t a = umma_desc_sw128(q_addr + (ks >> 2) * kPfRows * 128 + koff, 16, 1024);
+          const uint64_t bb = umma_desc_sw128(kst + (ks >> 2) * kPfKeys * 128 + koff, 16, 1024);
+          umma_f16(tm + (j & 1) * kPfKeys, a, bb, idesc_s, ks > 0);
+        }
+        umma_commit(&s_full[j & 1]);
+        return true;
+      };
+      ok = issue_s(0);
+      if (ok && nstages > 1) ok = issue_s(1);
+      for (int j = 0; ok && j < nstages; ++j) {
+        if (!ring_wait_pf(&p_full[j & 1], (j >> 1) & 1, &s_abort, p.status)) break;
+        tc_fence_after();
+        const uint32_t vst = ring_addr + (j % kStages) * kStageBytes + kPartBytes;
+        const uint32_t pb = p_addr + (j & 1) * 2 * kPBytes;
 #pragma unroll
-    for (int k = 0; k < KSD; ++k) {
-      qa[k][0] = rvalid[0] ? q32[(rq[0] + 16 * k + 2 * cq) >> 1] : 0u;
-      qa[k][1] = rvalid[1] ? q32[(rq[1] + 16 * k + 2 * cq) >> 1] : 0u;
-      qa[k][2] = rvalid[0] ? q32[(rq[0] + 16 * k + 8 + 2 * cq) >> 1] : 0u;
-      qa[k][3] = rvalid[1] ? q32[(rq[1] + 16 * k + 8 + 2 * cq) >> 1] : 0u;
+        for (int ks = 0; ks < 2 * kPfKeys / 16; ++ks) {  // P_hi V, then P_lo V
+          const int kk = ks & (kPfKeys / 16 - 1);
+          const uint64_t a =
+              umma_desc_sw128(pb + (ks >= kPfKeys / 16 ? kPBytes : 0) + kk * 32, 16, 1024);
+          const uint64_t bb = umma_desc_sw128(vst + kk * 16 * 128, kPfKeys * 128, 1024);
+          umma_f16(tm + kOCol, a, bb, idesc_o, j > 0 || ks > 0);
+        }
+        umma_commit(&empty_bar[j % kStages]);
+        umma_commit(&o_done[j & 1]);
+        if (j + 2 < nstages) ok = issue_s(j + 2);
+      }
+      // every MMA issued has finished before TMEM can be released
+      umma_commit(&mma_idle);
+      mbar_wait(&mma_idle, 0, p.status, 100000000ull);
     }
-  }
-  const int wmin = min(rpos[0], rpos[1]);  // this lane's earliest row position
-  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
-  float oacc[D / 8][4];
+    __syncwarp();
+  } else {
+    // ============================================================ softmax
+    // Every softmax thread runs every stage and every named barrier, also
+    // after a timeout (the waits then return at once), so none is left
+    // waiting at a barrier.
+    const uint32_t trow = tm + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const int c0 = cg * kSCols;                      // first score column
+    float m_used = -INFINITY, l_run = 0.f;
+    for (int j = 0; j < nstages; ++j) {
+      const int s = j % kStages;
+      ring_wait_pf(&s_full[j & 1], (j >> 1) & 1, &s_abort, p.status);
+      // the stage's TMA has landed (its full phase cannot advance before
+      // P_j V_j is done): gives this thread the block mask and the V bytes
+      ring_wait_pf(&full_bar[s], (j / kStages) & 1, &s_abort, p.status);
+      tc_fence_after();
+      float sv[kSCols];
+      {
+        uint32_t r[kSCols];
+        tmem_ld<kSCols>(trow + (j & 1) * kPfKeys + c0, r);
+        tmem_wait_ld();
 #pragma unroll
-  for (int n = 0; n < D / 8; ++n) oacc[n][0] = oacc[n][1] = oacc[n][2] = oacc[n][3] = 0.f;
-  bool alive = true;
-
-  for (int st = 0; st < nstages; ++st) {
-    const int s = st % kPfStages;
-    if (alive) {
-      int okv = 1;
-      if (lane == 0) okv = ring_wait_pf(&full_bar[s], (st / kPfStages) & 1, &s_abort, p.status);
-      okv = __shfl_sync(kFull, okv, 0);
-      if (!okv) alive = false;
+        for (int c = 0; c < kSCols; ++c) sv[c] = __uint_as_float(r[c]) * p.scale_log2;
+      }
+      const int key0 = j * kPfKeys;
+      const uint32_t bmask = stage_mask[s];
+      const bool tail = key0 + kPfKeys > nkeys || bmask != kAllBlocks;
+      const bool need_mask = tail || key0 + c0 + kSCols - 1 > rpos;
+      float mx = -INFINITY;
+      if (need_mask) {
+#pragma unroll
+        for (int c = 0; c < kSCols; ++c) {
+          const int kp = key0 + c0 + c;
+          const bool ok = kp <= rpos && kp < nkeys && ((bmask >> ((c0 + c) / BS)) & 1u);
+          sv[c] = ok ? sv[c] : -INFINITY;
+          mx = fmaxf(mx, sv[c]);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < kSCols; ++c) mx = fmaxf(mx, sv[c]);
+      }
+      red[j & 1][cg][row] = mx;
+      bar_sync(1, kPfSoftmax);
+#pragma unroll
+      for (int q = 0; q < kPfGroups; ++q) mx = fmaxf(mx, red[j & 1][q][row]);
+      // lazy maximum: raise it only when a score exceeds it by more than 2^8
+      // (every thread of the row takes the same decision)
+      float alpha = 1.f;
+      if (m_used == -INFINITY) {
+        m_used = mx;
+      } else if (mx > m_used + kPfRescaleLog2) {
+        alpha = ex2f(m_used - mx);
+        m_used = mx;
+        l_run *= alpha;
+      }
+      if (__any_sync(kFull, alpha != 1.f)) {
+        // O holds P_0..P_{j-1} V: wait for the last of them, rescale this
+        // thread's columns of its row
+        ring_wait_pf(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, &s_abort, p.status);
+        tc_fence_after();
+        uint32_t o[kOCols];
+        tmem_ld<kOCols>(trow + kOCol + cg * kOCols, o);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < kOCols; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+        tmem_st<kOCols>(trow + kOCol + cg * kOCols, o);
+        tmem_wait_st();
+      }
+      const float ms = m_used == -INFINITY ? 0.f : m_used;
+      float ls = 0.f;
+      uint8_t *phi = ps + (j & 1) * 2 * kPBytes;
+      uint8_t *plo = phi + kPBytes;
+#pragma unroll
+      for (int c8 = 0; c8 < kSCols / 8; ++c8) {
+        uint32_t wh[4], wl[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float a0 = ex2f(sv[c8 * 8 + 2 * e] - ms);
+          const float a1 = ex2f(sv[c8 * 8 + 2 * e + 1] - ms);
+          ls += a0 + a1;
+          split_p<kBF>(a0, a1, wh[e], wl[e]);
+        }
+        const uint32_t off = pf_chunk(row, c0 / 8 + c8, kPfRows);
+        *reinterpret_cast<uint4 *>(phi + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+        *reinterpret_cast<uint4 *>(plo + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+      }
+      l_run += ls;
+      if (tail) {
+        // V rows that hold no real position of this stage (past the keys the
+        // tile reads, or of a block that was not loaded) may hold anything:
+        // zero them so that P = 0 there cannot meet a NaN.
+        uint8_t *vpart = ring + s * kStageBytes + kPartBytes;
+        constexpr int kChunks = kPfKeys * D / 8;     // 16-byte chunks of V
+#pragma unroll
+        for (int i = 0; i < kChunks / kPfSoftmax; ++i) {
+          const int idx = threadIdx.x + i * kPfSoftmax;
+          const int kr = idx / (D / 8), c = idx % (D / 8);
+          const bool real = key0 + kr < nkeys && ((bmask >> (kr / BS)) & 1u);
+          if (!real)
+            *reinterpret_cast<uint4 *>(vpart + (c >> 3) * kPfKeys * 128 + kr * 128 + (c & 7) * 16) =
+                make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&p_full[j & 1]);
     }
-    if (alive) {
-      while (!mbar_try_wait(&full_bar[s], (st / kPfStages) & 1)) {
-      }  // already complete: gives every lane the acquire
-      const uint32_t kbase = smem_u32(ring + s * kStageBytes);
-      const uint32_t vbase = kbase + kPartBytes;
-      const uint32_t vmask_blocks = stage_mask[s];
-      const int key0 = st * kPfKeys;
+    // ------------------------------------------------------------- output
+    // row sums through the buffer the last stage's maxima did not use
+    red[nstages & 1][cg][row] = l_run;
+    ring_wait_pf(&o_done[(nstages - 1) & 1], ((nstages - 1) >> 1) & 1, &s_abort, p.status);
+    bar_sync(1, kPfSoftmax);
+    float l_tot = 0.f;
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int hk = half * 32;  // first stage row of this half
-        // -------------------------------------------- S = Q K^T (16 x 32)
-        float sc[4][4];
+    for (int q = 0; q < kPfGroups; ++q) l_tot += red[nstages & 1][q][row];
+    if (!__any_sync(kFull, s_abort != 0)) {  // warp-uniform: TMEM loads are warp-wide
+      tc_fence_after();
+      const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
+      uint32_t o[kOCols];
+      tmem_ld<kOCols>(trow + kOCol + cg * kOCols, o);
+      tmem_wait_ld();
+      if (rvalid) {
+        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + rq + cg * kOCols);
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt) {
-          sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+        for (int c4 = 0; c4 < kOCols / 8; ++c4) {
+          uint32_t w[4];
 #pragma unroll
-          for (int k2 = 0; k2 < KSD / 2; ++k2) {
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4(pf_chunk(kbase, hk + nt * 8 + (lane & 7), 4 * k2 + (lane >> 3), kPfKeys),
-                    b0, b1, b2, b3);
-            mma16816<kBF>(sc[nt], qa[2 * k2][0], qa[2 * k2][1], qa[2 * k2][2], qa[2 * k2][3],
-                          b0, b1);
-            mma16816<kBF>(sc[nt], qa[2 * k2 + 1][0], qa[2 * k2 + 1][1], qa[2 * k2 + 1][2],
-                          qa[2 * k2 + 1][3], b2, b3);
-          }
-        }
-        // ------------------------------------- scale, mask, online softmax
-        const int kh = key0 + hk;  // position of this half's first row
-        constexpr uint32_t kAll = (1u << kBlocksPerStage) - 1u;
-        const bool need_mask =
-            (kh + 31 > wmin) || (kh + 32 > nkeys) || (vmask_blocks & kAll) != kAll;
-        float bm[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int i = e >> 1;
-            const int kp = kh + nt * 8 + 2 * cq + (e & 1);
-            float v = sc[nt][e] * p.scale_log2;
-            if (need_mask) {
-              const int blk = (kp - key0) / BS;
-              const bool ok = kp <= rpos[i] && kp < nkeys && ((vmask_blocks >> blk) & 1u);
-              v = ok ? v : -INFINITY;
-            }
-            sc[nt][e] = v;
-            bm[i] = fmaxf(bm[i], v);
-          }
-        }
-        float al[2];
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          bm[i] = fmaxf(bm[i], __shfl_xor_sync(kFull, bm[i], 1));
-          bm[i] = fmaxf(bm[i], __shfl_xor_sync(kFull, bm[i], 2));
-          const float mn = fmaxf(m_run[i], bm[i]);
-          al[i] = mn == m_run[i] ? 1.f : ex2f(m_run[i] - mn);
-          m_run[i] = mn;
-        }
-        const float ms0 = m_run[0] == -INFINITY ? 0.f : m_run[0];
-        const float ms1 = m_run[1] == -INFINITY ? 0.f : m_run[1];
-        float ls[2] = {0.f, 0.f};
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt) {
-          sc[nt][0] = ex2f(sc[nt][0] - ms0);
-          sc[nt][1] = ex2f(sc[nt][1] - ms0);
-          sc[nt][2] = ex2f(sc[nt][2] - ms1);
-          sc[nt][3] = ex2f(sc[nt][3] - ms1);
-          ls[0] += sc[nt][0] + sc[nt][1];
-          ls[1] += sc[nt][2] + sc[nt][3];
-        }
-        l_run[0] = l_run[0] * al[0] + ls[0];
-        l_run[1] = l_run[1] * al[1] + ls[1];
-        if (__any_sync(kFull, al[0] != 1.f || al[1] != 1.f)) {
-#pragma unroll
-          for (int n = 0; n < D / 8; ++n) {
-            oacc[n][0] *= al[0];
-            oacc[n][1] *= al[0];
-            oacc[n][2] *= al[1];
-            oacc[n][3] *= al[1];
-          }
-        }
-        // ---------------------------------------------------- O += P V
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {  // 16 positions each
-          uint32_t ph[4], pl[4];
-          split2<kBF>(sc[2 * kk][0], sc[2 * kk][1], ph[0], pl[0]);
-          split2<kBF>(sc[2 * kk][2], sc[2 * kk][3], ph[1], pl[1]);
-          split2<kBF>(sc[2 * kk + 1][0], sc[2 * kk + 1][1], ph[2], pl[2]);
-          split2<kBF>(sc[2 * kk + 1][2], sc[2 * kk + 1][3], ph[3], pl[3]);
-          // V rows this lane's B fragments cover: positions 2cq, 2cq+1 (b0)
-          // and 2cq+8, 2cq+9 (b1) of the 16; zero them when not real tokens
-          // (stale shared memory may hold anything)
-          uint32_t vm0 = 0xffffffffu, vm1 = 0xffffffffu;
-          if (need_mask) {
-            const int kb = kh + kk * 16 + 2 * cq;
-            auto real = [&](int kp) {
-              return kp < nkeys && ((vmask_blocks >> ((kp - key0) / BS)) & 1u);
-            };
-            vm0 = (real(kb) ? 0xffffu : 0u) | (real(kb + 1) ? 0xffff0000u : 0u);
-            vm1 = (real(kb + 8) ? 0xffffu : 0u) | (real(kb + 9) ? 0xffff0000u : 0u);
-          }
-#pragma unroll
-          for (int n2 = 0; n2 < D / 16; ++n2) {
-            uint32_t b0, b1, b2, b3;  // dims 16n2.. (b0, b1), 16n2+8.. (b2, b3)
-            const int vr = hk + kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-            ldsm_x4_t(pf_chunk(vbase, vr, 2 * n2 + (lane >> 4), kPfKeys), b0, b1, b2, b3);
-            b0 &= vm0;
-            b1 &= vm1;
-            b2 &= vm0;
-            b3 &= vm1;
-            mma16816<kBF>(oacc[2 * n2], ph[0], ph[1], ph[2], ph[3], b0, b1);
-            mma16816<kBF>(oacc[2 * n2], pl[0], pl[1], pl[2], pl[3], b0, b1);
-            mma16816<kBF>(oacc[2 * n2 + 1], ph[0], ph[1], ph[2], ph[3], b2, b3);
-            mma16816<kBF>(oacc[2 * n2 + 1], pl[0], pl[1], pl[2], pl[3], b2, b3);
-          }
+          for (int e = 0; e < 4; ++e)
+            w[e] = pack2<kBF>(__uint_as_float(o[c4 * 8 + 2 * e]) * inv,
+                              __uint_as_float(o[c4 * 8 + 2 * e + 1]) * inv);
+          dst[c4] = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty_bar[s]);
   }
-
-  // ------------------------------------------------------------- output
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    l_run[i] += __shfl_xor_sync(kFull, l_run[i], 1);
-    l_run[i] += __shfl_xor_sync(kFull, l_run[i], 2);
-  }
-  const float inv0 = (alive && l_run[0] > 0.f) ? 1.f / l_run[0] : 0.f;
-  const float inv1 = (alive && l_run[1] > 0.f) ? 1.f / l_run[1] : 0.f;
-  uint32_t *o32 = static_cast<uint32_t *>(p.out);
-#pragma unroll
-  for (int n = 0; n < D / 8; ++n) {
-    if (rvalid[0]) o32[(rq[0] + 8 * n + 2 * cq) >> 1] = pack2<kBF>(oacc[n][0] * inv0, oacc[n][1] * inv0);
-    if (rvalid[1]) o32[(rq[1] + 8 * n + 2 * cq) >> 1] = pack2<kBF>(oacc[n][2] * inv1, oacc[n][3] * inv1);
-  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kPfMmaWarp) tmem_dealloc(tm, kPfTmemCols);
 }
 
 template <int D, int BS, int KV_T>
 cudaError_t launch_prefill(const CUtensorMap &km, const CUtensorMap &vm, const PrefillParams &p,
                            int tiles, cudaStream_t st) {
-  constexpr int smem = kPfStages * 2 * kPfKeys * D * 2 + 1024;
+  constexpr int smem =
+      pf_stages(D) * 2 * kPfKeys * D * 2 + kPfRows * D * 2 + 4 * kPfRows * kPfKeys * 2 + 1024;
   auto kern = attn_prefill_kernel<D, BS, KV_T>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;

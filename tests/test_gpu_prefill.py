@@ -107,3 +107,37 @@ def test_prefill_bad_chunk_is_reported(pkv):
     ref = attention.paged_prefill(to_np(pw.q[:10], np.float64), pw.cu_q[:2], k, v,
                                   wl.block_tables[:1], wl.context_lens[:1], wl.scale)
     compare(out[:10], ref, what="good sequence")
+
+
+@pytest.mark.parametrize("D,bs", [(128, 16), (64, 32)])
+def test_prefill_ignores_nan_past_the_context(pkv, D, bs):
+    """Cache rows past each sequence's last position (the tail of its last
+    block) and blocks no table names hold NaN: they are never attended, so
+    the output is finite and matches the oracle."""
+    pw = W.make_prefill_workload("nan", 16, 2, D, bs, "bf16", [37, 300, 129, 70], [37, 45, 9, 70],
+                                 seed=14, device=DEV)
+    wl = pw.cache
+    pool = build_pool(pkv, wl, DEV)
+    K, V, _, _ = pool.layer_views(0)
+    used = set()
+    for b, L in enumerate(wl.context_lens):
+        nb = (int(L) + bs - 1) // bs
+        used.update(int(x) for x in wl.block_tables[b][:nb])
+        last = int(wl.block_tables[b][nb - 1])
+        if L % bs:
+            K[last, :, int(L) % bs:] = float("nan")
+            V[last, :, int(L) % bs:] = float("nan")
+    for blk in range(wl.num_blocks):
+        if blk not in used:
+            K[blk] = float("nan")
+            V[blk] = float("nan")
+    tables, lens = device_inputs(wl, DEV)
+    cu = torch.from_numpy(pw.cu_q).to(DEV)
+    out = pkv.paged_attn_prefill(pool, 0, pw.q, cu, int(pw.chunk_lens.max()), tables, lens,
+                                 int(wl.context_lens.max()), wl.scale)
+    torch.cuda.synchronize()
+    assert pool.status() == 0
+    k, v = _cache_16(wl)
+    ref = attention.paged_prefill(to_np(pw.q, np.float64), pw.cu_q, k, v, wl.block_tables,
+                                  wl.context_lens, wl.scale)
+    compare(out, ref, what="nan tail")
