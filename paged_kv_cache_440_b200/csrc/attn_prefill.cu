@@ -12,15 +12,18 @@
 //   are (token, query head of the KV head's group) pairs, head fastest:
 //   128 / G tokens x G heads. Row r lives in TMEM lane r.
 // * The producer warp streams the KV head's cached blocks, 64 positions per
-//   stage (K then V, 128-byte swizzled TMA boxes of one block-head slab), into
-//   a 4-stage ring.
-// * The MMA warp (one thread) issues tcgen05 MMAs: S_j = Q K_j^T (M 128,
-//   N 64, K head_dim; Q and K both K-major in shared memory) into one of two
-//   TMEM score buffers, and O += P_j V_j (M 128, N head_dim, K 64; P K-major,
-//   V MN-major straight from the TMA stage) into a TMEM accumulator that stays
-//   resident for the whole key range. Order: S_0, S_1, then per stage j
-//   O += P_j V_j followed by S_{j+2}, so the tensor core computes the next
-//   scores while the softmax warps work on the current ones.
+//   stage (K then V, 128-byte swizzled TMA boxes of one block-head slab, one
+//   box per lane), into a ring of 6 (head_dim 128) or 8 (64) stages; block
+//   ids are read a 32-block window ahead.
+// * The MMA warp (one thread) issues tcgen05 MMAs with the A operand in
+//   tensor memory and B in shared memory: S_j = Q K_j^T (M 128, N 64,
+//   K head_dim; Q in TMEM, K K-major from the TMA stage) into one of two TMEM
+//   score buffers, and O += P_j V_j (M 128, N head_dim, K 64; P in TMEM, V
+//   MN-major from the TMA stage) into a TMEM accumulator that stays resident
+//   for the whole key range. Order: S_0, S_1, then per stage j O += P_j V_j
+//   followed by S_{j+2}, so the tensor core computes the next scores while
+//   the softmax warps work on the current ones. Shared memory only carries
+//   K and V: its bandwidth, not the tensor core, is the tighter limit.
 // * 16 softmax warps: warp w reads TMEM lanes 32 (w mod 4) .. + 31 (the
 //   lanes a warp may access) and columns of group w / 4, so four threads share
 //   a row, 16 scores each per stage; the row maximum is combined through
@@ -29,10 +32,10 @@
 //   l rescaled in TMEM) when a new score exceeds it by more than 2^8;
 //   otherwise the stale maximum stays in use, which keeps every P value below
 //   256 and leaves the result unchanged up to rounding.
-// * P_j goes to shared memory in the 128-byte swizzled K-major layout the MMA
-//   reads, as two 16-bit parts hi + lo; O accumulates P_hi V + P_lo V, so
-//   rounding P to 16 bits costs nothing measurable (bf16: hi and lo by
-//   truncation, bit masks only; fp16: by rounding conversions).
+// * P_j overwrites S_j in TMEM, each thread in its own 16 columns, as two
+//   16-bit parts hi + lo (8 columns of packed pairs each); O accumulates
+//   P_hi V + P_lo V, so rounding P to 16 bits costs nothing measurable (bf16:
+//   hi and lo by truncation, bit masks only; fp16: by rounding conversions).
 // * Synchronisation is by mbarriers: TMA -> MMA (full), MMA -> producer
 //   (stage free, by tcgen05.commit after P_j V_j), MMA -> softmax (S_j ready),
 //   softmax -> MMA (P_j written), MMA -> softmax (P_j V_j done, needed only to
@@ -53,14 +56,15 @@ using namespace dev;
 constexpr int kPfRows = 128;            // query rows per CTA (TMEM lanes)
 constexpr int kPfGroups = 4;            // softmax threads per row (column groups)
 constexpr int kPfSoftmax = 128 * kPfGroups;
-constexpr int kPfProducerWarp = kPfSoftmax / 32;
-constexpr int kPfMmaWarp = kPfProducerWarp + 1;
-constexpr int kPfThreads = kPfSoftmax + 64;
+constexpr int kPfProducerWarp = kPfSoftmax / 32;  // K boxes; the next warp: V boxes
+constexpr int kPfMmaWarp = kPfProducerWarp + 2;
+constexpr int kPfThreads = kPfSoftmax + 96;
 constexpr int kPfKeys = 64;             // positions per stage
-// Ring depth: 3 stages of 32 KB for head_dim 128 (shared memory then holds
-// the ring, Q, and two hi + lo P buffers: 193 KB), 4 of 16 KB for 64.
-__host__ __device__ constexpr int pf_stages(int D) { return D == 128 ? 3 : 4; }
-constexpr uint32_t kPfTmemCols = 256;   // S: 2 x 64 columns, O: head_dim columns
+// Ring depth: 6 stages of 32 KB for head_dim 128, 8 of 16 KB for 64.
+__host__ __device__ constexpr int pf_stages(int D) { return D == 128 ? 6 : 8; }
+constexpr int kPfSBufs = 3;             // S/P buffers in TMEM
+// TMEM columns: S/P 3 x 64, O head_dim, Q head_dim / 2 (packed pairs)
+constexpr uint32_t kPfTmemCols = 512;
 constexpr float kPfRescaleLog2 = 8.f;   // raise the running max only beyond 2^8
 
 struct PrefillParams {
@@ -83,28 +87,21 @@ __device__ __forceinline__ float ex2f(float x) {
 
 // Bounded wait on a pipeline barrier; gives up (false) when another role has
 // given up or after the time limit, recording KV_DEVERR_TIMEOUT.
+// The waiting thread sleeps in the barrier (woken when the phase completes)
+// rather than spinning, leaving issue slots to the warps that do the work.
 __device__ __forceinline__ bool ring_wait_pf(uint64_t *bar, uint32_t parity, volatile int *abort,
                                              int *status) {
   if (mbar_try_wait(bar, parity)) return true;
-  if (*abort) return false;
   const uint64_t t0 = globaltimer();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63) == 0) {
-      if (*abort) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
-        *abort = 1;
-        atomicOr(status, kDevErrTimeout);
-        return false;
-      }
+  for (;;) {
+    if (*abort) return false;
+    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      *abort = 1;
+      atomicOr(status, kDevErrTimeout);
+      return false;
     }
   }
-}
-
-// Byte offset of 16-byte chunk c of row r in a tile of `rows` rows stored as
-// 128-byte slabs (slab-major), 128-byte swizzled.
-__device__ __forceinline__ uint32_t pf_chunk(int r, int c, int rows) {
-  return (c >> 3) * rows * 128 + (r << 7) + (((c & 7) ^ (r & 7)) << 4);
 }
 
 // Two P values -> 16-bit pairs hi + lo (low half = first value).
@@ -132,22 +129,22 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
   constexpr int kSlabs = D / 64;                     // 128-byte slabs per row
   constexpr int kPartBytes = kPfKeys * D * 2;        // K (or V) of one stage
   constexpr int kStageBytes = 2 * kPartBytes;
-  constexpr int kQBytes = kPfRows * D * 2;
-  constexpr int kPBytes = kPfRows * kPfKeys * 2;     // one part (hi or lo) of P
   constexpr int kBlocksPerStage = kPfKeys / BS;
   constexpr uint32_t kAllBlocks = (1u << kBlocksPerStage) - 1u;
-  constexpr uint32_t kOCol = 2 * kPfKeys;            // first TMEM column of O
+  constexpr uint32_t kOCol = kPfSBufs * kPfKeys;     // first TMEM column of O
+  constexpr uint32_t kQCol = kOCol + D;              // first TMEM column of Q
+  constexpr uint32_t kTmemCols = kPfTmemCols;
   constexpr int kSCols = kPfKeys / kPfGroups;        // scores per thread per stage
   constexpr int kOCols = D / kPfGroups;              // O columns per thread
   constexpr unsigned kFull = 0xffffffffu;
-  static_assert(kOCol + D <= kPfTmemCols, "TMEM budget");
-  static_assert(kSCols % 8 == 0 && (kOCols == 16 || kOCols == 32), "column split");
+  static_assert(kQCol + D / 2 <= kTmemCols, "TMEM budget");
+  static_assert(kSCols == 16 && (kOCols == 16 || kOCols == 32), "column split");
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[kStages];
   __shared__ __align__(8) uint64_t empty_bar[kStages];
-  __shared__ __align__(8) uint64_t s_full[2];
-  __shared__ __align__(8) uint64_t p_full[2];
+  __shared__ __align__(8) uint64_t s_full[kPfSBufs];
+  __shared__ __align__(8) uint64_t p_full[kPfSBufs];
   __shared__ __align__(8) uint64_t o_done[2];
   __shared__ __align__(8) uint64_t mma_idle;
   __shared__ uint32_t stage_mask[kStages];         // valid blocks of the stage
@@ -156,8 +153,6 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
   __shared__ int s_abort;
   uint8_t *ring = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t *qs = ring + kStages * kStageBytes;
-  uint8_t *ps = qs + kQBytes;
 
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -183,15 +178,19 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
       mbar_init(&full_bar[i], 1);
       mbar_init(&empty_bar[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kPfSBufs; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], kPfSoftmax);
-      mbar_init(&o_done[i], 1);
     }
+    for (int i = 0; i < 2; ++i) mbar_init(&o_done[i], 1);
     mbar_init(&mma_idle, 1);
     fence_barrier_init();
   }
-  if (warp == kPfMmaWarp) tmem_alloc(&tmem_slot, kPfTmemCols);
+  if (warp == kPfMmaWarp) tmem_alloc(&tmem_slot, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tm = tmem_slot;
 
   // softmax threads: row and column group
   const int row = (warp & 3) * 32 + lane;
@@ -204,66 +203,82 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
     rvalid = tl < p.tile_tokens && t0 + tl < cb;
     if (rvalid) rpos = L - cb + t0 + tl;
     rq = (static_cast<int64_t>(q0 + t0 + tl) * p.q_heads + g * p.group + hl) * D;
-    // this thread's share of the Q row -> shared memory, K-major, 128-byte
-    // swizzled (zeros past the tile)
-    const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(p.q) + rq);
-    constexpr int kQc = D / 8 / kPfGroups;
+    // Q row -> TMEM as packed 16-bit pairs (zeros past the tile): groups
+    // 0 .. D/32 - 1 each write 32 dims (16 columns)
+    if (cg < D / 32) {
+      const uint4 *src =
+          reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(p.q) + rq) + cg * 4;
+      uint32_t v[16];
 #pragma unroll
-    for (int i = 0; i < kQc; ++i) {
-      const int c = cg * kQc + i;
-      const uint4 v = rvalid ? src[c] : make_uint4(0u, 0u, 0u, 0u);
-      *reinterpret_cast<uint4 *>(qs + pf_chunk(row, c, kPfRows)) = v;
+      for (int i = 0; i < 4; ++i) {
+        const uint4 x = rvalid ? src[i] : make_uint4(0u, 0u, 0u, 0u);
+        v[4 * i] = x.x;
+        v[4 * i + 1] = x.y;
+        v[4 * i + 2] = x.z;
+        v[4 * i + 3] = x.w;
+      }
+      tmem_st16(tm + (static_cast<uint32_t>((warp & 3) * 32) << 16) + kQCol + cg * 16, v);
+      tmem_wait_st();
     }
-    fence_proxy_async_smem();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tm = tmem_slot;
 
-  if (warp == kPfProducerWarp) {
-    // ============================================================ producer
+  if (warp == kPfProducerWarp || warp == kPfProducerWarp + 1) {
+    // ============================================================ producers
     if (lane == 0) {
       prefetch_tmap(&kmap);
       prefetch_tmap(&vmap);
     }
+    // Two warps, one for the K boxes and one for the V boxes of every stage
+    // (one box per block and slab, each issued by its own lane). Block ids
+    // travel one 32-block window per lane-wide load, fetched a window ahead.
+    const int kv = warp - kPfProducerWarp;
     const int32_t *btab = p.block_tables + static_cast<int64_t>(b) * p.max_blocks;
+    const int nblocks = (nkeys + BS - 1) / BS;
+    auto load_ids = [&](int w) {
+      const int jb = w * 32 + lane;
+      int id = -1;
+      if (jb < nblocks) {
+        id = btab[jb];
+        if (id < 0 || id >= p.num_blocks) {
+          if (kv == 0) atomicOr(p.status, kErrBlockId);
+          id = -1;
+        }
+      }
+      return id;
+    };
+    int cur = load_ids(0), nxt = load_ids(1);
+    uint32_t cur_ok = __ballot_sync(kFull, cur >= 0);
     int issued = 0;
+    constexpr int kBoxes = kBlocksPerStage * kSlabs;  // this warp's TMA boxes of a full stage
+    static_assert(kBoxes <= 32, "one box per lane");
     for (int st = 0; st < nstages; ++st) {
       const int s = st % kStages;
+      const int jb0 = st * kBlocksPerStage;        // first block of the stage
+      if (jb0 > 0 && (jb0 & 31) == 0) {            // next window
+        cur = nxt;
+        cur_ok = __ballot_sync(kFull, cur >= 0);
+        nxt = load_ids(jb0 / 32 + 1);
+      }
       int okv = 1;
       if (lane == 0 && st >= kStages)
         okv = ring_wait_pf(&empty_bar[s], ((st / kStages) - 1) & 1, &s_abort, p.status);
       okv = __shfl_sync(kFull, okv, 0);
       if (!okv) break;
-      const int j0 = st * kBlocksPerStage;
-      const int nblk = min(kBlocksPerStage, (nkeys - st * kPfKeys + BS - 1) / BS);
-      int id = -1;
-      if (lane < nblk) {
-        id = btab[j0 + lane];
-        if (id < 0 || id >= p.num_blocks) {
-          atomicOr(p.status, kErrBlockId);
-          id = -1;
-        }
-      }
-      const uint32_t valid = __ballot_sync(kFull, id >= 0);
-      if (lane == 0) {
+      const int nblk = min(kBlocksPerStage, nblocks - jb0);
+      const uint32_t valid = (cur_ok >> (jb0 & 31)) & ((1u << nblk) - 1u);
+      if (lane == 0 && kv == 0) {  // the V warp's bytes may land first: tx counts may go negative
         stage_mask[s] = valid;
         mbar_arrive_expect_tx(&full_bar[s], __popc(valid) * 2 * BS * D * 2);
       }
-      for (int j = 0; j < nblk; ++j) {
-        const int bid = __shfl_sync(kFull, id, j);
-        if (lane == 0 && bid >= 0) {
-          uint8_t *kst = ring + s * kStageBytes;
-          uint8_t *vst = kst + kPartBytes;
-          const int y = (bid * p.kv_heads + g) * BS;
-#pragma unroll
-          for (int sl = 0; sl < kSlabs; ++sl) {
-            const int off = (sl * kPfKeys + j * BS) * 128;
-            tma_load_2d(kst + off, &kmap, &full_bar[s], sl * 64, y);
-            tma_load_2d(vst + off, &vmap, &full_bar[s], sl * 64, y);
-          }
-        }
+      // lane -> (block j, slab)
+      const int j = lane / kSlabs, sl = lane % kSlabs;
+      const int bid = __shfl_sync(kFull, cur, (jb0 & 31) + (j < kBlocksPerStage ? j : 0));
+      if (lane < kBoxes && j < nblk && ((valid >> j) & 1u)) {
+        uint8_t *dst = ring + s * kStageBytes + kv * kPartBytes + (sl * kPfKeys + j * BS) * 128;
+        tma_load_2d(dst, kv ? &vmap : &kmap, &full_bar[s], sl * 64, (bid * p.kv_heads + g) * BS);
       }
       __syncwarp();
       ++issued;
@@ -279,42 +294,41 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
     if (lane == 0) {
       const uint32_t idesc_s = umma_idesc_f16<kBF>(kPfRows, kPfKeys, false);
       const uint32_t idesc_o = umma_idesc_f16<kBF>(kPfRows, D, true);
-      const uint32_t q_addr = smem_u32(qs), p_addr = smem_u32(ps);
-      const uint32_t ring_addr = smem_u32(ring);
+      // descriptors of stage 0; other stages and K steps add their byte
+      // offset / 16 to the start-address field (no carry: shared addresses
+      // stay below 256 KB)
+      const uint64_t kdesc0 = umma_desc_sw128(smem_u32(ring), 16, 1024);
+      const uint64_t vdesc0 = umma_desc_sw128(smem_u32(ring) + kPartBytes, kPfKeys * 128, 1024);
       bool ok = true;
       auto issue_s = [&](int j) {
         const int s = j % kStages;
         if (!ring_wait_pf(&full_bar[s], (j / kStages) & 1, &s_abort, p.status)) return false;
         tc_fence_after();
-        const uint32_t kst = ring_addr + s * kStageBytes;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t koff = (ks & 3) * 32;
-          const uint64_t a = umma_desc_sw128(q_addr + (ks >> 2) * kPfRows * 128 + koff, 16, 1024);
-          const uint64_t bb = umma_desc_sw128(kst + (ks >> 2) * kPfKeys * 128 + koff, 16, 1024);
-          umma_f16(tm + (j & 1) * kPfKeys, a, bb, idesc_s, ks > 0);
+          const uint32_t off = s * kStageBytes + (ks >> 2) * kPfKeys * 128 + (ks & 3) * 32;
+          umma_f16_tmem_a(tm + (j % kPfSBufs) * kPfKeys, tm + kQCol + ks * 8, kdesc0 + (off >> 4),
+                          idesc_s, ks > 0);
         }
-        umma_commit(&s_full[j & 1]);
+        umma_commit(&s_full[j % kPfSBufs]);
         return true;
       };
-      ok = issue_s(0);
-      if (ok && nstages > 1) ok = issue_s(1);
+      for (int j = 0; ok && j < min(nstages, kPfSBufs); ++j) ok = issue_s(j);
       for (int j = 0; ok && j < nstages; ++j) {
-        if (!ring_wait_pf(&p_full[j & 1], (j >> 1) & 1, &s_abort, p.status)) break;
+        if (!ring_wait_pf(&p_full[j % kPfSBufs], (j / kPfSBufs) & 1, &s_abort, p.status)) break;
         tc_fence_after();
-        const uint32_t vst = ring_addr + (j % kStages) * kStageBytes + kPartBytes;
-        const uint32_t pb = p_addr + (j & 1) * 2 * kPBytes;
+        const uint32_t pcol = tm + (j % kPfSBufs) * kPfKeys;
 #pragma unroll
         for (int ks = 0; ks < 2 * kPfKeys / 16; ++ks) {  // P_hi V, then P_lo V
           const int kk = ks & (kPfKeys / 16 - 1);
-          const uint64_t a =
-              umma_desc_sw128(pb + (ks >= kPfKeys / 16 ? kPBytes : 0) + kk * 32, 16, 1024);
-          const uint64_t bb = umma_desc_sw128(vst + kk * 16 * 128, kPfKeys * 128, 1024);
-          umma_f16(tm + kOCol, a, bb, idesc_o, j > 0 || ks > 0);
+          const uint32_t off = (j % kStages) * kStageBytes + kk * 16 * 128;
+          umma_f16_tmem_a(tm + kOCol, pcol + kk * 16 + (ks >= kPfKeys / 16 ? 8 : 0),
+                          vdesc0 + (off >> 4), idesc_o, j > 0 || ks > 0);
         }
         umma_commit(&empty_bar[j % kStages]);
         umma_commit(&o_done[j & 1]);
-        if (j + 2 < nstages) ok = issue_s(j + 2);
+        // S_{j+3} reuses S_j's columns: issued after P_j V_j, which reads them
+        if (j + kPfSBufs < nstages) ok = issue_s(j + kPfSBufs);
       }
       // every MMA issued has finished before TMEM can be released
       umma_commit(&mma_idle);
@@ -331,7 +345,7 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
     float m_used = -INFINITY, l_run = 0.f;
     for (int j = 0; j < nstages; ++j) {
       const int s = j % kStages;
-      ring_wait_pf(&s_full[j & 1], (j >> 1) & 1, &s_abort, p.status);
+      ring_wait_pf(&s_full[j % kPfSBufs], (j / kPfSBufs) & 1, &s_abort, p.status);
       // the stage's TMA has landed (its full phase cannot advance before
       // P_j V_j is done): gives this thread the block mask and the V bytes
       ring_wait_pf(&full_bar[s], (j / kStages) & 1, &s_abort, p.status);
@@ -339,7 +353,7 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
       float sv[kSCols];
       {
         uint32_t r[kSCols];
-        tmem_ld<kSCols>(trow + (j & 1) * kPfKeys + c0, r);
+        tmem_ld<kSCols>(trow + (j % kPfSBufs) * kPfKeys + c0, r);
         tmem_wait_ld();
 #pragma unroll
         for (int c = 0; c < kSCols; ++c) sv[c] = __uint_as_float(r[c]) * p.scale_log2;
@@ -390,22 +404,15 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
       }
       const float ms = m_used == -INFINITY ? 0.f : m_used;
       float ls = 0.f;
-      uint8_t *phi = ps + (j & 1) * 2 * kPBytes;
-      uint8_t *plo = phi + kPBytes;
+      uint32_t pw[16];                               // 8 hi pairs, then 8 lo pairs
 #pragma unroll
-      for (int c8 = 0; c8 < kSCols / 8; ++c8) {
-        uint32_t wh[4], wl[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float a0 = ex2f(sv[c8 * 8 + 2 * e] - ms);
-          const float a1 = ex2f(sv[c8 * 8 + 2 * e + 1] - ms);
-          ls += a0 + a1;
-          split_p<kBF>(a0, a1, wh[e], wl[e]);
-        }
-        const uint32_t off = pf_chunk(row, c0 / 8 + c8, kPfRows);
-        *reinterpret_cast<uint4 *>(phi + off) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
-        *reinterpret_cast<uint4 *>(plo + off) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+      for (int e = 0; e < 8; ++e) {
+        const float a0 = ex2f(sv[2 * e] - ms);
+        const float a1 = ex2f(sv[2 * e + 1] - ms);
+        ls += a0 + a1;
+        split_p<kBF>(a0, a1, pw[e], pw[8 + e]);
       }
+      tmem_st16(trow + (j % kPfSBufs) * kPfKeys + c0, pw);
       l_run += ls;
       if (tail) {
         // V rows that hold no real position of this stage (past the keys the
@@ -423,9 +430,10 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
                 make_uint4(0u, 0u, 0u, 0u);
         }
       }
-      fence_proxy_async_smem();
+      if (tail) fence_proxy_async_smem();           // zeroed V rows -> tensor core
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&p_full[j & 1]);
+      mbar_arrive(&p_full[j % kPfSBufs]);
     }
     // ------------------------------------------------------------- output
     // row sums through the buffer the last stage's maxima did not use
@@ -458,14 +466,13 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == kPfMmaWarp) tmem_dealloc(tm, kPfTmemCols);
+  if (warp == kPfMmaWarp) tmem_dealloc(tm, kTmemCols);
 }
 
 template <int D, int BS, int KV_T>
 cudaError_t launch_prefill(const CUtensorMap &km, const CUtensorMap &vm, const PrefillParams &p,
                            int tiles, cudaStream_t st) {
-  constexpr int smem =
-      pf_stages(D) * 2 * kPfKeys * D * 2 + kPfRows * D * 2 + 4 * kPfRows * kPfKeys * 2 + 1024;
+  constexpr int smem = pf_stages(D) * 2 * kPfKeys * D * 2 + 1024;
   auto kern = attn_prefill_kernel<D, BS, KV_T>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
