@@ -2,6 +2,10 @@
 
     python -m paged_kv_cache_440_b200.build [--force] [--debug]
 
+Extra nvcc flags (for example tuning defines such as -DPAGEDKV_PF_GROUPS=2)
+come from the environment variable PAGEDKV_NVCC_FLAGS; pass --force after
+changing them.
+
 Each source under csrc/ is compiled by nvcc to an object in _build/ (rebuilt
 only when it or a header is newer), then linked with the static CUDA runtime
 into paged_kv_cache_440_b200/libpagedkv.so. No GPU is needed to build.
@@ -58,6 +62,7 @@ def _compile(src, obj, extra, verbose_log):
 def build(force=False, debug=False, jobs=None):
     os.makedirs(BUILD, exist_ok=True)
     extra = ["-DPAGEDKV_DEBUG=1"] if debug else []
+    extra += os.environ.get("PAGEDKV_NVCC_FLAGS", "").split()
     newest_header = max((os.path.getmtime(h) for h in _headers()), default=0)
     todo, objs = [], []
     for src in _sources():

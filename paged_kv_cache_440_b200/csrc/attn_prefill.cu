@@ -11,29 +11,34 @@
 // * One CTA per (tile of new tokens, KV head, sequence). The tile's 128 rows
 //   are (token, query head of the KV head's group) pairs, head fastest:
 //   128 / G tokens x G heads. Row r lives in TMEM lane r.
-// * The producer warp streams the KV head's cached blocks, 64 positions per
-//   stage (K then V, 128-byte swizzled TMA boxes of one block-head slab, one
-//   box per lane), into a ring of 6 (head_dim 128) or 8 (64) stages; block
-//   ids are read a 32-block window ahead.
+// * Two producer warps (K boxes, V boxes) stream the KV head's cached
+//   blocks, 64 positions per stage (128-byte swizzled TMA boxes of one
+//   block-head slab, one box per lane), into a ring of 6 (head_dim 128) or 8
+//   (64) stages; block ids are read a 32-block window ahead.
 // * The MMA warp (one thread) issues tcgen05 MMAs with the A operand in
 //   tensor memory and B in shared memory: S_j = Q K_j^T (M 128, N 64,
-//   K head_dim; Q in TMEM, K K-major from the TMA stage) into one of two TMEM
-//   score buffers, and O += P_j V_j (M 128, N head_dim, K 64; P in TMEM, V
-//   MN-major from the TMA stage) into a TMEM accumulator that stays resident
-//   for the whole key range. Order: S_0, S_1, then per stage j O += P_j V_j
-//   followed by S_{j+2}, so the tensor core computes the next scores while
-//   the softmax warps work on the current ones. Shared memory only carries
-//   K and V: its bandwidth, not the tensor core, is the tighter limit.
-// * 16 softmax warps: warp w reads TMEM lanes 32 (w mod 4) .. + 31 (the
-//   lanes a warp may access) and columns of group w / 4, so four threads share
-//   a row, 16 scores each per stage; the row maximum is combined through
-//   shared memory once per stage. Scale, causal and tail masks and the online
-//   softmax run in fp32 (base 2). The running maximum is only raised (and O,
-//   l rescaled in TMEM) when a new score exceeds it by more than 2^8;
+//   K head_dim; Q in TMEM, K K-major from the TMA stage) into one of three
+//   TMEM score buffers, and O += P_j V_j (M 128, N head_dim, K 64; P in
+//   TMEM, V MN-major from the TMA stage) into a TMEM accumulator that stays
+//   resident for the whole key range. Order: S_0, S_1, S_2, then per stage j
+//   O += P_j V_j followed by S_{j+3}, so the scores of the next stages are
+//   ready before the softmax warps ask for them. Measured on B200, an MMA of
+//   this size takes the tensor core 45-65 cycles but its issuing thread can
+//   spend more when it runs extra instructions between MMAs: the issue loop
+//   carries precomputed descriptors and compile-time accumulate flags only.
+// * 8 softmax warps (PAGEDKV_PF_GROUPS = 2 column groups; 4 gives 16 warps,
+//   measured slower): warp w reads TMEM lanes 32 (w mod 4) .. + 31 (the lanes
+//   a warp may access) and columns of group w / 4, so two threads share a
+//   row, 32 scores each per stage; the row maximum is combined through shared
+//   memory once per stage. Scale, causal and tail masks and the online
+//   softmax run in fp32 (base 2), two lanes per instruction where the
+//   hardware has packed fp32 arithmetic. The running maximum is only raised
+//   (and O, l rescaled in TMEM) when a new score exceeds it by more than 2^8;
 //   otherwise the stale maximum stays in use, which keeps every P value below
 //   256 and leaves the result unchanged up to rounding.
-// * P_j overwrites S_j in TMEM, each thread in its own 16 columns, as two
-//   16-bit parts hi + lo (8 columns of packed pairs each); O accumulates
+// * P_j overwrites S_j in TMEM, each thread in its own columns, as two
+//   16-bit parts hi + lo (per 16 scores: 8 columns of packed hi pairs, then
+//   8 of lo pairs, the layout of one K step of the MMA's A); O accumulates
 //   P_hi V + P_lo V, so rounding P to 16 bits costs nothing measurable (bf16:
 //   hi and lo by truncation, bit masks only; fp16: by rounding conversions).
 // * Synchronisation is by mbarriers: TMA -> MMA (full), MMA -> producer
@@ -54,7 +59,10 @@ namespace {
 using namespace dev;
 
 constexpr int kPfRows = 128;            // query rows per CTA (TMEM lanes)
-constexpr int kPfGroups = 4;            // softmax threads per row (column groups)
+#ifndef PAGEDKV_PF_GROUPS
+#define PAGEDKV_PF_GROUPS 2
+#endif
+constexpr int kPfGroups = PAGEDKV_PF_GROUPS;  // softmax threads per row (column groups): 2 or 4
 constexpr int kPfSoftmax = 128 * kPfGroups;
 constexpr int kPfProducerWarp = kPfSoftmax / 32;  // K boxes; the next warp: V boxes
 constexpr int kPfMmaWarp = kPfProducerWarp + 2;
@@ -104,22 +112,6 @@ __device__ __forceinline__ bool ring_wait_pf(uint64_t *bar, uint32_t parity, vol
   }
 }
 
-// Two P values -> 16-bit pairs hi + lo (low half = first value).
-template <bool BF16>
-__device__ __forceinline__ void split_p(float a, float b, uint32_t &hi, uint32_t &lo) {
-  if constexpr (BF16) {
-    // bf16 is the upper half of fp32: truncate for hi, the exact remainder
-    // truncated again for lo (hi + lo within 2^-14 relative of the value)
-    const uint32_t ua = __float_as_uint(a), ub = __float_as_uint(b);
-    const float ra = a - __uint_as_float(ua & 0xFFFF0000u);
-    const float rb = b - __uint_as_float(ub & 0xFFFF0000u);
-    hi = prmt(ua, ub, 0x7632);
-    lo = prmt(__float_as_uint(ra), __float_as_uint(rb), 0x7632);
-  } else {
-    split2<false>(a, b, hi, lo);
-  }
-}
-
 template <int D, int BS, int KV_T>
 __global__ void __launch_bounds__(kPfThreads, 1)
 attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
@@ -138,7 +130,9 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
   constexpr int kOCols = D / kPfGroups;              // O columns per thread
   constexpr unsigned kFull = 0xffffffffu;
   static_assert(kQCol + D / 2 <= kTmemCols, "TMEM budget");
-  static_assert(kSCols == 16 && (kOCols == 16 || kOCols == 32), "column split");
+  constexpr int kOChunk = kOCols < 32 ? kOCols : 32;  // O columns per TMEM access
+  constexpr int kQGCols = D / 2 / kPfGroups < 16 ? 16 : D / 2 / kPfGroups;  // Q columns per group
+  static_assert((kSCols == 16 || kSCols == 32) && kOCols % kOChunk == 0, "column split");
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[kStages];
@@ -203,21 +197,21 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
     rvalid = tl < p.tile_tokens && t0 + tl < cb;
     if (rvalid) rpos = L - cb + t0 + tl;
     rq = (static_cast<int64_t>(q0 + t0 + tl) * p.q_heads + g * p.group + hl) * D;
-    // Q row -> TMEM as packed 16-bit pairs (zeros past the tile): groups
-    // 0 .. D/32 - 1 each write 32 dims (16 columns)
-    if (cg < D / 32) {
+    // Q row -> TMEM as packed 16-bit pairs (zeros past the tile): the first
+    // D / 2 / kQGCols groups write kQGCols columns (2 kQGCols dims) each
+    if (cg < D / 2 / kQGCols) {
       const uint4 *src =
-          reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(p.q) + rq) + cg * 4;
-      uint32_t v[16];
+          reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(p.q) + rq) + cg * kQGCols / 4;
+      uint32_t v[kQGCols];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < kQGCols / 4; ++i) {
         const uint4 x = rvalid ? src[i] : make_uint4(0u, 0u, 0u, 0u);
         v[4 * i] = x.x;
         v[4 * i + 1] = x.y;
         v[4 * i + 2] = x.z;
         v[4 * i + 3] = x.w;
       }
-      tmem_st16(tm + (static_cast<uint32_t>((warp & 3) * 32) << 16) + kQCol + cg * 16, v);
+      tmem_st<kQGCols>(tm + (static_cast<uint32_t>((warp & 3) * 32) << 16) + kQCol + cg * kQGCols, v);
       tmem_wait_st();
     }
   }
@@ -300,16 +294,19 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
       const uint64_t kdesc0 = umma_desc_sw128(smem_u32(ring), 16, 1024);
       const uint64_t vdesc0 = umma_desc_sw128(smem_u32(ring) + kPartBytes, kPfKeys * 128, 1024);
       bool ok = true;
+      // Between two MMAs this thread runs only immediate adds: the issuing
+      // thread, not the tensor core, limits small MMAs.
       auto issue_s = [&](int j) {
         const int s = j % kStages;
         if (!ring_wait_pf(&full_bar[s], (j / kStages) & 1, &s_abort, p.status)) return false;
         tc_fence_after();
+        const uint64_t kd = kdesc0 + static_cast<uint64_t>(s * (kStageBytes >> 4));
+        const uint32_t sd = tm + (j % kPfSBufs) * kPfKeys;
+        umma_f16_tmem_a_c<false>(sd, tm + kQCol, kd, idesc_s);
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t off = s * kStageBytes + (ks >> 2) * kPfKeys * 128 + (ks & 3) * 32;
-          umma_f16_tmem_a(tm + (j % kPfSBufs) * kPfKeys, tm + kQCol + ks * 8, kdesc0 + (off >> 4),
-                          idesc_s, ks > 0);
-        }
+        for (int ks = 1; ks < D / 16; ++ks)
+          umma_f16_tmem_a_c<true>(sd, tm + kQCol + ks * 8,
+                                  kd + (((ks >> 2) * kPfKeys * 128 + (ks & 3) * 32) >> 4), idesc_s);
         umma_commit(&s_full[j % kPfSBufs]);
         return true;
       };
@@ -318,12 +315,15 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
         if (!ring_wait_pf(&p_full[j % kPfSBufs], (j / kPfSBufs) & 1, &s_abort, p.status)) break;
         tc_fence_after();
         const uint32_t pcol = tm + (j % kPfSBufs) * kPfKeys;
+        const uint64_t vd = vdesc0 + static_cast<uint64_t>((j % kStages) * (kStageBytes >> 4));
+        // P_hi V over the stage's 4 K steps, then P_lo V (the first MMA of
+        // the first stage starts the accumulator)
+        umma_f16_tmem_a(tm + kOCol, pcol, vd, idesc_o, j > 0);
 #pragma unroll
-        for (int ks = 0; ks < 2 * kPfKeys / 16; ++ks) {  // P_hi V, then P_lo V
+        for (int ks = 1; ks < 2 * kPfKeys / 16; ++ks) {
           const int kk = ks & (kPfKeys / 16 - 1);
-          const uint32_t off = (j % kStages) * kStageBytes + kk * 16 * 128;
-          umma_f16_tmem_a(tm + kOCol, pcol + kk * 16 + (ks >= kPfKeys / 16 ? 8 : 0),
-                          vdesc0 + (off >> 4), idesc_o, j > 0 || ks > 0);
+          umma_f16_tmem_a_c<true>(tm + kOCol, pcol + kk * 16 + (ks >= kPfKeys / 16 ? 8 : 0),
+                                  vd + ((kk * 16 * 128) >> 4), idesc_o);
         }
         umma_commit(&empty_bar[j % kStages]);
         umma_commit(&o_done[j & 1]);
@@ -342,6 +342,7 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
     // waiting at a barrier.
     const uint32_t trow = tm + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const int c0 = cg * kSCols;                      // first score column
+    const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
     float m_used = -INFINITY, l_run = 0.f;
     for (int j = 0; j < nstages; ++j) {
       const int s = j % kStages;
@@ -356,25 +357,27 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
         tmem_ld<kSCols>(trow + (j % kPfSBufs) * kPfKeys + c0, r);
         tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < kSCols; ++c) sv[c] = __uint_as_float(r[c]) * p.scale_log2;
+        for (int c = 0; c < kSCols; c += 2) {
+          const float2 v = mul2(make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), sc2);
+          sv[c] = v.x;
+          sv[c + 1] = v.y;
+        }
       }
       const int key0 = j * kPfKeys;
       const uint32_t bmask = stage_mask[s];
       const bool tail = key0 + kPfKeys > nkeys || bmask != kAllBlocks;
       const bool need_mask = tail || key0 + c0 + kSCols - 1 > rpos;
-      float mx = -INFINITY;
       if (need_mask) {
 #pragma unroll
         for (int c = 0; c < kSCols; ++c) {
           const int kp = key0 + c0 + c;
           const bool ok = kp <= rpos && kp < nkeys && ((bmask >> ((c0 + c) / BS)) & 1u);
           sv[c] = ok ? sv[c] : -INFINITY;
-          mx = fmaxf(mx, sv[c]);
         }
-      } else {
-#pragma unroll
-        for (int c = 0; c < kSCols; ++c) mx = fmaxf(mx, sv[c]);
       }
+      float mx = fmaxf(sv[0], sv[1]);
+#pragma unroll
+      for (int c = 2; c < kSCols; c += 2) mx = fmax3(mx, sv[c], sv[c + 1]);
       red[j & 1][cg][row] = mx;
       bar_sync(1, kPfSoftmax);
 #pragma unroll
@@ -394,26 +397,42 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
         // thread's columns of its row
         ring_wait_pf(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, &s_abort, p.status);
         tc_fence_after();
-        uint32_t o[kOCols];
-        tmem_ld<kOCols>(trow + kOCol + cg * kOCols, o);
-        tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < kOCols; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-        tmem_st<kOCols>(trow + kOCol + cg * kOCols, o);
+        for (int oc = 0; oc < kOCols; oc += kOChunk) {
+          uint32_t o[kOChunk];
+          tmem_ld<kOChunk>(trow + kOCol + cg * kOCols + oc, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < kOChunk; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+          tmem_st<kOChunk>(trow + kOCol + cg * kOCols + oc, o);
+        }
         tmem_wait_st();
       }
       const float ms = m_used == -INFINITY ? 0.f : m_used;
-      float ls = 0.f;
-      uint32_t pw[16];                               // 8 hi pairs, then 8 lo pairs
+      const float2 nm = make_float2(-ms, -ms);
+      float2 ls = make_float2(0.f, 0.f);
+      // per 16 scores (one K step of P V): 8 hi pairs, then 8 lo pairs
+      uint32_t pw[kSCols];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float a0 = ex2f(sv[2 * e] - ms);
-        const float a1 = ex2f(sv[2 * e + 1] - ms);
-        ls += a0 + a1;
-        split_p<kBF>(a0, a1, pw[e], pw[8 + e]);
+      for (int e = 0; e < kSCols / 2; ++e) {
+        const float2 d = add2(make_float2(sv[2 * e], sv[2 * e + 1]), nm);
+        const float2 a = make_float2(ex2f(d.x), ex2f(d.y));
+        ls = add2(ls, a);
+        const int w = (e / 8) * 16 + (e % 8);
+        if constexpr (kBF) {
+          // bf16 is the upper half of fp32: truncate for hi, the exact
+          // remainder truncated again for lo (hi + lo within 2^-14 relative)
+          const uint32_t ua = __float_as_uint(a.x), ub = __float_as_uint(a.y);
+          const float2 r = sub2(a, make_float2(__uint_as_float(ua & 0xFFFF0000u),
+                                               __uint_as_float(ub & 0xFFFF0000u)));
+          pw[w] = prmt(ua, ub, 0x7632);
+          pw[w + 8] = prmt(__float_as_uint(r.x), __float_as_uint(r.y), 0x7632);
+        } else {
+          split2<false>(a.x, a.y, pw[w], pw[w + 8]);
+        }
       }
-      tmem_st16(trow + (j % kPfSBufs) * kPfKeys + c0, pw);
-      l_run += ls;
+      tmem_st<kSCols>(trow + (j % kPfSBufs) * kPfKeys + c0, pw);
+      l_run += ls.x + ls.y;
       if (tail) {
         // V rows that hold no real position of this stage (past the keys the
         // tile reads, or of a block that was not loaded) may hold anything:
@@ -446,19 +465,23 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
     if (!__any_sync(kFull, s_abort != 0)) {  // warp-uniform: TMEM loads are warp-wide
       tc_fence_after();
       const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
-      uint32_t o[kOCols];
-      tmem_ld<kOCols>(trow + kOCol + cg * kOCols, o);
-      tmem_wait_ld();
-      if (rvalid) {
-        uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + rq + cg * kOCols);
 #pragma unroll
-        for (int c4 = 0; c4 < kOCols / 8; ++c4) {
-          uint32_t w[4];
+      for (int oc = 0; oc < kOCols; oc += kOChunk) {
+        uint32_t o[kOChunk];
+        tmem_ld<kOChunk>(trow + kOCol + cg * kOCols + oc, o);
+        tmem_wait_ld();
+        if (rvalid) {
+          uint4 *dst =
+              reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + rq + cg * kOCols + oc);
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            w[e] = pack2<kBF>(__uint_as_float(o[c4 * 8 + 2 * e]) * inv,
-                              __uint_as_float(o[c4 * 8 + 2 * e + 1]) * inv);
-          dst[c4] = make_uint4(w[0], w[1], w[2], w[3]);
+          for (int c4 = 0; c4 < kOChunk / 8; ++c4) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              w[e] = pack2<kBF>(__uint_as_float(o[c4 * 8 + 2 * e]) * inv,
+                                __uint_as_float(o[c4 * 8 + 2 * e + 1]) * inv);
+            dst[c4] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
         }
       }
     }

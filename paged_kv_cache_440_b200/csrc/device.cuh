@@ -364,6 +364,30 @@ __device__ __forceinline__ void store_codes(uint8_t *dst, int lane, uint32_t pac
   }
 }
 
+// ------------------------------------------------------------ packed fp32
+// Two fp32 lanes per instruction (sm_100 f32x2 arithmetic), round to nearest.
+
+#define PAGEDKV_F32X2(NAME, OP)                                                          \
+  __device__ __forceinline__ float2 NAME(float2 a, float2 b) {                            \
+    float2 r;                                                                             \
+    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t" OP \
+        " d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"                                          \
+        : "=f"(r.x), "=f"(r.y)                                                            \
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));                                        \
+    return r;                                                                             \
+  }
+PAGEDKV_F32X2(mul2, "mul.rn.f32x2")
+PAGEDKV_F32X2(add2, "add.rn.f32x2")
+PAGEDKV_F32X2(sub2, "sub.rn.f32x2")
+#undef PAGEDKV_F32X2
+
+// max(a, b, c) in one instruction.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // ------------------------------------------------------------------ tcgen05
 // Fifth-generation tensor core: MMAs issued by one thread read both operands
 // from shared memory through 64-bit matrix descriptors and accumulate in
@@ -409,6 +433,25 @@ __device__ __forceinline__ void umma_f16_tmem_a(uint32_t tmem_d, uint32_t tmem_a
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
       "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate ? 1u : 0u)
       : "memory");
+}
+
+// As umma_f16_tmem_a with a compile-time accumulate flag (no predicate setup).
+template <bool ACC>
+__device__ __forceinline__ void umma_f16_tmem_a_c(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc,
+                                                  uint32_t idesc) {
+  if constexpr (ACC) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.eq.u32 p, 0, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(bdesc), "r"(idesc)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.u32 p, 0, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(bdesc), "r"(idesc)
+        : "memory");
+  }
 }
 
 // Arrive on `bar` once every tcgen05 operation this thread issued so far is done.
