@@ -67,11 +67,12 @@ constexpr int kPfSoftmax = 128 * kPfGroups;
 constexpr int kPfProducerWarp = kPfSoftmax / 32;  // K boxes; the next warp: V boxes
 constexpr int kPfMmaWarp = kPfProducerWarp + 2;
 constexpr int kPfThreads = kPfSoftmax + 96;
-constexpr int kPfKeys = 64;             // positions per stage
+constexpr int kPfKeys = 64;             // positions per stage (TMA ring granularity)
+constexpr int kPfUnit = 128;            // positions per score tile (two stages)
 // Ring depth: 6 stages of 32 KB for head_dim 128, 8 of 16 KB for 64.
 __host__ __device__ constexpr int pf_stages(int D) { return D == 128 ? 6 : 8; }
-constexpr int kPfSBufs = 3;             // S/P buffers in TMEM
-// TMEM columns: S/P 3 x 64, O head_dim, Q head_dim / 2 (packed pairs)
+constexpr int kPfSBufs = 2;             // S/P buffers in TMEM, 128 columns each
+// TMEM columns: S/P 2 x 128, O head_dim, Q head_dim / 2 (packed pairs)
 constexpr uint32_t kPfTmemCols = 512;
 constexpr float kPfRescaleLog2 = 8.f;   // raise the running max only beyond 2^8
 
@@ -112,7 +113,10 @@ __device__ __forceinline__ bool ring_wait_pf(uint64_t *bar, uint32_t parity, vol
   }
 }
 
-template <int D, int BS, int KV_T>
+// VBLK: V comes one box per block (both 128-byte slabs, the 3-D map), landing
+// per stage as [block][slab][row][128 B]; otherwise one box per block and
+// slab, landing as [slab][key][128 B].
+template <int D, int BS, int KV_T, bool VBLK>
 __global__ void __launch_bounds__(kPfThreads, 1)
 attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
                     const __grid_constant__ CUtensorMap vmap, const PrefillParams p) {
@@ -120,33 +124,46 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
   constexpr int kStages = pf_stages(D);
   constexpr int kSlabs = D / 64;                     // 128-byte slabs per row
   constexpr int kPartBytes = kPfKeys * D * 2;        // K (or V) of one stage
-  constexpr int kStageBytes = 2 * kPartBytes;
+  constexpr int kKSlabBytes = kStages * kPfKeys * 128;  // one slab of the K ring
   constexpr int kBlocksPerStage = kPfKeys / BS;
-  constexpr uint32_t kAllBlocks = (1u << kBlocksPerStage) - 1u;
-  constexpr uint32_t kOCol = kPfSBufs * kPfKeys;     // first TMEM column of O
+  constexpr uint32_t kAllBlocks = (1u << (2 * kBlocksPerStage)) - 1u;  // of a full unit
+  constexpr uint32_t kOCol = kPfSBufs * kPfUnit;     // first TMEM column of O
   constexpr uint32_t kQCol = kOCol + D;              // first TMEM column of Q
   constexpr uint32_t kTmemCols = kPfTmemCols;
-  constexpr int kSCols = kPfKeys / kPfGroups;        // scores per thread per stage
+  constexpr int kSCols = kPfUnit / kPfGroups;        // scores per thread per unit
+  constexpr int kSChunk = 32;                        // scores per TMEM access
   constexpr int kOCols = D / kPfGroups;              // O columns per thread
-  constexpr unsigned kFull = 0xffffffffu;
-  static_assert(kQCol + D / 2 <= kTmemCols, "TMEM budget");
   constexpr int kOChunk = kOCols < 32 ? kOCols : 32;  // O columns per TMEM access
   constexpr int kQGCols = D / 2 / kPfGroups < 16 ? 16 : D / 2 / kPfGroups;  // Q columns per group
-  static_assert((kSCols == 16 || kSCols == 32) && kOCols % kOChunk == 0, "column split");
+  constexpr unsigned kFull = 0xffffffffu;
+  static_assert(kQCol + D / 2 <= kTmemCols, "TMEM budget");
+  static_assert(kSCols % kSChunk == 0 && kOCols % kOChunk == 0, "column split");
+  static_assert(kStages % 2 == 0, "a unit's two stages are adjacent ring slots");
+  static_assert(!VBLK || kSlabs == 2, "block boxes carry two slabs");
+  // V of one stage: byte offset of (key, 16-byte chunk c) and the slab stride
+  auto v_off = [](int key, int c) {
+    if constexpr (VBLK)
+      return (key / BS) * BS * 256 + (c >> 3) * BS * 128 + (key % BS) * 128 + (c & 7) * 16;
+    else
+      return (c >> 3) * kPfKeys * 128 + key * 128 + (c & 7) * 16;
+  };
+  constexpr uint32_t kVSlabStride = VBLK ? BS * 128 : kPfKeys * 128;
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[kStages];
   __shared__ __align__(8) uint64_t empty_bar[kStages];
   __shared__ __align__(8) uint64_t s_full[kPfSBufs];
   __shared__ __align__(8) uint64_t p_full[kPfSBufs];
-  __shared__ __align__(8) uint64_t o_done[2];
   __shared__ __align__(8) uint64_t mma_idle;
-  __shared__ uint32_t stage_mask[kStages];         // valid blocks of the stage
+  __shared__ uint32_t stage_mask[kStages];           // valid blocks of the stage
   __shared__ float red[2][kPfGroups][kPfRows];       // row maxima, then row sums
   __shared__ uint32_t tmem_slot;
   __shared__ int s_abort;
-  uint8_t *ring = reinterpret_cast<uint8_t *>(
+  // K ring: [slab][slot * 64 + key][128 B], so that the two stages of a unit
+  // (slots 2i, 2i + 1) form one 128-row operand; V ring: [slot][slab][key][128 B]
+  uint8_t *ring_k = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *ring_v = ring_k + kStages * kPartBytes;
 
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -165,6 +182,7 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
   const int t_last = min(t0 + p.tile_tokens, cb) - 1;  // last token of the tile
   const int nkeys = L - cb + t_last + 1;               // positions the tile reads
   const int nstages = (nkeys + kPfKeys - 1) / kPfKeys;
+  const int nunits = (nstages + 1) / 2;
 
   if (threadIdx.x == 0) {
     s_abort = 0;
@@ -176,7 +194,6 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], kPfSoftmax);
     }
-    for (int i = 0; i < 2; ++i) mbar_init(&o_done[i], 1);
     mbar_init(&mma_idle, 1);
     fence_barrier_init();
   }
@@ -246,8 +263,9 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
     int cur = load_ids(0), nxt = load_ids(1);
     uint32_t cur_ok = __ballot_sync(kFull, cur >= 0);
     int issued = 0;
-    constexpr int kBoxes = kBlocksPerStage * kSlabs;  // this warp's TMA boxes of a full stage
-    static_assert(kBoxes <= 32, "one box per lane");
+    // this warp's TMA boxes of a full stage
+    const int kBoxes = (kv && VBLK) ? kBlocksPerStage : kBlocksPerStage * kSlabs;
+    static_assert(kBlocksPerStage * kSlabs <= 32, "one box per lane");
     for (int st = 0; st < nstages; ++st) {
       const int s = st % kStages;
       const int jb0 = st * kBlocksPerStage;        // first block of the stage
@@ -268,11 +286,19 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
         mbar_arrive_expect_tx(&full_bar[s], __popc(valid) * 2 * BS * D * 2);
       }
       // lane -> (block j, slab)
-      const int j = lane / kSlabs, sl = lane % kSlabs;
+      const int per = (kv && VBLK) ? 1 : kSlabs;
+      const int j = lane / per, sl = lane % per;
       const int bid = __shfl_sync(kFull, cur, (jb0 & 31) + (j < kBlocksPerStage ? j : 0));
       if (lane < kBoxes && j < nblk && ((valid >> j) & 1u)) {
-        uint8_t *dst = ring + s * kStageBytes + kv * kPartBytes + (sl * kPfKeys + j * BS) * 128;
-        tma_load_2d(dst, kv ? &vmap : &kmap, &full_bar[s], sl * 64, (bid * p.kv_heads + g) * BS);
+        const int y = (bid * p.kv_heads + g) * BS;
+        if (kv == 0)
+          tma_load_2d(ring_k + sl * kKSlabBytes + (s * kPfKeys + j * BS) * 128, &kmap, &full_bar[s],
+                      sl * 64, y);
+        else if (VBLK)
+          tma_load_3d(ring_v + s * kPartBytes + j * BS * 256, &vmap, &full_bar[s], 0, y, 0);
+        else
+          tma_load_2d(ring_v + s * kPartBytes + (sl * kPfKeys + j * BS) * 128, &vmap, &full_bar[s],
+                      sl * 64, y);
       }
       __syncwarp();
       ++issued;
@@ -286,49 +312,64 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
   } else if (warp == kPfMmaWarp) {
     // ============================================================ MMA issue
     if (lane == 0) {
-      const uint32_t idesc_s = umma_idesc_f16<kBF>(kPfRows, kPfKeys, false);
+      const uint32_t idesc_s = umma_idesc_f16<kBF>(kPfRows, kPfUnit, false);
       const uint32_t idesc_o = umma_idesc_f16<kBF>(kPfRows, D, true);
-      // descriptors of stage 0; other stages and K steps add their byte
-      // offset / 16 to the start-address field (no carry: shared addresses
-      // stay below 256 KB)
-      const uint64_t kdesc0 = umma_desc_sw128(smem_u32(ring), 16, 1024);
-      const uint64_t vdesc0 = umma_desc_sw128(smem_u32(ring) + kPartBytes, kPfKeys * 128, 1024);
+      // descriptors of slot 0; other slots and K steps add their byte offset
+      // / 16 to the start-address field (no carry: shared addresses stay below
+      // 256 KB)
+      const uint64_t kdesc0 = umma_desc_sw128(smem_u32(ring_k), 16, 1024);
+      const uint64_t vdesc0 = umma_desc_sw128(smem_u32(ring_v), kVSlabStride, 1024);
       bool ok = true;
       // Between two MMAs this thread runs only immediate adds: the issuing
       // thread, not the tensor core, limits small MMAs.
-      auto issue_s = [&](int j) {
-        const int s = j % kStages;
-        if (!ring_wait_pf(&full_bar[s], (j / kStages) & 1, &s_abort, p.status)) return false;
+      auto issue_s = [&](int u) {
+        const int a = 2 * u;
+        if (!ring_wait_pf(&full_bar[a % kStages], (a / kStages) & 1, &s_abort, p.status))
+          return false;
+        if (a + 1 < nstages &&
+            !ring_wait_pf(&full_bar[(a + 1) % kStages], ((a + 1) / kStages) & 1, &s_abort, p.status))
+          return false;
         tc_fence_after();
-        const uint64_t kd = kdesc0 + static_cast<uint64_t>(s * (kStageBytes >> 4));
-        const uint32_t sd = tm + (j % kPfSBufs) * kPfKeys;
+        // a unit's 128 keys: rows of slots a mod kStages and the next one
+        const uint64_t kd = kdesc0 + static_cast<uint64_t>(((a % kStages) * kPfKeys * 128) >> 4);
+        const uint32_t sd = tm + (u & 1) * kPfUnit;
         umma_f16_tmem_a_c<false>(sd, tm + kQCol, kd, idesc_s);
 #pragma unroll
         for (int ks = 1; ks < D / 16; ++ks)
           umma_f16_tmem_a_c<true>(sd, tm + kQCol + ks * 8,
-                                  kd + (((ks >> 2) * kPfKeys * 128 + (ks & 3) * 32) >> 4), idesc_s);
-        umma_commit(&s_full[j % kPfSBufs]);
+                                  kd + (((ks >> 2) * kKSlabBytes + (ks & 3) * 32) >> 4), idesc_s);
+        umma_commit(&s_full[u & 1]);
         return true;
       };
-      for (int j = 0; ok && j < min(nstages, kPfSBufs); ++j) ok = issue_s(j);
-      for (int j = 0; ok && j < nstages; ++j) {
-        if (!ring_wait_pf(&p_full[j % kPfSBufs], (j / kPfSBufs) & 1, &s_abort, p.status)) break;
+      for (int u = 0; ok && u < min(nunits, kPfSBufs); ++u) ok = issue_s(u);
+      for (int u = 0; ok && u < nunits; ++u) {
+        if (!ring_wait_pf(&p_full[u & 1], (u >> 1) & 1, &s_abort, p.status)) break;
         tc_fence_after();
-        const uint32_t pcol = tm + (j % kPfSBufs) * kPfKeys;
-        const uint64_t vd = vdesc0 + static_cast<uint64_t>((j % kStages) * (kStageBytes >> 4));
-        // P_hi V over the stage's 4 K steps, then P_lo V (the first MMA of
-        // the first stage starts the accumulator)
-        umma_f16_tmem_a(tm + kOCol, pcol, vd, idesc_o, j > 0);
+        const uint32_t pcol = tm + (u & 1) * kPfUnit;
+        const int a = 2 * u, nh = a + 1 < nstages ? 2 : 1;
+        // per stage of the unit: P_hi V over its 4 K steps, then P_lo V (the
+        // first MMA of the first unit starts the accumulator)
 #pragma unroll
-        for (int ks = 1; ks < 2 * kPfKeys / 16; ++ks) {
-          const int kk = ks & (kPfKeys / 16 - 1);
-          umma_f16_tmem_a_c<true>(tm + kOCol, pcol + kk * 16 + (ks >= kPfKeys / 16 ? 8 : 0),
-                                  vd + ((kk * 16 * 128) >> 4), idesc_o);
+        for (int h = 0; h < 2; ++h) {
+          if (h < nh) {
+            const uint64_t vd =
+                vdesc0 + static_cast<uint64_t>((((a + h) % kStages) * kPartBytes) >> 4);
+            const uint32_t ph = pcol + h * 64;
+            if (h == 0) umma_f16_tmem_a(tm + kOCol, ph, vd, idesc_o, u > 0);
+            else umma_f16_tmem_a_c<true>(tm + kOCol, ph, vd, idesc_o);
+#pragma unroll
+            for (int ks = 1; ks < 2 * kPfKeys / 16; ++ks) {
+              const int kk = ks & (kPfKeys / 16 - 1);
+              umma_f16_tmem_a_c<true>(tm + kOCol, ph + kk * 16 + (ks >= kPfKeys / 16 ? 8 : 0),
+                                      vd + (v_off(kk * 16, 0) >> 4), idesc_o);
+            }
+          }
         }
-        umma_commit(&empty_bar[j % kStages]);
-        umma_commit(&o_done[j & 1]);
-        // S_{j+3} reuses S_j's columns: issued after P_j V_j, which reads them
-        if (j + kPfSBufs < nstages) ok = issue_s(j + kPfSBufs);
+        // a unit's stages are free (and O holds P_0..P_u V) once these finish
+        umma_commit(&empty_bar[a % kStages]);
+        if (nh == 2) umma_commit(&empty_bar[(a + 1) % kStages]);
+        // S_{u+2} reuses S_u's columns: issued after P_u V, which reads them
+        if (u + kPfSBufs < nunits) ok = issue_s(u + kPfSBufs);
       }
       // every MMA issued has finished before TMEM can be released
       umma_commit(&mma_idle);
@@ -337,51 +378,62 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
     __syncwarp();
   } else {
     // ============================================================ softmax
-    // Every softmax thread runs every stage and every named barrier, also
+    // Every softmax thread runs every unit and every named barrier, also
     // after a timeout (the waits then return at once), so none is left
     // waiting at a barrier.
     const uint32_t trow = tm + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const int c0 = cg * kSCols;                      // first score column
     const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
     float m_used = -INFINITY, l_run = 0.f;
-    for (int j = 0; j < nstages; ++j) {
-      const int s = j % kStages;
-      ring_wait_pf(&s_full[j % kPfSBufs], (j / kPfSBufs) & 1, &s_abort, p.status);
-      // the stage's TMA has landed (its full phase cannot advance before
-      // P_j V_j is done): gives this thread the block mask and the V bytes
-      ring_wait_pf(&full_bar[s], (j / kStages) & 1, &s_abort, p.status);
+    for (int u = 0; u < nunits; ++u) {
+      const int a = 2 * u;
+      const bool two = a + 1 < nstages;
+      ring_wait_pf(&s_full[u & 1], (u >> 1) & 1, &s_abort, p.status);
+      // the stages' TMA has landed (their full phases cannot advance before
+      // P_u V is done): gives this thread the block masks and the V bytes
+      ring_wait_pf(&full_bar[a % kStages], (a / kStages) & 1, &s_abort, p.status);
+      if (two) ring_wait_pf(&full_bar[(a + 1) % kStages], ((a + 1) / kStages) & 1, &s_abort, p.status);
       tc_fence_after();
-      float sv[kSCols];
-      {
-        uint32_t r[kSCols];
-        tmem_ld<kSCols>(trow + (j % kPfSBufs) * kPfKeys + c0, r);
+      const int key0 = u * kPfUnit;
+      const uint32_t bmask =
+          stage_mask[a % kStages] | (two ? stage_mask[(a + 1) % kStages] << kBlocksPerStage : 0u);
+      const bool tail = key0 + kPfUnit > nkeys || bmask != kAllBlocks;
+      const bool need_mask = tail || key0 + c0 + kSCols - 1 > rpos;
+      const uint32_t sbuf = trow + (u & 1) * kPfUnit + c0;
+      // scores of chunk ch (scaled to base 2, masked)
+      auto scores = [&](int ch, float (&sv)[kSChunk]) {
+        uint32_t r[kSChunk];
+        tmem_ld<kSChunk>(sbuf + ch * kSChunk, r);
         tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < kSCols; c += 2) {
+        for (int c = 0; c < kSChunk; c += 2) {
           const float2 v = mul2(make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), sc2);
           sv[c] = v.x;
           sv[c + 1] = v.y;
         }
-      }
-      const int key0 = j * kPfKeys;
-      const uint32_t bmask = stage_mask[s];
-      const bool tail = key0 + kPfKeys > nkeys || bmask != kAllBlocks;
-      const bool need_mask = tail || key0 + c0 + kSCols - 1 > rpos;
-      if (need_mask) {
+        if (need_mask) {
 #pragma unroll
-        for (int c = 0; c < kSCols; ++c) {
-          const int kp = key0 + c0 + c;
-          const bool ok = kp <= rpos && kp < nkeys && ((bmask >> ((c0 + c) / BS)) & 1u);
-          sv[c] = ok ? sv[c] : -INFINITY;
+          for (int c = 0; c < kSChunk; ++c) {
+            const int cu = c0 + ch * kSChunk + c;       // column in the unit
+            const int kp = key0 + cu;
+            const bool okk = kp <= rpos && kp < nkeys && ((bmask >> (cu / BS)) & 1u);
+            sv[c] = okk ? sv[c] : -INFINITY;
+          }
         }
-      }
-      float mx = fmaxf(sv[0], sv[1]);
+      };
+      // pass 1: the row maximum over this thread's columns, then the row's
+      float mx = -INFINITY;
 #pragma unroll
-      for (int c = 2; c < kSCols; c += 2) mx = fmax3(mx, sv[c], sv[c + 1]);
-      red[j & 1][cg][row] = mx;
+      for (int ch = 0; ch < kSCols / kSChunk; ++ch) {
+        float sv[kSChunk];
+        scores(ch, sv);
+#pragma unroll
+        for (int c = 0; c < kSChunk; c += 2) mx = fmax3(mx, sv[c], sv[c + 1]);
+      }
+      red[u & 1][cg][row] = mx;
       bar_sync(1, kPfSoftmax);
 #pragma unroll
-      for (int q = 0; q < kPfGroups; ++q) mx = fmaxf(mx, red[j & 1][q][row]);
+      for (int q = 0; q < kPfGroups; ++q) mx = fmaxf(mx, red[u & 1][q][row]);
       // lazy maximum: raise it only when a score exceeds it by more than 2^8
       // (every thread of the row takes the same decision)
       float alpha = 1.f;
@@ -393,9 +445,10 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
         l_run *= alpha;
       }
       if (__any_sync(kFull, alpha != 1.f)) {
-        // O holds P_0..P_{j-1} V: wait for the last of them, rescale this
-        // thread's columns of its row
-        ring_wait_pf(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, &s_abort, p.status);
+        // O holds P_0..P_{u-1} V: wait for the last of them (the commit that
+        // freed unit u-1's first stage), rescale this thread's columns of O
+        const int pa = 2 * (u - 1);
+        ring_wait_pf(&empty_bar[pa % kStages], (pa / kStages) & 1, &s_abort, p.status);
         tc_fence_after();
 #pragma unroll
         for (int oc = 0; oc < kOCols; oc += kOChunk) {
@@ -408,60 +461,67 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
         }
         tmem_wait_st();
       }
+      // pass 2: P = 2^(s - m) over the same columns, written over S as
+      // hi + lo parts (per 16 scores: 8 hi pairs, then 8 lo pairs)
       const float ms = m_used == -INFINITY ? 0.f : m_used;
       const float2 nm = make_float2(-ms, -ms);
       float2 ls = make_float2(0.f, 0.f);
-      // per 16 scores (one K step of P V): 8 hi pairs, then 8 lo pairs
-      uint32_t pw[kSCols];
 #pragma unroll
-      for (int e = 0; e < kSCols / 2; ++e) {
-        const float2 d = add2(make_float2(sv[2 * e], sv[2 * e + 1]), nm);
-        const float2 a = make_float2(ex2f(d.x), ex2f(d.y));
-        ls = add2(ls, a);
-        const int w = (e / 8) * 16 + (e % 8);
-        if constexpr (kBF) {
-          // bf16 is the upper half of fp32: truncate for hi, the exact
-          // remainder truncated again for lo (hi + lo within 2^-14 relative)
-          const uint32_t ua = __float_as_uint(a.x), ub = __float_as_uint(a.y);
-          const float2 r = sub2(a, make_float2(__uint_as_float(ua & 0xFFFF0000u),
-                                               __uint_as_float(ub & 0xFFFF0000u)));
-          pw[w] = prmt(ua, ub, 0x7632);
-          pw[w + 8] = prmt(__float_as_uint(r.x), __float_as_uint(r.y), 0x7632);
-        } else {
-          split2<false>(a.x, a.y, pw[w], pw[w + 8]);
+      for (int ch = 0; ch < kSCols / kSChunk; ++ch) {
+        float sv[kSChunk];
+        scores(ch, sv);
+        uint32_t pw[kSChunk];
+#pragma unroll
+        for (int e = 0; e < kSChunk / 2; ++e) {
+          const float2 d = add2(make_float2(sv[2 * e], sv[2 * e + 1]), nm);
+          const float2 pa2 = make_float2(ex2f(d.x), ex2f(d.y));
+          ls = add2(ls, pa2);
+          const int w = (e / 8) * 16 + (e % 8);
+          if constexpr (kBF) {
+            // bf16 is the upper half of fp32: truncate for hi, the exact
+            // remainder truncated again for lo (hi + lo within 2^-14 relative)
+            const uint32_t ua = __float_as_uint(pa2.x), ub = __float_as_uint(pa2.y);
+            const float2 r = sub2(pa2, make_float2(__uint_as_float(ua & 0xFFFF0000u),
+                                                   __uint_as_float(ub & 0xFFFF0000u)));
+            pw[w] = prmt(ua, ub, 0x7632);
+            pw[w + 8] = prmt(__float_as_uint(r.x), __float_as_uint(r.y), 0x7632);
+          } else {
+            split2<false>(pa2.x, pa2.y, pw[w], pw[w + 8]);
+          }
         }
+        tmem_st<kSChunk>(sbuf + ch * kSChunk, pw);
       }
-      tmem_st<kSCols>(trow + (j % kPfSBufs) * kPfKeys + c0, pw);
       l_run += ls.x + ls.y;
       if (tail) {
-        // V rows that hold no real position of this stage (past the keys the
+        // V rows that hold no real position of this unit (past the keys the
         // tile reads, or of a block that was not loaded) may hold anything:
         // zero them so that P = 0 there cannot meet a NaN.
-        uint8_t *vpart = ring + s * kStageBytes + kPartBytes;
-        constexpr int kChunks = kPfKeys * D / 8;     // 16-byte chunks of V
+        constexpr int kChunks = kPfUnit * D / 8;     // 16-byte chunks of the unit's V
 #pragma unroll
         for (int i = 0; i < kChunks / kPfSoftmax; ++i) {
           const int idx = threadIdx.x + i * kPfSoftmax;
-          const int kr = idx / (D / 8), c = idx % (D / 8);
+          const int kr = idx / (D / 8), c = idx % (D / 8);  // row of the unit, chunk
+          const int h = kr / kPfKeys, kh = kr % kPfKeys;
           const bool real = key0 + kr < nkeys && ((bmask >> (kr / BS)) & 1u);
-          if (!real)
-            *reinterpret_cast<uint4 *>(vpart + (c >> 3) * kPfKeys * 128 + kr * 128 + (c & 7) * 16) =
+          if (!real && (h == 0 || two))
+            *reinterpret_cast<uint4 *>(ring_v + ((a + h) % kStages) * kPartBytes + v_off(kh, c)) =
                 make_uint4(0u, 0u, 0u, 0u);
         }
+        fence_proxy_async_smem();                    // zeroed V rows -> tensor core
       }
-      if (tail) fence_proxy_async_smem();           // zeroed V rows -> tensor core
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&p_full[j % kPfSBufs]);
+      mbar_arrive(&p_full[u & 1]);
     }
     // ------------------------------------------------------------- output
-    // row sums through the buffer the last stage's maxima did not use
-    red[nstages & 1][cg][row] = l_run;
-    ring_wait_pf(&o_done[(nstages - 1) & 1], ((nstages - 1) >> 1) & 1, &s_abort, p.status);
+    // row sums through the buffer the last unit's maxima did not use
+    red[nunits & 1][cg][row] = l_run;
+    const int la = 2 * (nunits - 1);                  // P_last V done frees this stage
+    ring_wait_pf(&empty_bar[la % kStages], (la / kStages) & 1, &s_abort, p.status);
     bar_sync(1, kPfSoftmax);
     float l_tot = 0.f;
 #pragma unroll
-    for (int q = 0; q < kPfGroups; ++q) l_tot += red[nstages & 1][q][row];
+    for (int q = 0; q < kPfGroups; ++q) l_tot += red[nunits & 1][q][row];
     if (!__any_sync(kFull, s_abort != 0)) {  // warp-uniform: TMEM loads are warp-wide
       tc_fence_after();
       const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
@@ -492,11 +552,11 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
   if (warp == kPfMmaWarp) tmem_dealloc(tm, kTmemCols);
 }
 
-template <int D, int BS, int KV_T>
-cudaError_t launch_prefill(const CUtensorMap &km, const CUtensorMap &vm, const PrefillParams &p,
-                           int tiles, cudaStream_t st) {
+template <int D, int BS, int KV_T, bool VBLK>
+cudaError_t launch_prefill_v(const CUtensorMap &km, const CUtensorMap &vm, const PrefillParams &p,
+                             int tiles, cudaStream_t st) {
   constexpr int smem = pf_stages(D) * 2 * kPfKeys * D * 2 + 1024;
-  auto kern = attn_prefill_kernel<D, BS, KV_T>;
+  auto kern = attn_prefill_kernel<D, BS, KV_T, VBLK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   e = launch_pdl(kern, dim3(tiles, p.kv_heads, p.num_seqs), dim3(kPfThreads), smem, st, km, vm, p);
@@ -504,8 +564,16 @@ cudaError_t launch_prefill(const CUtensorMap &km, const CUtensorMap &vm, const P
   return cudaGetLastError();
 }
 
-using PrefillFn = cudaError_t (*)(const CUtensorMap &, const CUtensorMap &, const PrefillParams &,
-                                  int, cudaStream_t);
+template <int D, int BS, int KV_T>
+cudaError_t launch_prefill(const LayerMaps &maps, const PrefillParams &p, int tiles,
+                           cudaStream_t st) {
+  if constexpr (D == 128) {
+    if (maps.v_blk_ok) return launch_prefill_v<D, BS, KV_T, true>(maps.k, maps.v_blk, p, tiles, st);
+  }
+  return launch_prefill_v<D, BS, KV_T, false>(maps.k, maps.v, p, tiles, st);
+}
+
+using PrefillFn = cudaError_t (*)(const LayerMaps &, const PrefillParams &, int, cudaStream_t);
 
 template <int D>
 PrefillFn pick_prefill_bs(int bs, int dt) {
@@ -572,6 +640,6 @@ extern "C" kv_status paged_attn_prefill(kv_pool *pool, int32_t layer, const void
   if (!layer_maps(pool, layer, pool->d.block_size, &maps, &code)) return code;
   const int D = pool->d.head_dim, bs = pool->d.block_size;
   PrefillFn fn = D == 128 ? pick_prefill_bs<128>(bs, cd) : pick_prefill_bs<64>(bs, cd);
-  kv_status s = cuda_check(fn(maps.k, maps.v, p, tiles, (cudaStream_t)stream), "prefill launch");
+  kv_status s = cuda_check(fn(maps, p, tiles, (cudaStream_t)stream), "prefill launch");
   return s == KV_OK ? ok() : s;
 }

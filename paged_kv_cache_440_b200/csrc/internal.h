@@ -52,6 +52,12 @@ struct Layout {
 struct LayerMaps {
   CUtensorMap k;
   CUtensorMap v;
+  // V as [row][slab of 128 bytes] with the slab as the outer coordinate: one
+  // box brings a block-head's rows of every slab, landing slab-major (16-bit
+  // caches with 256-byte rows only; v_blk_ok is false where the driver
+  // declined the encoding)
+  CUtensorMap v_blk;
+  bool v_blk_ok = false;
   int box_rows = 0;  // rows per box the maps were encoded for (0 = none yet)
 };
 

@@ -150,6 +150,26 @@ static bool encode_region(const kv_pool *p, void *base, int box_rows, CUtensorMa
   return true;
 }
 
+// 3-D view of a 16-bit region with 256-byte rows: (64 elements, row, slab),
+// strides (row: 256 bytes, slab: 128 bytes); a (64, box_rows, 2) box lands in
+// shared memory as [slab][row][128 bytes], 128-byte swizzled.
+static bool encode_region_slabs(const kv_pool *p, void *base, int box_rows, CUtensorMap *map) {
+  std::string why;
+  auto fn = encode_fn(&why);
+  if (!fn) return false;
+  const kv_pool_desc &d = p->d;
+  if ((d.cache_dtype != KV_BF16 && d.cache_dtype != KV_FP16) || p->row_bytes != 256) return false;
+  const CUtensorMapDataType dt =
+      d.cache_dtype == KV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  cuuint64_t gdim[3] = {64, (cuuint64_t)d.num_blocks * d.num_kv_heads * d.block_size, 2};
+  cuuint64_t gstride[2] = {256, 128};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 2};
+  cuuint32_t estride[3] = {1, 1, 1};
+  return fn(map, dt, 3, base, gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool layer_maps(kv_pool *p, int layer, int box_rows, LayerMaps *out, kv_status *code) {
   std::lock_guard<std::mutex> g(p->map_mu);
   std::vector<LayerMaps> &v = p->maps[layer];
@@ -167,6 +187,7 @@ bool layer_maps(kv_pool *p, int layer, int box_rows, LayerMaps *out, kv_status *
     *code = fail(KV_ERR_CUDA, "tensor map for layer %d: %s", layer, why.c_str());
     return false;
   }
+  m.v_blk_ok = encode_region_slabs(p, layer_v(p, layer), box_rows, &m.v_blk);
   m.box_rows = box_rows;
   v.push_back(m);
   *out = m;
