@@ -12,39 +12,45 @@
 //   are (token, query head of the KV head's group) pairs, head fastest:
 //   128 / G tokens x G heads. Row r lives in TMEM lane r.
 // * Two producer warps (K boxes, V boxes) stream the KV head's cached
-//   blocks, 64 positions per stage (128-byte swizzled TMA boxes of one
-//   block-head slab, one box per lane), into a ring of 6 (head_dim 128) or 8
-//   (64) stages; block ids are read a 32-block window ahead.
+//   blocks, 64 positions per stage, into a ring of 6 (head_dim 128) or 8 (64)
+//   stages; block ids are read a 32-block window ahead, each TMA box is issued
+//   by its own lane. K lands slab-major across the ring ([128-byte slab][slot
+//   x 64 + key][128 B], one box per block and slab), so two adjacent stages
+//   form one 128-key operand. V lands per stage, one box per block and slab,
+//   or one box per block where a 3-D (element, row, slab) view of the pool is
+//   accepted by the driver ([block][slab][row][128 B]).
 // * The MMA warp (one thread) issues tcgen05 MMAs with the A operand in
-//   tensor memory and B in shared memory: S_j = Q K_j^T (M 128, N 64,
-//   K head_dim; Q in TMEM, K K-major from the TMA stage) into one of three
-//   TMEM score buffers, and O += P_j V_j (M 128, N head_dim, K 64; P in
-//   TMEM, V MN-major from the TMA stage) into a TMEM accumulator that stays
-//   resident for the whole key range. Order: S_0, S_1, S_2, then per stage j
-//   O += P_j V_j followed by S_{j+3}, so the scores of the next stages are
-//   ready before the softmax warps ask for them. Measured on B200, an MMA of
-//   this size takes the tensor core 45-65 cycles but its issuing thread can
-//   spend more when it runs extra instructions between MMAs: the issue loop
-//   carries precomputed descriptors and compile-time accumulate flags only.
+//   tensor memory and B in shared memory, per unit of 128 keys (two stages):
+//   S_u = Q K_u^T (M 128, N 128, K head_dim; Q in TMEM, K K-major) into one
+//   of two TMEM score buffers, and O += P_u V_u (M 128, N head_dim, 16 keys
+//   per MMA; P in TMEM, V MN-major) into a TMEM accumulator that stays
+//   resident for the whole key range. Order: S_0, S_1, then per unit u
+//   O += P_u V_u followed by S_{u+2}, so the tensor core computes the next
+//   scores while the softmax warps work on the current ones. Measured on
+//   B200, an M 128 x N 128 x K 16 MMA takes the tensor core ~65 cycles, but
+//   its issuing thread can take longer when it runs other instructions
+//   between MMAs: the issue loop carries precomputed descriptors and
+//   compile-time accumulate flags only.
 // * 8 softmax warps (PAGEDKV_PF_GROUPS = 2 column groups; 4 gives 16 warps,
 //   measured slower): warp w reads TMEM lanes 32 (w mod 4) .. + 31 (the lanes
 //   a warp may access) and columns of group w / 4, so two threads share a
-//   row, 32 scores each per stage; the row maximum is combined through shared
-//   memory once per stage. Scale, causal and tail masks and the online
+//   row, 64 scores each per unit (read from TMEM twice: a max pass, then an
+//   exp pass, 32 columns at a time); the row maximum is combined through
+//   shared memory once per unit. Scale, causal and tail masks and the online
 //   softmax run in fp32 (base 2), two lanes per instruction where the
 //   hardware has packed fp32 arithmetic. The running maximum is only raised
 //   (and O, l rescaled in TMEM) when a new score exceeds it by more than 2^8;
 //   otherwise the stale maximum stays in use, which keeps every P value below
 //   256 and leaves the result unchanged up to rounding.
-// * P_j overwrites S_j in TMEM, each thread in its own columns, as two
+// * P_u overwrites S_u in TMEM, each thread in its own columns, as two
 //   16-bit parts hi + lo (per 16 scores: 8 columns of packed hi pairs, then
 //   8 of lo pairs, the layout of one K step of the MMA's A); O accumulates
 //   P_hi V + P_lo V, so rounding P to 16 bits costs nothing measurable (bf16:
 //   hi and lo by truncation, bit masks only; fp16: by rounding conversions).
 // * Synchronisation is by mbarriers: TMA -> MMA (full), MMA -> producer
-//   (stage free, by tcgen05.commit after P_j V_j), MMA -> softmax (S_j ready),
-//   softmax -> MMA (P_j written), MMA -> softmax (P_j V_j done, needed only to
-//   rescale O and for the final read). Every wait is bounded; after a timeout
+//   (stage free, by tcgen05.commit after P_u V; the softmax warps wait on the
+//   same commit before they rescale O or read it at the end), MMA -> softmax
+//   (S_u ready), softmax -> MMA (P_u written). Every wait is bounded; after a timeout
 //   every role runs to the end without waiting, the output is not written and
 //   the CTA frees its TMEM.
 #include <algorithm>
