@@ -58,6 +58,25 @@ def append_quantized(k_codes, v_codes, k_scales, v_scales, k_new, v_new,
         v_scales[blk, :, row] = vs[i]
 
 
+def append_quantized_kchan(k_codes, v_codes, v_scales, k_new, v_new, slot_mapping,
+                           block_size, chan_scales):
+    """As append_quantized for INT8 keys with per-channel scales: K rows are
+    quantized with the layer's fixed [Hkv, D] channel scales
+    (quant.quantize_k_channels), V rows per token and head (INT8 absmax).
+
+    k_codes, v_codes [NB, Hkv, bs, D] int8; v_scales [NB, Hkv, bs] float32.
+    """
+    kc = quant.quantize_k_channels(k_new, chan_scales)
+    vc, vs = quant.quantize_rows(v_new, "int8")
+    for i, slot in enumerate(np.asarray(slot_mapping).tolist()):
+        if slot < 0:
+            continue
+        blk, row = divmod(int(slot), block_size)
+        k_codes[blk, :, row, :] = kc[i]
+        v_codes[blk, :, row, :] = vc[i]
+        v_scales[blk, :, row] = vs[i]
+
+
 def block_copy(arrays, pairs):
     """In place: for each (src, dst) pair, every array's block dst := block src.
 

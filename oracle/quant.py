@@ -1,4 +1,5 @@
-"""KV-cache quantization reference: INT8 and FP8-E5M2 with per-token-head scales.
+"""KV-cache quantization reference: INT8 and FP8-E5M2 with per-token-head scales,
+INT8 keys with per-channel scales.
 
 Test infrastructure only (see ``oracle/__init__``).
 
@@ -171,3 +172,33 @@ def dequantize(codes, scales, kind):
     else:
         raise ValueError(kind)
     return v * np.asarray(scales, dtype=np.float32).astype(np.float64)[..., None]
+
+
+def quantize_k_channels(k, chan_scales):
+    """INT8 keys with one scale per (kv head, channel).
+
+    The pages list per-channel granularity (one scale per channel) beside
+    per-tensor and per-token-head, and suggest per-channel or per-token for K
+    while V may take a coarser one [bjdmk.com.cn/news/6246348, §5.2; KV Cache
+    原理与 PagedAttention, §四 table, INT8 row: per-tensor/per-channel].
+    Readings (the pages fix none of these): the scales are fixed for a layer
+    (calibrated or set by the caller, not derived from the rows being
+    written); y = fl32(k / s_c) (IEEE fp32 division); code = clamp(
+    round-half-even(y), -127, 127); a zero scale gives code 0.
+
+    k: [..., H, D] float32-representable values; chan_scales: [H, D] float32.
+    Returns int8 codes of k's shape.
+    """
+    k = np.asarray(k, dtype=np.float32)
+    s = np.asarray(chan_scales, dtype=np.float32)
+    nz = s > 0
+    safe = np.where(nz, s, np.float32(1.0))
+    y = np.divide(k, safe, dtype=np.float32)                  # fl32(k / s), broadcast [H, D]
+    codes = int8_encode(y)
+    return np.where(nz, codes, np.int8(0)).astype(np.int8)
+
+
+def dequantize_k_channels(codes, chan_scales):
+    """codes [..., H, D] int8, chan_scales [H, D] -> float64 code * s_c (exact)."""
+    return np.asarray(codes, dtype=np.int8).astype(np.float64) * \
+        np.asarray(chan_scales, dtype=np.float32).astype(np.float64)

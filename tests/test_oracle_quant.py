@@ -176,3 +176,65 @@ def test_int4_bounds_and_packing():
     allc = np.array([[a, b] for a in range(-8, 8) for b in range(-8, 8)], dtype=np.int8)
     assert np.array_equal(quant.unpack_int4(quant.pack_int4(allc)), allc)
     assert quant.pack_int4(allc).shape == (256, 1) and len(set(quant.pack_int4(allc)[:, 0])) == 256
+
+
+def test_kchan_hand_rows():
+    with open(GOLDEN) as f:
+        g = json.load(f)
+    for case in g["int8_kchan"]:
+        s = np.array(case["scales"], dtype=np.float32)[None, :]      # one kv head
+        k = np.array(case["k"], dtype=np.float32)[None, None, :]      # one token
+        codes = quant.quantize_k_channels(k, s)
+        assert list(codes[0, 0].astype(np.int64)) == case["codes"], case["why"]
+
+
+def test_kchan_equals_per_token_int8_when_the_scales_agree():
+    """With every channel of head h given that head's per-token absmax scale,
+    per-channel coding is the per-token INT8 coding of the same row."""
+    rng = np.random.default_rng(21)
+    k = (rng.standard_normal((1, 8, 128)) * rng.uniform(0.1, 10, (1, 8, 1))).astype(np.float32)
+    codes_tok, scale_tok = quant.quantize_rows(k, "int8")
+    chan = np.repeat(scale_tok[0][:, None], 128, axis=1)
+    codes_ch = quant.quantize_k_channels(k, chan)
+    assert np.array_equal(codes_ch, codes_tok)
+
+
+def test_kchan_error_bound_and_saturation():
+    rng = np.random.default_rng(22)
+    H, D = 4, 128
+    s = rng.uniform(0.001, 0.1, (H, D)).astype(np.float32)
+    k = (rng.standard_normal((512, H, D)) * 4.0).astype(np.float32)
+    codes = quant.quantize_k_channels(k, s)
+    deq = quant.dequantize_k_channels(codes, s)
+    sd = s.astype(np.float64)
+    kd = k.astype(np.float64)
+    inside = np.abs(kd) <= 126.5 * sd
+    # round to nearest of an fp32 quotient: within half a step (+ the quotient's rounding)
+    assert np.all(np.abs(deq - kd)[inside] <= (0.5 * sd * (1 + 1e-6) + np.abs(kd) * 2.0 ** -23)[inside])
+    big = np.abs(kd) >= 127.5 * sd * (1 + 1e-6)
+    assert big.any()
+    assert np.array_equal(np.abs(codes[big]).astype(np.int64), np.full(big.sum(), 127))
+    # integer multiples of a power-of-two scale come back exactly
+    s2 = np.full((H, D), 0.125, np.float32)
+    m = rng.integers(-127, 128, (64, H, D))
+    kk = (m * 0.125).astype(np.float32)
+    assert np.array_equal(quant.dequantize_k_channels(quant.quantize_k_channels(kk, s2), s2), kk)
+
+
+def test_kchan_append_places_codes_and_value_scales():
+    from oracle import cache_ops
+    rng = np.random.default_rng(23)
+    NB, H, bs, D = 5, 2, 16, 64
+    kc = np.zeros((NB, H, bs, D), np.int8)
+    vc = np.zeros((NB, H, bs, D), np.int8)
+    vs = np.zeros((NB, H, bs), np.float32)
+    chan = rng.uniform(0.01, 0.05, (H, D)).astype(np.float32)
+    k = rng.standard_normal((3, H, D)).astype(np.float32)
+    v = rng.standard_normal((3, H, D)).astype(np.float32)
+    slots = np.array([2 * bs + 5, -1, 4 * bs + 15])
+    cache_ops.append_quantized_kchan(kc, vc, vs, k, v, slots, bs, chan)
+    for i, blk, row in ((0, 2, 5), (2, 4, 15)):
+        assert np.array_equal(kc[blk, :, row], quant.quantize_k_channels(k[i], chan))
+        c, s = quant.quantize_rows(v[i], "int8")
+        assert np.array_equal(vc[blk, :, row], c) and np.array_equal(vs[blk, :, row], s)
+    assert not kc[[0, 1, 3]].any() and not vc[[0, 1, 3]].any()    # the skipped slot wrote nothing
