@@ -66,6 +66,9 @@ WORKLOADS = {
                      "block 32, 64 x 4096", lambda dev: W.quant_long("int4", "a", dev)),
     "quant_a_e5m2_cast": ("FP8-E5M2 KV cast with no scale: 64/8 heads, head_dim 128, block 32, "
                           "64 x 4096", lambda dev: W.quant_long("e5m2_cast", "a", dev)),
+    "quant_a_int8_kchan": ("INT8 KV, keys with fixed per-channel scales, values per token-head: "
+                           "64/8 heads, head_dim 128, block 32, 64 x 4096",
+                           lambda dev: W.quant_long("int8_kchan", "a", dev)),
     "shared_prefix": ("Shared prompt: 200 requests, 1500-token prefix in 94 shared blocks (the last "
                       "copied on write per request), suffixes U[1,512], 64/8 heads, D 128, bf16, "
                       "block 16; GB/s counts logical bytes (the shared prefix is read from L2)",
@@ -107,11 +110,14 @@ def step_bytes(wl):
     kv = tokens * wl.kv_heads * wl.head_dim * 2 * e
     if wl.cache_dtype in ("int8", "e5m2", "int4"):
         kv += tokens * wl.kv_heads * 2 * 4                   # per-token-head scales
+    elif wl.cache_dtype == "int8_kchan":
+        kv += tokens * wl.kv_heads * 4 + wl.kv_heads * wl.head_dim * 4   # V rows + K channels
     q_out = 2 * wl.batch * wl.q_heads * wl.head_dim * 2
     rows = wl.batch * wl.kv_heads
     append = rows * wl.head_dim * 2 * 2 + wl.batch * 8        # read new K, V and slots
     append += rows * wl.head_dim * 2 * e + \
-        (rows * 2 * 4 if wl.cache_dtype in ("int8", "e5m2", "int4") else 0)   # write rows
+        (rows * 2 * 4 if wl.cache_dtype in ("int8", "e5m2", "int4") else
+         rows * 4 if wl.cache_dtype == "int8_kchan" else 0)                  # write rows
     return int(kv + q_out), int(append)
 
 
@@ -438,7 +444,9 @@ def run_ours(args, rank, world, device):
     wl = make(device)
     pool = pkv.KVPool(1, wl.num_blocks, wl.block_size, wl.kv_heads, wl.head_dim,
                       wl.cache_dtype, device)
-    K, V, _, _ = pool.layer_views(0)
+    K, V, KS, _ = pool.layer_views(0)
+    if getattr(wl, "k_chan", None) is not None:
+        KS.copy_(torch.from_numpy(wl.k_chan).to(device))   # the layer's key channel scales
     if getattr(wl, "setup", None) is not None:
         wl.setup(pool, pkv)        # builds the cache through the allocator and CoW
     elif wl.k_fill is not None:

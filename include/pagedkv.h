@@ -67,8 +67,10 @@ typedef enum {
   KV_FP8_E5M2 = 2,         /* 1 sign, 5 exponent (bias 15), 2 mantissa bits     */
   KV_INT8 = 3,             /* two's complement, codes in [-127, 127]            */
   KV_FP8_E5M2_CAST = 4,    /* E5M2 codes cast from the values with no scale     */
-  KV_INT4 = 5              /* 4-bit codes in [-7, 7], two per byte (element 2i  */
+  KV_INT4 = 5,             /* 4-bit codes in [-7, 7], two per byte (element 2i  */
                            /* in the low nibble), head_dim 128 only             */
+  KV_INT8_KCHAN = 6        /* INT8 keys with one fixed fp32 scale per (kv head, */
+                           /* channel), INT8 values with per-token-head scales  */
 } kv_dtype;
 
 /* Bits of the device status word. */
@@ -100,8 +102,12 @@ typedef struct kv_pool kv_pool;   /* opaque host object */
  * starting on a 256-byte boundary:
  *   K       [num_blocks][num_kv_heads][block_size][head_dim]  cache_dtype
  *   V       same
- *   K scale [num_blocks][num_kv_heads][block_size]  fp32   (INT8 / E5M2 only)
- *   V scale same                                            (INT8 / E5M2 only)
+ *   K scale [num_blocks][num_kv_heads][block_size]  fp32   (INT8 / E5M2 / INT4)
+ *           [num_kv_heads][head_dim]                fp32   (INT8_KCHAN: the
+ *           layer's channel scales, written by the caller before any append;
+ *           per-channel granularity [bjdmk.com.cn/news/6246348, §5.2])
+ *   V scale [num_blocks][num_kv_heads][block_size]  fp32   (INT8 / E5M2 / INT4 /
+ *                                                            INT8_KCHAN)
  * followed by one 256-byte status region. One (block, head) tile of K or V is
  * contiguous (block_size * head_dim elements). K and V of a layer take exactly
  * 2 * num_kv_heads * head_dim * elem_bytes * (num_blocks * block_size) bytes,
@@ -124,7 +130,9 @@ kv_status kv_pool_create(const kv_pool_desc *desc, void *device_base,
 kv_status kv_pool_destroy(kv_pool *pool);
 
 /* Device addresses of one layer's regions. k_scale / v_scale are set to NULL
- * for 16-bit caches. Any output pointer may be NULL if not wanted. */
+ * for 16-bit and scale-less caches. For KV_INT8_KCHAN k_scale is the layer's
+ * [num_kv_heads][head_dim] channel-scale array (caller-written). Any output
+ * pointer may be NULL if not wanted. */
 kv_status kv_pool_layer_ptrs(const kv_pool *pool, int32_t layer, void **k,
                              void **v, float **k_scale, float **v_scale);
 
@@ -195,7 +203,11 @@ kv_status kv_append(kv_pool *pool, int32_t layer, const void *k_new,
                     const int64_t *slot_mapping, int32_t num_tokens,
                     kv_stream_t stream);
 
-/* Per-row symmetric absmax quantization [bjdmk.com.cn/news/6246348, §5.2:
+/* KV_INT8_KCHAN caches: each key value k of head h, channel c is stored as
+ *   clamp(round-half-even(fl32(k / s[h][c])), -127, 127) (0 where s[h][c] is
+ *   0) with s the layer's channel scales; each V row as for KV_INT8.
+ *
+ * Per-row symmetric absmax quantization [bjdmk.com.cn/news/6246348, §5.2:
  * one scale per token per head]:
  *   a = max|x|; scale = fl32(a / QMAX) (QMAX 127 for INT8, 57344 for E5M2);
  *   code = round-half-even(fl32(x / scale)), clamped to [-127, 127] (INT8) or

@@ -23,13 +23,15 @@ lib = ctypes.CDLL(LIB_PATH)
 # ----------------------------------------------------------------- constants
 KV_OK, KV_ERR_INVALID, KV_ERR_OOM, KV_ERR_CUDA, KV_ERR_UNSUPPORTED = 0, 1, 2, 3, 4
 KV_BF16, KV_FP16, KV_FP8_E5M2, KV_INT8, KV_FP8_E5M2_CAST, KV_INT4 = 0, 1, 2, 3, 4, 5
+KV_INT8_KCHAN = 6
 KV_DEVERR_BLOCK_ID, KV_DEVERR_CONTEXT, KV_DEVERR_SLOT, KV_DEVERR_TIMEOUT = 1, 2, 4, 8
 
 DTYPE_CODES = {"bf16": KV_BF16, "fp16": KV_FP16, "e5m2": KV_FP8_E5M2, "int8": KV_INT8,
-               "e5m2_cast": KV_FP8_E5M2_CAST, "int4": KV_INT4}
+               "e5m2_cast": KV_FP8_E5M2_CAST, "int4": KV_INT4, "int8_kchan": KV_INT8_KCHAN}
 TORCH_CODES = {torch.bfloat16: KV_BF16, torch.float16: KV_FP16}
 CACHE_TORCH = {"bf16": torch.bfloat16, "fp16": torch.float16, "e5m2": torch.uint8,
-               "int8": torch.int8, "e5m2_cast": torch.uint8, "int4": torch.uint8}
+               "int8": torch.int8, "e5m2_cast": torch.uint8, "int4": torch.uint8,
+               "int8_kchan": torch.int8}
 
 
 def code_row(kind, head_dim):
@@ -177,7 +179,8 @@ class KVPool:
     block_size = property(lambda s: s.desc.block_size)
     num_kv_heads = property(lambda s: s.desc.num_kv_heads)
     head_dim = property(lambda s: s.desc.head_dim)
-    quantized = property(lambda s: s.cache_dtype in ("int8", "e5m2", "e5m2_cast", "int4"))
+    quantized = property(lambda s: s.cache_dtype in ("int8", "e5m2", "e5m2_cast", "int4",
+                                                     "int8_kchan"))
 
     def close(self):
         if getattr(self, "handle", None):
@@ -201,7 +204,10 @@ class KVPool:
         return self.buffer[off:off + nbytes].view(dtype).view(shape)
 
     def layer_views(self, layer):
-        """(K, V, K_scale, V_scale) torch views of one layer's regions."""
+        """(K, V, K_scale, V_scale) torch views of one layer's regions.
+
+        For "int8_kchan" pools K_scale is the layer's [kv_heads, head_dim]
+        channel-scale array, which the caller fills before appending."""
         k, v, ks, vs = self.layer_ptrs(layer)
         row = code_row(self.cache_dtype, self.head_dim)   # elements per (token, head) row
         shape = (self.num_blocks, self.num_kv_heads, self.block_size, row)
@@ -213,8 +219,12 @@ class KVPool:
         if ks is None:
             return K, V, None, None
         sshape = shape[:3]
-        return K, V, self._view(ks, n * 4, torch.float32, sshape), \
-            self._view(vs, n * 4, torch.float32, sshape)
+        if self.cache_dtype == "int8_kchan":
+            KS = self._view(ks, self.num_kv_heads * self.head_dim * 4, torch.float32,
+                            (self.num_kv_heads, self.head_dim))
+        else:
+            KS = self._view(ks, n * 4, torch.float32, sshape)
+        return K, V, KS, self._view(vs, n * 4, torch.float32, sshape)
 
     # status word
     def status_clear(self, stream=None):

@@ -66,7 +66,7 @@ struct AttnParams {
   void *out;
   const int32_t *block_tables;
   const int32_t *context_lens;
-  const float *k_scale;
+  const float *k_scale;  // per-token K scales, or (INT8_KCHAN) the [kv_heads][D] channel scales
   const float *v_scale;
   float *part_o;   // [num_ctas][2][kNC][8][D]   unnormalised outputs of split units
   float *part_ml;  // [num_ctas][2][kNC][8][2]   their (max, sum), base 2
@@ -113,12 +113,17 @@ struct Tile {
   static constexpr int kSlabs = kRowBytes / kSlab;
   static constexpr bool kQuant = !is16<KV_T>();                 // 1-byte codes
   static constexpr bool kScaled = kQuant && KV_T != KV_FP8_E5M2_CAST;  // with fp32 scales
+  // per-token K scale rows (INT8_KCHAN keys use the layer's channel scales)
+  static constexpr bool kKRowScales = kScaled && KV_T != KV_INT8_KCHAN;
 
   // A stage holds `rows` = HG * BS rows (HG heads of one block) of K, then of
   // V, each as kSlabs slabs of rows x kSlab bytes, then (quantized caches) the
-  // K and V scales of those rows.
+  // K scales (per-token ones only) and the V scales of those rows.
   __host__ __device__ static constexpr int load_bytes(int rows) {
-    return 2 * rows * kRowBytes + (kScaled ? 2 * rows * 4 : 0);
+    return 2 * rows * kRowBytes + (kScaled ? (kKRowScales ? 2 : 1) * rows * 4 : 0);
+  }
+  __host__ __device__ static constexpr int vscale_off(int rows) {
+    return 2 * rows * kRowBytes + (kKRowScales ? rows * 4 : 0);
   }
 
   // Shared-memory address of 16-byte chunk c of row r of the K (or V) part of
@@ -155,10 +160,8 @@ __device__ __forceinline__ void issue_stage(uint8_t *stage, uint64_t *bar, const
     tma_load_2d(stage + s * rows * T::kSlab, km, bar, s * (T::kSlab / T::kElt), row0);
     tma_load_2d(stage + kv + s * rows * T::kSlab, vm, bar, s * (T::kSlab / T::kElt), row0);
   }
-  if constexpr (T::kScaled) {
-    bulk_load(stage + 2 * kv, p.k_scale + row0, rows * 4, bar);
-    bulk_load(stage + 2 * kv + rows * 4, p.v_scale + row0, rows * 4, bar);
-  }
+  if constexpr (T::kKRowScales) bulk_load(stage + 2 * kv, p.k_scale + row0, rows * 4, bar);
+  if constexpr (T::kScaled) bulk_load(stage + T::vscale_off(rows), p.v_scale + row0, rows * 4, bar);
 }
 
 __device__ __forceinline__ float warp_max_xor(float v, int from) {
@@ -286,10 +289,13 @@ struct Consumer {
   static constexpr bool kBF = (KV_T == KV_BF16);  // MMA operand type (bf16, else fp16)
   static constexpr int KS = D / 16;  // k-steps over head_dim
   static constexpr int MT = BS / 16;  // 16-token tiles per block
+  static constexpr bool KCH = (KV_T == KV_INT8_KCHAN);  // keys with channel scales
+  static constexpr bool kInt8Codes = (KV_T == KV_INT8 || KCH);  // INT8 codes (K and V)
 
   float m_run[2], m2_run[2], l_run[2];
   float oacc[D / 16][4];
   uint32_t qb[KS][2];
+  uint32_t qlo[KCH ? KS : 1][2];  // INT8_KCHAN: the query's low parts (hi + lo ~ fp32)
   float s_fac[2];
   float qcorr[2];  // INT8 keys enter the MMA as 1152 + code: 1152 * sum(q) per head
 
@@ -332,6 +338,11 @@ struct Consumer {
                               ? (ks >> 1) * 32 + 8 * cq + 2 * (ks & 1) + ((e & 1) << 2) + (e >> 1)
                               : 16 * ks + 4 * cq + e;
           qv[ks][e] = hv ? load_q<Q_T>(p.q, qrow + dim) : 0.f;
+          if constexpr (KCH) {
+            // keys code k / s_c: the channel scale moves to the query,
+            // q . k = sum_c (q_c s_c) code_c
+            qv[ks][e] *= p.k_scale[(h0 / p.group) * D + dim];
+          }
           amax = fmaxf(amax, fabsf(qv[ks][e]));
         }
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
@@ -343,15 +354,21 @@ struct Consumer {
       }
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
-        qb[ks][0] = pack2<false>(ldexpf(qv[ks][0], ex), ldexpf(qv[ks][1], ex));
-        qb[ks][1] = pack2<false>(ldexpf(qv[ks][2], ex), ldexpf(qv[ks][3], ex));
+        if constexpr (KCH) {
+          // q_c s_c is not a 16-bit value: hi + lo fp16 parts, two MMAs
+          split2<false>(ldexpf(qv[ks][0], ex), ldexpf(qv[ks][1], ex), qb[ks][0], qlo[ks][0]);
+          split2<false>(ldexpf(qv[ks][2], ex), ldexpf(qv[ks][3], ex), qb[ks][1], qlo[ks][1]);
+        } else {
+          qb[ks][0] = pack2<false>(ldexpf(qv[ks][0], ex), ldexpf(qv[ks][1], ex));
+          qb[ks][1] = pack2<false>(ldexpf(qv[ks][2], ex), ldexpf(qv[ks][3], ex));
+        }
       }
       // the score columns of this lane are heads 2cq and 2cq+1
       const int ex0 = __shfl_sync(0xffffffffu, ex, (2 * cq) * 4);
       const int ex1 = __shfl_sync(0xffffffffu, ex, (2 * cq + 1) * 4);
       s_fac[0] = ldexpf(p.scale_log2, -ex0);
       s_fac[1] = ldexpf(p.scale_log2, -ex1);
-      if constexpr (KV_T == KV_INT8 || KV_T == KV_INT4) {
+      if constexpr (kInt8Codes || KV_T == KV_INT4) {
         // sum of the fp16 query operands of head gq (as the MMA sees them)
         float qsum = 0.f;
 #pragma unroll
@@ -359,10 +376,15 @@ struct Consumer {
           const __half2 a = *reinterpret_cast<const __half2 *>(&qb[ks][0]);
           const __half2 c = *reinterpret_cast<const __half2 *>(&qb[ks][1]);
           qsum += (__low2float(a) + __high2float(a)) + (__low2float(c) + __high2float(c));
+          if constexpr (KCH) {
+            const __half2 al = *reinterpret_cast<const __half2 *>(&qlo[ks][0]);
+            const __half2 cl = *reinterpret_cast<const __half2 *>(&qlo[ks][1]);
+            qsum += (__low2float(al) + __high2float(al)) + (__low2float(cl) + __high2float(cl));
+          }
         }
         qsum += __shfl_xor_sync(0xffffffffu, qsum, 1);
         qsum += __shfl_xor_sync(0xffffffffu, qsum, 2);
-        constexpr float kBias = KV_T == KV_INT8 ? 1152.f : 1032.f;
+        constexpr float kBias = kInt8Codes ? 1152.f : 1032.f;
         qcorr[0] = kBias * __shfl_sync(0xffffffffu, qsum, (2 * cq) * 4);
         qcorr[1] = kBias * __shfl_sync(0xffffffffu, qsum, (2 * cq + 1) * 4);
       }
@@ -377,7 +399,7 @@ struct Consumer {
     const uint32_t vtile = ktile + rows * T::kRowBytes;
     const int r0 = hi * BS;  // the head's first row in the stage
     const float *ksc = reinterpret_cast<const float *>(st + 2 * rows * T::kRowBytes) + r0;
-    const float *vsc = ksc + rows;
+    const float *vsc = reinterpret_cast<const float *>(st + T::vscale_off(rows)) + r0;
     const int gq = lane >> 2, cq = lane & 3;
     // ---------------------------------------------------- scores S = K q
     float sc[MT][4];
@@ -418,16 +440,20 @@ struct Consumer {
         for (int kp = 0; kp < KS / 2; ++kp) {
           uint32_t q0, q1, q2, q3;  // byte matrices: rows 0-7 / 8-15 x chunks 2kp, 2kp+1
           ldsm_x4(T::chunk(ktile, r0 + row, 2 * kp + (lane >> 4), rows), q0, q1, q2, q3);
-          if constexpr (KV_T == KV_INT8) {
+          if constexpr (kInt8Codes) {
             // keys as 1152 + code (exact in fp16); the bias is removed per
             // score below with the query sums
             q0 ^= 0x80808080u; q1 ^= 0x80808080u; q2 ^= 0x80808080u; q3 ^= 0x80808080u;
-            mma16816<false>(acc, int8_pair_biased<0, 1>(q0), int8_pair_biased<0, 1>(q1),
-                            int8_pair_biased<2, 3>(q0), int8_pair_biased<2, 3>(q1),
-                            qb[2 * kp][0], qb[2 * kp][1]);
-            mma16816<false>(acc, int8_pair_biased<0, 1>(q2), int8_pair_biased<0, 1>(q3),
-                            int8_pair_biased<2, 3>(q2), int8_pair_biased<2, 3>(q3),
-                            qb[2 * kp + 1][0], qb[2 * kp + 1][1]);
+            const uint32_t a00 = int8_pair_biased<0, 1>(q0), a01 = int8_pair_biased<0, 1>(q1);
+            const uint32_t a02 = int8_pair_biased<2, 3>(q0), a03 = int8_pair_biased<2, 3>(q1);
+            const uint32_t a10 = int8_pair_biased<0, 1>(q2), a11 = int8_pair_biased<0, 1>(q3);
+            const uint32_t a12 = int8_pair_biased<2, 3>(q2), a13 = int8_pair_biased<2, 3>(q3);
+            mma16816<false>(acc, a00, a01, a02, a03, qb[2 * kp][0], qb[2 * kp][1]);
+            mma16816<false>(acc, a10, a11, a12, a13, qb[2 * kp + 1][0], qb[2 * kp + 1][1]);
+            if constexpr (KCH) {
+              mma16816<false>(acc, a00, a01, a02, a03, qlo[2 * kp][0], qlo[2 * kp][1]);
+              mma16816<false>(acc, a10, a11, a12, a13, qlo[2 * kp + 1][0], qlo[2 * kp + 1][1]);
+            }
           } else {
             mma16816<false>(acc, e5m2_pair<0, 1>(q0), e5m2_pair<0, 1>(q1),
                             e5m2_pair<2, 3>(q0), e5m2_pair<2, 3>(q1), qb[2 * kp][0],
@@ -441,11 +467,11 @@ struct Consumer {
       // acc: [0],[1] = token mt*16+gq, heads 2cq, 2cq+1; [2],[3] = token +8
       const int t0 = mt * 16 + gq, t1 = t0 + 8;
       float k0 = 1.f, k1 = 1.f;
-      if constexpr (kScaled) {
+      if constexpr (T::kKRowScales) {
         k0 = ksc[t0];
         k1 = ksc[t1];
       }
-      if constexpr (KV_T == KV_INT8 || KV_T == KV_INT4) {
+      if constexpr (kInt8Codes || KV_T == KV_INT4) {
         acc[0] -= qcorr[0];
         acc[1] -= qcorr[1];
         acc[2] -= qcorr[0];
@@ -608,7 +634,7 @@ struct Consumer {
           // after the transpose a lane holds tokens (2cq, 2cq+1) x dims (2gq, 2gq+1)
           // of each 16-dim chunk: bytes 0,2 -> dim 2gq; bytes 1,3 -> dim 2gq+1
           uint32_t a[8];
-          if constexpr (KV_T == KV_INT8) {
+          if constexpr (kInt8Codes) {
             q0 ^= 0x80808080u; q1 ^= 0x80808080u; q2 ^= 0x80808080u; q3 ^= 0x80808080u;
             a[0] = int8_pair<0, 2>(q0); a[1] = int8_pair<1, 3>(q0);
             a[2] = int8_pair<0, 2>(q1); a[3] = int8_pair<1, 3>(q1);
@@ -723,6 +749,15 @@ struct NewRow {
         v[0] = *reinterpret_cast<const uint32_t *>(vn + lane * 2);
         k[1] = v[1] = 0u;
       }
+    } else if constexpr (KV_T == KV_INT8_KCHAN) {
+      // keys with the layer's channel scales, values per row as INT8
+      float x[E];
+      load_row<D, Q_T>(kn, lane, x);
+      k[0] = quantize_row_chan<D>(x, p.k_scale + g * D, lane);
+      ks = 1.f;
+      load_row<D, Q_T>(vn, lane, x);
+      v[0] = quantize_row<D, KV_INT8>(x, &vs);
+      k[1] = v[1] = 0u;
     } else {
       float x[E];
       load_row<D, Q_T>(kn, lane, x);
@@ -766,10 +801,11 @@ struct NewRow {
     }
     if constexpr (kScaled) {
       if (lane == 0) {
-        float *sc = reinterpret_cast<float *>(st + 2 * rows * T::kRowBytes);
-        sc[r] = ks;
-        sc[rows + r] = vs;
-        p.k_scale_w[grow] = ks;
+        if constexpr (T::kKRowScales) {
+          reinterpret_cast<float *>(st + 2 * rows * T::kRowBytes)[r] = ks;
+          p.k_scale_w[grow] = ks;
+        }
+        reinterpret_cast<float *>(st + T::vscale_off(rows))[r] = vs;
         p.v_scale_w[grow] = vs;
       }
     }
@@ -1142,6 +1178,9 @@ PartFn pick_dtype(int kv, int q) {
     case KV_FP8_E5M2:
       return q == KV_BF16 ? launch_part<D, BS, KV_FP8_E5M2, KV_BF16>
                           : launch_part<D, BS, KV_FP8_E5M2, KV_FP16>;
+    case KV_INT8_KCHAN:
+      return q == KV_BF16 ? launch_part<D, BS, KV_INT8_KCHAN, KV_BF16>
+                          : launch_part<D, BS, KV_INT8_KCHAN, KV_FP16>;
     case KV_INT4:  // pools reject INT4 unless head_dim is 128
       if constexpr (D == 128)
         return q == KV_BF16 ? launch_part<D, BS, KV_INT4, KV_BF16> : launch_part<D, BS, KV_INT4, KV_FP16>;

@@ -7,7 +7,9 @@
 //   slot % block_size of physical block slot / block_size.
 // * Quantize: symmetric absmax per (token, head) row, fp32 scale
 //   [bjdmk.com.cn/news/6246348, §5.2]; INT8 or FP8-E5M2 codes
-//   [KV Cache 原理与 PagedAttention, §四].
+//   [KV Cache 原理与 PagedAttention, §四]. INT8_KCHAN caches code keys with
+//   the layer's fixed per-channel scales (per-channel granularity, §5.2 of
+//   the same page) and values per row as INT8.
 // * Block copy: the copy half of copy-on-write [bjdmk.com.cn/news/6246348,
 //   §3.2]: whole blocks, every layer, K, V and scales.
 //
@@ -91,17 +93,23 @@ append_quant_kernel(const uint16_t *__restrict__ k_new, const uint16_t *__restri
   const int row = static_cast<int>(slot - blk * block_size);
   const int64_t dst_row = (blk * kv_heads + h) * block_size + row;
   const int64_t src_row = static_cast<int64_t>(t) * kv_heads + h;
+  // INT8_KCHAN: ks holds the layer's [kv_heads][D] channel scales
+  constexpr int VQ = OUT_T == KV_INT8_KCHAN ? KV_INT8 : OUT_T;  // value coding
   float x[D / 32];
   float scale;
   load_row<D, IN_T>(k_new + src_row * D, lane, x);
-  uint32_t packed = quantize_row<D, OUT_T>(x, &scale);
   constexpr int kRow = OUT_T == KV_INT4 ? D / 2 : D;  // bytes per row
-  store_codes<D, OUT_T>(kc + dst_row * kRow, lane, packed);
-  if (OUT_T != KV_FP8_E5M2_CAST && lane == 0) ks[dst_row] = scale;
+  if constexpr (OUT_T == KV_INT8_KCHAN) {
+    store_codes<D, KV_INT8>(kc + dst_row * kRow, lane, quantize_row_chan<D>(x, ks + h * D, lane));
+  } else {
+    const uint32_t packed = quantize_row<D, OUT_T>(x, &scale);
+    store_codes<D, OUT_T>(kc + dst_row * kRow, lane, packed);
+    if (OUT_T != KV_FP8_E5M2_CAST && lane == 0) ks[dst_row] = scale;
+  }
   load_row<D, IN_T>(v_new + src_row * D, lane, x);
-  packed = quantize_row<D, OUT_T>(x, &scale);
-  store_codes<D, OUT_T>(vc + dst_row * kRow, lane, packed);
-  if (OUT_T != KV_FP8_E5M2_CAST && lane == 0) vs[dst_row] = scale;
+  const uint32_t vpacked = quantize_row<D, VQ>(x, &scale);
+  store_codes<D, VQ>(vc + dst_row * kRow, lane, vpacked);
+  if (VQ != KV_FP8_E5M2_CAST && lane == 0) vs[dst_row] = scale;
 }
 
 // Standalone: one warp per contiguous row.
@@ -129,14 +137,15 @@ struct CopyPairs {
   int32_t dst[kMaxPairsPerLaunch];
 };
 
-// grid (pair, layer, region): region 0 = K, 1 = V, 2 = K scale, 3 = V scale.
+// grid (pair, layer, region): region 0 = K, 1 = V, 2 = K scale, 3 = V scale
+// (no K-scale rows when the keys use channel scales: region 2 is then V's).
 __global__ void __launch_bounds__(256)
 block_copy_kernel(const __grid_constant__ CopyPairs pairs, char *__restrict__ base,
-                  uint64_t layer_stride, uint64_t kv_stride, uint64_t sc_stride,
-                  uint32_t kv_block_bytes, uint32_t sc_block_bytes) {
+                  uint64_t layer_stride, uint64_t kv_stride, uint64_t ksc_stride,
+                  uint32_t kv_block_bytes, uint32_t sc_block_bytes, int k_scale_rows) {
   const int i = blockIdx.x;
   const uint64_t layer = blockIdx.y;
-  const int region = blockIdx.z;
+  const int region = (blockIdx.z == 2 && !k_scale_rows) ? 3 : blockIdx.z;
   char *lb = base + layer * layer_stride;
   char *rb;
   uint32_t bytes;
@@ -144,7 +153,7 @@ block_copy_kernel(const __grid_constant__ CopyPairs pairs, char *__restrict__ ba
     case 0: rb = lb; bytes = kv_block_bytes; break;
     case 1: rb = lb + kv_stride; bytes = kv_block_bytes; break;
     case 2: rb = lb + 2 * kv_stride; bytes = sc_block_bytes; break;
-    default: rb = lb + 2 * kv_stride + sc_stride; bytes = sc_block_bytes; break;
+    default: rb = lb + 2 * kv_stride + ksc_stride; bytes = sc_block_bytes; break;
   }
   const uint4 *src = reinterpret_cast<const uint4 *>(rb + (uint64_t)pairs.src[i] * bytes);
   uint4 *dst = reinterpret_cast<uint4 *>(rb + (uint64_t)pairs.dst[i] * bytes);
@@ -236,6 +245,10 @@ kv_status kv_append(kv_pool *pool, int32_t layer, const void *k_new, const void 
     e = in_dtype == KV_BF16
             ? launch_append_quant<128, KV_BF16, KV_INT4>(pool, layer, k_new, v_new, slot_mapping, num_tokens, st)
             : launch_append_quant<128, KV_FP16, KV_INT4>(pool, layer, k_new, v_new, slot_mapping, num_tokens, st);
+  } else if (cd == KV_INT8_KCHAN) {
+    e = in_dtype == KV_BF16
+            ? dispatch_append_quant_d<KV_BF16, KV_INT8_KCHAN>(pool, layer, k_new, v_new, slot_mapping, num_tokens, st)
+            : dispatch_append_quant_d<KV_FP16, KV_INT8_KCHAN>(pool, layer, k_new, v_new, slot_mapping, num_tokens, st);
   } else if (cd == KV_FP8_E5M2) {
     e = in_dtype == KV_BF16
             ? dispatch_append_quant_d<KV_BF16, KV_FP8_E5M2>(pool, layer, k_new, v_new, slot_mapping, num_tokens, st)
@@ -306,7 +319,7 @@ kv_status kv_block_copy(kv_pool *pool, const int32_t *host_pairs, int32_t n_pair
   const kv_pool_desc &dd = pool->d;
   const uint32_t kv_block = (uint32_t)dd.num_kv_heads * dd.block_size * pool->row_bytes;
   const uint32_t sc_block = (uint32_t)dd.num_kv_heads * dd.block_size * sizeof(float);
-  const int regions = has_scales(dd.cache_dtype) ? 4 : 2;
+  const int regions = !has_scales(dd.cache_dtype) ? 2 : k_chan_scales(dd.cache_dtype) ? 3 : 4;
   cudaStream_t st = (cudaStream_t)stream;
   for (int32_t base = 0; base < n_pairs; base += kMaxPairsPerLaunch) {
     const int32_t n = std::min<int32_t>(kMaxPairsPerLaunch, n_pairs - base);
@@ -317,8 +330,8 @@ kv_status kv_block_copy(kv_pool *pool, const int32_t *host_pairs, int32_t n_pair
     }
     dim3 grid(n, dd.num_layers, regions);
     block_copy_kernel<<<grid, 256, 0, st>>>(cp, pool->base, pool->lay.layer_stride,
-                                            pool->lay.kv_stride, pool->lay.sc_stride, kv_block,
-                                            sc_block);
+                                            pool->lay.kv_stride, pool->lay.ksc_stride, kv_block,
+                                            sc_block, k_chan_scales(dd.cache_dtype) ? 0 : 1);
     kv_status s = cuda_check(cudaGetLastError(), "kv_block_copy launch");
     if (s != KV_OK) return s;
   }

@@ -360,6 +360,27 @@ __device__ __forceinline__ void load_row(const uint16_t *__restrict__ src, int l
   }
 }
 
+// INT8 codes of this lane's share of a key row with one fixed scale per
+// channel: code = clamp(round-half-even(fl32(x / s)), -127, 127), 0 where the
+// scale is not positive. cs: the head's head_dim channel scales.
+template <int D>
+__device__ __forceinline__ uint32_t quantize_row_chan(const float (&x)[D / 32], const float *cs,
+                                                      int lane) {
+  constexpr int E = D / 32;
+  uint32_t packed = 0;
+#pragma unroll
+  for (int i = 0; i < E; ++i) {
+    const float s = cs[lane * E + i];
+    int q = 0;
+    if (s > 0.f) {
+      q = __float2int_rn(__fdiv_rn(x[i], s));
+      q = max(-127, min(127, q));
+    }
+    packed |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * i);
+  }
+  return packed;
+}
+
 // Store this lane's codes of one row (row base `dst`): D/32 bytes, or D/64
 // for INT4 (4 bits per code).
 template <int D, int OUT_T = KV_INT8>

@@ -28,20 +28,24 @@ inline int row_bytes_of(int dtype, int head_dim) {
 // 1-byte codes (read through the code paths of the kernels)
 inline bool is_quant(int dtype) {
   return dtype == KV_INT8 || dtype == KV_FP8_E5M2 || dtype == KV_FP8_E5M2_CAST ||
-         dtype == KV_INT4;
+         dtype == KV_INT4 || dtype == KV_INT8_KCHAN;
 }
-// codes with a per-token-head fp32 scale (scale regions in the pool)
+// codes with fp32 scales (scale regions in the pool): per-token-head rows for
+// V, and for K too unless the keys use channel scales
 inline bool has_scales(int dtype) {
-  return dtype == KV_INT8 || dtype == KV_FP8_E5M2 || dtype == KV_INT4;
+  return dtype == KV_INT8 || dtype == KV_FP8_E5M2 || dtype == KV_INT4 || dtype == KV_INT8_KCHAN;
 }
+// keys with one fixed scale per (kv head, channel) of the layer
+inline bool k_chan_scales(int dtype) { return dtype == KV_INT8_KCHAN; }
 inline uint64_t round_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
 
 // Byte offsets of one layer's regions inside the pool buffer.
 struct Layout {
   uint64_t kv_bytes;      // one K (or V) region
   uint64_t kv_stride;     // kv_bytes rounded to 256
-  uint64_t sc_bytes;      // one scale region (0 for 16-bit caches)
+  uint64_t sc_bytes;      // the V-scale region (0 for 16-bit caches)
   uint64_t sc_stride;
+  uint64_t ksc_stride;    // the K-scale region (per-token rows, or channel scales)
   uint64_t layer_stride;  // K + V (+ K scale + V scale), each 256-aligned
   uint64_t status_off;    // 256-byte status region after the last layer
   uint64_t total;
@@ -99,7 +103,7 @@ inline float *layer_ks(const kv_pool *p, int layer) {
   return p->lay.sc_bytes ? (float *)(layer_v(p, layer) + p->lay.kv_stride) : nullptr;
 }
 inline float *layer_vs(const kv_pool *p, int layer) {
-  return p->lay.sc_bytes ? (float *)((char *)layer_ks(p, layer) + p->lay.sc_stride)
+  return p->lay.sc_bytes ? (float *)((char *)layer_ks(p, layer) + p->lay.ksc_stride)
                          : nullptr;
 }
 inline int32_t *status_word(const kv_pool *p) {

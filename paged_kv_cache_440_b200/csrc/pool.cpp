@@ -60,8 +60,9 @@ bool compute_layout(const kv_pool_desc &d, Layout *out, std::string *why,
     *why = "head_dim must be 64 or 128";
     return false;
   }
-  if (d.cache_dtype < KV_BF16 || d.cache_dtype > KV_INT4) {
-    *why = "cache_dtype must be KV_BF16, KV_FP16, KV_FP8_E5M2, KV_INT8, KV_FP8_E5M2_CAST or KV_INT4";
+  if (d.cache_dtype < KV_BF16 || d.cache_dtype > KV_INT8_KCHAN) {
+    *why = "cache_dtype must be KV_BF16, KV_FP16, KV_FP8_E5M2, KV_INT8, KV_FP8_E5M2_CAST, KV_INT4 "
+           "or KV_INT8_KCHAN";
     return false;
   }
   if (d.cache_dtype == KV_INT4 && d.head_dim != 128) {
@@ -79,7 +80,11 @@ bool compute_layout(const kv_pool_desc &d, Layout *out, std::string *why,
   L.kv_stride = round_up(L.kv_bytes, 256);
   L.sc_bytes = has_scales(d.cache_dtype) ? rows * sizeof(float) : 0;
   L.sc_stride = round_up(L.sc_bytes, 256);
-  L.layer_stride = 2 * L.kv_stride + 2 * L.sc_stride;
+  // K scales: per-token rows like V, or the layer's [heads][head_dim] channel scales
+  L.ksc_stride = k_chan_scales(d.cache_dtype)
+                     ? round_up((uint64_t)d.num_kv_heads * d.head_dim * sizeof(float), 256)
+                     : L.sc_stride;
+  L.layer_stride = 2 * L.kv_stride + L.ksc_stride + L.sc_stride;
   L.status_off = L.layer_stride * (uint64_t)d.num_layers;
   L.total = L.status_off + 256;
   *out = L;

@@ -54,6 +54,8 @@ def build_pool(pkv, wl, device, chunk=65536):
         for t in (K, V, KS, VS):
             if t is not None:                     # the scale-less cast has no scales
                 t.zero_()
+        if wl.cache_dtype == "int8_kchan":        # the layer's key channel scales
+            KS.copy_(torch.from_numpy(wl.k_chan).to(device))
         slots = torch.from_numpy(wl.slot_hist).to(device)
         for s in range(0, wl.k_hist.shape[0], chunk):
             pkv.kv_append(pool, 0, wl.k_hist[s:s + chunk].contiguous(),
@@ -89,21 +91,27 @@ def oracle_cache_quant(wl, seqs):
     sampled sequences' blocks, with block tables renumbered to match (the
     result does not depend on physical placement).
     """
+    kchan = wl.cache_dtype == "int8_kchan"
     row = wl.head_dim // 2 if wl.cache_dtype == "int4" else wl.head_dim
     shape = (wl.num_blocks, wl.kv_heads, wl.block_size, row)
-    cdt = np.int8 if wl.cache_dtype == "int8" else np.uint8
+    cdt = np.int8 if wl.cache_dtype in ("int8", "int8_kchan") else np.uint8
     kc, vc = np.zeros(shape, cdt), np.zeros(shape, cdt)
     ks, vs = np.zeros(shape[:3], np.float32), np.zeros(shape[:3], np.float32)
+    if kchan:
+        ks = wl.k_chan
+
+    def put(k, v, slots):
+        if kchan:
+            cache_ops.append_quantized_kchan(kc, vc, vs, k, v, slots, wl.block_size, wl.k_chan)
+        else:
+            cache_ops.append_quantized(kc, vc, ks, vs, k, v, slots, wl.block_size,
+                                       wl.cache_dtype)
     starts = np.concatenate([[0], np.cumsum(np.maximum(wl.context_lens - 1, 0))])
     used = []
     for b in seqs:
         lo, hi = int(starts[b]), int(starts[b + 1])
-        cache_ops.append_quantized(kc, vc, ks, vs, to_np(wl.k_hist[lo:hi]),
-                                   to_np(wl.v_hist[lo:hi]), wl.slot_hist[lo:hi],
-                                   wl.block_size, wl.cache_dtype)
-        cache_ops.append_quantized(kc, vc, ks, vs, to_np(wl.k_new[b:b + 1]),
-                                   to_np(wl.v_new[b:b + 1]), wl.slot_new[b:b + 1],
-                                   wl.block_size, wl.cache_dtype)
+        put(to_np(wl.k_hist[lo:hi]), to_np(wl.v_hist[lo:hi]), wl.slot_hist[lo:hi])
+        put(to_np(wl.k_new[b:b + 1]), to_np(wl.v_new[b:b + 1]), wl.slot_new[b:b + 1])
         nblk = -(-int(wl.context_lens[b]) // wl.block_size)
         used += wl.block_tables[b, :nblk].tolist()
     used = sorted(set(used)) or [0]
@@ -114,8 +122,13 @@ def oracle_cache_quant(wl, seqs):
         tables[b, :nblk] = [remap[x] for x in wl.block_tables[b, :nblk]]
     u = np.array(used)
     unpack = quant.unpack_int4 if wl.cache_dtype == "int4" else (lambda c: c)
-    kd = quant.dequantize(unpack(kc[u]), ks[u], wl.cache_dtype)
-    vd = quant.dequantize(unpack(vc[u]), vs[u], wl.cache_dtype)
+    if kchan:
+        kd = quant.dequantize_k_channels(kc[u].transpose(0, 2, 1, 3), wl.k_chan) \
+            .transpose(0, 2, 1, 3)                           # [U, bs, H, D] against [H, D]
+        vd = quant.dequantize(vc[u], vs[u], "int8")
+    else:
+        kd = quant.dequantize(unpack(kc[u]), ks[u], wl.cache_dtype)
+        vd = quant.dequantize(unpack(vc[u]), vs[u], wl.cache_dtype)
     return (kc, vc, ks, vs), (kd, vd, tables)
 
 

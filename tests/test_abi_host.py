@@ -269,3 +269,23 @@ def test_int4_layout_and_head_dim():
     d = B.PoolDesc(1, 8, 16, 2, 64, B.DTYPE_CODES["int4"])
     n = ctypes.c_uint64()
     assert B.lib.kv_pool_required_bytes(ctypes.byref(d), ctypes.byref(n)) == B.KV_ERR_UNSUPPORTED
+
+
+def test_kchan_layout_channel_scales_per_layer():
+    """INT8 keys with channel scales: 1-byte K and V rows, a [kv_heads][head_dim]
+    fp32 K-scale array per layer and per-token-head V scales."""
+    NB, layers, bs, hkv, D = 37, 2, 16, 8, 128
+    h, total = _make_pool(NB, layers, bs, hkv, D, "int8_kchan")
+    try:
+        tokens = NB * bs
+        kv = ref_pool.kv_cache_bytes(1, hkv, D, 1, tokens)
+        k, v, ks, vs = _ptrs(h, 0)
+        k1, _, _, _ = _ptrs(h, 1)
+        assert v - k >= kv // 2 and ks - v >= kv // 2
+        assert vs - ks == -(-hkv * D * 4 // 256) * 256          # channel scales, 256-aligned
+        assert k1 - vs >= tokens * hkv * 4                       # then per-token V scales
+        exact = ref_pool.kv_cache_bytes(layers, hkv, D, 1, tokens) + \
+            layers * (hkv * D * 4 + tokens * hkv * 4)
+        assert exact + 256 <= total <= exact + 256 + layers * 4 * 255
+    finally:
+        B.lib.kv_pool_destroy(h)

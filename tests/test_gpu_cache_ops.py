@@ -92,9 +92,10 @@ def test_quantize_bit_exact(pkv, kind, in_dt, D):
     assert np.array_equal(codes.cpu().numpy(), ref_codes)
 
 
-@pytest.mark.parametrize("cache", ["bf16", "int8", "e5m2", "e5m2_cast", "int4"])
+@pytest.mark.parametrize("cache", ["bf16", "int8", "e5m2", "e5m2_cast", "int4", "int8_kchan"])
 def test_block_copy_bit_exact(pkv, cache):
-    """Shared-prefix shapes: 200 copy-on-write pairs, 3 layers, random pool bytes."""
+    """Shared-prefix shapes: 200 copy-on-write pairs, 3 layers, random pool bytes.
+    Per-channel key scales belong to the layer, not to a block: left as they are."""
     layers, NB, bs, hkv, D = 3, 1500, 16, 8, 128
     pool = pkv.KVPool(layers, NB, bs, hkv, D, cache, DEV)
     g = torch.Generator(device=DEV).manual_seed(7)
@@ -107,11 +108,16 @@ def test_block_copy_bit_exact(pkv, cache):
     pairs = list(zip(ids[:200].tolist(), ids[200:].tolist()))
     pkv.kv_block_copy(pool, pairs)
     torch.cuda.synchronize()
-    regions = [a for lay in before for a in lay if a is not None]
+    per_block = [i for i in range(4) if not (cache == "int8_kchan" and i == 2)]
+    regions = [lay[i] for lay in before for i in per_block if lay[i] is not None]
     cache_ops.block_copy(regions, pairs)
-    after = [raw_bytes(t) for l in range(layers) for t in pool.layer_views(l) if t is not None]
+    views = [pool.layer_views(l) for l in range(layers)]
+    after = [raw_bytes(v[i]) for v in views for i in per_block if v[i] is not None]
     for a, r in zip(after, regions):
         assert np.array_equal(a, r)
+    if cache == "int8_kchan":
+        for l in range(layers):
+            assert np.array_equal(raw_bytes(views[l][2]), before[l][2])
 
 
 def test_bounded_wait_gives_up_and_reports(pkv):
@@ -148,3 +154,39 @@ def test_append_scale_less_e5m2_bit_exact(pkv, in_dt):
                                "e5m2_cast")
     assert np.array_equal(K.cpu().numpy(), kc)
     assert np.array_equal(V.cpu().numpy(), vc)
+
+
+@pytest.mark.parametrize("in_dt", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("D,bs", [(64, 16), (128, 32)])
+def test_append_kchan_bit_exact(pkv, in_dt, D, bs):
+    """INT8 keys with the layer's channel scales (one zero-scale channel, some
+    scales small enough to saturate), INT8 values per row: codes and value
+    scales bit-exact with the oracle; the channel scales stay as written."""
+    NB, hkv, T = 40, 4, 300
+    pool = pkv.KVPool(1, NB, bs, hkv, D, "int8_kchan", DEV)
+    K, V, KS, VS = pool.layer_views(0)
+    for t in (K, V, VS):
+        t.zero_()
+    rng = np.random.default_rng(D + bs)
+    sigma = rng.uniform(0.25, 4.0, (hkv, D)).astype(np.float32)
+    chan = (sigma * 4.0 / 127.0).astype(np.float32)
+    chan[1, 3] = 0.0                                    # a dropped channel
+    chan[2, :8] = np.float32(1e-4)                      # saturates
+    KS.copy_(torch.from_numpy(chan).to(DEV))
+    g = torch.Generator(device=DEV).manual_seed(D * bs)
+    k = (torch.randn(T, hkv, D, generator=g, device=DEV) * torch.from_numpy(sigma).to(DEV)).to(in_dt)
+    v = (torch.randn(T, hkv, D, generator=g, device=DEV) * 3).to(in_dt)
+    slots = rng.permutation(NB * bs)[:T].astype(np.int64)
+    slots[7] = -1                                       # padding token: skipped
+    pkv.kv_append(pool, 0, k, v, torch.from_numpy(slots).to(DEV))
+    torch.cuda.synchronize()
+    assert pool.status() == 0
+    kc = np.zeros((NB, hkv, bs, D), np.int8)
+    vc = np.zeros((NB, hkv, bs, D), np.int8)
+    vs = np.zeros((NB, hkv, bs), np.float32)
+    cache_ops.append_quantized_kchan(kc, vc, vs, to_np(k), to_np(v), slots, bs, chan)
+    assert np.array_equal(K.cpu().numpy(), kc)
+    assert np.array_equal(V.cpu().numpy(), vc)
+    assert np.array_equal(VS.cpu().numpy().view(np.uint32), vs.view(np.uint32))
+    assert np.array_equal(KS.cpu().numpy(), chan)
+    assert (np.abs(kc[..., 2, :, :8]) == 127).any()     # the saturating channels did saturate

@@ -70,7 +70,7 @@ def test_mha13b_every_output(pkv):
     _run_16(pkv, W.mha13b(DEV))
 
 
-@pytest.mark.parametrize("kind", ["int8", "e5m2", "int4"])
+@pytest.mark.parametrize("kind", ["int8", "e5m2", "int4", "int8_kchan"])
 @pytest.mark.parametrize("variant,seqs", [("a", [0, 13, 40, 63]), ("b", [0, 5])])
 def test_quantized_long_context(pkv, kind, variant, seqs):
     """INT8 / E5M2 per-token-head KV, bs 32, (a) 64 x 4096 and (b) 8 x 32768.
@@ -89,8 +89,11 @@ def test_quantized_long_context(pkv, kind, variant, seqs):
         idn = wl.block_tables[b, :nblk]
         assert np.array_equal(K[ids].cpu().numpy(), kc[idn]), "K codes, seq %d" % b
         assert np.array_equal(V[ids].cpu().numpy(), vc[idn]), "V codes, seq %d" % b
-        assert np.array_equal(KS[ids].cpu().numpy().view(np.uint32), ks[idn].view(np.uint32))
+        if kind != "int8_kchan":                 # channel scales: the layer's, checked below
+            assert np.array_equal(KS[ids].cpu().numpy().view(np.uint32), ks[idn].view(np.uint32))
         assert np.array_equal(VS[ids].cpu().numpy().view(np.uint32), vs[idn].view(np.uint32))
+    if kind == "int8_kchan":
+        assert np.array_equal(KS.cpu().numpy(), wl.k_chan)
     pairs = _all_pairs(wl, seqs)
     ref = oracle_outputs(wl, kd, vd, pairs, otab)
     compare(torch.stack([out[b, h] for b, h in pairs]), ref, what=wl.name)
@@ -190,7 +193,8 @@ def test_shared_prefix_copy_on_write(pkv):
 EDGE_LENS = [0, 1, 15, 16, 17, 63, 64, 65, 127, 128, 129, 300]
 
 
-@pytest.mark.parametrize("cache", ["bf16", "fp16", "int8", "e5m2", "e5m2_cast", "int4"])
+@pytest.mark.parametrize("cache", ["bf16", "fp16", "int8", "e5m2", "e5m2_cast", "int4",
+                                   "int8_kchan"])
 @pytest.mark.parametrize("G", [1, 2, 4, 8, 16])
 @pytest.mark.parametrize("D,bs", [(64, 16), (128, 32)])
 def test_edge_lengths_groups_dims(pkv, cache, G, D, bs):
@@ -271,6 +275,11 @@ def _fused_workloads():
                                                      [3, 32, 33, 200], seed=8, device=DEV)),
         ("int4", lambda: W.make_decode_workload("i4", 5, 16, 2, 128, 16, "bf16", "int4",
                                                 [1, 15, 16, 17, 300], seed=9, device=DEV)),
+        ("int8-kchan", lambda: W.make_decode_workload("kc", 4, 16, 2, 128, 32, "bf16", "int8_kchan",
+                                                      [1, 31, 32, 300], seed=10, device=DEV)),
+        ("int8-kchan-d64", lambda: W.make_decode_workload("kc64", 4, 8, 2, 64, 16, "fp16",
+                                                          "int8_kchan", [2, 16, 17, 129],
+                                                          seed=11, device=DEV)),
     ]
 
 
@@ -301,7 +310,10 @@ def test_fused_append_matches_oracle(pkv, name, make, num_ctas):
                        for x in wl.block_tables[b, :-(-int(wl.context_lens[b]) // wl.block_size)]})
         assert np.array_equal(K[used].cpu().numpy(), kc[used])
         assert np.array_equal(V[used].cpu().numpy(), vc[used])
-        if KS is not None:                       # the scale-less cast keeps no scales
+        if wl.cache_dtype == "int8_kchan":      # layer channel scales, per-token V scales
+            assert np.array_equal(KS.cpu().numpy(), wl.k_chan)
+            assert np.array_equal(VS[used].cpu().numpy().view(np.uint32), vs[used].view(np.uint32))
+        elif KS is not None:                     # the scale-less cast keeps no scales
             assert np.array_equal(KS[used].cpu().numpy().view(np.uint32), ks[used].view(np.uint32))
             assert np.array_equal(VS[used].cpu().numpy().view(np.uint32), vs[used].view(np.uint32))
     ref = oracle_outputs(wl, k, v, pairs, tab)

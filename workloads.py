@@ -48,6 +48,8 @@ class DecodeWorkload:
     k_hist: Optional[torch.Tensor] = None
     v_hist: Optional[torch.Tensor] = None
     slot_hist: Optional[np.ndarray] = None
+    # "int8_kchan" caches: the layer's fixed key channel scales, float32 [Hkv, D]
+    k_chan: Optional[np.ndarray] = None
     extra: dict = field(default_factory=dict)
 
     @property
@@ -143,6 +145,15 @@ def make_decode_workload(name, batch, q_heads, kv_heads, head_dim, block_size,
         wl.slot_hist = slots
     wl.k_new = randn(batch, kv_heads, head_dim)
     wl.v_new = randn(batch, kv_heads, head_dim)
+    if cache_dtype == "int8_kchan":
+        # keys whose channels differ in spread (sigma in [0.25, 4] per head and
+        # channel), with calibrated-style channel scales 4 sigma / 127: values
+        # beyond 4 sigma saturate
+        sigma = torch.empty(kv_heads, head_dim).uniform_(0.25, 4.0, generator=gen)
+        sig_d = sigma.to(device)
+        wl.k_hist = (wl.k_hist.float() * sig_d).to(dt)
+        wl.k_new = (wl.k_new.float() * sig_d).to(dt)
+        wl.k_chan = (sigma * 4.0 / 127.0).numpy().astype(np.float32)
     wl.slot_new = np.where(lens > 0, _slots(tables, lens, block_size,
                                             [max(int(n) - 1, 0) for n in lens]), -1)
     return wl
@@ -188,7 +199,8 @@ def mha13b(device="cpu", seed=0, batch=32, ctx=2048):
 
 def quant_long(kind, variant="a", device="cpu", seed=0):
     """Quantized KV: 64 q / 8 kv heads, D 128, bs 32, bf16 q; (a) 64 x 4096,
-    (b) 8 x 32768 tokens; K/V ~ N(0,1) stored as INT8 or FP8-E5M2."""
+    (b) 8 x 32768 tokens; K/V ~ N(0,1) stored as INT8 or FP8-E5M2 (and the
+    other 1-byte and 4-bit kinds; "int8_kchan" keys spread per channel)."""
     batch, ctx = (64, 4096) if variant == "a" else (8, 32768)
     return make_decode_workload("quant_%s_%s" % (variant, kind), batch, 64, 8, 128,
                                 32, "bf16", kind, [ctx] * batch, seed=seed,
