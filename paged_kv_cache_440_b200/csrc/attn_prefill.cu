@@ -238,9 +238,13 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
       tmem_wait_st();
     }
   }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
+  // Q in TMEM before the first MMA: softmax and MMA warps only, so that the
+  // producers start streaming K/V while Q is still being loaded
+  if (warp != kPfProducerWarp && warp != kPfProducerWarp + 1) {
+    tc_fence_before();
+    bar_sync(2, kPfSoftmax + 32);
+    tc_fence_after();
+  }
 
   if (warp == kPfProducerWarp || warp == kPfProducerWarp + 1) {
     // ============================================================ producers
