@@ -92,6 +92,7 @@ struct AttnParams {
   int units_per_seq;   // (kv_heads / hg) * cgroups
   int stage_bytes;     // bytes between ring stages (load size rounded to 1024)
   int stages;          // ring stages (R)
+  int unit_cost;       // positions charged for starting a unit (see Walk)
   int max_blocks;      // block-table row length
   int num_blocks;      // physical blocks in the pool
   int limit;           // valid lengths: 0 < L <= min(max_context, max_blocks * bs)
@@ -812,14 +813,23 @@ struct NewRow {
   }
 };
 
-// Position of a CTA's walk over the flattened (unit, block) list.
+// Position of a CTA's walk over the flattened (unit, block) list. Each unit
+// with blocks occupies unit_cost + nb positions: unit_cost positions that
+// stand for the fixed work of starting a unit (query load, partial write),
+// then one per block. The even split of positions over CTAs thus gives a CTA
+// whose share starts a unit fewer blocks.
 struct Walk {
   int b;         // sequence
   int gc;        // unit within the sequence: kv head * chunks + chunk
   int j;         // block within the unit
   int nb;        // blocks of sequence b
-  long long pos; // flattened position of (b, gc, j)
+  long long pos; // flattened position of block j of unit (b, gc)
 };
+
+// Positions of one unit of a sequence with nb blocks.
+__device__ __forceinline__ int unit_len(int nb, const AttnParams &p) {
+  return nb > 0 ? nb + p.unit_cost : 0;
+}
 
 template <int BS>
 __device__ __forceinline__ void walk_advance(Walk &w, int seg, const AttnParams &p) {
@@ -827,6 +837,7 @@ __device__ __forceinline__ void walk_advance(Walk &w, int seg, const AttnParams 
   w.j += seg;
   if (w.j == w.nb) {
     w.j = 0;
+    w.pos += p.unit_cost;  // the next unit's first block
     if (++w.gc == p.units_per_seq) {
       w.gc = 0;
       do {
@@ -877,7 +888,7 @@ attn_partition_kernel(const __grid_constant__ CUtensorMap kmap,
     if (L < 0 || L > p.limit) {
       if (c == 0) atomicOr(p.status, kErrContext);
     } else {
-      part += (L + BS - 1) / BS;
+      part += unit_len((L + BS - 1) / BS, p);
     }
   }
   const long long total = block_sum(part, red) * UH;
@@ -902,10 +913,10 @@ attn_partition_kernel(const __grid_constant__ CUtensorMap kmap,
   long long run = 0;
   for (int base = 0; base < B; base += kThreads) {
     const int b = base + threadIdx.x;
-    const int nb = b < B ? seq_blocks<BS>(p, b) : 0;
+    const int ln = b < B ? unit_len(seq_blocks<BS>(p, b), p) : 0;
     long long tot;
-    const long long excl = run + block_excl_scan(nb, red, &tot);
-    if (nb > 0 && excl * UH <= s0 && s0 < (excl + nb) * UH) {
+    const long long excl = run + block_excl_scan(ln, red, &tot);
+    if (ln > 0 && excl * UH <= s0 && s0 < (excl + ln) * UH) {
       s_loc[0] = b;
       s_loc[1] = excl;
     }
@@ -921,11 +932,15 @@ attn_partition_kernel(const __grid_constant__ CUtensorMap kmap,
   w0.b = static_cast<int>(s_loc[0]);
   w0.nb = seq_blocks<BS>(p, w0.b);
   {
+    // s0 may fall on the unit's start positions: the walk then begins at its
+    // first block (possibly past s1: nothing to do here)
+    const int ln = unit_len(w0.nb, p);
     const long long off = s0 - s_loc[1] * UH;
-    w0.gc = static_cast<int>(off / w0.nb);
-    w0.j = static_cast<int>(off - static_cast<long long>(w0.gc) * w0.nb);
+    w0.gc = static_cast<int>(off / ln);
+    const int jv = static_cast<int>(off - static_cast<long long>(w0.gc) * ln) - p.unit_cost;
+    w0.j = jv > 0 ? jv : 0;
+    w0.pos = s0 + (jv < 0 ? -jv : 0);
   }
-  w0.pos = s0;
 
   if (warp == kNC) {
     // ============================================================ producer
@@ -986,6 +1001,7 @@ attn_partition_kernel(const __grid_constant__ CUtensorMap kmap,
   Walk w = w0;
   uint32_t k = 0;
   bool alive = true;
+  int side = 0;  // the CTA's first piece goes to side 0, the others to side 1
   while (w.pos < s1) {
     if (w.b >= B || w.nb <= 0) {  // same test as the producer: both stop here
       if (warp == 0 && lane == 0) atomicOr(p.status, kErrContext);
@@ -1044,7 +1060,6 @@ attn_partition_kernel(const __grid_constant__ CUtensorMap kmap,
     }
     // ------------------------------------------ end of the unit's piece here
     const bool whole = (w.j == 0 && seg == w.nb);
-    const int side = (w.pos == s0) ? 0 : 1;
     if (active) {
       const int64_t pbase = ((static_cast<int64_t>(c) * 2 + side) * kNC + warp) * kChunkHeads;
       cs.finish(p, whole, w.b, h0, nh, pbase, alive, lane);
@@ -1054,6 +1069,7 @@ attn_partition_kernel(const __grid_constant__ CUtensorMap kmap,
       p.meta[static_cast<int64_t>(w.b) * UH + w.gc] = make_int4(c, nu, side, 0);
     }
     k += seg;
+    side = 1;
     walk_advance<BS>(w, seg, p);
   }
 }
@@ -1327,6 +1343,9 @@ kv_status fill_params(kv_pool *pool, int layer, const void *q, int num_seqs, int
   p.units_per_seq = u.units_per_seq;
   p.stage_bytes = u.stage_bytes;
   p.stages = u.stages;
+  // starting a unit (query load, partial write) costs about as much as
+  // streaming 192 KB on one SM: charged as that many blocks in the split
+  p.unit_cost = std::max(1, std::min(8, (192 * 1024 + u.stage_bytes / 2) / u.stage_bytes));
   p.max_blocks = max_blocks_per_seq;
   p.num_blocks = pool->d.num_blocks;
   const int64_t tbl_cap = static_cast<int64_t>(max_blocks_per_seq) * pool->d.block_size;
