@@ -289,3 +289,40 @@ def test_kchan_layout_channel_scales_per_layer():
         assert exact + 256 <= total <= exact + 256 + layers * 4 * 255
     finally:
         B.lib.kv_pool_destroy(h)
+
+
+def test_prefill_argument_validation():
+    """paged_attn_prefill rejects bad arguments before any device work; on a
+    host without a GPU a well-formed call fails loudly (KV_ERR_CUDA)."""
+    import torch
+    h, _ = _make_pool(64, 1, 16, 2, 64, "bf16")
+    hq, _ = _make_pool(64, 1, 16, 2, 64, "int8_kchan")
+    try:
+        fake = ctypes.c_void_p(FAKE_BASE)
+        nul = ctypes.c_void_p(0)
+
+        def call(pool=h, layer=0, q=fake, qdt=0, B_=2, Hq=8, total=10, maxq=5, mb=16, mc=64,
+                 scale=0.125, out=fake, cu=fake, tab=fake, lens=fake):
+            return B.lib.paged_attn_prefill(pool, layer, q, qdt, B_, Hq, cu, total, maxq, tab, mb,
+                                            lens, mc, scale, out, None)
+
+        assert call(layer=1) == B.KV_ERR_INVALID                     # layer out of range
+        assert call(pool=hq) == B.KV_ERR_UNSUPPORTED                 # 1-byte caches
+        assert call(qdt=1) == B.KV_ERR_UNSUPPORTED                   # q dtype != cache dtype
+        assert call(Hq=7) == B.KV_ERR_INVALID                        # not a multiple of Hkv
+        assert call(Hq=2 * 129) == B.KV_ERR_UNSUPPORTED              # > 128 heads per kv head
+        assert call(total=-1) == B.KV_ERR_INVALID
+        assert call(mb=0) == B.KV_ERR_INVALID
+        assert call(scale=float("inf")) == B.KV_ERR_INVALID
+        assert call(B_=0) == B.KV_OK                                 # nothing to do
+        assert call(q=nul) == B.KV_ERR_INVALID
+        assert call(q=ctypes.c_void_p(FAKE_BASE + 8)) == B.KV_ERR_INVALID   # misaligned
+        assert call(B_=65536) == B.KV_ERR_UNSUPPORTED
+        if not torch.cuda.is_available():
+            assert call() == B.KV_ERR_CUDA
+        # the per-channel key kind has no standalone per-row quantizer
+        assert B.lib.kv_quantize(fake, 0, 4, 64, B.KV_INT8_KCHAN, fake, fake, None) == \
+            B.KV_ERR_UNSUPPORTED
+    finally:
+        B.lib.kv_pool_destroy(h)
+        B.lib.kv_pool_destroy(hq)
