@@ -588,14 +588,87 @@ def run_ours(args, rank, world, device):
     return res
 
 
+CACHE_OPS = ("Cache ops of a LLaMA-70B-shaped layer (8 kv heads, head_dim 128, block 16): bf16 "
+             "append of one decode step (32 tokens) and of a 4096-token chunk, INT8 append of the "
+             "chunk, INT8 quantize of 32768 rows, copy-on-write copy of 200 blocks (K and V)")
+
+
+def cache_ops_main(args, device):
+    """Time kv_append, kv_quantize and kv_block_copy alone (CUDA events around
+    each launch, L2 flushed before each) and report their algorithmic GB/s."""
+    import paged_kv_cache_440_b200 as pkv
+    g = torch.Generator(device=device).manual_seed(0)
+    NB, bs, H, D, T = 5504, 16, 8, 128, 4096
+    pool = pkv.KVPool(1, NB, bs, H, D, "bf16", device)
+    qpool = pkv.KVPool(1, NB, bs, H, D, "int8", device)
+    for t in pool.layer_views(0) + qpool.layer_views(0):
+        if t is not None:
+            t.zero_()
+    k = torch.randn(T, H, D, generator=g, device=device).to(torch.bfloat16)
+    v = torch.randn(T, H, D, generator=g, device=device).to(torch.bfloat16)
+    perm = torch.randperm(NB * bs, generator=g, device=device)
+    slots = perm[:T].to(torch.int64).contiguous()
+    x = torch.randn(T * H, D, generator=g, device=device).to(torch.bfloat16)
+    codes = torch.empty(T * H, D, dtype=torch.int8, device=device)
+    scales = torch.empty(T * H, dtype=torch.float32, device=device)
+    ids = torch.randperm(NB, generator=torch.Generator().manual_seed(1))[:400].tolist()
+    pairs = list(zip(ids[:200], ids[200:]))
+    flush = torch.ones(64 << 20, dtype=torch.float32, device=device)   # 256 MiB
+    sink = torch.empty((), dtype=torch.float32, device=device)
+    row = H * D * 2
+    ops = [
+        ("append_step_bf16", lambda: pkv.kv_append(pool, 0, k[:32], v[:32], slots[:32]),
+         32 * (4 * row + 8)),
+        ("append_chunk_bf16", lambda: pkv.kv_append(pool, 0, k, v, slots), T * (4 * row + 8)),
+        ("append_chunk_int8", lambda: pkv.kv_append(qpool, 0, k, v, slots),
+         T * (2 * row + 2 * H * D + 2 * H * 4 + 8)),
+        ("quantize_int8", lambda: pkv.kv_quantize(x, "int8", codes=codes, scales=scales),
+         T * H * (D * 2 + D + 4)),
+        ("block_copy_200", lambda: pkv.kv_block_copy(pool, pairs), 200 * 2 * 2 * H * bs * D * 2),
+    ]
+    steps = max(1, min(args.steps, 200))
+    peak, peak_kind = measured_peak()
+    parts = {}
+    for name, fn, nbytes in ops:
+        for _ in range(args.warmup):
+            torch.sum(flush, 0, out=sink)
+            fn()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        for a, b_ in evs:
+            torch.sum(flush, 0, out=sink)
+            a.record()
+            fn()
+            b_.record()
+        torch.cuda.synchronize()
+        sec = sum(a.elapsed_time(b_) for a, b_ in evs) / steps / 1e3
+        parts[name] = {"us": round(sec * 1e6, 2), "bytes": int(nbytes),
+                       "GB/s": round(nbytes / sec / 1e9, 1),
+                       "frac": round(nbytes / sec / 1e9 / peak, 4)}
+    big = parts["append_chunk_bf16"]
+    print(json.dumps({
+        "metric": "KV cache ops GB/s (append, quantize, copy-on-write copy)",
+        "value": big["GB/s"], "unit": "GB/s", "n_gpus": 1, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": round(big["us"] / 1e3, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": CACHE_OPS, "l2": "L2 flushed before each launch by reading 256 MiB"},
+        "roofline": {"bound": "hbm", "achieved": big["GB/s"], "peak": peak, "unit": "GB/s",
+                     "frac": big["frac"], "traffic": None, "kernel": "append16_kernel",
+                     "peak_source": peak_kind},
+        "parts": parts, "gpu_launches": steps * len(ops), "device_status": pool.status()}),
+        flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(PREFILL_WORKLOADS),
-                    default="gqa70b")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(PREFILL_WORKLOADS) +
+                    ["cache_ops"], default="gqa70b")
     ap.add_argument("--ctas", type=int, default=0, help="CTAs of the attention kernel (0 = one per SM)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--separate-append", action="store_true",
@@ -659,6 +732,13 @@ def main():
 
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
+    if args.workload == "cache_ops":
+        if rank == 0:
+            cache_ops_main(args, device)
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+        return
     if args.workload in PREFILL_WORKLOADS:
         prefill_main(args, rank, world, device)
         if world > 1:
