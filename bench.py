@@ -130,7 +130,7 @@ class ClockSampler:
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
                0x100: "display_clock_setting"}
 
-    def __init__(self, index, period=0.01):
+    def __init__(self, index, period=0.002):
         self.index, self.period = index, period
         self.samples = []
         self.ok = False
@@ -186,37 +186,173 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(s)}
 
 
+def hold_gpu(seconds):
+    """Queue a GPU spin of about `seconds` so that the host can enqueue every
+    timed step while the GPU is busy: the device-timed region then holds no
+    gaps where the GPU waits for the host to launch the next kernel."""
+    torch.cuda._sleep(int(max(seconds, 1e-4) * 2.0e9))   # cycles at ~2 GHz
+
+
 # ------------------------------------------------------------------ oracle arm
 
-def oracle_sample(wl, budget_s=15.0):
-    """Time the fp64 CPU oracle (as it stands) on a bounded sample of the step:
-    the append and decode of whole sequences, taken in order until ~budget_s of
-    CPU work. Returns (GB/s in the metric's bytes, seconds, sequences, threads)."""
-    from threadpoolctl import threadpool_info
-    from oracle import attention, cache_ops
-    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    dt = np.float16 if wl.cache_dtype == "fp16" else np.float32
-    if wl.k_fill is None:
-        raise SystemExit("the CPU baseline covers 16-bit caches only")
-    kc = wl.k_fill.float().cpu().numpy().astype(dt)
-    vc = wl.v_fill.float().cpu().numpy().astype(dt)
-    kn = wl.k_new.float().cpu().numpy().astype(dt)
-    vn = wl.v_new.float().cpu().numpy().astype(dt)
-    q = wl.q.float().cpu().numpy().astype(np.float64)
-    e = elt_bytes(wl.cache_dtype)
-    done, nbytes, t_total = 0, 0, 0.0
-    for b in range(wl.batch):
-        t0 = time.perf_counter()
-        cache_ops.append(kc, vc, kn[b:b + 1], vn[b:b + 1], wl.slot_new[b:b + 1], wl.block_size)
+def _host_f32(t):
+    """Exact float32 host copy of a bf16 / fp16 tensor (through its bits)."""
+    u = t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    if t.dtype == torch.bfloat16:
+        return (u.astype(np.uint32) << 16).view(np.float32)
+    return u.view(np.float16).astype(np.float32)
+
+
+class OracleStep:
+    """The fp64 CPU oracle, as it stands, on one sequence of the workload at a
+    time: that sequence's append (quantized for a 1-byte or 4-bit cache) and its
+    decode attention for every query head. Quantized caches hold the oracle's
+    own codes of the whole history, made once before timing; the shared-prompt
+    workload holds the oracle's own copy-on-write cache. For a quantized cache a
+    sequence's history is quantized into it by prepare(b), outside the timing,
+    just before the sequence is first timed."""
+
+    def __init__(self, wl):
+        from oracle import cache_ops, quant
+        self.wl = wl
+        self.q = _host_f32(wl.q).astype(np.float64)
+        kind = wl.cache_dtype
+        self.kind = kind
+        if getattr(wl, "sp", None) is not None:          # shared prompt
+            self._init_shared(wl)
+        elif kind in ("bf16", "fp16"):
+            dt = np.float16 if kind == "fp16" else np.float32
+            self.kc, self.vc = _host_f32(wl.k_fill).astype(dt), _host_f32(wl.v_fill).astype(dt)
+            self.kn, self.vn = _host_f32(wl.k_new).astype(dt), _host_f32(wl.v_new).astype(dt)
+            self.tables = wl.block_tables
+        else:
+            H, bs, D = wl.kv_heads, wl.block_size, wl.head_dim
+            row = D // 2 if kind == "int4" else D
+            shape = (wl.num_blocks, H, bs, row)
+            cdt = np.int8 if kind in ("int8", "int8_kchan") else np.uint8
+            self.kc, self.vc = np.zeros(shape, cdt), np.zeros(shape, cdt)
+            self.ks = np.zeros(shape[:3], np.float32) if kind != "int8_kchan" else wl.k_chan
+            self.vs = np.zeros(shape[:3], np.float32)
+            self.kh, self.vh = _host_f32(wl.k_hist), _host_f32(wl.v_hist)
+            self.starts = np.concatenate([[0], np.cumsum(np.maximum(wl.context_lens - 1, 0))])
+            self.kn, self.vn = _host_f32(wl.k_new), _host_f32(wl.v_new)
+            self.tables = wl.block_tables
+        self.ready = set()
+
+    def prepare(self, b):
+        """Untimed: sequence b's cached history in the oracle's cache."""
+        from oracle import cache_ops
+        wl, kind = self.wl, self.kind
+        if b in self.ready or kind in ("bf16", "fp16") or getattr(wl, "sp", None) is not None:
+            return
+        sl = slice(int(self.starts[b]), int(self.starts[b + 1]))
+        if kind == "int8_kchan":
+            cache_ops.append_quantized_kchan(self.kc, self.vc, self.vs, self.kh[sl], self.vh[sl],
+                                             wl.slot_hist[sl], wl.block_size, wl.k_chan)
+        else:
+            cache_ops.append_quantized(self.kc, self.vc, self.ks, self.vs, self.kh[sl],
+                                       self.vh[sl], wl.slot_hist[sl], wl.block_size, kind)
+        self.ready.add(b)
+
+    def _init_shared(self, wl):
+        from oracle import allocator, cache_ops
+        sp = wl.sp
+        bs, H, D, P = sp.block_size, sp.kv_heads, sp.head_dim, sp.prefix_len
+        m = allocator.PoolModel(sp.num_blocks)
+        kc = np.zeros((sp.num_blocks, H, bs, D), np.float32)
+        vc = np.zeros_like(kc)
+        pre = m.alloc(-(-P // bs))
+        cache_ops.append(kc, vc, _host_f32(sp.prefix_k), _host_f32(sp.prefix_v),
+                         np.array([pre[t // bs] * bs + t % bs for t in range(P)]), bs)
+        sk, sv = _host_f32(sp.suffix_k), _host_f32(sp.suffix_v)
+        tables, off = [], 0
+        rows, slots = [], []
+        for b in range(sp.batch):
+            t = list(pre)
+            fresh = m.alloc(1)[0]
+            cache_ops.block_copy([kc, vc], [(t[-1], fresh)])
+            t[-1] = fresh
+            L = P + int(sp.suffix_lens[b])
+            t += m.alloc(-(-L // bs) - len(t))
+            for p_ in range(P, L - 1):                    # the history; the last is the step's
+                rows.append(off + p_ - P)
+                slots.append(t[p_ // bs] * bs + p_ % bs)
+            off += int(sp.suffix_lens[b])
+            tables.append(t)
+        cache_ops.append(kc, vc, sk[rows], sv[rows], np.array(slots), bs)
+        mb = max(len(t) for t in tables)
+        self.tables = np.full((sp.batch, mb), -1, np.int64)
+        for b, t in enumerate(tables):
+            self.tables[b, :len(t)] = t
+        self.kc, self.vc = kc, vc
+        self.kn, self.vn = _host_f32(wl.k_new), _host_f32(wl.v_new)
+        L = wl.context_lens
+        self.slot_new = np.array([tables[b][(L[b] - 1) // bs] * bs + (L[b] - 1) % bs
+                                  for b in range(sp.batch)], np.int64)
+
+    def run(self, b):
+        """Append and decode of sequence b; returns the metric's bytes for it."""
+        from oracle import attention, cache_ops, quant
+        wl, kind = self.wl, self.kind
+        slot = (self.slot_new if hasattr(self, "slot_new") else wl.slot_new)[b:b + 1]
+        if kind in ("bf16", "fp16"):
+            cache_ops.append(self.kc, self.vc, self.kn[b:b + 1], self.vn[b:b + 1], slot,
+                             wl.block_size)
+            kd, vd = self.kc, self.vc
+            nblk = -(-int(wl.context_lens[b]) // wl.block_size)
+            ids = self.tables[b, :nblk]
+            tab = self.tables
+        else:
+            if kind == "int8_kchan":
+                cache_ops.append_quantized_kchan(self.kc, self.vc, self.vs, self.kn[b:b + 1],
+                                                 self.vn[b:b + 1], slot, wl.block_size, wl.k_chan)
+            else:
+                cache_ops.append_quantized(self.kc, self.vc, self.ks, self.vs, self.kn[b:b + 1],
+                                           self.vn[b:b + 1], slot, wl.block_size, kind)
+            # dequantize the sequence's blocks (the oracle attends over values)
+            nblk = -(-int(wl.context_lens[b]) // wl.block_size)
+            ids = self.tables[b, :nblk]
+            unpack = quant.unpack_int4 if kind == "int4" else (lambda c: c)
+            if kind == "int8_kchan":
+                kd = quant.dequantize_k_channels(self.kc[ids].transpose(0, 2, 1, 3), wl.k_chan) \
+                    .transpose(0, 2, 1, 3)
+                vd = quant.dequantize(self.vc[ids], self.vs[ids], "int8")
+            else:
+                kd = quant.dequantize(unpack(self.kc[ids]), self.ks[ids], kind)
+                vd = quant.dequantize(unpack(self.vc[ids]), self.vs[ids], kind)
+            tab = np.full_like(self.tables, -1)
+            tab[b, :nblk] = np.arange(nblk)
         for h in range(wl.q_heads):
-            attention.decode_one(q, kc, vc, wl.block_tables, wl.context_lens, wl.scale, b, h)
-        t_total += time.perf_counter() - t0
-        done += 1
-        nbytes += int(wl.context_lens[b]) * wl.kv_heads * wl.head_dim * 2 * e \
+            attention.decode_one(self.q, kd, vd, tab, wl.context_lens, wl.scale, b, h)
+        e = elt_bytes(kind)
+        nb = int(wl.context_lens[b]) * wl.kv_heads * wl.head_dim * 2 * e \
             + 2 * wl.q_heads * wl.head_dim * 2 + wl.kv_heads * wl.head_dim * 2 * 2 * (1 + e)
-        if t_total >= budget_s:
-            break
-    return nbytes / t_total / 1e9, t_total, done, threads
+        if kind in ("int8", "e5m2", "int4", "int8_kchan"):
+            nb += int(wl.context_lens[b]) * wl.kv_heads * 8
+        return nb
+
+
+def oracle_sample(wl, budget_s=15.0, threads=None):
+    """Time the CPU oracle (as it stands) on a bounded sample of the step: the
+    append and decode of whole sequences, taken in order until ~budget_s of
+    CPU work. threads: BLAS threads for the run (None: as configured).
+    Returns (GB/s in the metric's bytes, seconds, sequences, threads used)."""
+    from threadpoolctl import threadpool_info, threadpool_limits
+    ost = OracleStep(wl)
+    with threadpool_limits(limits=threads):
+        used = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+        done, nbytes, t_total, t_setup = 0, 0, 0.0, 0.0
+        for b in range(wl.batch):
+            t0 = time.perf_counter()
+            ost.prepare(b)                         # untimed: the cache before the step
+            t1 = time.perf_counter()
+            nbytes += ost.run(b)
+            t_total += time.perf_counter() - t1
+            t_setup += t1 - t0
+            done += 1
+            if t_total >= budget_s or t_setup >= 2 * budget_s:
+                break
+    return nbytes / t_total / 1e9, t_total, done, used
 
 
 # ------------------------------------------------------------------ shared prefix
@@ -334,6 +470,7 @@ def run_prefill(args, rank, world, device):
         torch.distributed.barrier()
     torch.cuda.synchronize(device)
     t0 = time.time()
+    hold_gpu(1e-3 + 150e-6 * args.steps)
     for i in range(args.steps):
         torch.sum(flush, 0, out=sink)
         evs[i][0].record(stream)
@@ -353,6 +490,7 @@ def run_prefill(args, rank, world, device):
         for i in range(args.warmup + max(10, args.steps // 10)):
             torch.sum(flush, 0, out=sink)
             torch.cuda.synchronize(device)
+            hold_gpu(300e-6)
             a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
             d_q.copy_(h_q, non_blocking=True)
@@ -368,11 +506,16 @@ def run_prefill(args, rank, world, device):
             "status": pool.status(), "e2e": e2e, "launches": args.steps}
 
 
-def prefill_oracle_sample(pw, budget_s):
+def prefill_oracle_sample(pw, budget_s, threads=None):
     """TFLOP/s of the fp64 oracle on a bounded sample of the prefill rows."""
-    from threadpoolctl import threadpool_info
+    from threadpoolctl import threadpool_info, threadpool_limits
+    with threadpool_limits(limits=threads):
+        used = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+        return _prefill_oracle_sample(pw, budget_s) + (used,)
+
+
+def _prefill_oracle_sample(pw, budget_s):
     from oracle import attention
-    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
     wl = pw.cache
     k = wl.k_fill.float().cpu().numpy()
     v = wl.v_fill.float().cpu().numpy()
@@ -391,8 +534,8 @@ def prefill_oracle_sample(pw, budget_s):
             flops += 4 * wl.head_dim * wl.q_heads * (pos + 1)
             rows += 1
             if t >= budget_s:
-                return flops / t / 1e12, t, rows, threads
-    return flops / t / 1e12, t, rows, threads
+                return flops / t / 1e12, t, rows
+    return flops / t / 1e12, t, rows
 
 
 def prefill_main(args, rank, world, device):
@@ -409,8 +552,11 @@ def prefill_main(args, rank, world, device):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, secs, rows, threads = prefill_oracle_sample(pw, args.cpu_budget)
+        v1, secs1, rows1, _ = prefill_oracle_sample(pw, args.cpu_budget / 3, threads=1)
         cpu = {"value": round(v, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-               "sample": "%d new-token rows (all 64 heads each), %.1f s of fp64 numpy" % (rows, secs)}
+               "sample": "%d new-token rows (all 64 heads each), %.1f s of fp64 numpy" % (rows, secs),
+               "one_thread": {"value": round(v1, 6), "unit": "TFLOP/s",
+                              "sample": "%d rows, %.1f s" % (rows1, secs1)}}
     if rank == 0:
         line = {
             "metric": "chunked prefill attention TFLOP/s", "value": round(tflops, 2),
@@ -474,7 +620,7 @@ def run_ours(args, rank, world, device):
     fused = not args.separate_append and wl.group <= 8
 
     def one_step():
-        if fused:   # append folded into the attention kernel, then the merge
+        if fused:   # one kernel: append folded in, split units merged in place
             pkv.paged_attn_decode_append(pool, 0, wl.q, wl.k_new, wl.v_new, tables, lens,
                                          max_ctx, wl.scale, out=out, num_ctas=G, workspace=ws)
         else:
@@ -488,9 +634,9 @@ def run_ours(args, rank, world, device):
     torch.cuda.synchronize(device)
     pool.status_clear()
 
-    # Timed region: K steps, each bracketed by events with nothing between its
-    # kernels (so each may launch while its predecessor finishes); the L2 flush
-    # before each step is outside the events.
+    # Timed region: K steps, each bracketed by events; the L2 flush before each
+    # step is outside the events. A GPU spin queued first lets the host enqueue
+    # every step before the GPU reaches it, so no step waits on the host.
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
     sampler = ClockSampler(device.index if device.index is not None else 0).start()
@@ -498,6 +644,7 @@ def run_ours(args, rank, world, device):
         torch.distributed.barrier()
     torch.cuda.synchronize(device)
     t0 = time.time()
+    hold_gpu(1e-3 + 150e-6 * args.steps)
     for i in range(args.steps):
         flush_l2()
         evs[i][0].record(stream)
@@ -507,28 +654,27 @@ def run_ours(args, rank, world, device):
     t1 = time.time()
     if world > 1:
         torch.distributed.barrier()
-    # The attention kernel alone, same conditions (L2 flushed before each launch),
-    # for its roofline fraction.
-    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    for i in range(args.steps):
-        flush_l2()
-        kev[i][0].record(stream)
-        if fused:
-            pkv.paged_attn_partition_append(pool, 0, wl.q, wl.k_new, wl.v_new, tables, lens,
-                                            max_ctx, wl.scale, out, ws, num_ctas=G)
-        else:
-            pkv.paged_attn_partition(pool, 0, wl.q, tables, lens, max_ctx, wl.scale, out, ws,
-                                     num_ctas=G)
-        kev[i][1].record(stream)
-    torch.cuda.synchronize(device)
+    kev = None
+    if not fused:
+        # the attention kernel alone (the step also holds the append kernel),
+        # same conditions, for its roofline fraction
+        kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        hold_gpu(1e-3 + 150e-6 * args.steps)
+        for i in range(args.steps):
+            flush_l2()
+            kev[i][0].record(stream)
+            pkv.paged_attn_decode(pool, 0, wl.q, tables, lens, max_ctx, wl.scale, out=out,
+                                  num_ctas=G, workspace=ws)
+            kev[i][1].record(stream)
+        torch.cuda.synchronize(device)
     t2 = time.time()
     sampler.stop()
     status = pool.status()
     step_ms = np.array([a.elapsed_time(b) for a, b in evs])
-    part_ms = np.array([a.elapsed_time(b) for a, b in kev])
     step_s = float(step_ms.mean()) / 1e3
-    part_s = float(part_ms.mean()) / 1e3
+    # fused: the step is one launch of the attention kernel
+    part_s = step_s if kev is None else float(np.mean([a.elapsed_time(b) for a, b in kev])) / 1e3
     step_s, part_s = max_over_ranks([step_s, part_s], world, device)
     clocks = sampler.summary(t0, t2)
 
@@ -561,6 +707,7 @@ def run_ours(args, rank, world, device):
         for i in range(args.warmup + n_e2e):
             flush_l2()
             torch.cuda.synchronize(device)
+            hold_gpu(300e-6)    # the whole step is enqueued before the GPU reaches it
             a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
             d_in.copy_(h_in, non_blocking=True)
@@ -583,8 +730,8 @@ def run_ours(args, rank, world, device):
     dec_bytes, app_bytes = step_bytes(wl)
     res = {"wl": wl, "desc": desc, "G": G, "step_s": step_s, "part_s": part_s,
            "dec_bytes": dec_bytes, "app_bytes": app_bytes, "clocks": clocks, "fused": fused,
-           "status": status, "e2e": e2e, "launches": args.steps * (2 if fused else 3),
-           "wall": t1 - t0}
+           "status": status, "e2e": e2e, "launches": args.steps * (1 if fused else 2),
+           "wall": t1 - t0, "step_ms_median": float(np.median(step_ms))}
     return res
 
 
@@ -661,6 +808,73 @@ def cache_ops_main(args, device):
         flush=True)
 
 
+def reference_arm(args, world):
+    """The reference arm's JSON line: the CPU oracle timed over exactly
+    args.steps bounded steps after args.warmup untimed ones."""
+    from threadpoolctl import threadpool_info
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    if args.workload in PREFILL_WORKLOADS:
+        from oracle import attention
+        desc, make = PREFILL_WORKLOADS[args.workload]
+        pw = make("cpu")
+        wl = pw.cache
+        k, v = wl.k_fill.float().numpy(), wl.v_fill.float().numpy()
+        q = pw.q.float().numpy().astype(np.float64)
+        G = wl.q_heads // wl.kv_heads
+        rows = [(b, i) for b in range(wl.batch) for i in range(0, int(pw.chunk_lens[b]), 37)]
+
+        def one(n):
+            b, i = rows[n % len(rows)]
+            pos = int(wl.context_lens[b]) - int(pw.chunk_lens[b]) + i
+            for h in range(wl.q_heads):
+                attention.prefill_one(q[pw.cu_q[b] + i, h], k, v, wl.block_tables[b], pos,
+                                      h // G, wl.scale)
+            return 4 * wl.head_dim * wl.q_heads * (pos + 1)
+        metric, unit, what = ("chunked prefill attention TFLOP/s", "TFLOP/s",
+                              "one new-token row (all %d heads)" % wl.q_heads)
+        scale_out = 1e12
+    else:
+        desc, make = WORKLOADS[args.workload]
+        wl = make("cpu")
+        ost = OracleStep(wl)
+
+        def one(n):
+            b = n % wl.batch
+            ost.prepare(b)        # untimed below: the cache state before the step
+            return b
+        metric, unit, what = (METRIC, "GB/s",
+                              "one sequence's append and decode (all %d heads)" % wl.q_heads)
+        scale_out = 1e9
+    times, work = [], 0
+    for n in range(args.warmup + args.steps):
+        if args.workload in PREFILL_WORKLOADS:
+            t0 = time.perf_counter()
+            w = one(n)
+            dt = time.perf_counter() - t0
+        else:
+            b = one(n)
+            t0 = time.perf_counter()
+            w = ost.run(b)
+            dt = time.perf_counter() - t0
+        if n >= args.warmup:
+            times.append(dt)
+            work += w
+    secs = float(np.sum(times))
+    value = work / secs / scale_out
+    sample = "each step %s, in order; %d timed steps, %.2f s" % (what, args.steps, secs)
+    return {
+        "impl": "reference", "metric": metric, "value": round(value, 6), "unit": unit,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(secs / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": desc, "batch": wl.batch},
+        "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": threads,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -686,46 +900,12 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
 
-    if args.impl == "reference" and args.workload in PREFILL_WORKLOADS:
-        if rank == 0:
-            desc, make = PREFILL_WORKLOADS[args.workload]
-            pw = make("cpu")
-            v, secs, rows, threads = prefill_oracle_sample(pw, args.cpu_budget)
-            print(json.dumps({
-                "impl": "reference", "metric": "chunked prefill attention TFLOP/s",
-                "value": round(v, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": round(prefill_flops(pw) / (v * 1e12) * 1e3, 3),
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-                "data": "synthetic", "config": {"workload": desc, "batch": pw.cache.batch},
-                "cpu_baseline": {"value": round(v, 6), "unit": "TFLOP/s", "cores": threads,
-                                 "kind": "oracle",
-                                 "sample": "%d new-token rows, %.1f s" % (rows, secs)},
-                "e2e": {"value": round(v, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
-                        "d2h_bytes_per_step": 0}}), flush=True)
-        if world > 1:
-            torch.distributed.destroy_process_group()
-        return
-    desc, make = WORKLOADS.get(args.workload, (None, None))
     if args.impl == "reference":
+        # The oracle as it stands, on the host cores: W untimed and K timed steps,
+        # each a bounded sample of the workload (one sequence's append and decode,
+        # or one new-token row of a prefill), taken in order. Rank 0 alone.
         if rank == 0:
-            wl = make("cpu")
-            gbs, secs, nseq, threads = oracle_sample(wl, args.cpu_budget)
-            dec_bytes, app_bytes = step_bytes(wl)
-            step_s = (dec_bytes + app_bytes) / (gbs * 1e9)
-            line = {
-                "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s",
-                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-                "ms_per_step": round(step_s * 1e3, 3), "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": {"workload": desc, "batch": wl.batch},
-                "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": threads,
-                                 "kind": "oracle",
-                                 "sample": "%d of %d sequences (all %d heads each), %.1f s" %
-                                           (nseq, wl.batch, wl.q_heads, secs)},
-                "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
-                        "d2h_bytes_per_step": 0},
-            }
-            print(json.dumps(line), flush=True)
+            print(json.dumps(reference_arm(args, world)), flush=True)
         if world > 1:
             torch.distributed.destroy_process_group()
         return
@@ -762,12 +942,23 @@ def main():
             traffic = tr["bytes_per_launch"]
     except Exception:
         pass
+    bound_note = None
+    if args.workload == "shared_prefix":
+        # the shared prompt is read from L2, so logical bytes over time is no
+        # HBM fraction: the HBM figure is the DRAM bytes ncu counted per launch
+        achieved = traffic / r["part_s"] / 1e9 if traffic else None
+        bound_note = ("achieved = ncu DRAM bytes per launch / kernel time (the shared prompt is "
+                      "served from L2)" if traffic else
+                      "no DRAM capture of the current kernel source: HBM fraction not reported")
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and wl.k_fill is not None:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
         g_cpu, secs, nseq, threads = oracle_sample(wl, args.cpu_budget)
+        g_one, secs1, nseq1, _ = oracle_sample(wl, args.cpu_budget / 3, threads=1)
         cpu = {"value": round(g_cpu, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
-               "sample": "%d of %d sequences (all %d heads each), %.1f s of fp64 numpy" %
-                         (nseq, wl.batch, wl.q_heads, secs)}
+               "sample": "%d of %d sequences (append + all %d heads each), %.1f s of fp64 numpy"
+                         % (nseq, wl.batch, wl.q_heads, secs),
+               "one_thread": {"value": round(g_one, 4), "unit": "GB/s",
+                              "sample": "%d sequences, %.1f s" % (nseq1, secs1)}}
     if rank == 0:
         line = {
             "metric": METRIC, "value": round(gbs, 2), "unit": "GB/s", "n_gpus": world,
@@ -785,11 +976,14 @@ def main():
                        "bytes_per_step": r["dec_bytes"] + r["app_bytes"]},
             "pct_of_8tbs": round(100 * gbs / world / NOMINAL_HBM_GBS, 2),
             "decode_tokens_per_s": round(wl.batch * world / r["step_s"], 1),
-            "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
-                         "unit": "GB/s", "frac": round(achieved / peak, 4),
-                         "traffic": traffic,
-                         "kernel": "attn_partition_kernel" + (" (append fused)" if r.get("fused")
-                                                              else ""),
+            "roofline": {"bound": "hbm",
+                         "achieved": None if achieved is None else round(achieved, 2),
+                         "peak": peak, "unit": "GB/s",
+                         "frac": None if achieved is None else round(achieved / peak, 4),
+                         "traffic": traffic, "note": bound_note,
+                         "kernel": "attn_partition_kernel" + (
+                             " (append folded in, split units merged in the kernel)"
+                             if r.get("fused") else " (split units merged in the kernel)"),
                          "peak_source": peak_kind + " (MEASURED_PEAKS.json hbm_gbs)"
                          if peak_kind == "measured" else "fallback 6650 GB/s",
                          "kernel_ms": round(r["part_s"] * 1e3, 5)},
@@ -799,6 +993,7 @@ def main():
                 "h2d_bytes_per_step": r["e2e"][1], "d2h_bytes_per_step": r["e2e"][2]},
             "gpu_launches": r["launches"],
             "clocks": r["clocks"],
+            "step_ms_median": round(r["step_ms_median"], 5),
             "device_status": r["status"],
         }
         print(json.dumps(line), flush=True)

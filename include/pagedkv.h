@@ -117,7 +117,10 @@ typedef struct kv_pool kv_pool;   /* opaque host object */
  * KV_ERR_UNSUPPORTED for a block_size, head_dim or dtype outside the lists above. */
 kv_status kv_pool_required_bytes(const kv_pool_desc *desc, uint64_t *bytes);
 
-/* Create the host-side pool object over a caller-owned device buffer.
+/* Create the host-side pool object over a caller-owned device buffer: the
+ * preallocated pool of fixed-size physical blocks that every sequence's cache
+ * is cut into [KV Cache 原理与 PagedAttention, §三 "工作方式" 1; aiworkagent.org
+ * q17, "KV Memory Pool"].
  * device_base: 256-byte aligned device pointer to >= kv_pool_required_bytes
  * bytes; borrowed, never freed by the library. Its contents are not touched;
  * the caller zeroes the status region (kv_pool_status_clear) before first use.
@@ -126,10 +129,13 @@ kv_status kv_pool_required_bytes(const kv_pool_desc *desc, uint64_t *bytes);
 kv_status kv_pool_create(const kv_pool_desc *desc, void *device_base,
                          uint64_t bytes, kv_pool **out);
 
-/* Free the host object. Does not touch device memory. */
+/* Free the host object (the block pool's bookkeeping [KV Cache 原理与
+ * PagedAttention, §三 "工作方式" 3]). Does not touch device memory. */
 kv_status kv_pool_destroy(kv_pool *pool);
 
-/* Device addresses of one layer's regions. k_scale / v_scale are set to NULL
+/* Device addresses of one layer's regions (the layout of kv_pool_required_bytes;
+ * per-layer K and V as in the pages' KV size formula [KV Cache 原理与
+ * PagedAttention, §一 "显存占用公式"]). k_scale / v_scale are set to NULL
  * for 16-bit and scale-less caches. For KV_INT8_KCHAN k_scale is the layer's
  * [num_kv_heads][head_dim] channel-scale array (caller-written). Any output
  * pointer may be NULL if not wanted. */
@@ -184,7 +190,11 @@ kv_status kv_pool_stats(const kv_pool *pool, int32_t *used, int32_t *free_,
 /* Append (reshape_and_cache), quantize, copy-on-write block copy           */
 /* ------------------------------------------------------------------------ */
 
-/* Write each new token's K and V rows into the slot it maps to.
+/* Write each new token's K and V rows into the slot it maps to: each decode
+ * step computes only the new token's K and V and appends them to the cache end
+ * [KV Cache 原理与 PagedAttention, §一; bjdmk.com.cn/news/6246348, §2.1], which in
+ * a paged cache is a row of the block the sequence's table names for that
+ * position [KV Cache 原理与 PagedAttention, §三 "工作方式" 2].
  * k_new, v_new: device [num_tokens][num_kv_heads][head_dim] of in_dtype
  *   (KV_BF16 or KV_FP16), 16-byte aligned.
  * slot_mapping: device int64 [num_tokens]; slot = physical_block * block_size
@@ -252,6 +262,10 @@ kv_status kv_block_copy(kv_pool *pool, const int32_t *host_pairs,
  * finished by it; a unit cut by CTA boundaries leaves a running max m, sum l
  * and unnormalised output o per piece, which the merge combines:
  * out = sum_i e^(m_i - M) o_i / sum_i e^(m_i - M) l_i, M = max_i m_i.
+ * In paged_attn_decode (and _append, _static) the merge runs inside the same
+ * kernel: each CTA counts its pieces in at the unit's arrival counter, and the
+ * CTA whose piece completes the unit merges it. paged_attn_partition +
+ * paged_attn_merge run the two phases as separate kernels (same bits).
  *
  * Common arguments:
  *   q       device [num_seqs][num_q_heads][head_dim], q_dtype, 16-byte aligned.
@@ -267,14 +281,16 @@ kv_status kv_block_copy(kv_pool *pool, const int32_t *host_pairs,
  *           of the current device (the default), else 1 .. 65535.
  *   workspace     device, 256-byte aligned, >= paged_attn_workspace_bytes
  *           bytes for the same num_seqs, num_q_heads and num_ctas. Holds the
- *           per-unit bookkeeping and the split partials between the two
- *           kernels; its contents are scratch and need no initialisation.
+ *           per-unit bookkeeping and arrival counters and the split partials;
+ *           its contents are scratch and need no initialisation (a counter is
+ *           tagged with the launch that wrote it, and the merging CTA resets
+ *           it, so a replayed launch also starts from zero).
  *           Concurrent calls must use separate workspaces.
  */
 
-/* Workspace bytes for these sizes: 16 B per unit plus 2 x 64 x (head_dim + 2)
- * fp32 per CTA, each part rounded up to 256 B. num_ctas = 0 queries the
- * current device (KV_ERR_CUDA without one). */
+/* Workspace bytes for these sizes: 16 B of bookkeeping and an 8-byte counter
+ * per unit plus 2 x 64 x (head_dim + 2) fp32 per CTA, each part rounded up to
+ * 256 B. num_ctas = 0 queries the current device (KV_ERR_CUDA without one). */
 kv_status paged_attn_workspace_bytes(const kv_pool *pool, int32_t num_seqs,
                                      int32_t num_q_heads, int32_t num_ctas,
                                      uint64_t *bytes);
@@ -283,8 +299,9 @@ kv_status paged_attn_workspace_bytes(const kv_pool *pool, int32_t num_seqs,
  * device). */
 kv_status paged_attn_default_ctas(const kv_pool *pool, int32_t *num_ctas);
 
-/* Full decode attention: paged_attn_partition followed by paged_attn_merge on
- * the same stream. */
+/* Full decode attention in one kernel launch: the work split above, with the
+ * split units merged inside the kernel. The same bits as paged_attn_partition
+ * followed by paged_attn_merge on the same stream. */
 kv_status paged_attn_decode(kv_pool *pool, int32_t layer, const void *q,
                             int32_t q_dtype, int32_t num_seqs,
                             int32_t num_q_heads, const int32_t *block_tables,
@@ -302,7 +319,10 @@ kv_status paged_attn_decode(kv_pool *pool, int32_t layer, const void *q,
  * The split-K scratch lives in a 16 MiB array inside the library's own device
  * memory (every GPU that loads the library holds it until the process exits).
  * The first call on each device looks up that array's device address with the
- * device current; make that first call before any stream capture. Calls whose
+ * device current; make that first call before any stream capture. The stream
+ * must belong to the current device (else KV_ERR_INVALID), and the looked-up
+ * address does not survive a reset of the device (cudaDeviceReset): do not use
+ * this entry point across one. Calls whose
  * scratch would exceed 16 MiB (paged_attn_workspace_bytes for the same
  * num_seqs, num_q_heads, num_ctas) return KV_ERR_INVALID and queue nothing.
  * Every call uses the same array, so calls that overlap on the GPU (on

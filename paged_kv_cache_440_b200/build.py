@@ -1,10 +1,10 @@
 """Build libpagedkv.so for sm_100a, in the package directory.
 
-    python -m paged_kv_cache_440_b200.build [--force] [--debug]
+    python -m paged_kv_cache_440_b200.build [--force]
 
-Extra nvcc flags (for example tuning defines such as -DPAGEDKV_PF_GROUPS=2)
-come from the environment variable PAGEDKV_NVCC_FLAGS; pass --force after
-changing them.
+Extra nvcc flags (for example -lineinfo variants or -Xptxas options) come
+from the environment variable PAGEDKV_NVCC_FLAGS; pass --force after changing
+them.
 
 Each source under csrc/ is compiled by nvcc to an object in _build/ (rebuilt
 only when it or a header is newer), then linked with the static CUDA runtime
@@ -59,10 +59,9 @@ def _compile(src, obj, extra, verbose_log):
     return obj
 
 
-def build(force=False, debug=False, jobs=None):
+def build(force=False, jobs=None):
     os.makedirs(BUILD, exist_ok=True)
-    extra = ["-DPAGEDKV_DEBUG=1"] if debug else []
-    extra += os.environ.get("PAGEDKV_NVCC_FLAGS", "").split()
+    extra = os.environ.get("PAGEDKV_NVCC_FLAGS", "").split()
     newest_header = max((os.path.getmtime(h) for h in _headers()), default=0)
     todo, objs = [], []
     for src in _sources():
@@ -89,7 +88,6 @@ def build(force=False, debug=False, jobs=None):
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
-    ap.add_argument("--debug", action="store_true")
     a = ap.parse_args()
-    print(build(force=a.force, debug=a.debug))
+    print(build(force=a.force))
     sys.exit(0)

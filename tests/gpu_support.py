@@ -143,3 +143,63 @@ def oracle_outputs(wl, kcache, vcache, pairs, tables=None):
 def raw_bytes(t):
     """Host copy of a device tensor's bytes, shaped [..., last * itemsize]."""
     return t.detach().contiguous().view(torch.uint8).cpu().numpy()
+
+
+def host_f32(t):
+    """Exact float32 host copy of a bf16 / fp16 device tensor (via its bits)."""
+    u = t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    if t.dtype == torch.bfloat16:
+        return (u.astype(np.uint32) << 16).view(np.float32)
+    return u.view(np.float16).astype(np.float32)
+
+
+def check_quant_pool(wl, pool, threads=8):
+    """Every code and scale byte a quantized cache holds for every sequence's
+    positions 0 .. L-1 (its history, then the step's new token) against the
+    oracle's quantization of the same rows. Sequences are checked in parallel
+    threads (numpy releases the GIL); returns the number of rows checked."""
+    import concurrent.futures
+    K, V, KS, VS = pool.layer_views(0)
+    kc, vc = K.cpu().numpy(), V.cpu().numpy()
+    ks = KS.cpu().numpy() if KS is not None else None
+    vs = VS.cpu().numpy() if VS is not None else None
+    k_hist, v_hist = host_f32(wl.k_hist), host_f32(wl.v_hist)
+    k_new, v_new = host_f32(wl.k_new), host_f32(wl.v_new)
+    bs, H = wl.block_size, wl.kv_heads
+    starts = np.concatenate([[0], np.cumsum(np.maximum(wl.context_lens - 1, 0))])
+    kind = wl.cache_dtype
+
+    def one(b):
+        L = int(wl.context_lens[b])
+        if L <= 0:
+            return 0
+        nblk = -(-L // bs)
+        ids = wl.block_tables[b, :nblk]
+        tok = lambda a: a[ids].transpose(0, 2, 1, 3).reshape(nblk * bs, H, -1)[:L]
+        tok_s = lambda a: a[ids].transpose(0, 2, 1).reshape(nblk * bs, H)[:L]
+        lo, hi = int(starts[b]), int(starts[b + 1])
+        kx = np.concatenate([k_hist[lo:hi], k_new[b:b + 1]])
+        vx = np.concatenate([v_hist[lo:hi], v_new[b:b + 1]])
+        if kind == "int8_kchan":
+            kq, kscale = quant.quantize_k_channels(kx, wl.k_chan), None
+            vq, vscale = quant.quantize_rows(vx, "int8")
+        else:
+            kq, kscale = quant.quantize_rows(kx, kind)
+            vq, vscale = quant.quantize_rows(vx, kind)
+        if kind == "int4":
+            kq, vq = quant.pack_int4(kq), quant.pack_int4(vq)
+        assert np.array_equal(tok(kc).view(np.uint8), kq.view(np.uint8)), "K codes, seq %d" % b
+        assert np.array_equal(tok(vc).view(np.uint8), vq.view(np.uint8)), "V codes, seq %d" % b
+        if kscale is not None and ks is not None:
+            assert np.array_equal(tok_s(ks).view(np.uint32), kscale.view(np.uint32)), \
+                "K scales, seq %d" % b
+        if vs is not None and kind != "e5m2_cast":
+            assert np.array_equal(tok_s(vs).view(np.uint32), vscale.view(np.uint32)), \
+                "V scales, seq %d" % b
+        return L * H
+
+    with concurrent.futures.ThreadPoolExecutor(max_workers=threads) as ex:
+        rows = sum(ex.map(one, range(wl.batch)))
+    if kind == "int8_kchan":
+        assert np.array_equal(ks, wl.k_chan)      # the layer's channel scales, untouched
+    return rows

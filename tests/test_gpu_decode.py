@@ -13,8 +13,8 @@ import pytest
 import torch
 
 import workloads as W
-from gpu_support import (bits16, build_pool, compare, device_inputs, oracle_cache_16,
-                         oracle_cache_quant, oracle_outputs, step, to_np)
+from gpu_support import (bits16, build_pool, check_quant_pool, compare, device_inputs,
+                         oracle_cache_16, oracle_cache_quant, oracle_outputs, step, to_np)
 from oracle import cache_ops
 
 pytestmark = pytest.mark.gpu
@@ -70,30 +70,52 @@ def test_mha13b_every_output(pkv):
     _run_16(pkv, W.mha13b(DEV))
 
 
-@pytest.mark.parametrize("kind", ["int8", "e5m2", "int4", "int8_kchan"])
-@pytest.mark.parametrize("variant,seqs", [("a", [0, 13, 40, 63]), ("b", [0, 5])])
-def test_quantized_long_context(pkv, kind, variant, seqs):
-    """INT8 / E5M2 per-token-head KV, bs 32, (a) 64 x 4096 and (b) 8 x 32768.
-    Codes and scales of the sampled sequences are bit-exact; their outputs match
-    the oracle run on the same dequantized values."""
-    wl = W.quant_long(kind, variant, DEV)
+def test_gqa70b_benchmarked_call(pkv):
+    """Exactly the call the benchmark times: paged_attn_decode_append on the
+    LLaMA-70B-shaped layer (batch 32, lengths U[512, 4096]) with the default
+    CTA count and a workspace from make_workspace. Every pool row is bit-exact
+    with the oracle's append (the new token at position L - 1), and all 2048
+    outputs match the oracle."""
+    wl = W.gqa70b(DEV)
     pool = build_pool(pkv, wl, DEV)
-    out = step(pkv, pool, wl, DEV)
+    tables, lens = device_inputs(wl, DEV)
+    G = pkv.default_ctas(pool)
+    ws = pkv.make_workspace(pool, wl.batch, wl.q_heads, G)
+    out = torch.empty_like(wl.q)
+    pkv.paged_attn_decode_append(pool, 0, wl.q, wl.k_new, wl.v_new, tables, lens,
+                                 int(wl.context_lens.max()), wl.scale, out=out, num_ctas=G,
+                                 workspace=ws)
     torch.cuda.synchronize()
     assert pool.status() == 0
-    (kc, vc, ks, vs), (kd, vd, otab) = oracle_cache_quant(wl, seqs)
-    K, V, KS, VS = pool.layer_views(0)
-    for b in seqs:
-        nblk = -(-int(wl.context_lens[b]) // wl.block_size)
-        ids = torch.from_numpy(wl.block_tables[b, :nblk].astype(np.int64)).to(DEV)
-        idn = wl.block_tables[b, :nblk]
-        assert np.array_equal(K[ids].cpu().numpy(), kc[idn]), "K codes, seq %d" % b
-        assert np.array_equal(V[ids].cpu().numpy(), vc[idn]), "V codes, seq %d" % b
-        if kind != "int8_kchan":                 # channel scales: the layer's, checked below
-            assert np.array_equal(KS[ids].cpu().numpy().view(np.uint32), ks[idn].view(np.uint32))
-        assert np.array_equal(VS[ids].cpu().numpy().view(np.uint32), vs[idn].view(np.uint32))
-    if kind == "int8_kchan":
-        assert np.array_equal(KS.cpu().numpy(), wl.k_chan)
+    K, V, _, _ = pool.layer_views(0)
+    kb, vb = bits16(wl.k_fill), bits16(wl.v_fill)
+    cache_ops.append(kb, vb, bits16(wl.k_new), bits16(wl.v_new), wl.slot_new, wl.block_size)
+    assert np.array_equal(bits16(K), kb) and np.array_equal(bits16(V), vb)
+    k, v = oracle_cache_16(wl)
+    pairs = _all_pairs(wl)
+    compare(torch.stack([out[b, h] for b, h in pairs]), oracle_outputs(wl, k, v, pairs),
+            what="gqa70b benchmarked call")
+
+
+@pytest.mark.parametrize("kind", ["int8", "e5m2", "int4", "int8_kchan", "e5m2_cast"])
+@pytest.mark.parametrize("variant,seqs", [("a", [0, 9, 13, 27, 40, 51, 58, 63]), ("b", [0, 5])])
+def test_quantized_long_context(pkv, kind, variant, seqs):
+    """Quantized KV, bs 32, (a) 64 x 4096 and (b) 8 x 32768, through the call
+    the benchmark times (paged_attn_decode_append: history appended with
+    kv_append, the step's token quantized inside the attention kernel). Every
+    code and scale of every sequence is bit-exact with the oracle's
+    quantization of the same rows; outputs of the sampled sequences match the
+    oracle run on the same dequantized values."""
+    wl = W.quant_long(kind, variant, DEV)
+    pool = build_pool(pkv, wl, DEV)
+    tables, lens = device_inputs(wl, DEV)
+    out = pkv.paged_attn_decode_append(pool, 0, wl.q, wl.k_new, wl.v_new, tables, lens,
+                                       int(wl.context_lens.max()), wl.scale)
+    torch.cuda.synchronize()
+    assert pool.status() == 0
+    rows = check_quant_pool(wl, pool)
+    assert rows == int(wl.context_lens.sum()) * wl.kv_heads
+    _, (kd, vd, otab) = oracle_cache_quant(wl, seqs)
     pairs = _all_pairs(wl, seqs)
     ref = oracle_outputs(wl, kd, vd, pairs, otab)
     compare(torch.stack([out[b, h] for b, h in pairs]), ref, what=wl.name)
@@ -103,7 +125,7 @@ def test_shared_prefix_copy_on_write(pkv):
     """200 requests share a 1500-token prompt (94 blocks of 16, the last holding
     12 tokens). Every request copies the shared partial block before appending
     its private suffix. The oracle builds its own cache with its own allocator
-    model and copies; outputs agree for a sample of requests."""
+    model and copies; the outputs of all 200 requests agree."""
     from oracle import allocator, cache_ops
     wl = W.shared_prefix(DEV)
     bs, hkv, D = wl.block_size, wl.kv_heads, wl.head_dim
@@ -179,12 +201,14 @@ def test_shared_prefix_copy_on_write(pkv):
     o_tbl = np.full((wl.batch, mb), -1, np.int64)
     for b, t in enumerate(o_tables):
         o_tbl[b, :len(t)] = t
+    import concurrent.futures
     from oracle import attention
     q = to_np(wl.q, np.float64)
-    sample = [0, 1, 57, 123, 199]
-    got = torch.stack([out[b, h] for b in sample for h in range(wl.q_heads)])
-    ref = np.stack([attention.decode_one(q, kc, vc, o_tbl, lens, wl.scale, b, h)
-                    for b in sample for h in range(wl.q_heads)])
+    pairs = [(b, h) for b in range(wl.batch) for h in range(wl.q_heads)]
+    with concurrent.futures.ThreadPoolExecutor(max_workers=8) as ex:
+        ref = np.stack(list(ex.map(
+            lambda bh: attention.decode_one(q, kc, vc, o_tbl, lens, wl.scale, *bh), pairs)))
+    got = torch.stack([out[b, h] for b, h in pairs])
     compare(got, ref, what="shared_prefix")
 
 
@@ -382,4 +406,37 @@ def test_decode_whatever_the_workspace_held(pkv, name, make, G):
                                   num_ctas=G, workspace=ws)
             torch.cuda.synchronize()
             assert np.array_equal(bits16(out), bits16(ref)), name
+    assert pool.status() == 0
+
+
+def test_decode_graph_replays_match(pkv):
+    """A decode step captured in a CUDA graph replays with the same launch (the
+    same arrival-counter epoch) every time: the CTA that merges a split unit
+    resets its counter, so each replay merges again and gives the same bits as
+    a direct call (and as the separate partition + merge kernels)."""
+    wl = W.gqa70b(DEV, batch=12)
+    pool = build_pool(pkv, wl, DEV)
+    tables, lens = device_inputs(wl, DEV)
+    pkv.kv_append(pool, 0, wl.k_new, wl.v_new, torch.from_numpy(wl.slot_new).to(DEV))
+    max_ctx = int(wl.context_lens.max())
+    G = 53
+    ws = pkv.make_workspace(pool, wl.batch, wl.q_heads, G)
+    ref = torch.empty_like(wl.q)
+    pkv.paged_attn_partition(pool, 0, wl.q, tables, lens, max_ctx, wl.scale, ref, ws, num_ctas=G)
+    pkv.paged_attn_merge(pool, lens, tables.shape[1], max_ctx, ref, ws, num_ctas=G)
+    out = torch.empty_like(wl.q)
+    pkv.paged_attn_decode(pool, 0, wl.q, tables, lens, max_ctx, wl.scale, out=out, num_ctas=G,
+                          workspace=ws)           # warm-up outside the capture
+    torch.cuda.synchronize()
+    assert np.array_equal(bits16(out), bits16(ref))
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        pkv.paged_attn_decode(pool, 0, wl.q, tables, lens, max_ctx, wl.scale, out=out,
+                              num_ctas=G, workspace=ws)
+    for _ in range(3):
+        out.fill_(float("nan"))
+        graph.replay()
+        torch.cuda.synchronize()
+        assert np.array_equal(bits16(out), bits16(ref))
+    del graph
     assert pool.status() == 0
