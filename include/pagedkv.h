@@ -262,10 +262,6 @@ kv_status kv_block_copy(kv_pool *pool, const int32_t *host_pairs,
  * finished by it; a unit cut by CTA boundaries leaves a running max m, sum l
  * and unnormalised output o per piece, which the merge combines:
  * out = sum_i e^(m_i - M) o_i / sum_i e^(m_i - M) l_i, M = max_i m_i.
- * In paged_attn_decode (and _append, _static) the merge runs inside the same
- * kernel: each CTA counts its pieces in at the unit's arrival counter, and the
- * CTA whose piece completes the unit merges it. paged_attn_partition +
- * paged_attn_merge run the two phases as separate kernels (same bits).
  *
  * Common arguments:
  *   q       device [num_seqs][num_q_heads][head_dim], q_dtype, 16-byte aligned.
@@ -281,16 +277,14 @@ kv_status kv_block_copy(kv_pool *pool, const int32_t *host_pairs,
  *           of the current device (the default), else 1 .. 65535.
  *   workspace     device, 256-byte aligned, >= paged_attn_workspace_bytes
  *           bytes for the same num_seqs, num_q_heads and num_ctas. Holds the
- *           per-unit bookkeeping and arrival counters and the split partials;
- *           its contents are scratch and need no initialisation (a counter is
- *           tagged with the launch that wrote it, and the merging CTA resets
- *           it, so a replayed launch also starts from zero).
+ *           per-unit bookkeeping and the split partials between the two
+ *           kernels; its contents are scratch and need no initialisation.
  *           Concurrent calls must use separate workspaces.
  */
 
-/* Workspace bytes for these sizes: 16 B of bookkeeping and an 8-byte counter
- * per unit plus 2 x 64 x (head_dim + 2) fp32 per CTA, each part rounded up to
- * 256 B. num_ctas = 0 queries the current device (KV_ERR_CUDA without one). */
+/* Workspace bytes for these sizes: 16 B per unit plus 2 x 64 x (head_dim + 2)
+ * fp32 per CTA, each part rounded up to 256 B. num_ctas = 0 queries the
+ * current device (KV_ERR_CUDA without one). */
 kv_status paged_attn_workspace_bytes(const kv_pool *pool, int32_t num_seqs,
                                      int32_t num_q_heads, int32_t num_ctas,
                                      uint64_t *bytes);
@@ -299,9 +293,9 @@ kv_status paged_attn_workspace_bytes(const kv_pool *pool, int32_t num_seqs,
  * device). */
 kv_status paged_attn_default_ctas(const kv_pool *pool, int32_t *num_ctas);
 
-/* Full decode attention in one kernel launch: the work split above, with the
- * split units merged inside the kernel. The same bits as paged_attn_partition
- * followed by paged_attn_merge on the same stream. */
+/* Full decode attention: paged_attn_partition followed by paged_attn_merge on
+ * the same stream (the merge kernel is launched so that it is scheduled while
+ * the attention kernel drains). */
 kv_status paged_attn_decode(kv_pool *pool, int32_t layer, const void *q,
                             int32_t q_dtype, int32_t num_seqs,
                             int32_t num_q_heads, const int32_t *block_tables,

@@ -42,7 +42,6 @@
 //   multiply the scores, per-token V scales are folded into the softmax
 //   weights through log2(scale) so the fp16 weights stay within (0, 1].
 #include <algorithm>
-#include <atomic>
 #include <cfloat>
 
 #include "device.cuh"
@@ -72,9 +71,6 @@ struct AttnParams {
   float *part_o;   // [num_ctas][2][kNC][8][D]   unnormalised outputs of split units
   float *part_ml;  // [num_ctas][2][kNC][8][2]   their (max, sum), base 2
   int4 *meta;      // [num_seqs * units_per_seq]: first CTA, #CTAs, first side
-  // [num_seqs * units_per_seq] arrival counters of split units: launch epoch in
-  // the high 32 bits, pieces arrived in the low 32 (fused merge only)
-  unsigned long long *counters;
   int *status;
   // fused append (paged_attn_decode_append): each sequence's new token, written
   // at position L - 1 before it is attended; null when not fused
@@ -96,14 +92,11 @@ struct AttnParams {
   int units_per_seq;   // (kv_heads / hg) * cgroups
   int stage_bytes;     // bytes between ring stages (load size rounded to 1024)
   int stages;          // ring stages (R)
-  int merge_region;    // shared-memory bytes per consumer warp for the fused merge
-  int unit_cost4;      // quarter blocks charged for starting a unit (see Walk)
+  int unit_cost;       // positions charged for starting a unit (see Walk)
   int max_blocks;      // block-table row length
   int num_blocks;      // physical blocks in the pool
   int limit;           // valid lengths: 0 < L <= min(max_context, max_blocks * bs)
   int num_ctas;
-  int fuse_merge;      // 1: the CTA whose piece of a split unit arrives last merges it
-  uint32_t epoch;      // nonzero tag of this launch's counter arrivals
 };
 
 constexpr int align_up_c(int x, int a) { return (x + a - 1) / a * a; }
@@ -181,26 +174,9 @@ __device__ __forceinline__ float warp_max_xor(float v, int from) {
 __device__ __forceinline__ float exp2_rel(float x, float m) {
   return x == -INFINITY ? 0.f : exp2f(x - m);
 }
-// Folds one split piece (running max m, sum l, unnormalised outputs o, base 2)
-// into the running (M, Ls, acc) of the merge:
-//   out = sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i,  M = max_i m_i.
-// Every rounding is explicit, so the merge kernel and the merge inside the
-// attention kernel produce the same bits for the same pieces in the same order.
-template <int E>
-__device__ __forceinline__ void combine_piece(float &M, float &Ls, float (&acc)[E], float m,
-                                              float l, const float (&o)[E]) {
-  const float Mn = fmaxf(M, m);
-  if (Mn == -INFINITY) return;  // nothing seen yet, nothing added
-  const float a = exp2_rel(M, Mn), wt = exp2_rel(m, Mn);
-  Ls = __fmaf_rn(l, wt, __fmul_rn(Ls, a));
-#pragma unroll
-  for (int e = 0; e < E; ++e) acc[e] = __fmaf_rn(o[e], wt, __fmul_rn(acc[e], a));
-  M = Mn;
-}
-
-// Final normalisation of a merged output element.
-__device__ __forceinline__ float merged_value(float acc, float Ls) {
-  return Ls > 0.f ? __fmul_rn(acc, __fdiv_rn(1.f, Ls)) : 0.f;
+// Rescale factor exp2(m_old - m_new), 1 while nothing has been seen.
+__device__ __forceinline__ float rescale(float m_old, float m_new) {
+  return m_new == -INFINITY ? 1.f : exp2f(m_old - m_new);
 }
 
 // The SFU's base-2 exponential and logarithm (relative error about 2^-22,
@@ -248,10 +224,20 @@ __device__ __forceinline__ int cta_of(long long x, long long T, long long G) {
   return static_cast<int>(r + (x - r * (q + 1)) / q);
 }
 
+__device__ __forceinline__ long long block_sum(long long v, long long *red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  long long t = 0;
+#pragma unroll
+  for (int i = 0; i < kWarps; ++i) t += red[i];
+  __syncthreads();
+  return t;
+}
+
 // Exclusive prefix sum over the CTA's threads; *total gets the CTA's sum.
-// With reuse = false it takes a single __syncthreads and `red` must not be
-// written again; with reuse = true a second one makes `red` reusable.
-template <bool kReuse>
 __device__ __forceinline__ long long block_excl_scan(long long v, long long *red,
                                                      long long *total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -269,18 +255,9 @@ __device__ __forceinline__ long long block_excl_scan(long long v, long long *red
     before += i < warp ? red[i] : 0;
     tot += red[i];
   }
-  if constexpr (kReuse) __syncthreads();
+  __syncthreads();
   *total = tot;
   return before + x - v;
-}
-
-// A sequence's contribution to the split, packed in one integer so that one
-// prefix sum gives both: its blocks (bits 26 and up) and whether it has any
-// (bit 0; then each of its units carries one unit-start charge).
-constexpr int kUnitBits = 26;
-constexpr long long kUnitMask = (1ll << kUnitBits) - 1;
-__device__ __forceinline__ long long pack_seq(int nb) {
-  return (static_cast<long long>(nb) << kUnitBits) | (nb > 0 ? 1 : 0);
 }
 
 // Waits on a ring barrier; gives up when another warp has aborted or the time
@@ -792,25 +769,6 @@ struct NewRow {
     }
   }
 
-  // Park this lane's share in shared memory (buf: [6][32] words of this warp)
-  // between the piece start and the block that takes it.
-  __device__ __forceinline__ void stash(uint32_t *buf, int lane) const {
-    buf[lane] = k[0];
-    buf[32 + lane] = k[1];
-    buf[64 + lane] = v[0];
-    buf[96 + lane] = v[1];
-    buf[128 + lane] = __float_as_uint(ks);
-    buf[160 + lane] = __float_as_uint(vs);
-  }
-  __device__ __forceinline__ void unstash(const uint32_t *buf, int lane) {
-    k[0] = buf[lane];
-    k[1] = buf[32 + lane];
-    v[0] = buf[64 + lane];
-    v[1] = buf[96 + lane];
-    ks = __uint_as_float(buf[128 + lane]);
-    vs = __uint_as_float(buf[160 + lane]);
-  }
-
   // Put the row in the stage (row r0 + rl of the stage's K / V parts, where the
   // load brought whatever the pool held) and in the pool (block id, head g).
   __device__ __forceinline__ void store(const AttnParams &p, uint8_t *st, int rows, int r, int id,
@@ -856,19 +814,10 @@ struct NewRow {
 };
 
 // Position of a CTA's walk over the flattened (unit, block) list. Each unit
-// with blocks occupies cost + ppb * nb positions: `cost` positions that stand
-// for the fixed work of starting a unit (query load, partial write), then ppb
-// per block. The positions of all units are split evenly over the CTAs and a
-// CTA takes the blocks whose first position falls in its range, so a CTA
-// whose share starts a unit takes fewer blocks. With ppb = 4 (used whenever
-// every CTA gets at least 4 positions) shares are balanced to a quarter block;
-// with ppb = 1 (tiny workloads) every position past a unit's charge is a
-// block start, so every CTA between a unit's first and last block holds one.
-struct Split {
-  int ppb;   // positions per block: 4 or 1
-  int cost;  // positions charged per unit start
-};
-
+// with blocks occupies unit_cost + nb positions: unit_cost positions that
+// stand for the fixed work of starting a unit (query load, partial write),
+// then one per block. The even split of positions over CTAs thus gives a CTA
+// whose share starts a unit fewer blocks.
 struct Walk {
   int b;         // sequence
   int gc;        // unit within the sequence: kv head * chunks + chunk
@@ -878,193 +827,30 @@ struct Walk {
 };
 
 // Positions of one unit of a sequence with nb blocks.
-__device__ __forceinline__ long long unit_len(int nb, const Split &sp) {
-  return nb > 0 ? static_cast<long long>(sp.ppb) * nb + sp.cost : 0;
-}
-
-// Blocks from w.j whose first position lies before s1 (w.pos < s1).
-__device__ __forceinline__ int walk_seg(const Walk &w, long long s1, const Split &sp) {
-  const long long left = (s1 - w.pos + sp.ppb - 1) / sp.ppb;
-  return static_cast<int>(min(static_cast<long long>(w.nb - w.j), left));
-}
-
-// From the end of a unit (w.j == w.nb) to the first block of the next unit
-// with blocks.
-template <int BS>
-__device__ __forceinline__ void walk_next_unit(Walk &w, const Split &sp, const AttnParams &p) {
-  w.j = 0;
-  w.pos += sp.cost;  // past the next unit's charge: its first block
-  if (++w.gc == p.units_per_seq) {
-    w.gc = 0;
-    do {
-      ++w.b;
-      w.nb = w.b < p.num_seqs ? seq_blocks<BS>(p, w.b) : 0;
-    } while (w.b < p.num_seqs && w.nb == 0);
-  }
+__device__ __forceinline__ int unit_len(int nb, const AttnParams &p) {
+  return nb > 0 ? nb + p.unit_cost : 0;
 }
 
 template <int BS>
-__device__ __forceinline__ void walk_advance(Walk &w, int seg, const Split &sp,
-                                             const AttnParams &p) {
-  w.pos += static_cast<long long>(sp.ppb) * seg;
+__device__ __forceinline__ void walk_advance(Walk &w, int seg, const AttnParams &p) {
+  w.pos += seg;
   w.j += seg;
-  if (w.j == w.nb) walk_next_unit<BS>(w, sp, p);
-}
-
-// Head slot geometry of unit gc for consumer warp `warp`: kv head g, query
-// heads h0 .. h0 + nh - 1; active = false for a warp with no slot in the unit.
-struct Slot {
-  bool active;
-  int hi, g, h0, nh;
-};
-__device__ __forceinline__ Slot slot_of(const AttnParams &p, int gc, int warp) {
-  Slot s;
-  const int hgi = gc / p.cgroups;
-  const int cgi = gc - hgi * p.cgroups;
-  const int cpg = min(p.cpg, p.chunks - cgi * p.cpg);
-  s.active = warp < p.hg * cpg;
-  s.hi = s.active ? warp / cpg : 0;
-  const int cl = warp - s.hi * cpg;
-  s.g = hgi * p.hg + s.hi;
-  const int chunk = cgi * p.cpg + cl;
-  s.h0 = s.g * p.group + chunk * kChunkHeads;
-  s.nh = min(kChunkHeads, p.group - chunk * kChunkHeads);
-  return s;
-}
-
-__device__ __forceinline__ void prefetch_l2(const void *ptr) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
-}
-
-// Arrival of one piece of a split unit at its counter (launch epoch in the
-// high word, count in the low word; a stale epoch counts as 0). Returns true
-// for the arrival that completes the unit's nu pieces and then resets the
-// counter to 0, so a replay of the same launch (same epoch) starts afresh.
-__device__ __forceinline__ bool arrive_last(unsigned long long *ctr, uint32_t epoch, int nu,
-                                            int *status) {
-  unsigned long long old = *reinterpret_cast<volatile unsigned long long *>(ctr);
-  for (int it = 0; it < (1 << 20); ++it) {
-    const unsigned long long cnt =
-        static_cast<uint32_t>(old >> 32) == epoch ? (old & 0xffffffffull) : 0ull;
-    const unsigned long long nw = (static_cast<unsigned long long>(epoch) << 32) | (cnt + 1);
-    const unsigned long long prev = atomicCAS(ctr, old, nw);
-    if (prev == old) {
-      if (cnt + 1 != static_cast<unsigned long long>(nu)) return false;
-      *reinterpret_cast<volatile unsigned long long *>(ctr) = 0ull;
-      return true;
+  if (w.j == w.nb) {
+    w.j = 0;
+    w.pos += p.unit_cost;  // the next unit's first block
+    if (++w.gc == p.units_per_seq) {
+      w.gc = 0;
+      do {
+        ++w.b;
+        w.nb = w.b < p.num_seqs ? seq_blocks<BS>(p, w.b) : 0;
+      } while (w.b < p.num_seqs && w.nb == 0);
     }
-    old = prev;
   }
-  atomicOr(status, kErrTimeout);
-  return false;
 }
 
 // ============================================================================
 // Partition kernel: persistent, one producer warp + kNC consumer warps.
 // ============================================================================
-
-// Zeros for the outputs of sequence b when its length is empty or invalid
-// (threads t of n of the caller's group share the work).
-template <int D, int Q_T>
-__device__ __forceinline__ void zero_sequence(const AttnParams &p, int b, int t, int n) {
-  const int L = p.context_lens[b];
-  if (L > 0 && L <= p.limit) return;
-  uint4 *o = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) +
-                                       static_cast<int64_t>(b) * p.q_heads * D);
-  const int chunks = p.q_heads * D * 2 / 16;
-  for (int i = t; i < chunks; i += n) o[i] = make_uint4(0u, 0u, 0u, 0u);
-}
-
-// Merge of one split unit by consumer warp `warp` (its head slot), run by the
-// CTA whose piece arrived last: the unit's pieces are fetched with bulk
-// copies into this warp's share of the (drained) ring, folded in piece order
-// and normalised into out.
-template <int D, int BS, int Q_T>
-__device__ __forceinline__ void merge_unit(const AttnParams &p, int b, int gc, long long ustart,
-                                           int nb, const Split &sp, long long total, long long G,
-                                           uint8_t *region, int region_bytes, uint64_t *bar,
-                                           uint32_t &phase, int warp, int lane) {
-  constexpr int E = D / 32;
-  const Slot sl = slot_of(p, gc, warp);
-  if (!sl.active) return;
-  const long long first = ustart + sp.cost;  // block 0's position
-  const int c0 = cta_of(first, total, G);
-  const int c1 = cta_of(first + static_cast<long long>(sp.ppb) * (nb - 1), total, G);
-  const int nu = c1 - c0 + 1;
-  // c0 also holds the previous unit's last block (then this is its second
-  // piece, side 1) iff its range starts at or before that block's position
-  const int side0 = cta_start(c0, total, G) <= ustart - sp.ppb ? 1 : 0;
-  constexpr int kOBytes = kChunkHeads * D * 4;
-  constexpr int kMlBytes = kChunkHeads * 2 * 4;
-  const int per = region_bytes / (kOBytes + kMlBytes);  // pieces per batch
-  if (per < 1) {  // the host sizes the region for at least one piece
-    if (lane == 0) atomicOr(p.status, kErrTimeout);
-    return;
-  }
-  float *so = reinterpret_cast<float *>(region);
-  float *sml = reinterpret_cast<float *>(region + per * kOBytes);
-  float M[kChunkHeads], Ls[kChunkHeads], acc[kChunkHeads][E];
-#pragma unroll
-  for (int n = 0; n < kChunkHeads; ++n) {
-    M[n] = -INFINITY;
-    Ls[n] = 0.f;
-#pragma unroll
-    for (int e = 0; e < E; ++e) acc[n][e] = 0.f;
-  }
-  for (int k0 = 0; k0 < nu; k0 += per) {
-    const int cnt = min(per, nu - k0);
-    if (lane == 0) {
-      // the pieces were written by other CTAs' generic stores, published
-      // through the arrival counter; the bulk copies read them in the async
-      // proxy, and overwrite shared memory this warp last read generically
-      asm volatile("fence.proxy.async.global;" ::: "memory");
-      fence_proxy_async_smem();
-      mbar_arrive_expect_tx(bar, cnt * (kOBytes + kMlBytes));
-      for (int k = 0; k < cnt; ++k) {
-        const int i = k0 + k;
-        const int64_t rec =
-            ((static_cast<int64_t>(c0 + i) * 2 + (i == 0 ? side0 : 0)) * kNC + warp) * kChunkHeads;
-        bulk_load(so + k * (kOBytes / 4), p.part_o + rec * D, kOBytes, bar);
-        bulk_load(sml + k * (kMlBytes / 4), p.part_ml + rec * 2, kMlBytes, bar);
-      }
-    }
-    int okv = 1;
-    if (lane == 0) okv = mbar_wait(bar, phase, p.status);
-    okv = __shfl_sync(0xffffffffu, okv, 0);
-    if (!okv) return;  // gave up: the status word has the timeout bit
-    while (!mbar_try_wait(bar, phase)) {
-    }  // already complete: gives every lane the acquire
-    phase ^= 1u;
-    for (int k = 0; k < cnt; ++k) {
-#pragma unroll
-      for (int n = 0; n < kChunkHeads; ++n) {
-        if (n < sl.nh) {
-          const float2 ml = *reinterpret_cast<const float2 *>(sml + k * (kMlBytes / 4) + 2 * n);
-          float o[E];
-          const float *src = so + k * (kOBytes / 4) + n * D + lane * E;
-          if constexpr (E == 4) {
-            const float4 x = *reinterpret_cast<const float4 *>(src);
-            o[0] = x.x; o[1] = x.y; o[2] = x.z; o[3] = x.w;
-          } else {
-            const float2 x = *reinterpret_cast<const float2 *>(src);
-            o[0] = x.x; o[1] = x.y;
-          }
-          combine_piece<E>(M[n], Ls[n], acc[n], ml.x, ml.y, o);
-        }
-      }
-    }
-    __syncwarp();  // every lane has read the batch before the next overwrites it
-  }
-#pragma unroll
-  for (int n = 0; n < kChunkHeads; ++n) {
-    if (n < sl.nh) {
-      const int64_t o = (static_cast<int64_t>(b) * p.q_heads + sl.h0 + n) * D + lane * E;
-#pragma unroll
-      for (int e = 0; e < E; ++e) store_out<Q_T>(p.out, o + e, merged_value(acc[n][e], Ls[n]));
-    }
-  }
-}
-
 template <int D, int BS, int KV_T, int Q_T>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_partition_kernel(const __grid_constant__ CUtensorMap kmap,
@@ -1075,18 +861,10 @@ attn_partition_kernel(const __grid_constant__ CUtensorMap kmap,
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[kMaxStages];
   __shared__ __align__(8) uint64_t empty_bar[kMaxStages];
-  __shared__ __align__(8) uint64_t merge_bar[kNC];
   __shared__ int stage_id[kMaxStages];
   __shared__ long long red[kWarps];
   __shared__ long long s_loc[2];
   __shared__ int s_abort;
-  __shared__ int s_last[2];
-  // split of this launch and the CTA's split pieces, read by the consumers at
-  // piece boundaries only (keeps them out of the registers of the block loop)
-  __shared__ long long s_split[4];   // ppb, cost, total, s1
-  __shared__ long long s_pend[2][4];  // sequence, unit, unit start, blocks
-  __shared__ int s_npend;
-  __shared__ uint32_t s_newrow[kNC][6 * 32];  // fused append: each warp's new row
   uint8_t *ring = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
 
@@ -1101,120 +879,50 @@ attn_partition_kernel(const __grid_constant__ CUtensorMap kmap,
   const int R = p.stages;
 
   // ---------------------------------------------------------------- prologue
-  launch_dependents();      // let the next kernel be scheduled early
+  launch_dependents();      // let the merge kernel be scheduled early
   grid_dependency_wait();   // inputs may come from the previous kernel
+  // Total positions over all units, then this CTA's even share [s0, s1).
+  long long part = 0;
+  for (int b = threadIdx.x; b < B; b += kThreads) {
+    const int L = p.context_lens[b];
+    if (L < 0 || L > p.limit) {
+      if (c == 0) atomicOr(p.status, kErrContext);
+    } else {
+      part += unit_len((L + BS - 1) / BS, p);
+    }
+  }
+  const long long total = block_sum(part, red) * UH;
+  const long long s0 = cta_start(c, total, G), s1 = cta_start(c + 1, total, G);
+  if (s0 >= s1) return;  // same for every thread of the CTA
+
   if (threadIdx.x == 0) {
     s_loc[0] = -1;
     s_abort = 0;
-    s_npend = 0;
     for (int i = 0; i < R; ++i) {
       mbar_init(&full_bar[i], 1);
       mbar_init(&empty_bar[i], kNC);
     }
-    for (int i = 0; i < kNC; ++i) mbar_init(&merge_bar[i], 1);
     fence_barrier_init();
   }
-  if (warp == kNC) {
-    if (lane == 0) {
-      prefetch_tmap(&kmap);
-      prefetch_tmap(&vmap);
+  if (warp == kNC && lane == 0) {
+    prefetch_tmap(&kmap);
+    prefetch_tmap(&vmap);
+  }
+  __syncthreads();
+  // Sequence holding position s0 (chunked scan over the sequences).
+  long long run = 0;
+  for (int base = 0; base < B; base += kThreads) {
+    const int b = base + threadIdx.x;
+    const int ln = b < B ? unit_len(seq_blocks<BS>(p, b), p) : 0;
+    long long tot;
+    const long long excl = run + block_excl_scan(ln, red, &tot);
+    if (ln > 0 && excl * UH <= s0 && s0 < (excl + ln) * UH) {
+      s_loc[0] = b;
+      s_loc[1] = excl;
     }
-    // This CTA's share of the block tables into L2 (every CTA takes a share,
-    // at most 64 KB), so that the producers' table reads after the split
-    // below hit L2 instead of waiting on HBM.
-    const uintptr_t t0 = reinterpret_cast<uintptr_t>(p.block_tables) & ~static_cast<uintptr_t>(127);
-    const uintptr_t t1 = reinterpret_cast<uintptr_t>(p.block_tables + static_cast<int64_t>(B) * p.max_blocks);
-    const long long lines = static_cast<long long>((t1 - t0 + 127) >> 7);
-    const long long share = min((lines + G - 1) / G, 512ll);
-    for (long long l = c * share + lane; l < min((c + 1) * share, lines); l += 32)
-      prefetch_l2(reinterpret_cast<const void *>(t0 + (l << 7)));
-  }
-  // One prefix sum over the sequences gives every CTA the whole split: each
-  // sequence contributes its blocks and, if it has any, one unit start per
-  // unit. A single pass (one __syncthreads) when the batch fits the CTA.
-  long long my_excl = 0;  // packed prefix of this thread's sequence (one pass)
-  int my_nb = 0;
-  long long tot = 0;
-  if (B <= kThreads) {
-    if (threadIdx.x < B) {
-      const int L = p.context_lens[threadIdx.x];
-      if (L < 0 || L > p.limit) {
-        if (c == 0) atomicOr(p.status, kErrContext);
-      } else {
-        my_nb = (L + BS - 1) / BS;
-      }
-    }
-    my_excl = block_excl_scan<false>(pack_seq(my_nb), red, &tot);
-  } else {
-    for (int base = 0; base < B; base += kThreads) {
-      const int b = base + threadIdx.x;
-      int nb = 0;
-      if (b < B) {
-        const int L = p.context_lens[b];
-        if (L < 0 || L > p.limit) {
-          if (c == 0) atomicOr(p.status, kErrContext);
-        } else {
-          nb = (L + BS - 1) / BS;
-        }
-      }
-      long long t;
-      block_excl_scan<true>(pack_seq(nb), red, &t);
-      tot += t;
-    }
-  }
-  const long long TB = tot >> kUnitBits, NU = tot & kUnitMask;
-  Split sp;
-  if ((4 * TB + static_cast<long long>(p.unit_cost4) * NU) * UH >= 4 * G) {
-    sp.ppb = 4;
-    sp.cost = p.unit_cost4;
-  } else {
-    sp.ppb = 1;
-    sp.cost = (p.unit_cost4 + 3) / 4;
-  }
-  const long long total = (sp.ppb * TB + sp.cost * NU) * UH;
-  const long long s0 = cta_start(c, total, G), s1 = cta_start(c + 1, total, G);
-  if (threadIdx.x == 0) {  // visible to the consumers after the __syncthreads below
-    s_split[0] = sp.ppb;
-    s_split[1] = sp.cost;
-    s_split[2] = total;
-    s_split[3] = s1;
-  }
-  if (s0 >= s1) {  // no work: only this CTA's share of zero outputs (fused merge)
-    if (p.fuse_merge)
-      for (int b = c; b < B; b += static_cast<int>(G)) zero_sequence<D, Q_T>(p, b, threadIdx.x, kThreads);
-    return;  // same for every thread of the CTA
-  }
-  // Sequence holding position s0, and the position of its first unit.
-  auto seq_pos = [&](long long packed) {
-    return (sp.ppb * (packed >> kUnitBits) + sp.cost * (packed & kUnitMask)) * UH;
-  };
-  if (B <= kThreads) {
-    if (my_nb > 0) {
-      const long long lo = seq_pos(my_excl);
-      if (lo <= s0 && s0 < lo + unit_len(my_nb, sp) * UH) {
-        s_loc[0] = threadIdx.x;
-        s_loc[1] = lo;
-      }
-    }
+    run += tot;
     __syncthreads();
-  } else {
-    long long run = 0;
-    for (int base = 0; base < B; base += kThreads) {
-      const int b = base + threadIdx.x;
-      const int nb = b < B ? seq_blocks<BS>(p, b) : 0;
-      long long t;
-      const long long excl = run + block_excl_scan<true>(pack_seq(nb), red, &t);
-      if (nb > 0) {
-        const long long lo = seq_pos(excl);
-        if (lo <= s0 && s0 < lo + unit_len(nb, sp) * UH) {
-          s_loc[0] = b;
-          s_loc[1] = lo;
-        }
-      }
-      run += t;
-      __syncthreads();
-      if (s_loc[0] >= 0) break;
-    }
+    if (s_loc[0] >= 0) break;
   }
   if (s_loc[0] < 0) {  // lengths changed under the kernel: nothing consistent to do
     if (threadIdx.x == 0) atomicOr(p.status, kErrContext);
@@ -1224,16 +932,14 @@ attn_partition_kernel(const __grid_constant__ CUtensorMap kmap,
   w0.b = static_cast<int>(s_loc[0]);
   w0.nb = seq_blocks<BS>(p, w0.b);
   {
-    // s0 may fall on a unit's charged positions or inside a block's quarter
-    // positions: the walk begins at the first block that starts at or after it
-    const long long ln = unit_len(w0.nb, sp);
-    const long long off = s0 - s_loc[1];
+    // s0 may fall on the unit's start positions: the walk then begins at its
+    // first block (possibly past s1: nothing to do here)
+    const int ln = unit_len(w0.nb, p);
+    const long long off = s0 - s_loc[1] * UH;
     w0.gc = static_cast<int>(off / ln);
-    const long long r = off - static_cast<long long>(w0.gc) * ln;
-    const int j = r <= sp.cost ? 0 : static_cast<int>((r - sp.cost + sp.ppb - 1) / sp.ppb);
-    w0.j = j;
-    w0.pos = s_loc[1] + static_cast<long long>(w0.gc) * ln + sp.cost + static_cast<long long>(sp.ppb) * j;
-    if (w0.j == w0.nb) walk_next_unit<BS>(w0, sp, p);
+    const int jv = static_cast<int>(off - static_cast<long long>(w0.gc) * ln) - p.unit_cost;
+    w0.j = jv > 0 ? jv : 0;
+    w0.pos = s0 + (jv < 0 ? -jv : 0);
   }
 
   if (warp == kNC) {
@@ -1243,7 +949,7 @@ attn_partition_kernel(const __grid_constant__ CUtensorMap kmap,
     bool ok = true;
     while (w.pos < s1 && ok) {
       if (w.b >= B || w.nb <= 0) break;  // lengths changed under the kernel
-      const int seg = walk_seg(w, s1, sp);
+      const int seg = static_cast<int>(min(static_cast<long long>(w.nb - w.j), s1 - w.pos));
       const int head0 = (w.gc / p.cgroups) * p.hg;  // first kv head of the unit
       const int32_t *btrow = p.block_tables + static_cast<int64_t>(w.b) * p.max_blocks + w.j;
       for (int i0 = 0; i0 < seg && ok; i0 += 32) {
@@ -1277,7 +983,7 @@ attn_partition_kernel(const __grid_constant__ CUtensorMap kmap,
           ++k;
         }
       }
-      walk_advance<BS>(w, seg, sp, p);
+      walk_advance<BS>(w, seg, p);
     }
     if (!ok && lane == 0) {
       // aborted: let the loads still in flight land before the CTA can exit
@@ -1291,69 +997,38 @@ attn_partition_kernel(const __grid_constant__ CUtensorMap kmap,
   // Consumer warp `warp` owns slot `warp` of each unit: kv head hi = warp / cpg
   // of the unit's group, query-head chunk cl = warp % cpg. Every consumer visits
   // every position (an idle one only releases the stage).
-  if (p.k_new != nullptr) {  // the first piece's new rows into L2
-    const Slot s0l = slot_of(p, w0.gc, warp);
-    constexpr int kHalf = D * 2 / 128;  // 128-byte lines per new row
-    if (s0l.active && lane < 2 * kHalf)
-      prefetch_l2(static_cast<const char *>(lane < kHalf ? p.k_new : p.v_new) +
-                  (static_cast<int64_t>(w0.b) * p.kv_heads + s0l.g) * D * 2 + (lane % kHalf) * 128);
-  }
-  if (p.fuse_merge)  // zeros for empty / invalid sequences while the first stage loads
-    for (int b = c; b < B; b += static_cast<int>(G)) zero_sequence<D, Q_T>(p, b, threadIdx.x, kNC * 32);
   Consumer<D, BS, KV_T, Q_T> cs;
   Walk w = w0;
-  uint32_t k = 0;  // blocks consumed so far (the CTA's first piece has k == 0)
+  uint32_t k = 0;
   bool alive = true;
-  // the split, read from shared memory where it is used
-#define PKV_SPLIT_S1 (*reinterpret_cast<volatile long long *>(&s_split[3]))
-#define PKV_SPLIT_TOTAL (*reinterpret_cast<volatile long long *>(&s_split[2]))
-  auto split_now = [&]() {
-    Split r;
-    r.ppb = static_cast<int>(*reinterpret_cast<volatile long long *>(&s_split[0]));
-    r.cost = static_cast<int>(*reinterpret_cast<volatile long long *>(&s_split[1]));
-    return r;
-  };
-  while (w.pos < PKV_SPLIT_S1) {
+  int side = 0;  // the CTA's first piece goes to side 0, the others to side 1
+  while (w.pos < s1) {
     if (w.b >= B || w.nb <= 0) {  // same test as the producer: both stop here
       if (warp == 0 && lane == 0) atomicOr(p.status, kErrContext);
       break;
     }
-    const int seg = walk_seg(w, PKV_SPLIT_S1, split_now());
-    const Slot sl = slot_of(p, w.gc, warp);
-    const bool active = sl.active;
+    const int seg = static_cast<int>(min(static_cast<long long>(w.nb - w.j), s1 - w.pos));
+    const int hgi = w.gc / p.cgroups;
+    const int cgi = w.gc - hgi * p.cgroups;
+    const int cpg = min(p.cpg, p.chunks - cgi * p.cpg);
+    const bool active = warp < p.hg * cpg;
+    const int hi = active ? warp / cpg : 0;
+    const int cl = warp - hi * cpg;
+    const int g = hgi * p.hg + hi;
+    const int chunk = cgi * p.cpg + cl;
+    const int h0 = g * p.group + chunk * kChunkHeads;
+    const int nh = min(kChunkHeads, p.group - chunk * kChunkHeads);
     const int L = p.context_lens[w.b];
     // fused append: the new token (position L - 1) is in block jl of the unit;
     // with one query-head chunk per kv head this warp alone uses its rows
-    // (-1: none in this piece)
     const int jl = (L - 1) / BS;
-    const int jnew = (p.k_new != nullptr && active && L > 0 && jl >= w.j && jl < w.j + seg) ? jl : -1;
-    {
-      // the next unit's query rows (and new rows) into L2 while this piece streams
-      Walk wn = w;
-      walk_advance<BS>(wn, seg, split_now(), p);
-      if (wn.pos < PKV_SPLIT_S1 && wn.b < B) {
-        const Slot sn = slot_of(p, wn.gc, warp);
-        if (sn.active) {
-          const char *qr = static_cast<const char *>(p.q) +
-                           (static_cast<int64_t>(wn.b) * p.q_heads + sn.h0) * D * 2;
-          if (lane * 128 < sn.nh * D * 2) prefetch_l2(qr + lane * 128);
-          if (p.k_new != nullptr && lane < 2 * (D * 2 / 128)) {
-            constexpr int kHalf = D * 2 / 128;  // 128-byte lines per new row
-            const char *nrw = static_cast<const char *>(lane < kHalf ? p.k_new : p.v_new) +
-                              (static_cast<int64_t>(wn.b) * p.kv_heads + sn.g) * D * 2;
-            prefetch_l2(nrw + (lane % kHalf) * 128);
-          }
-        }
-      }
-    }
-    if (jnew >= 0) {  // loaded (and quantized) now, parked until its block arrives
-      NewRow<D, BS, KV_T, Q_T> nr;
-      nr.load(p, w.b, sl.g, lane);
-      nr.stash(s_newrow[warp], lane);
-    }
+    const bool has_new =
+        p.k_new != nullptr && active && L > 0 && jl >= w.j && jl < w.j + seg;
+    NewRow<D, BS, KV_T, Q_T> nr;
+    if (has_new) nr.load(p, w.b, g, lane);
     if (active) {
       cs.reset();
-      cs.load_query(p, w.b, sl.h0, sl.nh, lane);
+      cs.load_query(p, w.b, h0, nh, lane);
     }
     for (uint32_t kk = k; kk < k + seg; ++kk) {
       const int s = kk % R;
@@ -1370,82 +1045,33 @@ attn_partition_kernel(const __grid_constant__ CUtensorMap kmap,
           const int jb = w.j + static_cast<int>(kk - k);
           const int id = stage_id[s];
           const int valid = id >= 0 ? min(BS, L - jb * BS) : 0;
-          if (jb == jnew && id >= 0) {
-            const int rl = (L - 1) - jnew * BS;
-            NewRow<D, BS, KV_T, Q_T> nr;
-            nr.unstash(s_newrow[warp], lane);
-            nr.store(p, ring + s * stride, rows, sl.hi * BS + rl, id, sl.g, rl, lane);
+          if (has_new && jb == jl && id >= 0) {
+            const int rl = (L - 1) - jl * BS;
+            nr.store(p, ring + s * stride, rows, hi * BS + rl, id, g, rl, lane);
             // the producer's next TMA into this stage must come after these writes
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
           }
-          cs.block(ring + s * stride, rows, sl.hi, valid, lane);
+          cs.block(ring + s * stride, rows, hi, valid, lane);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty_bar[s]);
       }
     }
     // ------------------------------------------ end of the unit's piece here
-    const Split sp2 = split_now();
     const bool whole = (w.j == 0 && seg == w.nb);
-    const int side = k > 0 ? 1 : 0;  // the CTA's first piece is side 0, later ones side 1
     if (active) {
       const int64_t pbase = ((static_cast<int64_t>(c) * 2 + side) * kNC + warp) * kChunkHeads;
-      cs.finish(p, whole, w.b, sl.h0, sl.nh, pbase, alive, lane);
+      cs.finish(p, whole, w.b, h0, nh, pbase, alive, lane);
     }
-    if (warp == 0 && lane == 0) {
-      if (w.j == 0) {  // this CTA holds the unit's first block
-        const int nu =
-            cta_of(w.pos + static_cast<long long>(sp2.ppb) * (w.nb - 1), PKV_SPLIT_TOTAL, G) -
-            c + 1;
-        p.meta[static_cast<int64_t>(w.b) * UH + w.gc] = make_int4(c, nu, side, 0);
-      }
-      const int np = s_npend;
-      if (!whole && np < 2) {  // a CTA splits at most its first and its last piece
-        s_pend[np][0] = w.b;
-        s_pend[np][1] = w.gc;
-        s_pend[np][2] = w.pos - static_cast<long long>(sp2.ppb) * w.j - sp2.cost;
-        s_pend[np][3] = w.nb;
-        s_npend = np + 1;
-      }
+    if (warp == 0 && lane == 0 && w.j == 0) {  // this CTA holds the unit's first block
+      const int nu = cta_of(w.pos + w.nb - 1, total, G) - c + 1;
+      p.meta[static_cast<int64_t>(w.b) * UH + w.gc] = make_int4(c, nu, side, 0);
     }
     k += seg;
-    walk_advance<BS>(w, seg, sp2, p);
+    side = 1;
+    walk_advance<BS>(w, seg, p);
   }
-
-  // ------------------------------------------------ merge of split units
-  // Each CTA arrives once per split piece after publishing its partials; the
-  // arrival that completes a unit merges it, here, while the other CTAs'
-  // streams finish. Only consumer warps take part (named barrier 1).
-  if (p.fuse_merge) {
-    const Split sp2 = split_now();
-    const long long total2 = PKV_SPLIT_TOTAL;
-    __threadfence();  // this lane's partial stores, before the arrival below
-    bar_sync(1, kNC * 32);  // also makes s_pend / s_npend visible
-    const int npend = s_npend;
-    if (warp == 0 && lane == 0) {
-      const bool ok = !s_abort;
-      for (int i = 0; i < npend; ++i) {
-        const long long first = s_pend[i][2] + sp2.cost;
-        const int nu =
-            cta_of(first + static_cast<long long>(sp2.ppb) * (s_pend[i][3] - 1), total2, G) -
-            cta_of(first, total2, G) + 1;
-        s_last[i] = ok && arrive_last(p.counters + s_pend[i][0] * UH + s_pend[i][1], p.epoch, nu,
-                                      p.status);
-      }
-      __threadfence();  // the other pieces, before they are read
-    }
-    bar_sync(1, kNC * 32);
-    const int region = p.merge_region;
-    uint32_t phase = 0;
-    for (int i = 0; i < npend; ++i)
-      if (s_last[i])
-        merge_unit<D, BS, Q_T>(p, static_cast<int>(s_pend[i][0]), static_cast<int>(s_pend[i][1]),
-                               s_pend[i][2], static_cast<int>(s_pend[i][3]), sp2, total2, G,
-                               ring + warp * region, region, &merge_bar[warp], phase, warp, lane);
-  }
-#undef PKV_SPLIT_S1
-#undef PKV_SPLIT_TOTAL
 }
 
 // ============================================================================
@@ -1522,11 +1148,22 @@ __global__ void __launch_bounds__(kMergeWarps * 32) attn_merge_kernel(const Attn
       }
     }
 #pragma unroll
-    for (int k = 0; k < kBatch; ++k)
-      if (i0 + k < nu) combine_piece<E>(M, Ls, acc, ml[k].x, ml[k].y, o[k]);
-  }
+    for (int k = 0; k < kBatch; ++k) {
+      if (i0 + k < nu) {
+        const float Mn = fmaxf(M, ml[k].x);
+        if (Mn != -INFINITY) {
+          const float a = exp2_rel(M, Mn), wt = exp2_rel(ml[k].x, Mn);
+          Ls = Ls * a + ml[k].y * wt;
 #pragma unroll
-  for (int e = 0; e < E; ++e) store_out<OUT_T>(p.out, orow + e, merged_value(acc[e], Ls));
+          for (int e = 0; e < E; ++e) acc[e] = acc[e] * a + o[k][e] * wt;
+          M = Mn;
+        }
+      }
+    }
+  }
+  const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+#pragma unroll
+  for (int e = 0; e < E; ++e) store_out<OUT_T>(p.out, orow + e, acc[e] * inv);
 }
 
 // ============================================================================
@@ -1538,8 +1175,7 @@ using PartFn = cudaError_t (*)(const CUtensorMap &, const CUtensorMap &, const A
 template <int D, int BS, int KV_T, int Q_T>
 cudaError_t launch_part(const CUtensorMap &km, const CUtensorMap &vm, const AttnParams &p,
                         cudaStream_t st) {
-  // the ring, which the fused merge reuses as kNC regions of merge_region bytes
-  const int smem = std::max(p.stages * p.stage_bytes, kNC * p.merge_region) + 1024;
+  const int smem = p.stages * p.stage_bytes + 1024;
   auto kern = attn_partition_kernel<D, BS, KV_T, Q_T>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -1623,32 +1259,19 @@ UnitGeom unit_geom(const kv_pool *pool, int num_q_heads) {
   return u;
 }
 
-// Workspace: unit metadata, unit arrival counters, then per-CTA partials
-// (two sides x kNC slots x 8 heads).
+// Workspace: unit metadata, then per-CTA partials (two sides x kNC slots x 8 heads).
 struct WsLayout {
-  uint64_t meta_off, ctr_off, ml_off, o_off, total;
+  uint64_t meta_off, ml_off, o_off, total;
 };
 
 WsLayout ws_layout(int B, int units_per_seq, int G, int D) {
   WsLayout w{};
   const uint64_t recs = static_cast<uint64_t>(G) * 2 * kNC * kChunkHeads;
-  const uint64_t units = static_cast<uint64_t>(B) * units_per_seq;
   w.meta_off = 0;
-  w.ctr_off = round_up(units * 16, 256);
-  w.ml_off = w.ctr_off + round_up(units * 8, 256);
+  w.ml_off = round_up(static_cast<uint64_t>(B) * units_per_seq * 16, 256);
   w.o_off = w.ml_off + round_up(recs * 2 * 4, 256);
   w.total = w.o_off + round_up(recs * D * 4, 256);
   return w;
-}
-
-// Launch epochs for the fused merge's arrival counters: nonzero and never
-// all ones, so neither zeroed nor 0xFF-filled memory looks like a live count.
-std::atomic<uint32_t> g_epoch{0};
-uint32_t next_epoch() {
-  for (;;) {
-    const uint32_t e = g_epoch.fetch_add(1, std::memory_order_relaxed) + 1;
-    if (e != 0u && e != 0xffffffffu) return e;
-  }
 }
 
 kv_status sm_count(int *n) {
@@ -1705,7 +1328,6 @@ kv_status fill_params(kv_pool *pool, int layer, const void *q, int num_seqs, int
   p.v_scale = layer >= 0 ? layer_vs(pool, layer) : nullptr;
   char *ws = static_cast<char *>(workspace);
   p.meta = reinterpret_cast<int4 *>(ws + wl.meta_off);
-  p.counters = reinterpret_cast<unsigned long long *>(ws + wl.ctr_off);
   p.part_ml = reinterpret_cast<float *>(ws + wl.ml_off);
   p.part_o = reinterpret_cast<float *>(ws + wl.o_off);
   p.status = status_word(pool);
@@ -1721,13 +1343,9 @@ kv_status fill_params(kv_pool *pool, int layer, const void *q, int num_seqs, int
   p.units_per_seq = u.units_per_seq;
   p.stage_bytes = u.stage_bytes;
   p.stages = u.stages;
-  // per consumer warp: its share of the ring, but room for at least one piece
-  // (8 heads x (head_dim + 2) fp32) however small the ring
-  p.merge_region = std::max((u.stages * u.stage_bytes / kNC) & ~1023,
-                            static_cast<int>(round_up(kChunkHeads * (D + 2) * 4, 1024)));
   // starting a unit (query load, partial write) costs about as much as
-  // streaming 64 KB on one SM: charged as that many quarter blocks
-  p.unit_cost4 = std::max(1, std::min(32, (4 * 64 * 1024 + u.stage_bytes / 2) / u.stage_bytes));
+  // streaming 192 KB on one SM: charged as that many blocks in the split
+  p.unit_cost = std::max(1, std::min(8, (192 * 1024 + u.stage_bytes / 2) / u.stage_bytes));
   p.max_blocks = max_blocks_per_seq;
   p.num_blocks = pool->d.num_blocks;
   const int64_t tbl_cap = static_cast<int64_t>(max_blocks_per_seq) * pool->d.block_size;
@@ -1741,7 +1359,7 @@ kv_status run_partition(kv_pool *pool, int32_t layer, const void *q, int32_t q_d
                         int32_t max_blocks_per_seq, const int32_t *context_lens,
                         int32_t max_context, float scale, void *out, int32_t num_ctas,
                         void *workspace, uint64_t workspace_bytes, const void *k_new,
-                        const void *v_new, bool fuse_merge, cudaStream_t st) {
+                        const void *v_new, cudaStream_t st) {
   if (!pool) return fail(KV_ERR_INVALID, "null pool");
   if (layer < 0 || layer >= pool->d.num_layers) return fail(KV_ERR_INVALID, "layer %d out of range", layer);
   const int cd = pool->d.cache_dtype;
@@ -1781,8 +1399,6 @@ kv_status run_partition(kv_pool *pool, int32_t layer, const void *q, int32_t q_d
     p.v_scale_w = layer_vs(pool, layer);
   }
   if (num_seqs == 0) return KV_OK;
-  p.fuse_merge = fuse_merge ? 1 : 0;
-  p.epoch = fuse_merge ? next_epoch() : 0u;
   kv_status code;
   LayerMaps maps;
   if (!layer_maps(pool, layer, p.hg * pool->d.block_size, &maps, &code)) return code;
@@ -1846,8 +1462,7 @@ kv_status paged_attn_partition(kv_pool *pool, int32_t layer, const void *q, int3
                                void *workspace, uint64_t workspace_bytes, kv_stream_t stream) {
   kv_status s = run_partition(pool, layer, q, q_dtype, num_seqs, num_q_heads, block_tables,
                               max_blocks_per_seq, context_lens, max_context, scale, out, num_ctas,
-                              workspace, workspace_bytes, nullptr, nullptr, false,
-                              (cudaStream_t)stream);
+                              workspace, workspace_bytes, nullptr, nullptr, (cudaStream_t)stream);
   return s == KV_OK ? ok() : s;
 }
 
@@ -1861,8 +1476,7 @@ kv_status paged_attn_partition_append(kv_pool *pool, int32_t layer, const void *
   if (num_seqs > 0 && (!k_new || !v_new)) return fail(KV_ERR_INVALID, "null k_new / v_new");
   kv_status s = run_partition(pool, layer, q, q_dtype, num_seqs, num_q_heads, block_tables,
                               max_blocks_per_seq, context_lens, max_context, scale, out, num_ctas,
-                              workspace, workspace_bytes, k_new, v_new, false,
-                              (cudaStream_t)stream);
+                              workspace, workspace_bytes, k_new, v_new, (cudaStream_t)stream);
   return s == KV_OK ? ok() : s;
 }
 
@@ -1881,12 +1495,16 @@ kv_status paged_attn_decode(kv_pool *pool, int32_t layer, const void *q, int32_t
                             int32_t max_blocks_per_seq, const int32_t *context_lens,
                             int32_t max_context, float scale, void *out, int32_t num_ctas,
                             void *workspace, uint64_t workspace_bytes, kv_stream_t stream) {
-  // one launch: the attention kernel merges split units itself
   kv_status s = run_partition(pool, layer, q, q_dtype, num_seqs, num_q_heads, block_tables,
                               max_blocks_per_seq, context_lens, max_context, scale, out, num_ctas,
-                              workspace, workspace_bytes, nullptr, nullptr, true,
-                              (cudaStream_t)stream);
-  return s == KV_OK ? ok() : s;
+                              workspace, workspace_bytes, nullptr, nullptr, (cudaStream_t)stream);
+  if (s != KV_OK) return s;
+  if (num_seqs > 0) {
+    s = run_merge(pool, num_seqs, num_q_heads, context_lens, max_blocks_per_seq, max_context,
+                  num_ctas, q_dtype, out, workspace, workspace_bytes, (cudaStream_t)stream);
+    if (s != KV_OK) return s;
+  }
+  return ok();
 }
 
 kv_status paged_attn_decode_append(kv_pool *pool, int32_t layer, const void *q,
@@ -1899,9 +1517,14 @@ kv_status paged_attn_decode_append(kv_pool *pool, int32_t layer, const void *q,
   if (num_seqs > 0 && (!k_new || !v_new)) return fail(KV_ERR_INVALID, "null k_new / v_new");
   kv_status s = run_partition(pool, layer, q, q_dtype, num_seqs, num_q_heads, block_tables,
                               max_blocks_per_seq, context_lens, max_context, scale, out, num_ctas,
-                              workspace, workspace_bytes, k_new, v_new, true,
-                              (cudaStream_t)stream);
-  return s == KV_OK ? ok() : s;
+                              workspace, workspace_bytes, k_new, v_new, (cudaStream_t)stream);
+  if (s != KV_OK) return s;
+  if (num_seqs > 0) {
+    s = run_merge(pool, num_seqs, num_q_heads, context_lens, max_blocks_per_seq, max_context,
+                  num_ctas, q_dtype, out, workspace, workspace_bytes, (cudaStream_t)stream);
+    if (s != KV_OK) return s;
+  }
+  return ok();
 }
 
 }  // extern "C"
@@ -1983,9 +1606,8 @@ extern "C" kv_status paged_attn_decode_static(kv_pool *pool, int32_t layer, cons
   void *ws = nullptr;
   s = scratch_address((cudaStream_t)stream, &ws);
   if (s != KV_OK) return s;
-  // Nothing in the scratch needs to start at zero: the kernel writes every
-  // bookkeeping entry and partial before it reads it, and its arrival counters
-  // carry the tag of the launch that wrote them (a stale one counts as zero).
+  // Nothing in the scratch needs to start at zero: the partition kernel writes
+  // every bookkeeping entry and partial that the merge kernel then reads.
   return paged_attn_decode(pool, layer, q, q_dtype, num_seqs, num_q_heads, block_tables,
                            max_blocks_per_seq, context_lens, max_context, scale, out, num_ctas,
                            ws, kStaticScratchBytes, stream);

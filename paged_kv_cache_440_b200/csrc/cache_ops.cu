@@ -13,8 +13,9 @@
 // * Block copy: the copy half of copy-on-write [bjdmk.com.cn/news/6246348,
 //   §3.2]: whole blocks, every layer, K, V and scales.
 //
-// All three are pure data movement at a few hundred KB per decode step; each
-// warp handles one row (or one block) with 16-byte vector accesses.
+// All three are pure data movement at a few hundred KB per decode step; a
+// warp handles one token's rows (or a CTA one block region) with 16-byte
+// vector accesses, its loads in flight together before its stores.
 #include <cstring>
 #include <vector>
 
@@ -30,45 +31,64 @@ constexpr int kWarpsPerCta = 8;
 
 // ---------------------------------------------------------------- 16-bit copy
 
-// One warp per (token, kv head): lanes [0, 16) copy the K row, [16, 32) the V
-// row, 16 bytes each (row_bytes <= 256).
+// Up to this many 16-byte chunks per lane are loaded before any is stored, so
+// a warp has all of them in flight at once (one memory round trip per batch).
+constexpr int kBatch = 8;
+
+// One warp per token: the K and V rows of all its kv heads (2 * kv_heads *
+// row_chunks 16-byte chunks), spread over the lanes.
 __global__ void __launch_bounds__(kWarpsPerCta * 32)
 append16_kernel(const uint4 *__restrict__ k_new, const uint4 *__restrict__ v_new,
                 const int64_t *__restrict__ slots, int num_tokens, int kv_heads,
-                int block_size, int row_chunks, int64_t num_slots, char *__restrict__ kc,
-                char *__restrict__ vc, int *status) {
+                int block_size, int row_chunks, int64_t num_slots, uint4 *__restrict__ kc,
+                uint4 *__restrict__ vc, int *status) {
   launch_dependents();
   grid_dependency_wait();
-  const int warp = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
+  const int t = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (warp >= num_tokens * kv_heads) return;
-  const int t = warp / kv_heads;
-  const int h = warp - t * kv_heads;
+  if (t >= num_tokens) return;
+  const int per_kv = kv_heads * row_chunks;  // chunks of one token's K (or V)
+  const int n = 2 * per_kv;
   const int64_t slot = slots[t];
-  if (slot < 0) return;
-  if (slot >= num_slots) {
-    if (lane == 0 && h == 0) atomicOr(status, kErrSlot);
-    return;
-  }
-  const int64_t blk = slot / block_size;
-  const int row = static_cast<int>(slot - blk * block_size);
-  const int64_t dst_row = (blk * kv_heads + h) * block_size + row;
-  const int c = lane & 15;
-  if (c >= row_chunks) return;
-  const int64_t src_row = static_cast<int64_t>(t) * kv_heads + h;
-  if (lane < 16) {
-    uint4 x = k_new[src_row * row_chunks + c];
-    reinterpret_cast<uint4 *>(kc)[dst_row * row_chunks + c] = x;
-  } else {
-    uint4 x = v_new[src_row * row_chunks + c];
-    reinterpret_cast<uint4 *>(vc)[dst_row * row_chunks + c] = x;
+  int64_t blk = 0;
+  int row = 0;
+  for (int i0 = 0; i0 < n; i0 += kBatch * 32) {
+    uint4 x[kBatch];
+    // the rows do not depend on the slot: their loads go out with its load
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = i0 + u * 32 + lane;
+      if (i < n) {
+        const int j = i < per_kv ? i : i - per_kv;  // head * row_chunks + chunk
+        x[u] = (i < per_kv ? k_new : v_new)[static_cast<int64_t>(t) * per_kv + j];
+      }
+    }
+    if (i0 == 0) {
+      if (slot < 0) return;
+      if (slot >= num_slots) {
+        if (lane == 0) atomicOr(status, kErrSlot);
+        return;
+      }
+      blk = slot / block_size;
+      row = static_cast<int>(slot - blk * block_size);
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = i0 + u * 32 + lane;
+      if (i < n) {
+        const int j = i < per_kv ? i : i - per_kv;
+        const int h = j / row_chunks, c = j - h * row_chunks;
+        (i < per_kv ? kc : vc)[((blk * kv_heads + h) * block_size + row) * row_chunks + c] = x[u];
+      }
+    }
   }
 }
 
 // ---------------------------------------------------------------- quantize
 
 // One warp per (token, kv head): quantize the K row and the V row, store the
-// codes and scales at the slot.
+// codes and scales at the slot. The rows are loaded together with the slot
+// (they do not depend on it), so the warp waits on memory once.
 template <int D, int IN_T, int OUT_T>
 __global__ void __launch_bounds__(kWarpsPerCta * 32)
 append_quant_kernel(const uint16_t *__restrict__ k_new, const uint16_t *__restrict__ v_new,
@@ -83,7 +103,11 @@ append_quant_kernel(const uint16_t *__restrict__ k_new, const uint16_t *__restri
   if (warp >= num_tokens * kv_heads) return;
   const int t = warp / kv_heads;
   const int h = warp - t * kv_heads;
+  const int64_t src_row = static_cast<int64_t>(t) * kv_heads + h;
+  float xk[D / 32], xv[D / 32];
   const int64_t slot = slots[t];
+  load_row<D, IN_T>(k_new + src_row * D, lane, xk);
+  load_row<D, IN_T>(v_new + src_row * D, lane, xv);
   if (slot < 0) return;
   if (slot >= num_slots) {
     if (lane == 0 && h == 0) atomicOr(status, kErrSlot);
@@ -92,22 +116,18 @@ append_quant_kernel(const uint16_t *__restrict__ k_new, const uint16_t *__restri
   const int64_t blk = slot / block_size;
   const int row = static_cast<int>(slot - blk * block_size);
   const int64_t dst_row = (blk * kv_heads + h) * block_size + row;
-  const int64_t src_row = static_cast<int64_t>(t) * kv_heads + h;
   // INT8_KCHAN: ks holds the layer's [kv_heads][D] channel scales
   constexpr int VQ = OUT_T == KV_INT8_KCHAN ? KV_INT8 : OUT_T;  // value coding
-  float x[D / 32];
-  float scale;
-  load_row<D, IN_T>(k_new + src_row * D, lane, x);
   constexpr int kRow = OUT_T == KV_INT4 ? D / 2 : D;  // bytes per row
+  float scale;
   if constexpr (OUT_T == KV_INT8_KCHAN) {
-    store_codes<D, KV_INT8>(kc + dst_row * kRow, lane, quantize_row_chan<D>(x, ks + h * D, lane));
+    store_codes<D, KV_INT8>(kc + dst_row * kRow, lane, quantize_row_chan<D>(xk, ks + h * D, lane));
   } else {
-    const uint32_t packed = quantize_row<D, OUT_T>(x, &scale);
+    const uint32_t packed = quantize_row<D, OUT_T>(xk, &scale);
     store_codes<D, OUT_T>(kc + dst_row * kRow, lane, packed);
     if (OUT_T != KV_FP8_E5M2_CAST && lane == 0) ks[dst_row] = scale;
   }
-  load_row<D, IN_T>(v_new + src_row * D, lane, x);
-  const uint32_t vpacked = quantize_row<D, VQ>(x, &scale);
+  const uint32_t vpacked = quantize_row<D, VQ>(xv, &scale);
   store_codes<D, VQ>(vc + dst_row * kRow, lane, vpacked);
   if (VQ != KV_FP8_E5M2_CAST && lane == 0) vs[dst_row] = scale;
 }
@@ -158,7 +178,16 @@ block_copy_kernel(const __grid_constant__ CopyPairs pairs, char *__restrict__ ba
   const uint4 *src = reinterpret_cast<const uint4 *>(rb + (uint64_t)pairs.src[i] * bytes);
   uint4 *dst = reinterpret_cast<uint4 *>(rb + (uint64_t)pairs.dst[i] * bytes);
   const uint32_t n = bytes / 16;
-  for (uint32_t j = threadIdx.x; j < n; j += blockDim.x) dst[j] = src[j];
+  // every load of a batch before its stores: one round trip per batch
+  for (uint32_t j0 = threadIdx.x; j0 < n; j0 += kBatch * blockDim.x) {
+    uint4 x[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u)
+      if (j0 + u * blockDim.x < n) x[u] = src[j0 + u * blockDim.x];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u)
+      if (j0 + u * blockDim.x < n) dst[j0 + u * blockDim.x] = x[u];
+  }
 }
 
 template <int D, int IN_T, int OUT_T>
@@ -173,7 +202,7 @@ cudaError_t launch_quantize(const void *x, int64_t rows, void *codes, float *sca
 template <int D, int IN_T, int OUT_T>
 cudaError_t launch_append_quant(kv_pool *p, int layer, const void *k, const void *v,
                                 const int64_t *slots, int T, cudaStream_t st) {
-  const int64_t warps = (int64_t)T * p->d.num_kv_heads;
+  const int64_t warps = static_cast<int64_t>(T) * p->d.num_kv_heads;
   const int64_t grid = (warps + kWarpsPerCta - 1) / kWarpsPerCta;
   cudaError_t e = launch_pdl(
       append_quant_kernel<D, IN_T, OUT_T>, dim3((unsigned)grid), dim3(kWarpsPerCta * 32), 0, st,
@@ -221,21 +250,19 @@ kv_status kv_append(kv_pool *pool, int32_t layer, const void *k_new, const void 
     return fail(KV_ERR_INVALID, "k_new / v_new must be 16-byte aligned, slot_mapping 8-byte");
   if (in_dtype != KV_BF16 && in_dtype != KV_FP16)
     return fail(KV_ERR_UNSUPPORTED, "in_dtype must be KV_BF16 or KV_FP16");
-  const int64_t warps = (int64_t)num_tokens * pool->d.num_kv_heads;
-  if ((warps + kWarpsPerCta - 1) / kWarpsPerCta > 0x7FFFFFFF)
-    return fail(KV_ERR_INVALID, "too many tokens");
   cudaStream_t st = (cudaStream_t)stream;
   const int cd = pool->d.cache_dtype;
   cudaError_t e;
   if (!is_quant(cd)) {
     if (in_dtype != cd)
       return fail(KV_ERR_UNSUPPORTED, "a 16-bit cache takes rows of its own dtype");
-    const int64_t grid = (warps + kWarpsPerCta - 1) / kWarpsPerCta;
+    const int64_t grid = (static_cast<int64_t>(num_tokens) + kWarpsPerCta - 1) / kWarpsPerCta;
     e = launch_pdl(append16_kernel, dim3((unsigned)grid), dim3(kWarpsPerCta * 32), 0, st,
                    static_cast<const uint4 *>(k_new), static_cast<const uint4 *>(v_new),
                    slot_mapping, num_tokens, pool->d.num_kv_heads, pool->d.block_size,
                    pool->row_bytes / 16, (int64_t)pool->d.num_blocks * pool->d.block_size,
-                   layer_k(pool, layer), layer_v(pool, layer), status_word(pool));
+                   reinterpret_cast<uint4 *>(layer_k(pool, layer)),
+                   reinterpret_cast<uint4 *>(layer_v(pool, layer)), status_word(pool));
     if (e == cudaSuccess) e = cudaGetLastError();
   } else if (cd == KV_INT8) {
     e = in_dtype == KV_BF16

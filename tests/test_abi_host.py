@@ -196,13 +196,12 @@ def test_attention_argument_validation_and_workspace_size():
         # Hq must be a multiple of Hkv
         assert B.lib.paged_attn_workspace_bytes(h, 4, 3, 10, ctypes.byref(n)) == B.KV_ERR_INVALID
         assert B.lib.paged_attn_workspace_bytes(h, 4, 8, -1, ctypes.byref(n)) == B.KV_ERR_INVALID
-        # 16 B of bookkeeping and an 8-byte arrival counter per unit (here one
-        # unit per sequence: both kv heads in one group) plus 10 CTAs x 2 sides x
-        # 8 slots x 8 heads x (64 + 2) fp32, 256-aligned parts
+        # 16 B per unit (here one unit per sequence: both kv heads in one group)
+        # plus 10 CTAs x 2 sides x 8 slots x 8 heads x (64 + 2) fp32, 256-aligned parts
         B.check(B.lib.paged_attn_workspace_bytes(h, 4, 8, 10, ctypes.byref(n)))
         r256 = lambda x: -(-x // 256) * 256
         recs = 10 * 2 * 8 * 8
-        want = r256(4 * 1 * 16) + r256(4 * 1 * 8) + r256(recs * 2 * 4) + r256(recs * 64 * 4)
+        want = r256(4 * 1 * 16) + r256(recs * 2 * 4) + r256(recs * 64 * 4)
         assert n.value == want
         # 16 query heads per kv head (two 8-head chunks): still one unit per sequence
         B.check(B.lib.paged_attn_workspace_bytes(h, 4, 32, 10, ctypes.byref(n)))

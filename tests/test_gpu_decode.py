@@ -410,10 +410,9 @@ def test_decode_whatever_the_workspace_held(pkv, name, make, G):
 
 
 def test_decode_graph_replays_match(pkv):
-    """A decode step captured in a CUDA graph replays with the same launch (the
-    same arrival-counter epoch) every time: the CTA that merges a split unit
-    resets its counter, so each replay merges again and gives the same bits as
-    a direct call (and as the separate partition + merge kernels)."""
+    """A decode step captured in a CUDA graph (both kernels, launched so that
+    the merge may start while the attention kernel drains) gives, replay after
+    replay, the bits of the separate partition + merge calls."""
     wl = W.gqa70b(DEV, batch=12)
     pool = build_pool(pkv, wl, DEV)
     tables, lens = device_inputs(wl, DEV)
