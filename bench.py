@@ -490,7 +490,6 @@ def run_prefill(args, rank, world, device):
         for i in range(args.warmup + max(10, args.steps // 10)):
             torch.sum(flush, 0, out=sink)
             torch.cuda.synchronize(device)
-            hold_gpu(300e-6)
             a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
             d_q.copy_(h_q, non_blocking=True)
@@ -708,7 +707,6 @@ def run_ours(args, rank, world, device):
         for i in range(args.warmup + n_e2e):
             flush_l2()
             torch.cuda.synchronize(device)
-            hold_gpu(300e-6)    # the whole step is enqueued before the GPU reaches it
             a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
             d_in.copy_(h_in, non_blocking=True)

@@ -38,7 +38,11 @@
 //   M, the probabilities turned from accumulator to operand layout by an
 //   in-register 8x8 transpose and fed as two 16-bit parts (hi + lo) so P V
 //   keeps fp32-level accuracy. Online softmax in fp32 (base 2) per head.
-// * INT8 / E5M2 codes convert exactly to fp16 in registers; per-token K scales
+// * INT8 and INT4 keys meet the query on the 8-bit integer tensor core
+//   (m16n8k32, int32 accumulation): the key codes enter as stored (INT4 as
+//   offset nibbles), the query as two exact signed 8-bit digits of its value
+//   against the head's absmax, so no key code is converted. E5M2 keys and all
+//   value codes convert exactly to fp16 in registers. Per-token K scales
 //   multiply the scores, per-token V scales are folded into the softmax
 //   weights through log2(scale) so the fp16 weights stay within (0, 1].
 #include <algorithm>
@@ -98,8 +102,6 @@ struct AttnParams {
   int limit;           // valid lengths: 0 < L <= min(max_context, max_blocks * bs)
   int num_ctas;
 };
-
-constexpr int align_up_c(int x, int a) { return (x + a - 1) / a * a; }
 
 template <int KV_T>
 constexpr bool is16() {
@@ -173,10 +175,6 @@ __device__ __forceinline__ float warp_max_xor(float v, int from) {
 // exp2(x - m) with exp2(-inf) = 0 and no NaN when both are -inf.
 __device__ __forceinline__ float exp2_rel(float x, float m) {
   return x == -INFINITY ? 0.f : exp2f(x - m);
-}
-// Rescale factor exp2(m_old - m_new), 1 while nothing has been seen.
-__device__ __forceinline__ float rescale(float m_old, float m_new) {
-  return m_new == -INFINITY ? 1.f : exp2f(m_old - m_new);
 }
 
 // The SFU's base-2 exponential and logarithm (relative error about 2^-22,
@@ -292,13 +290,17 @@ struct Consumer {
   static constexpr int MT = BS / 16;  // 16-token tiles per block
   static constexpr bool KCH = (KV_T == KV_INT8_KCHAN);  // keys with channel scales
   static constexpr bool kInt8Codes = (KV_T == KV_INT8 || KCH);  // INT8 codes (K and V)
+  // integer keys (INT8, INT4) meet the query on the 8-bit integer tensor core:
+  // the query as three signed 8-bit digits, int32 accumulation
+  static constexpr bool kIntK = kInt8Codes || KV_T == KV_INT4;
+  static constexpr int kDig = 3;
 
   float m_run[2], m2_run[2], l_run[2];
   float oacc[D / 16][4];
-  uint32_t qb[KS][2];
-  uint32_t qlo[KCH ? KS : 1][2];  // INT8_KCHAN: the query's low parts (hi + lo ~ fp32)
+  uint32_t qb[kIntK ? 1 : KS][2];           // 16-bit query operands (fp16 / bf16 MMA)
+  uint32_t qi[kIntK ? D / 32 : 1][2][kDig];  // [k32 step][b0 / b1][digit, most significant first]
+  float qcf[2];  // INT4: what the offset codes add to each score column
   float s_fac[2];
-  float qcorr[2];  // INT8 keys enter the MMA as 1152 + code: 1152 * sum(q) per head
 
   __device__ __forceinline__ void reset() {
     m_run[0] = m_run[1] = m2_run[0] = m2_run[1] = -INFINITY;
@@ -322,28 +324,94 @@ struct Consumer {
         qb[ks][0] = hv ? q32[(qrow + 16 * ks + 2 * cq) >> 1] : 0u;
         qb[ks][1] = hv ? q32[(qrow + 16 * ks + 8 + 2 * cq) >> 1] : 0u;
       }
+    } else if constexpr (kIntK) {
+      // Three signed 8-bit digits per query value: x = rint(q * qs) with
+      // qs = 127 * 2^16 / max|q| of the head (about 23 bits, as fp32 holds
+      // q), split as x = 2^16 h + 2^8 m + l (h in [-127, 127], m and l in
+      // [-128, 127]). The key codes enter as they are stored (INT8), or as
+      // offset nibbles code + 8 (INT4, unsigned), so each digit's dot product
+      // is exact in int32 and a score is (2^16 acc_h + 2^8 acc_m + acc_l) / qs
+      // (INT4: less 8 * the same combination of the digit sums). Two digits
+      // (15 bits) measured up to 2e-2 relative error on near-zero outputs of
+      // per-channel keys; three keep it near 1e-5.
+      // B fragment of k32 step kp: lane (gq, cq) holds 4 k-slots of head gq
+      // in each half; INT8 slot (kp, half, e) is dim 32kp + 16half + 4cq + e;
+      // INT4 nibbles split into even and odd dims, slot (kp, half, e) is dim
+      // 64(kp / 2) + 32half + 8cq + 2e + kp % 2.
+      float qv[D / 32][2][4];
+      float amax = 0.f;
+#pragma unroll
+      for (int kp = 0; kp < D / 32; ++kp)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int dim = KV_T == KV_INT4 ? (kp >> 1) * 64 + 32 * hf + 8 * cq + 2 * e + (kp & 1)
+                                            : 32 * kp + 16 * hf + 4 * cq + e;
+            float v = hv ? load_q<Q_T>(p.q, qrow + dim) : 0.f;
+            if constexpr (KCH) {
+              // keys code k / s_c: the channel scale moves to the query,
+              // q . k = sum_c (q_c s_c) code_c
+              v *= p.k_scale[(h0 / p.group) * D + dim];
+            }
+            qv[kp][hf][e] = v;
+            amax = fmaxf(amax, fabsf(v));
+          }
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+      const float qs = amax > 0.f ? __fdiv_rn(8323072.f, amax) : 0.f;  // 127 * 2^16
+      int dsum[kDig] = {0, 0, 0};
+#pragma unroll
+      for (int kp = 0; kp < D / 32; ++kp)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t w[kDig] = {0u, 0u, 0u};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int x = __float2int_rn(qv[kp][hf][e] * qs);
+            const int h = (x + 32896) >> 16;  // floors: h in [-127, 127]
+            const int r = x - (h << 16);       // [-32896, 32639]
+            const int m = (r + 128) >> 8;      // [-128, 127]
+            const int l = r - (m << 8);        // [-128, 127]
+            w[0] |= (static_cast<uint32_t>(h) & 0xFFu) << (8 * e);
+            w[1] |= (static_cast<uint32_t>(m) & 0xFFu) << (8 * e);
+            w[2] |= (static_cast<uint32_t>(l) & 0xFFu) << (8 * e);
+            dsum[0] += h;
+            dsum[1] += m;
+            dsum[2] += l;
+          }
+#pragma unroll
+          for (int d = 0; d < kDig; ++d) qi[kp][hf][d] = w[d];
+        }
+      // the score columns of this lane are heads 2cq and 2cq+1
+      const float f = qs > 0.f ? __fdiv_rn(p.scale_log2, qs) : 0.f;
+      s_fac[0] = __shfl_sync(0xffffffffu, f, (2 * cq) * 4);
+      s_fac[1] = __shfl_sync(0xffffffffu, f, (2 * cq + 1) * 4);
+      if constexpr (KV_T == KV_INT4) {
+#pragma unroll
+        for (int d = 0; d < kDig; ++d) {
+          dsum[d] += __shfl_xor_sync(0xffffffffu, dsum[d], 1);
+          dsum[d] += __shfl_xor_sync(0xffffffffu, dsum[d], 2);
+        }
+        const float corr = 8.f * fmaf(static_cast<float>(dsum[0]), 65536.f,
+                                      fmaf(static_cast<float>(dsum[1]), 256.f,
+                                           static_cast<float>(dsum[2])));
+        qcf[0] = __shfl_sync(0xffffffffu, corr, (2 * cq) * 4);
+        qcf[1] = __shfl_sync(0xffffffffu, corr, (2 * cq + 1) * 4);
+      }
     } else {
-      // fp16 operands: q scaled per head by a power of two so its largest
-      // magnitude is in [2^14, 2^15) (exact), the scale folded into s_fac.
-      // k-slot order matches the code fragments: lane (gq, cq) holds dims
-      // 16ks + 4cq .. 16ks + 4cq + 3.
-      // INT4 codes unpack in another order: k-step ks = 2c + s takes dims
-      // 32c + 8cq + 2s + {0, 4} (first pair) and {1, 5} (second pair).
+      // E5M2 codes are exact fp16 values: fp16 operands, q scaled per head by
+      // a power of two so its largest magnitude is in [2^14, 2^15) (exact),
+      // the scale folded into s_fac. k-slot order matches the code fragments:
+      // lane (gq, cq) holds dims 16ks + 4cq .. 16ks + 4cq + 3.
       float qv[KS][4];
       float amax = 0.f;
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int dim = KV_T == KV_INT4
-                              ? (ks >> 1) * 32 + 8 * cq + 2 * (ks & 1) + ((e & 1) << 2) + (e >> 1)
-                              : 16 * ks + 4 * cq + e;
+          const int dim = 16 * ks + 4 * cq + e;
           qv[ks][e] = hv ? load_q<Q_T>(p.q, qrow + dim) : 0.f;
-          if constexpr (KCH) {
-            // keys code k / s_c: the channel scale moves to the query,
-            // q . k = sum_c (q_c s_c) code_c
-            qv[ks][e] *= p.k_scale[(h0 / p.group) * D + dim];
-          }
           amax = fmaxf(amax, fabsf(qv[ks][e]));
         }
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
@@ -355,40 +423,14 @@ struct Consumer {
       }
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
-        if constexpr (KCH) {
-          // q_c s_c is not a 16-bit value: hi + lo fp16 parts, two MMAs
-          split2<false>(ldexpf(qv[ks][0], ex), ldexpf(qv[ks][1], ex), qb[ks][0], qlo[ks][0]);
-          split2<false>(ldexpf(qv[ks][2], ex), ldexpf(qv[ks][3], ex), qb[ks][1], qlo[ks][1]);
-        } else {
-          qb[ks][0] = pack2<false>(ldexpf(qv[ks][0], ex), ldexpf(qv[ks][1], ex));
-          qb[ks][1] = pack2<false>(ldexpf(qv[ks][2], ex), ldexpf(qv[ks][3], ex));
-        }
+        qb[ks][0] = pack2<false>(ldexpf(qv[ks][0], ex), ldexpf(qv[ks][1], ex));
+        qb[ks][1] = pack2<false>(ldexpf(qv[ks][2], ex), ldexpf(qv[ks][3], ex));
       }
       // the score columns of this lane are heads 2cq and 2cq+1
       const int ex0 = __shfl_sync(0xffffffffu, ex, (2 * cq) * 4);
       const int ex1 = __shfl_sync(0xffffffffu, ex, (2 * cq + 1) * 4);
       s_fac[0] = ldexpf(p.scale_log2, -ex0);
       s_fac[1] = ldexpf(p.scale_log2, -ex1);
-      if constexpr (kInt8Codes || KV_T == KV_INT4) {
-        // sum of the fp16 query operands of head gq (as the MMA sees them)
-        float qsum = 0.f;
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-          const __half2 a = *reinterpret_cast<const __half2 *>(&qb[ks][0]);
-          const __half2 c = *reinterpret_cast<const __half2 *>(&qb[ks][1]);
-          qsum += (__low2float(a) + __high2float(a)) + (__low2float(c) + __high2float(c));
-          if constexpr (KCH) {
-            const __half2 al = *reinterpret_cast<const __half2 *>(&qlo[ks][0]);
-            const __half2 cl = *reinterpret_cast<const __half2 *>(&qlo[ks][1]);
-            qsum += (__low2float(al) + __high2float(al)) + (__low2float(cl) + __high2float(cl));
-          }
-        }
-        qsum += __shfl_xor_sync(0xffffffffu, qsum, 1);
-        qsum += __shfl_xor_sync(0xffffffffu, qsum, 2);
-        constexpr float kBias = kInt8Codes ? 1152.f : 1032.f;
-        qcorr[0] = kBias * __shfl_sync(0xffffffffu, qsum, (2 * cq) * 4);
-        qcorr[1] = kBias * __shfl_sync(0xffffffffu, qsum, (2 * cq + 1) * 4);
-      }
     }
   }
 
@@ -415,54 +457,54 @@ struct Consumer {
           ldsm_x4(T::chunk(ktile, r0 + row, 2 * ks + (lane >> 4), rows), a0, a1, a2, a3);
           mma16816<kBF>(acc, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
         }
-      } else if constexpr (KV_T == KV_INT4) {
-        // 16-byte chunk c of a row = dims 32c .. 32c + 31; a lane's word holds
-        // dims 32c + 8cq .. + 7 of its token (nibble k = dim 8cq + k)
+      } else if constexpr (kIntK) {
+        // ldmatrix.x4 of rows 0-7 / 8-15 x 16-byte chunks 2c, 2c+1 gives the
+        // A fragments of one k32 step as stored bytes
+        int ai[kDig][4] = {};  // one accumulator per query digit
+        if constexpr (KV_T == KV_INT4) {
+          // a chunk holds 32 dims as nibbles (dim 2i low, 2i + 1 high nibble of
+          // byte i); offset to u = code + 8 and split into even / odd dims:
+          // k32 steps 2c (even dims) and 2c + 1 (odd dims)
 #pragma unroll
-        for (int cpair = 0; cpair < 2; ++cpair) {
-          uint32_t w0, w1, w2, w3;  // rows 0-7 / 8-15 x chunks 2cpair, 2cpair+1
-          ldsm_x4(T::chunk(ktile, r0 + row, 2 * cpair + (lane >> 4), rows), w0, w1, w2, w3);
-          w0 ^= 0x88888888u; w1 ^= 0x88888888u; w2 ^= 0x88888888u; w3 ^= 0x88888888u;
-          const int kc = 4 * cpair;  // k-steps 4cpair .. 4cpair + 3
-          mma16816<false>(acc, int4_pair_biased<0>(w0), int4_pair_biased<0>(w1),
-                          int4_pair_biased<1>(w0), int4_pair_biased<1>(w1), qb[kc][0], qb[kc][1]);
-          mma16816<false>(acc, int4_pair_biased<2>(w0), int4_pair_biased<2>(w1),
-                          int4_pair_biased<3>(w0), int4_pair_biased<3>(w1), qb[kc + 1][0],
-                          qb[kc + 1][1]);
-          mma16816<false>(acc, int4_pair_biased<0>(w2), int4_pair_biased<0>(w3),
-                          int4_pair_biased<1>(w2), int4_pair_biased<1>(w3), qb[kc + 2][0],
-                          qb[kc + 2][1]);
-          mma16816<false>(acc, int4_pair_biased<2>(w2), int4_pair_biased<2>(w3),
-                          int4_pair_biased<3>(w2), int4_pair_biased<3>(w3), qb[kc + 3][0],
-                          qb[kc + 3][1]);
+          for (int c = 0; c < D / 64; ++c) {
+            uint32_t w0, w1, w2, w3;
+            ldsm_x4(T::chunk(ktile, r0 + row, 2 * c + (lane >> 4), rows), w0, w1, w2, w3);
+            w0 ^= 0x88888888u; w1 ^= 0x88888888u; w2 ^= 0x88888888u; w3 ^= 0x88888888u;
+            const uint32_t e0 = w0 & 0x0F0F0F0Fu, e1 = w1 & 0x0F0F0F0Fu;
+            const uint32_t e2 = w2 & 0x0F0F0F0Fu, e3 = w3 & 0x0F0F0F0Fu;
+            const uint32_t o0 = (w0 >> 4) & 0x0F0F0F0Fu, o1 = (w1 >> 4) & 0x0F0F0F0Fu;
+            const uint32_t o2 = (w2 >> 4) & 0x0F0F0F0Fu, o3 = (w3 >> 4) & 0x0F0F0F0Fu;
+#pragma unroll
+            for (int d = 0; d < kDig; ++d) {
+              mma16832_i8<true>(ai[d], e0, e1, e2, e3, qi[2 * c][0][d], qi[2 * c][1][d]);
+              mma16832_i8<true>(ai[d], o0, o1, o2, o3, qi[2 * c + 1][0][d], qi[2 * c + 1][1][d]);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int kp = 0; kp < D / 32; ++kp) {
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(T::chunk(ktile, r0 + row, 2 * kp + (lane >> 4), rows), a0, a1, a2, a3);
+#pragma unroll
+            for (int d = 0; d < kDig; ++d)
+              mma16832_i8<false>(ai[d], a0, a1, a2, a3, qi[kp][0][d], qi[kp][1][d]);
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          acc[i] = fmaf(static_cast<float>(ai[0][i]), 65536.f,
+                        fmaf(static_cast<float>(ai[1][i]), 256.f, static_cast<float>(ai[2][i])));
+          if constexpr (KV_T == KV_INT4) acc[i] -= qcf[i & 1];  // columns 2cq, 2cq + 1
         }
       } else {
 #pragma unroll
         for (int kp = 0; kp < KS / 2; ++kp) {
           uint32_t q0, q1, q2, q3;  // byte matrices: rows 0-7 / 8-15 x chunks 2kp, 2kp+1
           ldsm_x4(T::chunk(ktile, r0 + row, 2 * kp + (lane >> 4), rows), q0, q1, q2, q3);
-          if constexpr (kInt8Codes) {
-            // keys as 1152 + code (exact in fp16); the bias is removed per
-            // score below with the query sums
-            q0 ^= 0x80808080u; q1 ^= 0x80808080u; q2 ^= 0x80808080u; q3 ^= 0x80808080u;
-            const uint32_t a00 = int8_pair_biased<0, 1>(q0), a01 = int8_pair_biased<0, 1>(q1);
-            const uint32_t a02 = int8_pair_biased<2, 3>(q0), a03 = int8_pair_biased<2, 3>(q1);
-            const uint32_t a10 = int8_pair_biased<0, 1>(q2), a11 = int8_pair_biased<0, 1>(q3);
-            const uint32_t a12 = int8_pair_biased<2, 3>(q2), a13 = int8_pair_biased<2, 3>(q3);
-            mma16816<false>(acc, a00, a01, a02, a03, qb[2 * kp][0], qb[2 * kp][1]);
-            mma16816<false>(acc, a10, a11, a12, a13, qb[2 * kp + 1][0], qb[2 * kp + 1][1]);
-            if constexpr (KCH) {
-              mma16816<false>(acc, a00, a01, a02, a03, qlo[2 * kp][0], qlo[2 * kp][1]);
-              mma16816<false>(acc, a10, a11, a12, a13, qlo[2 * kp + 1][0], qlo[2 * kp + 1][1]);
-            }
-          } else {
-            mma16816<false>(acc, e5m2_pair<0, 1>(q0), e5m2_pair<0, 1>(q1),
-                            e5m2_pair<2, 3>(q0), e5m2_pair<2, 3>(q1), qb[2 * kp][0],
-                            qb[2 * kp][1]);
-            mma16816<false>(acc, e5m2_pair<0, 1>(q2), e5m2_pair<0, 1>(q3),
-                            e5m2_pair<2, 3>(q2), e5m2_pair<2, 3>(q3), qb[2 * kp + 1][0],
-                            qb[2 * kp + 1][1]);
-          }
+          mma16816<false>(acc, e5m2_pair<0, 1>(q0), e5m2_pair<0, 1>(q1), e5m2_pair<2, 3>(q0),
+                          e5m2_pair<2, 3>(q1), qb[2 * kp][0], qb[2 * kp][1]);
+          mma16816<false>(acc, e5m2_pair<0, 1>(q2), e5m2_pair<0, 1>(q3), e5m2_pair<2, 3>(q2),
+                          e5m2_pair<2, 3>(q3), qb[2 * kp + 1][0], qb[2 * kp + 1][1]);
         }
       }
       // acc: [0],[1] = token mt*16+gq, heads 2cq, 2cq+1; [2],[3] = token +8
@@ -471,12 +513,6 @@ struct Consumer {
       if constexpr (T::kKRowScales) {
         k0 = ksc[t0];
         k1 = ksc[t1];
-      }
-      if constexpr (kInt8Codes || KV_T == KV_INT4) {
-        acc[0] -= qcorr[0];
-        acc[1] -= qcorr[1];
-        acc[2] -= qcorr[0];
-        acc[3] -= qcorr[1];
       }
       sc[mt][0] = t0 < valid ? acc[0] * s_fac[0] * k0 : -INFINITY;
       sc[mt][1] = t0 < valid ? acc[1] * s_fac[1] * k0 : -INFINITY;
@@ -769,6 +805,26 @@ struct NewRow {
     }
   }
 
+  // Park this lane's share in shared memory (buf: this warp's [6][32] words)
+  // from the piece start to the block that takes it, so that it holds no
+  // registers through the blocks before.
+  __device__ __forceinline__ void stash(uint32_t *buf, int lane) const {
+    buf[lane] = k[0];
+    buf[32 + lane] = k[1];
+    buf[64 + lane] = v[0];
+    buf[96 + lane] = v[1];
+    buf[128 + lane] = __float_as_uint(ks);
+    buf[160 + lane] = __float_as_uint(vs);
+  }
+  __device__ __forceinline__ void unstash(const uint32_t *buf, int lane) {
+    k[0] = buf[lane];
+    k[1] = buf[32 + lane];
+    v[0] = buf[64 + lane];
+    v[1] = buf[96 + lane];
+    ks = __uint_as_float(buf[128 + lane]);
+    vs = __uint_as_float(buf[160 + lane]);
+  }
+
   // Put the row in the stage (row r0 + rl of the stage's K / V parts, where the
   // load brought whatever the pool held) and in the pool (block id, head g).
   __device__ __forceinline__ void store(const AttnParams &p, uint8_t *st, int rows, int r, int id,
@@ -865,6 +921,7 @@ attn_partition_kernel(const __grid_constant__ CUtensorMap kmap,
   __shared__ long long red[kWarps];
   __shared__ long long s_loc[2];
   __shared__ int s_abort;
+  __shared__ uint32_t s_newrow[kNC][6 * 32];  // fused append: each warp's new row
   uint8_t *ring = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
 
@@ -1024,8 +1081,11 @@ attn_partition_kernel(const __grid_constant__ CUtensorMap kmap,
     const int jl = (L - 1) / BS;
     const bool has_new =
         p.k_new != nullptr && active && L > 0 && jl >= w.j && jl < w.j + seg;
-    NewRow<D, BS, KV_T, Q_T> nr;
-    if (has_new) nr.load(p, w.b, g, lane);
+    if (has_new) {  // loaded (quantized) now, parked until its block arrives
+      NewRow<D, BS, KV_T, Q_T> nr;
+      nr.load(p, w.b, g, lane);
+      nr.stash(s_newrow[warp], lane);
+    }
     if (active) {
       cs.reset();
       cs.load_query(p, w.b, h0, nh, lane);
@@ -1047,6 +1107,8 @@ attn_partition_kernel(const __grid_constant__ CUtensorMap kmap,
           const int valid = id >= 0 ? min(BS, L - jb * BS) : 0;
           if (has_new && jb == jl && id >= 0) {
             const int rl = (L - 1) - jl * BS;
+            NewRow<D, BS, KV_T, Q_T> nr;
+            nr.unstash(s_newrow[warp], lane);
             nr.store(p, ring + s * stride, rows, hi * BS + rl, id, g, rl, lane);
             // the producer's next TMA into this stage must come after these writes
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -1131,8 +1193,10 @@ __global__ void __launch_bounds__(kMergeWarps * 32) attn_merge_kernel(const Attn
   };
   // One online pass over the pieces in order: running max M, sum Ls and
   // output acc. The loads of up to kBatch pieces are issued together, so a
-  // unit costs one round trip per kBatch pieces rather than one per piece.
-  constexpr int kBatch = 8;
+  // unit costs one round trip per kBatch pieces rather than one per piece
+  // (10 keeps the kernel at about 90 registers, so a CTA still fits beside an
+  // attention CTA's 48k).
+  constexpr int kBatch = 10;
   float M = -INFINITY, Ls = 0.f;
   float acc[E];
 #pragma unroll
@@ -1213,17 +1277,24 @@ PartFn pick_partition(int D, int BS, int kv, int q) {
   return BS == 16 ? pick_dtype<64, 16>(kv, q) : pick_dtype<64, 32>(kv, q);
 }
 
+// Dynamic shared memory a merge CTA reserves without using it: it caps how
+// many merge CTAs one SM takes when the attention CTAs drain (measured: CTAs
+// piling onto the first SMs to free up made slow outlier steps), while two
+// still fit beside a resident attention CTA, so the merge is scheduled early.
+constexpr int kMergeSmemReserve = 12 * 1024;
+
 cudaError_t launch_merge(int D, int out_t, const AttnParams &p, cudaStream_t st) {
   const int64_t warps = static_cast<int64_t>(p.num_seqs) * p.q_heads;
   const unsigned grid = static_cast<unsigned>((warps + kMergeWarps - 1) / kMergeWarps);
   const int th = kMergeWarps * 32;
+  const int sm = kMergeSmemReserve;
   cudaError_t e;
   if (D == 128) {
-    e = out_t == KV_BF16 ? launch_pdl(attn_merge_kernel<128, KV_BF16>, dim3(grid), dim3(th), 0, st, p)
-                         : launch_pdl(attn_merge_kernel<128, KV_FP16>, dim3(grid), dim3(th), 0, st, p);
+    e = out_t == KV_BF16 ? launch_pdl(attn_merge_kernel<128, KV_BF16>, dim3(grid), dim3(th), sm, st, p)
+                         : launch_pdl(attn_merge_kernel<128, KV_FP16>, dim3(grid), dim3(th), sm, st, p);
   } else {
-    e = out_t == KV_BF16 ? launch_pdl(attn_merge_kernel<64, KV_BF16>, dim3(grid), dim3(th), 0, st, p)
-                         : launch_pdl(attn_merge_kernel<64, KV_FP16>, dim3(grid), dim3(th), 0, st, p);
+    e = out_t == KV_BF16 ? launch_pdl(attn_merge_kernel<64, KV_BF16>, dim3(grid), dim3(th), sm, st, p)
+                         : launch_pdl(attn_merge_kernel<64, KV_FP16>, dim3(grid), dim3(th), sm, st, p);
   }
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

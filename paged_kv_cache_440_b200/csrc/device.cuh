@@ -191,6 +191,28 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
   }
 }
 
+// D = A(16x32, row) * B(32x8, col) + D on 8-bit integers, exact int32
+// accumulation. A signed (s8) or unsigned (u8) as kUnsignedA says, B signed.
+// A's four registers are what one ldmatrix.x4 of a 16-row x 32-byte tile
+// gives (rows 0-7 / 8-15 of bytes 0-15, then of bytes 16-31).
+template <bool kUnsignedA>
+__device__ __forceinline__ void mma16832_i8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                            uint32_t a3, uint32_t b0, uint32_t b1) {
+  if constexpr (kUnsignedA) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  } else {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  }
+}
+
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t d;
   asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
@@ -261,14 +283,6 @@ template <int A, int B>
 __device__ __forceinline__ uint32_t e5m2_pair(uint32_t src) {
   // result bytes: [0] = 0, [1] = src[A], [2] = 0, [3] = src[B]
   return prmt(src, 0u, (B << 12) | (4 << 8) | (A << 4) | 4);
-}
-
-// Two INT8 codes (sign bit flipped by the caller) as fp16 1152 + code, exact:
-// the bias stays in and is removed from the dot product by the caller.
-template <int A, int B>
-__device__ __forceinline__ uint32_t int8_pair_biased(uint32_t src_biased) {
-  // result bytes: [0] = u[A], [1] = 0x64, [2] = u[B], [3] = 0x64 -> 1024 + u
-  return prmt(src_biased, 0x64646464u, (4 << 12) | (B << 8) | (4 << 4) | A);
 }
 
 template <int A, int B>
