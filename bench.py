@@ -974,7 +974,9 @@ def main():
                        "l2": "K/V %.1fx L2 (126 MB); L2 flushed before each timed step by "
                              "reading 256 MiB" % (r["dec_bytes"] / 126e6),
                        "bytes_per_step": r["dec_bytes"] + r["app_bytes"]},
-            "pct_of_8tbs": round(100 * gbs / world / NOMINAL_HBM_GBS, 2),
+            # the shared prompt's value counts logical bytes (read from L2): no HBM percentage
+            "pct_of_8tbs": None if args.workload == "shared_prefix"
+            else round(100 * gbs / world / NOMINAL_HBM_GBS, 2),
             "decode_tokens_per_s": round(wl.batch * world / r["step_s"], 1),
             "roofline": {"bound": "hbm",
                          "achieved": None if achieved is None else round(achieved, 2),
