@@ -469,11 +469,13 @@ struct Consumer {
           for (int c = 0; c < D / 64; ++c) {
             uint32_t w0, w1, w2, w3;
             ldsm_x4(T::chunk(ktile, r0 + row, 2 * c + (lane >> 4), rows), w0, w1, w2, w3);
-            w0 ^= 0x88888888u; w1 ^= 0x88888888u; w2 ^= 0x88888888u; w3 ^= 0x88888888u;
-            const uint32_t e0 = w0 & 0x0F0F0F0Fu, e1 = w1 & 0x0F0F0F0Fu;
-            const uint32_t e2 = w2 & 0x0F0F0F0Fu, e3 = w3 & 0x0F0F0F0Fu;
-            const uint32_t o0 = (w0 >> 4) & 0x0F0F0F0Fu, o1 = (w1 >> 4) & 0x0F0F0F0Fu;
-            const uint32_t o2 = (w2 >> 4) & 0x0F0F0F0Fu, o3 = (w3 >> 4) & 0x0F0F0F0Fu;
+            // u = code + 8: mask the nibbles and flip their top bit in one op
+            const uint32_t e0 = (w0 & 0x0F0F0F0Fu) ^ 0x08080808u, e1 = (w1 & 0x0F0F0F0Fu) ^ 0x08080808u;
+            const uint32_t e2 = (w2 & 0x0F0F0F0Fu) ^ 0x08080808u, e3 = (w3 & 0x0F0F0F0Fu) ^ 0x08080808u;
+            const uint32_t o0 = ((w0 >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
+            const uint32_t o1 = ((w1 >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
+            const uint32_t o2 = ((w2 >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
+            const uint32_t o3 = ((w3 >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
 #pragma unroll
             for (int d = 0; d < kDig; ++d) {
               mma16832_i8<true>(ai[d], e0, e1, e2, e3, qi[2 * c][0][d], qi[2 * c][1][d]);
@@ -640,8 +642,7 @@ struct Consumer {
           uint32_t w0, w1, w2, w3;  // tokens 0-7 / 8-15 x chunks 2cp, 2cp+1
           const int vr = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
           ldsm_x4_t(T::chunk(vtile, r0 + vr, 2 * cp + (lane >> 4), rows), w0, w1, w2, w3);
-          w0 ^= 0x88888888u; w1 ^= 0x88888888u; w2 ^= 0x88888888u; w3 ^= 0x88888888u;
-          uint32_t a[16];
+          uint32_t a[16];  // codes as fp16 (the offset flip is inside int4_pair)
           a[0] = int4_pair<0>(w0); a[1] = int4_pair<1>(w0); a[2] = int4_pair<0>(w1); a[3] = int4_pair<1>(w1);
           a[4] = int4_pair<2>(w0); a[5] = int4_pair<3>(w0); a[6] = int4_pair<2>(w1); a[7] = int4_pair<3>(w1);
           a[8] = int4_pair<0>(w2); a[9] = int4_pair<1>(w2); a[10] = int4_pair<0>(w3); a[11] = int4_pair<1>(w3);

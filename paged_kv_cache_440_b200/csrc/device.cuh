@@ -250,17 +250,18 @@ __device__ __forceinline__ void split2(float a, float b, uint32_t &hi, uint32_t 
 
 // -------------------------------------------------- 4-bit codes -> fp16 pairs
 //
-// INT4 codes (two's complement nibbles) become offset binary u = code + 8 when
-// the caller xors the word with 0x88888888. Nibbles K and K + 4 of a 32-bit
-// word, placed under the fp16 exponent byte 0x64, are 1024 + u: an exact pair,
-// 1032 above the codes.
+// An INT4 code c (two's complement nibble) is offset binary u = c + 8 after
+// flipping its top bit. Nibbles K and K + 4 of a 32-bit word of codes, masked,
+// flipped and placed under the fp16 exponent byte 0x64 in one logic op
+// ((x & 0x000F000F) ^ 0x64086408), are 1024 + u: an exact pair, 1032 above the
+// codes.
 template <int K>
-__device__ __forceinline__ uint32_t int4_pair_biased(uint32_t w_biased) {
-  return ((w_biased >> (4 * K)) & 0x000F000Fu) | 0x64006400u;
+__device__ __forceinline__ uint32_t int4_pair_biased(uint32_t w) {
+  return ((w >> (4 * K)) & 0x000F000Fu) ^ 0x64086408u;
 }
 template <int K>
-__device__ __forceinline__ uint32_t int4_pair(uint32_t w_biased) {
-  uint32_t h = int4_pair_biased<K>(w_biased);
+__device__ __forceinline__ uint32_t int4_pair(uint32_t w) {
+  uint32_t h = int4_pair_biased<K>(w);
   __half2 v = *reinterpret_cast<__half2 *>(&h);
   const __half2 bias = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));
   v = __hsub2(v, bias);
