@@ -14,11 +14,18 @@
 // * Two producer warps (K boxes, V boxes) stream the KV head's cached
 //   blocks, 64 positions per stage, into a ring of 6 (head_dim 128) or 8 (64)
 //   stages; block ids are read a 32-block window ahead, each TMA box is issued
-//   by its own lane. K lands slab-major across the ring ([128-byte slab][slot
-//   x 64 + key][128 B], one box per block and slab), so two adjacent stages
-//   form one 128-key operand. V lands per stage, one box per block and slab,
-//   or one box per block where a 3-D (element, row, slab) view of the pool is
-//   accepted by the driver ([block][slab][row][128 B]).
+//   by its own lane. With head_dim 128 each block comes in one box for K and
+//   one for V, through 4-D and 3-D views of the pool whose boxes cover both
+//   128-byte slabs of a row: K lands as [block][8-row group][slab][8 rows][128
+//   B], so that the 8-row groups of all keys of two adjacent stages sit 2048
+//   bytes apart and form one 128-key operand; V as [block][slab][row][128 B].
+//   (Where the driver declines those views: one box per block and slab, K
+//   slab-major across the ring.) The copy engine's cost grows with the number
+//   of boxes, not only with the bytes: one box per block streams the same
+//   bytes about 25% faster than two.
+// * K and V of a stage have their own full and empty barriers: a K slot is
+//   released as soon as S of its unit is done, long before P V frees the V
+//   slot, so the K loads run up to a ring ahead of the scores.
 // * The MMA warp (one thread) issues tcgen05 MMAs with the A operand in
 //   tensor memory and B in shared memory, per unit of 128 keys (two stages):
 //   S_u = Q K_u^T (M 128, N 128, K head_dim; Q in TMEM, K K-major) into one
@@ -34,11 +41,16 @@
 // * 8 softmax warps (PAGEDKV_PF_GROUPS = 2 column groups; 4 gives 16 warps,
 //   measured slower): warp w reads TMEM lanes 32 (w mod 4) .. + 31 (the lanes
 //   a warp may access) and columns of group w / 4, so two threads share a
-//   row, 64 scores each per unit (read from TMEM twice: a max pass, then an
-//   exp pass, 32 columns at a time); the row maximum is combined through
-//   shared memory once per unit. Scale, causal and tail masks and the online
-//   softmax run in fp32 (base 2), two lanes per instruction where the
-//   hardware has packed fp32 arithmetic. The running maximum is only raised
+//   row, 64 scores each per unit, read from TMEM once (both 32-column loads
+//   in flight together) and kept in registers for the max and the exp pass.
+//   The row maximum of the raw scores is combined through shared memory once
+//   per unit, under a named barrier of the warps sharing those TMEM lanes
+//   only. The scale is applied with the maximum in one packed fused
+//   multiply-add per score pair (exp2(s scale - m)); it is kept positive: a
+//   negative scale enters as q's sign, a zero one as q = 0. Causal and tail
+//   masks set raw scores to -inf; the online softmax runs in fp32 (base 2),
+//   two lanes per instruction where the hardware has packed fp32
+//   arithmetic. The running maximum is only raised
 //   (and O, l rescaled in TMEM) when a new score exceeds it by more than 2^8;
 //   otherwise the stale maximum stays in use, which keeps every P value below
 //   256 and leaves the result unchanged up to rounding.
@@ -47,14 +59,17 @@
 //   8 of lo pairs, the layout of one K step of the MMA's A); O accumulates
 //   P_hi V + P_lo V, so rounding P to 16 bits costs nothing measurable (bf16:
 //   hi and lo by truncation, bit masks only; fp16: by rounding conversions).
-// * Synchronisation is by mbarriers: TMA -> MMA (full), MMA -> producer
-//   (stage free, by tcgen05.commit after P_u V; the softmax warps wait on the
-//   same commit before they rescale O or read it at the end), MMA -> softmax
-//   (S_u ready), softmax -> MMA (P_u written). Every wait is bounded; after a timeout
+// * Synchronisation is by mbarriers: TMA -> MMA (K full, V full), MMA ->
+//   producers (K slot free by tcgen05.commit after S_u; V slot free after P_u
+//   V, and the softmax warps wait on that commit before they rescale O or
+//   read it at the end), MMA -> softmax (S_u ready), softmax -> MMA (P_u
+//   written; the softmax warps wait for V full too, for the block masks and
+//   the tail rows they zero). Every wait is bounded; after a timeout
 //   every role runs to the end without waiting, the output is not written and
 //   the CTA frees its TMEM.
 #include <algorithm>
 #include <cfloat>
+#include <cmath>
 
 #include "device.cuh"
 #include "internal.h"
@@ -89,7 +104,10 @@ struct PrefillParams {
   const int32_t *block_tables;
   const int32_t *context_lens;
   int *status;
-  float scale_log2;
+  float scale_log2;           // |scale| log2(e), or 1 where scale is 0
+  // q enters TMEM as (bits & q_keep) ^ q_sign: its sign flipped where scale <
+  // 0, zeroed where scale is 0 (all scores 0), so that the scale used is > 0
+  uint32_t q_keep, q_sign;
   int num_seqs, q_heads, kv_heads, group, tile_tokens, total_q;
   int max_blocks, num_blocks, limit;
 };
@@ -119,9 +137,11 @@ __device__ __forceinline__ bool ring_wait_pf(uint64_t *bar, uint32_t parity, vol
   }
 }
 
-// VBLK: V comes one box per block (both 128-byte slabs, the 3-D map), landing
-// per stage as [block][slab][row][128 B]; otherwise one box per block and
-// slab, landing as [slab][key][128 B].
+// VBLK: K and V come one box per block (both 128-byte slabs): K through the
+// 4-D map, landing per stage as [block][8-row group][slab][8 rows][128 B], V
+// through the 3-D map as [block][slab][row][128 B]; otherwise one box per
+// block and slab, K landing as [slab][slot * 64 + key][128 B] across the ring
+// and V per stage as [slab][key][128 B].
 template <int D, int BS, int KV_T, bool VBLK>
 __global__ void __launch_bounds__(kPfThreads, 1)
 attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
@@ -154,19 +174,31 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
       return (c >> 3) * kPfKeys * 128 + key * 128 + (c & 7) * 16;
   };
   constexpr uint32_t kVSlabStride = VBLK ? BS * 128 : kPfKeys * 128;
+  constexpr uint32_t kKGroupStride = VBLK ? 2048 : 1024;   // 8-row groups of K
+  constexpr uint32_t kKSlotBytes = VBLK ? kPartBytes : kPfKeys * 128;  // K slot stride
+  constexpr uint32_t kKSlabOff = VBLK ? 1024 : kKSlabBytes;            // second 64 dims
 
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t full_bar[kStages];
-  __shared__ __align__(8) uint64_t empty_bar[kStages];
+  // K and V of a stage land and are released separately: a K slot is free
+  // once S of its unit is done, a V slot once P V is
+  __shared__ __align__(8) uint64_t k_full[kStages];
+  __shared__ __align__(8) uint64_t v_full[kStages];
+  __shared__ __align__(8) uint64_t k_empty[kStages];
+  __shared__ __align__(8) uint64_t v_empty[kStages];
   __shared__ __align__(8) uint64_t s_full[kPfSBufs];
   __shared__ __align__(8) uint64_t p_full[kPfSBufs];
   __shared__ __align__(8) uint64_t mma_idle;
-  __shared__ uint32_t stage_mask[kStages];           // valid blocks of the stage
+  // valid blocks of a stage, written by the V warp before its full arrival:
+  // a V slot (unlike a K slot) is not refilled before the softmax warps are
+  // done with its unit
+  __shared__ uint32_t stage_mask[kStages];
   __shared__ float red[2][kPfGroups][kPfRows];       // row maxima, then row sums
   __shared__ uint32_t tmem_slot;
   __shared__ int s_abort;
-  // K ring: [slab][slot * 64 + key][128 B], so that the two stages of a unit
-  // (slots 2i, 2i + 1) form one 128-row operand; V ring: [slot][slab][key][128 B]
+  // K ring: with block boxes [slot][block][8-row group][slab][8 rows][128 B]
+  // (8-row groups 2048 bytes apart, slabs 1024), else [slab][slot * 64 + key][128
+  // B] (8-row groups 1024 apart); either way the two stages of a unit (slots
+  // 2i, 2i + 1) form one 128-row operand. V ring: [slot][...] as v_off says.
   uint8_t *ring_k = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t *ring_v = ring_k + kStages * kPartBytes;
@@ -193,8 +225,10 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
   if (threadIdx.x == 0) {
     s_abort = 0;
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&full_bar[i], 1);
-      mbar_init(&empty_bar[i], 1);
+      mbar_init(&k_full[i], 1);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_empty[i], 1);
     }
     for (int i = 0; i < kPfSBufs; ++i) {
       mbar_init(&s_full[i], 1);
@@ -229,10 +263,10 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
 #pragma unroll
       for (int i = 0; i < kQGCols / 4; ++i) {
         const uint4 x = rvalid ? src[i] : make_uint4(0u, 0u, 0u, 0u);
-        v[4 * i] = x.x;
-        v[4 * i + 1] = x.y;
-        v[4 * i + 2] = x.z;
-        v[4 * i + 3] = x.w;
+        v[4 * i] = (x.x & p.q_keep) ^ p.q_sign;
+        v[4 * i + 1] = (x.y & p.q_keep) ^ p.q_sign;
+        v[4 * i + 2] = (x.z & p.q_keep) ^ p.q_sign;
+        v[4 * i + 3] = (x.w & p.q_keep) ^ p.q_sign;
       }
       tmem_st<kQGCols>(tm + (static_cast<uint32_t>((warp & 3) * 32) << 16) + kQCol + cg * kQGCols, v);
       tmem_wait_st();
@@ -253,9 +287,13 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
       prefetch_tmap(&vmap);
     }
     // Two warps, one for the K boxes and one for the V boxes of every stage
-    // (one box per block and slab, each issued by its own lane). Block ids
-    // travel one 32-block window per lane-wide load, fetched a window ahead.
+    // (one box per block, or per block and slab where the block maps are not
+    // available, each issued by its own lane), each warp with its own full
+    // and empty barriers. Block ids travel one 32-block window per lane-wide
+    // load, fetched a window ahead.
     const int kv = warp - kPfProducerWarp;
+    uint64_t *fullb = kv ? v_full : k_full;
+    uint64_t *emptyb = kv ? v_empty : k_empty;
     const int32_t *btab = p.block_tables + static_cast<int64_t>(b) * p.max_blocks;
     const int nblocks = (nkeys + BS - 1) / BS;
     auto load_ids = [&](int w) {
@@ -274,7 +312,7 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
     uint32_t cur_ok = __ballot_sync(kFull, cur >= 0);
     int issued = 0;
     // this warp's TMA boxes of a full stage
-    const int kBoxes = (kv && VBLK) ? kBlocksPerStage : kBlocksPerStage * kSlabs;
+    const int kBoxes = VBLK ? kBlocksPerStage : kBlocksPerStage * kSlabs;
     static_assert(kBlocksPerStage * kSlabs <= 32, "one box per lane");
     for (int st = 0; st < nstages; ++st) {
       const int s = st % kStages;
@@ -286,29 +324,34 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
       }
       int okv = 1;
       if (lane == 0 && st >= kStages)
-        okv = ring_wait_pf(&empty_bar[s], ((st / kStages) - 1) & 1, &s_abort, p.status);
+        okv = ring_wait_pf(&emptyb[s], ((st / kStages) - 1) & 1, &s_abort, p.status);
       okv = __shfl_sync(kFull, okv, 0);
       if (!okv) break;
       const int nblk = min(kBlocksPerStage, nblocks - jb0);
       const uint32_t valid = (cur_ok >> (jb0 & 31)) & ((1u << nblk) - 1u);
-      if (lane == 0 && kv == 0) {  // the V warp's bytes may land first: tx counts may go negative
-        stage_mask[s] = valid;
-        mbar_arrive_expect_tx(&full_bar[s], __popc(valid) * 2 * BS * D * 2);
+      if (lane == 0) {
+        if (kv == 1) stage_mask[s] = valid;
+        mbar_arrive_expect_tx(&fullb[s], __popc(valid) * BS * D * 2);
       }
       // lane -> (block j, slab)
-      const int per = (kv && VBLK) ? 1 : kSlabs;
+      const int per = VBLK ? 1 : kSlabs;
       const int j = lane / per, sl = lane % per;
       const int bid = __shfl_sync(kFull, cur, (jb0 & 31) + (j < kBlocksPerStage ? j : 0));
       if (lane < kBoxes && j < nblk && ((valid >> j) & 1u)) {
         const int y = (bid * p.kv_heads + g) * BS;
-        if (kv == 0)
-          tma_load_2d(ring_k + sl * kKSlabBytes + (s * kPfKeys + j * BS) * 128, &kmap, &full_bar[s],
-                      sl * 64, y);
-        else if (VBLK)
-          tma_load_3d(ring_v + s * kPartBytes + j * BS * 256, &vmap, &full_bar[s], 0, y, 0);
-        else
-          tma_load_2d(ring_v + s * kPartBytes + (sl * kPfKeys + j * BS) * 128, &vmap, &full_bar[s],
-                      sl * 64, y);
+        if constexpr (VBLK) {
+          if (kv == 0)
+            tma_load_4d(ring_k + s * kPartBytes + j * BS * 256, &kmap, &fullb[s], 0, 0, 0, y / 8);
+          else
+            tma_load_3d(ring_v + s * kPartBytes + j * BS * 256, &vmap, &fullb[s], 0, y, 0);
+        } else {
+          if (kv == 0)
+            tma_load_2d(ring_k + sl * kKSlabBytes + (s * kPfKeys + j * BS) * 128, &kmap, &fullb[s],
+                        sl * 64, y);
+          else
+            tma_load_2d(ring_v + s * kPartBytes + (sl * kPfKeys + j * BS) * 128, &vmap, &fullb[s],
+                        sl * 64, y);
+        }
       }
       __syncwarp();
       ++issued;
@@ -316,7 +359,7 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
     if (lane == 0) {
       // let the loads still in flight land before the CTA can exit
       for (int st = max(0, issued - kStages); st < issued; ++st)
-        mbar_wait(&full_bar[st % kStages], (st / kStages) & 1, nullptr, 100000000ull);
+        mbar_wait(&fullb[st % kStages], (st / kStages) & 1, nullptr, 100000000ull);
     }
     __syncwarp();
   } else if (warp == kPfMmaWarp) {
@@ -327,28 +370,32 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
       // descriptors of slot 0; other slots and K steps add their byte offset
       // / 16 to the start-address field (no carry: shared addresses stay below
       // 256 KB)
-      const uint64_t kdesc0 = umma_desc_sw128(smem_u32(ring_k), 16, 1024);
+      const uint64_t kdesc0 = umma_desc_sw128(smem_u32(ring_k), 16, kKGroupStride);
       const uint64_t vdesc0 = umma_desc_sw128(smem_u32(ring_v), kVSlabStride, 1024);
       bool ok = true;
       // Between two MMAs this thread runs only immediate adds: the issuing
       // thread, not the tensor core, limits small MMAs.
       auto issue_s = [&](int u) {
         const int a = 2 * u;
-        if (!ring_wait_pf(&full_bar[a % kStages], (a / kStages) & 1, &s_abort, p.status))
+        const bool two = a + 1 < nstages;
+        if (!ring_wait_pf(&k_full[a % kStages], (a / kStages) & 1, &s_abort, p.status))
           return false;
-        if (a + 1 < nstages &&
-            !ring_wait_pf(&full_bar[(a + 1) % kStages], ((a + 1) / kStages) & 1, &s_abort, p.status))
+        if (two &&
+            !ring_wait_pf(&k_full[(a + 1) % kStages], ((a + 1) / kStages) & 1, &s_abort, p.status))
           return false;
         tc_fence_after();
         // a unit's 128 keys: rows of slots a mod kStages and the next one
-        const uint64_t kd = kdesc0 + static_cast<uint64_t>(((a % kStages) * kPfKeys * 128) >> 4);
+        const uint64_t kd = kdesc0 + static_cast<uint64_t>(((a % kStages) * kKSlotBytes) >> 4);
         const uint32_t sd = tm + (u & 1) * kPfUnit;
         umma_f16_tmem_a_c<false>(sd, tm + kQCol, kd, idesc_s);
 #pragma unroll
         for (int ks = 1; ks < D / 16; ++ks)
           umma_f16_tmem_a_c<true>(sd, tm + kQCol + ks * 8,
-                                  kd + (((ks >> 2) * kKSlabBytes + (ks & 3) * 32) >> 4), idesc_s);
+                                  kd + (((ks >> 2) * kKSlabOff + (ks & 3) * 32) >> 4), idesc_s);
         umma_commit(&s_full[u & 1]);
+        // the unit's K slots are free once S is done
+        umma_commit(&k_empty[a % kStages]);
+        if (two) umma_commit(&k_empty[(a + 1) % kStages]);
         return true;
       };
       for (int u = 0; ok && u < min(nunits, kPfSBufs); ++u) ok = issue_s(u);
@@ -357,6 +404,12 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
         tc_fence_after();
         const uint32_t pcol = tm + (u & 1) * kPfUnit;
         const int a = 2 * u, nh = a + 1 < nstages ? 2 : 1;
+        // V has landed (the softmax warps waited for it too)
+        if (!ring_wait_pf(&v_full[a % kStages], (a / kStages) & 1, &s_abort, p.status)) break;
+        if (nh == 2 &&
+            !ring_wait_pf(&v_full[(a + 1) % kStages], ((a + 1) / kStages) & 1, &s_abort, p.status))
+          break;
+        tc_fence_after();
         // per stage of the unit: P_hi V over its 4 K steps, then P_lo V (the
         // first MMA of the first unit starts the accumulator)
 #pragma unroll
@@ -375,9 +428,9 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
             }
           }
         }
-        // a unit's stages are free (and O holds P_0..P_u V) once these finish
-        umma_commit(&empty_bar[a % kStages]);
-        if (nh == 2) umma_commit(&empty_bar[(a + 1) % kStages]);
+        // the unit's V slots are free (and O holds P_0..P_u V) once these finish
+        umma_commit(&v_empty[a % kStages]);
+        if (nh == 2) umma_commit(&v_empty[(a + 1) % kStages]);
         // S_{u+2} reuses S_u's columns: issued after P_u V, which reads them
         if (u + kPfSBufs < nunits) ok = issue_s(u + kPfSBufs);
       }
@@ -399,10 +452,12 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
       const int a = 2 * u;
       const bool two = a + 1 < nstages;
       ring_wait_pf(&s_full[u & 1], (u >> 1) & 1, &s_abort, p.status);
-      // the stages' TMA has landed (their full phases cannot advance before
-      // P_u V is done): gives this thread the block masks and the V bytes
-      ring_wait_pf(&full_bar[a % kStages], (a / kStages) & 1, &s_abort, p.status);
-      if (two) ring_wait_pf(&full_bar[(a + 1) % kStages], ((a + 1) / kStages) & 1, &s_abort, p.status);
+      // the stages' V has landed (a V slot's full phase cannot advance before
+      // P_u V is done; a K slot may already hold the next round, so K
+      // barriers are not waited on here): gives this thread the block masks
+      // and the V bytes
+      ring_wait_pf(&v_full[a % kStages], (a / kStages) & 1, &s_abort, p.status);
+      if (two) ring_wait_pf(&v_full[(a + 1) % kStages], ((a + 1) / kStages) & 1, &s_abort, p.status);
       tc_fence_after();
       const int key0 = u * kPfUnit;
       const uint32_t bmask =
@@ -410,40 +465,37 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
       const bool tail = key0 + kPfUnit > nkeys || bmask != kAllBlocks;
       const bool need_mask = tail || key0 + c0 + kSCols - 1 > rpos;
       const uint32_t sbuf = trow + (u & 1) * kPfUnit + c0;
-      // scores of chunk ch (scaled to base 2, masked)
-      auto scores = [&](int ch, float (&sv)[kSChunk]) {
-        uint32_t r[kSChunk];
-        tmem_ld<kSChunk>(sbuf + ch * kSChunk, r);
-        tmem_wait_ld();
+      // this thread's scores of the unit, read from TMEM once and kept in
+      // registers; masked positions become -inf
+      uint32_t sr[kSCols / kSChunk][kSChunk];
 #pragma unroll
-        for (int c = 0; c < kSChunk; c += 2) {
-          const float2 v = mul2(make_float2(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), sc2);
-          sv[c] = v.x;
-          sv[c + 1] = v.y;
-        }
-        if (need_mask) {
-#pragma unroll
-          for (int c = 0; c < kSChunk; ++c) {
-            const int cu = c0 + ch * kSChunk + c;       // column in the unit
-            const int kp = key0 + cu;
-            const bool okk = kp <= rpos && kp < nkeys && ((bmask >> (cu / BS)) & 1u);
-            sv[c] = okk ? sv[c] : -INFINITY;
-          }
-        }
+      for (int ch = 0; ch < kSCols / kSChunk; ++ch) tmem_ld<kSChunk>(sbuf + ch * kSChunk, sr[ch]);
+      tmem_wait_ld();
+      auto keep = [&](int cu) {                      // column cu of the unit is attended
+        const int kp = key0 + cu;
+        return kp <= rpos && kp < nkeys && ((bmask >> (cu / BS)) & 1u);
       };
-      // pass 1: the row maximum over this thread's columns, then the row's
+      if (need_mask) {
+#pragma unroll
+        for (int ch = 0; ch < kSCols / kSChunk; ++ch)
+#pragma unroll
+          for (int c = 0; c < kSChunk; ++c)
+            if (!keep(c0 + ch * kSChunk + c)) sr[ch][c] = __float_as_uint(-INFINITY);
+      }
+      // the row maximum of the raw scores (the scale is not negative: a
+      // negative one enters as q's sign), over this thread's columns and then
+      // the row's, exchanged with the warps holding the row's other columns
       float mx = -INFINITY;
 #pragma unroll
-      for (int ch = 0; ch < kSCols / kSChunk; ++ch) {
-        float sv[kSChunk];
-        scores(ch, sv);
+      for (int ch = 0; ch < kSCols / kSChunk; ++ch)
 #pragma unroll
-        for (int c = 0; c < kSChunk; c += 2) mx = fmax3(mx, sv[c], sv[c + 1]);
-      }
+        for (int c = 0; c < kSChunk; c += 2)
+          mx = fmax3(mx, __uint_as_float(sr[ch][c]), __uint_as_float(sr[ch][c + 1]));
       red[u & 1][cg][row] = mx;
-      bar_sync(1, kPfSoftmax);
+      bar_sync(3 + (warp & 3), 32 * kPfGroups);
 #pragma unroll
       for (int q = 0; q < kPfGroups; ++q) mx = fmaxf(mx, red[u & 1][q][row]);
+      mx = mx == -INFINITY ? -INFINITY : mx * p.scale_log2;  // base 2
       // lazy maximum: raise it only when a score exceeds it by more than 2^8
       // (every thread of the row takes the same decision)
       float alpha = 1.f;
@@ -456,9 +508,9 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
       }
       if (__any_sync(kFull, alpha != 1.f)) {
         // O holds P_0..P_{u-1} V: wait for the last of them (the commit that
-        // freed unit u-1's first stage), rescale this thread's columns of O
+        // freed unit u-1's first V slot), rescale this thread's columns of O
         const int pa = 2 * (u - 1);
-        ring_wait_pf(&empty_bar[pa % kStages], (pa / kStages) & 1, &s_abort, p.status);
+        ring_wait_pf(&v_empty[pa % kStages], (pa / kStages) & 1, &s_abort, p.status);
         tc_fence_after();
 #pragma unroll
         for (int oc = 0; oc < kOCols; oc += kOChunk) {
@@ -471,20 +523,21 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
         }
         tmem_wait_st();
       }
-      // pass 2: P = 2^(s - m) over the same columns, written over S as
-      // hi + lo parts (per 16 scores: 8 hi pairs, then 8 lo pairs)
+      // pass 2: P = 2^(s scale - m) over the same columns (one fused
+      // multiply-add per pair; the scale is positive, so masked columns give
+      // 2^-inf = 0), written over S as hi + lo parts (per 16 scores: 8 hi
+      // pairs, then 8 lo pairs)
       const float ms = m_used == -INFINITY ? 0.f : m_used;
       const float2 nm = make_float2(-ms, -ms);
       float2 ls = make_float2(0.f, 0.f);
 #pragma unroll
       for (int ch = 0; ch < kSCols / kSChunk; ++ch) {
-        float sv[kSChunk];
-        scores(ch, sv);
         uint32_t pw[kSChunk];
 #pragma unroll
         for (int e = 0; e < kSChunk / 2; ++e) {
-          const float2 d = add2(make_float2(sv[2 * e], sv[2 * e + 1]), nm);
-          const float2 pa2 = make_float2(ex2f(d.x), ex2f(d.y));
+          const float2 d = fma2(make_float2(__uint_as_float(sr[ch][2 * e]),
+                                            __uint_as_float(sr[ch][2 * e + 1])), sc2, nm);
+          float2 pa2 = make_float2(ex2f(d.x), ex2f(d.y));
           ls = add2(ls, pa2);
           const int w = (e / 8) * 16 + (e % 8);
           if constexpr (kBF) {
@@ -527,8 +580,8 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
     // row sums through the buffer the last unit's maxima did not use
     red[nunits & 1][cg][row] = l_run;
     const int la = 2 * (nunits - 1);                  // P_last V done frees this stage
-    ring_wait_pf(&empty_bar[la % kStages], (la / kStages) & 1, &s_abort, p.status);
-    bar_sync(1, kPfSoftmax);
+    ring_wait_pf(&v_empty[la % kStages], (la / kStages) & 1, &s_abort, p.status);
+    bar_sync(3 + (warp & 3), 32 * kPfGroups);
     float l_tot = 0.f;
 #pragma unroll
     for (int q = 0; q < kPfGroups; ++q) l_tot += red[nunits & 1][q][row];
@@ -578,7 +631,8 @@ template <int D, int BS, int KV_T>
 cudaError_t launch_prefill(const LayerMaps &maps, const PrefillParams &p, int tiles,
                            cudaStream_t st) {
   if constexpr (D == 128) {
-    if (maps.v_blk_ok) return launch_prefill_v<D, BS, KV_T, true>(maps.k, maps.v_blk, p, tiles, st);
+    if (maps.v_blk_ok && maps.k_grp_ok)
+      return launch_prefill_v<D, BS, KV_T, true>(maps.k_grp, maps.v_blk, p, tiles, st);
   }
   return launch_prefill_v<D, BS, KV_T, false>(maps.k, maps.v, p, tiles, st);
 }
@@ -633,7 +687,10 @@ extern "C" kv_status paged_attn_prefill(kv_pool *pool, int32_t layer, const void
   p.block_tables = block_tables;
   p.context_lens = context_lens;
   p.status = status_word(pool);
-  p.scale_log2 = scale * 1.4426950408889634f;
+  // scores s scale = (sign(scale) q) k |scale|: the kernel's scale is positive
+  p.scale_log2 = scale == 0.f ? 1.f : std::fabs(scale) * 1.4426950408889634f;
+  p.q_keep = scale == 0.f ? 0u : 0xFFFFFFFFu;
+  p.q_sign = scale < 0.f ? 0x80008000u : 0u;
   p.num_seqs = num_seqs;
   p.q_heads = num_q_heads;
   p.kv_heads = hkv;

@@ -62,6 +62,12 @@ struct LayerMaps {
   // declined the encoding)
   CUtensorMap v_blk;
   bool v_blk_ok = false;
+  // K as (64 elements, 8 rows, slab, 8-row group): one box brings a
+  // block-head's rows of both slabs, landing as [8-row group][slab][8 rows][128
+  // bytes], so that the 8-row groups of consecutive blocks sit 2048 bytes
+  // apart (same conditions as v_blk)
+  CUtensorMap k_grp;
+  bool k_grp_ok = false;
   int box_rows = 0;  // rows per box the maps were encoded for (0 = none yet)
 };
 

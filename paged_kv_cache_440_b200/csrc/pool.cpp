@@ -175,6 +175,30 @@ static bool encode_region_slabs(const kv_pool *p, void *base, int box_rows, CUte
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 4-D view of a 16-bit region with 256-byte rows: (64 elements, row within an
+// 8-row group, slab, 8-row group), strides (256, 128, 2048 bytes); a (64, 8, 2,
+// box_rows / 8) box lands in shared memory as [group][slab][8 rows][128 bytes],
+// 128-byte swizzled: every 1024-byte swizzle atom is 8 rows of one slab.
+static bool encode_region_groups(const kv_pool *p, void *base, int box_rows, CUtensorMap *map) {
+  std::string why;
+  auto fn = encode_fn(&why);
+  if (!fn) return false;
+  const kv_pool_desc &d = p->d;
+  if ((d.cache_dtype != KV_BF16 && d.cache_dtype != KV_FP16) || p->row_bytes != 256 ||
+      box_rows % 8 != 0)
+    return false;
+  const CUtensorMapDataType dt =
+      d.cache_dtype == KV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const cuuint64_t rows = (cuuint64_t)d.num_blocks * d.num_kv_heads * d.block_size;
+  cuuint64_t gdim[4] = {64, 8, 2, rows / 8};
+  cuuint64_t gstride[3] = {256, 128, 2048};
+  cuuint32_t box[4] = {64, 8, 2, (cuuint32_t)(box_rows / 8)};
+  cuuint32_t estride[4] = {1, 1, 1, 1};
+  return fn(map, dt, 4, base, gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool layer_maps(kv_pool *p, int layer, int box_rows, LayerMaps *out, kv_status *code) {
   std::lock_guard<std::mutex> g(p->map_mu);
   std::vector<LayerMaps> &v = p->maps[layer];
@@ -193,6 +217,7 @@ bool layer_maps(kv_pool *p, int layer, int box_rows, LayerMaps *out, kv_status *
     return false;
   }
   m.v_blk_ok = encode_region_slabs(p, layer_v(p, layer), box_rows, &m.v_blk);
+  m.k_grp_ok = encode_region_groups(p, layer_k(p, layer), box_rows, &m.k_grp);
   m.box_rows = box_rows;
   v.push_back(m);
   *out = m;

@@ -56,6 +56,62 @@ def test_prefill_matches_oracle(pkv, case):
     compare(out, ref, what=name)
 
 
+# Several hundred work items (token tile x KV head), more than one per SM: each
+# CTA walks 2 to 5 items, so Q buffers, ring stages and S/P buffers carry over
+# from one item to the next; prefixes and chunks vary (odd and even stage
+# counts, tiles past a short chunk).
+MANY = [
+    ("many-g8-d128-bs16", 32, 4, 128, 16, "bf16",
+     [400, 387, 397, 400, 262, 500, 162, 257, 117, 267],
+     [400, 350, 333, 300, 257, 200, 161, 129, 100, 17]),
+    ("many-g8-d64-bs32", 32, 4, 64, 32, "fp16",
+     [700, 650, 600, 513, 64, 999],
+     [640, 533, 500, 457, 64, 450]),
+]
+
+
+@pytest.mark.parametrize("case", MANY, ids=[c[0] for c in MANY])
+def test_prefill_many_items_per_cta(pkv, case):
+    from concurrent.futures import ThreadPoolExecutor
+    name, hq, hkv, D, bs, dt, lens, chunks = case
+    pw = W.make_prefill_workload(name, hq, hkv, D, bs, dt, lens, chunks, seed=17, device=DEV)
+    pool, out = _run(pkv, pw)
+    assert pool.status() == 0
+    wl = pw.cache
+    k, v = _cache_16(wl)
+    q64 = to_np(pw.q, np.float64)
+
+    def one(b):
+        lo, hi = int(pw.cu_q[b]), int(pw.cu_q[b + 1])
+        return attention.paged_prefill(q64[lo:hi], np.array([0, hi - lo]), k, v,
+                                       wl.block_tables[b:b + 1], wl.context_lens[b:b + 1],
+                                       wl.scale)
+
+    with ThreadPoolExecutor(8) as ex:
+        ref = np.concatenate(list(ex.map(one, range(wl.batch))))
+    compare(out, ref, what=name)
+
+
+@pytest.mark.parametrize("scale", [0.0, -0.3, 0.25])
+def test_prefill_any_finite_scale(pkv, scale):
+    """The softmax scale may be zero (every attended position weighs the same)
+    or negative; the kernel folds its sign into q and keeps its own scale
+    positive."""
+    pw = W.make_prefill_workload("scale", 16, 2, 128, 16, "bf16", [200, 77, 40], [150, 77, 3],
+                                 seed=19, device=DEV)
+    wl = pw.cache
+    pool = build_pool(pkv, wl, DEV)
+    tables, lens = device_inputs(wl, DEV)
+    cu = torch.from_numpy(pw.cu_q).to(DEV)
+    out = pkv.paged_attn_prefill(pool, 0, pw.q, cu, 150, tables, lens, 200, scale)
+    torch.cuda.synchronize()
+    assert pool.status() == 0
+    k, v = _cache_16(wl)
+    ref = attention.paged_prefill(to_np(pw.q, np.float64), pw.cu_q, k, v, wl.block_tables,
+                                  wl.context_lens, scale)
+    compare(out, ref, what="scale %g" % scale)
+
+
 def test_prefill_last_token_agrees_with_decode(pkv):
     """A one-token chunk is a decode step: both paths give the same output
     within the tolerance (different kernels, different orders)."""
