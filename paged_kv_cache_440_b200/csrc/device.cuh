@@ -368,21 +368,39 @@ __device__ __forceinline__ uint32_t quantize_row(const float (&x)[D / 32], float
   return packed;
 }
 
+// One row's D/32 16-bit values of this lane, as loaded (the loads of the
+// next row can be in flight while this one is converted and quantized).
+template <int D>
+struct RawRow {
+  uint32_t w[D / 64];
+};
+
+template <int D>
+__device__ __forceinline__ RawRow<D> load_row_raw(const uint16_t *__restrict__ src, int lane) {
+  RawRow<D> r;
+  if constexpr (D / 32 == 4) {
+    const uint2 v = *reinterpret_cast<const uint2 *>(src + lane * 4);
+    r.w[0] = v.x;
+    r.w[1] = v.y;
+  } else {
+    r.w[0] = *reinterpret_cast<const uint32_t *>(src + lane * 2);
+  }
+  return r;
+}
+
+template <int D, int IN_T>
+__device__ __forceinline__ void raw_to_f32(const RawRow<D> &r, float (&x)[D / 32]) {
+#pragma unroll
+  for (int i = 0; i < D / 64; ++i) {
+    x[2 * i] = to_f32<IN_T>(r.w[i] & 0xFFFF);
+    x[2 * i + 1] = to_f32<IN_T>(r.w[i] >> 16);
+  }
+}
+
 template <int D, int IN_T>
 __device__ __forceinline__ void load_row(const uint16_t *__restrict__ src, int lane,
                                          float (&x)[D / 32]) {
-  constexpr int E = D / 32;
-  if constexpr (E == 4) {
-    uint2 v = *reinterpret_cast<const uint2 *>(src + lane * 4);
-    x[0] = to_f32<IN_T>(v.x & 0xFFFF);
-    x[1] = to_f32<IN_T>(v.x >> 16);
-    x[2] = to_f32<IN_T>(v.y & 0xFFFF);
-    x[3] = to_f32<IN_T>(v.y >> 16);
-  } else {
-    uint32_t v = *reinterpret_cast<const uint32_t *>(src + lane * 2);
-    x[0] = to_f32<IN_T>(v & 0xFFFF);
-    x[1] = to_f32<IN_T>(v >> 16);
-  }
+  raw_to_f32<D, IN_T>(load_row_raw<D>(src, lane), x);
 }
 
 // INT8 codes of this lane's share of a key row with one fixed scale per
