@@ -471,16 +471,23 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
 #pragma unroll
       for (int ch = 0; ch < kSCols / kSChunk; ++ch) tmem_ld<kSChunk>(sbuf + ch * kSChunk, sr[ch]);
       tmem_wait_ld();
-      auto keep = [&](int cu) {                      // column cu of the unit is attended
-        const int kp = key0 + cu;
-        return kp <= rpos && kp < nkeys && ((bmask >> (cu / BS)) & 1u);
-      };
       if (need_mask) {
+        // columns past the row's last attended key (causal or tail limit),
+        // then columns of blocks whose id was invalid
+        const int lim = min(rpos, nkeys - 1) - key0 - c0;
 #pragma unroll
         for (int ch = 0; ch < kSCols / kSChunk; ++ch)
 #pragma unroll
           for (int c = 0; c < kSChunk; ++c)
-            if (!keep(c0 + ch * kSChunk + c)) sr[ch][c] = __float_as_uint(-INFINITY);
+            if (ch * kSChunk + c > lim) sr[ch][c] = __float_as_uint(-INFINITY);
+        if (bmask != kAllBlocks) {
+#pragma unroll
+          for (int ch = 0; ch < kSCols / kSChunk; ++ch)
+#pragma unroll
+            for (int c = 0; c < kSChunk; ++c)
+              if (!((bmask >> ((c0 + ch * kSChunk + c) / BS)) & 1u))
+                sr[ch][c] = __float_as_uint(-INFINITY);
+        }
       }
       // the row maximum of the raw scores (the scale is not negative: a
       // negative one enters as q's sign), over this thread's columns and then
