@@ -790,6 +790,8 @@ def cache_ops_main(args, device):
     steps = max(1, min(args.steps, 200))
     peak, peak_kind = measured_peak()
     parts = {}
+    sampler = ClockSampler(device.index if device.index is not None else 0).start()
+    t0 = time.time()
     for name, fn, inner, nbytes in ops:
         n = steps if inner == 1 and nbytes < (1 << 30) else max(1, min(steps, 20))
         for _ in range(args.warmup):
@@ -812,6 +814,8 @@ def cache_ops_main(args, device):
                        "regions": n,
                        "GB/s": round(nbytes / sec / 1e9, 1),
                        "frac": round(nbytes / sec / 1e9 / peak, 4)}
+    t1 = time.time()
+    sampler.stop()
     big = parts["append_chunk_bf16_stream"]
     print(json.dumps({
         "metric": "KV cache ops GB/s (append, quantize, copy-on-write copy)",
@@ -824,7 +828,7 @@ def cache_ops_main(args, device):
         "roofline": {"bound": "hbm", "achieved": big["GB/s"], "peak": peak, "unit": "GB/s",
                      "frac": big["frac"], "traffic": None, "kernel": "append16_kernel",
                      "peak_source": peak_kind},
-        "parts": parts,
+        "parts": parts, "clocks": sampler.summary(t0, t1),
         "gpu_launches": sum(p["regions"] * p["launches"] for p in parts.values()),
         "device_status": pool.status() | pool1.status() | qpool.status()}),
         flush=True)
