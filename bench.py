@@ -548,6 +548,14 @@ def prefill_main(args, rank, world, device):
             peak, kind = float(json.load(f)["bf16_tflops"]), "measured (MEASURED_PEAKS.json bf16_tflops, cuBLAS burst)"
     except Exception:
         peak, kind = 1590.0, "fallback 1590 TFLOP/s"
+    traffic = None
+    try:
+        with open(TRAFFIC_FILE) as f:
+            tr = json.load(f).get(args.workload)
+        if tr and tr.get("kernel_source_hash") == kernel_hash("attn_prefill.cu"):
+            traffic = tr["bytes_per_launch"]
+    except (OSError, ValueError):
+        pass
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, secs, rows, threads = prefill_oracle_sample(pw, args.cpu_budget)
@@ -570,7 +578,7 @@ def prefill_main(args, rank, world, device):
                        "l2": "L2 flushed before each timed step by reading 256 MiB"},
             "roofline": {"bound": "tensor", "achieved": round(tflops / world, 2), "peak": peak,
                          "unit": "TFLOP/s", "frac": round(tflops / world / peak, 4),
-                         "traffic": None, "kernel": "attn_prefill_kernel", "peak_source": kind,
+                         "traffic": traffic, "kernel": "attn_prefill_kernel", "peak_source": kind,
                          "kernel_ms": round(r["step_s"] * 1e3, 5)},
             "cpu_baseline": cpu,
             "e2e": None if r["e2e"] is None else {
@@ -1029,10 +1037,10 @@ def main():
         torch.distributed.destroy_process_group()
 
 
-def kernel_hash():
-    """Hash of the attention kernel source; ncu traffic figures apply only to it."""
+def kernel_hash(src="attn_decode.cu"):
+    """Hash of a kernel's source file; ncu traffic figures apply only to it."""
     import hashlib
-    with open(os.path.join(ROOT, "paged_kv_cache_440_b200", "csrc", "attn_decode.cu"), "rb") as f:
+    with open(os.path.join(ROOT, "paged_kv_cache_440_b200", "csrc", src), "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
