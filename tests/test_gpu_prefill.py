@@ -92,7 +92,7 @@ def test_prefill_many_items_per_cta(pkv, case):
     compare(out, ref, what=name)
 
 
-@pytest.mark.parametrize("scale", [0.0, -0.3, 0.25])
+@pytest.mark.parametrize("scale", [0.0, -0.3, 0.15])
 def test_prefill_any_finite_scale(pkv, scale):
     """The softmax scale may be zero (every attended position weighs the same)
     or negative; the kernel folds its sign into q and keeps its own scale
