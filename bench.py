@@ -759,7 +759,8 @@ def cache_ops_main(args, device):
     import paged_kv_cache_440_b200 as pkv
     g = torch.Generator(device=device).manual_seed(0)
     NB, bs, H, D, T, NC = 5504, 16, 8, 128, 4096, 16
-    pool = pkv.KVPool(CACHE_LAYERS, NB, bs, H, D, "bf16", device)
+    layers = max(1, args.cache_layers)
+    pool = pkv.KVPool(layers, NB, bs, H, D, "bf16", device)
     qpool = pkv.KVPool(1, NB, bs, H, D, "int8", device)
     pool1 = pkv.KVPool(1, NB, bs, H, D, "bf16", device)
     for pl in (qpool, pool1):
@@ -785,7 +786,7 @@ def cache_ops_main(args, device):
         ("append_step_bf16", lambda i: pkv.kv_append(pool1, 0, ks[0][:32], vs[0][:32], slots[0][:32]),
          1, 32 * (4 * row + 8)),
         ("append_chunk_bf16", lambda i: pkv.kv_append(pool1, 0, ks[0], vs[0], slots[0]), 1, chunk),
-        ("append_chunk_bf16_stream", lambda i: pkv.kv_append(pool, i, ks[i], vs[i], slots[i]),
+        ("append_chunk_bf16_stream", lambda i: pkv.kv_append(pool, i % layers, ks[i], vs[i], slots[i]),
          NC, chunk),
         ("append_chunk_int8", lambda i: pkv.kv_append(qpool, 0, ks[0], vs[0], slots[0]), 1,
          T * (2 * row + 2 * H * D + 2 * H * 4 + 8)),
@@ -793,7 +794,7 @@ def cache_ops_main(args, device):
          T * H * (D * 2 + D + 4)),
         ("block_copy_200_one_layer", lambda i: pkv.kv_block_copy(pool1, pairs), 1, 200 * blk),
         ("block_copy_200_all_layers", lambda i: pkv.kv_block_copy(pool, pairs), 1,
-         200 * CACHE_LAYERS * blk),
+         200 * layers * blk),
     ]
     steps = max(1, min(args.steps, 200))
     peak, peak_kind = measured_peak()
@@ -831,7 +832,8 @@ def cache_ops_main(args, device):
         "warmup": args.warmup, "ms_per_step": round(big["us"] * big["launches"] / 1e3, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": CACHE_OPS, "l2": "L2 flushed before each timed region by reading "
+        "config": {"workload": CACHE_OPS, "layers": layers,
+                   "l2": "L2 flushed before each timed region by reading "
                    "256 MiB; a stream's 16 chunks are distinct (537 MB, above the L2)"},
         "roofline": {"bound": "hbm", "achieved": big["GB/s"], "peak": peak, "unit": "GB/s",
                      "frac": big["frac"], "traffic": None, "kernel": "append16_kernel",
@@ -923,6 +925,8 @@ def main():
                     help="kv_append + paged_attn_decode instead of paged_attn_decode_append")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--cache-layers", type=int, default=CACHE_LAYERS,
+                    help="cache_ops: layers of the pool (the copy-on-write copy covers all of them)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
