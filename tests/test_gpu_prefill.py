@@ -41,6 +41,7 @@ CASES = [
     ("g16-d64-bs16", 32, 2, 64, 16, "bf16", [90, 17], [41, 17]),
     ("g3-d128-bs16", 6, 2, 128, 16, "fp16", [70, 140], [70, 60]),
     ("g64-d128-bs16", 64, 1, 128, 16, "bf16", [40, 3], [9, 3]),
+    ("g4-fp16-d128-bs32", 8, 2, 128, 32, "fp16", [333, 97, 64], [200, 97, 33]),
 ]
 
 
@@ -143,6 +144,29 @@ def test_prefill_70b_shape_sampled(pkv):
                                                     h // 8, wl.scale)
                               for h in range(64)]) for b, i in rows])
     compare(got, ref, what="prefill70b")
+
+
+def test_prefill_bad_block_id_is_reported(pkv):
+    """A block id outside the pool is reported in the status word and its
+    positions are skipped; outputs stay finite and the other sequence's rows
+    match the oracle."""
+    pw = W.make_prefill_workload("badid", 16, 2, 128, 16, "bf16", [300, 90], [120, 40], seed=21,
+                                 device=DEV)
+    wl = pw.cache
+    pool = build_pool(pkv, wl, DEV)
+    tables, lens = device_inputs(wl, DEV)
+    tables[0, 3] = wl.num_blocks + 5              # outside the pool
+    cu = torch.from_numpy(pw.cu_q).to(DEV)
+    pool.status_clear()
+    out = pkv.paged_attn_prefill(pool, 0, pw.q, cu, 120, tables, lens, 300, wl.scale)
+    torch.cuda.synchronize()
+    assert pool.status() & 1
+    assert torch.all(torch.isfinite(out.float()))
+    k, v = _cache_16(wl)
+    lo = int(pw.cu_q[1])
+    ref = attention.paged_prefill(to_np(pw.q[lo:], np.float64), np.array([0, 40]), k, v,
+                                  wl.block_tables[1:], wl.context_lens[1:], wl.scale)
+    compare(out[lo:], ref, what="good sequence")
 
 
 def test_prefill_bad_chunk_is_reported(pkv):
