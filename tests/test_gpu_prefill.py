@@ -113,6 +113,34 @@ def test_prefill_any_finite_scale(pkv, scale):
     compare(out, ref, what="scale %g" % scale)
 
 
+def _random_case(seed):
+    """A seeded random prefill shape: group size, head_dim, block size, dtype,
+    2 to 5 sequences with prefixes of 0 to 300 and chunks of 1 to 160 tokens."""
+    rng = np.random.default_rng(seed)
+    hkv = int(rng.choice([1, 2, 4]))
+    g = int(rng.choice([1, 2, 4, 8, 16]))
+    D = int(rng.choice([64, 128]))
+    bs = int(rng.choice([16, 32]))
+    dt = str(rng.choice(["bf16", "fp16"]))
+    n = int(rng.integers(2, 6))
+    chunks = [int(x) for x in rng.integers(1, 161, n)]
+    lens = [c + int(rng.integers(0, 301)) for c in chunks]
+    return ("rand%d" % seed, g * hkv, hkv, D, bs, dt, lens, chunks)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_prefill_random_shapes(pkv, seed):
+    name, hq, hkv, D, bs, dt, lens, chunks = _random_case(seed)
+    pw = W.make_prefill_workload(name, hq, hkv, D, bs, dt, lens, chunks, seed=100 + seed,
+                                 device=DEV)
+    pool, out = _run(pkv, pw)
+    assert pool.status() == 0
+    k, v = _cache_16(pw.cache)
+    ref = attention.paged_prefill(to_np(pw.q, np.float64), pw.cu_q, k, v, pw.cache.block_tables,
+                                  pw.cache.context_lens, pw.cache.scale)
+    compare(out, ref, what=name)
+
+
 def test_prefill_last_token_agrees_with_decode(pkv):
     """A one-token chunk is a decode step: both paths give the same output
     within the tolerance (different kernels, different orders)."""
