@@ -869,6 +869,24 @@ def reference_arm(args, world):
         metric, unit, what = ("chunked prefill attention TFLOP/s", "TFLOP/s",
                               "one new-token row (all %d heads)" % wl.q_heads)
         scale_out = 1e12
+    elif args.workload == "cache_ops":
+        from oracle import cache_ops
+        NB, bs, H, D, T = 5504, 16, 8, 128, 4096
+        rng = np.random.default_rng(0)
+        kc = np.zeros((NB, H, bs, D), dtype=np.uint16)
+        vc = np.zeros_like(kc)
+        kn = rng.integers(0, 1 << 16, (T, H, D), dtype=np.uint16)
+        vn = rng.integers(0, 1 << 16, (T, H, D), dtype=np.uint16)
+        slots = rng.permutation(NB * bs)[:T].astype(np.int64)
+
+        def one(n):
+            cache_ops.append(kc, vc, kn, vn, slots, bs)
+            return T * (4 * H * D * 2 + 8)
+        desc = CACHE_OPS
+        wl = type("CacheOps", (), {"batch": T})
+        metric, unit, what = ("KV cache ops GB/s (append, quantize, copy-on-write copy)", "GB/s",
+                              "one 4096-token bf16 chunk appended at random rows")
+        scale_out = 1e9
     else:
         desc, make = WORKLOADS[args.workload]
         wl = make("cpu")
@@ -883,7 +901,7 @@ def reference_arm(args, world):
         scale_out = 1e9
     times, work = [], 0
     for n in range(args.warmup + args.steps):
-        if args.workload in PREFILL_WORKLOADS:
+        if args.workload in PREFILL_WORKLOADS or args.workload == "cache_ops":
             t0 = time.perf_counter()
             w = one(n)
             dt = time.perf_counter() - t0
@@ -902,7 +920,8 @@ def reference_arm(args, world):
         "impl": "reference", "metric": metric, "value": round(value, 6), "unit": unit,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(secs / args.steps * 1e3, 3), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "u16" if args.workload == "cache_ops" else "f64", "data": "synthetic",
         "config": {"workload": desc, "batch": wl.batch},
         "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": threads,
                          "kind": "oracle", "sample": sample},
