@@ -1,6 +1,6 @@
 // Device-side building blocks for sm_100a: mbarrier waits with a time limit,
-// TMA tile loads and 1-D bulk copies into shared memory (CTA-local, never
-// multicast), warp-level fragment loads and tensor-core MMA, and the
+// TMA tile loads and 1-D bulk copies into this CTA's own shared memory only,
+// warp-level fragment loads and tensor-core MMA, and the
 // conversions of 1-byte KV codes to fp16.
 #pragma once
 
