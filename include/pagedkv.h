@@ -403,7 +403,9 @@ kv_status paged_attn_merge(kv_pool *pool, int32_t num_seqs, int32_t num_q_heads,
  *              sequences one after another (row cu_q_lens[b] + i).
  *   cu_q_lens  device int32 [num_seqs + 1], non-decreasing, cu_q_lens[0] = 0,
  *              cu_q_lens[num_seqs] = total_q; max_q_len >= every c_b (host).
- *   Other arguments as paged_attn_decode. Up to 128 query heads per kv head.
+ *   Other arguments as paged_attn_decode (any finite scale: zero weighs every
+ *   attended position the same). Up to 128 query heads per kv head and 65535
+ *   sequences per call (KV_ERR_UNSUPPORTED beyond).
  * A sequence with c_b > context_lens[b], a length beyond the table, or rows
  * outside [0, total_q) sets KV_DEVERR_CONTEXT and its rows are not written;
  * an invalid block id sets KV_DEVERR_BLOCK_ID and its positions are skipped.
