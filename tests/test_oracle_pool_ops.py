@@ -6,7 +6,9 @@ pool model.
 * internal waste below one block (at most 15 tokens for 16-token blocks);
 * append and copy checked at explicit flat byte offsets, computed here from the
   [block][kv_head][row][dim] layout, not through the oracle;
-* copy-on-write leaves every other sharer's logical sequence unchanged.
+* copy-on-write leaves every other sharer's logical sequence unchanged;
+* the scale-bytes product against a count of the scales the oracle's append
+  writes.
 """
 import json
 import os
@@ -83,6 +85,26 @@ def test_append_quantized_places_codes_and_scales():
     codes, sc = quant.quantize_rows(kn, "int8")
     assert np.array_equal(kc[1, :, 1], codes[0]) and np.array_equal(ks[3, :, 7], sc[1])
     assert np.array_equal(kc[0, :, 0], codes[2])
+
+
+def test_scale_bytes_counts_the_scales_append_writes():
+    """scale_bytes against a brute-force count: append T tokens of a quantized
+    cache in each of 3 layers through the oracle's own append and count the
+    fp32 scale entries it writes (K and V, every head), 4 bytes each."""
+    rng = np.random.default_rng(4)
+    layers, NB, Hkv, bs, D, T = 3, 6, 2, 8, 16, 29
+    written = 0
+    for _ in range(layers):
+        kc = np.zeros((NB, Hkv, bs, D), np.int8)
+        vc = np.zeros((NB, Hkv, bs, D), np.int8)
+        ks = np.full((NB, Hkv, bs), np.nan, np.float32)
+        vs = np.full((NB, Hkv, bs), np.nan, np.float32)
+        kn = rng.standard_normal((T, Hkv, D)).astype(np.float32)
+        vn = rng.standard_normal((T, Hkv, D)).astype(np.float32)
+        slots = rng.permutation(NB * bs)[:T]
+        cache_ops.append_quantized(kc, vc, ks, vs, kn, vn, slots, bs, "int8")
+        written += int(np.count_nonzero(~np.isnan(ks)) + np.count_nonzero(~np.isnan(vs)))
+    assert written * 4 == pool.scale_bytes(layers, Hkv, 4, T)
 
 
 def test_block_copy_and_cow_keeps_sharers_intact():
