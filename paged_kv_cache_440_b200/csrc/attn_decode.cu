@@ -198,6 +198,19 @@ __device__ __forceinline__ float load_q(const void *q, int64_t idx) {
   else return __half2float(__ushort_as_half(bits));
 }
 
+// Query elements idx .. idx + 3 (idx a multiple of 4) with one 8-byte load.
+template <int Q_T>
+__device__ __forceinline__ void load_q4(const void *q, int64_t idx, float (&v)[4]) {
+  const uint2 u = *reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(q) + idx);
+  const uint32_t w[2] = {u.x, u.y};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint16_t bits = static_cast<uint16_t>(w[i >> 1] >> (16 * (i & 1)));
+    if constexpr (Q_T == KV_BF16) v[i] = __uint_as_float(static_cast<uint32_t>(bits) << 16);
+    else v[i] = __half2float(__ushort_as_half(bits));
+  }
+}
+
 template <int Q_T>
 __device__ __forceinline__ void store_out(void *out, int64_t idx, float v) {
   if constexpr (Q_T == KV_BF16) static_cast<__nv_bfloat16 *>(out)[idx] = __float2bfloat16_rn(v);
@@ -340,6 +353,31 @@ struct Consumer {
       // 64(kp / 2) + 32half + 8cq + 2e + kp % 2.
       float qv[D / 32][2][4];
       float amax = 0.f;
+      // INT8 slots (kp, hf, 0..3) are 4 consecutive dims; INT4 slots (kp, hf,
+      // 0..3) of kp = 2c and 2c + 1 interleave 8 consecutive dims
+#pragma unroll
+      for (int kp = 0; kp < D / 32; ++kp)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          if constexpr (KV_T == KV_INT4) {
+            if ((kp & 1) == 0) {
+              float lo[4] = {0.f, 0.f, 0.f, 0.f}, hi4[4] = {0.f, 0.f, 0.f, 0.f};
+              const int64_t base = qrow + (kp >> 1) * 64 + 32 * hf + 8 * cq;
+              if (hv) {
+                load_q4<Q_T>(p.q, base, lo);
+                load_q4<Q_T>(p.q, base + 4, hi4);
+              }
+              qv[kp][hf][0] = lo[0]; qv[kp][hf][1] = lo[2]; qv[kp][hf][2] = hi4[0]; qv[kp][hf][3] = hi4[2];
+              qv[kp + 1][hf][0] = lo[1]; qv[kp + 1][hf][1] = lo[3];
+              qv[kp + 1][hf][2] = hi4[1]; qv[kp + 1][hf][3] = hi4[3];
+            }
+          } else {
+            float v4[4] = {0.f, 0.f, 0.f, 0.f};
+            if (hv) load_q4<Q_T>(p.q, qrow + 32 * kp + 16 * hf + 4 * cq, v4);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) qv[kp][hf][e] = v4[e];
+          }
+        }
 #pragma unroll
       for (int kp = 0; kp < D / 32; ++kp)
 #pragma unroll
@@ -348,7 +386,7 @@ struct Consumer {
           for (int e = 0; e < 4; ++e) {
             const int dim = KV_T == KV_INT4 ? (kp >> 1) * 64 + 32 * hf + 8 * cq + 2 * e + (kp & 1)
                                             : 32 * kp + 16 * hf + 4 * cq + e;
-            float v = hv ? load_q<Q_T>(p.q, qrow + dim) : 0.f;
+            float v = qv[kp][hf][e];
             if constexpr (KCH) {
               // keys code k / s_c: the channel scale moves to the query,
               // q . k = sum_c (q_c s_c) code_c
@@ -407,13 +445,15 @@ struct Consumer {
       float qv[KS][4];
       float amax = 0.f;
 #pragma unroll
-      for (int ks = 0; ks < KS; ++ks)
+      for (int ks = 0; ks < KS; ++ks) {
+        float v4[4] = {0.f, 0.f, 0.f, 0.f};
+        if (hv) load_q4<Q_T>(p.q, qrow + 16 * ks + 4 * cq, v4);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int dim = 16 * ks + 4 * cq + e;
-          qv[ks][e] = hv ? load_q<Q_T>(p.q, qrow + dim) : 0.f;
-          amax = fmaxf(amax, fabsf(qv[ks][e]));
+          qv[ks][e] = v4[e];
+          amax = fmaxf(amax, fabsf(v4[e]));
         }
+      }
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
       int ex = 0;
@@ -421,10 +461,18 @@ struct Consumer {
         frexpf(amax, &ex);
         ex = 15 - ex;  // amax * 2^ex in [2^14, 2^15)
       }
+      // x * 2^ex is exact while 2^ex is a normal float (ex >= -113 here, as
+      // amax * 2^ex < 2^15); ex > 127 only for amax below 2^-112
+      const bool pw = ex <= 127;
+      const float p2 = __int_as_float((127 + (pw ? ex : 0)) << 23);
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) qv[ks][e] = pw ? qv[ks][e] * p2 : ldexpf(qv[ks][e], ex);
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
-        qb[ks][0] = pack2<false>(ldexpf(qv[ks][0], ex), ldexpf(qv[ks][1], ex));
-        qb[ks][1] = pack2<false>(ldexpf(qv[ks][2], ex), ldexpf(qv[ks][3], ex));
+        qb[ks][0] = pack2<false>(qv[ks][0], qv[ks][1]);
+        qb[ks][1] = pack2<false>(qv[ks][2], qv[ks][3]);
       }
       // the score columns of this lane are heads 2cq and 2cq+1
       const int ex0 = __shfl_sync(0xffffffffu, ex, (2 * cq) * 4);
