@@ -238,6 +238,7 @@ class OracleStep:
             self.kn, self.vn = _host_f32(wl.k_new), _host_f32(wl.v_new)
             self.tables = wl.block_tables
         self.ready = set()
+        self.outs = {}          # sequence -> the oracle's outputs of all its heads
 
     def prepare(self, b):
         """Untimed: sequence b's cached history in the oracle's cache."""
@@ -322,8 +323,8 @@ class OracleStep:
                 vd = quant.dequantize(unpack(self.vc[ids]), self.vs[ids], kind)
             tab = np.full_like(self.tables, -1)
             tab[b, :nblk] = np.arange(nblk)
-        for h in range(wl.q_heads):
-            attention.decode_one(self.q, kd, vd, tab, wl.context_lens, wl.scale, b, h)
+        self.outs[b] = np.stack([attention.decode_one(self.q, kd, vd, tab, wl.context_lens,
+                                                      wl.scale, b, h) for h in range(wl.q_heads)])
         e = elt_bytes(kind)
         nb = int(wl.context_lens[b]) * wl.kv_heads * wl.head_dim * 2 * e \
             + 2 * wl.q_heads * wl.head_dim * 2 + wl.kv_heads * wl.head_dim * 2 * 2 * (1 + e)
@@ -336,7 +337,8 @@ def oracle_sample(wl, budget_s=15.0, threads=None):
     """Time the CPU oracle (as it stands) on a bounded sample of the step: the
     append and decode of whole sequences, taken in order until ~budget_s of
     CPU work. threads: BLAS threads for the run (None: as configured).
-    Returns (GB/s in the metric's bytes, seconds, sequences, threads used)."""
+    Returns (GB/s in the metric's bytes, seconds, sequences, threads used,
+    {sequence: the oracle's outputs [Hq, D]})."""
     from threadpoolctl import threadpool_info, threadpool_limits
     ost = OracleStep(wl)
     with threadpool_limits(limits=threads):
@@ -352,7 +354,20 @@ def oracle_sample(wl, budget_s=15.0, threads=None):
             done += 1
             if t_total >= budget_s or t_setup >= 2 * budget_s:
                 break
-    return nbytes / t_total / 1e9, t_total, done, used
+    return nbytes / t_total / 1e9, t_total, done, used, ost.outs
+
+
+def output_check(gpu_out, oracle_outs, tol=1e-2):
+    """The step's GPU outputs against the oracle's on the sampled sequences:
+    max abs and max rel (floor 1e-2 on |oracle|) error, both within tol."""
+    g = _host_f32(gpu_out).astype(np.float64)
+    ea = er = 0.0
+    for b, o in oracle_outs.items():
+        err = np.abs(g[b] - o)
+        ea = max(ea, float(err.max()))
+        er = max(er, float((err / np.maximum(np.abs(o), 1e-2)).max()))
+    return {"sequences": sorted(int(b) for b in oracle_outs), "max_abs": ea, "max_rel": er,
+            "tolerance": tol, "ok": bool(ea <= tol and er <= tol)}
 
 
 # ------------------------------------------------------------------ shared prefix
@@ -659,6 +674,7 @@ def run_ours(args, rank, world, device):
         evs[i][1].record(stream)
     torch.cuda.synchronize(device)
     t1 = time.time()
+    out_timed = out.clone()        # the last timed step's outputs, for the output check
     if world > 1:
         torch.distributed.barrier()
     # The attention kernel alone, same conditions (L2 flushed before each launch),
@@ -735,7 +751,7 @@ def run_ours(args, rank, world, device):
         e2e = (e2e_s, h2d, d2h)
 
     dec_bytes, app_bytes = step_bytes(wl)
-    res = {"wl": wl, "desc": desc, "G": G, "step_s": step_s, "part_s": part_s,
+    res = {"wl": wl, "desc": desc, "G": G, "step_s": step_s, "part_s": part_s, "out": out_timed,
            "dec_bytes": dec_bytes, "app_bytes": app_bytes, "clocks": clocks, "fused": fused,
            "status": status, "e2e": e2e, "launches": args.steps * (2 if fused else 3),
            "wall": t1 - t0, "step_ms_median": float(np.median(step_ms))}
@@ -1009,13 +1025,15 @@ def main():
                       "no DRAM capture of the current kernel source: HBM fraction not reported")
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        g_cpu, secs, nseq, threads = oracle_sample(wl, args.cpu_budget)
-        g_one, secs1, nseq1, _ = oracle_sample(wl, args.cpu_budget / 3, threads=1)
+        g_cpu, secs, nseq, threads, oouts = oracle_sample(wl, args.cpu_budget)
+        g_one, secs1, nseq1, _, _ = oracle_sample(wl, args.cpu_budget / 3, threads=1)
         cpu = {"value": round(g_cpu, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
                "sample": "%d of %d sequences (append + all %d heads each), %.1f s of fp64 numpy"
                          % (nseq, wl.batch, wl.q_heads, secs),
                "one_thread": {"value": round(g_one, 4), "unit": "GB/s",
-                              "sample": "%d sequences, %.1f s" % (nseq1, secs1)}}
+                              "sample": "%d sequences, %.1f s" % (nseq1, secs1)},
+               # the timed step's outputs of the sampled sequences against the oracle's
+               "output_check": output_check(r["out"], oouts)}
     if rank == 0:
         line = {
             "metric": METRIC, "value": round(gbs, 2), "unit": "GB/s", "n_gpus": world,
