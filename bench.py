@@ -358,15 +358,16 @@ def oracle_sample(wl, budget_s=15.0, threads=None):
 
 
 def output_check(gpu_out, oracle_outs, tol=1e-2):
-    """The step's GPU outputs against the oracle's on the sampled sequences:
-    max abs and max rel (floor 1e-2 on |oracle|) error, both within tol."""
+    """The step's GPU outputs against the oracle's on the sampled sequences
+    (the first ones of the batch, in order): how many, max abs and max rel
+    (floor 1e-2 on |oracle|) error, both within tol."""
     g = _host_f32(gpu_out).astype(np.float64)
     ea = er = 0.0
     for b, o in oracle_outs.items():
         err = np.abs(g[b] - o)
         ea = max(ea, float(err.max()))
         er = max(er, float((err / np.maximum(np.abs(o), 1e-2)).max()))
-    return {"sequences": sorted(int(b) for b in oracle_outs), "max_abs": ea, "max_rel": er,
+    return {"sequences": len(oracle_outs), "max_abs": ea, "max_rel": er,
             "tolerance": tol, "ok": bool(ea <= tol and er <= tol)}
 
 
