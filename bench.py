@@ -359,8 +359,9 @@ def oracle_sample(wl, budget_s=15.0, threads=None):
 
 def output_check(gpu_out, oracle_outs, tol=1e-2):
     """The step's GPU outputs against the oracle's on the sampled sequences
-    (the first ones of the batch, in order): how many, max abs and max rel
-    (floor 1e-2 on |oracle|) error, both within tol."""
+    (decode: the first ones of the batch, in order) or new-token rows
+    (prefill): how many, max abs and max rel (floor 1e-2 on |oracle|) error,
+    both within tol. gpu_out's first index is the sample's key."""
     g = _host_f32(gpu_out).astype(np.float64)
     ea = er = 0.0
     for b, o in oracle_outs.items():
@@ -495,6 +496,7 @@ def run_prefill(args, rank, world, device):
     torch.cuda.synchronize(device)
     t1 = time.time()
     sampler.stop()
+    out_timed = out.clone()        # the last timed step's outputs, for the output check
     step_s = float(np.mean([a.elapsed_time(b_) for a, b_ in evs])) / 1e3
     step_s, = max_over_ranks([step_s], world, device)
     e2e = None
@@ -517,12 +519,14 @@ def run_prefill(args, rank, world, device):
                 times.append(a.elapsed_time(b_) / 1e3)
         e2e_s, = max_over_ranks([float(np.mean(times))], world, device)
         e2e = (e2e_s, h_q.numel() * 2, h_out.numel() * 2)
-    return {"pw": pw, "desc": desc, "step_s": step_s, "clocks": sampler.summary(t0, t1),
+    return {"pw": pw, "desc": desc, "step_s": step_s, "out": out_timed,
+            "clocks": sampler.summary(t0, t1),
             "status": pool.status(), "e2e": e2e, "launches": args.steps}
 
 
 def prefill_oracle_sample(pw, budget_s, threads=None):
-    """TFLOP/s of the fp64 oracle on a bounded sample of the prefill rows."""
+    """TFLOP/s of the fp64 oracle on a bounded sample of the prefill rows:
+    (TFLOP/s, seconds, rows, {new-token row: its outputs [Hq, D]}, threads)."""
     from threadpoolctl import threadpool_info, threadpool_limits
     with threadpool_limits(limits=threads):
         used = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
@@ -536,21 +540,22 @@ def _prefill_oracle_sample(pw, budget_s):
     v = wl.v_fill.float().cpu().numpy()
     q = pw.q.float().cpu().numpy().astype(np.float64)
     G = wl.q_heads // wl.kv_heads
-    flops, t, rows = 0, 0.0, 0
+    flops, t, rows, outs = 0, 0.0, 0, {}
     for b in range(wl.batch):
         L, c = int(wl.context_lens[b]), int(pw.chunk_lens[b])
         for i in range(0, c, 37):                     # a spread of positions
             pos = L - c + i
+            r = int(pw.cu_q[b]) + i
             t0 = time.perf_counter()
-            for h in range(wl.q_heads):
-                attention.prefill_one(q[pw.cu_q[b] + i, h], k, v, wl.block_tables[b], pos,
-                                      h // G, wl.scale)
+            outs[r] = np.stack([attention.prefill_one(q[r, h], k, v, wl.block_tables[b], pos,
+                                                      h // G, wl.scale)
+                                for h in range(wl.q_heads)])
             t += time.perf_counter() - t0
             flops += 4 * wl.head_dim * wl.q_heads * (pos + 1)
             rows += 1
             if t >= budget_s:
-                return flops / t / 1e12, t, rows
-    return flops / t / 1e12, t, rows
+                return flops / t / 1e12, t, rows, outs
+    return flops / t / 1e12, t, rows, outs
 
 
 def prefill_main(args, rank, world, device):
@@ -574,12 +579,14 @@ def prefill_main(args, rank, world, device):
         pass
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, secs, rows, threads = prefill_oracle_sample(pw, args.cpu_budget)
-        v1, secs1, rows1, _ = prefill_oracle_sample(pw, args.cpu_budget / 3, threads=1)
+        v, secs, rows, oouts, threads = prefill_oracle_sample(pw, args.cpu_budget)
+        v1, secs1, rows1, _, _ = prefill_oracle_sample(pw, args.cpu_budget / 3, threads=1)
         cpu = {"value": round(v, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                "sample": "%d new-token rows (all 64 heads each), %.1f s of fp64 numpy" % (rows, secs),
                "one_thread": {"value": round(v1, 6), "unit": "TFLOP/s",
-                              "sample": "%d rows, %.1f s" % (rows1, secs1)}}
+                              "sample": "%d rows, %.1f s" % (rows1, secs1)},
+               # the timed step's outputs of the sampled rows against the oracle's
+               "output_check": output_check(r["out"], oouts)}
     if rank == 0:
         line = {
             "metric": "chunked prefill attention TFLOP/s", "value": round(tflops, 2),

@@ -60,3 +60,23 @@ def test_output_check_covers_a_quantized_cache():
     good = torch.from_numpy(np.stack([outs[b] for b in range(3)]).astype(np.float32))
     assert bench.output_check(good.to(torch.bfloat16), outs)["ok"]
     assert not bench.output_check(torch.zeros_like(good).to(torch.bfloat16), outs)["ok"]
+
+
+def test_prefill_output_check_rows_are_the_oracle_prefill():
+    """The prefill line's oracle rows are those of the chunked-prefill oracle
+    (new token i of sequence b at position L_b - c_b + i), and a wrong row is
+    flagged."""
+    pw = W.make_prefill_workload("p", 8, 2, 64, 16, "bf16", [90, 120], [80, 41], seed=5)
+    v, secs, rows, outs, threads = bench.prefill_oracle_sample(pw, budget_s=60.0)
+    assert rows == len(outs) and sorted(outs) == [0, 37, 74, 80, 117]
+    wl = pw.cache
+    q = bench._host_f32(pw.q).astype(np.float64)
+    ref = attention.paged_prefill(q, pw.cu_q, bench._host_f32(wl.k_fill),
+                                  bench._host_f32(wl.v_fill), wl.block_tables, wl.context_lens,
+                                  wl.scale)
+    for r, o in outs.items():
+        np.testing.assert_allclose(o, ref[r], rtol=1e-12, atol=1e-14)
+    gpu = torch.from_numpy(ref.astype(np.float32)).to(torch.bfloat16)
+    assert bench.output_check(gpu, outs)["ok"]
+    gpu[74, 3, 0] += 0.5
+    assert not bench.output_check(gpu, outs)["ok"]
