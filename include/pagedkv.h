@@ -354,6 +354,55 @@ kv_status paged_attn_decode_append(kv_pool *pool, int32_t layer, const void *q,
                                    int32_t num_ctas, void *workspace,
                                    uint64_t workspace_bytes, kv_stream_t stream);
 
+/* A decode step for sequences that share a prompt prefix: the first
+ * prefix_blocks entries of every row of block_tables are the same block ids,
+ * the shared prefix's blocks [bjdmk.com.cn/news/6246348, §3.2: requests with
+ * one system prompt map it to the same physical blocks]. Results are those of
+ * paged_attn_decode_append (k_new, v_new given) or paged_attn_decode (both
+ * null) on the same arguments, within their tolerance. The work is split three
+ * ways; the pages give no method for it.
+ *   1. The shared positions 0 .. P - 1 (P = prefix_blocks * block_size) for
+ *      all sequences at once. Per kv head this is a dense (sequences x group)
+ *      by P contraction, run on the tensor cores (the chunked-prefill kernel,
+ *      without its causal limit); its per-(sequence, head) partials go to the
+ *      workspace. Row 0 of block_tables names the prefix's blocks.
+ *   2. Each sequence's positions P .. L_b - 1, with the step's append, through
+ *      the decode kernel.
+ *   3. The merge, with the prefix partial folded in.
+ * 16-bit caches only (a 1-byte or 4-bit cache: KV_ERR_UNSUPPORTED);
+ * q_dtype must be the cache dtype. At most 128 query heads per kv head (8 with
+ * an append), else KV_ERR_UNSUPPORTED.
+ *   prefix_blocks  1 <= prefix_blocks < max_blocks_per_seq, and
+ *                  P <= max_context, else KV_ERR_INVALID.
+ *   context_lens   P <= L_b <= max_context for every sequence. L_b = P gives
+ *                  the prefix's attention alone. On the device, a length
+ *                  outside that range raises KV_DEVERR_CONTEXT and zeros the
+ *                  sequence's outputs. With an append, L_b = P also raises
+ *                  KV_DEVERR_CONTEXT: the new token would fall in the shared
+ *                  blocks, so it is not written.
+ *   workspace      device, 256-byte aligned, at least
+ *                  paged_attn_cascade_workspace_bytes for the same num_seqs,
+ *                  num_q_heads and num_ctas.
+ * Other arguments as paged_attn_decode_append. Three kernels on the stream;
+ * asynchronous; no allocation. */
+kv_status paged_attn_decode_cascade(kv_pool *pool, int32_t layer, const void *q,
+                                    const void *k_new, const void *v_new,
+                                    int32_t q_dtype, int32_t num_seqs,
+                                    int32_t num_q_heads, const int32_t *block_tables,
+                                    int32_t max_blocks_per_seq,
+                                    const int32_t *context_lens, int32_t max_context,
+                                    int32_t prefix_blocks, float scale, void *out,
+                                    int32_t num_ctas, void *workspace,
+                                    uint64_t workspace_bytes, kv_stream_t stream);
+
+/* Workspace bytes for paged_attn_decode_cascade: the decode workspace
+ * (paged_attn_workspace_bytes) plus the prefix pass's partials,
+ * num_seqs * num_q_heads * (head_dim + 2) * 4 bytes (each part rounded up to
+ * 256 bytes). */
+kv_status paged_attn_cascade_workspace_bytes(const kv_pool *pool, int32_t num_seqs,
+                                             int32_t num_q_heads, int32_t num_ctas,
+                                             uint64_t *bytes);
+
 /* Phase 1 alone: the persistent attention kernel. Writes out for the units it
  * finishes and the workspace partials and bookkeeping for split units. */
 kv_status paged_attn_partition(kv_pool *pool, int32_t layer, const void *q,

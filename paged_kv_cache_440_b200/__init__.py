@@ -8,7 +8,8 @@ been built (``python -m paged_kv_cache_440_b200.build``). There is no fallback.
 _EXPORTS = (
     "KVPool", "PagedKVError", "PrefixCache", "default_ctas", "kv_append", "kv_block_copy",
     "kv_quantize", "make_workspace", "paged_attn_decode", "paged_attn_decode_append",
-    "paged_attn_decode_static", "paged_attn_partition_append",
+    "paged_attn_decode_static", "paged_attn_partition_append", "paged_attn_decode_cascade",
+    "cascade_workspace_bytes", "make_cascade_workspace",
     "paged_attn_merge", "paged_attn_prefill",
     "paged_attn_partition", "required_bytes", "selftest_wait_timeout", "version",
     "workspace_bytes",

@@ -99,6 +99,9 @@ _SIGS = {
     "paged_attn_partition_append": [_P, _I32, _P, _P, _P, _I32, _I32, _I32, _P, _I32, _P, _I32,
                                     _F, _P, _I32, _P, _U64, _P],
     "paged_attn_merge": [_P, _I32, _I32, _P, _I32, _I32, _I32, _I32, _P, _P, _U64, _P],
+    "paged_attn_decode_cascade": [_P, _I32, _P, _P, _P, _I32, _I32, _I32, _P, _I32, _P, _I32,
+                                  _I32, _F, _P, _I32, _P, _U64, _P],
+    "paged_attn_cascade_workspace_bytes": [_P, _I32, _I32, _I32, _PU64],
     "kv_selftest_wait_timeout": [_P, ctypes.c_uint32, _P],
     "paged_attn_decode_static": [_P, _I32, _P, _I32, _I32, _I32, _P, _I32, _P, _I32, _F, _P,
                                  _I32, _P],
@@ -440,6 +443,47 @@ def paged_attn_decode_append(pool, layer, q, k_new, v_new, block_tables, context
                                        block_tables.shape[1], _ptr(context_lens), max_context,
                                        float(scale), _ptr(out), num_ctas, _ptr(workspace),
                                        workspace.numel(), _stream(stream, pool.device)))
+    return out
+
+
+def cascade_workspace_bytes(pool, num_seqs, num_q_heads, num_ctas=0):
+    n = ctypes.c_uint64()
+    check(lib.paged_attn_cascade_workspace_bytes(pool.handle, num_seqs, num_q_heads, num_ctas,
+                                                 ctypes.byref(n)))
+    return n.value
+
+
+def make_cascade_workspace(pool, num_seqs, num_q_heads, num_ctas=0):
+    n = cascade_workspace_bytes(pool, num_seqs, num_q_heads, num_ctas)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=pool.device)
+
+
+def paged_attn_decode_cascade(pool, layer, q, block_tables, context_lens, max_context,
+                              prefix_blocks, scale, k_new=None, v_new=None, out=None,
+                              num_ctas=0, workspace=None, stream=None):
+    """Decode step for sequences whose block tables begin with the same
+    prefix_blocks shared blocks: the prefix once for all of them on the tensor
+    cores, each sequence's remaining positions (with the new token's append
+    when k_new, v_new [B, Hkv, D] are given) through the decode kernel, then
+    the merge. Returns out."""
+    B, Hq, out = _attn_args(pool, q, block_tables, context_lens, out)
+    if (k_new is None) != (v_new is None):
+        raise ValueError("k_new and v_new go together")
+    if k_new is not None:
+        _need(k_new, "k_new", q.dtype, pool.device)
+        _need(v_new, "v_new", q.dtype, pool.device)
+        if tuple(k_new.shape) != (B, pool.num_kv_heads, pool.head_dim) or v_new.shape != k_new.shape:
+            raise ValueError("k_new, v_new must be [B, kv_heads, head_dim]")
+    if workspace is None:
+        workspace = make_cascade_workspace(pool, B, Hq, num_ctas)
+    kn = None if k_new is None else _ptr(k_new)
+    vn = None if v_new is None else _ptr(v_new)
+    check(lib.paged_attn_decode_cascade(pool.handle, layer, _ptr(q), kn, vn,
+                                        TORCH_CODES[q.dtype], B, Hq, _ptr(block_tables),
+                                        block_tables.shape[1], _ptr(context_lens), max_context,
+                                        prefix_blocks, float(scale), _ptr(out), num_ctas,
+                                        _ptr(workspace), workspace.numel(),
+                                        _stream(stream, pool.device)))
     return out
 
 

@@ -101,7 +101,21 @@ struct AttnParams {
   int num_blocks;      // physical blocks in the pool
   int limit;           // valid lengths: 0 < L <= min(max_context, max_blocks * bs)
   int num_ctas;
+  // Cascade step (paged_attn_decode_cascade): the first len_off positions of
+  // every sequence (a shared prefix) are attended by the prefix pass, this
+  // call attends positions len_off .. L - 1 through tables that start at
+  // them (lengths below are L - len_off), every unit leaves partials, and
+  // the merge folds in each (sequence, head)'s prefix partial from pre_o
+  // ([num_seqs][q_heads][D], unnormalised) and pre_ml ((max, sum), base 2).
+  int len_off;
+  const float *pre_o;
+  const float *pre_ml;
 };
+
+// Positions of sequence b this call attends.
+__device__ __forceinline__ int seq_len(const AttnParams &p, int b) {
+  return p.context_lens[b] - p.len_off;
+}
 
 template <int KV_T>
 constexpr bool is16() {
@@ -220,7 +234,7 @@ __device__ __forceinline__ void store_out(void *out, int64_t idx, float v) {
 // KV blocks of sequence b; 0 for an empty or invalid length.
 template <int BS>
 __device__ __forceinline__ int seq_blocks(const AttnParams &p, int b) {
-  const int L = p.context_lens[b];
+  const int L = seq_len(p, b);
   return (L > 0 && L <= p.limit) ? (L + BS - 1) / BS : 0;
 }
 
@@ -764,9 +778,34 @@ struct Consumer {
       for (int i = 0; i < 2; ++i)
         f[i] = (m2_run[i] == -INFINITY || !alive) ? 0.f : exp2f(m2_run[i] - m_run[i]);
     }
+    // cascade step (16-bit caches): a whole unit folds in the shared prefix's
+    // partial of each of its heads here (the prefix pass finished before this
+    // kernel passed its dependency wait); fp weights that partial's output
+    float fp[2] = {0.f, 0.f};
+    int64_t prow[2] = {0, 0};
+    const bool pre = !kScaled && whole && p.pre_o != nullptr;  // (O against m_run)
     if (whole) {
 #pragma unroll
-      for (int i = 0; i < 2; ++i) f[i] = l_run[i] > 0.f ? f[i] / l_run[i] : 0.f;
+      for (int i = 0; i < 2; ++i) {
+        if (!pre) {
+          f[i] = l_run[i] > 0.f ? f[i] / l_run[i] : 0.f;
+          continue;
+        }
+        float lp = 0.f, wp = 0.f, ws = 0.f;
+        if (2 * cq + i < nh) {
+          prow[i] = (static_cast<int64_t>(b) * p.q_heads + h0 + 2 * cq + i) * D;
+          const float2 ml = *reinterpret_cast<const float2 *>(p.pre_ml + prow[i] / D * 2);
+          const float M = fmaxf(alive ? m_run[i] : -INFINITY, ml.x);
+          if (M != -INFINITY) {
+            ws = alive ? exp2_rel(m_run[i], M) : 0.f;
+            wp = exp2_rel(ml.x, M);
+            lp = ml.y * wp;
+          }
+        }
+        const float den = l_run[i] * ws + lp;
+        f[i] = den > 0.f ? ws / den : 0.f;
+        fp[i] = den > 0.f ? wp / den : 0.f;
+      }
     }
 #pragma unroll
     for (int dt = 0; dt < D / 16; ++dt) {
@@ -788,8 +827,13 @@ struct Consumer {
           const float v0 = oacc[dt][i] * f[i], v1 = oacc[dt][i + 2] * f[i];
           if (whole) {
             const int64_t o = (static_cast<int64_t>(b) * p.q_heads + h0 + n) * D;
-            store_out<Q_T>(p.out, o + d0, v0);
-            store_out<Q_T>(p.out, o + d1, v1);
+            if (pre) {
+              store_out<Q_T>(p.out, o + d0, v0 + p.pre_o[prow[i] + d0] * fp[i]);
+              store_out<Q_T>(p.out, o + d1, v1 + p.pre_o[prow[i] + d1] * fp[i]);
+            } else {
+              store_out<Q_T>(p.out, o + d0, v0);
+              store_out<Q_T>(p.out, o + d1, v1);
+            }
           } else {
             float *po = p.part_o + (pbase + n) * D;
             po[d0] = v0;
@@ -990,8 +1034,9 @@ attn_partition_kernel(const __grid_constant__ CUtensorMap kmap,
   // Total positions over all units, then this CTA's even share [s0, s1).
   long long part = 0;
   for (int b = threadIdx.x; b < B; b += kThreads) {
-    const int L = p.context_lens[b];
-    if (L < 0 || L > p.limit) {
+    const int L = seq_len(p, b);
+    // (cascade with an append: the new token must lie past the shared prefix)
+    if (L < 0 || L > p.limit || (L == 0 && p.len_off > 0 && p.k_new != nullptr)) {
       if (c == 0) atomicOr(p.status, kErrContext);
     } else {
       part += unit_len((L + BS - 1) / BS, p);
@@ -1124,7 +1169,7 @@ attn_partition_kernel(const __grid_constant__ CUtensorMap kmap,
     const int chunk = cgi * p.cpg + cl;
     const int h0 = g * p.group + chunk * kChunkHeads;
     const int nh = min(kChunkHeads, p.group - chunk * kChunkHeads);
-    const int L = p.context_lens[w.b];
+    const int L = seq_len(p, w.b);
     // fused append: the new token (position L - 1) is in block jl of the unit;
     // with one query-head chunk per kv head this warp alone uses its rows
     const int jl = (L - 1) / BS;
@@ -1213,17 +1258,19 @@ __global__ void __launch_bounds__(kMergeWarps * 32) attn_merge_kernel(const Attn
   const int slot = hi * cpg + cl;
   // length and bookkeeping in one round trip (the bookkeeping is used only
   // for a valid, non-empty length: it is rewritten for such units every call)
-  const int L = p.context_lens[b];
+  const int L = seq_len(p, b);
   const int4 mt = p.meta[static_cast<int64_t>(b) * p.units_per_seq + hgi * p.cgroups + cgi];
   const int64_t orow = static_cast<int64_t>(w) * D + lane * E;
-  if (!(L > 0 && L <= p.limit)) {
+  const bool pre = p.pre_o != nullptr;  // cascade: fold in the prefix partial
+  const bool valid = L > 0 && L <= p.limit;
+  if (!valid && !(pre && L == 0)) {     // (cascade: no position past the prefix)
 #pragma unroll
     for (int e = 0; e < E; ++e) store_out<OUT_T>(p.out, orow + e, 0.f);
     return;
   }
-  const int nu = mt.y;
-  if (nu <= 1) return;  // finished by the partition kernel
-  if (mt.x < 0 || mt.x >= p.num_ctas || nu > p.num_ctas - mt.x || (mt.z & ~1)) {
+  const int nu = valid ? mt.y : 0;
+  if (valid && nu <= 1) return;  // finished by the partition kernel
+  if (valid && (mt.x < 0 || mt.x >= p.num_ctas || nu < 1 || nu > p.num_ctas - mt.x || (mt.z & ~1))) {
     if (lane == 0) atomicOr(p.status, kErrTimeout);  // bookkeeping not written: phase 1 aborted
     return;
   }
@@ -1272,6 +1319,20 @@ __global__ void __launch_bounds__(kMergeWarps * 32) attn_merge_kernel(const Attn
           M = Mn;
         }
       }
+    }
+  }
+  if (pre) {  // the prefix pass's piece, last
+    const float2 ml = *reinterpret_cast<const float2 *>(p.pre_ml + static_cast<int64_t>(w) * 2);
+    float o[E];
+    const float *src = p.pre_o + orow;
+#pragma unroll
+    for (int e = 0; e < E; ++e) o[e] = src[e];
+    const float Mn = fmaxf(M, ml.x);
+    if (Mn != -INFINITY) {
+      const float a = exp2_rel(M, Mn), wt = exp2_rel(ml.x, Mn);
+      Ls = Ls * a + ml.y * wt;
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[e] = acc[e] * a + o[e] * wt;
     }
   }
   const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
@@ -1474,12 +1535,34 @@ kv_status fill_params(kv_pool *pool, int layer, const void *q, int num_seqs, int
   return KV_OK;
 }
 
+// A cascade step's view of the call: the shared prefix's blocks and where the
+// prefix pass leaves its partials.
+struct Cascade {
+  int prefix_blocks;
+  float *pre_o;
+  float *pre_ml;
+};
+
+// Suffix view of a cascade step: tables from the first block past the prefix
+// (same row stride), lengths and limit counted from there.
+void apply_cascade(const kv_pool *pool, const Cascade *cas, int32_t max_blocks_per_seq,
+                   int32_t max_context, AttnParams *p) {
+  if (!cas) return;
+  const int bs = pool->d.block_size;
+  p->len_off = cas->prefix_blocks * bs;
+  if (p->block_tables) p->block_tables += cas->prefix_blocks;
+  const int64_t cap = static_cast<int64_t>(max_blocks_per_seq - cas->prefix_blocks) * bs;
+  p->limit = static_cast<int>(std::min<int64_t>(max_context - p->len_off, cap));
+  p->pre_o = cas->pre_o;
+  p->pre_ml = cas->pre_ml;
+}
+
 kv_status run_partition(kv_pool *pool, int32_t layer, const void *q, int32_t q_dtype,
                         int32_t num_seqs, int32_t num_q_heads, const int32_t *block_tables,
                         int32_t max_blocks_per_seq, const int32_t *context_lens,
                         int32_t max_context, float scale, void *out, int32_t num_ctas,
                         void *workspace, uint64_t workspace_bytes, const void *k_new,
-                        const void *v_new, cudaStream_t st) {
+                        const void *v_new, cudaStream_t st, const Cascade *cas = nullptr) {
   if (!pool) return fail(KV_ERR_INVALID, "null pool");
   if (layer < 0 || layer >= pool->d.num_layers) return fail(KV_ERR_INVALID, "layer %d out of range", layer);
   const int cd = pool->d.cache_dtype;
@@ -1503,6 +1586,7 @@ kv_status run_partition(kv_pool *pool, int32_t layer, const void *q, int32_t q_d
   s = fill_params(pool, layer, q, num_seqs, num_q_heads, block_tables, max_blocks_per_seq,
                   context_lens, max_context, scale, out, G, workspace, workspace_bytes, &p);
   if (s != KV_OK) return s;
+  apply_cascade(pool, cas, max_blocks_per_seq, max_context, &p);
   if (k_new || v_new) {
     if (!k_new || !v_new) return fail(KV_ERR_INVALID, "k_new and v_new go together");
     if ((reinterpret_cast<uintptr_t>(k_new) & 15) || (reinterpret_cast<uintptr_t>(v_new) & 15))
@@ -1530,7 +1614,7 @@ kv_status run_partition(kv_pool *pool, int32_t layer, const void *q, int32_t q_d
 kv_status run_merge(kv_pool *pool, int32_t num_seqs, int32_t num_q_heads,
                     const int32_t *context_lens, int32_t max_blocks_per_seq, int32_t max_context,
                     int32_t num_ctas, int32_t out_dtype, void *out, void *workspace,
-                    uint64_t workspace_bytes, cudaStream_t st) {
+                    uint64_t workspace_bytes, cudaStream_t st, const Cascade *cas = nullptr) {
   if (!pool) return fail(KV_ERR_INVALID, "null pool");
   if (out_dtype != KV_BF16 && out_dtype != KV_FP16)
     return fail(KV_ERR_UNSUPPORTED, "out_dtype must be KV_BF16 or KV_FP16");
@@ -1545,7 +1629,75 @@ kv_status run_merge(kv_pool *pool, int32_t num_seqs, int32_t num_q_heads,
   s = fill_params(pool, -1, nullptr, num_seqs, num_q_heads, nullptr, max_blocks_per_seq,
                   context_lens, max_context, 1.f, out, G, workspace, workspace_bytes, &p);
   if (s != KV_OK) return s;
+  apply_cascade(pool, cas, max_blocks_per_seq, max_context, &p);
   return cuda_check(launch_merge(pool->d.head_dim, out_dtype, p, st), "merge launch");
+}
+
+// Workspace of a cascade step: the decode workspace, then the prefix pass's
+// outputs [num_seqs][Hq][D] and (max, sum) pairs [num_seqs][Hq][2], fp32.
+uint64_t cascade_ws(int B, int Hq, int units_per_seq, int G, int D, uint64_t *o_off,
+                    uint64_t *ml_off) {
+  *o_off = round_up(ws_layout(B, units_per_seq, G, D).total, 256);
+  *ml_off = *o_off + round_up(static_cast<uint64_t>(B) * Hq * D * 4, 256);
+  return *ml_off + round_up(static_cast<uint64_t>(B) * Hq * 2 * 4, 256);
+}
+
+kv_status run_cascade(kv_pool *pool, int32_t layer, const void *q, const void *k_new,
+                      const void *v_new, int32_t q_dtype, int32_t num_seqs, int32_t num_q_heads,
+                      const int32_t *block_tables, int32_t max_blocks_per_seq,
+                      const int32_t *context_lens, int32_t max_context, int32_t prefix_blocks,
+                      float scale, void *out, int32_t num_ctas, void *workspace,
+                      uint64_t workspace_bytes, cudaStream_t st) {
+  if (!pool) return fail(KV_ERR_INVALID, "null pool");
+  if (layer < 0 || layer >= pool->d.num_layers) return fail(KV_ERR_INVALID, "layer %d out of range", layer);
+  if (is_quant(pool->d.cache_dtype))
+    return fail(KV_ERR_UNSUPPORTED, "the cascade step reads 16-bit caches only");
+  if (q_dtype != pool->d.cache_dtype) return fail(KV_ERR_UNSUPPORTED, "q_dtype must be the cache dtype");
+  if (prefix_blocks < 1 || prefix_blocks >= max_blocks_per_seq)
+    return fail(KV_ERR_INVALID, "prefix_blocks must be in [1, max_blocks_per_seq)");
+  if (static_cast<int64_t>(prefix_blocks) * pool->d.block_size > max_context)
+    return fail(KV_ERR_INVALID, "max_context is shorter than the prefix");
+  int G = 0;
+  kv_status s = check_attn(pool, num_seqs, num_q_heads, max_context, num_ctas, &G);
+  if (s != KV_OK) return s;
+  if (num_q_heads / pool->d.num_kv_heads > 128)
+    return fail(KV_ERR_UNSUPPORTED, "at most 128 query heads per kv head");
+  if (num_seqs == 0) return KV_OK;
+  if (!q || !out || !block_tables || !context_lens) return fail(KV_ERR_INVALID, "null pointer");
+  if ((reinterpret_cast<uintptr_t>(q) & 15) || (reinterpret_cast<uintptr_t>(out) & 15) ||
+      (reinterpret_cast<uintptr_t>(block_tables) & 3) || (reinterpret_cast<uintptr_t>(context_lens) & 3))
+    return fail(KV_ERR_INVALID, "q and out must be 16-byte aligned, tables and lengths 4-byte");
+  if (k_new || v_new) {  // checked before any launch
+    if (!k_new || !v_new) return fail(KV_ERR_INVALID, "k_new and v_new go together");
+    if ((reinterpret_cast<uintptr_t>(k_new) & 15) || (reinterpret_cast<uintptr_t>(v_new) & 15))
+      return fail(KV_ERR_INVALID, "k_new and v_new must be 16-byte aligned");
+    if (num_q_heads / pool->d.num_kv_heads > kChunkHeads)
+      return fail(KV_ERR_UNSUPPORTED, "the fused append supports up to 8 query heads per kv head");
+  }
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255))
+    return fail(KV_ERR_INVALID, "workspace must be 256-byte aligned");
+  const UnitGeom u = unit_geom(pool, num_q_heads);
+  uint64_t o_off = 0, ml_off = 0;
+  const uint64_t need = cascade_ws(num_seqs, num_q_heads, u.units_per_seq, G, pool->d.head_dim,
+                                   &o_off, &ml_off);
+  if (!workspace || workspace_bytes < need)
+    return fail(KV_ERR_INVALID, "workspace of %llu bytes needed, %llu given",
+                static_cast<unsigned long long>(need), static_cast<unsigned long long>(workspace_bytes));
+  Cascade cas{prefix_blocks, reinterpret_cast<float *>(static_cast<char *>(workspace) + o_off),
+              reinterpret_cast<float *>(static_cast<char *>(workspace) + ml_off)};
+  // 1. the shared prefix, once for all sequences, on the tensor cores (row 0
+  //    of the tables names the prefix's blocks, as every row does)
+  s = prefix_pass(pool, layer, q, num_seqs, num_q_heads, block_tables, prefix_blocks, scale,
+                  cas.pre_o, cas.pre_ml, st);
+  if (s != KV_OK) return s;
+  // 2. each sequence's positions past the prefix (with the step's append),
+  //    every unit as partials; 3. the merge, prefix partial folded in
+  s = run_partition(pool, layer, q, q_dtype, num_seqs, num_q_heads, block_tables,
+                    max_blocks_per_seq, context_lens, max_context, scale, out, num_ctas,
+                    workspace, workspace_bytes, k_new, v_new, st, &cas);
+  if (s != KV_OK) return s;
+  return run_merge(pool, num_seqs, num_q_heads, context_lens, max_blocks_per_seq, max_context,
+                   num_ctas, q_dtype, out, workspace, workspace_bytes, st, &cas);
 }
 
 }  // namespace
@@ -1564,6 +1716,34 @@ kv_status paged_attn_workspace_bytes(const kv_pool *pool, int32_t num_seqs, int3
   const UnitGeom u = unit_geom(pool, num_q_heads);
   *bytes = ws_layout(num_seqs, u.units_per_seq, G, pool->d.head_dim).total;
   return ok();
+}
+
+kv_status paged_attn_cascade_workspace_bytes(const kv_pool *pool, int32_t num_seqs,
+                                             int32_t num_q_heads, int32_t num_ctas,
+                                             uint64_t *bytes) {
+  if (!bytes) return fail(KV_ERR_INVALID, "null bytes");
+  int G = 0;
+  kv_status s = check_attn(pool, num_seqs, num_q_heads, 0, num_ctas, &G);
+  if (s != KV_OK) return s;
+  const UnitGeom u = unit_geom(pool, num_q_heads);
+  uint64_t o_off = 0, ml_off = 0;
+  *bytes = cascade_ws(num_seqs, num_q_heads, u.units_per_seq, G, pool->d.head_dim, &o_off, &ml_off);
+  return ok();
+}
+
+kv_status paged_attn_decode_cascade(kv_pool *pool, int32_t layer, const void *q,
+                                    const void *k_new, const void *v_new, int32_t q_dtype,
+                                    int32_t num_seqs, int32_t num_q_heads,
+                                    const int32_t *block_tables, int32_t max_blocks_per_seq,
+                                    const int32_t *context_lens, int32_t max_context,
+                                    int32_t prefix_blocks, float scale, void *out,
+                                    int32_t num_ctas, void *workspace, uint64_t workspace_bytes,
+                                    kv_stream_t stream) {
+  kv_status s = run_cascade(pool, layer, q, k_new, v_new, q_dtype, num_seqs, num_q_heads,
+                            block_tables, max_blocks_per_seq, context_lens, max_context,
+                            prefix_blocks, scale, out, num_ctas, workspace, workspace_bytes,
+                            (cudaStream_t)stream);
+  return s == KV_OK ? ok() : s;
 }
 
 kv_status paged_attn_default_ctas(const kv_pool *pool, int32_t *num_ctas) {

@@ -110,6 +110,14 @@ struct PrefillParams {
   uint32_t q_keep, q_sign;
   int num_seqs, q_heads, kv_heads, group, tile_tokens, total_q;
   int max_blocks, num_blocks, limit;
+  // Shared-prefix pass of a cascade decode step (prefix_len > 0): the
+  // total_q "new tokens" are total_q sequences' decode queries, every one
+  // attending all prefix_len positions of the one block-table row (no causal
+  // limit); each row's unnormalised output goes to pre_o ([total_q][Hq][D]
+  // fp32) and its (maximum, sum), base 2, to pre_ml, in place of out.
+  int prefix_len;
+  float *pre_o;
+  float *pre_ml;
 };
 
 __device__ __forceinline__ float ex2f(float x) {
@@ -209,16 +217,17 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
   const int t0 = blockIdx.x * p.tile_tokens;
 
   grid_dependency_wait();
-  const int q0 = p.cu_q[b];
-  const int cb = p.cu_q[b + 1] - q0;
-  const int L = p.context_lens[b];
+  const bool pre = p.prefix_len > 0;  // shared-prefix pass: no causal limit
+  const int q0 = pre ? 0 : p.cu_q[b];
+  const int cb = pre ? p.total_q : p.cu_q[b + 1] - q0;
+  const int L = pre ? p.prefix_len : p.context_lens[b];
   if (t0 >= cb) return;  // also when cb <= 0: same for the whole CTA
-  if (cb > L || L > p.limit || q0 < 0 || q0 + cb > p.total_q) {
+  if ((!pre && cb > L) || L > p.limit || q0 < 0 || q0 + cb > p.total_q) {
     if (threadIdx.x == 0 && blockIdx.x == 0 && g == 0) atomicOr(p.status, kErrContext);
     return;
   }
   const int t_last = min(t0 + p.tile_tokens, cb) - 1;  // last token of the tile
-  const int nkeys = L - cb + t_last + 1;               // positions the tile reads
+  const int nkeys = pre ? L : L - cb + t_last + 1;     // positions the tile reads
   const int nstages = (nkeys + kPfKeys - 1) / kPfKeys;
   const int nunits = (nstages + 1) / 2;
 
@@ -252,7 +261,7 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
   if (warp < kPfProducerWarp) {
     const int tl = row / p.group, hl = row - tl * p.group;
     rvalid = tl < p.tile_tokens && t0 + tl < cb;
-    if (rvalid) rpos = L - cb + t0 + tl;
+    if (rvalid) rpos = pre ? L - 1 : L - cb + t0 + tl;
     rq = (static_cast<int64_t>(q0 + t0 + tl) * p.q_heads + g * p.group + hl) * D;
     // Q row -> TMEM as packed 16-bit pairs (zeros past the tile): the first
     // D / 2 / kQGCols groups write kQGCols columns (2 kQGCols dims) each
@@ -595,12 +604,22 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
     if (!__any_sync(kFull, s_abort != 0)) {  // warp-uniform: TMEM loads are warp-wide
       tc_fence_after();
       const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
+      if (pre && rvalid && cg == 0) {
+        p.pre_ml[rq / D * 2] = m_used;
+        p.pre_ml[rq / D * 2 + 1] = l_tot;
+      }
 #pragma unroll
       for (int oc = 0; oc < kOCols; oc += kOChunk) {
         uint32_t o[kOChunk];
         tmem_ld<kOChunk>(trow + kOCol + cg * kOCols + oc, o);
         tmem_wait_ld();
-        if (rvalid) {
+        if (pre && rvalid) {  // the partial, against m_used: O and l as they stand
+          float4 *dst = reinterpret_cast<float4 *>(p.pre_o + rq + cg * kOCols + oc);
+#pragma unroll
+          for (int c4 = 0; c4 < kOChunk / 4; ++c4)
+            dst[c4] = make_float4(__uint_as_float(o[4 * c4]), __uint_as_float(o[4 * c4 + 1]),
+                                  __uint_as_float(o[4 * c4 + 2]), __uint_as_float(o[4 * c4 + 3]));
+        } else if (rvalid) {
           uint4 *dst =
               reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.out) + rq + cg * kOCols + oc);
 #pragma unroll
@@ -653,6 +672,41 @@ PrefillFn pick_prefill_bs(int bs, int dt) {
 }
 
 }  // namespace
+
+kv_status prefix_pass(kv_pool *pool, int layer, const void *q, int num_seqs, int num_q_heads,
+                      const int32_t *prefix_table, int prefix_blocks, float scale, float *pre_o,
+                      float *pre_ml, cudaStream_t st) {
+  const int hkv = pool->d.num_kv_heads, G = num_q_heads / hkv;
+  if (G > kPfRows) return fail(KV_ERR_UNSUPPORTED, "at most %d query heads per kv head", kPfRows);
+  PrefillParams p{};
+  p.q = q;
+  p.block_tables = prefix_table;
+  p.status = status_word(pool);
+  p.scale_log2 = scale == 0.f ? 1.f : std::fabs(scale) * 1.4426950408889634f;
+  p.q_keep = scale == 0.f ? 0u : 0xFFFFFFFFu;
+  p.q_sign = scale < 0.f ? 0x80008000u : 0u;
+  p.num_seqs = 1;  // the one block-table row of the prefix
+  p.q_heads = num_q_heads;
+  p.kv_heads = hkv;
+  p.group = G;
+  p.tile_tokens = kPfRows / G;
+  p.total_q = num_seqs;
+  p.max_blocks = prefix_blocks;
+  p.num_blocks = pool->d.num_blocks;
+  p.prefix_len = prefix_blocks * pool->d.block_size;
+  p.limit = p.prefix_len;
+  p.pre_o = pre_o;
+  p.pre_ml = pre_ml;
+  const int tiles = (num_seqs + p.tile_tokens - 1) / p.tile_tokens;
+  kv_status code;
+  LayerMaps maps;
+  if (!layer_maps(pool, layer, pool->d.block_size, &maps, &code)) return code;
+  const int D = pool->d.head_dim, bs = pool->d.block_size;
+  PrefillFn fn = D == 128 ? pick_prefill_bs<128>(bs, pool->d.cache_dtype)
+                          : pick_prefill_bs<64>(bs, pool->d.cache_dtype);
+  return cuda_check(fn(maps, p, tiles, st), "cascade prefix launch");
+}
+
 }  // namespace pagedkv
 
 using namespace pagedkv;
@@ -687,7 +741,7 @@ extern "C" kv_status paged_attn_prefill(kv_pool *pool, int32_t layer, const void
       (reinterpret_cast<uintptr_t>(context_lens) & 3) || (reinterpret_cast<uintptr_t>(cu_q_lens) & 3))
     return fail(KV_ERR_INVALID, "q and out must be 16-byte aligned, index arrays 4-byte");
   if (num_seqs > 65535) return fail(KV_ERR_UNSUPPORTED, "at most 65535 sequences per call");
-  PrefillParams p;
+  PrefillParams p{};
   p.q = q;
   p.out = out;
   p.cu_q = cu_q_lens;

@@ -140,4 +140,14 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
 // message on failure.
 bool layer_maps(kv_pool *p, int layer, int box_rows, LayerMaps *out, kv_status *code);
 
+// Shared-prefix pass of a cascade decode step (attn_prefill.cu): the decode
+// query of each of num_seqs sequences (q [num_seqs][Hq][D], the cache dtype)
+// attends the prefix_blocks blocks of prefix_table, all positions, no causal
+// limit; writes each (sequence, head)'s unnormalised output to pre_o
+// ([num_seqs][Hq][D] fp32) and its (maximum, sum), base 2, to pre_ml. The
+// caller has checked the cache dtype, the head counts and the pointers.
+kv_status prefix_pass(kv_pool *pool, int layer, const void *q, int num_seqs, int num_q_heads,
+                      const int32_t *prefix_table, int prefix_blocks, float scale, float *pre_o,
+                      float *pre_ml, cudaStream_t st);
+
 }  // namespace pagedkv

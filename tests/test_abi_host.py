@@ -327,3 +327,46 @@ def test_prefill_argument_validation():
     finally:
         B.lib.kv_pool_destroy(h)
         B.lib.kv_pool_destroy(hq)
+
+
+def test_cascade_argument_validation_and_workspace_size():
+    """paged_attn_decode_cascade checks its arguments before any launch (the
+    prefix pass included); its workspace is the decode workspace plus the
+    prefix partials; on a host without a GPU a well-formed call fails loudly."""
+    import torch
+    h, _ = _make_pool(64, 1, 16, 2, 64, "bf16")
+    hq, _ = _make_pool(64, 1, 16, 2, 64, "int8")
+    try:
+        r256 = lambda x: -(-x // 256) * 256
+        n, nd = ctypes.c_uint64(), ctypes.c_uint64()
+        B.check(B.lib.paged_attn_cascade_workspace_bytes(h, 4, 8, 10, ctypes.byref(n)))
+        B.check(B.lib.paged_attn_workspace_bytes(h, 4, 8, 10, ctypes.byref(nd)))
+        assert n.value == r256(nd.value) + r256(4 * 8 * 64 * 4) + r256(4 * 8 * 2 * 4)
+        fake = ctypes.c_void_p(FAKE_BASE)
+        nul = ctypes.c_void_p(0)
+
+        def call(pool=h, layer=0, q=fake, kn=None, vn=None, qdt=0, B_=4, Hq=8, mb=16, mc=250,
+                 pb=4, scale=0.125, out=fake, ctas=10, ws=fake, wsb=1 << 22):
+            return B.lib.paged_attn_decode_cascade(pool, layer, q, kn, vn, qdt, B_, Hq, fake, mb,
+                                                   fake, mc, pb, scale, out, ctas, ws, wsb, None)
+
+        assert call(layer=1) == B.KV_ERR_INVALID
+        assert call(pool=hq) == B.KV_ERR_UNSUPPORTED                 # 16-bit caches only
+        assert call(qdt=1) == B.KV_ERR_UNSUPPORTED                   # q dtype != cache dtype
+        assert call(pb=0) == B.KV_ERR_INVALID                        # no prefix
+        assert call(pb=16) == B.KV_ERR_INVALID                       # no block past the prefix
+        assert call(mc=63) == B.KV_ERR_INVALID                       # prefix longer than max
+        assert call(Hq=7) == B.KV_ERR_INVALID
+        assert call(Hq=2 * 129) == B.KV_ERR_UNSUPPORTED              # > 128 heads per kv head
+        assert call(kn=fake) == B.KV_ERR_INVALID                     # k_new without v_new
+        assert call(kn=fake, vn=fake, Hq=32) == B.KV_ERR_UNSUPPORTED  # append: <= 8 per kv head
+        assert call(wsb=16) == B.KV_ERR_INVALID                      # workspace too small
+        assert call(ws=ctypes.c_void_p(FAKE_BASE + 128)) == B.KV_ERR_INVALID   # misaligned
+        assert call(q=nul) == B.KV_ERR_INVALID
+        assert call(B_=0) == B.KV_OK                                 # nothing to do
+        if not torch.cuda.is_available():
+            assert call() == B.KV_ERR_CUDA
+            assert call(kn=fake, vn=fake) == B.KV_ERR_CUDA
+    finally:
+        B.lib.kv_pool_destroy(h)
+        B.lib.kv_pool_destroy(hq)

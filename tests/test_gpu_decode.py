@@ -210,6 +210,16 @@ def test_shared_prefix_copy_on_write(pkv):
             lambda bh: attention.decode_one(q, kc, vc, o_tbl, lens, wl.scale, *bh), pairs)))
     got = torch.stack([out[b, h] for b, h in pairs])
     compare(got, ref, what="shared_prefix")
+    # the cascade step on the same pool: the 93 blocks every request still
+    # shares once for all requests on the tensor cores, the rest per request
+    t_dev = torch.from_numpy(tbl).to(DEV)
+    l_dev = torch.from_numpy(lens.astype(np.int32)).to(DEV)
+    assert all(t[:nprefix - 1] == tables[0][:nprefix - 1] for t in tables)
+    out_c = pkv.paged_attn_decode_cascade(pool, 0, wl.q, t_dev, l_dev, int(lens.max()),
+                                          nprefix - 1, wl.scale)
+    torch.cuda.synchronize()
+    assert pool.status() == 0
+    compare(torch.stack([out_c[b, h] for b, h in pairs]), ref, what="shared_prefix cascade")
 
 
 # --------------------------------------------------------------- edge cases
@@ -439,3 +449,97 @@ def test_decode_graph_replays_match(pkv):
         assert np.array_equal(bits16(out), bits16(ref))
     del graph
     assert pool.status() == 0
+
+
+# ------------------------------------------------ cascade (shared prefix) step
+
+def _cascade_case(seed):
+    """Sequences whose tables start with the same pb blocks: seeded shapes over
+    dtype, head_dim, block size, heads, batch, prefix and suffix lengths (some
+    suffixes empty when there is no append)."""
+    rng = np.random.default_rng(1000 + seed)
+    dtype = ("bf16", "fp16")[seed % 2]
+    D = (64, 128)[(seed // 2) % 2]
+    bs = (16, 32)[(seed // 4) % 2]
+    hkv = int(rng.choice([1, 2, 4, 8]))
+    append = seed % 3 != 2
+    G = (1, 2, 4, 8)[seed % 4] if append else (16, 64, 8, 1)[(seed // 3) % 4]
+    B = int(rng.integers(1, 48))
+    pb = int(rng.integers(1, 9))
+    suffix = rng.integers(1 if append else 0, 5 * bs, size=B)
+    if not append:
+        suffix[0] = 0                       # the prefix alone
+    lens = pb * bs + suffix
+    nblk = -(-lens // bs)
+    N = pb + int((nblk - pb).sum()) + 8
+    perm = rng.permutation(N).astype(np.int32)
+    mb = int(nblk.max()) + 1
+    tables = np.full((B, mb), -1, np.int32)
+    pos = pb
+    for b in range(B):
+        tables[b, :pb] = perm[:pb]
+        k = int(nblk[b]) - pb
+        tables[b, pb:pb + k] = perm[pos:pos + k]
+        pos += k
+    wl = W.make_decode_workload("cascade%d" % seed, B, G * hkv, hkv, D, bs, dtype, dtype, lens,
+                                num_blocks=N, seed=seed, device=DEV, placement=tables)
+    return wl, pb, append
+
+
+@pytest.mark.parametrize("seed", range(10))
+def test_cascade_matches_oracle(pkv, seed):
+    """paged_attn_decode_cascade: every output against the oracle's decode over
+    the whole tables (prefix included); with an append, the new rows are in the
+    pool bit for bit."""
+    wl, pb, append = _cascade_case(seed)
+    pool = build_pool(pkv, wl, DEV)
+    tables, lens = device_inputs(wl, DEV)
+    kw = dict(k_new=wl.k_new, v_new=wl.v_new) if append else {}
+    out = pkv.paged_attn_decode_cascade(pool, 0, wl.q, tables, lens, int(wl.context_lens.max()),
+                                        pb, wl.scale, **kw)
+    torch.cuda.synchronize()
+    assert pool.status() == 0
+    if append:
+        k, v = oracle_cache_16(wl)
+    else:
+        dt = np.float16 if wl.cache_dtype == "fp16" else np.float32
+        k, v = to_np(wl.k_fill, dt), to_np(wl.v_fill, dt)
+    pairs = _all_pairs(wl)
+    ref = oracle_outputs(wl, k, v, pairs)
+    compare(torch.stack([out[b, h] for b, h in pairs]), ref, what=wl.name)
+    if append:
+        K, V, _, _ = pool.layer_views(0)
+        bs = wl.block_size
+        for b in range(wl.batch):
+            s_ = int(wl.slot_new[b])
+            assert np.array_equal(bits16(K[s_ // bs, :, s_ % bs]), bits16(wl.k_new[b]))
+            assert np.array_equal(bits16(V[s_ // bs, :, s_ % bs]), bits16(wl.v_new[b]))
+
+
+def test_cascade_reports_lengths_inside_the_prefix(pkv):
+    """A length shorter than the prefix, or (with an append) equal to it, is
+    reported on the device; the other sequences' outputs stay exact."""
+    wl, pb, _ = _cascade_case(0)
+    assert wl.batch >= 3
+    bs = wl.block_size
+    pool = build_pool(pkv, wl, DEV)
+    pool.status_clear()
+    tables, lens = device_inputs(wl, DEV)
+    bad = lens.clone()
+    bad[1] = pb * bs - 1
+    out = pkv.paged_attn_decode_cascade(pool, 0, wl.q, tables, bad, int(wl.context_lens.max()),
+                                        pb, wl.scale)
+    torch.cuda.synchronize()
+    assert pool.status() & 2                 # KV_DEVERR_CONTEXT
+    assert torch.count_nonzero(out[1]) == 0
+    dt = np.float16 if wl.cache_dtype == "fp16" else np.float32
+    k, v = to_np(wl.k_fill, dt), to_np(wl.v_fill, dt)
+    pairs = [(b, h) for b in (0, 2) for h in range(wl.q_heads)]
+    compare(torch.stack([out[b, h] for b, h in pairs]), oracle_outputs(wl, k, v, pairs))
+    pool.status_clear()
+    bad = lens.clone()
+    bad[2] = pb * bs                      # the new token would land in the shared blocks
+    pkv.paged_attn_decode_cascade(pool, 0, wl.q, tables, bad, int(wl.context_lens.max()), pb,
+                                  wl.scale, k_new=wl.k_new, v_new=wl.v_new)
+    torch.cuda.synchronize()
+    assert pool.status() & 2                 # KV_DEVERR_CONTEXT
