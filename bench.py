@@ -73,6 +73,11 @@ WORKLOADS = {
                       "copied on write per request), suffixes U[1,512], 64/8 heads, D 128, bf16, "
                       "block 16; GB/s counts logical bytes (the shared prefix is read from L2)",
                       lambda dev: SharedPrefixStep(dev)),
+    "shared_prefix_cascade": ("Shared prompt as above through the cascade step: the 93 blocks all "
+                              "200 requests still share once for all of them on the tensor cores, "
+                              "each request's remaining positions through the decode kernel, then "
+                              "the merge; GB/s counts the same logical bytes",
+                              lambda dev: SharedPrefixStep(dev, cascade=True)),
 }
 
 
@@ -119,6 +124,16 @@ def step_bytes(wl):
         (rows * 2 * 4 if wl.cache_dtype in ("int8", "e5m2", "int4") else
          rows * 4 if wl.cache_dtype == "int8_kchan" else 0)                  # write rows
     return int(kv + q_out), int(append)
+
+
+def cascade_hbm_bytes(wl):
+    """Bytes a cascade step must read or write in HBM: the shared blocks' K/V
+    once, the K/V of every position past them, q, out and the new rows."""
+    bs, row = wl.block_size, wl.kv_heads * wl.head_dim * 2 * 2      # K + V of one position
+    shared = wl.cascade_blocks * bs
+    later = int((wl.context_lens - shared).sum())
+    q_out = 2 * wl.batch * wl.q_heads * wl.head_dim * 2
+    return (shared + later) * row + q_out + step_bytes(wl)[1]
 
 
 # ------------------------------------------------------------------ clocks
@@ -381,8 +396,10 @@ class SharedPrefixStep:
     copies the partial one on write, and appends its suffix except the last
     token, which is the step's append."""
 
-    def __init__(self, device):
+    def __init__(self, device, cascade=False):
         self.sp = sp = W.shared_prefix(device)
+        # cascade step: the prompt's full blocks, shared by every request
+        self.cascade_blocks = sp.prefix_len // sp.block_size if cascade else 0
         self.batch, self.q_heads, self.kv_heads = sp.batch, sp.q_heads, sp.kv_heads
         self.head_dim, self.block_size, self.cache_dtype = sp.head_dim, sp.block_size, "bf16"
         self.group = sp.q_heads // sp.kv_heads
@@ -638,7 +655,9 @@ def run_ours(args, rank, world, device):
     slot_new = torch.from_numpy(wl.slot_new).to(device)
     max_ctx = int(wl.context_lens.max())
     G = args.ctas or pkv.default_ctas(pool)
-    ws = pkv.make_workspace(pool, wl.batch, wl.q_heads, G)
+    casc = getattr(wl, "cascade_blocks", 0)
+    ws = (pkv.make_cascade_workspace if casc else pkv.make_workspace)(pool, wl.batch,
+                                                                       wl.q_heads, G)
     out = torch.empty_like(wl.q)
     flush = torch.ones(64 << 20, dtype=torch.float32, device=device)   # 256 MiB
     flush_sink = torch.empty((), dtype=torch.float32, device=device)
@@ -650,7 +669,11 @@ def run_ours(args, rank, world, device):
     fused = not args.separate_append and wl.group <= 8
 
     def one_step():
-        if fused:   # append folded into the attention kernel, then the merge
+        if casc:    # shared prefix once for all requests, then per request, then the merge
+            pkv.paged_attn_decode_cascade(pool, 0, wl.q, tables, lens, max_ctx, casc, wl.scale,
+                                          k_new=wl.k_new, v_new=wl.v_new, out=out, num_ctas=G,
+                                          workspace=ws)
+        elif fused:   # append folded into the attention kernel, then the merge
             pkv.paged_attn_decode_append(pool, 0, wl.q, wl.k_new, wl.v_new, tables, lens,
                                          max_ctx, wl.scale, out=out, num_ctas=G, workspace=ws)
         else:
@@ -690,7 +713,7 @@ def run_ours(args, rank, world, device):
     kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
     hold_gpu(1e-3 + 150e-6 * args.steps)
-    for i in range(args.steps):
+    for i in range(args.steps if not casc else 0):   # (cascade: the step is the figure)
         flush_l2()
         kev[i][0].record(stream)
         if fused:
@@ -706,7 +729,8 @@ def run_ours(args, rank, world, device):
     status = pool.status()
     step_ms = np.array([a.elapsed_time(b) for a, b in evs])
     step_s = float(step_ms.mean()) / 1e3
-    part_s = float(np.mean([a.elapsed_time(b) for a, b in kev])) / 1e3
+    part_s = float(np.mean([a.elapsed_time(b) for a, b in kev])) / 1e3 if not casc else \
+        float(step_ms.mean()) / 1e3
     step_s, part_s = max_over_ranks([step_s, part_s], world, device)
     clocks = sampler.summary(t0, t2)
 
@@ -742,7 +766,11 @@ def run_ours(args, rank, world, device):
             a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
             d_in.copy_(h_in, non_blocking=True)
-            if fused:
+            if casc:
+                pkv.paged_attn_decode_cascade(pool, 0, d_q, d_tab, d_len, max_ctx, casc, wl.scale,
+                                              k_new=d_kn, v_new=d_vn, out=d_out, num_ctas=G,
+                                              workspace=ws)
+            elif fused:
                 pkv.paged_attn_decode_append(pool, 0, d_q, d_kn, d_vn, d_tab, d_len, max_ctx,
                                              wl.scale, out=d_out, num_ctas=G, workspace=ws)
             else:
@@ -761,7 +789,8 @@ def run_ours(args, rank, world, device):
     dec_bytes, app_bytes = step_bytes(wl)
     res = {"wl": wl, "desc": desc, "G": G, "step_s": step_s, "part_s": part_s, "out": out_timed,
            "dec_bytes": dec_bytes, "app_bytes": app_bytes, "clocks": clocks, "fused": fused,
-           "status": status, "e2e": e2e, "launches": args.steps * (2 if fused else 3),
+           "status": status, "e2e": e2e,
+           "launches": args.steps * (2 if fused and not casc else 3), "cascade": casc,
            "wall": t1 - t0, "step_ms_median": float(np.median(step_ms))}
     return res
 
@@ -1031,6 +1060,13 @@ def main():
         bound_note = ("achieved = ncu DRAM bytes per launch / kernel time (the shared prompt is "
                       "served from L2)" if traffic else
                       "no DRAM capture of the current kernel source: HBM fraction not reported")
+    elif r.get("cascade"):
+        # the step's three kernels as one: the bytes HBM must deliver are the
+        # shared blocks' K/V once, every position past them, q, out and the new
+        # rows; the timed figure is the whole step
+        achieved = cascade_hbm_bytes(wl) / r["step_s"] / 1e9
+        bound_note = ("whole step (prefix pass, attention, merge): achieved = the shared blocks' "
+                      "K/V once + every later position's K/V + q + out + new rows, / step time")
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         g_cpu, secs, nseq, threads, oouts = oracle_sample(wl, args.cpu_budget)
@@ -1058,7 +1094,7 @@ def main():
                              "reading 256 MiB" % (r["dec_bytes"] / 126e6),
                        "bytes_per_step": r["dec_bytes"] + r["app_bytes"]},
             # the shared prompt's value counts logical bytes (read from L2): no HBM percentage
-            "pct_of_8tbs": None if args.workload == "shared_prefix"
+            "pct_of_8tbs": None if args.workload.startswith("shared_prefix")
             else round(100 * gbs / world / NOMINAL_HBM_GBS, 2),
             "decode_tokens_per_s": round(wl.batch * world / r["step_s"], 1),
             "roofline": {"bound": "hbm",
@@ -1066,8 +1102,10 @@ def main():
                          "peak": peak, "unit": "GB/s",
                          "frac": None if achieved is None else round(achieved / peak, 4),
                          "traffic": traffic, "note": bound_note,
-                         "kernel": "attn_partition_kernel" + (" (append fused)" if r.get("fused")
-                                                              else ""),
+                         "kernel": "cascade step: attn_prefill_kernel (prefix pass) + "
+                                   "attn_partition_kernel + attn_merge_kernel" if r.get("cascade")
+                         else "attn_partition_kernel" + (" (append fused)" if r.get("fused")
+                                                         else ""),
                          "peak_source": peak_kind + " (MEASURED_PEAKS.json hbm_gbs)"
                          if peak_kind == "measured" else "fallback 6650 GB/s",
                          "kernel_ms": round(r["part_s"] * 1e3, 5)},

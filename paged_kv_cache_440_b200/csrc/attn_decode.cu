@@ -763,6 +763,7 @@ struct Consumer {
   // End of the unit's piece in this CTA: write the normalised output of heads
   // h0 .. h0 + nh - 1 (whole unit) or the unnormalised partial (m, l, O) to
   // record `pbase` + head of the workspace.
+  template <bool CASC>
   __device__ __forceinline__ void finish(const AttnParams &p, bool whole, int b, int h0, int nh,
                                          int64_t pbase, bool alive, int lane) {
     const int gq = lane >> 2, cq = lane & 3;
@@ -783,7 +784,7 @@ struct Consumer {
     // kernel passed its dependency wait); fp weights that partial's output
     float fp[2] = {0.f, 0.f};
     int64_t prow[2] = {0, 0};
-    const bool pre = !kScaled && whole && p.pre_o != nullptr;  // (O against m_run)
+    const bool pre = CASC && !kScaled && whole;  // (cascade kernels: O against m_run)
     if (whole) {
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
@@ -807,6 +808,20 @@ struct Consumer {
         fp[i] = den > 0.f ? wp / den : 0.f;
       }
     }
+    // the prefix partial's values this lane adds, all loaded before the first
+    // output store (the stores could alias them, so later loads would wait)
+    float pv[D / 16][2][2];
+    if (pre) {
+#pragma unroll
+      for (int dt = 0; dt < D / 16; ++dt)
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int d0 = dt * 16 + gq;  // 16-bit caches: rows gq / gq + 8
+          const bool hv = 2 * cq + i < nh;
+          pv[dt][i][0] = hv ? p.pre_o[prow[i] + d0] * fp[i] : 0.f;
+          pv[dt][i][1] = hv ? p.pre_o[prow[i] + d0 + 8] * fp[i] : 0.f;
+        }
+    }
 #pragma unroll
     for (int dt = 0; dt < D / 16; ++dt) {
       int d0, d1;
@@ -828,8 +843,8 @@ struct Consumer {
           if (whole) {
             const int64_t o = (static_cast<int64_t>(b) * p.q_heads + h0 + n) * D;
             if (pre) {
-              store_out<Q_T>(p.out, o + d0, v0 + p.pre_o[prow[i] + d0] * fp[i]);
-              store_out<Q_T>(p.out, o + d1, v1 + p.pre_o[prow[i] + d1] * fp[i]);
+              store_out<Q_T>(p.out, o + d0, v0 + pv[dt][i][0]);
+              store_out<Q_T>(p.out, o + d1, v1 + pv[dt][i][1]);
             } else {
               store_out<Q_T>(p.out, o + d0, v0);
               store_out<Q_T>(p.out, o + d1, v1);
@@ -999,8 +1014,11 @@ __device__ __forceinline__ void walk_advance(Walk &w, int seg, const AttnParams 
 
 // ============================================================================
 // Partition kernel: persistent, one producer warp + kNC consumer warps.
+// CASC: the attention pass of a cascade step (whole units fold in the shared
+// prefix's partials); a separate instantiation, so the plain kernels carry no
+// trace of it.
 // ============================================================================
-template <int D, int BS, int KV_T, int Q_T>
+template <int D, int BS, int KV_T, int Q_T, bool CASC>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_partition_kernel(const __grid_constant__ CUtensorMap kmap,
                       const __grid_constant__ CUtensorMap vmap, const AttnParams p) {
@@ -1218,7 +1236,7 @@ attn_partition_kernel(const __grid_constant__ CUtensorMap kmap,
     const bool whole = (w.j == 0 && seg == w.nb);
     if (active) {
       const int64_t pbase = ((static_cast<int64_t>(c) * 2 + side) * kNC + warp) * kChunkHeads;
-      cs.finish(p, whole, w.b, h0, nh, pbase, alive, lane);
+      cs.template finish<CASC>(p, whole, w.b, h0, nh, pbase, alive, lane);
     }
     if (warp == 0 && lane == 0 && w.j == 0) {  // this CTA holds the unit's first block
       const int nu = cta_of(w.pos + w.nb - 1, total, G) - c + 1;
@@ -1346,11 +1364,11 @@ __global__ void __launch_bounds__(kMergeWarps * 32) attn_merge_kernel(const Attn
 using PartFn = cudaError_t (*)(const CUtensorMap &, const CUtensorMap &, const AttnParams &,
                                cudaStream_t);
 
-template <int D, int BS, int KV_T, int Q_T>
+template <int D, int BS, int KV_T, int Q_T, bool CASC = false>
 cudaError_t launch_part(const CUtensorMap &km, const CUtensorMap &vm, const AttnParams &p,
                         cudaStream_t st) {
   const int smem = p.stages * p.stage_bytes + 1024;
-  auto kern = attn_partition_kernel<D, BS, KV_T, Q_T>;
+  auto kern = attn_partition_kernel<D, BS, KV_T, Q_T, CASC>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   e = launch_pdl(kern, dim3(p.num_ctas), dim3(kThreads), smem, st, km, vm, p);
@@ -1385,6 +1403,18 @@ PartFn pick_dtype(int kv, int q) {
 PartFn pick_partition(int D, int BS, int kv, int q) {
   if (D == 128) return BS == 16 ? pick_dtype<128, 16>(kv, q) : pick_dtype<128, 32>(kv, q);
   return BS == 16 ? pick_dtype<64, 16>(kv, q) : pick_dtype<64, 32>(kv, q);
+}
+
+// The cascade step's attention pass: 16-bit caches only.
+template <int D, int BS>
+PartFn pick_cascade_dtype(int kv) {
+  return kv == KV_BF16 ? launch_part<D, BS, KV_BF16, KV_BF16, true>
+                       : launch_part<D, BS, KV_FP16, KV_FP16, true>;
+}
+PartFn pick_cascade(int D, int BS, int kv) {
+  if (kv != KV_BF16 && kv != KV_FP16) return nullptr;
+  if (D == 128) return BS == 16 ? pick_cascade_dtype<128, 16>(kv) : pick_cascade_dtype<128, 32>(kv);
+  return BS == 16 ? pick_cascade_dtype<64, 16>(kv) : pick_cascade_dtype<64, 32>(kv);
 }
 
 // Dynamic shared memory a merge CTA reserves without using it: it caps how
@@ -1606,7 +1636,8 @@ kv_status run_partition(kv_pool *pool, int32_t layer, const void *q, int32_t q_d
   kv_status code;
   LayerMaps maps;
   if (!layer_maps(pool, layer, p.hg * pool->d.block_size, &maps, &code)) return code;
-  PartFn fn = pick_partition(pool->d.head_dim, pool->d.block_size, cd, q_dtype);
+  PartFn fn = cas ? pick_cascade(pool->d.head_dim, pool->d.block_size, cd)
+                  : pick_partition(pool->d.head_dim, pool->d.block_size, cd, q_dtype);
   if (!fn) return fail(KV_ERR_UNSUPPORTED, "no attention kernel for this cache shape");
   return cuda_check(fn(maps.k, maps.v, p, st), "paged attention launch");
 }
