@@ -150,7 +150,9 @@ __device__ __forceinline__ bool ring_wait_pf(uint64_t *bar, uint32_t parity, vol
 // through the 3-D map as [block][slab][row][128 B]; otherwise one box per
 // block and slab, K landing as [slab][slot * 64 + key][128 B] across the ring
 // and V per stage as [slab][key][128 B].
-template <int D, int BS, int KV_T, bool VBLK>
+// PRE: the shared-prefix pass of a cascade decode step (prefix_len, pre_o,
+// pre_ml), a separate instantiation so the prefill kernels carry no trace of it.
+template <int D, int BS, int KV_T, bool VBLK, bool PRE>
 __global__ void __launch_bounds__(kPfThreads, 1)
 attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
                     const __grid_constant__ CUtensorMap vmap, const PrefillParams p) {
@@ -217,7 +219,7 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
   const int t0 = blockIdx.x * p.tile_tokens;
 
   grid_dependency_wait();
-  const bool pre = p.prefix_len > 0;  // shared-prefix pass: no causal limit
+  constexpr bool pre = PRE;  // shared-prefix pass: no causal limit
   const int q0 = pre ? 0 : p.cu_q[b];
   const int cb = pre ? p.total_q : p.cu_q[b + 1] - q0;
   const int L = pre ? p.prefix_len : p.context_lens[b];
@@ -641,11 +643,11 @@ attn_prefill_kernel(const __grid_constant__ CUtensorMap kmap,
   if (warp == kPfMmaWarp) tmem_dealloc(tm, kTmemCols);
 }
 
-template <int D, int BS, int KV_T, bool VBLK>
+template <int D, int BS, int KV_T, bool VBLK, bool PRE>
 cudaError_t launch_prefill_v(const CUtensorMap &km, const CUtensorMap &vm, const PrefillParams &p,
                              int tiles, cudaStream_t st) {
   constexpr int smem = pf_stages(D) * 2 * kPfKeys * D * 2 + 1024;
-  auto kern = attn_prefill_kernel<D, BS, KV_T, VBLK>;
+  auto kern = attn_prefill_kernel<D, BS, KV_T, VBLK, PRE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   e = launch_pdl(kern, dim3(tiles, p.kv_heads, p.num_seqs), dim3(kPfThreads), smem, st, km, vm, p);
@@ -653,22 +655,23 @@ cudaError_t launch_prefill_v(const CUtensorMap &km, const CUtensorMap &vm, const
   return cudaGetLastError();
 }
 
-template <int D, int BS, int KV_T>
+template <int D, int BS, int KV_T, bool PRE>
 cudaError_t launch_prefill(const LayerMaps &maps, const PrefillParams &p, int tiles,
                            cudaStream_t st) {
   if constexpr (D == 128) {
     if (maps.v_blk_ok && maps.k_grp_ok)
-      return launch_prefill_v<D, BS, KV_T, true>(maps.k_grp, maps.v_blk, p, tiles, st);
+      return launch_prefill_v<D, BS, KV_T, true, PRE>(maps.k_grp, maps.v_blk, p, tiles, st);
   }
-  return launch_prefill_v<D, BS, KV_T, false>(maps.k, maps.v, p, tiles, st);
+  return launch_prefill_v<D, BS, KV_T, false, PRE>(maps.k, maps.v, p, tiles, st);
 }
 
 using PrefillFn = cudaError_t (*)(const LayerMaps &, const PrefillParams &, int, cudaStream_t);
 
-template <int D>
+template <int D, bool PRE = false>
 PrefillFn pick_prefill_bs(int bs, int dt) {
-  if (bs == 16) return dt == KV_BF16 ? launch_prefill<D, 16, KV_BF16> : launch_prefill<D, 16, KV_FP16>;
-  return dt == KV_BF16 ? launch_prefill<D, 32, KV_BF16> : launch_prefill<D, 32, KV_FP16>;
+  if (bs == 16)
+    return dt == KV_BF16 ? launch_prefill<D, 16, KV_BF16, PRE> : launch_prefill<D, 16, KV_FP16, PRE>;
+  return dt == KV_BF16 ? launch_prefill<D, 32, KV_BF16, PRE> : launch_prefill<D, 32, KV_FP16, PRE>;
 }
 
 }  // namespace
@@ -702,8 +705,8 @@ kv_status prefix_pass(kv_pool *pool, int layer, const void *q, int num_seqs, int
   LayerMaps maps;
   if (!layer_maps(pool, layer, pool->d.block_size, &maps, &code)) return code;
   const int D = pool->d.head_dim, bs = pool->d.block_size;
-  PrefillFn fn = D == 128 ? pick_prefill_bs<128>(bs, pool->d.cache_dtype)
-                          : pick_prefill_bs<64>(bs, pool->d.cache_dtype);
+  PrefillFn fn = D == 128 ? pick_prefill_bs<128, true>(bs, pool->d.cache_dtype)
+                          : pick_prefill_bs<64, true>(bs, pool->d.cache_dtype);
   return cuda_check(fn(maps, p, tiles, st), "cascade prefix launch");
 }
 
