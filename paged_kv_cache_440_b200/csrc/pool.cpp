@@ -233,7 +233,7 @@ extern "C" {
 
 const char *kv_last_error(void) { return g_last_error.c_str(); }
 
-const char *kv_version(void) { return "pagedkv 0.1 (sm_100a)"; }
+const char *kv_version(void) { return "pagedkv 0.2 (sm_100a)"; }
 
 kv_status kv_pool_required_bytes(const kv_pool_desc *desc, uint64_t *bytes) {
   if (!desc || !bytes) return fail(KV_ERR_INVALID, "null argument");
