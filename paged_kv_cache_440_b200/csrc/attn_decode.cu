@@ -1730,8 +1730,9 @@ kv_status run_cascade(kv_pool *pool, int32_t layer, const void *q, const void *k
   s = prefix_pass(pool, layer, q, num_seqs, num_q_heads, block_tables, prefix_blocks, scale,
                   cas.pre_o, cas.pre_ml, st);
   if (s != KV_OK) return s;
-  // 2. each sequence's positions past the prefix (with the step's append),
-  //    every unit as partials; 3. the merge, prefix partial folded in
+  // 2. each sequence's positions past the prefix (with the step's append):
+  //    a unit finished in one CTA folds in its prefix partials there, split
+  //    units leave partials; 3. the merge folds the prefix partial into those
   s = run_partition(pool, layer, q, q_dtype, num_seqs, num_q_heads, block_tables,
                     max_blocks_per_seq, context_lens, max_context, scale, out, num_ctas,
                     workspace, workspace_bytes, k_new, v_new, st, &cas);
